@@ -1,0 +1,491 @@
+"""Plain fp64 CPU oracle of Block-GTQ / TQ-MSE packed-KV decode attention.
+
+TEST INFRASTRUCTURE: used only by the tests, by ``__graft_entry__.smoke()`` and by the
+CPU-baseline leg of ``bench.py``. Never on the product path.
+
+Sources (cited by page title and passage):
+
+* [BGTQ] "Block-GTQ: RoPE-Block Rate Allocation for KV-Cache Quantization", abstract.
+  Sentence 2: RoPE 2-D frequency blocks carry the key precision. Sentence 3: a blockwise
+  logit-error bound motivates a label-free query-key energy score, combined with
+  codec-dependent rate penalties. Sentence 4: largest-marginal-gain allocation is
+  exactly optimal for the separable integer proxy under equal-cost budgets and
+  diminishing gains. Sentence 5: TQ-MSE instantiation, equal-rate blocks grouped, and
+  attention over packed caches with no decoded fp16 KV. Sentence 7: "K2V2" = average
+  logical bits per K/V coordinate. Sentence 8: no fp16 sink or recent-token buffer.
+* [TQ] "TurboQuant: paper algorithm and vLLM engineering implementation" (pipeline
+  diagram). Box "input vector x" (a per-head K or V vector); box "random rotation /
+  Hadamard" (makes coordinates concentrated and near-independent); box "per-coordinate
+  MSE scalar quantisation" (a few centroids approximate the rotated coordinates);
+  exercise box 1 (KV-cache memory for a batch/context/kv-head count).
+* [Philox] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3"
+  (SC'11): the Philox4x32-10 counter-based generator.
+* [BoxMuller] Box and Muller (1958): two uniforms to two independent N(0,1) draws.
+
+Readings where the pages leave a step open (each one is also listed in the design doc):
+energy score = mean query block energy x mean key block energy (blockwise bound,
+Cauchy-Schwarz per block); rate penalty D(b) = Gaussian Lloyd-Max per-coordinate MSE;
+block j = coordinates {j, j+64} (rotate-half RoPE); groups ordered by descending rate,
+blocks ascending, coordinate j before j+64; dense Haar rotation per group from a
+Philox-seeded Gaussian matrix (QR, positive triangular diagonal); y = sqrt(d) R x/|x|;
+code = number of thresholds <= y; one fp32 norm per (token, group); V coded as one
+128-dim TQ-MSE group at the V rate.
+
+Parity pins (tests/test_oracle_pins.py): Philox known-answer vectors; Lloyd-Max closed
+form at 1 bit, the published per-coordinate MSE figures and Monte Carlo; greedy vs
+exhaustive search; rotation orthogonality / QR definition; encode-decode against the
+closed-form distortion; attention against the rotated-space identity and its special
+cases. No function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+HEAD_DIM = 128
+N_BLOCKS = 64
+TILE_TOKENS = 64
+CHUNK_TOKENS = 16
+_MASK32 = np.uint64(0xFFFFFFFF)
+
+# ----------------------------------------------------------------------------------------
+# Counter-based randomness [Philox], [BoxMuller]
+# ----------------------------------------------------------------------------------------
+_PHILOX_M0 = np.uint64(0xD2511F53)
+_PHILOX_M1 = np.uint64(0xCD9E8D57)
+_PHILOX_W0 = np.uint64(0x9E3779B9)
+_PHILOX_W1 = np.uint64(0xBB67AE85)
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds [Philox, section 3]. ctr: 4 arrays, key: 2 ints/arrays.
+
+    One round multiplies words 0 and 2 by the two Philox constants, takes the 64-bit
+    products apart into high and low halves, and mixes the high halves with the other
+    two counter words and the round key. The key is bumped by the Weyl constants
+    before every round but the first.
+    """
+    c0, c1, c2, c3 = (np.asarray(c, dtype=np.uint64) & _MASK32 for c in ctr)
+    k0 = np.asarray(key[0], dtype=np.uint64) & _MASK32
+    k1 = np.asarray(key[1], dtype=np.uint64) & _MASK32
+    for rnd in range(10):
+        if rnd:
+            k0 = (k0 + _PHILOX_W0) & _MASK32
+            k1 = (k1 + _PHILOX_W1) & _MASK32
+        p0 = _PHILOX_M0 * c0
+        p1 = _PHILOX_M1 * c2
+        c0, c1, c2, c3 = ((p1 >> np.uint64(32)) ^ c1 ^ k0, p1 & _MASK32,
+                          (p0 >> np.uint64(32)) ^ c3 ^ k1, p0 & _MASK32)
+    return c0, c1, c2, c3
+
+
+def _u53(hi, lo):
+    """Uniform in (0,1) from two 32-bit words: 27 high bits of hi, 26 of lo, plus half."""
+    a = (hi >> np.uint64(5)).astype(np.float64)
+    b = (lo >> np.uint64(6)).astype(np.float64)
+    return (a * 67108864.0 + b + 0.5) / 9007199254740992.0
+
+
+def gaussian_stream(seed: int, stream: int, count: int) -> np.ndarray:
+    """Draws 0..count-1 of the N(0,1) stream (seed, stream).
+
+    Philox block n has counter (n mod 2^32, n div 2^32, stream, 0) and key (seed mod 2^32,
+    seed div 2^32); its words (0,1) and (2,3) give two uniforms u1, u2 and Box-Muller
+    turns them into draws 2n (radius times cosine) and 2n+1 (radius times sine).
+    """
+    nblk = (count + 1) // 2
+    n = np.arange(nblk, dtype=np.uint64)
+    x0, x1, x2, x3 = philox4x32_10((n & _MASK32, n >> np.uint64(32), np.full_like(n, stream), np.zeros_like(n)),
+                                   (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF))
+    u1, u2 = _u53(x0, x1), _u53(x2, x3)
+    r = np.sqrt(-2.0 * np.log(u1))
+    out = np.empty(2 * nblk)
+    out[0::2] = r * np.cos(2.0 * math.pi * u2)
+    out[1::2] = r * np.sin(2.0 * math.pi * u2)
+    return out[:count]
+
+
+def haar_rotation(seed: int, stream: int, d: int) -> np.ndarray:
+    """Seeded random orthogonal d x d matrix [TQ, "random rotation" box].
+
+    A[i, j] = draw i*d + j of the stream; A = Q T with T upper triangular and a positive
+    diagonal; the rotation is Q (Haar distributed). numpy's QR returns some sign pattern
+    on T's diagonal, fixed here by flipping the matching columns of Q.
+    """
+    a = gaussian_stream(seed, stream, d * d).reshape(d, d)
+    q, t = np.linalg.qr(a)
+    sgn = np.sign(np.diag(t))
+    sgn[sgn == 0] = 1.0
+    return q * sgn[None, :]
+
+
+# ----------------------------------------------------------------------------------------
+# Lloyd-Max scalar quantiser on N(0,1) [TQ, "per-coordinate MSE scalar quantisation" box]
+# ----------------------------------------------------------------------------------------
+def _phi(x):
+    return math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi) if math.isfinite(x) else 0.0
+
+
+def _upper_tail(x):
+    return 0.5 * math.erfc(x / math.sqrt(2.0)) if math.isfinite(x) else 0.0
+
+
+def lloyd_max(bits: int, tol: float = 1e-15, max_iter: int = 200000):
+    """MSE-optimal 2^bits-level quantiser for N(0,1): (centroids, thresholds, mse).
+
+    Lloyd's two conditions, iterated to a fixed point: each threshold is the midpoint of
+    its neighbouring centroids; each centroid is the conditional mean of its cell,
+    E[X | a < X <= b] = (phi(a) - phi(b)) / (P(X > a) - P(X > b)). The density is
+    symmetric, so only the positive half (middle threshold 0) is iterated and then
+    mirrored. mse = 1 - sum_i P(cell i) c_i^2 (the centroid condition makes the cross
+    term vanish).
+    """
+    if bits < 1 or bits > 8:
+        raise ValueError("bits in 1..8")
+    n = 1 << (bits - 1)
+    t = [0.0] + [3.0 * i / n for i in range(1, n)] + [math.inf]
+    mu = [0.0] * n
+    for _ in range(max_iter):
+        for i in range(n):
+            mu[i] = (_phi(t[i]) - _phi(t[i + 1])) / (_upper_tail(t[i]) - _upper_tail(t[i + 1]))
+        change = 0.0
+        for i in range(1, n):
+            nt = 0.5 * (mu[i - 1] + mu[i])
+            change = max(change, abs(nt - t[i]))
+            t[i] = nt
+        if change < tol:
+            break
+    for i in range(n):
+        mu[i] = (_phi(t[i]) - _phi(t[i + 1])) / (_upper_tail(t[i]) - _upper_tail(t[i + 1]))
+    cent = np.array([-m for m in reversed(mu)] + mu)
+    thr = np.array([-x for x in reversed(t[1:n])] + [0.0] + t[1:n])
+    mse = 1.0 - 2.0 * sum((_upper_tail(t[i]) - _upper_tail(t[i + 1])) * mu[i] ** 2 for i in range(n))
+    return cent, thr, mse
+
+
+def lloyd_max_mse_table(max_bits: int = 4) -> dict:
+    return {b: lloyd_max(b)[2] for b in range(1, max_bits + 1)}
+
+
+# ----------------------------------------------------------------------------------------
+# Energy score and rate allocation [BGTQ sentences 2-4]
+# ----------------------------------------------------------------------------------------
+def block_energy(q_cal: np.ndarray, k_cal: np.ndarray) -> np.ndarray:
+    """Label-free query-key energy per RoPE block [BGTQ sentence 3].
+
+    q_cal [n_q, h_q, 128], k_cal [n_k, h_kv, 128]. Block j holds coordinates j and j+64.
+    For KV head h: (mean over calibration queries and the h_q/h_kv query heads of h of
+    |q_j|^2) times (mean over calibration keys of |k_j|^2); the layer score sums the KV
+    heads. Cauchy-Schwarz per block bounds the logit error q.(k - k_hat) by
+    sum_j |q_j| |e_j|, and E|e_j|^2 grows with D(b_j) |k_j|^2, which is this product.
+    """
+    q = np.asarray(q_cal, dtype=np.float64)
+    k = np.asarray(k_cal, dtype=np.float64)
+    h_q, h_kv = q.shape[1], k.shape[1]
+    g = h_q // h_kv
+    qe = q[..., :N_BLOCKS] ** 2 + q[..., N_BLOCKS:] ** 2      # [n, h_q, 64]
+    ke = k[..., :N_BLOCKS] ** 2 + k[..., N_BLOCKS:] ** 2      # [n, h_kv, 64]
+    s = np.zeros(N_BLOCKS)
+    for h in range(h_kv):
+        s += qe[:, h * g:(h + 1) * g, :].mean(axis=(0, 1)) * ke[:, h, :].mean(axis=0)
+    return s
+
+
+def proxy_objective(score, rates, distortion) -> float:
+    """Separable integer proxy sum_j s_j D(b_j) [BGTQ sentence 4]."""
+    return float(sum(score[j] * distortion[rates[j]] for j in range(len(rates))))
+
+
+def greedy_rates(score, distortion, r_min: int, r_max: int, total_bits: int) -> np.ndarray:
+    """Largest-marginal-gain allocation [BGTQ sentence 4].
+
+    Every block starts at r_min; each step gives one more bit to the block whose proxy
+    drops the most, s_j (D(b_j) - D(b_j + 1)), among blocks still below r_max, until the
+    rates sum to total_bits. Ties go to the lowest block index.
+    """
+    n = len(score)
+    if total_bits < n * r_min or total_bits > n * r_max:
+        raise ValueError("infeasible budget")
+    rates = np.full(n, r_min, dtype=np.int64)
+    for _ in range(total_bits - n * r_min):
+        best, best_gain = -1, -math.inf
+        for j in range(n):
+            if rates[j] < r_max:
+                gain = score[j] * (distortion[rates[j]] - distortion[rates[j] + 1])
+                if gain > best_gain:
+                    best, best_gain = j, gain
+        rates[best] += 1
+    return rates
+
+
+def brute_force_rates(score, distortion, r_min: int, r_max: int, total_bits: int):
+    """Exhaustive minimum of the proxy over every rate vector with the given sum."""
+    import itertools
+    n = len(score)
+    best, arg = math.inf, []
+    for r in itertools.product(range(r_min, r_max + 1), repeat=n):
+        if sum(r) != total_bits:
+            continue
+        v = proxy_objective(score, r, distortion)
+        tol = 1e-12 * max(1.0, abs(v))
+        if not arg or v < best - tol:
+            best, arg = v, [r]
+        elif abs(v - best) <= tol:
+            arg.append(r)
+    return best, arg
+
+
+# ----------------------------------------------------------------------------------------
+# Layout: groups, rotations, packed format [BGTQ sentence 5], [TQ]
+# ----------------------------------------------------------------------------------------
+def chunk_slot(j: int) -> int:
+    """Bit slot of token j (0..15) inside a 16-token row of packed V codes."""
+    return 4 * ((j % 8) // 2) + 2 * (j // 8) + (j % 2)
+
+
+@dataclass
+class Layout:
+    k_rates: np.ndarray                  # [64] rate per RoPE block
+    v_rate: int
+    seed: int
+    groups: list                         # [(rate, coords ndarray)] in descending rate order
+    k_rot: list                          # R_g, d_g x d_g
+    v_rot: np.ndarray                    # 128 x 128
+    codebooks: dict                      # rate -> (centroids, thresholds)
+
+    @property
+    def n_kgroups(self):
+        return len(self.groups)
+
+    @property
+    def k_bits(self):                    # bits per token of the K code record
+        return int(sum(r * len(c) for r, c in self.groups))
+
+    @property
+    def k_record_bytes(self):
+        return self.k_bits // 8
+
+    @property
+    def v_record_bytes(self):
+        return HEAD_DIM * self.v_rate // 8
+
+    @property
+    def bytes_per_token(self):
+        """Resident bytes per (token, KV head): codes plus one fp32 norm per group."""
+        return self.k_record_bytes + self.v_record_bytes + 4 * (self.n_kgroups + 1)
+
+    @property
+    def tile_bytes(self):
+        return TILE_TOKENS * self.bytes_per_token
+
+    def packed_rates(self):
+        return np.concatenate([np.full(len(c), r) for r, c in self.groups])
+
+    def packed_coords(self):
+        return np.concatenate([c for _, c in self.groups])
+
+
+def group_coordinates(k_rates) -> list:
+    """Equal-rate blocks form one group [BGTQ sentence 5]; descending rate, blocks ascending,
+    coordinate j before j+64 inside block j."""
+    rates = np.asarray(k_rates)
+    out = []
+    for r in sorted(set(int(x) for x in rates), reverse=True):
+        blocks = [j for j in range(N_BLOCKS) if rates[j] == r]
+        coords = np.array([c for j in blocks for c in (j, j + N_BLOCKS)], dtype=np.int64)
+        out.append((r, coords))
+    return out
+
+
+def make_layout(k_rates, v_rate: int, seed: int) -> Layout:
+    """K record = a whole number of bytes: the 64 block rates must sum to a multiple of 4."""
+    if len(k_rates) != N_BLOCKS or (2 * int(np.sum(k_rates))) % 8 or not 1 <= v_rate <= 4:
+        raise ValueError("64 block rates summing to a multiple of 4, and a V rate in 1..4")
+    groups = group_coordinates(k_rates)
+    k_rot = [haar_rotation(seed, r, len(c)) for r, c in groups]
+    v_rot = haar_rotation(seed, 0, HEAD_DIM)
+    books = {}
+    for r in set([r for r, _ in groups] + [v_rate]):
+        c, t, _ = lloyd_max(r)
+        books[r] = (c, t)
+    return Layout(np.asarray(k_rates, dtype=np.int64), int(v_rate), int(seed), groups, k_rot, v_rot, books)
+
+
+def cache_bytes(layout: Layout, batch: int, h_kv: int, tokens: int) -> int:
+    """Resident bytes of a packed cache [TQ exercise box 1]: per (token, KV head)
+    128 b_K/8 + 128 b_V/8 code bytes plus 4 (n_gK + 1) norm bytes; capacity in whole
+    64-token tiles."""
+    tiles = -(-tokens // TILE_TOKENS)
+    return batch * h_kv * tiles * layout.tile_bytes
+
+
+# ----------------------------------------------------------------------------------------
+# TQ-MSE encode / decode [TQ pipeline boxes], [BGTQ sentence 5]
+# ----------------------------------------------------------------------------------------
+def _tq_encode_group(x: np.ndarray, rot: np.ndarray, thresholds: np.ndarray):
+    """x [n, d] -> (codes [n, d], norms [n], margin [n, d]).
+
+    |x| is the group norm; the unit vector is rotated and scaled by sqrt(d) so each
+    coordinate has unit variance, then each coordinate is compared with the Lloyd-Max
+    thresholds: code = number of thresholds <= y (a value on a threshold goes up).
+    A zero vector gives y = 0. margin = distance from y to the nearest threshold.
+    """
+    d = x.shape[1]
+    norms = np.sqrt(np.sum(x * x, axis=1))
+    y = np.zeros_like(x)
+    nz = norms > 0
+    y[nz] = math.sqrt(d) * (x[nz] @ rot.T) / norms[nz, None]
+    codes = np.searchsorted(thresholds, y, side="right")
+    margin = np.min(np.abs(y[..., None] - thresholds[None, None, :]), axis=-1)
+    return codes.astype(np.int64), norms, margin
+
+
+def encode(layout: Layout, k: np.ndarray, v: np.ndarray) -> dict:
+    """k, v [n, 128] (any float; promoted to fp64). Codes are in packed-dimension order."""
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    kc, kn, km = [], [], []
+    for (r, coords), rot in zip(layout.groups, layout.k_rot):
+        c, nrm, m = _tq_encode_group(k[:, coords], rot, layout.codebooks[r][1])
+        kc.append(c)
+        kn.append(nrm)
+        km.append(m)
+    vc, vn, vm = _tq_encode_group(v, layout.v_rot, layout.codebooks[layout.v_rate][1])
+    return {
+        "k_codes": np.concatenate(kc, axis=1), "k_norms": np.stack(kn, axis=1), "k_margin": np.concatenate(km, axis=1),
+        "v_codes": vc, "v_norm": vn, "v_margin": vm,
+    }
+
+
+def reconstruct(layout: Layout, k_codes, k_norms, v_codes, v_norm):
+    """Decoded k_hat, v_hat [n, 128] in original coordinates (fp64): per group
+    x_hat = (|x| / sqrt(d)) R^T c[code], scattered back to the group's coordinates."""
+    n = k_codes.shape[0]
+    kh = np.zeros((n, HEAD_DIM))
+    col = 0
+    for gi, ((r, coords), rot) in enumerate(zip(layout.groups, layout.k_rot)):
+        d = len(coords)
+        cvals = layout.codebooks[r][0][k_codes[:, col:col + d]]
+        kh[:, coords] = (np.asarray(k_norms[:, gi], dtype=np.float64) / math.sqrt(d))[:, None] * (cvals @ rot)
+        col += d
+    cv = layout.codebooks[layout.v_rate][0][v_codes]
+    vh = (np.asarray(v_norm, dtype=np.float64) / math.sqrt(HEAD_DIM))[:, None] * (cv @ layout.v_rot)
+    return kh, vh
+
+
+def attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, scale: float) -> np.ndarray:
+    """Exact softmax attention of queries q [G, 128] over every cached token (no sink or
+    recent-token window [BGTQ sentence 8]). Returns [G, 128]; an empty cache gives 0."""
+    q = np.asarray(q, dtype=np.float64)
+    if k_hat.shape[0] == 0:
+        return np.zeros_like(q)
+    s = (q @ k_hat.T) * scale
+    s -= s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ v_hat
+
+
+# ----------------------------------------------------------------------------------------
+# Packed tile format (the byte layout both sides implement)
+# ----------------------------------------------------------------------------------------
+def _put_bits(bitbuf: np.ndarray, pos: np.ndarray, codes: np.ndarray, rate: int):
+    for i in range(rate):
+        bitbuf[..., pos + i] = (codes >> i) & 1
+
+
+def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
+    """Bytes of one (batch row, KV head) cache holding tokens 0..n-1 of ``enc``.
+
+    Tile of 64 tokens = [K records, token-major, LSB-first bitstream in packed-dim order]
+    [V codes: four 16-token chunks, each a bitstream where (dim d, token j) sits at bit
+    (16 d + slot(j)) b_V] [K norms fp32, group-major] [V norms fp32]. Unused slots are 0.
+    """
+    n = enc["k_codes"].shape[0]
+    if capacity % TILE_TOKENS or n > capacity:
+        raise ValueError("capacity must be a multiple of 64 and hold the tokens")
+    ntile = capacity // TILE_TOKENS
+    out = np.zeros((ntile, layout.tile_bytes), dtype=np.uint8)
+    rates = layout.packed_rates()
+    koff = np.concatenate([[0], np.cumsum(rates)[:-1]])
+    kb, vb, ng = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups
+    # K records
+    kbits = np.zeros((ntile * TILE_TOKENS, kb * 8), dtype=np.uint8)
+    for p in range(HEAD_DIM):
+        for i in range(rates[p]):
+            kbits[:n, koff[p] + i] = (enc["k_codes"][:, p] >> i) & 1
+    krec = np.packbits(kbits, axis=1, bitorder="little").reshape(ntile, TILE_TOKENS * kb)
+    out[:, :TILE_TOKENS * kb] = krec
+    # V chunks
+    br = layout.v_rate
+    vcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
+    vcodes[:n] = enc["v_codes"]
+    vcodes = vcodes.reshape(ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS, HEAD_DIM)
+    vbits = np.zeros((ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS * HEAD_DIM * br), dtype=np.uint8)
+    for j in range(CHUNK_TOKENS):
+        pos = (CHUNK_TOKENS * np.arange(HEAD_DIM) + chunk_slot(j)) * br
+        for i in range(br):
+            vbits[:, :, pos + i] = (vcodes[:, :, j, :] >> i) & 1
+    vrec = np.packbits(vbits, axis=2, bitorder="little").reshape(ntile, TILE_TOKENS * vb)
+    base = TILE_TOKENS * kb
+    out[:, base:base + TILE_TOKENS * vb] = vrec
+    # norms
+    base += TILE_TOKENS * vb
+    kn = np.zeros((ntile * TILE_TOKENS, ng), dtype=np.float32)
+    kn[:n] = enc["k_norms"].astype(np.float32)
+    kn = kn.reshape(ntile, TILE_TOKENS, ng).transpose(0, 2, 1).reshape(ntile, -1)
+    out[:, base:base + 4 * TILE_TOKENS * ng] = kn.view(np.uint8).reshape(ntile, -1)
+    base += 4 * TILE_TOKENS * ng
+    vn = np.zeros(ntile * TILE_TOKENS, dtype=np.float32)
+    vn[:n] = enc["v_norm"].astype(np.float32)
+    out[:, base:base + 4 * TILE_TOKENS] = vn.reshape(ntile, TILE_TOKENS).view(np.uint8)
+    return out.reshape(-1)
+
+
+def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
+    """Inverse of ``pack`` for tokens 0..n-1 (codes, fp32 norms promoted to fp64)."""
+    ntile = len(buf) // layout.tile_bytes
+    t = np.asarray(buf, dtype=np.uint8).reshape(ntile, layout.tile_bytes)
+    kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
+    rates = layout.packed_rates()
+    koff = np.concatenate([[0], np.cumsum(rates)[:-1]])
+    kbits = np.unpackbits(t[:, :TILE_TOKENS * kb].reshape(-1, kb), axis=1, bitorder="little").astype(np.int64)
+    kc = np.zeros((kbits.shape[0], HEAD_DIM), dtype=np.int64)
+    for p in range(HEAD_DIM):
+        for i in range(rates[p]):
+            kc[:, p] |= kbits[:, koff[p] + i] << i
+    base = TILE_TOKENS * kb
+    vbits = np.unpackbits(t[:, base:base + TILE_TOKENS * vb].reshape(ntile, TILE_TOKENS // CHUNK_TOKENS, -1),
+                          axis=2, bitorder="little").astype(np.int64)
+    vc = np.zeros((ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS, HEAD_DIM), dtype=np.int64)
+    for j in range(CHUNK_TOKENS):
+        pos = (CHUNK_TOKENS * np.arange(HEAD_DIM) + chunk_slot(j)) * br
+        for i in range(br):
+            vc[:, :, j, :] |= vbits[:, :, pos + i] << i
+    base += TILE_TOKENS * vb
+    kn = t[:, base:base + 4 * TILE_TOKENS * ng].copy().view(np.float32).reshape(ntile, ng, TILE_TOKENS)
+    kn = kn.transpose(0, 2, 1).reshape(-1, ng)
+    base += 4 * TILE_TOKENS * ng
+    vn = t[:, base:base + 4 * TILE_TOKENS].copy().view(np.float32).reshape(-1)
+    return {"k_codes": kc[:n], "k_norms": kn[:n].astype(np.float64),
+            "v_codes": vc.reshape(-1, HEAD_DIM)[:n], "v_norm": vn[:n].astype(np.float64)}
+
+
+def boundary_mask(layout: Layout, enc: dict, capacity: int, eps: float = 1e-6):
+    """Byte mask (same shape as ``pack``) covering the code bits of every coordinate whose
+    rotated value lies within eps of a decision threshold; also returns their count."""
+    rates = layout.packed_rates()
+    kmask = np.where(enc["k_margin"] < eps, (1 << rates)[None, :] - 1, 0)
+    vmask = np.where(enc["v_margin"] < eps, (1 << layout.v_rate) - 1, 0)
+    fake = {"k_codes": kmask, "v_codes": vmask,
+            "k_norms": np.zeros_like(enc["k_norms"]), "v_norm": np.zeros_like(enc["v_norm"])}
+    return pack(layout, fake, capacity), int((enc["k_margin"] < eps).sum() + (enc["v_margin"] < eps).sum())
+
+
+def decode_attention(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int, scale: float) -> np.ndarray:
+    """Attention of the G query heads q [G, 128] of one KV head over its packed cache."""
+    u = unpack(layout, buf, length)
+    kh, vh = reconstruct(layout, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
+    return attention(q, kh, vh, scale)

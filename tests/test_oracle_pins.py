@@ -1,0 +1,357 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a wrong
+sign or index, a transposed operand) fails it. No GPU needed.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from packed_cache_decode_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ------------------------------------------------------------------ randomness
+def test_philox_known_answers():
+    for row in _rows("philox4x32_10_kat.txt"):
+        v = [int(x, 16) for x in row if x != "->"]
+        ctr, key, want = v[:4], v[4:6], v[6:10]
+        got = O.philox4x32_10(tuple([c] for c in ctr), tuple(key))
+        assert [int(g[0]) for g in got] == want
+
+
+def test_gaussian_stream_statistics_and_determinism():
+    z = O.gaussian_stream(12345, 3, 400001)
+    assert z.shape == (400001,)
+    assert abs(z.mean()) < 0.01 and abs(z.var() - 1) < 0.01
+    assert abs(np.mean(z ** 4) - 3) < 0.05          # Gaussian kurtosis
+    assert abs(np.corrcoef(z[0:-1:2], z[1::2])[0, 1]) < 0.01  # the cos/sin pair is uncorrelated
+    np.testing.assert_array_equal(z[:1000], O.gaussian_stream(12345, 3, 1000))
+    assert not np.allclose(z[:100], O.gaussian_stream(12345, 4, 100))
+    assert not np.allclose(z[:100], O.gaussian_stream(12346, 3, 100))
+
+
+def test_haar_rotation_is_the_qr_factor_of_the_seeded_matrix():
+    for d in (2, 6, 34, 128):
+        r = O.haar_rotation(7, 2, d)
+        np.testing.assert_allclose(r @ r.T, np.eye(d), atol=1e-12)
+        a = O.gaussian_stream(7, 2, d * d).reshape(d, d)
+        t = r.T @ a                                   # must be upper triangular, positive diagonal
+        assert np.max(np.abs(np.tril(t, -1))) < 1e-10 * np.max(np.abs(t))
+        assert np.all(np.diag(t) > 0)
+        x = np.random.default_rng(d).standard_normal((50, d))
+        np.testing.assert_allclose(np.linalg.norm(x @ r.T, axis=1) / np.linalg.norm(x, axis=1), 1.0, atol=1e-6)
+
+
+def test_haar_rotation_first_moment():
+    # For Haar-distributed Q, E[Q] = 0 and E[Q_ij^2] = 1/d.
+    d = 16
+    qs = np.stack([O.haar_rotation(s, 1, d) for s in range(300)])
+    assert abs(qs.mean()) < 0.01
+    assert abs((qs ** 2).mean() - 1.0 / d) < 0.002
+
+
+# ------------------------------------------------------------------ Lloyd-Max
+def test_lloyd_max_one_bit_closed_form():
+    c, t, mse = O.lloyd_max(1)
+    assert t.tolist() == [0.0]
+    assert c[1] == pytest.approx(math.sqrt(2 / math.pi), rel=1e-14)
+    assert mse == pytest.approx(1 - 2 / math.pi, rel=1e-13)
+
+
+def test_lloyd_max_published_mse():
+    for b, want in _rows("gaussian_lloyd_max_mse.txt"):
+        assert O.lloyd_max(int(b))[2] == pytest.approx(float(want), rel=1e-3)
+
+
+def test_lloyd_max_conditions_by_quadrature():
+    from scipy import integrate
+    from scipy.stats import norm
+    for b in (2, 3, 4):
+        c, t, mse = O.lloyd_max(b)
+        np.testing.assert_allclose(c, -c[::-1], rtol=0, atol=0)
+        assert t[len(t) // 2] == 0.0
+        np.testing.assert_allclose(t, 0.5 * (c[1:] + c[:-1]), atol=1e-14)
+        edges = np.concatenate([[-np.inf], t, [np.inf]])
+        tot = 0.0
+        for i in range(len(c)):
+            p = norm.cdf(edges[i + 1]) - norm.cdf(edges[i])
+            m1 = integrate.quad(lambda x: x * norm.pdf(x), edges[i], edges[i + 1])[0]
+            assert m1 / p == pytest.approx(c[i], abs=1e-9)
+            tot += integrate.quad(lambda x: (x - c[i]) ** 2 * norm.pdf(x), edges[i], edges[i + 1])[0]
+        assert tot == pytest.approx(mse, rel=1e-8)
+
+
+def test_lloyd_max_monte_carlo():
+    x = np.random.default_rng(0).standard_normal(2_000_000)
+    for b in (1, 2, 3, 4):
+        c, t, mse = O.lloyd_max(b)
+        xq = c[np.searchsorted(t, x, side="right")]
+        assert np.mean((x - xq) ** 2) == pytest.approx(mse, rel=0.01)
+
+
+def test_diminishing_marginal_gains():
+    D = O.lloyd_max_mse_table()
+    gains = [D[b] - D[b + 1] for b in (1, 2, 3)]
+    assert all(g > 0 for g in gains) and gains[0] > gains[1] > gains[2]
+
+
+# ------------------------------------------------------------------ energy + allocation
+def test_block_energy_constructed_cases():
+    n = 5
+    # two KV heads, GQA 2: query heads 0,1 -> kv 0; 2,3 -> kv 1
+    q = np.zeros((n, 4, 128))
+    k = np.zeros((n, 2, 128))
+    q[:, 0:2, 3] = 2.0           # kv-0 queries: energy 4 in block 3 (coordinate 3)
+    q[:, 2:4, 64 + 10] = 1.0     # kv-1 queries: energy 1 in block 10 (coordinate 74)
+    k[:, 0, 3 + 64] = 3.0        # kv-0 keys: energy 9 in block 3 (coordinate 67)
+    k[:, 1, 10] = 5.0            # kv-1 keys: energy 25 in block 10
+    k[:, 1, 3] = 7.0             # kv-1 key energy in block 3 meets no kv-1 query energy
+    s = O.block_energy(q, k)
+    want = np.zeros(64)
+    want[3] = 4 * 9
+    want[10] = 1 * 25
+    np.testing.assert_allclose(s, want)
+
+
+def test_block_energy_is_rope_invariant():
+    m = synth.make_layer_model(8, 2, seed=3)
+    q = torch.stack([torch.randn(64, 128) for _ in range(8)], 1).double()
+    k = torch.stack([torch.randn(64, 128) for _ in range(2)], 1).double()
+    pos = torch.arange(64) * 37 + 5
+    qr = synth.rope_rotate_half(q.transpose(0, 1), pos, 5e5).transpose(0, 1)
+    kr = synth.rope_rotate_half(k.transpose(0, 1), pos, 5e5).transpose(0, 1)
+    np.testing.assert_allclose(O.block_energy(qr.numpy(), kr.numpy()), O.block_energy(q.numpy(), k.numpy()), rtol=1e-12)
+    assert m.group == 4
+
+
+def test_greedy_equals_exhaustive_optimum():
+    rng = np.random.default_rng(1)
+    D = O.lloyd_max_mse_table()
+    cases = 0
+    for n in (1, 2, 3, 4, 5, 6):
+        for trial in range(3 if n < 6 else 1):
+            s = rng.exponential(size=n) * rng.choice([1, 10, 100], size=n)
+            if trial == 2:
+                s[: n // 2] = s[-1]                 # ties
+            for budget in range(n, 4 * n + 1):
+                g = O.greedy_rates(s, D, 1, 4, budget)
+                best, args = O.brute_force_rates(s, D, 1, 4, budget)
+                assert g.sum() == budget
+                assert O.proxy_objective(s, g, D) == pytest.approx(best, rel=1e-12, abs=1e-15)
+                if len(args) == 1:
+                    assert tuple(g) == args[0]
+                cases += 1
+    assert cases > 60
+
+
+def test_greedy_infeasible_budget():
+    D = O.lloyd_max_mse_table()
+    with pytest.raises(ValueError):
+        O.greedy_rates(np.ones(4), D, 1, 4, 3)
+    with pytest.raises(ValueError):
+        O.greedy_rates(np.ones(4), D, 1, 4, 17)
+
+
+def test_greedy_prefers_high_energy_blocks():
+    D = O.lloyd_max_mse_table()
+    s = np.array([1.0, 100.0, 10.0, 0.01])
+    r = O.greedy_rates(s, D, 1, 4, 8)
+    assert r[1] >= r[2] >= r[0] >= r[3]
+
+
+# ------------------------------------------------------------------ layout + format
+def _random_rates(rng):
+    r = rng.integers(1, 5, 64)
+    while r.sum() % 4:
+        j = rng.integers(0, 64)
+        r[j] = r[j] % 4 + 1
+    return r
+
+
+def test_grouping_and_byte_formula():
+    with pytest.raises(ValueError):
+        O.make_layout(np.array([1] * 63 + [2]), 2, 0)           # 130 bits: not whole bytes
+    lay = O.make_layout(np.array([2] * 64), 2, 0)
+    assert lay.n_kgroups == 1 and lay.bytes_per_token == 32 + 32 + 8
+    lay = O.make_layout(np.array([4] * 32 + [2] * 32), 2, 0)
+    assert [r for r, _ in lay.groups] == [4, 2]
+    assert list(lay.groups[0][1][:4]) == [0, 64, 1, 65]
+    assert lay.bytes_per_token == 48 + 32 + 12
+    mixed = np.array([1] * 16 + [2] * 16 + [3] * 16 + [4] * 16)        # average 2.5 bits
+    lay = O.make_layout(mixed, 3, 0)
+    assert [r for r, _ in lay.groups] == [4, 3, 2, 1]
+    assert lay.k_bits == 2 * (16 + 32 + 48 + 64)
+    # K2V2 with four groups: 32 + 32 + 20 = 84 bytes, K3V3 four groups 116, K4V4 one group 136
+    k2 = np.array([1] * 22 + [2] * 22 + [3] * 18 + [4] * 2)
+    assert k2.sum() == 128
+    assert O.make_layout(k2, 2, 0).bytes_per_token == 84
+    k3 = np.array([1] * 4 + [2] * 10 + [3] * 32 + [4] * 18)
+    assert k3.sum() == 192
+    assert O.make_layout(k3, 3, 0).bytes_per_token == 116
+    assert O.make_layout(np.full(64, 4), 4, 0).bytes_per_token == 136
+    lay = O.make_layout(k2, 2, 0)
+    assert O.cache_bytes(lay, 2, 8, 128) == 2 * 8 * 128 * 84
+    assert O.cache_bytes(lay, 1, 1, 65) == 128 * 84
+
+
+def test_pack_places_bits_where_the_format_says():
+    lay = O.make_layout(np.array([2] * 32 + [1] * 32), 3, 5)   # packed dims 0..63 rate 2, 64..127 rate 1
+    enc = {"k_codes": np.zeros((3, 128), dtype=np.int64), "v_codes": np.zeros((3, 128), dtype=np.int64),
+           "k_norms": np.zeros((3, 2)), "v_norm": np.zeros(3)}
+    enc["k_codes"][2, 5] = 3          # token 2, packed dim 5 (rate 2): bits 10,11 of record 2
+    enc["k_codes"][1, 64] = 1         # token 1, packed dim 64 (rate 1): bit 128 of record 1
+    enc["v_codes"][1, 7] = 5          # token 1, dim 7, rate 3: chunk 0, bit (16*7 + slot(1))*3
+    enc["v_codes"][2, 0] = 6          # token 2 -> slot 4: bits 12..14 of chunk 0
+    enc["k_norms"][1] = [1.5, -2.0]
+    enc["v_norm"][2] = 0.25
+    buf = O.pack(lay, enc, 64)
+    kb = lay.k_record_bytes
+    assert kb == 24 and lay.tile_bytes == 64 * (24 + 48 + 12) and buf.size == lay.tile_bytes
+    assert buf[2 * kb + 1] == 0b00001100
+    assert buf[1 * kb + 16] == 1
+    vbase = 64 * kb
+    bit = (16 * 7 + 1) * 3
+    assert (int.from_bytes(buf[vbase:vbase + 8 * 48].tobytes(), "little") >> bit) & 7 == 5
+    assert (int.from_bytes(buf[vbase:vbase + 8 * 48].tobytes(), "little") >> 12) & 7 == 6
+    nbase = vbase + 64 * 48
+    kn = buf[nbase:nbase + 4 * 128].view(np.float32)
+    assert kn[1] == 1.5 and kn[64 + 1] == -2.0
+    assert buf[nbase + 512:nbase + 768].view(np.float32)[2] == 0.25
+    # nothing else written: one byte per code, and 1.5 / -2.0 / 0.25 have 2 / 1 / 2 nonzero bytes
+    assert int(np.count_nonzero(buf)) == 4 + 2 + 1 + 2
+    u = O.unpack(lay, buf, 3)
+    np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
+    np.testing.assert_array_equal(u["v_codes"], enc["v_codes"])
+
+
+def test_chunk_slot_is_a_permutation():
+    assert sorted(O.chunk_slot(j) for j in range(16)) == list(range(16))
+    assert [O.chunk_slot(j) for j in (0, 1, 8, 9, 2, 3)] == [0, 1, 2, 3, 4, 5]
+
+
+def test_pack_unpack_round_trip():
+    rng = np.random.default_rng(3)
+    rates = _random_rates(rng)
+    lay = O.make_layout(rates, 2, 11)
+    n = 150
+    k = rng.standard_normal((n, 128)) * 3
+    v = rng.standard_normal((n, 128))
+    enc = O.encode(lay, k, v)
+    buf = O.pack(lay, enc, 192)
+    assert buf.size == O.cache_bytes(lay, 1, 1, 192)
+    u = O.unpack(lay, buf, n)
+    np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
+    np.testing.assert_array_equal(u["v_codes"], enc["v_codes"])
+    np.testing.assert_array_equal(u["k_norms"], enc["k_norms"].astype(np.float32))
+    np.testing.assert_array_equal(u["v_norm"], enc["v_norm"].astype(np.float32))
+
+
+# ------------------------------------------------------------------ encode / decode
+def test_codes_are_nearest_centroids():
+    rng = np.random.default_rng(4)
+    for b in (1, 2, 3, 4):
+        lay = O.make_layout(np.full(64, b), b, 9)
+        x = rng.standard_normal((40, 128))
+        enc = O.encode(lay, x, x)
+        y = math.sqrt(128) * (x @ lay.k_rot[0].T) / np.linalg.norm(x, axis=1, keepdims=True)
+        c = lay.codebooks[b][0]
+        nearest = np.argmin(np.abs(y[..., None] - c[None, None, :]), axis=-1)
+        # packed order == group order for a single group: coordinates (0,64,1,65,...)
+        y_packed = math.sqrt(128) * (x[:, lay.groups[0][1]] @ lay.k_rot[0].T) / np.linalg.norm(x, axis=1, keepdims=True)
+        nearest_p = np.argmin(np.abs(y_packed[..., None] - c[None, None, :]), axis=-1)
+        np.testing.assert_array_equal(enc["k_codes"], nearest_p)
+        assert nearest.shape == nearest_p.shape
+
+
+def test_zero_vector_and_threshold_ties():
+    lay = O.make_layout(np.full(64, 2), 2, 1)
+    enc = O.encode(lay, np.zeros((2, 128)), np.zeros((2, 128)))
+    assert np.all(enc["k_codes"] == 2) and np.all(enc["v_codes"] == 2)
+    kh, vh = O.reconstruct(lay, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+    assert np.all(kh == 0) and np.all(vh == 0)
+
+
+def test_reconstruction_error_matches_lloyd_max_distortion():
+    # After a Haar rotation of a 128-dim vector the coordinates are close to N(0,1)
+    # (scaled), so the relative squared error approaches D(b). A transposed rotation
+    # or a missing sqrt(d) would give an O(1) error instead.
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3000, 128))
+    for b in (1, 2, 3, 4):
+        lay = O.make_layout(np.full(64, b), b, 21)
+        enc = O.encode(lay, x, x)
+        kh, vh = O.reconstruct(lay, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+        D = O.lloyd_max(b)[2]
+        for xh in (kh, vh):
+            rel = np.sum((xh - x) ** 2) / np.sum(x ** 2)
+            assert rel == pytest.approx(D, rel=0.05)
+
+
+def test_mixed_rate_reconstruction_error_by_group():
+    rng = np.random.default_rng(6)
+    rates = np.array([1] * 16 + [2] * 16 + [3] * 16 + [4] * 16)
+    lay = O.make_layout(rates, 2, 8)
+    x = rng.standard_normal((4000, 128))
+    enc = O.encode(lay, x, x)
+    kh, _ = O.reconstruct(lay, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+    for r, coords in lay.groups:
+        rel = np.sum((kh[:, coords] - x[:, coords]) ** 2) / np.sum(x[:, coords] ** 2)
+        # 32-dim groups: the rotated coordinates are only roughly Gaussian; allow 15%
+        assert rel == pytest.approx(O.lloyd_max(r)[2], rel=0.15)
+
+
+# ------------------------------------------------------------------ attention
+def test_attention_special_cases():
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal((9, 128))
+    k = rng.standard_normal((9, 128))
+    q = rng.standard_normal((3, 128))
+    np.testing.assert_allclose(O.attention(q, k[:1], v[:1], 0.1), np.repeat(v[:1], 3, 0), rtol=1e-15)
+    np.testing.assert_allclose(O.attention(np.zeros((2, 128)), k, v, 0.1), np.repeat(v.mean(0, keepdims=True), 2, 0), rtol=1e-13)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None, :, None, :], torch.tensor(k)[None, None].expand(1, 3, 9, 128),
+        torch.tensor(v)[None, None].expand(1, 3, 9, 128), scale=0.1)[0, :, 0].numpy()
+    np.testing.assert_allclose(O.attention(q, k, v, 0.1), ref, rtol=1e-12, atol=1e-12)
+    assert np.all(O.attention(q, k[:0], v[:0], 0.1) == 0)
+
+
+def test_decode_attention_equals_rotated_space_form():
+    """Scores and values computed from codes in the rotated space (q' = R q per group,
+    centroid lookups, inverse rotation of the value sum) equal the original-space result."""
+    rng = np.random.default_rng(8)
+    rates = _random_rates(rng)
+    lay = O.make_layout(rates, 3, 4)
+    n, G = 70, 4
+    k = rng.standard_normal((n, 128)) * 2
+    v = rng.standard_normal((n, 128))
+    q = rng.standard_normal((G, 128))
+    enc = O.encode(lay, k, v)
+    buf = O.pack(lay, enc, 128)
+    out = O.decode_attention(lay, q, buf, n, 0.088)
+    u = O.unpack(lay, buf, n)
+    s = np.zeros((G, n))
+    col = 0
+    for gi, ((r, coords), rot) in enumerate(zip(lay.groups, lay.k_rot)):
+        d = len(coords)
+        qp = q[:, coords] @ rot.T
+        cv = lay.codebooks[r][0][u["k_codes"][:, col:col + d]]
+        s += (qp @ cv.T) * (u["k_norms"][:, gi] / math.sqrt(d))[None, :]
+        col += d
+    s *= 0.088
+    p = np.exp(s - s.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    cv = lay.codebooks[3][0][u["v_codes"]] * (u["v_norm"] / math.sqrt(128))[:, None]
+    out_rot = (p @ cv) @ lay.v_rot
+    np.testing.assert_allclose(out, out_rot, rtol=1e-11, atol=1e-12)
