@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark: packed-KV decode attention (Block-GTQ / TQ-MSE) on B200.
+
+One step = one decode step of a whole model's attention: for every layer, encode-append
+the new token's key/value (TQ-MSE) into that layer's packed cache and run decode
+attention of all query heads over the packed cache (split-K + log-sum-exp combine).
+Each layer has its own cache, so a step reads every layer's cache once (far more than
+the 126 MB L2). The step is captured in a CUDA graph and replayed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|qwen3b|llama70b|tiny]
+    python bench.py --impl reference ...      # the CPU oracle, timed on the host cores
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from packed_cache_decode_b200 import binding as B  # noqa: E402
+from packed_cache_decode_b200 import synth  # noqa: E402
+
+METRIC = "packed-KV decode attention: cached keys/s (HBM GB/s as % of B200 peak in roofline)"
+UNIT = "keys/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ workload
+class Model:
+    """Per-layer packed caches and per-step inputs of one workload on one GPU."""
+
+    def __init__(self, wl: synth.Workload, device: torch.device, seed_offset: int = 0):
+        self.wl = wl
+        self.dev = device
+        L, Bt, hq, hkv = wl.length, wl.batch, wl.h_q, wl.h_kv
+        self.capacity = 64 * math.ceil(L / 64)
+        self.layers = []
+        gen = torch.Generator(device=device)
+        for layer in range(wl.layers):
+            seed = wl.seed * 1000 + layer + seed_offset
+            m = synth.make_layer_model(hq, hkv, seed)
+            q_cal, k_cal = synth.make_calibration(m, 256, seed + 1, wl.theta)
+            rates = B.plan_layer_rates(q_cal.numpy(), k_cal.numpy(), wl.k_bits)
+            lay = B.Layout(rates, wl.v_bits, seed).upload(device.index)
+            cache = torch.zeros(lay.cache_bytes(Bt, hkv, self.capacity), dtype=torch.uint8, device=device)
+            gen.manual_seed(seed)
+            k, v = self._draw_kv(m, Bt, L, hkv, gen)
+            lens0 = torch.zeros(Bt, dtype=torch.int32, device=device)
+            chunk = 16384
+            for a in range(0, L - 1, chunk):
+                b = min(L - 1, a + chunk)
+                lens0.fill_(a)
+                B.encode_append(lay, k[:, a:b].contiguous(), v[:, a:b].contiguous(), lens0, cache, self.capacity)
+            q = self._draw_q(m, Bt, hq, L - 1, gen)
+            self.layers.append({
+                "layout": lay, "cache": cache,
+                "k_new": k[:, L - 1:L].contiguous(), "v_new": v[:, L - 1:L].contiguous(), "q": q,
+                "out": torch.empty(Bt, hq, 128, dtype=torch.float32, device=device),
+            })
+            del k, v
+        torch.cuda.synchronize(device)
+        self.lens_before = torch.full((Bt,), L - 1, dtype=torch.int32, device=device)
+        self.lens_after = torch.full((Bt,), L, dtype=torch.int32, device=device)
+        ws = max(B.workspace_bytes(x["layout"], Bt, hq, hkv, L) for x in self.layers)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.bytes_per_step = sum(Bt * hkv * L * x["layout"].bytes_per_token for x in self.layers)
+        self.keys_per_step = Bt * hkv * L * wl.layers
+
+    def _draw_kv(self, m, Bt, L, hkv, gen):
+        # Same recipe as synth.key_slice / value_slice, drawn on the device in bulk.
+        dt = self.wl.dtype
+        x = torch.randn(Bt, L, hkv, 128, generator=gen, device=self.dev)
+        x *= torch.cat([m.k_scale, m.k_scale], 1).to(self.dev)[None, None]
+        for h in range(hkv):
+            x[:, :, h, m.outliers[h].to(self.dev)] *= m.outlier_gain
+        x = _rope_dev(x, torch.arange(L, device=self.dev), self.wl.theta)
+        v = torch.randn(Bt, L, hkv, 128, generator=gen, device=self.dev)
+        return x.to(dt), v.to(dt)
+
+    def _draw_q(self, m, Bt, hq, pos, gen):
+        x = torch.randn(Bt, 1, hq, 128, generator=gen, device=self.dev)
+        x *= torch.cat([m.q_scale, m.q_scale], 1).to(self.dev)[None, None]
+        for i in range(hq):
+            x[:, :, i, m.outliers[i // m.group].to(self.dev)] *= m.outlier_gain
+        x = _rope_dev(x, torch.tensor([pos], device=self.dev), self.wl.theta)
+        return x[:, 0].contiguous().to(self.wl.dtype)
+
+    def step(self, stream, timing_events=None):
+        cap = self.capacity
+        for i, x in enumerate(self.layers):
+            B.encode_append(x["layout"], x["k_new"], x["v_new"], self.lens_before, x["cache"], cap, stream=stream)
+            B.decode_attention(x["layout"], x["q"], x["cache"], self.lens_after, cap, self.wl.length, x["out"],
+                               self.workspace, self.wl.h_kv, stream=stream)
+
+    def decode_only(self, stream):
+        for x in self.layers:
+            B.decode_attention(x["layout"], x["q"], x["cache"], self.lens_after, self.capacity, self.wl.length,
+                               x["out"], self.workspace, self.wl.h_kv, stream=stream)
+
+
+def _rope_dev(x, pos, theta):
+    inv = theta ** (-torch.arange(64, dtype=torch.float64, device=x.device) * 2.0 / 128)
+    ang = pos.double()[:, None] * inv[None, :]
+    c = torch.cos(ang)[None, :, None, :].float()
+    s = torch.sin(ang)[None, :, None, :].float()
+    a, b = x[..., :64], x[..., 64:]
+    return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+
+
+# ------------------------------------------------------------------------ oracle timing
+def oracle_sample(wl: synth.Workload, budget_s: float):
+    """Time the CPU oracle on whole (batch row, KV head) units of one layer of the
+    workload: encode the new token, then unpack + reconstruct + attend over the cache."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    m = synth.make_layer_model(wl.h_q, wl.h_kv, wl.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, wl.seed + 1, wl.theta)
+    rates = O.greedy_rates(O.block_energy(q_cal.double().numpy(), k_cal.double().numpy()),
+                           O.lloyd_max_mse_table(), 1, 4, 64 * wl.k_bits)
+    lay = O.make_layout(rates, wl.v_bits, wl.seed)
+    G = wl.h_q // wl.h_kv
+    cap = 64 * math.ceil(wl.length / 64)
+    prepared = []
+    for h in range(min(2, wl.h_kv)):
+        k = synth.key_slice(m, 0, h, wl.length, 0, wl.seed, wl.theta).double().numpy()
+        v = synth.value_slice(m, 0, h, wl.length, wl.seed).double().numpy()
+        q = torch.stack([synth.query_slice(m, 0, h * G + i, 1, wl.length - 1, wl.seed, wl.theta)[0]
+                         for i in range(G)]).double().numpy()
+        prepared.append((k, v, q, O.pack(lay, O.encode(lay, k[:-1], v[:-1]), cap)))
+    units, keys, elapsed = 0, 0, 0.0
+    while elapsed < budget_s:
+        k, v, q, buf = prepared[units % len(prepared)]
+        t0 = time.perf_counter()
+        new = O.encode(lay, k[-1:], v[-1:])                        # the step's append
+        u = O.unpack(lay, buf, wl.length - 1)
+        for key in ("k_codes", "v_codes"):
+            u[key] = np.concatenate([u[key], new[key]])
+        u["k_norms"] = np.concatenate([u["k_norms"], new["k_norms"].astype(np.float32)])
+        u["v_norm"] = np.concatenate([u["v_norm"], new["v_norm"].astype(np.float32)])
+        kh, vh = O.reconstruct(lay, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
+        O.attention(q, kh, vh, 1 / math.sqrt(128))
+        elapsed += time.perf_counter() - t0
+        units += 1
+        keys += wl.length
+    return {"value": keys / elapsed, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{units} (batch row, KV head) unit passes over {len(prepared)} distinct unit(s) of one "
+                      f"layer, {wl.length} cached tokens each: append 1 token + decode attention, {elapsed:.1f} s"}
+
+
+# ------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8b", choices=list(synth.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=None)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    if args.layers:
+        wl = synth.Workload(**{**wl.__dict__, "layers": args.layers})
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        for _ in range(args.warmup):
+            oracle_sample(wl, args.cpu_budget / max(1, args.steps + args.warmup))
+        for _ in range(args.steps):
+            per_step.append(oracle_sample(wl, args.cpu_budget / max(1, args.steps)))
+        v = statistics.median([p["value"] for p in per_step])
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "layers": wl.layers},
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": per_step[0]["cores"], "kind": "oracle",
+                                 "sample": "per step: " + per_step[0]["sample"]},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    model = Model(wl, dev, seed_offset=rank * 100000)
+    stream = torch.cuda.Stream(device=dev)
+
+    # capture one step and the decode-only sequence as CUDA graphs
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            model.step(stream)
+    torch.cuda.synchronize(dev)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        model.step(stream)
+    g_dec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dec, stream=stream):
+        model.decode_only(stream)
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            g_step.replay()
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                g_step.replay()
+            ev1.record(stream)
+        barrier()
+        step_ms = ev0.elapsed_time(ev1) / args.steps
+        # dominant kernel: decode attention, timed on its own stream over the same caches
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            d0.record(stream)
+            for _ in range(args.steps):
+                g_dec.replay()
+            d1.record(stream)
+        barrier()
+        dec_ms = d0.elapsed_time(d1) / (args.steps * wl.layers)
+    clocks = clk.summary()
+
+    # end to end through the public API with host buffers (pinned), copies inside the timing
+    h_q = [x["q"].cpu().pin_memory() for x in model.layers]
+    h_k = [x["k_new"].cpu().pin_memory() for x in model.layers]
+    h_v = [x["v_new"].cpu().pin_memory() for x in model.layers]
+    h_out = [torch.empty_like(x["out"], device="cpu").pin_memory() for x in model.layers]
+    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for i, x in enumerate(model.layers):
+            x["q"].copy_(h_q[i], non_blocking=True)
+            x["k_new"].copy_(h_k[i], non_blocking=True)
+            x["v_new"].copy_(h_v[i], non_blocking=True)
+        g_step.replay()
+        for i, x in enumerate(model.layers):
+            h_out[i].copy_(x["out"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    times = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(times, op=pg.ReduceOp.MAX)
+    step_ms, dec_ms, e2e_ms = times.tolist()
+    del g_step, g_dec
+
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        keys = model.keys_per_step * world
+        dec_bytes = model.bytes_per_step / wl.layers
+        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": keys / (step_ms * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "context": wl.length,
+                       "h_q": wl.h_q, "h_kv": wl.h_kv, "rates": f"K{wl.k_bits}V{wl.v_bits}",
+                       "bytes_per_token_head": model.layers[0]["layout"].bytes_per_token,
+                       "step": "per layer: encode-append 1 token + decode attention; CUDA graph",
+                       "l2": f"inputs larger than L2: {model.bytes_per_step / 1e6:.0f} MB of packed caches per step",
+                       "parallelism": f"replicas x{world} (independent sequences per GPU)"},
+            "gbs": model.bytes_per_step / (step_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "decode_attention (split + combine), per layer launch",
+                         "peak_kind": peak_kind},
+            "clocks": clocks,
+            "gpu_launches": args.steps * wl.layers * 3,
+            "e2e": {"value": keys / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(wl, args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

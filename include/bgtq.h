@@ -1,0 +1,175 @@
+/*
+ * bgtq.h -- C ABI of libbgtq: Block-GTQ / TQ-MSE packed-KV decode attention on B200.
+ *
+ * Sources of the operations (page title, passage):
+ *  [BGTQ] "Block-GTQ: RoPE-Block Rate Allocation for KV-Cache Quantization", abstract:
+ *         s2 RoPE 2-D frequency blocks carry the key precision; s3 label-free query-key
+ *         energy score with codec-dependent rate penalties; s4 largest-marginal-gain
+ *         allocation; s5 TQ-MSE instantiation, equal-rate blocks grouped, attention over
+ *         packed caches without a decoded fp16 KV cache; s7 "K2V2" logical rates;
+ *         s8 no fp16 sink or recent-token buffer.
+ *  [TQ]   "TurboQuant: paper algorithm and vLLM engineering implementation" (pipeline
+ *         diagram): input vector x (per-head K or V) -> random rotation -> per-coordinate
+ *         MSE scalar quantisation with a few centroids; exercise 1: KV memory footprint.
+ *
+ * Conventions for every call:
+ *  - head_dim is 128; RoPE block j (0..63) is the coordinate pair {j, j+64}
+ *    (rotate-half RoPE). Keys are passed AFTER RoPE.
+ *  - All device buffers are allocated and owned by the caller. A layout owns only its
+ *    host tables and, after bgtq_layout_upload, one device allocation of constants.
+ *  - Device calls are asynchronous on the given stream (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream). They never allocate, never synchronise, and check
+ *    every argument before launching; on error nothing is written.
+ *  - A failing call returns a status and leaves a message for bgtq_last_error_string()
+ *    (per host thread). No C++ exception crosses the ABI.
+ *
+ * Packed cache format (one (batch row, KV head) = capacity/64 consecutive tiles):
+ *  tile of 64 tokens = [K records | V codes | K norms | V norms]
+ *   K records: 64 x Kb bytes, token-major, Kb = 128*avg_k_bits/8. A record is an
+ *              LSB-first bitstream (bit n = bit n%8 of byte n/8) of the 128 key codes in
+ *              packed-dimension order: K groups by descending rate; in a group, blocks
+ *              ascending, coordinate j before j+64. A code of rate r takes r bits.
+ *   V codes:   four 16-token chunks of 256*b_V bytes; each an LSB-first bitstream where
+ *              the code of (dimension d, token j of the chunk) starts at bit
+ *              (16*d + slot(j))*b_V, slot(j) = 4*((j%8)/2) + 2*(j/8) + j%2.
+ *   K norms:   n_kgroups x 64 fp32, group-major: |x_g| of each token's group g.
+ *   V norms:   64 fp32.
+ *  tile_bytes = 64*(Kb + 16*b_V) + 256*(n_kgroups + 1).
+ *  A code c of a group with rate r stands for the Lloyd-Max centroid c of N(0,1) with 2^r
+ *  levels (ascending); the coordinate it encodes is y = sqrt(d_g) * (R_g x_g)_i / |x_g|.
+ */
+#ifndef BGTQ_H
+#define BGTQ_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BGTQ_OK = 0,
+  BGTQ_ERR_INVALID = 1,     /* bad argument: null pointer, bad size, unsupported shape */
+  BGTQ_ERR_INFEASIBLE = 2,  /* rate budget outside [n*min_rate, n*max_rate] */
+  BGTQ_ERR_CAPACITY = 3,    /* capacity not a multiple of 64 or too small for the call */
+  BGTQ_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  BGTQ_ERR_NOMEM = 5,       /* host or device allocation failed (layout calls only) */
+  BGTQ_ERR_WORKSPACE = 6,   /* workspace pointer null or smaller than required */
+  BGTQ_ERR_DEVICE = 7       /* layout not uploaded, or uploaded to another device */
+} bgtq_status;
+
+enum { BGTQ_F32 = 0, BGTQ_BF16 = 1, BGTQ_F16 = 2 };
+
+#define BGTQ_HEAD_DIM 128
+#define BGTQ_N_BLOCKS 64
+#define BGTQ_TILE_TOKENS 64
+#define BGTQ_MAX_GQA 8
+#define BGTQ_MAX_KGROUPS 4
+
+/* Device status bits reported by bgtq_device_status. */
+#define BGTQ_STATUS_ENCODE_OVERFLOW 1u  /* encode: seq_len + n_new > capacity; those tokens skipped */
+#define BGTQ_STATUS_DECODE_CLAMPED 2u   /* decode: seq_len > capacity or > max_seq_len; clamped */
+
+typedef struct bgtq_layout bgtq_layout;
+
+typedef struct {
+  int head_dim;                       /* 128 */
+  int n_blocks;                       /* 64 */
+  int n_kgroups;                      /* number of distinct key rates, 1..4 */
+  int group_rate[BGTQ_MAX_KGROUPS];   /* descending */
+  int group_dim[BGTQ_MAX_KGROUPS];    /* d_g = 2 x blocks in the group */
+  int v_rate;
+  int k_record_bytes;                 /* Kb */
+  int v_record_bytes;                 /* 16 * v_rate */
+  int bytes_per_token;                /* Kb + 16 v_rate + 4 (n_kgroups + 1) */
+  int tile_tokens;                    /* 64 */
+  int tile_bytes;
+  unsigned long long seed;
+} bgtq_layout_info;
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* bgtq_last_error_string(void);
+int bgtq_version(void);
+
+/* ---------------------------------------------------------------- host planning ---- */
+
+/* Gaussian Lloyd-Max quantiser [TQ, "per-coordinate MSE scalar quantisation"]:
+ * bits in 1..4; writes 2^bits ascending centroids, 2^bits - 1 thresholds (midpoints,
+ * middle one exactly 0) and the per-coordinate MSE on N(0,1). Any output may be NULL. */
+bgtq_status bgtq_lloyd_max(int bits, double* centroids, double* thresholds, double* mse);
+
+/* Energy score per RoPE block [BGTQ s3]. q_cal [n_q, h_q, 128] and k_cal [n_k, h_kv, 128]
+ * fp32 host arrays (post-RoPE is fine: RoPE rotates inside each block). score_out[64]:
+ * sum over KV heads of (mean over calibration queries and that head's h_q/h_kv query
+ * heads of |q_j|^2) x (mean over calibration keys of |k_j|^2). */
+bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q,
+                              const float* k_cal, long long n_k, int h_kv, double* score_out);
+
+/* Largest-marginal-gain rate allocation [BGTQ s4]. Rates start at min_rate; each step
+ * adds one bit to the block with the largest score[j] * (D[b_j] - D[b_j + 1]) among
+ * blocks below max_rate (ties: lowest j) until the rates sum to total_bits.
+ * distortion: array indexed by rate (entries min_rate..max_rate used), or NULL for the
+ * Gaussian Lloyd-Max MSE. 1 <= min_rate <= max_rate <= 4. BGTQ_ERR_INFEASIBLE if
+ * total_bits is outside [n_blocks*min_rate, n_blocks*max_rate]. rates_out[n_blocks]. */
+bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate, int max_rate,
+                                long long total_bits, const double* distortion, int* rates_out);
+
+/* Layout of one layer [BGTQ s5]: k_rates[64] in 1..4 summing to a multiple of 4 (so a K
+ * record is whole bytes), v_rate in 1..4, seed of the rotations. Groups equal-rate blocks,
+ * draws one seeded Haar rotation per K group (Philox4x32-10 stream = rate) and one for V
+ * (stream 0), and builds the Lloyd-Max tables. Host only. */
+bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long long seed,
+                               bgtq_layout** out);
+void bgtq_layout_destroy(bgtq_layout* layout);
+bgtq_status bgtq_layout_get_info(const bgtq_layout* layout, bgtq_layout_info* info);
+/* Rotation of K group g (0..n_kgroups-1) or of V (g = n_kgroups), row-major d x d fp64,
+ * y = R x. max_elems bounds the write. */
+bgtq_status bgtq_layout_rotation(const bgtq_layout* layout, int group, double* out, long long max_elems);
+/* packed_to_coord[128]: original coordinate of each packed key dimension. */
+bgtq_status bgtq_layout_coords(const bgtq_layout* layout, int* packed_to_coord);
+
+/* Resident bytes of a packed cache [TQ exercise 1]: batch x h_kv x ceil(tokens/64) tiles.
+ * Returns -1 on bad arguments. */
+long long bgtq_cache_bytes(const bgtq_layout* layout, int batch, int h_kv, long long tokens);
+
+/* ---------------------------------------------------------------- device calls ----- */
+
+/* Copies the layout's constants to `device` (one cudaMalloc, freed by destroy). Must
+ * precede the device calls; not for use during stream capture. */
+bgtq_status bgtq_layout_upload(bgtq_layout* layout, int device);
+
+/* TQ-MSE encode and append [TQ pipeline; BGTQ s5]. k, v: [batch, n_new, h_kv, 128]
+ * contiguous, dtype BGTQ_F32/BF16/F16, device memory. seq_lens_dev[batch] int32 device:
+ * the position of token 0 of row b (not modified; the caller advances it). cache: device
+ * buffer of bgtq_cache_bytes(layout, batch, h_kv, capacity) bytes. Tokens whose position
+ * is >= capacity are skipped and set BGTQ_STATUS_ENCODE_OVERFLOW. Writes each token's
+ * K record, V codes and norms; the rest of the cache is untouched. */
+bgtq_status bgtq_encode_append(const bgtq_layout* layout, const void* k, const void* v, int dtype,
+                               int batch, int n_new, int h_kv, const int* seq_lens_dev,
+                               void* cache, long long capacity, void* stream);
+
+/* Workspace bytes that bgtq_decode_attention needs for this shape on the current device
+ * (split-K partials). 0 on bad arguments. */
+size_t bgtq_workspace_bytes(const bgtq_layout* layout, int batch, int h_q, int h_kv,
+                            long long max_seq_len);
+
+/* Single-token decode attention over the packed cache [BGTQ s5, s8]. q [batch, h_q, 128]
+ * (dtype as above, device; query head i uses KV head i / (h_q/h_kv)), cache as written by
+ * bgtq_encode_append, seq_lens_dev[batch] int32 device = number of cached tokens of each
+ * row (0 gives a zero output row), max_seq_len >= every seq_len (plans the split-K grid;
+ * larger lengths are clamped and flagged), softmax_scale (e.g. 1/sqrt(128)).
+ * out [batch, h_q, 128] fp32 device. workspace: device buffer of at least
+ * bgtq_workspace_bytes(...). h_q/h_kv must be 1..8. */
+bgtq_status bgtq_decode_attention(const bgtq_layout* layout, const void* q, int q_dtype,
+                                  int batch, int h_q, int h_kv, const void* cache,
+                                  const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                                  float softmax_scale, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Reads (synchronously) the layout's device status bits; clears them if clear != 0. */
+bgtq_status bgtq_device_status(const bgtq_layout* layout, unsigned* flags, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BGTQ_H */

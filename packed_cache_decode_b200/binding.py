@@ -1,0 +1,259 @@
+"""Thin ctypes binding of libbgtq (include/bgtq.h): argument marshalling only.
+
+Every step of the path runs inside the library. If ``libbgtq.so`` is missing the
+binding raises; there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbgtq.so")
+_lib = None
+
+OK, ERR_INVALID, ERR_INFEASIBLE, ERR_CAPACITY, ERR_CUDA, ERR_NOMEM, ERR_WORKSPACE, ERR_DEVICE = range(8)
+F32, BF16, F16 = 0, 1, 2
+HEAD_DIM = 128
+TILE_TOKENS = 64
+STATUS_ENCODE_OVERFLOW = 1
+STATUS_DECODE_CLAMPED = 2
+
+EXPORTED = [
+    "bgtq_last_error_string", "bgtq_version", "bgtq_lloyd_max", "bgtq_block_energy", "bgtq_allocate_rates",
+    "bgtq_layout_create", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
+    "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
+    "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
+]
+
+
+class LayoutInfo(C.Structure):
+    _fields_ = [("head_dim", C.c_int), ("n_blocks", C.c_int), ("n_kgroups", C.c_int),
+                ("group_rate", C.c_int * 4), ("group_dim", C.c_int * 4), ("v_rate", C.c_int),
+                ("k_record_bytes", C.c_int), ("v_record_bytes", C.c_int), ("bytes_per_token", C.c_int),
+                ("tile_tokens", C.c_int), ("tile_bytes", C.c_int), ("seed", C.c_ulonglong)]
+
+
+class BgtqError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: status {status}: {msg}")
+        self.status = status
+
+
+def load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libbgtq.so not built ({_LIB_PATH}); run python -m packed_cache_decode_b200.build_lib")
+    lib = C.CDLL(_LIB_PATH)
+    P, I, LL, D, F, U = C.c_void_p, C.c_int, C.c_longlong, C.c_double, C.c_float, C.c_ulonglong
+    sig = {
+        "bgtq_last_error_string": (C.c_char_p, []),
+        "bgtq_version": (I, []),
+        "bgtq_lloyd_max": (I, [I, P, P, P]),
+        "bgtq_block_energy": (I, [P, LL, I, P, LL, I, P]),
+        "bgtq_allocate_rates": (I, [P, I, I, I, LL, P, P]),
+        "bgtq_layout_create": (I, [P, I, U, C.POINTER(P)]),
+        "bgtq_layout_destroy": (None, [P]),
+        "bgtq_layout_get_info": (I, [P, C.POINTER(LayoutInfo)]),
+        "bgtq_layout_rotation": (I, [P, I, P, LL]),
+        "bgtq_layout_coords": (I, [P, P]),
+        "bgtq_cache_bytes": (LL, [P, I, I, LL]),
+        "bgtq_layout_upload": (I, [P, I]),
+        "bgtq_encode_append": (I, [P, P, P, I, I, I, I, P, P, LL, P]),
+        "bgtq_workspace_bytes": (C.c_size_t, [P, I, I, I, LL]),
+        "bgtq_decode_attention": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_device_status": (I, [P, C.POINTER(C.c_uint), I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise BgtqError(status, where, load().bgtq_last_error_string().decode())
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+# ---------------------------------------------------------------- host planning
+def lloyd_max(bits: int):
+    c = np.zeros(1 << bits)
+    t = np.zeros((1 << bits) - 1)
+    m = np.zeros(1)
+    _check(load().bgtq_lloyd_max(bits, _ptr(c), _ptr(t), _ptr(m)), "lloyd_max")
+    return c, t, float(m[0])
+
+
+def block_energy(q_cal, k_cal) -> np.ndarray:
+    q = np.ascontiguousarray(q_cal, dtype=np.float32)
+    k = np.ascontiguousarray(k_cal, dtype=np.float32)
+    s = np.zeros(64)
+    _check(load().bgtq_block_energy(_ptr(q), q.shape[0], q.shape[1], _ptr(k), k.shape[0], k.shape[1], _ptr(s)),
+           "block_energy")
+    return s
+
+
+def allocate_rates(score, min_rate: int, max_rate: int, total_bits: int, distortion=None) -> np.ndarray:
+    s = np.ascontiguousarray(score, dtype=np.float64)
+    out = np.zeros(len(s), dtype=np.int32)
+    dptr = None
+    if distortion is not None:
+        d = np.zeros(6)
+        for r, v in dict(distortion).items():
+            d[r] = v
+        dptr = _ptr(d)
+    _check(load().bgtq_allocate_rates(_ptr(s), len(s), min_rate, max_rate, total_bits, dptr, _ptr(out)),
+           "allocate_rates")
+    return out
+
+
+class Layout:
+    """A layer's packing layout (owns the C handle)."""
+
+    def __init__(self, k_rates, v_rate: int, seed: int):
+        lib = load()
+        r = np.ascontiguousarray(k_rates, dtype=np.int32)
+        if r.shape != (64,):
+            raise ValueError("64 block rates expected")
+        h = C.c_void_p()
+        _check(lib.bgtq_layout_create(_ptr(r), int(v_rate), C.c_ulonglong(seed), C.byref(h)), "layout_create")
+        self._h = h
+        self.k_rates = r.copy()
+        self.v_rate = int(v_rate)
+        self.seed = int(seed)
+        info = LayoutInfo()
+        _check(lib.bgtq_layout_get_info(h, C.byref(info)), "layout_get_info")
+        self.info = info
+        self.device = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def n_kgroups(self):
+        return self.info.n_kgroups
+
+    @property
+    def bytes_per_token(self):
+        return self.info.bytes_per_token
+
+    @property
+    def tile_bytes(self):
+        return self.info.tile_bytes
+
+    def rotation(self, group: int) -> np.ndarray:
+        d = self.info.group_dim[group] if group < self.n_kgroups else HEAD_DIM
+        out = np.zeros((d, d))
+        _check(load().bgtq_layout_rotation(self._h, group, _ptr(out), out.size), "layout_rotation")
+        return out
+
+    def coords(self) -> np.ndarray:
+        out = np.zeros(128, dtype=np.int32)
+        _check(load().bgtq_layout_coords(self._h, _ptr(out)), "layout_coords")
+        return out
+
+    def cache_bytes(self, batch: int, h_kv: int, tokens: int) -> int:
+        n = load().bgtq_cache_bytes(self._h, batch, h_kv, tokens)
+        if n < 0:
+            _check(ERR_INVALID, "cache_bytes")
+        return int(n)
+
+    def upload(self, device: int = 0):
+        _check(load().bgtq_layout_upload(self._h, device), "layout_upload")
+        self.device = device
+        return self
+
+    def status(self, clear: bool = True) -> int:
+        f = C.c_uint(0)
+        _check(load().bgtq_device_status(self._h, C.byref(f), int(clear)), "device_status")
+        return int(f.value)
+
+    def close(self):
+        if self._h:
+            load().bgtq_layout_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---------------------------------------------------------------- device calls
+_DTYPES = {}
+
+
+def dtype_code(t) -> int:
+    import torch
+    if not _DTYPES:
+        _DTYPES.update({torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16})
+    return _DTYPES[t.dtype]
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def encode_append(layout: Layout, k, v, seq_lens, cache, capacity: int, stream=None):
+    """k, v [B, n_new, h_kv, 128] CUDA tensors; seq_lens [B] int32 CUDA; cache uint8 CUDA."""
+    B, n_new, h_kv, d = k.shape
+    assert d == HEAD_DIM and k.is_contiguous() and v.is_contiguous() and v.shape == k.shape and v.dtype == k.dtype
+    _check(load().bgtq_encode_append(layout.handle, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()),
+                                     dtype_code(k), B, n_new, h_kv, C.c_void_p(seq_lens.data_ptr()),
+                                     C.c_void_p(cache.data_ptr()), capacity, _stream_ptr(stream)),
+           "encode_append")
+
+
+def workspace_bytes(layout: Layout, batch: int, h_q: int, h_kv: int, max_seq_len: int) -> int:
+    n = load().bgtq_workspace_bytes(layout.handle, batch, h_q, h_kv, max_seq_len)
+    if n == 0:
+        _check(ERR_INVALID, "workspace_bytes")
+    return int(n)
+
+
+def decode_attention(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out, workspace,
+                     h_kv: int, softmax_scale: float | None = None, stream=None):
+    """q [B, h_q, 128] CUDA; out [B, h_q, 128] fp32 CUDA; workspace uint8 CUDA."""
+    B, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B, h_q, h_kv,
+                                        C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                        max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                        C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_attention")
+
+
+@dataclass
+class PackedLayer:
+    """One layer's packed cache and the device buffers its calls need (caller-owned)."""
+
+    layout: Layout
+    cache: object
+    seq_lens: object
+    capacity: int
+    batch: int
+    h_q: int
+    h_kv: int
+    workspace: object = None
+    out: object = None
+
+
+def plan_layer_rates(q_cal, k_cal, avg_bits: int, min_rate: int = 1, max_rate: int = 4) -> np.ndarray:
+    """Energy score + largest-marginal-gain allocation for one layer (library calls)."""
+    s = block_energy(q_cal, k_cal)
+    return allocate_rates(s, min_rate, max_rate, 64 * avg_bits)

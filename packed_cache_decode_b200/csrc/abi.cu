@@ -1,0 +1,191 @@
+// Device-side entry points of the C ABI (include/bgtq.h): layout upload, encode-append,
+// decode attention, workspace sizing and the device status word. Every argument is
+// checked before anything is launched; CUDA errors are mapped to BGTQ_ERR_CUDA.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "bgtq_internal.h"
+#include "kernels.h"
+
+using namespace bgtq;
+
+namespace {
+
+bgtq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(BGTQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool valid_dtype(int d) { return d == BGTQ_F32 || d == BGTQ_BF16 || d == BGTQ_F16; }
+
+bgtq_status check_device(const bgtq_layout* L, const char* who) {
+  if (!L) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null layout");
+  if (L->device < 0 || !L->dev_block)
+    return fail(BGTQ_ERR_DEVICE, std::string(who) + ": layout not uploaded (bgtq_layout_upload)");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  if (cur != L->device) return fail(BGTQ_ERR_DEVICE, std::string(who) + ": layout lives on another device");
+  return BGTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void bgtq_layout_destroy(bgtq_layout* L) {
+  if (!L) return;
+  if (L->dev_block) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != L->device) cudaSetDevice(L->device);
+    cudaFree(L->dev_block);
+    if (cur >= 0 && cur != L->device) cudaSetDevice(cur);
+  }
+  delete L;
+}
+
+bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
+  if (!L) return fail(BGTQ_ERR_INVALID, "layout_upload: null layout");
+  if (L->dev_block) return fail(BGTQ_ERR_INVALID, "layout_upload: already uploaded");
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess) return cuda_fail(e, "layout_upload");
+  if (device < 0 || device >= ndev) return fail(BGTQ_ERR_INVALID, "layout_upload: bad device");
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (cur != device && (e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "layout_upload");
+
+  const int ng = L->n_kgroups;
+  size_t n64 = 0;
+  for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
+  const size_t bytes = 256 + n64 * sizeof(double) + n64 * sizeof(float) + 256;
+  std::vector<unsigned char> host(bytes, 0);
+  void* dblock = nullptr;
+  if ((e = cudaMalloc(&dblock, bytes)) != cudaSuccess) {
+    if (cur != device) cudaSetDevice(cur);
+    return fail(BGTQ_ERR_NOMEM, std::string("layout_upload: ") + cudaGetErrorString(e));
+  }
+  DevLayout& D = L->dev;
+  std::memset(&D, 0, sizeof(D));
+  unsigned char* dptr = static_cast<unsigned char*>(dblock);
+  size_t off = 256;  // status word first
+  D.status = reinterpret_cast<unsigned*>(dptr);
+  for (int g = 0; g <= ng; ++g) {
+    std::memcpy(host.data() + off, L->rot[g].data(), L->rot[g].size() * sizeof(double));
+    const double* p = reinterpret_cast<const double*>(dptr + off);
+    if (g < ng) D.k_rot64[g] = p; else D.v_rot64 = p;
+    off += L->rot[g].size() * sizeof(double);
+  }
+  for (int g = 0; g <= ng; ++g) {
+    float* h32 = reinterpret_cast<float*>(host.data() + off);
+    for (size_t i = 0; i < L->rot[g].size(); ++i) h32[i] = float(L->rot[g][i]);
+    const float* p = reinterpret_cast<const float*>(dptr + off);
+    if (g < ng) D.k_rot32[g] = p; else D.v_rot32 = p;
+    off += L->rot[g].size() * sizeof(float);
+  }
+  D.n_kgroups = ng;
+  D.v_rate = L->v_rate;
+  D.k_record_bytes = L->k_record_bytes;
+  D.tile_bytes = L->tile_bytes;
+  D.vcode_off = kTile * L->k_record_bytes;
+  D.knorm_off = D.vcode_off + kTile * L->v_record_bytes;
+  D.vnorm_off = D.knorm_off + 4 * kTile * ng;
+  for (int g = 0; g < kMaxGroups; ++g) {
+    D.group_rate[g] = L->group_rate[g];
+    D.group_dim[g] = L->group_dim[g];
+    D.group_off[g] = L->group_off[g];
+    D.group_bitoff[g] = L->group_bitoff[g];
+  }
+  for (int p = 0; p < kD; ++p) D.packed_coord[p] = short(L->packed_coord[p]);
+  for (int r = 0; r < 5; ++r)
+    for (int i = 0; i < 16; ++i) {
+      D.centroid[r][i] = float(L->centroid[r][i]);
+      D.threshold[r][i] = L->threshold[r][i];
+    }
+  e = cudaMemcpy(dblock, host.data(), bytes, cudaMemcpyHostToDevice);
+  if (cur != device) cudaSetDevice(cur);
+  if (e != cudaSuccess) {
+    cudaFree(dblock);
+    return cuda_fail(e, "layout_upload");
+  }
+  L->dev_block = dblock;
+  L->device = device;
+  return BGTQ_OK;
+}
+
+bgtq_status bgtq_encode_append(const bgtq_layout* L, const void* k, const void* v, int dtype, int batch,
+                               int n_new, int h_kv, const int* seq_lens_dev, void* cache, long long capacity,
+                               void* stream) {
+  bgtq_status st = check_device(L, "encode_append");
+  if (st != BGTQ_OK) return st;
+  if (!valid_dtype(dtype)) return fail(BGTQ_ERR_INVALID, "encode_append: bad dtype");
+  if (batch <= 0 || batch > 65535 || h_kv <= 0 || h_kv > 65535 || n_new < 0)
+    return fail(BGTQ_ERR_INVALID, "encode_append: bad batch / h_kv / n_new");
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, "encode_append: capacity must be a positive multiple of 64");
+  if (n_new == 0) return BGTQ_OK;
+  if (!k || !v || !seq_lens_dev || !cache) return fail(BGTQ_ERR_INVALID, "encode_append: null pointer");
+  cudaError_t e = launch_tq_encode(L->dev, k, v, dtype, batch, n_new, h_kv, seq_lens_dev, cache,
+                                   capacity / kTile, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "encode_append");
+  return BGTQ_OK;
+}
+
+size_t bgtq_workspace_bytes(const bgtq_layout* L, int batch, int h_q, int h_kv, long long max_seq_len) {
+  if (!L || batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG || max_seq_len < 0) {
+    set_error("workspace_bytes: bad arguments");
+    return 0;
+  }
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    set_error("workspace_bytes: no CUDA device");
+    return 0;
+  }
+  return plan_decode(batch, h_q, h_kv, max_seq_len, sms).workspace_bytes;
+}
+
+bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q, int h_kv,
+                                  const void* cache, const int* seq_lens_dev, long long capacity,
+                                  long long max_seq_len, float softmax_scale, float* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_device(L, "decode_attention");
+  if (st != BGTQ_OK) return st;
+  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_attention: bad dtype");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
+    return fail(BGTQ_ERR_INVALID, "decode_attention: need h_q = G * h_kv with G in 1..8");
+  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_attention: batch * h_kv > 65535");
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, "decode_attention: capacity must be a positive multiple of 64");
+  if (max_seq_len < 0 || max_seq_len > capacity)
+    return fail(BGTQ_ERR_CAPACITY, "decode_attention: max_seq_len must be in [0, capacity]");
+  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_attention: bad softmax_scale");
+  if (!q || !cache || !seq_lens_dev || !out) return fail(BGTQ_ERR_INVALID, "decode_attention: null pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attention");
+  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  if (!workspace || workspace_bytes < plan.workspace_bytes)
+    return fail(BGTQ_ERR_WORKSPACE, "decode_attention: workspace missing or smaller than bgtq_workspace_bytes()");
+  e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, cache, seq_lens_dev, capacity / kTile,
+                    softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attention");
+  return BGTQ_OK;
+}
+
+bgtq_status bgtq_device_status(const bgtq_layout* L, unsigned* flags, int clear) {
+  bgtq_status st = check_device(L, "device_status");
+  if (st != BGTQ_OK) return st;
+  if (!flags) return fail(BGTQ_ERR_INVALID, "device_status: null pointer");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(flags, L->dev.status, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && clear) e = cudaMemset(L->dev.status, 0, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "device_status");
+  return BGTQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+// Internal types shared by the host planner, the ABI layer and the kernels of libbgtq.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/bgtq.h"
+
+namespace bgtq {
+
+constexpr int kD = BGTQ_HEAD_DIM;        // 128
+constexpr int kBlocks = BGTQ_N_BLOCKS;   // 64
+constexpr int kTile = BGTQ_TILE_TOKENS;  // 64 tokens per tile
+constexpr int kChunk = 16;               // tokens per V-code chunk
+constexpr int kMaxG = BGTQ_MAX_GQA;
+constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
+
+// Everything a kernel needs about one layer's packing, passed by value.
+struct DevLayout {
+  int n_kgroups;
+  int v_rate;
+  int k_record_bytes;   // Kb
+  int tile_bytes;
+  int vcode_off;        // byte offsets inside a tile
+  int knorm_off;
+  int vnorm_off;
+  int group_rate[kMaxGroups];
+  int group_dim[kMaxGroups];
+  int group_off[kMaxGroups];     // first packed dimension of the group
+  int group_bitoff[kMaxGroups];  // first bit of the group inside a K record
+  short packed_coord[kD];        // packed key dimension -> original coordinate
+  float centroid[5][16];         // [rate][code], fp32
+  double threshold[5][16];       // [rate][k], fp64 (2^rate - 1 used)
+  const double* k_rot64[kMaxGroups];  // d_g x d_g row-major, y = R x
+  const double* v_rot64;
+  const float* k_rot32[kMaxGroups];
+  const float* v_rot32;
+  unsigned* status;
+};
+
+}  // namespace bgtq
+
+struct bgtq_layout {
+  int k_rates[bgtq::kBlocks];
+  int v_rate;
+  unsigned long long seed;
+  int n_kgroups;
+  int group_rate[bgtq::kMaxGroups];
+  int group_dim[bgtq::kMaxGroups];
+  int group_off[bgtq::kMaxGroups];
+  int group_bitoff[bgtq::kMaxGroups];
+  int packed_coord[bgtq::kD];
+  std::vector<double> rot[bgtq::kMaxGroups + 1];  // K groups, then V at index n_kgroups
+  double centroid[5][16];
+  double threshold[5][16];
+  double mse[5];
+  int k_record_bytes, v_record_bytes, bytes_per_token, tile_bytes;
+  // device copy
+  int device = -1;
+  void* dev_block = nullptr;
+  bgtq::DevLayout dev{};
+};
+
+namespace bgtq {
+void set_error(const std::string& msg);
+bgtq_status fail(bgtq_status s, const std::string& msg);
+// Host Lloyd-Max, also used by the layout builder.
+void lloyd_max_host(int bits, double* centroids, double* thresholds, double* mse);
+}  // namespace bgtq

@@ -1,0 +1,116 @@
+"""Shared pieces of the parity tests: build one layer's inputs, run the CUDA path through
+the C ABI, run the oracle, and compare the two."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+import oracle as O
+from packed_cache_decode_b200 import binding as B
+from packed_cache_decode_b200 import synth
+
+CODE_EPS = 1e-6        # coordinates this close to a threshold may code either way
+ATTN_REL_L2 = 2e-3     # attention output tolerance (relative L2 per query head)
+
+
+@dataclass
+class Case:
+    h_q: int
+    h_kv: int
+    batch: int
+    length: int
+    k_bits: int
+    v_bits: int
+    dtype: torch.dtype = torch.bfloat16
+    theta: float = 5e5
+    seed: int = 0
+    scale_v: bool = False
+    capacity: int | None = None
+
+    @property
+    def cap(self):
+        return self.capacity or 64 * math.ceil(self.length / 64)
+
+
+def oracle_rates(model, case: Case) -> np.ndarray:
+    """Per-layer rates from 256 calibration tokens (seed + 1), computed by the oracle."""
+    q_cal, k_cal = synth.make_calibration(model, 256, case.seed + 1, case.theta)
+    s = O.block_energy(q_cal.double().numpy(), k_cal.double().numpy())
+    return O.greedy_rates(s, O.lloyd_max_mse_table(), 1, 4, 64 * case.k_bits)
+
+
+def build_inputs(case: Case):
+    model = synth.make_layer_model(case.h_q, case.h_kv, case.seed, scale_v=case.scale_v)
+    rates = oracle_rates(model, case)
+    q, k, v = synth.make_cache_inputs(model, case.batch, case.length, case.seed, case.theta, case.dtype)
+    return model, rates, q, k, v
+
+
+def gpu_encode(case: Case, rates, k, v, n_chunks: int = 1, layout=None):
+    """Encode-append all tokens on the GPU (in n_chunks appends); returns (layout, cache)."""
+    lay = layout or B.Layout(rates, case.v_bits, case.seed).upload(0)
+    cap = case.cap
+    cache = torch.zeros(lay.cache_bytes(case.batch, case.h_kv, cap), dtype=torch.uint8, device="cuda")
+    kd, vd = k.cuda(), v.cuda()
+    bounds = np.linspace(0, case.length, n_chunks + 1).astype(int)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if b == a:
+            continue
+        lens = torch.full((case.batch,), int(a), dtype=torch.int32, device="cuda")
+        B.encode_append(lay, kd[:, a:b].contiguous(), vd[:, a:b].contiguous(), lens, cache, cap)
+    torch.cuda.synchronize()
+    return lay, cache
+
+
+def gpu_decode(lay, case: Case, q, cache, seq_lens=None, max_seq_len=None, scale=None):
+    lens = torch.full((case.batch,), case.length, dtype=torch.int32) if seq_lens is None else seq_lens
+    lens = lens.to(torch.int32).cuda()
+    msl = case.length if max_seq_len is None else max_seq_len
+    ws = torch.empty(B.workspace_bytes(lay, case.batch, case.h_q, case.h_kv, msl), dtype=torch.uint8, device="cuda")
+    out = torch.full((case.batch, case.h_q, 128), float("nan"), dtype=torch.float32, device="cuda")
+    B.decode_attention(lay, q.cuda().contiguous(), cache, lens, case.cap, msl, out, ws, case.h_kv, scale)
+    torch.cuda.synchronize()
+    return out.cpu().double().numpy()
+
+
+def oracle_slice(case: Case, rates, k, v, b: int, h: int, n: int | None = None):
+    lay = O.make_layout(rates, case.v_bits, case.seed)
+    n = case.length if n is None else n
+    enc = O.encode(lay, k[b, :n, h].double().numpy(), v[b, :n, h].double().numpy())
+    buf = O.pack(lay, enc, case.cap)
+    return lay, enc, buf
+
+
+def slice_bytes(case: Case, lay_bytes_per_tile: int, cache_cpu: np.ndarray, b: int, h: int) -> np.ndarray:
+    n_tiles = case.cap // 64
+    per = n_tiles * lay_bytes_per_tile
+    u = b * case.h_kv + h
+    return cache_cpu[u * per:(u + 1) * per]
+
+
+def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, capacity: int):
+    """Codes bit-exact except near-threshold coordinates; norms to 1 fp32 ulp.
+    Returns (near-boundary count, how many of those differ)."""
+    mask, n_near = O.boundary_mask(lay, enc, capacity, CODE_EPS)
+    nt = capacity // 64
+    tb = lay.tile_bytes
+    code_bytes = 64 * (lay.k_record_bytes + lay.v_record_bytes)
+    w = want.reshape(nt, tb)
+    g = got.reshape(nt, tb)
+    m = mask.reshape(nt, tb)
+    diff = (w[:, :code_bytes] ^ g[:, :code_bytes]) & ~m[:, :code_bytes]
+    bad = np.argwhere(diff != 0)
+    assert bad.size == 0, f"{len(bad)} code bytes differ away from thresholds, first at tile/byte {bad[:5].tolist()}"
+    wn = w[:, code_bytes:].copy().view(np.float32)
+    gn = g[:, code_bytes:].copy().view(np.float32)
+    ulp = np.abs(wn.view(np.int32).astype(np.int64) - gn.view(np.int32).astype(np.int64))
+    assert ulp.max() <= 1, f"norm differs by {ulp.max()} ulp"
+    near_diff = int(np.count_nonzero((w[:, :code_bytes] ^ g[:, :code_bytes]) & m[:, :code_bytes]))
+    return n_near, near_diff
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))

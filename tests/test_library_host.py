@@ -1,0 +1,135 @@
+"""The C-ABI library's host-side planning against the oracle (no GPU needed), and the
+library's exported symbols against include/bgtq.h."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from packed_cache_decode_b200 import binding as B
+from packed_cache_decode_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "bgtq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bgtq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(B.EXPORTED) == names
+
+
+def test_lloyd_max_matches_oracle(lib):
+    for b in (1, 2, 3, 4):
+        c, t, m = B.lloyd_max(b)
+        oc, ot, om = O.lloyd_max(b)
+        np.testing.assert_allclose(c, oc, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(t, ot, rtol=0, atol=1e-13)
+        assert m == pytest.approx(om, rel=1e-12)
+        assert t[len(t) // 2] == 0.0
+    with pytest.raises(B.BgtqError):
+        B.lloyd_max(5)
+
+
+def _k2_rates():
+    return np.array([1] * 22 + [2] * 22 + [3] * 18 + [4] * 2)
+
+
+@pytest.mark.parametrize("seed", [0, 12345, 2**40 + 7])
+def test_layout_matches_oracle(lib, seed):
+    rng = np.random.default_rng(seed % 1000)
+    rates = rng.permutation(_k2_rates())
+    lay = B.Layout(rates, 3, seed)
+    ref = O.make_layout(rates, 3, seed)
+    assert lay.n_kgroups == ref.n_kgroups
+    assert lay.bytes_per_token == ref.bytes_per_token and lay.tile_bytes == ref.tile_bytes
+    assert lay.info.k_record_bytes == ref.k_record_bytes
+    np.testing.assert_array_equal(lay.coords(), ref.packed_coords())
+    for g, (r, coords) in enumerate(ref.groups):
+        assert lay.info.group_rate[g] == r and lay.info.group_dim[g] == len(coords)
+        np.testing.assert_allclose(lay.rotation(g), ref.k_rot[g], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lay.rotation(lay.n_kgroups), ref.v_rot, rtol=0, atol=1e-12)
+    for tokens in (1, 64, 65, 32768):
+        assert lay.cache_bytes(2, 8, tokens) == O.cache_bytes(ref, 2, 8, tokens)
+
+
+def test_rotation_preserves_norms_to_1e6(lib):
+    lay = B.Layout(_k2_rates(), 2, 7)
+    x = np.random.default_rng(0).standard_normal((100, 128))
+    for g in range(lay.n_kgroups + 1):
+        r = lay.rotation(g)
+        r32 = r.astype(np.float32).astype(np.float64)   # the decode kernels use the fp32 copy
+        d = r.shape[0]
+        for rr in (r, r32):
+            ratio = np.linalg.norm(x[:, :d] @ rr.T, axis=1) / np.linalg.norm(x[:, :d], axis=1)
+            assert np.max(np.abs(ratio - 1)) < 1e-6
+        assert np.max(np.abs(r32 @ r32.T - np.eye(d))) < 1e-6
+
+
+def test_layout_rejects_bad_rates(lib):
+    with pytest.raises(B.BgtqError):
+        B.Layout(np.array([1] * 63 + [2]), 2, 0)          # 130 bits
+    with pytest.raises(B.BgtqError):
+        B.Layout(np.array([0] * 64), 2, 0)
+    with pytest.raises(B.BgtqError):
+        B.Layout(np.full(64, 2), 5, 0)
+
+
+def test_block_energy_matches_oracle(lib):
+    m = synth.make_layer_model(32, 8, seed=1)
+    q, k = synth.make_calibration(m, 256, 2, 5e5)
+    s_lib = B.block_energy(q.numpy(), k.numpy())
+    s_ref = O.block_energy(q.numpy().astype(np.float64), k.numpy().astype(np.float64))
+    np.testing.assert_allclose(s_lib, s_ref, rtol=1e-12)
+
+
+def test_allocation_matches_oracle_greedy(lib):
+    rng = np.random.default_rng(2)
+    D = O.lloyd_max_mse_table()
+    for trial in range(20):
+        s = rng.exponential(size=64) * rng.choice([0.01, 1, 100], size=64)
+        if trial % 5 == 0:
+            s[:20] = 3.0                                  # ties
+        for avg in (1, 2, 3, 4):
+            want = O.greedy_rates(s, D, 1, 4, 64 * avg)
+            got = B.allocate_rates(s, 1, 4, 64 * avg)
+            np.testing.assert_array_equal(got, want)
+        budget = int(rng.integers(64, 257))
+        np.testing.assert_array_equal(B.allocate_rates(s, 1, 4, budget), O.greedy_rates(s, D, 1, 4, budget))
+
+
+def test_allocation_custom_distortion_and_errors(lib):
+    s = np.array([5.0, 1.0, 3.0, 0.5])
+    D = {1: 1.0, 2: 0.5, 3: 0.3, 4: 0.2}
+    np.testing.assert_array_equal(B.allocate_rates(s, 1, 4, 9, D), O.greedy_rates(s, D, 1, 4, 9))
+    with pytest.raises(B.BgtqError) as e:
+        B.allocate_rates(s, 1, 4, 17)
+    assert e.value.status == B.ERR_INFEASIBLE
+    with pytest.raises(B.BgtqError) as e:
+        B.allocate_rates(s, 2, 1, 6)
+    assert e.value.status == B.ERR_INVALID
+
+
+def test_host_validation_without_device(lib):
+    lay = B.Layout(np.full(64, 2), 2, 0)
+    assert lib.bgtq_block_energy(None, 1, 1, None, 1, 1, None) == B.ERR_INVALID
+    assert lib.bgtq_cache_bytes(None, 1, 1, 1) == -1
+    assert lib.bgtq_layout_rotation(lay.handle, 9, None, 0) == B.ERR_INVALID
+    # device calls before an upload report DEVICE, never crash
+    f = C.c_uint(0)
+    assert lib.bgtq_device_status(lay.handle, C.byref(f), 0) == B.ERR_DEVICE
+    assert lib.bgtq_encode_append(lay.handle, None, None, 0, 1, 1, 1, None, None, 64, None) == B.ERR_DEVICE
+    assert lib.bgtq_decode_attention(lay.handle, None, 0, 1, 1, 1, None, None, 64, 64, 0.1, None, None, 0,
+                                     None) == B.ERR_DEVICE
+    if not torch.cuda.is_available():
+        assert lib.bgtq_layout_upload(lay.handle, 0) in (B.ERR_CUDA, B.ERR_INVALID)
