@@ -166,6 +166,28 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* layout, const void* q, int 
                                   float softmax_scale, float* out, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- no-allocation variant */
+
+/* The pages have no counterpart to this call: it is a library convenience.
+ * bgtq_decode_attention without the workspace argument, for callers that cannot call
+ * cudaMalloc (an inference server that gives all device memory to its own pool at
+ * start-up, a plugin whose framework forbids allocation inside its execute callback,
+ * a fixed and audited memory budget). The split-K scratch is one file-scope device array
+ * of BGTQ_NOALLOC_SCRATCH_BYTES (8 MiB), held on every GPU that loads the library until
+ * exit; shapes whose scratch would exceed it return BGTQ_ERR_WORKSPACE with a message.
+ * Nothing is allocated. The first call on a device looks up the array's device address
+ * (once per device, that device current): make it before any stream capture. All calls
+ * share the array, so calls whose kernels overlap on the GPU race and give wrong
+ * results; serialise them (one stream). Arguments and results as bgtq_decode_attention. */
+#define BGTQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+bgtq_status bgtq_decode_attention_noalloc(const bgtq_layout* layout, const void* q, int q_dtype,
+                                          int batch, int h_q, int h_kv, const void* cache,
+                                          const int* seq_lens_dev, long long capacity,
+                                          long long max_seq_len, float softmax_scale, float* out,
+                                          void* stream);
+/* BGTQ_NOALLOC_SCRATCH_BYTES, as compiled into the library. */
+size_t bgtq_noalloc_scratch_capacity(void);
+
 /* Reads (synchronously) the layout's device status bits; clears them if clear != 0. */
 bgtq_status bgtq_device_status(const bgtq_layout* layout, unsigned* flags, int clear);
 

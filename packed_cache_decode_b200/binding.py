@@ -26,6 +26,7 @@ EXPORTED = [
     "bgtq_layout_create", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
     "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
+    "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity",
 ]
 
 
@@ -67,6 +68,8 @@ def load():
         "bgtq_workspace_bytes": (C.c_size_t, [P, I, I, I, LL]),
         "bgtq_decode_attention": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
         "bgtq_device_status": (I, [P, C.POINTER(C.c_uint), I]),
+        "bgtq_decode_attention_noalloc": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P]),
+        "bgtq_noalloc_scratch_capacity": (C.c_size_t, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -236,6 +239,21 @@ def decode_attention(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_
                                         max_seq_len, scale, C.c_void_p(out.data_ptr()),
                                         C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_attention")
+
+
+def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out,
+                             h_kv: int, softmax_scale: float | None = None, stream=None):
+    """decode_attention for callers that cannot allocate device memory: the split-K
+    scratch is the library's fixed device array, not a caller workspace. Calls that
+    overlap on the GPU race on that array, so keep them on one stream."""
+    B_, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_noalloc(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q,
+                                                h_kv, C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()),
+                                                capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                                _stream_ptr(stream)),
+           "decode_attention_noalloc")
 
 
 @dataclass
