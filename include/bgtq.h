@@ -69,6 +69,8 @@ enum { BGTQ_F32 = 0, BGTQ_BF16 = 1, BGTQ_F16 = 2 };
 /* Device status bits reported by bgtq_device_status. */
 #define BGTQ_STATUS_ENCODE_OVERFLOW 1u  /* encode: seq_len + n_new > capacity; those tokens skipped */
 #define BGTQ_STATUS_DECODE_CLAMPED 2u   /* decode: seq_len > capacity or > max_seq_len; clamped */
+#define BGTQ_STATUS_TIMEOUT 4u          /* decode: a bulk copy did not complete within the kernel's bounded
+                                           wait; that call's output is invalid */
 
 typedef struct bgtq_layout bgtq_layout;
 

@@ -19,7 +19,7 @@ BUILD = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3,-Wall", "-I", os.path.join(ROOT, "include")]
-SOURCES = ["host_plan.cpp", "abi.cu", "encode.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["host_plan.cpp", "abi.cu", "encode.cu", "decode_mma.cu", "noalloc.cu"]
 HEADERS = ["bgtq_internal.h", "kernels.h"]
 
 
@@ -43,7 +43,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if src.endswith(".cpp"):
                 cmd = ["g++", "-O3", "-std=c++17", "-fPIC", "-Wall", "-I", os.path.join(ROOT, "include"),
                        "-c", path, "-o", obj]
-            if verbose:
+            if verbose and not src.endswith(".cpp"):
                 cmd.insert(1, "-Xptxas=-v")
                 print(" ".join(cmd), flush=True)
             subprocess.run(cmd, check=True)

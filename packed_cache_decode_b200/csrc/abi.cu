@@ -1,6 +1,7 @@
 // Device-side entry points of the C ABI (include/bgtq.h): layout upload, encode-append,
 // decode attention, workspace sizing and the device status word. Every argument is
 // checked before anything is launched; CUDA errors are mapped to BGTQ_ERR_CUDA.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -20,6 +21,45 @@ bgtq_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 bool valid_dtype(int d) { return d == BGTQ_F32 || d == BGTQ_BF16 || d == BGTQ_F16; }
+
+// Nearest fp16 value of v (round half to even), as a double.
+double round_fp16(double v) {
+  if (v == 0.0) return 0.0;
+  const double a = std::fabs(v);
+  const int e = std::max(int(std::floor(std::log2(a))), -14);
+  const double ulp = std::ldexp(1.0, e - 10);
+  return std::copysign(std::nearbyint(a / ulp) * ulp, v);
+}
+
+unsigned short fp16_bits(double v) {
+  __half h = __float2half_rn(float(v));
+  return *reinterpret_cast<unsigned short*>(&h);
+}
+
+unsigned pack_half2(double lo, double hi) { return unsigned(fp16_bits(lo)) | (unsigned(fp16_bits(hi)) << 16); }
+
+// Scale kappa_r such that fp16(kappa_r * c) represents the rate-r codebook as exactly as
+// possible: +-1 for rate 1; otherwise the best of the 1024 scales that map the outer
+// magnitude to an integer in [1024, 2048) (max relative error 2.3e-7 at rate 2, 1.8e-5
+// at rate 3, 9.3e-5 at rate 4).
+double codebook_kappa(const double* c, int r) {
+  const int m = 1 << (r - 1);
+  if (r == 1) return 1.0 / c[m];
+  double best = 1.0, best_err = INFINITY;
+  for (int A = 1024; A < 2048; ++A) {
+    const double k = A / c[2 * m - 1];
+    double err = 0.0;
+    for (int i = m; i < 2 * m; ++i) {
+      const double v = k * c[i];
+      err = std::max(err, std::fabs(round_fp16(v) - v) / v);
+    }
+    if (err < best_err) {
+      best_err = err;
+      best = k;
+    }
+  }
+  return best;
+}
 
 bgtq_status check_device(const bgtq_layout* L, const char* who) {
   if (!L) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null layout");
@@ -62,7 +102,8 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t bytes = 256 + n64 * sizeof(double) + n64 * sizeof(float) + 256;
+  const size_t lut_words = 20 + 2 * (64 + 256) + 256;
+  const size_t bytes = 256 + n64 * sizeof(double) + 2 * n64 * sizeof(float) + lut_words * 4 + 256;
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
   if ((e = cudaMalloc(&dblock, bytes)) != cudaSuccess) {
@@ -86,6 +127,63 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     const float* p = reinterpret_cast<const float*>(dptr + off);
     if (g < ng) D.k_rot32[g] = p; else D.v_rot32 = p;
     off += L->rot[g].size() * sizeof(float);
+  }
+  for (int g = 0; g < ng; ++g) {
+    const int d = L->group_dim[g];
+    float* h32 = reinterpret_cast<float*>(host.data() + off);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) h32[size_t(j) * d + i] = float(L->rot[g][size_t(i) * d + j]);
+    D.k_rot32t[g] = reinterpret_cast<const float*>(dptr + off);
+    off += L->rot[g].size() * sizeof(float);
+  }
+  {
+    // pair tables for the tensor-core decode
+    unsigned* w = reinterpret_cast<unsigned*>(host.data() + off);
+    // keys: rates 1-2 scaled (exact), rates 3-4 carry an explicit low part (kappa 1);
+    // values: one fp16 table, scaled by the best kappa of the value rate
+    double kap[5] = {1, 1, 1, 1, 1};
+    for (int r = 1; r <= 2; ++r) kap[r] = codebook_kappa(L->centroid[r], r);
+    const double kap_v = codebook_kappa(L->centroid[L->v_rate], L->v_rate);
+    for (int r = 1; r <= 2; ++r)
+      for (int idx = 0; idx < (1 << (2 * r)); ++idx) {
+        const int a = idx & ((1 << r) - 1), b = idx >> r;
+        w[(r == 1 ? 0 : 4) + idx] = pack_half2(kap[r] * L->centroid[r][a], kap[r] * L->centroid[r][b]);
+      }
+    for (int r = 3; r <= 4; ++r)
+      for (int idx = 0; idx < (1 << (2 * r)); ++idx) {
+        const int a = idx & ((1 << r) - 1), b = idx >> r;
+        const double ca = L->centroid[r][a], cb = L->centroid[r][b];
+        const double ha = double(__half2float(__float2half_rn(float(ca))));
+        const double hb = double(__half2float(__float2half_rn(float(cb))));
+        unsigned* e = w + 20 + 2 * ((r == 3 ? 0 : 64) + idx);
+        e[0] = pack_half2(ha, hb);
+        e[1] = pack_half2(ca - ha, cb - hb);
+      }
+    for (int idx = 0; idx < (1 << (2 * L->v_rate)); ++idx) {
+      const int a = idx & ((1 << L->v_rate) - 1), b = idx >> L->v_rate;
+      w[20 + 2 * 320 + idx] = pack_half2(kap_v * L->centroid[L->v_rate][a], kap_v * L->centroid[L->v_rate][b]);
+    }
+    D.klut12 = reinterpret_cast<const unsigned*>(dptr + off);
+    D.klut34 = reinterpret_cast<const unsigned*>(dptr + off + 20 * 4);
+    D.vlut = reinterpret_cast<const unsigned*>(dptr + off + (20 + 2 * 320) * 4);
+    for (int r = 0; r < 5; ++r) D.kappa[r] = float(kap[r]);
+    D.kappa_v = float(kap_v);
+    off += lut_words * 4;
+  }
+  {
+    int ci = 0;
+    for (int g = 0; g < ng; ++g) {
+      const int r = L->group_rate[g], d = L->group_dim[g];
+      D.group_chunk0[g] = ci;
+      D.group_nchunks[g] = (d + 15) / 16;
+      for (int cc = 0; cc < D.group_nchunks[g]; ++cc, ++ci) {
+        D.chunk_bit[ci] = L->group_bitoff[g] + 16 * cc * r;
+        D.chunk_dim0[ci] = L->group_off[g] + 16 * cc;
+        D.chunk_ndim[ci] = std::min(16, d - 16 * cc);
+        D.chunk_group[ci] = g;
+      }
+    }
+    D.n_kchunks = ci;
   }
   D.n_kgroups = ng;
   D.v_rate = L->v_rate;

@@ -15,6 +15,7 @@ constexpr int kTile = BGTQ_TILE_TOKENS;  // 64 tokens per tile
 constexpr int kChunk = 16;               // tokens per V-code chunk
 constexpr int kMaxG = BGTQ_MAX_GQA;
 constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
+constexpr int kMaxChunks = 12;           // sum over groups of ceil(d_g / 16) <= 128/16 + 4
 
 // Everything a kernel needs about one layer's packing, passed by value.
 struct DevLayout {
@@ -35,8 +36,23 @@ struct DevLayout {
   const double* k_rot64[kMaxGroups];  // d_g x d_g row-major, y = R x
   const double* v_rot64;
   const float* k_rot32[kMaxGroups];
+  const float* k_rot32t[kMaxGroups];  // transposed copies (column-major)
   const float* v_rot32;
   unsigned* status;
+  // Tensor-core decode: 16-dimension chunks of the K record, per group.
+  int n_kchunks;
+  int group_chunk0[kMaxGroups];
+  int group_nchunks[kMaxGroups];
+  int chunk_bit[kMaxChunks];     // first bit of the chunk inside a K record
+  int chunk_dim0[kMaxChunks];    // first packed dimension of the chunk
+  int chunk_ndim[kMaxChunks];    // valid dimensions in the chunk (<= 16)
+  int chunk_group[kMaxChunks];
+  float kappa[5];                // per-rate scale making the rate-1/2 fp16 key codebooks exact
+  float kappa_v;                 // scale of the fp16 value codebook
+  // Pair tables: entry (a | b << r) holds the fp16 pair (value(a), value(b)).
+  const unsigned* klut12;        // rate 1: 4 entries at 0; rate 2: 16 entries at 4 (kappa-scaled)
+  const unsigned* klut34;        // rate 3: 64 entries at 0; rate 4: 256 at 64; entry = {hi pair, lo pair}
+  const unsigned* vlut;          // value codebook pairs, 2^(2 v_rate) entries (fp16, times kappa_v)
 };
 
 }  // namespace bgtq

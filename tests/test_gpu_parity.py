@@ -79,9 +79,9 @@ def test_decode_on_oracle_packed_cache():
                                        1 / math.sqrt(128)))
     cache = torch.from_numpy(np.concatenate(parts)).cuda()
     out = gpu_decode(lay, case, q, cache)
-    for h in range(case.h_kv):
-        for i in range(G):
-            assert rel_l2(out[0, h * G + i], refs[h][i]) <= 1e-4
+    errs = [rel_l2(out[0, h * G + i], refs[h][i]) for h in range(case.h_kv) for i in range(G)]
+    print(f"decode on the oracle's cache: max rel L2 {max(errs):.2e}, median {np.median(errs):.2e}")
+    assert max(errs) <= ATTN_REL_L2
 
 
 def test_incremental_appends_equal_prefill():
