@@ -102,7 +102,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t lut_words = 20 + 2 * (64 + 256) + 256;
+  const size_t lut_words = 20 + 2 * (64 + 256) + 256 + 32;
   const size_t bytes = 256 + n64 * sizeof(double) + 2 * n64 * sizeof(float) + lut_words * 4 + 256;
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
@@ -134,6 +134,8 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     for (int i = 0; i < d; ++i)
       for (int j = 0; j < d; ++j) h32[size_t(j) * d + i] = float(L->rot[g][size_t(i) * d + j]);
     D.k_rot32t[g] = reinterpret_cast<const float*>(dptr + off);
+    D.k_rot32t_off[g] = int((D.k_rot32t[g] - D.k_rot32t[0]));
+    D.k_rot32t_floats += int(L->rot[g].size());
     off += L->rot[g].size() * sizeof(float);
   }
   {
@@ -163,11 +165,19 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
       const int a = idx & ((1 << L->v_rate) - 1), b = idx >> L->v_rate;
       w[20 + 2 * 320 + idx] = pack_half2(kap_v * L->centroid[L->v_rate][a], kap_v * L->centroid[L->v_rate][b]);
     }
+    for (int idx = 0; idx < 16; ++idx) {
+      const double* c1 = L->centroid[1];
+      unsigned* e = w + 20 + 2 * 320 + 256 + 2 * idx;
+      e[0] = pack_half2(kap[1] * c1[idx & 1], kap[1] * c1[(idx >> 1) & 1]);
+      e[1] = pack_half2(kap[1] * c1[(idx >> 2) & 1], kap[1] * c1[(idx >> 3) & 1]);
+    }
+    D.klut1q = reinterpret_cast<const unsigned*>(dptr + off + (20 + 2 * 320 + 256) * 4);
     D.klut12 = reinterpret_cast<const unsigned*>(dptr + off);
     D.klut34 = reinterpret_cast<const unsigned*>(dptr + off + 20 * 4);
     D.vlut = reinterpret_cast<const unsigned*>(dptr + off + (20 + 2 * 320) * 4);
     for (int r = 0; r < 5; ++r) D.kappa[r] = float(kap[r]);
     D.kappa_v = float(kap_v);
+    for (int g = 0; g < ng; ++g) D.inv_kappa_group[g] = float(1.0 / kap[L->group_rate[g]]);
     off += lut_words * 4;
   }
   {
@@ -181,6 +191,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
         D.chunk_dim0[ci] = L->group_off[g] + 16 * cc;
         D.chunk_ndim[ci] = std::min(16, d - 16 * cc);
         D.chunk_group[ci] = g;
+        D.chunk_rate[ci] = r;
       }
     }
     D.n_kchunks = ci;

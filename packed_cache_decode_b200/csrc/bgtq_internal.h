@@ -36,7 +36,9 @@ struct DevLayout {
   const double* k_rot64[kMaxGroups];  // d_g x d_g row-major, y = R x
   const double* v_rot64;
   const float* k_rot32[kMaxGroups];
-  const float* k_rot32t[kMaxGroups];  // transposed copies (column-major)
+  const float* k_rot32t[kMaxGroups];  // transposed copies (column-major), back to back
+  int k_rot32t_off[kMaxGroups];       // float offset of group g's copy from k_rot32t[0]
+  int k_rot32t_floats;                // sum of d_g^2
   const float* v_rot32;
   unsigned* status;
   // Tensor-core decode: 16-dimension chunks of the K record, per group.
@@ -47,11 +49,14 @@ struct DevLayout {
   int chunk_dim0[kMaxChunks];    // first packed dimension of the chunk
   int chunk_ndim[kMaxChunks];    // valid dimensions in the chunk (<= 16)
   int chunk_group[kMaxChunks];
+  int chunk_rate[kMaxChunks];
+  float inv_kappa_group[kMaxGroups];  // 1 / kappa of each group's rate
   float kappa[5];                // per-rate scale making the rate-1/2 fp16 key codebooks exact
   float kappa_v;                 // scale of the fp16 value codebook
   // Pair tables: entry (a | b << r) holds the fp16 pair (value(a), value(b)).
   const unsigned* klut12;        // rate 1: 4 entries at 0; rate 2: 16 entries at 4 (kappa-scaled)
   const unsigned* klut34;        // rate 3: 64 entries at 0; rate 4: 256 at 64; entry = {hi pair, lo pair}
+  const unsigned* klut1q;        // rate 1, 16 entries: four codes -> {pair (0,1), pair (2,3)} (kappa-scaled)
   const unsigned* vlut;          // value codebook pairs, 2^(2 v_rate) entries (fp16, times kappa_v)
 };
 

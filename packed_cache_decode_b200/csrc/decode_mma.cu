@@ -6,9 +6,9 @@
 //   o           = R_V^T sum_t p_t (|v_t| / sqrt(128)) c[vcodes_t] / sum_t p_t.
 //
 // Three kernels per call:
-//  * qprep_kernel (one CTA per batch row x KV head): q' = R_g q_g for the G query heads,
-//    scaled by softmax_scale * log2(e) / sqrt(d_g), split into fp16 hi + lo parts and laid
-//    out as mma B fragments; also clears the per-unit completion counters.
+//  * qprep_kernel (one CTA per batch row x KV head): q' = R_g q_g for the G query heads
+//    (rotations staged in shared memory), scaled by softmax_scale * log2(e) / sqrt(d_g),
+//    split into fp16 hi + lo parts and laid out as mma B fragments.
 //  * split_kernel (one CTA per (split, unit), 4 warps): 64-token tiles arrive by 1-D bulk
 //    async copies (cp.async.bulk + mbarrier, no multicast) into a 4-stage ring. Warp w
 //    takes tokens 16w..16w+15 of each tile. Scores: for every 16-dimension chunk of a key
@@ -17,9 +17,12 @@
 //    multiplies them with q' hi and lo (fp32 accumulators per group, then times the group
 //    norm). Online softmax in base 2 with warp shuffles. Values: the probabilities times
 //    |v|/sqrt(128) in fp16, transposed with movmatrix, against value-code pair lookups,
-//    accumulated in V's rotated space (fp32). The four warps merge, the CTA writes its
-//    partial (o', m, l); the last CTA of the unit to finish (atomic counter, no waiting)
-//    merges all splits by log-sum-exp and applies R_V^T.
+//    accumulated in V's rotated space (fp32). The four warps merge and the CTA writes its
+//    partial (o', m, l). A fifth warp only issues the copies (full/empty mbarriers).
+//  * combine_kernel (one CTA per batch row x query head, 512 threads): log-sum-exp merge
+//    of the splits and o = R_V^T o'.
+// The three launches are chained with programmatic dependent launch, so each kernel's
+// set-up (and the split kernel's first tile copies) overlaps the previous kernel.
 //
 // Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, waits
 // (bounded) for its own copies in flight and returns.
@@ -40,10 +43,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kStages = 4;
 constexpr int kWarps = 4;
 constexpr unsigned kWaitLimit = 1u << 22;
-constexpr int kMaxSplitHeads = 1536;  // n_splits * G cap: the merging CTA stages S x G values
-// shared floats of the merge area: the four warps' [8][128] partials, and later the
-// split merge (3 S G staged values, 2 x 8 per-head scalars, G x 128 outputs)
-constexpr int kMergeFloats = 3 * kMaxSplitHeads + 16 + kMaxG * kD;
+constexpr int kMergeFloats = kWarps * 8 * kD;  // the consumer warps' [8][128] partials
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ unsigned smem_addr(const void* p) { return unsigned(__cvta_generic_to_shared(p)); }
@@ -107,7 +107,6 @@ __device__ __forceinline__ float load_q(const void* p, int dtype, size_t i) {
 
 // Workspace layout of one call (all offsets 256-byte aligned).
 struct Workspace {
-  unsigned* counters;  // [units]
   uint2* qfrag;        // [units][kMaxChunks][2][32]
   float* part_ml;      // [units][splits][G][2]
   float* part_o;       // [units][splits][G][128]
@@ -118,8 +117,6 @@ __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_
 __host__ __device__ inline Workspace carve(void* base, long long units, int splits, int G) {
   Workspace w;
   char* p = static_cast<char*>(base);
-  w.counters = reinterpret_cast<unsigned*>(p);
-  p += align256(units * sizeof(unsigned));
   w.qfrag = reinterpret_cast<uint2*>(p);
   p += align256(size_t(units) * kMaxChunks * 2 * 32 * sizeof(uint2));
   w.part_ml = reinterpret_cast<float*>(p);
@@ -129,49 +126,64 @@ __host__ __device__ inline Workspace carve(void* base, long long units, int spli
 }
 
 inline size_t workspace_size(long long units, int splits, int G) {
-  return align256(units * sizeof(unsigned)) + align256(size_t(units) * kMaxChunks * 2 * 32 * sizeof(uint2)) +
+  return align256(size_t(units) * kMaxChunks * 2 * 32 * sizeof(uint2)) +
          align256(size_t(units) * splits * G * 2 * sizeof(float)) + size_t(units) * splits * G * kD * sizeof(float);
 }
 
 // ------------------------------------------------------------------ q preparation
-__global__ void __launch_bounds__(128) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype, int h_q,
-                                                    int h_kv, int G, float qscale, Workspace ws) {
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
+                                                             int h_q, int h_kv, int G, float qscale, Workspace ws) {
+  extern __shared__ __align__(16) float prep_smem[];
   const int u = blockIdx.x, b = u / h_kv, h = u % h_kv;
   const int tid = threadIdx.x;
-  __shared__ float qs[kMaxG][kD];
-  __shared__ float qr[kMaxG][kD];
-  for (int hh = 0; hh < kMaxG; ++hh)
-    qs[hh][tid] = hh < G ? load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + tid) : 0.f;
-  if (tid == 0) ws.counters[u] = 0u;
+  float* rot = prep_smem;                       // the K-group rotations, transposed, back to back
+  float* qs = rot + L.k_rot32t_floats;          // [8][128] q in original coordinates
+  float* qr = qs + kMaxG * kD;                  // [8][128] q' in packed order
+  {
+    const float4* src = reinterpret_cast<const float4*>(L.k_rot32t[0]);
+    float4* dst = reinterpret_cast<float4*>(rot);
+    const int n4 = L.k_rot32t_floats / 4;
+#pragma unroll 4
+    for (int i = tid; i < n4; i += kPrepThreads) dst[i] = __ldg(src + i);
+  }
+  // q in packed order: qs[hh][p] = q[hh][packed_coord[p]]
+  for (int e = tid; e < kMaxG * kD; e += kPrepThreads) {
+    const int hh = e / kD, p = e % kD;
+    qs[e] = hh < G ? load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + L.packed_coord[p]) : 0.f;
+  }
   __syncthreads();
   {
+    // thread = (packed dimension p, half of the heads)
+    const int p = tid & (kD - 1), hbase = (tid >> 7) * (kMaxG / 2);
     int g = 0;
-    while (g + 1 < L.n_kgroups && tid >= L.group_off[g + 1]) ++g;
-    const int d = L.group_dim[g], off = L.group_off[g], i = tid - off;
-    const float* col = L.k_rot32t[g] + i;  // transposed: element (i, j) at j * d + i
+    while (g + 1 < L.n_kgroups && p >= L.group_off[g + 1]) ++g;
+    const int d = L.group_dim[g], off = L.group_off[g], i = p - off;
+    const float* col = rot + L.k_rot32t_off[g] + i;  // element (i, j) at j * d + i
     const float f = qscale * rsqrtf(float(d));
-    float acc[kMaxG];
+    float acc[kMaxG / 2];
 #pragma unroll
-    for (int hh = 0; hh < kMaxG; ++hh) acc[hh] = 0.f;
+    for (int k = 0; k < kMaxG / 2; ++k) acc[k] = 0.f;
+    const float* qg = qs + hbase * kD + off;
 #pragma unroll 4
     for (int j = 0; j < d; ++j) {
-      const float rj = __ldg(col + (size_t)j * d);
-      const int c = L.packed_coord[off + j];
+      const float rj = col[j * d];
 #pragma unroll
-      for (int hh = 0; hh < kMaxG; ++hh) acc[hh] = fmaf(rj, qs[hh][c], acc[hh]);
+      for (int k = 0; k < kMaxG / 2; ++k) acc[k] = fmaf(rj, qg[k * kD + j], acc[k]);
     }
 #pragma unroll
-    for (int hh = 0; hh < kMaxG; ++hh) qr[hh][tid] = acc[hh] * f;
+    for (int k = 0; k < kMaxG / 2; ++k) qr[(hbase + k) * kD + p] = acc[k] * f;
   }
   __syncthreads();
   // B fragments: lane (g = lane/4 -> head, t = lane%4). k-slots 2t, 2t+1 -> chunk dims 4t, 4t+1;
   // k-slots 2t+8, 2t+9 -> chunk dims 4t+2, 4t+3. Dims beyond the group are zero.
-  for (int e = tid; e < L.n_kchunks * 32; e += 128) {
+  for (int e = tid; e < L.n_kchunks * 32; e += kPrepThreads) {
     const int ci = e >> 5, lane = e & 31, hh = lane >> 2, t = lane & 3;
     const int d0 = L.chunk_dim0[ci], nd = L.chunk_ndim[ci];
     float v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) v[j] = (4 * t + j < nd) ? qr[hh][d0 + 4 * t + j] : 0.f;
+    for (int j = 0; j < 4; ++j) v[j] = (4 * t + j < nd) ? qr[hh * kD + d0 + 4 * t + j] : 0.f;
     float hi[4], lo[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -184,6 +196,89 @@ __global__ void __launch_bounds__(128) qprep_kernel(DevLayout L, const void* __r
   }
   __syncthreads();
   pdl_trigger();
+}
+
+size_t prep_smem_bytes(const DevLayout& L) { return (size_t(L.k_rot32t_floats) + 2 * kMaxG * kD) * sizeof(float); }
+
+// ------------------------------------------------------------------ combine
+constexpr int kCombThreads = 512;
+constexpr int kMaxSplits = 1024;
+
+// One CTA per (batch row, query head): log-sum-exp merge of the splits, then o = R_V^T o'.
+// Four threads per output dimension. R_V (not written by the split kernel) is read into
+// registers before waiting for the split kernel to finish.
+__global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* __restrict__ part_ml,
+                                                              const float* __restrict__ part_o, int S, int G,
+                                                              int h_q, int h_kv, const float* __restrict__ v_rot,
+                                                              float* __restrict__ out) {
+  const int bq = blockIdx.x, b = bq / h_q, hq = bq % h_q;
+  const int u = b * h_kv + hq / G, hh = hq % G;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = tid & (kD - 1), qtr = tid >> 7;
+  __shared__ float w[kMaxSplits];
+  __shared__ float red[2][kCombThreads / 32];
+  __shared__ float part[4][kD];
+  __shared__ float op[kD];
+  float rv[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) rv[i] = __ldg(v_rot + (size_t)(qtr * 32 + i) * kD + d);
+  pdl_wait();  // partials come from split_kernel
+  const float2* ml = reinterpret_cast<const float2*>(part_ml) + (size_t)u * S * G + hh;  // split sp at ml[sp * G]
+  float mloc[2], lloc[2];
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int sp = tid + k * kCombThreads;
+    const float2 v = sp < S ? ml[(size_t)sp * G] : make_float2(-INFINITY, 0.f);
+    mloc[k] = v.x;
+    lloc[k] = v.y;
+    M = fmaxf(M, v.x);
+  }
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[0][warp] = M;
+  __syncthreads();
+  M = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kCombThreads / 32; ++i) M = fmaxf(M, red[0][i]);
+  float l = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int sp = tid + k * kCombThreads;
+    if (sp < S) {
+      const float wt = (M == -INFINITY || mloc[k] == -INFINITY) ? 0.f : exp2f(mloc[k] - M);
+      w[sp] = wt;
+      l = fmaf(wt, lloc[k], l);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) red[1][warp] = l;
+  __syncthreads();
+  l = 0.f;
+#pragma unroll
+  for (int i = 0; i < kCombThreads / 32; ++i) l += red[1][i];
+  {
+    const float* po = part_o + ((size_t)u * S * G + hh) * kD + d;  // split sp at po[sp * G * kD]
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    int sp = qtr;
+    for (; sp + 12 < S; sp += 16) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] = fmaf(w[sp + 4 * k], __ldg(po + (size_t)(sp + 4 * k) * G * kD), o[k]);
+    }
+    for (; sp < S; sp += 4) o[0] = fmaf(w[sp], __ldg(po + (size_t)sp * G * kD), o[0]);
+    part[qtr][d] = (o[0] + o[1]) + (o[2] + o[3]);
+  }
+  __syncthreads();
+  if (tid < kD) op[tid] = l > 0.f ? ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) / l : 0.f;
+  __syncthreads();
+  float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    r0 = fmaf(rv[i], op[qtr * 32 + i], r0);
+    r1 = fmaf(rv[i + 1], op[qtr * 32 + i + 1], r1);
+  }
+  part[qtr][d] = r0 + r1;
+  __syncthreads();
+  if (tid < kD) out[((size_t)b * h_q + hq) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
 }
 
 // ------------------------------------------------------------------ split kernel
@@ -199,14 +294,134 @@ struct SplitArgs {
   float* out;
 };
 
-// fields of value codes: 4 codes of dimension d, tokens 2t, 2t+1, 2t+8, 2t+9 of a chunk
-template <int VR>
-__device__ __forceinline__ unsigned vfield(const unsigned* chunk_words, int d, int t) {
-  return bits32(chunk_words, (16 * d + 4 * t) * VR);
+constexpr int kConsumers = 4;                 // consumer warps, one 16-token slice of a tile each
+constexpr int kThreads = 32 * (kConsumers + 1);  // + one producer warp
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
+
+// Scores of one key group with compile-time rate R: for each 16-dimension chunk, the
+// thread's four codes (dims 4t..4t+3 of the chunk) of tokens g and g+8 index the pair
+// tables; q' hi and lo are the B operands. The bit offset advances 16 R per chunk.
+// Per chunk the thread forms its A fragments from the four codes of tokens g and g+8
+// (dims 4t..4t+3 of the chunk). Products with q' hi and q' lo (and, for rates 3-4, the
+// centroid low parts) go to separate accumulators, and consecutive chunks alternate
+// between two accumulator sets, so the mma dependency chains stay short.
+template <int R>
+__device__ __forceinline__ void key_chunk(float (&ah)[4], float (&al)[4], unsigned f0, unsigned f1, uint2 bh,
+                                          uint2 bl, const unsigned* klut12, const uint2* klut1q,
+                                          const uint2* klut34) {
+  constexpr unsigned M = (1u << (2 * R)) - 1u;
+  if constexpr (R == 1) {
+    // the four 1-bit codes of a token index one entry: {pair (4t, 4t+1), pair (4t+2, 4t+3)}
+    const uint2 e0 = klut1q[f0 & 15u], e1 = klut1q[f1 & 15u];
+    mma16816(ah, e0.x, e1.x, e0.y, e1.y, bh.x, bh.y);
+    mma16816(al, e0.x, e1.x, e0.y, e1.y, bl.x, bl.y);
+  } else if constexpr (R == 2) {
+    const unsigned* lut = klut12 + 4;
+    const unsigned a0 = lut[f0 & M], a2 = lut[(f0 >> 4) & M];
+    const unsigned a1 = lut[f1 & M], a3 = lut[(f1 >> 4) & M];
+    mma16816(ah, a0, a1, a2, a3, bh.x, bh.y);
+    mma16816(al, a0, a1, a2, a3, bl.x, bl.y);
+  } else {
+    const uint2* lut = klut34 + (R == 3 ? 0 : 64);
+    const uint2 e0 = lut[f0 & M], e2 = lut[(f0 >> (2 * R)) & M];
+    const uint2 e1 = lut[f1 & M], e3 = lut[(f1 >> (2 * R)) & M];
+    mma16816(ah, e0.x, e1.x, e2.x, e3.x, bh.x, bh.y);
+    mma16816(al, e0.x, e1.x, e2.x, e3.x, bl.x, bl.y);
+    mma16816(al, e0.y, e1.y, e2.y, e3.y, bh.x, bh.y);
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void key_group(float (&acc)[4], const unsigned* rec0, const unsigned* rec1,
+                                          const uint2* qf, int c0, int c1, int bit, int lane,
+                                          const unsigned* klut12, const uint2* klut1q, const uint2* klut34) {
+  float a[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) a[i][j] = 0.f;
+  const uint2* qp = qf + c0 * 64 + lane;
+  int ci = c0;
+  for (; ci + 1 < c1; ci += 2, bit += 32 * R, qp += 128) {
+    const int b1 = bit + 16 * R;
+    const unsigned* p0 = rec0 + (bit >> 5);
+    const unsigned* p1 = rec1 + (bit >> 5);
+    const unsigned* q0 = rec0 + (b1 >> 5);
+    const unsigned* q1 = rec1 + (b1 >> 5);
+    const unsigned f0 = __funnelshift_r(p0[0], p0[1], bit & 31), f1 = __funnelshift_r(p1[0], p1[1], bit & 31);
+    const unsigned g0 = __funnelshift_r(q0[0], q0[1], b1 & 31), g1 = __funnelshift_r(q1[0], q1[1], b1 & 31);
+    const uint2 bh0 = qp[0], bl0 = qp[32], bh1 = qp[64], bl1 = qp[96];
+    key_chunk<R>(a[0], a[1], f0, f1, bh0, bl0, klut12, klut1q, klut34);
+    key_chunk<R>(a[2], a[3], g0, g1, bh1, bl1, klut12, klut1q, klut34);
+  }
+  if (ci < c1) {
+    const unsigned* p0 = rec0 + (bit >> 5);
+    const unsigned* p1 = rec1 + (bit >> 5);
+    const unsigned f0 = __funnelshift_r(p0[0], p0[1], bit & 31), f1 = __funnelshift_r(p1[0], p1[1], bit & 31);
+    key_chunk<R>(a[0], a[1], f0, f1, qp[0], qp[32], klut12, klut1q, klut34);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = (a[0][j] + a[1][j]) + (a[2][j] + a[3][j]);
+}
+
+// Value codes for the PV product. MMA row r of m-tile mt stands for value dimension
+// 16 (r % 8) + 2 mt + r / 8, so thread g owns the contiguous dimensions 16g .. 16g+15 of
+// the 16-token chunk (16 rows of 16 VR bits starting at word 8 VR g). For m-tile mt the
+// thread needs rows 2mt (MMA row g) and 2mt+1 (row g+8), and in each row the 4 VR bits of
+// tokens 2t, 2t+1, 2t+8, 2t+9 (slots 4t..4t+3). Rates 1 and 2 keep all 16 rows in
+// registers (one tile load); rates 3 and 4 read the two rows per m-tile.
 template <int VR>
-__global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a) {
+struct ValueRows {
+  unsigned w[VR <= 2 ? 8 * VR : 1];
+  const unsigned* base;
+  int t;
+  __device__ __forceinline__ void load(const unsigned* chunk, int g, int t_) {
+    t = t_;
+    base = chunk + 8 * VR * g;
+    if constexpr (VR <= 2) {
+      const uint4* p = reinterpret_cast<const uint4*>(base);
+#pragma unroll
+      for (int i = 0; i < 2 * VR; ++i) {
+        const uint4 v = p[i];
+        w[4 * i] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+      }
+    }
+  }
+  __device__ __forceinline__ void fields(int mt, unsigned& fx, unsigned& fy) const {
+    if constexpr (VR == 1) {
+      fx = w[mt] >> (4 * t);
+      fy = w[mt] >> (16 + 4 * t);
+    } else if constexpr (VR == 2) {
+      fx = w[2 * mt] >> (8 * t);
+      fy = w[2 * mt + 1] >> (8 * t);
+    } else if constexpr (VR == 3) {
+      const unsigned w0 = base[3 * mt], w1 = base[3 * mt + 1], w2 = base[3 * mt + 2];
+      fx = unsigned((((unsigned long long)w1 << 32) | w0) >> (12 * t));
+      fy = unsigned((((unsigned long long)w2 << 32) | w1) >> (16 + 12 * t));
+    } else {
+      const uint4 v = reinterpret_cast<const uint4*>(base)[mt];
+      const int sh = 16 * (t & 1);
+      fx = ((t < 2) ? v.x : v.y) >> sh;
+      fy = ((t < 2) ? v.z : v.w) >> sh;
+    }
+  }
+};
+
+template <int VR>
+__global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int s = blockIdx.x, u = blockIdx.y;
   const int b = u / a.h_kv;
@@ -214,17 +429,18 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
   const int g = lane >> 2, t = lane & 3;
   const int TB = L.tile_bytes;
 
-  // shared memory carve-up
   unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);
+  unsigned long long* empty = full + kStages;
   unsigned char* ring = smem + 128;
   uint2* qf = reinterpret_cast<uint2*>(ring + kStages * TB + 64);
   unsigned* klut12 = reinterpret_cast<unsigned*>(qf + kMaxChunks * 2 * 32);
   uint2* klut34 = reinterpret_cast<uint2*>(klut12 + 32);
-  unsigned* vlut = reinterpret_cast<unsigned*>(klut34 + 320);
+  uint2* klut1q = klut34 + 320;                       // rate 1, four codes per entry
+  unsigned* vlut = reinterpret_cast<unsigned*>(klut1q + 16);
   float* mo = reinterpret_cast<float*>(vlut + 256);  // merge: [warp][8][128]
   float* mm = mo + kMergeFloats;                      // [warp][8]
-  float* ml = mm + kWarps * 8;                        // [warp][8]
-  __shared__ int s_last;
+  float* ml = mm + kConsumers * 8;                    // [warp][8]
+  __shared__ int s_timeout;
 
   long long len = a.seq_lens[b];
   if (len < 0) len = 0;
@@ -235,86 +451,96 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
   }
   const int len_tiles = int((len + kTile - 1) / kTile);
   const int t0 = s * a.tiles_per_split;
-  const int t1 = min(t0 + a.tiles_per_split, len_tiles);
-  const int ntiles = max(0, t1 - t0);
+  const int ntiles = max(0, min(t0 + a.tiles_per_split, len_tiles) - t0);
   const uint8_t* src = a.cache + ((size_t)u * a.n_tiles + t0) * (size_t)TB;
 
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&full[i], 1);
+  if (tid == kConsumers * 32) {
+    // the producer lane: barriers, then the first copies before anything else
+    s_timeout = 0;
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kConsumers);
+    }
     fence_mbar_init();
-    for (int i = 0; i < min(kStages, ntiles); ++i) {
-      mbar_expect_tx(&full[i], TB);
-      bulk_load(ring + i * TB, src + (size_t)i * TB, TB, &full[i]);
+    for (int it = 0; it < min(kStages, ntiles); ++it) {
+      mbar_expect_tx(&full[it], TB);
+      bulk_load(ring + it * TB, src + (size_t)it * TB, TB, &full[it]);
     }
   }
-  // constant tables (written by the layout upload, not by the previous kernel)
-  for (int i = tid; i < 20; i += 128) klut12[i] = L.klut12[i];
-  for (int i = tid; i < 320; i += 128)
-    klut34[i] = make_uint2(L.klut34[2 * i], L.klut34[2 * i + 1]);
-  for (int i = tid; i < (1 << (2 * VR)); i += 128) vlut[i] = L.vlut[i];
-  pdl_wait();  // q fragments and counters come from qprep_kernel
+  for (int i = tid; i < 20; i += kThreads) klut12[i] = L.klut12[i];
+  for (int i = tid; i < 320; i += kThreads) klut34[i] = make_uint2(L.klut34[2 * i], L.klut34[2 * i + 1]);
+  for (int i = tid; i < 16; i += kThreads) klut1q[i] = make_uint2(L.klut1q[2 * i], L.klut1q[2 * i + 1]);
+  for (int i = tid; i < (1 << (2 * VR)); i += kThreads) vlut[i] = L.vlut[i];
+  __syncthreads();
+
+  if (warp == kConsumers) {
+    // ------------------------------------------------ producer warp: one lane streams tiles
+    if (lane == 0) {
+      int issued = min(kStages, ntiles);
+      for (int it = issued; it < ntiles; ++it) {
+        const int stage = it % kStages;
+        if (it >= kStages && !mbar_wait_bounded(&empty[stage], ((it / kStages) - 1) & 1)) {
+          atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
+          break;
+        }
+        mbar_expect_tx(&full[stage], TB);
+        bulk_load(ring + stage * TB, src + (size_t)it * TB, TB, &full[stage]);
+        issued = it + 1;
+      }
+      // do not leave while copies into this CTA's shared memory are still in flight
+      for (int j = max(0, issued - kStages); j < issued; ++j) mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------- consumer warps
+  pdl_wait();  // q fragments come from qprep_kernel
   {
     const uint4* qsrc = reinterpret_cast<const uint4*>(a.ws.qfrag + (size_t)u * kMaxChunks * 2 * 32);
     uint4* qdst = reinterpret_cast<uint4*>(qf);
     for (int i = tid; i < L.n_kchunks * 32; i += 128) qdst[i] = qsrc[i];
   }
-  __syncthreads();
+  consumer_sync();
 
   const float vscale = rsqrtf(float(kD)) / L.kappa_v;
-
   float O[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
     for (int j = 0; j < 4; ++j) O[mt][j] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  bool ok = true;
+  const int tok0 = 16 * warp + g;
 
   for (int it = 0; it < ntiles; ++it) {
     const int stage = it % kStages;
-    // A timed-out wait still runs the tile on whatever is in shared memory (every index
-    // stays in bounds); the CTA-wide vote at the end of the tile then stops the loop.
-    if (!mbar_wait_bounded(&full[stage], (it / kStages) & 1)) ok = false;
+    if (!mbar_wait_bounded(&full[stage], (it / kStages) & 1)) {
+      // stop consuming; the producer waits for its own copies and this unit's result
+      // is not written (every consumer warp still reaches the merge barriers below)
+      if (lane == 0) {
+        atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
+        s_timeout = 1;
+      }
+      break;
+    }
     const unsigned char* tb = ring + stage * TB;
-    const int tok0 = 16 * warp + g;  // token rows g and g+8 of this warp's chunk
     const long long gtok = (long long)(t0 + it) * kTile + tok0;
 
-    // ---------------- scores
+    // ---------------- scores: per key group, rate as a template parameter
     const unsigned* rec0 = reinterpret_cast<const unsigned*>(tb + tok0 * L.k_record_bytes);
     const unsigned* rec1 = reinterpret_cast<const unsigned*>(tb + (tok0 + 8) * L.k_record_bytes);
     const float* kn = reinterpret_cast<const float*>(tb + L.knorm_off);
     float sc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int gi = 0; gi < L.n_kgroups; ++gi) {
-      const int r = L.group_rate[gi];
-      const int c0 = L.group_chunk0[gi], c1 = c0 + L.group_nchunks[gi];
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (r <= 2) {
-        const unsigned* lut = klut12 + (r == 1 ? 0 : 4);
-        const unsigned msk = (1u << (2 * r)) - 1u;
-        for (int ci = c0; ci < c1; ++ci) {
-          const int bit = L.chunk_bit[ci] + 4 * t * r;
-          const unsigned f0 = bits32(rec0, bit), f1 = bits32(rec1, bit);
-          const unsigned a0 = lut[f0 & msk], a2 = lut[(f0 >> (2 * r)) & msk];
-          const unsigned a1 = lut[f1 & msk], a3 = lut[(f1 >> (2 * r)) & msk];
-          const uint2 bh = qf[ci * 64 + lane], bl = qf[ci * 64 + 32 + lane];
-          mma16816(acc, a0, a1, a2, a3, bh.x, bh.y);
-          mma16816(acc, a0, a1, a2, a3, bl.x, bl.y);
-        }
-      } else {
-        const uint2* lut = klut34 + (r == 3 ? 0 : 64);
-        const unsigned msk = (1u << (2 * r)) - 1u;
-        for (int ci = c0; ci < c1; ++ci) {
-          const int bit = L.chunk_bit[ci] + 4 * t * r;
-          const unsigned f0 = bits32(rec0, bit), f1 = bits32(rec1, bit);
-          const uint2 e0 = lut[f0 & msk], e2 = lut[(f0 >> (2 * r)) & msk];
-          const uint2 e1 = lut[f1 & msk], e3 = lut[(f1 >> (2 * r)) & msk];
-          const uint2 bh = qf[ci * 64 + lane], bl = qf[ci * 64 + 32 + lane];
-          mma16816(acc, e0.x, e1.x, e2.x, e3.x, bh.x, bh.y);
-          mma16816(acc, e0.x, e1.x, e2.x, e3.x, bl.x, bl.y);
-          mma16816(acc, e0.y, e1.y, e2.y, e3.y, bh.x, bh.y);
-        }
+      const int r = L.group_rate[gi], c0 = L.group_chunk0[gi], c1 = c0 + L.group_nchunks[gi];
+      const int bit = L.group_bitoff[gi] + 4 * t * r;
+      switch (r) {
+        case 1: key_group<1>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
+        case 2: key_group<2>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
+        case 3: key_group<3>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
+        default: key_group<4>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
       }
-      const float ik = 1.0f / L.kappa[r];
+      const float ik = L.inv_kappa_group[gi];
       const float n0 = kn[gi * kTile + tok0] * ik;
       const float n1 = kn[gi * kTile + tok0 + 8] * ik;
       sc[0] = fmaf(acc[0], n0, sc[0]);
@@ -325,7 +551,7 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
     if (gtok >= len) sc[0] = sc[1] = -INFINITY;
     if (gtok + 8 >= len) sc[2] = sc[3] = -INFINITY;
 
-    // ---------------- online softmax (heads 2t and 2t+1; rows g and g+8)
+    // ---------------- online softmax (heads 2t, 2t+1; token rows g, g+8), base 2
     float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -333,22 +559,24 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
       x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
     }
     const float n0m = fmaxf(m0, x0), n1m = fmaxf(m1, x1);
-    const float corr0 = n0m == -INFINITY ? 1.f : exp2f(m0 - n0m);
-    const float corr1 = n1m == -INFINITY ? 1.f : exp2f(m1 - n1m);
-    const float p0 = n0m == -INFINITY ? 0.f : exp2f(sc[0] - n0m);
-    const float p1 = n1m == -INFINITY ? 0.f : exp2f(sc[1] - n1m);
-    const float p2 = n0m == -INFINITY ? 0.f : exp2f(sc[2] - n0m);
-    const float p3 = n1m == -INFINITY ? 0.f : exp2f(sc[3] - n1m);
+    // rows that are still all -inf keep a zero weight and leave the accumulators alone
+    const float b0m = n0m == -INFINITY ? 0.f : n0m, b1m = n1m == -INFINITY ? 0.f : n1m;
+    const float corr0 = fast_exp2(m0 - b0m), corr1 = fast_exp2(m1 - b1m);
+    const float p0 = fast_exp2(sc[0] - b0m), p1 = fast_exp2(sc[1] - b1m);
+    const float p2 = fast_exp2(sc[2] - b0m), p3 = fast_exp2(sc[3] - b1m);
+    const bool rescale = !__all_sync(0xffffffffu, n0m == m0 && n1m == m1);
     m0 = n0m;
     m1 = n1m;
     l0 = fmaf(l0, corr0, p0 + p2);
     l1 = fmaf(l1, corr1, p1 + p3);
+    if (rescale) {
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      O[mt][0] *= corr0;
-      O[mt][1] *= corr1;
-      O[mt][2] *= corr0;
-      O[mt][3] *= corr1;
+      for (int mt = 0; mt < 8; ++mt) {
+        O[mt][0] *= corr0;
+        O[mt][1] *= corr1;
+        O[mt][2] *= corr0;
+        O[mt][3] *= corr1;
+      }
     }
     const float* vn = reinterpret_cast<const float*>(tb + L.vnorm_off);
     const float av0 = vn[tok0] * vscale, av1 = vn[tok0 + 8] * vscale;
@@ -356,33 +584,24 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
     const unsigned pb1 = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
 
     // ---------------- values
-    const unsigned* vw = reinterpret_cast<const unsigned*>(tb + L.vcode_off + warp * 256 * VR);
-    constexpr unsigned vm = (1u << (2 * VR)) - 1u;
+    {
+      ValueRows<VR> vr;
+      vr.load(reinterpret_cast<const unsigned*>(tb + L.vcode_off + warp * 256 * VR), g, t);
+      constexpr unsigned vm = (1u << (2 * VR)) - 1u;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const unsigned f0 = vfield<VR>(vw, 16 * mt + g, t);
-      const unsigned f1 = vfield<VR>(vw, 16 * mt + g + 8, t);
-      mma16816(O[mt], vlut[f0 & vm], vlut[f1 & vm], vlut[(f0 >> (2 * VR)) & vm], vlut[(f1 >> (2 * VR)) & vm], pb0,
-               pb1);
-    }
-
-    // every warp is done with this stage
-    if (!__syncthreads_and(ok)) {
-      // A copy never completed: record it, wait (bounded) for the copies this CTA still
-      // has in flight, and leave without a result for this unit.
-      if (tid == 0) {
-        atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
-        for (int j = it; j < min(it + kStages, ntiles); ++j) mbar_wait_bounded(&full[j % kStages], (j / kStages) & 1);
+      for (int mt = 0; mt < 8; ++mt) {
+        unsigned fx, fy;
+        vr.fields(mt, fx, fy);
+        mma16816(O[mt], vlut[fx & vm], vlut[fy & vm], vlut[(fx >> (2 * VR)) & vm], vlut[(fy >> (2 * VR)) & vm],
+                 pb0, pb1);
       }
-      return;
     }
-    if (tid == 0 && it + kStages < ntiles) {
-      mbar_expect_tx(&full[stage], TB);
-      bulk_load(ring + stage * TB, src + (size_t)(it + kStages) * TB, TB, &full[stage]);
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
   }
 
-  // ---------------- merge the warps
+  pdl_trigger();
+  // ---------------- merge the consumer warps
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -390,11 +609,11 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
   }
   float* mow = mo + warp * 8 * kD;
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    mow[(2 * t) * kD + 16 * mt + g] = O[mt][0];
-    mow[(2 * t + 1) * kD + 16 * mt + g] = O[mt][1];
-    mow[(2 * t) * kD + 16 * mt + g + 8] = O[mt][2];
-    mow[(2 * t + 1) * kD + 16 * mt + g + 8] = O[mt][3];
+  for (int mt = 0; mt < 8; ++mt) {  // row g -> dim 16g + 2mt, row g+8 -> dim 16g + 2mt + 1
+    mow[(2 * t) * kD + 16 * g + 2 * mt] = O[mt][0];
+    mow[(2 * t + 1) * kD + 16 * g + 2 * mt] = O[mt][1];
+    mow[(2 * t) * kD + 16 * g + 2 * mt + 1] = O[mt][2];
+    mow[(2 * t + 1) * kD + 16 * g + 2 * mt + 1] = O[mt][3];
   }
   if (g == 0) {
     mm[warp * 8 + 2 * t] = m0;
@@ -402,17 +621,18 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
     ml[warp * 8 + 2 * t] = l0;
     ml[warp * 8 + 2 * t + 1] = l1;
   }
-  __syncthreads();
+  consumer_sync();
+  if (*static_cast<volatile int*>(&s_timeout)) return;  // uniform over the consumer warps
   const int G = a.G;
   for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * 8 + hh]);
+    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, mm[w * 8 + hh]);
     float o = 0.f, l = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float f = exp2f(mm[w * 8 + hh] - M);
+      for (int w = 0; w < kConsumers; ++w) {
+        const float f = fast_exp2(mm[w * 8 + hh] - M);
         o = fmaf(f, mo[(w * 8 + hh) * kD + tid], o);
         l = fmaf(f, ml[w * 8 + hh], l);
       }
@@ -424,71 +644,11 @@ __global__ void __launch_bounds__(128, 3) split_kernel(DevLayout L, SplitArgs a)
       a.ws.part_ml[idx * 2 + 1] = l;
     }
   }
-
-  // ---------------- the last CTA of this unit merges the splits
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.ws.counters[u], 1u) == unsigned(a.n_splits - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // stage every split's (m, l) of this unit, then the per-split weights exp2(m_s - M)
-  const int S = a.n_splits;
-  float* sml = mo;                    // [S][G][2]  (S * G <= kMaxSplitHeads)
-  float* sw = mo + 2 * S * G;         // [S][G] weights, then [G] sums l
-  float* op = sw + S * G + 2 * kMaxG; // [G][128] normalised rotated outputs
-  {
-    const float* src_ml = a.ws.part_ml + (size_t)u * S * G * 2;
-    for (int i = tid; i < S * G * 2; i += 128) sml[i] = __ldcg(src_ml + i);
-  }
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, sml[(sp * G + tid) * 2]);
-    float l = 0.f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float m = sml[(sp * G + tid) * 2];
-      const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M);
-      sw[sp * G + tid] = w;
-      l = fmaf(w, sml[(sp * G + tid) * 2 + 1], l);
-    }
-    sw[S * G + tid] = l;
-  }
-  __syncthreads();
-  {
-    const float* po = a.ws.part_o + (size_t)u * S * G * kD + tid;
-    for (int hh = 0; hh < G; ++hh) {
-      float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-      int sp = 0;
-      for (; sp + 4 <= S; sp += 4) {
-        o0 = fmaf(sw[(sp + 0) * G + hh], __ldcg(po + ((size_t)(sp + 0) * G + hh) * kD), o0);
-        o1 = fmaf(sw[(sp + 1) * G + hh], __ldcg(po + ((size_t)(sp + 1) * G + hh) * kD), o1);
-        o2 = fmaf(sw[(sp + 2) * G + hh], __ldcg(po + ((size_t)(sp + 2) * G + hh) * kD), o2);
-        o3 = fmaf(sw[(sp + 3) * G + hh], __ldcg(po + ((size_t)(sp + 3) * G + hh) * kD), o3);
-      }
-      for (; sp < S; ++sp) o0 = fmaf(sw[sp * G + hh], __ldcg(po + ((size_t)sp * G + hh) * kD), o0);
-      const float l = sw[S * G + hh];
-      op[hh * kD + tid] = l > 0.f ? ((o0 + o1) + (o2 + o3)) / l : 0.f;
-    }
-  }
-  __syncthreads();
-  float r[kMaxG];
-#pragma unroll
-  for (int hh = 0; hh < kMaxG; ++hh) r[hh] = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < kD; ++i) {
-    const float rv = __ldg(L.v_rot32 + i * kD + tid);
-#pragma unroll
-    for (int hh = 0; hh < kMaxG; ++hh) r[hh] = fmaf(rv, op[(hh < G ? hh : 0) * kD + i], r[hh]);
-  }
-  const int h = u % a.h_kv;
-  for (int hh = 0; hh < G; ++hh) a.out[((size_t)b * a.h_q + (size_t)h * G + hh) * kD + tid] = r[hh];
-  if (tid == 0) a.ws.counters[u] = 0u;
 }
 
 size_t split_smem_bytes(int tile_bytes) {
-  return 128 + size_t(kStages) * tile_bytes + 64 + kMaxChunks * 2 * 32 * sizeof(uint2) + 32 * 4 + 320 * 8 +
-         256 * 4 + (kMergeFloats + 2 * kWarps * 8) * sizeof(float);
+  return 128 + size_t(kStages) * tile_bytes + 64 + kMaxChunks * 2 * 32 * sizeof(uint2) + 32 * 4 + 320 * 8 + 16 * 8 +
+         256 * 4 + (kMergeFloats + 2 * kConsumers * 8) * sizeof(float);
 }
 
 template <int VR>
@@ -505,7 +665,7 @@ cudaError_t launch_split(const DevLayout& L, const SplitArgs& a, dim3 grid, cuda
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -524,11 +684,11 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
   p.max_tiles = int((max_seq_len + kTile - 1) / kTile);
   if (p.max_tiles < 1) p.max_tiles = 1;
   const long long units = (long long)batch * h_kv;
-  const long long target = 3LL * num_sms;
+  const long long target = 4LL * num_sms;
   long long splits = (target + units - 1) / units;
   if (splits < 1) splits = 1;
   if (splits > p.max_tiles) splits = p.max_tiles;
-  if (splits * G > kMaxSplitHeads) splits = kMaxSplitHeads / G;
+  if (splits > kMaxSplits) splits = kMaxSplits;
   p.tiles_per_split = int((p.max_tiles + splits - 1) / splits);
   p.n_splits = (p.max_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
   p.workspace_bytes = workspace_size(units, p.n_splits, G);
@@ -541,7 +701,19 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
   const int G = h_q / h_kv;
   const long long units = (long long)batch * h_kv;
   Workspace ws = carve(workspace, units, plan.n_splits, G);
-  qprep_kernel<<<unsigned(units), 128, 0, stream>>>(L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, ws);
+  {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int((kD * kD + 2 * kMaxG * kD) * sizeof(float)));
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
+  }
+  qprep_kernel<<<unsigned(units), kPrepThreads, prep_smem_bytes(L), stream>>>(L, q, q_dtype, h_q, h_kv, G,
+                                                                              softmax_scale * kLog2e, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   SplitArgs a;
@@ -558,12 +730,24 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
   a.out = out;
   dim3 grid(plan.n_splits, unsigned(units));
   switch (L.v_rate) {
-    case 1: return launch_split<1>(L, a, grid, stream);
-    case 2: return launch_split<2>(L, a, grid, stream);
-    case 3: return launch_split<3>(L, a, grid, stream);
-    case 4: return launch_split<4>(L, a, grid, stream);
-    default: return cudaErrorInvalidValue;
+    case 1: e = launch_split<1>(L, a, grid, stream); break;
+    case 2: e = launch_split<2>(L, a, grid, stream); break;
+    case 3: e = launch_split<3>(L, a, grid, stream); break;
+    case 4: e = launch_split<4>(L, a, grid, stream); break;
+    default: e = cudaErrorInvalidValue;
   }
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(batch * h_q));
+  cfg.blockDim = dim3(kCombThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)ws.part_ml, (const float*)ws.part_o, plan.n_splits,
+                            G, h_q, h_kv, L.v_rot32, out);
 }
 
 }  // namespace bgtq
