@@ -9,6 +9,8 @@ the 126 MB L2). The step is captured in a CUDA graph and replayed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|qwen3b|llama70b|tiny]
     python bench.py --impl reference ...      # the CPU oracle, timed on the host cores
+    python bench.py --mode sweep              # decode over the 32q/8kv context x batch x rate grid
+    python bench.py --mode encode             # tq_encode append throughput, 1 and 64 new tokens
 
 Prints one JSON line (rank 0).
 """
@@ -119,20 +121,26 @@ class Model:
             lay = B.Layout(rates, wl.v_bits, seed).upload(device.index)
             cache = torch.zeros(lay.cache_bytes(Bt, hkv, self.capacity), dtype=torch.uint8, device=device)
             gen.manual_seed(seed)
-            k, v = self._draw_kv(m, Bt, L, hkv, gen)
+            # prefill tokens 0..L-2 in bounded chunks (about 1 GB of fp32 draws at a time);
+            # token L-1 is the one every step appends again
+            chunk = int(max(64, min(16384, 1e9 // (Bt * hkv * 128 * 4 * 3))))
             lens0 = torch.zeros(Bt, dtype=torch.int32, device=device)
-            chunk = 16384
-            for a in range(0, L - 1, chunk):
-                b = min(L - 1, a + chunk)
-                lens0.fill_(a)
-                B.encode_append(lay, k[:, a:b].contiguous(), v[:, a:b].contiguous(), lens0, cache, self.capacity)
+            for a in range(0, L, chunk):
+                b = min(L, a + chunk)
+                k, v = self._draw_kv(m, Bt, a, b, hkv, gen)
+                n_enc = min(b, L - 1) - a
+                if n_enc > 0:
+                    lens0.fill_(a)
+                    B.encode_append(lay, k[:, :n_enc].contiguous(), v[:, :n_enc].contiguous(), lens0, cache,
+                                    self.capacity)
+                if b == L:
+                    k_new, v_new = k[:, -1:].contiguous(), v[:, -1:].contiguous()
+                del k, v
             q = self._draw_q(m, Bt, hq, L - 1, gen)
             self.layers.append({
-                "layout": lay, "cache": cache,
-                "k_new": k[:, L - 1:L].contiguous(), "v_new": v[:, L - 1:L].contiguous(), "q": q,
+                "layout": lay, "cache": cache, "k_new": k_new, "v_new": v_new, "q": q,
                 "out": torch.empty(Bt, hq, 128, dtype=torch.float32, device=device),
             })
-            del k, v
         torch.cuda.synchronize(device)
         self.lens_before = torch.full((Bt,), L - 1, dtype=torch.int32, device=device)
         self.lens_after = torch.full((Bt,), L, dtype=torch.int32, device=device)
@@ -141,15 +149,15 @@ class Model:
         self.bytes_per_step = sum(Bt * hkv * L * x["layout"].bytes_per_token for x in self.layers)
         self.keys_per_step = Bt * hkv * L * wl.layers
 
-    def _draw_kv(self, m, Bt, L, hkv, gen):
-        # Same recipe as synth.key_slice / value_slice, drawn on the device in bulk.
+    def _draw_kv(self, m, Bt, a, b, hkv, gen):
+        # Same recipe as synth.key_slice / value_slice (positions a..b-1), drawn on the device.
         dt = self.wl.dtype
-        x = torch.randn(Bt, L, hkv, 128, generator=gen, device=self.dev)
+        x = torch.randn(Bt, b - a, hkv, 128, generator=gen, device=self.dev)
         x *= torch.cat([m.k_scale, m.k_scale], 1).to(self.dev)[None, None]
         for h in range(hkv):
             x[:, :, h, m.outliers[h].to(self.dev)] *= m.outlier_gain
-        x = _rope_dev(x, torch.arange(L, device=self.dev), self.wl.theta)
-        v = torch.randn(Bt, L, hkv, 128, generator=gen, device=self.dev)
+        x = _rope_dev(x, torch.arange(a, b, device=self.dev), self.wl.theta)
+        v = torch.randn(Bt, b - a, hkv, 128, generator=gen, device=self.dev)
         return x.to(dt), v.to(dt)
 
     def _draw_q(self, m, Bt, hq, pos, gen):
@@ -226,6 +234,78 @@ def oracle_sample(wl: synth.Workload, budget_s: float):
                       f"layer, {wl.length} cached tokens each: append 1 token + decode attention, {elapsed:.1f} s"}
 
 
+# ------------------------------------------------------------------------ sweep / encode modes
+def _time_graph(fn, stream, reps):
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fn(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    return ms
+
+
+def run_sweep(args):
+    """Decode attention over the 32q/8kv grid; each point cycles enough per-layer caches
+    to exceed L2 (>= 256 MB per replay, at most 32 layers)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = _peaks()
+    stream = torch.cuda.Stream()
+    for wl in synth.sweep_workloads():
+        bpt = 128 * wl.k_bits // 8 + 128 * wl.v_bits // 8 + 20
+        per_layer = wl.batch * wl.h_kv * wl.length * bpt
+        layers = int(min(32, max(1, math.ceil(256e6 / per_layer))))
+        if per_layer * layers > 40e9:
+            continue
+        w = synth.Workload(**{**wl.__dict__, "layers": layers})
+        model = Model(w, dev)
+        ms = _time_graph(model.decode_only, stream, max(5, args.steps))
+        keys = w.batch * w.h_kv * w.length * layers
+        gbs = model.bytes_per_step / (ms * 1e-3) / 1e9
+        print(json.dumps({"mode": "sweep", "workload": w.name, "layers_cycled": layers,
+                          "us_per_layer": ms * 1e3 / layers, "keys_per_s": keys / (ms * 1e-3), "GBs": gbs,
+                          "hbm_frac": gbs / peak, "peak_kind": peak_kind}), flush=True)
+        del model
+        torch.cuda.empty_cache()
+
+
+def run_encode(args):
+    """tq_encode append throughput on the 32q/8kv shape (K2V2 layout), n_new in {1, 64}."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream()
+    m = synth.make_layer_model(32, 8, 4)
+    q_cal, k_cal = synth.make_calibration(m, 256, 5, 5e5)
+    rates = B.plan_layer_rates(q_cal.numpy(), k_cal.numpy(), 2)
+    lay = B.Layout(rates, 2, 4).upload(0)
+    for batch in (1, 8, 32):
+        for n_new in (1, 64):
+            cap = 4096
+            cache = torch.zeros(lay.cache_bytes(batch, 8, cap), dtype=torch.uint8, device=dev)
+            k = torch.randn(batch, n_new, 8, 128, device=dev).to(torch.bfloat16)
+            v = torch.randn_like(k)
+            lens = torch.full((batch,), 1000, dtype=torch.int32, device=dev)
+            ms = _time_graph(lambda st: B.encode_append(lay, k, v, lens, cache, cap, stream=st), stream,
+                             max(20, args.steps))
+            toks = batch * n_new
+            print(json.dumps({"mode": "encode", "batch": batch, "n_new": n_new, "h_kv": 8, "rates": "K2V2",
+                              "us_per_call": ms * 1e3, "tokens_per_s": toks / (ms * 1e-3),
+                              "token_heads_per_s": toks * 8 / (ms * 1e-3)}), flush=True)
+
+
 # ------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -237,7 +317,12 @@ def main():
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="step", choices=["step", "sweep", "encode"])
     args = ap.parse_args()
+    if args.mode == "sweep":
+        return run_sweep(args)
+    if args.mode == "encode":
+        return run_encode(args)
     wl = synth.WORKLOADS[args.workload]
     if args.layers:
         wl = synth.Workload(**{**wl.__dict__, "layers": args.layers})

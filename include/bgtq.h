@@ -24,11 +24,14 @@
  *    (per host thread). No C++ exception crosses the ABI.
  *
  * Packed cache format (one (batch row, KV head) = capacity/64 consecutive tiles):
- *  tile of 64 tokens = [K records | V codes | K norms | V norms]
- *   K records: 64 x Kb bytes, token-major, Kb = 128*avg_k_bits/8. A record is an
- *              LSB-first bitstream (bit n = bit n%8 of byte n/8) of the 128 key codes in
- *              packed-dimension order: K groups by descending rate; in a group, blocks
- *              ascending, coordinate j before j+64. A code of rate r takes r bits.
+ *  tile of 64 tokens = [K codes | V codes | K norms | V norms]
+ *   K codes:   64 x Kb bytes, Kb = 128*avg_k_bits/8. Packed key dimensions: K groups by
+ *              descending rate; in a group, blocks ascending, coordinate j before j+64.
+ *              Each group is cut into 16-dimension chunks (the last one may be shorter).
+ *              Chunk c (dims_c dimensions of rate r_c) owns a block of 8*dims_c*r_c bytes,
+ *              blocks in chunk order; a block is an LSB-first bitstream (bit n = bit n%8
+ *              of byte n/8) in which token j's codes of the chunk start at bit
+ *              j*dims_c*r_c, dimension i of the chunk at + i*r_c.
  *   V codes:   four 16-token chunks of 256*b_V bytes; each an LSB-first bitstream where
  *              the code of (dimension d, token j of the chunk) starts at bit
  *              (16*d + slot(j))*b_V, slot(j) = 4*((j%8)/2) + 2*(j/8) + j%2.

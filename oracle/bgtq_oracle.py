@@ -280,6 +280,20 @@ class Layout:
     def tile_bytes(self):
         return TILE_TOKENS * self.bytes_per_token
 
+    def k_chunks(self):
+        """16-dimension chunks of the key groups in order: (first packed dim, dims, rate,
+        byte offset of the chunk's block inside a tile). A block holds the 64 tokens'
+        fields of that chunk back to back (token j's field at bit j * dims * rate)."""
+        out, p, off = [], 0, 0
+        for r, coords in self.groups:
+            d = len(coords)
+            for c0 in range(0, d, 16):
+                nd = min(16, d - c0)
+                out.append((p + c0, nd, r, off))
+                off += TILE_TOKENS * nd * r // 8
+            p += d
+        return out
+
     def packed_rates(self):
         return np.concatenate([np.full(len(c), r) for r, c in self.groups])
 
@@ -399,25 +413,29 @@ def _put_bits(bitbuf: np.ndarray, pos: np.ndarray, codes: np.ndarray, rate: int)
 def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
     """Bytes of one (batch row, KV head) cache holding tokens 0..n-1 of ``enc``.
 
-    Tile of 64 tokens = [K records, token-major, LSB-first bitstream in packed-dim order]
-    [V codes: four 16-token chunks, each a bitstream where (dim d, token j) sits at bit
-    (16 d + slot(j)) b_V] [K norms fp32, group-major] [V norms fp32]. Unused slots are 0.
+    Tile of 64 tokens = [K codes: one block per 16-dimension key chunk, in chunk order; a
+    block is an LSB-first bitstream where token j's codes of the chunk's dims sit at bit
+    j * dims * rate, dim i of the chunk at + i * rate] [V codes: four 16-token chunks, each
+    a bitstream where (dim d, token j) sits at bit (16 d + slot(j)) b_V] [K norms fp32,
+    group-major] [V norms fp32]. Unused slots are 0.
     """
     n = enc["k_codes"].shape[0]
     if capacity % TILE_TOKENS or n > capacity:
         raise ValueError("capacity must be a multiple of 64 and hold the tokens")
     ntile = capacity // TILE_TOKENS
     out = np.zeros((ntile, layout.tile_bytes), dtype=np.uint8)
-    rates = layout.packed_rates()
-    koff = np.concatenate([[0], np.cumsum(rates)[:-1]])
     kb, vb, ng = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups
-    # K records
-    kbits = np.zeros((ntile * TILE_TOKENS, kb * 8), dtype=np.uint8)
-    for p in range(HEAD_DIM):
-        for i in range(rates[p]):
-            kbits[:n, koff[p] + i] = (enc["k_codes"][:, p] >> i) & 1
-    krec = np.packbits(kbits, axis=1, bitorder="little").reshape(ntile, TILE_TOKENS * kb)
-    out[:, :TILE_TOKENS * kb] = krec
+    # K area: chunk-major blocks (see Layout.k_chunks)
+    kcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
+    kcodes[:n] = enc["k_codes"]
+    kcodes = kcodes.reshape(ntile, TILE_TOKENS, HEAD_DIM)
+    for p0, nd, r, off in layout.k_chunks():
+        w = nd * r
+        bits = np.zeros((ntile, TILE_TOKENS * w), dtype=np.uint8)
+        for i in range(nd):
+            for bit in range(r):
+                bits[:, np.arange(TILE_TOKENS) * w + i * r + bit] = (kcodes[:, :, p0 + i] >> bit) & 1
+        out[:, off:off + TILE_TOKENS * w // 8] = np.packbits(bits, axis=1, bitorder="little")
     # V chunks
     br = layout.v_rate
     vcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
@@ -449,13 +467,14 @@ def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
     ntile = len(buf) // layout.tile_bytes
     t = np.asarray(buf, dtype=np.uint8).reshape(ntile, layout.tile_bytes)
     kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
-    rates = layout.packed_rates()
-    koff = np.concatenate([[0], np.cumsum(rates)[:-1]])
-    kbits = np.unpackbits(t[:, :TILE_TOKENS * kb].reshape(-1, kb), axis=1, bitorder="little").astype(np.int64)
-    kc = np.zeros((kbits.shape[0], HEAD_DIM), dtype=np.int64)
-    for p in range(HEAD_DIM):
-        for i in range(rates[p]):
-            kc[:, p] |= kbits[:, koff[p] + i] << i
+    kc = np.zeros((ntile, TILE_TOKENS, HEAD_DIM), dtype=np.int64)
+    for p0, nd, r, off in layout.k_chunks():
+        w = nd * r
+        bits = np.unpackbits(t[:, off:off + TILE_TOKENS * w // 8], axis=1, bitorder="little").astype(np.int64)
+        for i in range(nd):
+            for bit in range(r):
+                kc[:, :, p0 + i] |= bits[:, np.arange(TILE_TOKENS) * w + i * r + bit] << bit
+    kc = kc.reshape(-1, HEAD_DIM)
     base = TILE_TOKENS * kb
     vbits = np.unpackbits(t[:, base:base + TILE_TOKENS * vb].reshape(ntile, TILE_TOKENS // CHUNK_TOKENS, -1),
                           axis=2, bitorder="little").astype(np.int64)

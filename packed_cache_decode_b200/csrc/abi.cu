@@ -116,7 +116,11 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   size_t off = 256;  // status word first
   D.status = reinterpret_cast<unsigned*>(dptr);
   for (int g = 0; g <= ng; ++g) {
-    std::memcpy(host.data() + off, L->rot[g].data(), L->rot[g].size() * sizeof(double));
+    // fp64 copies are stored transposed (element (i, j) at j * d + i) for coalesced reads
+    const int d = int(std::lround(std::sqrt(double(L->rot[g].size()))));
+    double* h64 = reinterpret_cast<double*>(host.data() + off);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) h64[size_t(j) * d + i] = L->rot[g][size_t(i) * d + j];
     const double* p = reinterpret_cast<const double*>(dptr + off);
     if (g < ng) D.k_rot64[g] = p; else D.v_rot64 = p;
     off += L->rot[g].size() * sizeof(double);
@@ -181,13 +185,14 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     off += lut_words * 4;
   }
   {
-    int ci = 0;
+    int ci = 0, koff = 0;
     for (int g = 0; g < ng; ++g) {
       const int r = L->group_rate[g], d = L->group_dim[g];
       D.group_chunk0[g] = ci;
       D.group_nchunks[g] = (d + 15) / 16;
       for (int cc = 0; cc < D.group_nchunks[g]; ++cc, ++ci) {
-        D.chunk_bit[ci] = L->group_bitoff[g] + 16 * cc * r;
+        D.chunk_koff[ci] = koff;
+        koff += kTile * std::min(16, d - 16 * cc) * r / 8;
         D.chunk_dim0[ci] = L->group_off[g] + 16 * cc;
         D.chunk_ndim[ci] = std::min(16, d - 16 * cc);
         D.chunk_group[ci] = g;

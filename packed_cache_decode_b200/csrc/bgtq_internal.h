@@ -33,8 +33,8 @@ struct DevLayout {
   short packed_coord[kD];        // packed key dimension -> original coordinate
   float centroid[5][16];         // [rate][code], fp32
   double threshold[5][16];       // [rate][k], fp64 (2^rate - 1 used)
-  const double* k_rot64[kMaxGroups];  // d_g x d_g row-major, y = R x
-  const double* v_rot64;
+  const double* k_rot64[kMaxGroups];  // d_g x d_g, TRANSPOSED: element (i, j) of R at j * d + i
+  const double* v_rot64;              // 128 x 128, transposed likewise
   const float* k_rot32[kMaxGroups];
   const float* k_rot32t[kMaxGroups];  // transposed copies (column-major), back to back
   int k_rot32t_off[kMaxGroups];       // float offset of group g's copy from k_rot32t[0]
@@ -45,7 +45,7 @@ struct DevLayout {
   int n_kchunks;
   int group_chunk0[kMaxGroups];
   int group_nchunks[kMaxGroups];
-  int chunk_bit[kMaxChunks];     // first bit of the chunk inside a K record
+  int chunk_koff[kMaxChunks];    // byte offset of the chunk's block inside a tile (chunk-major keys)
   int chunk_dim0[kMaxChunks];    // first packed dimension of the chunk
   int chunk_ndim[kMaxChunks];    // valid dimensions in the chunk (<= 16)
   int chunk_group[kMaxChunks];

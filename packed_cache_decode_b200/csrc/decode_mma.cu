@@ -40,7 +40,7 @@ namespace bgtq {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kStages = 4;
+constexpr int kStages = 8;
 constexpr int kWarps = 4;
 constexpr unsigned kWaitLimit = 1u << 22;
 constexpr int kMergeFloats = kWarps * 8 * kD;  // the consumer warps' [8][128] partials
@@ -311,67 +311,76 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // Scores of one key group with compile-time rate R: for each 16-dimension chunk, the
 // thread's four codes (dims 4t..4t+3 of the chunk) of tokens g and g+8 index the pair
 // tables; q' hi and lo are the B operands. The bit offset advances 16 R per chunk.
-// Per chunk the thread forms its A fragments from the four codes of tokens g and g+8
-// (dims 4t..4t+3 of the chunk). Products with q' hi and q' lo (and, for rates 3-4, the
-// centroid low parts) go to separate accumulators, and consecutive chunks alternate
-// between two accumulator sets, so the mma dependency chains stay short.
+// Per chunk the thread forms its A fragments from the four codes (dims 4t..4t+3 of the
+// chunk) of its two tokens in each of the tile's four 16-token row blocks, and multiplies
+// them with the q' hi and lo fragments (and, for rates 3-4, the centroid low parts).
+// The four row blocks are independent accumulation chains.
 template <int R>
-__device__ __forceinline__ void key_chunk(float (&ah)[4], float (&al)[4], unsigned f0, unsigned f1, uint2 bh,
-                                          uint2 bl, const unsigned* klut12, const uint2* klut1q,
-                                          const uint2* klut34) {
+__device__ __forceinline__ void key_chunk(float (&acc)[4], unsigned f0, unsigned f1, uint2 bh, uint2 bl,
+                                          const unsigned* klut12, const uint2* klut1q, const uint2* klut34) {
   constexpr unsigned M = (1u << (2 * R)) - 1u;
   if constexpr (R == 1) {
     // the four 1-bit codes of a token index one entry: {pair (4t, 4t+1), pair (4t+2, 4t+3)}
     const uint2 e0 = klut1q[f0 & 15u], e1 = klut1q[f1 & 15u];
-    mma16816(ah, e0.x, e1.x, e0.y, e1.y, bh.x, bh.y);
-    mma16816(al, e0.x, e1.x, e0.y, e1.y, bl.x, bl.y);
+    mma16816(acc, e0.x, e1.x, e0.y, e1.y, bh.x, bh.y);
+    mma16816(acc, e0.x, e1.x, e0.y, e1.y, bl.x, bl.y);
   } else if constexpr (R == 2) {
     const unsigned* lut = klut12 + 4;
     const unsigned a0 = lut[f0 & M], a2 = lut[(f0 >> 4) & M];
     const unsigned a1 = lut[f1 & M], a3 = lut[(f1 >> 4) & M];
-    mma16816(ah, a0, a1, a2, a3, bh.x, bh.y);
-    mma16816(al, a0, a1, a2, a3, bl.x, bl.y);
+    mma16816(acc, a0, a1, a2, a3, bh.x, bh.y);
+    mma16816(acc, a0, a1, a2, a3, bl.x, bl.y);
   } else {
     const uint2* lut = klut34 + (R == 3 ? 0 : 64);
     const uint2 e0 = lut[f0 & M], e2 = lut[(f0 >> (2 * R)) & M];
     const uint2 e1 = lut[f1 & M], e3 = lut[(f1 >> (2 * R)) & M];
-    mma16816(ah, e0.x, e1.x, e2.x, e3.x, bh.x, bh.y);
-    mma16816(al, e0.x, e1.x, e2.x, e3.x, bl.x, bl.y);
-    mma16816(al, e0.y, e1.y, e2.y, e3.y, bh.x, bh.y);
+    mma16816(acc, e0.x, e1.x, e2.x, e3.x, bh.x, bh.y);
+    mma16816(acc, e0.x, e1.x, e2.x, e3.x, bl.x, bl.y);
+    mma16816(acc, e0.y, e1.y, e2.y, e3.y, bh.x, bh.y);
   }
 }
 
+// Keys are chunk-major inside a tile: chunk c's block holds the 64 tokens' fields of
+// dims_c * R bits back to back. For a full chunk (16 dims) the thread's four codes of
+// token j sit in one word: R = 1: word j/2 at bit 16 (j%2) + 4t; R = 2: word j at 8t;
+// R = 4: word 2j + t/2 at 16 (t%2). Rate 3 and partial chunks use a 64-bit window.
 template <int R>
-__device__ __forceinline__ void key_group(float (&acc)[4], const unsigned* rec0, const unsigned* rec1,
-                                          const uint2* qf, int c0, int c1, int bit, int lane,
-                                          const unsigned* klut12, const uint2* klut1q, const uint2* klut34) {
-  float a[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a[i][j] = 0.f;
+__device__ __forceinline__ void key_group(float (&acc)[4][4], const unsigned char* tb, const DevLayout& L,
+                                          const uint2* qf, int c0, int c1, int lane, const unsigned* klut12,
+                                          const uint2* klut1q, const uint2* klut34) {
+  const int g = lane >> 2, t = lane & 3;
   const uint2* qp = qf + c0 * 64 + lane;
-  int ci = c0;
-  for (; ci + 1 < c1; ci += 2, bit += 32 * R, qp += 128) {
-    const int b1 = bit + 16 * R;
-    const unsigned* p0 = rec0 + (bit >> 5);
-    const unsigned* p1 = rec1 + (bit >> 5);
-    const unsigned* q0 = rec0 + (b1 >> 5);
-    const unsigned* q1 = rec1 + (b1 >> 5);
-    const unsigned f0 = __funnelshift_r(p0[0], p0[1], bit & 31), f1 = __funnelshift_r(p1[0], p1[1], bit & 31);
-    const unsigned g0 = __funnelshift_r(q0[0], q0[1], b1 & 31), g1 = __funnelshift_r(q1[0], q1[1], b1 & 31);
-    const uint2 bh0 = qp[0], bl0 = qp[32], bh1 = qp[64], bl1 = qp[96];
-    key_chunk<R>(a[0], a[1], f0, f1, bh0, bl0, klut12, klut1q, klut34);
-    key_chunk<R>(a[2], a[3], g0, g1, bh1, bl1, klut12, klut1q, klut34);
-  }
-  if (ci < c1) {
-    const unsigned* p0 = rec0 + (bit >> 5);
-    const unsigned* p1 = rec1 + (bit >> 5);
-    const unsigned f0 = __funnelshift_r(p0[0], p0[1], bit & 31), f1 = __funnelshift_r(p1[0], p1[1], bit & 31);
-    key_chunk<R>(a[0], a[1], f0, f1, qp[0], qp[32], klut12, klut1q, klut34);
-  }
+  for (int ci = c0; ci < c1; ++ci, qp += 64) {
+    const uint2 bh = qp[0], bl = qp[32];
+    const unsigned* blk = reinterpret_cast<const unsigned*>(tb + L.chunk_koff[ci]);
+    const int nd = L.chunk_ndim[ci];
+    if (R != 3 && nd == 16) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) acc[j] = (a[0][j] + a[1][j]) + (a[2][j] + a[3][j]);
+      for (int rt = 0; rt < 4; ++rt) {
+        const int j0 = 16 * rt + g, j1 = j0 + 8;
+        unsigned f0, f1;
+        if constexpr (R == 1) {
+          f0 = blk[j0 >> 1] >> (16 * (g & 1) + 4 * t);
+          f1 = blk[j1 >> 1] >> (16 * (g & 1) + 4 * t);
+        } else if constexpr (R == 2) {
+          f0 = blk[j0] >> (8 * t);
+          f1 = blk[j1] >> (8 * t);
+        } else {
+          f0 = blk[2 * j0 + (t >> 1)] >> (16 * (t & 1));
+          f1 = blk[2 * j1 + (t >> 1)] >> (16 * (t & 1));
+        }
+        key_chunk<R>(acc[rt], f0, f1, bh, bl, klut12, klut1q, klut34);
+      }
+    } else {
+      const int w = nd * R;
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt) {
+        const int j0 = 16 * rt + g;
+        const unsigned f0 = bits32(blk, j0 * w + 4 * t * R), f1 = bits32(blk, (j0 + 8) * w + 4 * t * R);
+        key_chunk<R>(acc[rt], f0, f1, bh, bl, klut12, klut1q, klut34);
+      }
+    }
+  }
 }
 
 // Value codes for the PV product. MMA row r of m-tile mt stands for value dimension
@@ -421,7 +430,7 @@ struct ValueRows {
 };
 
 template <int VR>
-__global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int s = blockIdx.x, u = blockIdx.y;
   const int b = u / a.h_kv;
@@ -437,9 +446,10 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
   uint2* klut34 = reinterpret_cast<uint2*>(klut12 + 32);
   uint2* klut1q = klut34 + 320;                       // rate 1, four codes per entry
   unsigned* vlut = reinterpret_cast<unsigned*>(klut1q + 16);
-  float* mo = reinterpret_cast<float*>(vlut + 256);  // merge: [warp][8][128]
-  float* mm = mo + kMergeFloats;                      // [warp][8]
+  float* mm = reinterpret_cast<float*>(vlut + 256);  // [warp][8]
   float* ml = mm + kConsumers * 8;                    // [warp][8]
+  // the warps' [8][128] partials reuse the ring once every tile has been consumed
+  float* mo = reinterpret_cast<float*>(ring);
   __shared__ int s_timeout;
 
   long long len = a.seq_lens[b];
@@ -459,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
     s_timeout = 0;
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kConsumers);
+      mbar_init(&empty[i], 1);
     }
     fence_mbar_init();
     for (int it = 0; it < min(kStages, ntiles); ++it) {
@@ -509,9 +519,9 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
 #pragma unroll
     for (int j = 0; j < 4; ++j) O[mt][j] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const int tok0 = 16 * warp + g;
 
-  for (int it = 0; it < ntiles; ++it) {
+  // warp w takes tiles w, w+4, w+8, ... of this split; a whole 64-token tile per warp
+  for (int it = warp; it < ntiles; it += kConsumers) {
     const int stage = it % kStages;
     if (!mbar_wait_bounded(&full[stage], (it / kStages) & 1)) {
       // stop consuming; the producer waits for its own copies and this unit's result
@@ -523,36 +533,53 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
       break;
     }
     const unsigned char* tb = ring + stage * TB;
-    const long long gtok = (long long)(t0 + it) * kTile + tok0;
+    const long long gt0 = (long long)(t0 + it) * kTile + g;  // token of row g in row block 0
 
-    // ---------------- scores: per key group, rate as a template parameter
-    const unsigned* rec0 = reinterpret_cast<const unsigned*>(tb + tok0 * L.k_record_bytes);
-    const unsigned* rec1 = reinterpret_cast<const unsigned*>(tb + (tok0 + 8) * L.k_record_bytes);
+    // ---------------- scores of the tile's 64 tokens: per key group (rate as a template
+    // parameter), per chunk, four row blocks; then times the group norms
     const float* kn = reinterpret_cast<const float*>(tb + L.knorm_off);
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    float sc[4][4];
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sc[rt][j] = 0.f;
     for (int gi = 0; gi < L.n_kgroups; ++gi) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc[4][4];
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[rt][j] = 0.f;
       const int r = L.group_rate[gi], c0 = L.group_chunk0[gi], c1 = c0 + L.group_nchunks[gi];
-      const int bit = L.group_bitoff[gi] + 4 * t * r;
       switch (r) {
-        case 1: key_group<1>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
-        case 2: key_group<2>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
-        case 3: key_group<3>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
-        default: key_group<4>(acc, rec0, rec1, qf, c0, c1, bit, lane, klut12, klut1q, klut34); break;
+        case 1: key_group<1>(acc, tb, L, qf, c0, c1, lane, klut12, klut1q, klut34); break;
+        case 2: key_group<2>(acc, tb, L, qf, c0, c1, lane, klut12, klut1q, klut34); break;
+        case 3: key_group<3>(acc, tb, L, qf, c0, c1, lane, klut12, klut1q, klut34); break;
+        default: key_group<4>(acc, tb, L, qf, c0, c1, lane, klut12, klut1q, klut34); break;
       }
       const float ik = L.inv_kappa_group[gi];
-      const float n0 = kn[gi * kTile + tok0] * ik;
-      const float n1 = kn[gi * kTile + tok0 + 8] * ik;
-      sc[0] = fmaf(acc[0], n0, sc[0]);
-      sc[1] = fmaf(acc[1], n0, sc[1]);
-      sc[2] = fmaf(acc[2], n1, sc[2]);
-      sc[3] = fmaf(acc[3], n1, sc[3]);
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt) {
+        const float n0 = kn[gi * kTile + 16 * rt + g] * ik;
+        const float n1 = kn[gi * kTile + 16 * rt + g + 8] * ik;
+        sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
+        sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
+        sc[rt][2] = fmaf(acc[rt][2], n1, sc[rt][2]);
+        sc[rt][3] = fmaf(acc[rt][3], n1, sc[rt][3]);
+      }
     }
-    if (gtok >= len) sc[0] = sc[1] = -INFINITY;
-    if (gtok + 8 >= len) sc[2] = sc[3] = -INFINITY;
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt) {
+      if (gt0 + 16 * rt >= len) sc[rt][0] = sc[rt][1] = -INFINITY;
+      if (gt0 + 16 * rt + 8 >= len) sc[rt][2] = sc[rt][3] = -INFINITY;
+    }
 
-    // ---------------- online softmax (heads 2t, 2t+1; token rows g, g+8), base 2
-    float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+    // ---------------- online softmax over the 64 tokens (heads 2t, 2t+1), base 2
+    float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt) {
+      x0 = fmaxf(x0, fmaxf(sc[rt][0], sc[rt][2]));
+      x1 = fmaxf(x1, fmaxf(sc[rt][1], sc[rt][3]));
+    }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
@@ -562,14 +589,12 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
     // rows that are still all -inf keep a zero weight and leave the accumulators alone
     const float b0m = n0m == -INFINITY ? 0.f : n0m, b1m = n1m == -INFINITY ? 0.f : n1m;
     const float corr0 = fast_exp2(m0 - b0m), corr1 = fast_exp2(m1 - b1m);
-    const float p0 = fast_exp2(sc[0] - b0m), p1 = fast_exp2(sc[1] - b1m);
-    const float p2 = fast_exp2(sc[2] - b0m), p3 = fast_exp2(sc[3] - b1m);
     const bool rescale = !__all_sync(0xffffffffu, n0m == m0 && n1m == m1);
     m0 = n0m;
     m1 = n1m;
-    l0 = fmaf(l0, corr0, p0 + p2);
-    l1 = fmaf(l1, corr1, p1 + p3);
     if (rescale) {
+      l0 *= corr0;
+      l1 *= corr1;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
         O[mt][0] *= corr0;
@@ -579,14 +604,19 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
       }
     }
     const float* vn = reinterpret_cast<const float*>(tb + L.vnorm_off);
-    const float av0 = vn[tok0] * vscale, av1 = vn[tok0 + 8] * vscale;
-    const unsigned pb0 = movmatrix_trans(pack_h2(p0 * av0, p1 * av0));
-    const unsigned pb1 = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
 
-    // ---------------- values
-    {
+    // ---------------- values: row block rt is value chunk rt of the tile
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt) {
+      const float p0 = fast_exp2(sc[rt][0] - b0m), p1 = fast_exp2(sc[rt][1] - b1m);
+      const float p2 = fast_exp2(sc[rt][2] - b0m), p3 = fast_exp2(sc[rt][3] - b1m);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+      const float av0 = vn[16 * rt + g] * vscale, av1 = vn[16 * rt + g + 8] * vscale;
+      const unsigned pb0 = movmatrix_trans(pack_h2(p0 * av0, p1 * av0));
+      const unsigned pb1 = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
       ValueRows<VR> vr;
-      vr.load(reinterpret_cast<const unsigned*>(tb + L.vcode_off + warp * 256 * VR), g, t);
+      vr.load(reinterpret_cast<const unsigned*>(tb + L.vcode_off + rt * 256 * VR), g, t);
       constexpr unsigned vm = (1u << (2 * VR)) - 1u;
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
@@ -601,7 +631,10 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
   }
 
   pdl_trigger();
-  // ---------------- merge the consumer warps
+  // ---------------- merge the consumer warps (their partials reuse the ring: wait until
+  // every warp is done with its tiles; after a timeout copies may still be in flight)
+  consumer_sync();
+  if (*static_cast<volatile int*>(&s_timeout)) return;  // uniform over the consumer warps
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -622,7 +655,6 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
     ml[warp * 8 + 2 * t + 1] = l1;
   }
   consumer_sync();
-  if (*static_cast<volatile int*>(&s_timeout)) return;  // uniform over the consumer warps
   const int G = a.G;
   for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
@@ -648,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 4) split_kernel(DevLayout L, SplitAr
 
 size_t split_smem_bytes(int tile_bytes) {
   return 128 + size_t(kStages) * tile_bytes + 64 + kMaxChunks * 2 * 32 * sizeof(uint2) + 32 * 4 + 320 * 8 + 16 * 8 +
-         256 * 4 + (kMergeFloats + 2 * kConsumers * 8) * sizeof(float);
+         256 * 4 + 2 * kConsumers * 8 * sizeof(float);
 }
 
 template <int VR>
@@ -684,7 +716,7 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
   p.max_tiles = int((max_seq_len + kTile - 1) / kTile);
   if (p.max_tiles < 1) p.max_tiles = 1;
   const long long units = (long long)batch * h_kv;
-  const long long target = 4LL * num_sms;
+  const long long target = 3LL * num_sms;
   long long splits = (target + units - 1) / units;
   if (splits < 1) splits = 1;
   if (splits > p.max_tiles) splits = p.max_tiles;

@@ -147,10 +147,11 @@ def test_capacity_overflow_is_flagged_and_skipped():
     assert lay.status() == 0                           # cleared by the previous read
     # positions 60..63 were written, 64..67 skipped: only tokens 60..63 of the tile changed
     olay = O.make_layout(rates, 2, case.seed)
-    diff = np.nonzero((before != cache).cpu().numpy())[0]
-    kb = olay.k_record_bytes
-    krec_changed = sorted(set(i // kb for i in diff if i < 64 * kb))
-    assert krec_changed and min(krec_changed) >= 60
+    u0 = O.unpack(olay, before.cpu().numpy(), 64)
+    u1 = O.unpack(olay, cache.cpu().numpy(), 64)
+    changed = sorted(set(np.nonzero((u0["k_codes"] != u1["k_codes"]).any(1) | (u0["v_codes"] != u1["v_codes"]).any(1)
+                                    | (u0["k_norms"] != u1["k_norms"]).any(1) | (u0["v_norm"] != u1["v_norm"]))[0]))
+    assert changed and min(changed) >= 60
 
 
 def test_decode_clamps_overlong_lengths():

@@ -208,10 +208,13 @@ def test_grouping_and_byte_formula():
 
 def test_pack_places_bits_where_the_format_says():
     lay = O.make_layout(np.array([2] * 32 + [1] * 32), 3, 5)   # packed dims 0..63 rate 2, 64..127 rate 1
+    assert [c[1:] for c in lay.k_chunks()] == [(16, 2, 0), (16, 2, 256), (16, 2, 512), (16, 2, 768),
+                                               (16, 1, 1024), (16, 1, 1152), (16, 1, 1280), (16, 1, 1408)]
     enc = {"k_codes": np.zeros((3, 128), dtype=np.int64), "v_codes": np.zeros((3, 128), dtype=np.int64),
            "k_norms": np.zeros((3, 2)), "v_norm": np.zeros(3)}
-    enc["k_codes"][2, 5] = 3          # token 2, packed dim 5 (rate 2): bits 10,11 of record 2
-    enc["k_codes"][1, 64] = 1         # token 1, packed dim 64 (rate 1): bit 128 of record 1
+    enc["k_codes"][2, 5] = 3          # token 2, packed dim 5: chunk 0 (32 bits per token), bits 64+10, 64+11
+    enc["k_codes"][1, 64] = 1         # token 1, packed dim 64: chunk 4 at byte 1024, 16 bits per token: bit 16
+    enc["k_codes"][0, 127] = 1        # token 0, packed dim 127: chunk 7 at byte 1408, dim 15: bit 15
     enc["v_codes"][1, 7] = 5          # token 1, dim 7, rate 3: chunk 0, bit (16*7 + slot(1))*3
     enc["v_codes"][2, 0] = 6          # token 2 -> slot 4: bits 12..14 of chunk 0
     enc["k_norms"][1] = [1.5, -2.0]
@@ -219,8 +222,9 @@ def test_pack_places_bits_where_the_format_says():
     buf = O.pack(lay, enc, 64)
     kb = lay.k_record_bytes
     assert kb == 24 and lay.tile_bytes == 64 * (24 + 48 + 12) and buf.size == lay.tile_bytes
-    assert buf[2 * kb + 1] == 0b00001100
-    assert buf[1 * kb + 16] == 1
+    assert buf[9] == 0b00001100
+    assert buf[1024 + 2] == 1
+    assert buf[1408 + 1] == 0b10000000
     vbase = 64 * kb
     bit = (16 * 7 + 1) * 3
     assert (int.from_bytes(buf[vbase:vbase + 8 * 48].tobytes(), "little") >> bit) & 7 == 5
@@ -230,10 +234,22 @@ def test_pack_places_bits_where_the_format_says():
     assert kn[1] == 1.5 and kn[64 + 1] == -2.0
     assert buf[nbase + 512:nbase + 768].view(np.float32)[2] == 0.25
     # nothing else written: one byte per code, and 1.5 / -2.0 / 0.25 have 2 / 1 / 2 nonzero bytes
-    assert int(np.count_nonzero(buf)) == 4 + 2 + 1 + 2
+    assert int(np.count_nonzero(buf)) == 5 + 2 + 1 + 2
     u = O.unpack(lay, buf, 3)
     np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
     np.testing.assert_array_equal(u["v_codes"], enc["v_codes"])
+
+
+def test_partial_chunks_are_packed_densely():
+    rates = np.array([4] * 3 + [3] * 5 + [2] * 9 + [1] * 47)     # group dims 6, 10, 18, 94
+    assert rates.sum() % 4 == 0
+    lay = O.make_layout(rates, 2, 1)
+    ch = lay.k_chunks()
+    assert [(nd, r) for _, nd, r, _ in ch] == [(6, 4), (10, 3), (16, 2), (2, 2), (16, 1), (16, 1), (16, 1),
+                                               (16, 1), (16, 1), (14, 1)]
+    end = ch[-1][3] + 64 * ch[-1][1] * ch[-1][2] // 8
+    assert end == 64 * lay.k_record_bytes                      # no padding
+    assert all(off % 16 == 0 for *_, off in ch)                # every block starts 16-byte aligned
 
 
 def test_chunk_slot_is_a_permutation():
