@@ -21,7 +21,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -50,56 +49,85 @@ def _peaks():
 
 # ------------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples the GPU's SM clock and clock-event reasons through NVML every 10 ms on a
+    host thread (reads only; nothing is set). mark() notes host times; summary(t0, t1)
+    reports the samples taken between two marks."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    REASONS = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+               "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap",
+               "hw_power_brake": "HwPowerBrakeSlowdown"}
 
-    def __enter__(self):
+    def __init__(self, device: torch.device):
+        self.dev = device
+        self.samples = []          # (host time, sm MHz, reason bits)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nv = None
+        self._h = None
+        self.error = None
+
+    def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            p = torch.cuda.get_device_properties(self.dev)
+            try:
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                self._h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+            self._nv = nv
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM))
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+            t_end = time.monotonic() + 5.0
+            while not self.samples and time.monotonic() < t_end:
+                time.sleep(0.005)
+        except Exception as e:       # no NVML: the line says so instead of guessing
+            self.error = f"{type(e).__name__}: {e}"
         return self
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
-
-    def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
             try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+                mhz = float(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+                self.samples.append((time.monotonic(), mhz, bits))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            self._stop.wait(0.01)
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+    @staticmethod
+    def mark():
+        return time.monotonic()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        if self.error and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled: " + self.error], "samples": 0}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if not win:                    # timed region shorter than the sampling period
+            later = [s for s in self.samples if s[0] >= t0]
+            win = later[:1]
+            window = "first sample after the timed region started"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        reasons = set()
+        for _, _, bits in win:
+            for name, nvname in self.REASONS.items():
+                mask = getattr(self._nv, "nvmlClocksEventReason" + nvname, 0)
+                if bits & mask:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in win]), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win), "window": window}
 
 
 # ------------------------------------------------------------------------ workload
@@ -142,7 +170,7 @@ class Model:
                 "out": torch.empty(Bt, hq, 128, dtype=torch.float32, device=device),
             })
         torch.cuda.synchronize(device)
-        self.lens_before = torch.full((Bt,), L - 1, dtype=torch.int32, device=device)
+        self.lens_before = torch.full((Bt,), L - 1, dtype=torch.int32, device=device)   # the step appends token L-1
         self.lens_after = torch.full((Bt,), L, dtype=torch.int32, device=device)
         ws = max(B.workspace_bytes(x["layout"], Bt, hq, hkv, L) for x in self.layers)
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
@@ -168,12 +196,15 @@ class Model:
         x = _rope_dev(x, torch.tensor([pos], device=self.dev), self.wl.theta)
         return x[:, 0].contiguous().to(self.wl.dtype)
 
-    def step(self, stream, timing_events=None):
-        cap = self.capacity
-        for i, x in enumerate(self.layers):
-            B.encode_append(x["layout"], x["k_new"], x["v_new"], self.lens_before, x["cache"], cap, stream=stream)
-            B.decode_attention(x["layout"], x["q"], x["cache"], self.lens_after, cap, self.wl.length, x["out"],
-                               self.workspace, self.wl.h_kv, stream=stream)
+    # kernel launches of one layer: step = step_prep + split + combine; decode_only =
+    # qprep + split + combine
+    LAUNCHES_PER_LAYER = 3
+
+    def step(self, stream):
+        """Every layer: append the step's token and attend (one bgtq_decode_step call)."""
+        for x in self.layers:
+            B.decode_step(x["layout"], x["k_new"], x["v_new"], x["q"], x["cache"], self.lens_before, self.capacity,
+                          self.wl.length, x["out"], self.workspace, stream=stream)
 
     def decode_only(self, stream):
         for x in self.layers:
@@ -310,7 +341,7 @@ def run_encode(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama8b", choices=list(synth.WORKLOADS))
@@ -383,29 +414,35 @@ def main():
             pg.barrier()
         torch.cuda.synchronize(dev)
 
+    clk = ClockSampler(dev).start()
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             g_step.replay()
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(args.steps):
-                g_step.replay()
-            ev1.record(stream)
-        barrier()
-        step_ms = ev0.elapsed_time(ev1) / args.steps
-        # dominant kernel: decode attention, timed on its own stream over the same caches
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            d0.record(stream)
-            for _ in range(args.steps):
-                g_dec.replay()
-            d1.record(stream)
-        barrier()
-        dec_ms = d0.elapsed_time(d1) / (args.steps * wl.layers)
-    clocks = clk.summary()
+    t_on = clk.mark()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            g_step.replay()
+        ev1.record(stream)
+    barrier()
+    t_off = clk.mark()
+    step_ms = ev0.elapsed_time(ev1) / args.steps
+    # dominant kernels: the decode attention call of each layer (qprep -> split -> combine),
+    # timed on their own stream over the same caches
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_dec.replay()
+        d0.record(stream)
+        for _ in range(args.steps):
+            g_dec.replay()
+        d1.record(stream)
+    barrier()
+    dec_ms = d0.elapsed_time(d1) / (args.steps * wl.layers)
+    clk.stop()
+    clocks = clk.summary(t_on, t_off)
 
     # end to end through the public API with host buffers (pinned), copies inside the timing
     h_q = [x["q"].cpu().pin_memory() for x in model.layers]
@@ -455,16 +492,16 @@ def main():
             "config": {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "context": wl.length,
                        "h_q": wl.h_q, "h_kv": wl.h_kv, "rates": f"K{wl.k_bits}V{wl.v_bits}",
                        "bytes_per_token_head": model.layers[0]["layout"].bytes_per_token,
-                       "step": "per layer: encode-append 1 token + decode attention; CUDA graph",
+                       "step": "per layer: bgtq_decode_step (append 1 token + decode attention); CUDA graph",
                        "l2": f"inputs larger than L2: {model.bytes_per_step / 1e6:.0f} MB of packed caches per step",
                        "parallelism": f"replicas x{world} (independent sequences per GPU)"},
             "gbs": model.bytes_per_step / (step_ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
-                         "kernel": "decode_attention (split + combine), per layer launch",
+                         "kernel": "decode attention call per layer (qprep -> split -> combine, PDL-chained)",
                          "peak_kind": peak_kind},
             "clocks": clocks,
-            "gpu_launches": args.steps * wl.layers * 3,
+            "gpu_launches": args.steps * wl.layers * Model.LAUNCHES_PER_LAYER,
             "e2e": {"value": keys / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }

@@ -171,6 +171,19 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* layout, const void* q, int 
                                   float softmax_scale, float* out, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* One decode step of one layer [TQ pipeline; BGTQ s5, s8]: appends n_new tokens per row,
+ * then attends the query over the grown cache. The same results as bgtq_encode_append
+ * (k_new, v_new, kv_dtype, n_new, seq_lens_dev) followed by bgtq_decode_attention over
+ * seq_lens_dev[b] + n_new tokens, in one chain of three kernels: the encode and the
+ * rotation of q share the first launch. seq_lens_dev[batch] int32 device = tokens cached
+ * before the step (not modified; the caller advances it). max_seq_len >= every
+ * seq_lens_dev[b] + n_new; workspace as for bgtq_decode_attention. n_new = 0 attends only. */
+bgtq_status bgtq_decode_step(const bgtq_layout* layout, const void* k_new, const void* v_new,
+                             int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,
+                             int h_kv, void* cache, const int* seq_lens_dev, long long capacity,
+                             long long max_seq_len, float softmax_scale, float* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- no-allocation variant */
 
 /* The pages have no counterpart to this call: it is a library convenience.

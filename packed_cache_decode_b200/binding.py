@@ -26,7 +26,7 @@ EXPORTED = [
     "bgtq_layout_create", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
     "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
-    "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity",
+    "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step",
 ]
 
 
@@ -70,6 +70,7 @@ def load():
         "bgtq_device_status": (I, [P, C.POINTER(C.c_uint), I]),
         "bgtq_decode_attention_noalloc": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P]),
         "bgtq_noalloc_scratch_capacity": (C.c_size_t, []),
+        "bgtq_decode_step": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -241,6 +242,24 @@ def decode_attention(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_
            "decode_attention")
 
 
+def decode_step(layout: Layout, k_new, v_new, q, cache, seq_lens, capacity: int, max_seq_len: int, out, workspace,
+                softmax_scale: float | None = None, stream=None):
+    """Append k_new, v_new [B, n_new, h_kv, 128] at seq_lens[b] (int32 CUDA, not advanced)
+    and attend q [B, h_q, 128] over seq_lens[b] + n_new tokens; out [B, h_q, 128] fp32."""
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and k_new.is_contiguous() and v_new.is_contiguous()
+    assert v_new.shape == k_new.shape and v_new.dtype == k_new.dtype
+    Bq, h_q, dq = q.shape
+    assert Bq == B_ and dq == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step(layout.handle, C.c_void_p(k_new.data_ptr()), C.c_void_p(v_new.data_ptr()),
+                                   dtype_code(k_new), n_new, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q, h_kv,
+                                   C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                   max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                   C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_step")
+
+
 def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out,
                              h_kv: int, softmax_scale: float | None = None, stream=None):
     """decode_attention for callers that cannot allocate device memory: the split-K
@@ -254,21 +273,6 @@ def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, 
                                                 capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
                                                 _stream_ptr(stream)),
            "decode_attention_noalloc")
-
-
-@dataclass
-class PackedLayer:
-    """One layer's packed cache and the device buffers its calls need (caller-owned)."""
-
-    layout: Layout
-    cache: object
-    seq_lens: object
-    capacity: int
-    batch: int
-    h_q: int
-    h_kv: int
-    workspace: object = None
-    out: object = None
 
 
 def plan_layer_rates(q_cal, k_cal, avg_bits: int, min_rate: int = 1, max_rate: int = 4) -> np.ndarray:

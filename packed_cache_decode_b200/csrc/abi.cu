@@ -291,6 +291,39 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dty
   return BGTQ_OK;
 }
 
+bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype, int n_new,
+                             const void* q, int q_dtype, int batch, int h_q, int h_kv, void* cache,
+                             const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                             float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  bgtq_status st = check_device(L, "decode_step");
+  if (st != BGTQ_OK) return st;
+  if (!valid_dtype(kv_dtype) || !valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_step: bad dtype");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
+    return fail(BGTQ_ERR_INVALID, "decode_step: need h_q = G * h_kv with G in 1..8");
+  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_step: batch * h_kv > 65535");
+  if (n_new < 0 || (long long)n_new * kEncodeParts * batch * h_kv + (long long)batch * h_kv > 0x7fffffffLL)
+    return fail(BGTQ_ERR_INVALID, "decode_step: bad n_new");
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, "decode_step: capacity must be a positive multiple of 64");
+  if (max_seq_len < 0 || max_seq_len > capacity)
+    return fail(BGTQ_ERR_CAPACITY, "decode_step: max_seq_len must be in [0, capacity]");
+  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_step: bad softmax_scale");
+  if (!q || !cache || !seq_lens_dev || !out || (n_new > 0 && (!k_new || !v_new)))
+    return fail(BGTQ_ERR_INVALID, "decode_step: null pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step");
+  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  if (!workspace || workspace_bytes < plan.workspace_bytes)
+    return fail(BGTQ_ERR_WORKSPACE, "decode_step: workspace missing or smaller than bgtq_workspace_bytes()");
+  e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch, h_q, h_kv,
+                         cache, capacity / kTile, softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step");
+  return BGTQ_OK;
+}
+
 bgtq_status bgtq_device_status(const bgtq_layout* L, unsigned* flags, int clear) {
   bgtq_status st = check_device(L, "device_status");
   if (st != BGTQ_OK) return st;

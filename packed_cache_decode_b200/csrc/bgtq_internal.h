@@ -16,6 +16,7 @@ constexpr int kChunk = 16;               // tokens per V-code chunk
 constexpr int kMaxG = BGTQ_MAX_GQA;
 constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
 constexpr int kMaxChunks = 12;           // sum over groups of ceil(d_g / 16) <= 128/16 + 4
+constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32 outputs each
 
 // Everything a kernel needs about one layer's packing, passed by value.
 struct DevLayout {

@@ -5,24 +5,26 @@
 //   q . k_hat   = sum_g (|k_g| / sqrt(d_g)) (R_g q_g) . c[codes_g]
 //   o           = R_V^T sum_t p_t (|v_t| / sqrt(128)) c[vcodes_t] / sum_t p_t.
 //
-// Three kernels per call:
+// Three kernels per call (a decode step that also appends the new token fuses the append
+// into the first one: step_prep_kernel runs the encode CTAs and the q-preparation CTAs):
 //  * qprep_kernel (one CTA per batch row x KV head): q' = R_g q_g for the G query heads
 //    (rotations staged in shared memory), scaled by softmax_scale * log2(e) / sqrt(d_g),
 //    split into fp16 hi + lo parts and laid out as mma B fragments.
-//  * split_kernel (one CTA per (split, unit), 4 warps): 64-token tiles arrive by 1-D bulk
-//    async copies (cp.async.bulk + mbarrier, no multicast) into a 4-stage ring. Warp w
-//    takes tokens 16w..16w+15 of each tile. Scores: for every 16-dimension chunk of a key
-//    group, the thread's code pairs index a pair table in shared memory (fp16 values, exact
-//    for rates 1-2 after a per-rate scale; hi + lo parts for rates 3-4) and mma.m16n8k16
-//    multiplies them with q' hi and lo (fp32 accumulators per group, then times the group
-//    norm). Online softmax in base 2 with warp shuffles. Values: the probabilities times
-//    |v|/sqrt(128) in fp16, transposed with movmatrix, against value-code pair lookups,
-//    accumulated in V's rotated space (fp32). The four warps merge and the CTA writes its
-//    partial (o', m, l). A fifth warp only issues the copies (full/empty mbarriers).
+//  * split_kernel (one CTA per (split, unit), 4 consumer warps + 1 producer warp): 64-token
+//    tiles arrive by 1-D bulk async copies (cp.async.bulk + mbarrier, no multicast) into an
+//    8-stage ring; consumer warp w takes tiles w, w+4, ... whole, as four 16-token row
+//    blocks. Scores: for every 16-dimension chunk of a key group, the thread's code pairs
+//    index a pair table in shared memory (fp16 values, exact for rates 1-2 after a per-rate
+//    scale; hi + lo parts for rates 3-4) and mma.m16n8k16 multiplies them with q' hi and lo
+//    (fp32 accumulators per group, then times the group norm). Online softmax in base 2
+//    with warp shuffles. Values: the probabilities times |v|/sqrt(128) in fp16, transposed
+//    with movmatrix, against value-code pair lookups, accumulated in V's rotated space
+//    (fp32). The four warps merge and the CTA writes its partial (o', m, l).
 //  * combine_kernel (one CTA per batch row x query head, 512 threads): log-sum-exp merge
 //    of the splits and o = R_V^T o'.
 // The three launches are chained with programmatic dependent launch, so each kernel's
-// set-up (and the split kernel's first tile copies) overlaps the previous kernel.
+// set-up (and, when the first kernel does not write the cache, the split kernel's first
+// tile copies) overlaps the previous kernel.
 //
 // Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, waits
 // (bounded) for its own copies in flight and returns.
@@ -33,6 +35,7 @@
 #include <cmath>
 
 #include "bgtq_internal.h"
+#include "encode_body.cuh"
 #include "kernels.h"
 
 namespace bgtq {
@@ -43,7 +46,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kStages = 8;
 constexpr int kWarps = 4;
 constexpr unsigned kWaitLimit = 1u << 22;
-constexpr int kMergeFloats = kWarps * 8 * kD;  // the consumer warps' [8][128] partials
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ unsigned smem_addr(const void* p) { return unsigned(__cvta_generic_to_shared(p)); }
@@ -132,11 +134,12 @@ inline size_t workspace_size(long long units, int splits, int G) {
 
 // ------------------------------------------------------------------ q preparation
 constexpr int kPrepThreads = 256;
+static_assert(kPrepThreads == enc::kEncodeThreads, "the fused step kernel runs both bodies");
 
-__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
-                                                             int h_q, int h_kv, int G, float qscale, Workspace ws) {
-  extern __shared__ __align__(16) float prep_smem[];
-  const int u = blockIdx.x, b = u / h_kv, h = u % h_kv;
+__device__ __forceinline__ void qprep_unit(const DevLayout& L, const void* __restrict__ q, int q_dtype, int h_q,
+                                           int h_kv, int G, float qscale, const Workspace& ws, int u,
+                                           float* prep_smem) {
+  const int b = u / h_kv, h = u % h_kv;
   const int tid = threadIdx.x;
   float* rot = prep_smem;                       // the K-group rotations, transposed, back to back
   float* qs = rot + L.k_rot32t_floats;          // [8][128] q in original coordinates
@@ -194,8 +197,40 @@ __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const 
     dst[lane] = make_uint2(pack_h2(hi[0], hi[1]), pack_h2(hi[2], hi[3]));
     dst[32 + lane] = make_uint2(pack_h2(lo[0], lo[1]), pack_h2(lo[2], lo[3]));
   }
+}
+
+__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
+                                                             int h_q, int h_kv, int G, float qscale, Workspace ws) {
+  extern __shared__ __align__(16) float prep_smem[];
+  qprep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, ws, blockIdx.x, prep_smem);
   __syncthreads();
   pdl_trigger();
+}
+
+// Fused first kernel of a decode step: blocks [0, n_enc) append the new tokens (four
+// blocks per token and KV head), the remaining blocks prepare q' for one unit each.
+// It lets the attention kernels launch at once (they wait for it before reading).
+__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
+                                                                 const void* __restrict__ v, int kv_dtype, int n_new,
+                                                                 int batch, long long n_tiles,
+                                                                 const int* __restrict__ seq_lens_before,
+                                                                 uint8_t* __restrict__ cache,
+                                                                 const void* __restrict__ q, int q_dtype, int h_q,
+                                                                 int h_kv, int G, float qscale, Workspace ws,
+                                                                 int n_enc) {
+  extern __shared__ __align__(16) float prep_smem[];
+  pdl_trigger();
+  const int e = blockIdx.x;
+  if (e < n_enc) {
+    const int part = e % kEncodeParts;
+    int rest = e / kEncodeParts;
+    const int t = rest % n_new;
+    rest /= n_new;
+    const int b = rest % batch, h = rest / batch;
+    enc::encode_token_part(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, n_tiles, t, part, b, h);
+  } else {
+    qprep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, ws, e - n_enc, prep_smem);
+  }
 }
 
 size_t prep_smem_bytes(const DevLayout& L) { return (size_t(L.k_rot32t_floats) + 2 * kMaxG * kD) * sizeof(float); }
@@ -292,6 +327,8 @@ struct SplitArgs {
   int h_q, h_kv, G;
   Workspace ws;
   float* out;
+  int len_add;           // tokens appended by the previous kernel: row b attends over seq_lens[b] + len_add
+  int wait_before_copy;  // the previous kernel writes the cache: wait for it before copying
 };
 
 constexpr int kConsumers = 4;                 // consumer warps, one 16-token slice of a tile each
@@ -452,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 3) split_kernel(DevLayout L, SplitAr
   float* mo = reinterpret_cast<float*>(ring);
   __shared__ int s_timeout;
 
-  long long len = a.seq_lens[b];
+  long long len = (long long)a.seq_lens[b] + a.len_add;
   if (len < 0) len = 0;
   const long long cap_tokens = min(a.n_tiles, (long long)a.max_tiles) * kTile;
   if (len > cap_tokens) {
@@ -472,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 3) split_kernel(DevLayout L, SplitAr
       mbar_init(&empty[i], 1);
     }
     fence_mbar_init();
+    if (a.wait_before_copy) pdl_wait();
     for (int it = 0; it < min(kStages, ntiles); ++it) {
       mbar_expect_tx(&full[it], TB);
       bulk_load(ring + it * TB, src + (size_t)it * TB, TB, &full[it]);
@@ -727,27 +765,22 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
   return p;
 }
 
-cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                          int h_q, int h_kv, const void* cache, const int* seq_lens, long long n_tiles,
-                          float softmax_scale, float* out, void* workspace, cudaStream_t stream) {
+namespace {
+
+cudaError_t set_prep_smem(const void* fn) {
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, fn);
+  if (e != cudaSuccess) return e;
+  if (attr.maxDynamicSharedSizeBytes >= int((kD * kD + 2 * kMaxG * kD) * sizeof(float))) return cudaSuccess;
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int((kD * kD + 2 * kMaxG * kD) * sizeof(float)));
+}
+
+cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int batch, int h_q, int h_kv,
+                             const void* cache, const int* seq_lens, long long n_tiles, float* out,
+                             const Workspace& ws, int len_add, int wait_before_copy, cudaStream_t stream) {
   const int G = h_q / h_kv;
   const long long units = (long long)batch * h_kv;
-  Workspace ws = carve(workspace, units, plan.n_splits, G);
-  {
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int((kD * kD + 2 * kMaxG * kD) * sizeof(float)));
-      if (e != cudaSuccess) return e;
-      configured[dev] = true;
-    }
-  }
-  qprep_kernel<<<unsigned(units), kPrepThreads, prep_smem_bytes(L), stream>>>(L, q, q_dtype, h_q, h_kv, G,
-                                                                              softmax_scale * kLog2e, ws);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   SplitArgs a;
   a.cache = static_cast<const uint8_t*>(cache);
   a.seq_lens = seq_lens;
@@ -760,7 +793,10 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
   a.G = G;
   a.ws = ws;
   a.out = out;
+  a.len_add = len_add;
+  a.wait_before_copy = wait_before_copy;
   dim3 grid(plan.n_splits, unsigned(units));
+  cudaError_t e;
   switch (L.v_rate) {
     case 1: e = launch_split<1>(L, a, grid, stream); break;
     case 2: e = launch_split<2>(L, a, grid, stream); break;
@@ -780,6 +816,42 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)ws.part_ml, (const float*)ws.part_o, plan.n_splits,
                             G, h_q, h_kv, L.v_rot32, out);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
+                          int h_q, int h_kv, const void* cache, const int* seq_lens, long long n_tiles,
+                          float softmax_scale, float* out, void* workspace, cudaStream_t stream) {
+  const int G = h_q / h_kv;
+  const long long units = (long long)batch * h_kv;
+  Workspace ws = carve(workspace, units, plan.n_splits, G);
+  cudaError_t e = set_prep_smem((const void*)qprep_kernel);
+  if (e != cudaSuccess) return e;
+  qprep_kernel<<<unsigned(units), kPrepThreads, prep_smem_bytes(L), stream>>>(L, q, q_dtype, h_q, h_kv, G,
+                                                                              softmax_scale * kLog2e, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the cache is not written by qprep: the split kernel may start copying tiles at once
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, n_tiles, out, ws, 0, 0, stream);
+}
+
+cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
+                               int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
+                               int batch, int h_q, int h_kv, void* cache, long long n_tiles, float softmax_scale, float* out, void* workspace,
+                               cudaStream_t stream) {
+  const int G = h_q / h_kv;
+  const long long units = (long long)batch * h_kv;
+  Workspace ws = carve(workspace, units, plan.n_splits, G);
+  cudaError_t e = set_prep_smem((const void*)step_prep_kernel);
+  if (e != cudaSuccess) return e;
+  const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
+  step_prep_kernel<<<unsigned(n_enc + units), kPrepThreads, prep_smem_bytes(L), stream>>>(
+      L, k_new, v_new, kv_dtype, n_new, batch, n_tiles, seq_lens_before, static_cast<uint8_t*>(cache), q, q_dtype,
+      h_q, h_kv, G, softmax_scale * kLog2e, ws, int(n_enc));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens_before, n_tiles, out, ws, n_new, 1, stream);
 }
 
 }  // namespace bgtq

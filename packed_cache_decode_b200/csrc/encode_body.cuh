@@ -1,0 +1,164 @@
+// Device code of tq_encode shared by the append kernel and the fused decode-step kernel.
+//
+// "TurboQuant: paper algorithm and vLLM engineering implementation" (pipeline diagram):
+// input vector x (per-head K or V) -> seeded random rotation -> per-coordinate scalar
+// quantisation against a few centroids. "Block-GTQ" abstract, sentence 5: equal-rate RoPE
+// blocks are grouped and each group is TQ-MSE coded.
+//
+// Every decision (norm, rotation, threshold comparison) is taken in fp64 so that the
+// codes agree with an fp64 reading of the method except for values within rounding
+// distance of a threshold.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "bgtq_internal.h"
+
+namespace bgtq {
+namespace enc {
+
+
+__device__ __forceinline__ double load_elem(const void* p, int dtype, size_t i) {
+  if (dtype == BGTQ_F32) return double(static_cast<const float*>(p)[i]);
+  if (dtype == BGTQ_BF16) return double(__bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]));
+  return double(__half2float(static_cast<const __half*>(p)[i]));
+}
+
+// Position of token j (0..15) inside a 16-token row of packed V codes.
+__device__ __forceinline__ int chunk_slot(int j) { return 4 * ((j & 7) >> 1) + 2 * (j >> 3) + (j & 1); }
+
+__device__ __forceinline__ int quantize(double y, const double* thr, int rate) {
+  int code = 0;
+  const int nthr = (1 << rate) - 1;
+  for (int m = 0; m < nthr; ++m) code += (y >= thr[m]) ? 1 : 0;
+  return code;
+}
+
+// Sets `width` (<= 64) bits at bit offset `bit` of a little-endian word array to `val`,
+// word by word with atomics (other tokens' fields share these words, possibly
+// concurrently).
+__device__ __forceinline__ void put_field_atomic(unsigned* words, int bit, unsigned long long val, int width) {
+  while (width > 0) {
+    const int w = bit >> 5, sh = bit & 31;
+    const int n = min(width, 32 - sh);
+    const unsigned mask = (n == 32 ? 0xffffffffu : ((1u << n) - 1u)) << sh;
+    atomicAnd(&words[w], ~mask);
+    atomicOr(&words[w], (unsigned(val) << sh) & mask);
+    val >>= n;
+    bit += n;
+    width -= n;
+  }
+}
+
+// Sets `width` bits at bit offset `bit` of a little-endian word array to `val`, leaving
+// the other bits alone (other tokens' codes share these words, possibly concurrently).
+__device__ __forceinline__ void put_bits_atomic(unsigned* words, int bit, unsigned val, int width) {
+  const unsigned mask = (1u << width) - 1u;
+  const int w = bit >> 5, sh = bit & 31;
+  atomicAnd(&words[w], ~(mask << sh));
+  atomicOr(&words[w], (val & mask) << sh);
+  if (sh + width > 32) {
+    const int s2 = 32 - sh;
+    atomicAnd(&words[w + 1], ~(mask >> s2));
+    atomicOr(&words[w + 1], (val & mask) >> s2);
+  }
+}
+
+// Four CTAs of 256 threads code one (token, KV head); CTA `part` owns packed key
+// dimensions and value dimensions [32 part, 32 part + 32). Each of its 64 outputs is
+// computed by four consecutive threads, each over a quarter of the rotation row (read
+// from the transposed fp64 copy: consecutive outputs, consecutive addresses), eight
+// loads in flight, summed with two shuffles. Every CTA recomputes the group norms (the
+// inputs are 256 values). Codes are written with atomics: the key fields of a chunk and
+// the value rows are shared with other tokens and other parts.
+constexpr int kEncodeThreads = 256;
+
+// Body of one encode CTA (256 threads): token t of batch row b, KV head h, output part
+// `part` (0..3).
+__device__ __forceinline__ void encode_token_part(const DevLayout& L, const void* __restrict__ k,
+                                                  const void* __restrict__ v, int dtype, int n_new, int h_kv,
+                                                  const int* __restrict__ seq_lens, uint8_t* __restrict__ cache,
+                                                  long long n_tiles, int t, int part, int b, int h) {
+  const int tid = threadIdx.x;
+  const long long pos = (long long)seq_lens[b] + t;
+  if (pos < 0 || pos >= n_tiles * kTile) {
+    if (tid == 0 && part == 0) atomicOr(L.status, BGTQ_STATUS_ENCODE_OVERFLOW);
+    return;
+  }
+  __shared__ double xp[kD], xv[kD];
+  __shared__ double gnorm[kMaxGroups + 1];
+
+  const size_t base = (((size_t)b * n_new + t) * h_kv + h) * kD;
+  if (tid < kD) xp[tid] = load_elem(k, dtype, base + L.packed_coord[tid]);  // keys in packed order
+  else xv[tid - kD] = load_elem(v, dtype, base + tid - kD);
+  __syncthreads();
+
+  if (tid < L.n_kgroups || tid == kD) {
+    const double* x = tid < kD ? xp + L.group_off[tid] : xv;
+    const int d = tid < kD ? L.group_dim[tid] : kD;
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    int i = 0;
+    for (; i + 4 <= d; i += 4) {
+      s0 = fma(x[i], x[i], s0);
+      s1 = fma(x[i + 1], x[i + 1], s1);
+      s2 = fma(x[i + 2], x[i + 2], s2);
+      s3 = fma(x[i + 3], x[i + 3], s3);
+    }
+    for (; i < d; ++i) s0 = fma(x[i], x[i], s0);
+    gnorm[tid < kD ? tid : kMaxGroups] = sqrt((s0 + s1) + (s2 + s3));
+  }
+  __syncthreads();
+
+  // thread = (output o of this part, quarter q of its dot product)
+  const int o = tid >> 2, q = tid & 3;
+  const bool is_key = o < 32;
+  const int p = 32 * part + (o & 31);
+  int g = 0;
+  if (is_key)
+    while (g + 1 < L.n_kgroups && p >= L.group_off[g + 1]) ++g;
+  const int d = is_key ? L.group_dim[g] : kD;
+  const int off = is_key ? L.group_off[g] : 0;
+  const int i = p - off;
+  const double* col = (is_key ? L.k_rot64[g] : L.v_rot64) + i;  // element (i, j) at j * d + i
+  const double* x = is_key ? xp + off : xv;
+  const int j0 = (q * d) / 4, j1 = ((q + 1) * d) / 4;
+  double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+  int j = j0;
+  for (; j + 8 <= j1; j += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = fma(__ldg(col + (size_t)(j + u) * d), x[j + u], a[u]);
+  }
+  for (; j < j1; ++j) a[0] = fma(__ldg(col + (size_t)j * d), x[j], a[0]);
+  double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  if (q != 0) return;
+
+  const double nrm = gnorm[is_key ? g : kMaxGroups];
+  const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
+  const int r = is_key ? L.group_rate[g] : L.v_rate;
+  const int code = quantize(y, L.threshold[r], r);
+
+  const long long tile = pos / kTile;
+  const int tt = int(pos % kTile);
+  uint8_t* tp = cache + (((size_t)b * h_kv + h) * n_tiles + tile) * (size_t)L.tile_bytes;
+  if (is_key) {
+    // chunk-major keys: token tt's field of chunk c sits at bit tt * dims_c * rate_c of
+    // the chunk's block; dimension i % 16 of the chunk at + (i % 16) * rate
+    const int ci = L.group_chunk0[g] + (i >> 4);
+    const int w = L.chunk_ndim[ci] * r;
+    put_bits_atomic(reinterpret_cast<unsigned*>(tp + L.chunk_koff[ci]), tt * w + (i & 15) * r, unsigned(code), r);
+    if (part == 0 && p < L.n_kgroups)
+      reinterpret_cast<float*>(tp + L.knorm_off)[p * kTile + tt] = float(gnorm[p]);
+  } else {
+    unsigned* vchunk = reinterpret_cast<unsigned*>(tp + L.vcode_off + (tt / kChunk) * 256 * L.v_rate);
+    put_bits_atomic(vchunk, (kChunk * p + chunk_slot(tt % kChunk)) * L.v_rate, unsigned(code), L.v_rate);
+    if (p == 0) reinterpret_cast<float*>(tp + L.vnorm_off)[tt] = float(gnorm[kMaxGroups]);
+  }
+}
+
+
+}  // namespace enc
+}  // namespace bgtq

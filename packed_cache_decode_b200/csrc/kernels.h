@@ -27,4 +27,11 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
                           int h_q, int h_kv, const void* cache, const int* seq_lens, long long n_tiles,
                           float softmax_scale, float* out, void* workspace, cudaStream_t stream);
 
+// Append n_new tokens at seq_lens_before[b] and attend over seq_lens_before[b] + n_new
+// tokens, as one chain of three kernels (append + q preparation, split, combine).
+cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
+                               int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
+                               int batch, int h_q, int h_kv, void* cache, long long n_tiles, float softmax_scale, float* out, void* workspace,
+                               cudaStream_t stream);
+
 }  // namespace bgtq
