@@ -196,8 +196,7 @@ class Model:
         x = _rope_dev(x, torch.tensor([pos], device=self.dev), self.wl.theta)
         return x[:, 0].contiguous().to(self.wl.dtype)
 
-    # kernel launches of one layer: step = step_prep + split + combine; decode_only =
-    # qprep + split + combine
+    # kernel launches of one layer in a step: encode + split + combine
     LAUNCHES_PER_LAYER = 3
 
     def step(self, stream):
@@ -498,7 +497,7 @@ def main():
             "gbs": model.bytes_per_step / (step_ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
-                         "kernel": "decode attention call per layer (qprep -> split -> combine, PDL-chained)",
+                         "kernel": "decode attention call per layer (split -> combine, PDL-chained)",
                          "peak_kind": peak_kind},
             "clocks": clocks,
             "gpu_launches": args.steps * wl.layers * Model.LAUNCHES_PER_LAYER,

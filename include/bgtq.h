@@ -25,16 +25,26 @@
  *
  * Packed cache format (one (batch row, KV head) = capacity/64 consecutive tiles):
  *  tile of 64 tokens = [K codes | V codes | K norms | V norms]
+ *   Both code areas are fragment-major: cut into per-lane bit strings (lane l = 4g + t of
+ *   a 32-lane warp) that hold exactly the codes one lane turns into its tensor-core
+ *   operands. Words are little-endian; bit n of a string is bit n%8 of its byte n/8.
  *   K codes:   64 x Kb bytes, Kb = 128*avg_k_bits/8. Packed key dimensions: K groups by
  *              descending rate; in a group, blocks ascending, coordinate j before j+64.
- *              Each group is cut into 16-dimension chunks (the last one may be shorter).
- *              Chunk c (dims_c dimensions of rate r_c) owns a block of 8*dims_c*r_c bytes,
- *              blocks in chunk order; a block is an LSB-first bitstream (bit n = bit n%8
- *              of byte n/8) in which token j's codes of the chunk start at bit
- *              j*dims_c*r_c, dimension i of the chunk at + i*r_c.
- *   V codes:   four 16-token chunks of 256*b_V bytes; each an LSB-first bitstream where
- *              the code of (dimension d, token j of the chunk) starts at bit
- *              (16*d + slot(j))*b_V, slot(j) = 4*((j%8)/2) + 2*(j/8) + j%2.
+ *              Each group is cut into quads of 4 dimension pairs (8 dimensions); the
+ *              group's last quad holds the remaining P = 1..3 pairs when its dimension
+ *              count is not a multiple of 8. Quad blocks follow one another, 16*P*r bytes
+ *              each. In a quad, lane i = g*P + e (g = 0..7, pair e = 0..P-1) holds for
+ *              the tokens g + 8m (m = 0..7) the codes lo (dim 2e) and hi (dim 2e+1) as a
+ *              16r-bit string: r = 1: bit m = lo, bit 8+m = hi; r = 2..4: field m of 2r
+ *              bits at bit 2rm = lo | hi << r. The string sits at bit 16r*i of the block,
+ *              except r = 3: bits 0..31 at bit 32i, bits 32..47 at bit 256P + 16i.
+ *   V codes:   four 16-token chunks of 256*b_V bytes (tokens 16c..16c+15). Lane l = 4g+t
+ *              holds 32 fields n = 4mt + k (mt = 0..7, k = 0..3): value dimension
+ *              16g + 2mt + (k&1), tokens lo = 2t + 8(k>>1) and hi = lo + 1 of the chunk,
+ *              as a 64*b_V-bit string: b_V = 1: word u = 0,1 has bit f = lo and bit
+ *              16+f = hi of field 16u+f; b_V = 2..4: field n of 2b_V bits at bit 2b_V*n
+ *              = lo | hi << b_V. The string sits at bit 64*b_V*l of the chunk, except
+ *              b_V = 3, 4: bits 0..127 at bit 128l, the rest at bit 4096 + (64b_V-128)l.
  *   K norms:   n_kgroups x 64 fp32, group-major: |x_g| of each token's group g.
  *   V norms:   64 fp32.
  *  tile_bytes = 64*(Kb + 16*b_V) + 256*(n_kgroups + 1).

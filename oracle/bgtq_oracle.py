@@ -240,11 +240,6 @@ def brute_force_rates(score, distortion, r_min: int, r_max: int, total_bits: int
 # ----------------------------------------------------------------------------------------
 # Layout: groups, rotations, packed format [BGTQ sentence 5], [TQ]
 # ----------------------------------------------------------------------------------------
-def chunk_slot(j: int) -> int:
-    """Bit slot of token j (0..15) inside a 16-token row of packed V codes."""
-    return 4 * ((j % 8) // 2) + 2 * (j // 8) + (j % 2)
-
-
 @dataclass
 class Layout:
     k_rates: np.ndarray                  # [64] rate per RoPE block
@@ -280,17 +275,20 @@ class Layout:
     def tile_bytes(self):
         return TILE_TOKENS * self.bytes_per_token
 
-    def k_chunks(self):
-        """16-dimension chunks of the key groups in order: (first packed dim, dims, rate,
-        byte offset of the chunk's block inside a tile). A block holds the 64 tokens'
-        fields of that chunk back to back (token j's field at bit j * dims * rate)."""
+    def k_quads(self):
+        """Quads of the key groups in order: (first packed dim, pairs, rate, byte offset of
+        the quad's block inside a tile). A group's packed dims are cut into quads of 4 pairs
+        (8 dims); its last quad holds the remaining 1-3 pairs when the group's dim count is
+        not a multiple of 8. A quad block holds the codes of its pairs for the tile's 64
+        tokens: 64 x 2 pairs x r bits = 16 x pairs x r bytes, so blocks start 16-byte
+        aligned and the K area has no padding."""
         out, p, off = [], 0, 0
         for r, coords in self.groups:
             d = len(coords)
-            for c0 in range(0, d, 16):
-                nd = min(16, d - c0)
-                out.append((p + c0, nd, r, off))
-                off += TILE_TOKENS * nd * r // 8
+            for c0 in range(0, d, 8):
+                npairs = min(8, d - c0) // 2
+                out.append((p + c0, npairs, r, off))
+                off += 16 * npairs * r
             p += d
         return out
 
@@ -404,51 +402,152 @@ def attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, scale: float)
 
 # ----------------------------------------------------------------------------------------
 # Packed tile format (the byte layout both sides implement)
+#
+# Tile of 64 tokens = [K area][V area][K norms fp32, group-major: [group][token]]
+# [V norms fp32 [token]]. Both code areas are "fragment-major": they are cut into per-lane
+# bit strings, lane l = 4 g + t of a 32-lane warp, holding exactly the codes that lane
+# turns into its tensor-core operand registers, so a lane reads its codes with one or two
+# aligned loads and no two lanes share a word. Words are little-endian; bit b of a bit
+# string is bit b % 8 of its byte b // 8.
+#
+# K quad with P pairs at rate r (Layout.k_quads): lane i = g P + e (g 0..7 = token row,
+# e 0..P-1 = pair) holds, for the eight tokens j = g + 8 m (m 0..7), the codes lo = dim
+# 2e and hi = dim 2e + 1 of the quad. Its 16 r-bit string: rate 1: bit m = lo(m), bit
+# 8 + m = hi(m); rates 2-4: field m (2 r bits) at bit 2 r m = lo(m) | hi(m) << r. Storage
+# inside the quad block: rate 1: halfword i; rate 2: word i; rate 4: 8 bytes at 8 i;
+# rate 3: bits 0..31 in word i, bits 32..47 in halfword i after the 8 P words.
+#
+# V: four 16-token chunks (tokens 16 c .. 16 c + 15), each a block of 256 b bytes. Lane
+# l = 4 g + t holds 32 fields n = 4 mt + k (mt 0..7, k 0..3): value dim 16 g + 2 mt +
+# (k & 1), tokens lo = 2 t + 8 (k >> 1) and hi = lo + 1 of the chunk. Its 64 b-bit
+# string: rate 1: word u (0, 1) has bit f = lo(16 u + f) and bit 16 + f = hi(16 u + f);
+# rates 2-4: field n at bit 2 b n = lo | hi << b. Storage: rate 1: 8 bytes at 8 l; rate
+# 2: 16 bytes at 16 l; rates 3-4: bits 0..127 at 16 l and the rest (64 or 128 bits) at
+# 512 + (8 or 16) l.
 # ----------------------------------------------------------------------------------------
-def _put_bits(bitbuf: np.ndarray, pos: np.ndarray, codes: np.ndarray, rate: int):
-    for i in range(rate):
-        bitbuf[..., pos + i] = (codes >> i) & 1
+def _k_lane_bits(r: int, lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
+    """lo, hi [..., 8] codes of slots m = 0..7 -> [..., 16 r] bits of one K lane."""
+    out = np.zeros(lo.shape[:-1] + (16 * r,), dtype=np.uint8)
+    for m in range(8):
+        if r == 1:
+            out[..., m] = lo[..., m] & 1
+            out[..., 8 + m] = hi[..., m] & 1
+        else:
+            for b in range(r):
+                out[..., 2 * r * m + b] = (lo[..., m] >> b) & 1
+                out[..., 2 * r * m + r + b] = (hi[..., m] >> b) & 1
+    return out
+
+
+def _k_lane_codes(r: int, bits: np.ndarray):
+    """Inverse of _k_lane_bits: [..., 16 r] bits -> (lo, hi) [..., 8]."""
+    bits = bits.astype(np.int64)
+    lo = np.zeros(bits.shape[:-1] + (8,), dtype=np.int64)
+    hi = np.zeros_like(lo)
+    for m in range(8):
+        if r == 1:
+            lo[..., m] = bits[..., m]
+            hi[..., m] = bits[..., 8 + m]
+        else:
+            for b in range(r):
+                lo[..., m] |= bits[..., 2 * r * m + b] << b
+                hi[..., m] |= bits[..., 2 * r * m + r + b] << b
+    return lo, hi
+
+
+def _k_lane_spans(r: int, npairs: int, i: int):
+    """(lane bit range, block bit range) pieces where K lane i of a quad is stored."""
+    if r == 3:
+        return [((0, 32), (32 * i, 32 * i + 32)), ((32, 48), (256 * npairs + 16 * i, 256 * npairs + 16 * i + 16))]
+    return [((0, 16 * r), (16 * r * i, 16 * r * (i + 1)))]
+
+
+def _v_fields():
+    """For lane l = 4 g + t and field n: (value dim, lo token, hi token) in a V chunk."""
+    out = np.zeros((32, 32, 3), dtype=np.int64)
+    for lane in range(32):
+        g, t = lane // 4, lane % 4
+        for n in range(32):
+            mt, k = n // 4, n % 4
+            lo = 2 * t + 8 * (k >> 1)
+            out[lane, n] = (16 * g + 2 * mt + (k & 1), lo, lo + 1)
+    return out
+
+
+def _v_lane_bits(b: int, lo: np.ndarray, hi: np.ndarray) -> np.ndarray:
+    """lo, hi [..., 32] codes of fields n = 0..31 -> [..., 64 b] bits of one V lane."""
+    out = np.zeros(lo.shape[:-1] + (64 * b,), dtype=np.uint8)
+    for n in range(32):
+        if b == 1:
+            u, f = divmod(n, 16)
+            out[..., 32 * u + f] = lo[..., n] & 1
+            out[..., 32 * u + 16 + f] = hi[..., n] & 1
+        else:
+            for i in range(b):
+                out[..., 2 * b * n + i] = (lo[..., n] >> i) & 1
+                out[..., 2 * b * n + b + i] = (hi[..., n] >> i) & 1
+    return out
+
+
+def _v_lane_codes(b: int, bits: np.ndarray):
+    bits = bits.astype(np.int64)
+    lo = np.zeros(bits.shape[:-1] + (32,), dtype=np.int64)
+    hi = np.zeros_like(lo)
+    for n in range(32):
+        if b == 1:
+            u, f = divmod(n, 16)
+            lo[..., n] = bits[..., 32 * u + f]
+            hi[..., n] = bits[..., 32 * u + 16 + f]
+        else:
+            for i in range(b):
+                lo[..., n] |= bits[..., 2 * b * n + i] << i
+                hi[..., n] |= bits[..., 2 * b * n + b + i] << i
+    return lo, hi
+
+
+def _v_lane_spans(b: int, lane: int):
+    """(lane bit range, chunk-block bit range) pieces where V lane l is stored."""
+    if b <= 2:
+        return [((0, 64 * b), (64 * b * lane, 64 * b * (lane + 1)))]
+    rest = 64 * b - 128
+    return [((0, 128), (128 * lane, 128 * lane + 128)), ((128, 64 * b), (4096 + rest * lane, 4096 + rest * (lane + 1)))]
 
 
 def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
-    """Bytes of one (batch row, KV head) cache holding tokens 0..n-1 of ``enc``.
-
-    Tile of 64 tokens = [K codes: one block per 16-dimension key chunk, in chunk order; a
-    block is an LSB-first bitstream where token j's codes of the chunk's dims sit at bit
-    j * dims * rate, dim i of the chunk at + i * rate] [V codes: four 16-token chunks, each
-    a bitstream where (dim d, token j) sits at bit (16 d + slot(j)) b_V] [K norms fp32,
-    group-major] [V norms fp32]. Unused slots are 0.
-    """
+    """Bytes of one (batch row, KV head) cache holding tokens 0..n-1 of ``enc`` in the
+    fragment-major tile format described above. Unused token slots are 0."""
     n = enc["k_codes"].shape[0]
     if capacity % TILE_TOKENS or n > capacity:
         raise ValueError("capacity must be a multiple of 64 and hold the tokens")
     ntile = capacity // TILE_TOKENS
     out = np.zeros((ntile, layout.tile_bytes), dtype=np.uint8)
-    kb, vb, ng = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups
-    # K area: chunk-major blocks (see Layout.k_chunks)
+    kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
+    # K area
     kcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
     kcodes[:n] = enc["k_codes"]
-    kcodes = kcodes.reshape(ntile, TILE_TOKENS, HEAD_DIM)
-    for p0, nd, r, off in layout.k_chunks():
-        w = nd * r
-        bits = np.zeros((ntile, TILE_TOKENS * w), dtype=np.uint8)
-        for i in range(nd):
-            for bit in range(r):
-                bits[:, np.arange(TILE_TOKENS) * w + i * r + bit] = (kcodes[:, :, p0 + i] >> bit) & 1
-        out[:, off:off + TILE_TOKENS * w // 8] = np.packbits(bits, axis=1, bitorder="little")
-    # V chunks
-    br = layout.v_rate
+    kcodes = kcodes.reshape(ntile, 8, 8, HEAD_DIM)          # [tile, m, g, dim]: token g + 8 m
+    for p0, npairs, r, off in layout.k_quads():
+        blk = np.zeros((ntile, 128 * npairs * r), dtype=np.uint8)
+        for g in range(8):
+            for e in range(npairs):
+                lane = _k_lane_bits(r, kcodes[:, :, g, p0 + 2 * e], kcodes[:, :, g, p0 + 2 * e + 1])
+                for (a0, a1), (b0, b1) in _k_lane_spans(r, npairs, g * npairs + e):
+                    blk[:, b0:b1] = lane[:, a0:a1]
+        out[:, off:off + 16 * npairs * r] = np.packbits(blk, axis=1, bitorder="little")
+    # V area
     vcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
     vcodes[:n] = enc["v_codes"]
-    vcodes = vcodes.reshape(ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS, HEAD_DIM)
-    vbits = np.zeros((ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS * HEAD_DIM * br), dtype=np.uint8)
-    for j in range(CHUNK_TOKENS):
-        pos = (CHUNK_TOKENS * np.arange(HEAD_DIM) + chunk_slot(j)) * br
-        for i in range(br):
-            vbits[:, :, pos + i] = (vcodes[:, :, j, :] >> i) & 1
-    vrec = np.packbits(vbits, axis=2, bitorder="little").reshape(ntile, TILE_TOKENS * vb)
+    vcodes = vcodes.reshape(ntile, 4, CHUNK_TOKENS, HEAD_DIM)
+    fld = _v_fields()
     base = TILE_TOKENS * kb
-    out[:, base:base + TILE_TOKENS * vb] = vrec
+    for c in range(4):
+        blk = np.zeros((ntile, 2048 * br), dtype=np.uint8)
+        for lane in range(32):
+            dims, lot, hit = fld[lane, :, 0], fld[lane, :, 1], fld[lane, :, 2]
+            bits = _v_lane_bits(br, vcodes[:, c, lot, dims], vcodes[:, c, hit, dims])
+            for (a0, a1), (b0, b1) in _v_lane_spans(br, lane):
+                blk[:, b0:b1] = bits[:, a0:a1]
+        out[:, base + 256 * br * c:base + 256 * br * (c + 1)] = np.packbits(blk, axis=1, bitorder="little")
     # norms
     base += TILE_TOKENS * vb
     kn = np.zeros((ntile * TILE_TOKENS, ng), dtype=np.float32)
@@ -467,22 +566,31 @@ def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
     ntile = len(buf) // layout.tile_bytes
     t = np.asarray(buf, dtype=np.uint8).reshape(ntile, layout.tile_bytes)
     kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
-    kc = np.zeros((ntile, TILE_TOKENS, HEAD_DIM), dtype=np.int64)
-    for p0, nd, r, off in layout.k_chunks():
-        w = nd * r
-        bits = np.unpackbits(t[:, off:off + TILE_TOKENS * w // 8], axis=1, bitorder="little").astype(np.int64)
-        for i in range(nd):
-            for bit in range(r):
-                kc[:, :, p0 + i] |= bits[:, np.arange(TILE_TOKENS) * w + i * r + bit] << bit
+    kc = np.zeros((ntile, 8, 8, HEAD_DIM), dtype=np.int64)
+    for p0, npairs, r, off in layout.k_quads():
+        blk = np.unpackbits(t[:, off:off + 16 * npairs * r], axis=1, bitorder="little")
+        for g in range(8):
+            for e in range(npairs):
+                lane = np.zeros((ntile, 16 * r), dtype=np.uint8)
+                for (a0, a1), (b0, b1) in _k_lane_spans(r, npairs, g * npairs + e):
+                    lane[:, a0:a1] = blk[:, b0:b1]
+                lo, hi = _k_lane_codes(r, lane)
+                kc[:, :, g, p0 + 2 * e] = lo
+                kc[:, :, g, p0 + 2 * e + 1] = hi
     kc = kc.reshape(-1, HEAD_DIM)
+    vc = np.zeros((ntile, 4, CHUNK_TOKENS, HEAD_DIM), dtype=np.int64)
+    fld = _v_fields()
     base = TILE_TOKENS * kb
-    vbits = np.unpackbits(t[:, base:base + TILE_TOKENS * vb].reshape(ntile, TILE_TOKENS // CHUNK_TOKENS, -1),
-                          axis=2, bitorder="little").astype(np.int64)
-    vc = np.zeros((ntile, TILE_TOKENS // CHUNK_TOKENS, CHUNK_TOKENS, HEAD_DIM), dtype=np.int64)
-    for j in range(CHUNK_TOKENS):
-        pos = (CHUNK_TOKENS * np.arange(HEAD_DIM) + chunk_slot(j)) * br
-        for i in range(br):
-            vc[:, :, j, :] |= vbits[:, :, pos + i] << i
+    for c in range(4):
+        blk = np.unpackbits(t[:, base + 256 * br * c:base + 256 * br * (c + 1)], axis=1, bitorder="little")
+        for lane in range(32):
+            bits = np.zeros((ntile, 64 * br), dtype=np.uint8)
+            for (a0, a1), (b0, b1) in _v_lane_spans(br, lane):
+                bits[:, a0:a1] = blk[:, b0:b1]
+            lo, hi = _v_lane_codes(br, bits)
+            dims, lot, hit = fld[lane, :, 0], fld[lane, :, 1], fld[lane, :, 2]
+            vc[:, c, lot, dims] = lo
+            vc[:, c, hit, dims] = hi
     base += TILE_TOKENS * vb
     kn = t[:, base:base + 4 * TILE_TOKENS * ng].copy().view(np.float32).reshape(ntile, ng, TILE_TOKENS)
     kn = kn.transpose(0, 2, 1).reshape(-1, ng)

@@ -36,7 +36,6 @@ unsigned short fp16_bits(double v) {
   return *reinterpret_cast<unsigned short*>(&h);
 }
 
-unsigned pack_half2(double lo, double hi) { return unsigned(fp16_bits(lo)) | (unsigned(fp16_bits(hi)) << 16); }
 
 // Scale kappa_r such that fp16(kappa_r * c) represents the rate-r codebook as exactly as
 // possible: +-1 for rate 1; otherwise the best of the 1024 scales that map the outer
@@ -102,8 +101,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t lut_words = 20 + 2 * (64 + 256) + 256 + 32;
-  const size_t bytes = 256 + n64 * sizeof(double) + 2 * n64 * sizeof(float) + lut_words * 4 + 256;
+  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256;
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
   if ((e = cudaMalloc(&dblock, bytes)) != cudaSuccess) {
@@ -126,80 +124,57 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     off += L->rot[g].size() * sizeof(double);
   }
   for (int g = 0; g <= ng; ++g) {
-    float* h32 = reinterpret_cast<float*>(host.data() + off);
-    for (size_t i = 0; i < L->rot[g].size(); ++i) h32[i] = float(L->rot[g][i]);
-    const float* p = reinterpret_cast<const float*>(dptr + off);
-    if (g < ng) D.k_rot32[g] = p; else D.v_rot32 = p;
-    off += L->rot[g].size() * sizeof(float);
-  }
-  for (int g = 0; g < ng; ++g) {
-    const int d = L->group_dim[g];
+    // fp32 copies, row-major; key rows padded to a multiple of 4 floats (16-byte rows)
+    const int d = int(std::lround(std::sqrt(double(L->rot[g].size()))));
+    const int ld = g < ng ? (d + 3) / 4 * 4 : d;
     float* h32 = reinterpret_cast<float*>(host.data() + off);
     for (int i = 0; i < d; ++i)
-      for (int j = 0; j < d; ++j) h32[size_t(j) * d + i] = float(L->rot[g][size_t(i) * d + j]);
-    D.k_rot32t[g] = reinterpret_cast<const float*>(dptr + off);
-    D.k_rot32t_off[g] = int((D.k_rot32t[g] - D.k_rot32t[0]));
-    D.k_rot32t_floats += int(L->rot[g].size());
-    off += L->rot[g].size() * sizeof(float);
+      for (int j = 0; j < ld; ++j) h32[size_t(i) * ld + j] = j < d ? float(L->rot[g][size_t(i) * d + j]) : 0.f;
+    const float* p = reinterpret_cast<const float*>(dptr + off);
+    if (g < ng) {
+      D.k_rot32[g] = p;
+      D.k_rot32_ld[g] = ld;
+    } else {
+      D.v_rot32 = p;
+    }
+    off += size_t(d) * ld * sizeof(float);
   }
   {
-    // pair tables for the tensor-core decode
-    unsigned* w = reinterpret_cast<unsigned*>(host.data() + off);
-    // keys: rates 1-2 scaled (exact), rates 3-4 carry an explicit low part (kappa 1);
-    // values: one fp16 table, scaled by the best kappa of the value rate
+    // codebooks of the tensor-core decode: keys of rates 1-2 scaled (exact in fp16), rates
+    // 3-4 as explicit hi + lo parts (kappa 1); values: one fp16 table scaled by the best
+    // kappa of the value rate
     double kap[5] = {1, 1, 1, 1, 1};
     for (int r = 1; r <= 2; ++r) kap[r] = codebook_kappa(L->centroid[r], r);
     const double kap_v = codebook_kappa(L->centroid[L->v_rate], L->v_rate);
-    for (int r = 1; r <= 2; ++r)
-      for (int idx = 0; idx < (1 << (2 * r)); ++idx) {
-        const int a = idx & ((1 << r) - 1), b = idx >> r;
-        w[(r == 1 ? 0 : 4) + idx] = pack_half2(kap[r] * L->centroid[r][a], kap[r] * L->centroid[r][b]);
-      }
-    for (int r = 3; r <= 4; ++r)
-      for (int idx = 0; idx < (1 << (2 * r)); ++idx) {
-        const int a = idx & ((1 << r) - 1), b = idx >> r;
-        const double ca = L->centroid[r][a], cb = L->centroid[r][b];
-        const double ha = double(__half2float(__float2half_rn(float(ca))));
-        const double hb = double(__half2float(__float2half_rn(float(cb))));
-        unsigned* e = w + 20 + 2 * ((r == 3 ? 0 : 64) + idx);
-        e[0] = pack_half2(ha, hb);
-        e[1] = pack_half2(ca - ha, cb - hb);
-      }
-    for (int idx = 0; idx < (1 << (2 * L->v_rate)); ++idx) {
-      const int a = idx & ((1 << L->v_rate) - 1), b = idx >> L->v_rate;
-      w[20 + 2 * 320 + idx] = pack_half2(kap_v * L->centroid[L->v_rate][a], kap_v * L->centroid[L->v_rate][b]);
+    for (int i = 0; i < 4; ++i) D.kc2[i] = fp16_bits(kap[2] * L->centroid[2][i]);
+    for (int i = 0; i < 8; ++i) {
+      D.kc3[0][i] = fp16_bits(round_fp16(L->centroid[3][i]));
+      D.kc3[1][i] = fp16_bits(L->centroid[3][i] - round_fp16(L->centroid[3][i]));
     }
-    for (int idx = 0; idx < 16; ++idx) {
-      const double* c1 = L->centroid[1];
-      unsigned* e = w + 20 + 2 * 320 + 256 + 2 * idx;
-      e[0] = pack_half2(kap[1] * c1[idx & 1], kap[1] * c1[(idx >> 1) & 1]);
-      e[1] = pack_half2(kap[1] * c1[(idx >> 2) & 1], kap[1] * c1[(idx >> 3) & 1]);
+    for (int i = 0; i < 16; ++i) {
+      D.kc4[0][i] = fp16_bits(round_fp16(L->centroid[4][i]));
+      D.kc4[1][i] = fp16_bits(L->centroid[4][i] - round_fp16(L->centroid[4][i]));
     }
-    D.klut1q = reinterpret_cast<const unsigned*>(dptr + off + (20 + 2 * 320 + 256) * 4);
-    D.klut12 = reinterpret_cast<const unsigned*>(dptr + off);
-    D.klut34 = reinterpret_cast<const unsigned*>(dptr + off + 20 * 4);
-    D.vlut = reinterpret_cast<const unsigned*>(dptr + off + (20 + 2 * 320) * 4);
+    for (int i = 0; i < (1 << L->v_rate); ++i) D.vc[i] = fp16_bits(kap_v * L->centroid[L->v_rate][i]);
     for (int r = 0; r < 5; ++r) D.kappa[r] = float(kap[r]);
     D.kappa_v = float(kap_v);
     for (int g = 0; g < ng; ++g) D.inv_kappa_group[g] = float(1.0 / kap[L->group_rate[g]]);
-    off += lut_words * 4;
   }
   {
-    int ci = 0, koff = 0;
+    int qi = 0, koff = 0;
     for (int g = 0; g < ng; ++g) {
       const int r = L->group_rate[g], d = L->group_dim[g];
-      D.group_chunk0[g] = ci;
-      D.group_nchunks[g] = (d + 15) / 16;
-      for (int cc = 0; cc < D.group_nchunks[g]; ++cc, ++ci) {
-        D.chunk_koff[ci] = koff;
-        koff += kTile * std::min(16, d - 16 * cc) * r / 8;
-        D.chunk_dim0[ci] = L->group_off[g] + 16 * cc;
-        D.chunk_ndim[ci] = std::min(16, d - 16 * cc);
-        D.chunk_group[ci] = g;
-        D.chunk_rate[ci] = r;
+      D.group_quad0[g] = qi;
+      D.group_nquads[g] = (d + 7) / 8;
+      for (int c0 = 0; c0 < d; c0 += 8, ++qi) {
+        const int np = std::min(8, d - c0) / 2;
+        D.quad_off[qi] = koff;
+        D.quad_np[qi] = np;
+        D.quad_dim0[qi] = L->group_off[g] + c0;
+        koff += 16 * np * r;
       }
     }
-    D.n_kchunks = ci;
+    D.n_kquads = qi;
   }
   D.n_kgroups = ng;
   D.v_rate = L->v_rate;
@@ -216,10 +191,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   }
   for (int p = 0; p < kD; ++p) D.packed_coord[p] = short(L->packed_coord[p]);
   for (int r = 0; r < 5; ++r)
-    for (int i = 0; i < 16; ++i) {
-      D.centroid[r][i] = float(L->centroid[r][i]);
-      D.threshold[r][i] = L->threshold[r][i];
-    }
+    for (int i = 0; i < 16; ++i) D.threshold[r][i] = L->threshold[r][i];
   e = cudaMemcpy(dblock, host.data(), bytes, cudaMemcpyHostToDevice);
   if (cur != device) cudaSetDevice(cur);
   if (e != cudaSuccess) {

@@ -15,7 +15,7 @@ constexpr int kTile = BGTQ_TILE_TOKENS;  // 64 tokens per tile
 constexpr int kChunk = 16;               // tokens per V-code chunk
 constexpr int kMaxG = BGTQ_MAX_GQA;
 constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
-constexpr int kMaxChunks = 12;           // sum over groups of ceil(d_g / 16) <= 128/16 + 4
+constexpr int kMaxQuads = 20;            // sum over groups of ceil(d_g / 8) <= 128/8 + 3
 constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32 outputs each
 
 // Everything a kernel needs about one layer's packing, passed by value.
@@ -32,33 +32,31 @@ struct DevLayout {
   int group_off[kMaxGroups];     // first packed dimension of the group
   int group_bitoff[kMaxGroups];  // first bit of the group inside a K record
   short packed_coord[kD];        // packed key dimension -> original coordinate
-  float centroid[5][16];         // [rate][code], fp32
   double threshold[5][16];       // [rate][k], fp64 (2^rate - 1 used)
   const double* k_rot64[kMaxGroups];  // d_g x d_g, TRANSPOSED: element (i, j) of R at j * d + i
   const double* v_rot64;              // 128 x 128, transposed likewise
-  const float* k_rot32[kMaxGroups];
-  const float* k_rot32t[kMaxGroups];  // transposed copies (column-major), back to back
-  int k_rot32t_off[kMaxGroups];       // float offset of group g's copy from k_rot32t[0]
-  int k_rot32t_floats;                // sum of d_g^2
+  const float* k_rot32[kMaxGroups];  // row-major, rows padded to k_rot32_ld[g] floats (a multiple of 4)
+  int k_rot32_ld[kMaxGroups];
   const float* v_rot32;
   unsigned* status;
-  // Tensor-core decode: 16-dimension chunks of the K record, per group.
-  int n_kchunks;
-  int group_chunk0[kMaxGroups];
-  int group_nchunks[kMaxGroups];
-  int chunk_koff[kMaxChunks];    // byte offset of the chunk's block inside a tile (chunk-major keys)
-  int chunk_dim0[kMaxChunks];    // first packed dimension of the chunk
-  int chunk_ndim[kMaxChunks];    // valid dimensions in the chunk (<= 16)
-  int chunk_group[kMaxChunks];
-  int chunk_rate[kMaxChunks];
+  // Fragment-major K area: each group's packed dims cut into quads of 4 pairs (8 dims),
+  // the last quad of a group holding the remaining 1-3 pairs.
+  int n_kquads;
+  int group_quad0[kMaxGroups];
+  int group_nquads[kMaxGroups];
+  int quad_off[kMaxQuads];       // byte offset of the quad's block inside a tile
+  int quad_np[kMaxQuads];        // pairs in the quad (1..4)
+  int quad_dim0[kMaxQuads];      // first packed dimension of the quad
   float inv_kappa_group[kMaxGroups];  // 1 / kappa of each group's rate
   float kappa[5];                // per-rate scale making the rate-1/2 fp16 key codebooks exact
   float kappa_v;                 // scale of the fp16 value codebook
-  // Pair tables: entry (a | b << r) holds the fp16 pair (value(a), value(b)).
-  const unsigned* klut12;        // rate 1: 4 entries at 0; rate 2: 16 entries at 4 (kappa-scaled)
-  const unsigned* klut34;        // rate 3: 64 entries at 0; rate 4: 256 at 64; entry = {hi pair, lo pair}
-  const unsigned* klut1q;        // rate 1, 16 entries: four codes -> {pair (0,1), pair (2,3)} (kappa-scaled)
-  const unsigned* vlut;          // value codebook pairs, 2^(2 v_rate) entries (fp16, times kappa_v)
+  // fp16 bit patterns of the codebooks the decode kernels build their pair tables from:
+  // keys of rates 1-2 scaled by kappa (exact), rates 3-4 as hi + lo parts (kappa 1);
+  // values scaled by kappa_v.
+  unsigned short kc2[4];
+  unsigned short kc3[2][8];      // [hi, lo][code]
+  unsigned short kc4[2][16];
+  unsigned short vc[16];
 };
 
 }  // namespace bgtq

@@ -14,6 +14,9 @@ __global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayou
                                                                         int n_new, int h_kv,
                                                                         const int* __restrict__ seq_lens,
                                                                         uint8_t* __restrict__ cache, long long n_tiles) {
+  // a split kernel launched as this kernel's programmatic dependent may start streaming
+  // the tiles that do not receive the new tokens (it waits before the one that does)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   enc::encode_token_part(L, k, v, dtype, n_new, h_kv, seq_lens, cache, n_tiles, blockIdx.x / kEncodeParts,
                          blockIdx.x % kEncodeParts, blockIdx.y, blockIdx.z);
 }

@@ -26,30 +26,11 @@ __device__ __forceinline__ double load_elem(const void* p, int dtype, size_t i) 
   return double(__half2float(static_cast<const __half*>(p)[i]));
 }
 
-// Position of token j (0..15) inside a 16-token row of packed V codes.
-__device__ __forceinline__ int chunk_slot(int j) { return 4 * ((j & 7) >> 1) + 2 * (j >> 3) + (j & 1); }
-
 __device__ __forceinline__ int quantize(double y, const double* thr, int rate) {
   int code = 0;
   const int nthr = (1 << rate) - 1;
   for (int m = 0; m < nthr; ++m) code += (y >= thr[m]) ? 1 : 0;
   return code;
-}
-
-// Sets `width` (<= 64) bits at bit offset `bit` of a little-endian word array to `val`,
-// word by word with atomics (other tokens' fields share these words, possibly
-// concurrently).
-__device__ __forceinline__ void put_field_atomic(unsigned* words, int bit, unsigned long long val, int width) {
-  while (width > 0) {
-    const int w = bit >> 5, sh = bit & 31;
-    const int n = min(width, 32 - sh);
-    const unsigned mask = (n == 32 ? 0xffffffffu : ((1u << n) - 1u)) << sh;
-    atomicAnd(&words[w], ~mask);
-    atomicOr(&words[w], (unsigned(val) << sh) & mask);
-    val >>= n;
-    bit += n;
-    width -= n;
-  }
 }
 
 // Sets `width` bits at bit offset `bit` of a little-endian word array to `val`, leaving
@@ -63,6 +44,63 @@ __device__ __forceinline__ void put_bits_atomic(unsigned* words, int bit, unsign
     const int s2 = 32 - sh;
     atomicAnd(&words[w + 1], ~(mask >> s2));
     atomicOr(&words[w + 1], (val & mask) >> s2);
+  }
+}
+
+// Writes a code field that starts at bit `lb` of a lane's bit string, where the string's
+// bits below `split` are stored from block bit a0 and the others from block bit b0 (the
+// second plane of rate-3 keys and rate 3-4 values); a field may straddle the split.
+__device__ __forceinline__ void put_lane_field(unsigned* blk, int lb, unsigned val, int width, int split, int a0,
+                                               int b0) {
+  if (lb + width <= split) {
+    put_bits_atomic(blk, a0 + lb, val, width);
+  } else if (lb >= split) {
+    put_bits_atomic(blk, b0 + lb - split, val, width);
+  } else {
+    const int n = split - lb;
+    put_bits_atomic(blk, a0 + lb, val, n);
+    put_bits_atomic(blk, b0, val >> n, width - n);
+  }
+}
+
+// Fragment-major placement of the code of token tt (0..63 in its tile).
+// Key packed dim at offset i of group g (rate r): quad Q = group_quad0[g] + i / 8 with P
+// pairs; pair e = (i % 8) / 2, hi = i & 1; lane = (tt % 8) P + e, slot m = tt / 8. The
+// lane's string: rate 1: bit m (lo) or 8 + m (hi); rates 2-4: field 2 r m + r hi. Stored
+// at 16 r lane bits into the quad block (rate 3: bits 0..31 at 32 lane, bits 32..47 at
+// 256 P + 16 lane).
+__device__ __forceinline__ void put_key_code(const DevLayout& L, uint8_t* tile, int g, int i, int tt, unsigned code) {
+  const int r = L.group_rate[g];
+  const int Q = L.group_quad0[g] + (i >> 3), P = L.quad_np[Q];
+  const int e = (i & 7) >> 1, hi = i & 1;
+  const int lane = (tt & 7) * P + e, m = tt >> 3;
+  unsigned* blk = reinterpret_cast<unsigned*>(tile + L.quad_off[Q]);
+  if (r == 1) {
+    put_bits_atomic(blk, 16 * lane + 8 * hi + m, code, 1);
+  } else if (r == 3) {
+    put_lane_field(blk, 6 * m + 3 * hi, code, 3, 32, 32 * lane, 256 * P + 16 * lane);
+  } else {
+    put_bits_atomic(blk, 16 * r * lane + 2 * r * m + r * hi, code, r);
+  }
+}
+
+// Value dim d of token tt: chunk c = tt / 16, jj = tt % 16; lane = 4 (d / 16) + (jj % 8) / 2,
+// field n = 4 ((d % 16) / 2) + 2 (jj / 8) + (d % 2), hi = jj % 2. The lane's string: rate
+// 1: word n / 16, bit n % 16 (+ 16 for hi); rates 2-4: field 2 b n + b hi. Stored at 64 b
+// lane bits into the chunk block (rates 3-4: bits 0..127 at 128 lane, the rest at
+// 4096 + (64 b - 128) lane).
+__device__ __forceinline__ void put_value_code(const DevLayout& L, uint8_t* tile, int d, int tt, unsigned code) {
+  const int br = L.v_rate;
+  const int jj = tt & 15;
+  const int lane = 4 * (d >> 4) + ((jj & 7) >> 1);
+  const int n = 4 * ((d & 15) >> 1) + 2 * (jj >> 3) + (d & 1), hi = jj & 1;
+  unsigned* blk = reinterpret_cast<unsigned*>(tile + L.vcode_off + (tt >> 4) * 256 * br);
+  if (br == 1) {
+    put_bits_atomic(blk, 64 * lane + 32 * (n >> 4) + 16 * hi + (n & 15), code, 1);
+  } else if (br == 2) {
+    put_bits_atomic(blk, 128 * lane + 4 * n + 2 * hi, code, 2);
+  } else {
+    put_lane_field(blk, 2 * br * n + br * hi, code, br, 128, 128 * lane, 4096 + (64 * br - 128) * lane);
   }
 }
 
@@ -145,16 +183,11 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   const int tt = int(pos % kTile);
   uint8_t* tp = cache + (((size_t)b * h_kv + h) * n_tiles + tile) * (size_t)L.tile_bytes;
   if (is_key) {
-    // chunk-major keys: token tt's field of chunk c sits at bit tt * dims_c * rate_c of
-    // the chunk's block; dimension i % 16 of the chunk at + (i % 16) * rate
-    const int ci = L.group_chunk0[g] + (i >> 4);
-    const int w = L.chunk_ndim[ci] * r;
-    put_bits_atomic(reinterpret_cast<unsigned*>(tp + L.chunk_koff[ci]), tt * w + (i & 15) * r, unsigned(code), r);
+    put_key_code(L, tp, g, i, tt, unsigned(code));
     if (part == 0 && p < L.n_kgroups)
       reinterpret_cast<float*>(tp + L.knorm_off)[p * kTile + tt] = float(gnorm[p]);
   } else {
-    unsigned* vchunk = reinterpret_cast<unsigned*>(tp + L.vcode_off + (tt / kChunk) * 256 * L.v_rate);
-    put_bits_atomic(vchunk, (kChunk * p + chunk_slot(tt % kChunk)) * L.v_rate, unsigned(code), L.v_rate);
+    put_value_code(L, tp, p, tt, unsigned(code));
     if (p == 0) reinterpret_cast<float*>(tp + L.vnorm_off)[tt] = float(gnorm[kMaxGroups]);
   }
 }

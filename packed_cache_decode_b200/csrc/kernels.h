@@ -8,16 +8,20 @@
 
 namespace bgtq {
 
-// Split-K plan of one decode call: the cache of each (batch row, KV head) is cut into
-// n_splits ranges of tiles_per_split 64-token tiles.
+// Plan of one decode call: the units' caches (batch rows x KV heads, max_tiles 64-token
+// tiles each) are one sequence of T tiles; CTA c takes tiles [c T / n_ctas, (c+1) T /
+// n_ctas) (at most tiles_per_cta, never more than one unit long); a unit meets at most
+// n_parts slices, each leaving one partial result.
 struct DecodePlan {
   int max_tiles;        // ceil(max_seq_len / 64)
-  int tiles_per_split;
-  int n_splits;
+  int tiles_per_cta;
+  int n_ctas;
+  int n_parts;
   size_t workspace_bytes;
 };
 
-DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms);
+// ctas_per_sm <= 0: the most split CTAs that fit an SM (the workspace of any launch plan).
+DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms, int ctas_per_sm = 0);
 
 cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, int dtype, int batch,
                              int n_new, int h_kv, const int* seq_lens, void* cache, long long n_tiles,
@@ -28,7 +32,8 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
                           float softmax_scale, float* out, void* workspace, cudaStream_t stream);
 
 // Append n_new tokens at seq_lens_before[b] and attend over seq_lens_before[b] + n_new
-// tokens, as one chain of three kernels (append + q preparation, split, combine).
+// tokens: the encode kernel, then the split kernel as its programmatic dependent (only the
+// tile receiving the new tokens waits for the encode), then the combine.
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
                                int batch, int h_q, int h_kv, void* cache, long long n_tiles, float softmax_scale, float* out, void* workspace,

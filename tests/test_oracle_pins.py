@@ -207,54 +207,79 @@ def test_grouping_and_byte_formula():
 
 
 def test_pack_places_bits_where_the_format_says():
+    """Worked by hand from the fragment-major format: K quad lane i = 4 g + e holds the pair
+    e codes of tokens g + 8 m; V lane 4 g + t holds field n = 4 mt + k = (dim 16 g + 2 mt +
+    (k & 1), tokens 2 t + 8 (k >> 1) and +1)."""
     lay = O.make_layout(np.array([2] * 32 + [1] * 32), 3, 5)   # packed dims 0..63 rate 2, 64..127 rate 1
-    assert [c[1:] for c in lay.k_chunks()] == [(16, 2, 0), (16, 2, 256), (16, 2, 512), (16, 2, 768),
-                                               (16, 1, 1024), (16, 1, 1152), (16, 1, 1280), (16, 1, 1408)]
-    enc = {"k_codes": np.zeros((3, 128), dtype=np.int64), "v_codes": np.zeros((3, 128), dtype=np.int64),
-           "k_norms": np.zeros((3, 2)), "v_norm": np.zeros(3)}
-    enc["k_codes"][2, 5] = 3          # token 2, packed dim 5: chunk 0 (32 bits per token), bits 64+10, 64+11
-    enc["k_codes"][1, 64] = 1         # token 1, packed dim 64: chunk 4 at byte 1024, 16 bits per token: bit 16
-    enc["k_codes"][0, 127] = 1        # token 0, packed dim 127: chunk 7 at byte 1408, dim 15: bit 15
-    enc["v_codes"][1, 7] = 5          # token 1, dim 7, rate 3: chunk 0, bit (16*7 + slot(1))*3
-    enc["v_codes"][2, 0] = 6          # token 2 -> slot 4: bits 12..14 of chunk 0
+    assert [q[1:] for q in lay.k_quads()] == ([(4, 2, 128 * i) for i in range(8)]
+                                              + [(4, 1, 1024 + 64 * i) for i in range(8)])
+    n = 58
+    enc = {"k_codes": np.zeros((n, 128), dtype=np.int64), "v_codes": np.zeros((n, 128), dtype=np.int64),
+           "k_norms": np.zeros((n, 2)), "v_norm": np.zeros(n)}
+    enc["k_codes"][2, 5] = 3     # quad 0, pair 2 hi; token 2 = (g 2, m 0): lane 10 -> word 10, bits 2-3
+    enc["k_codes"][57, 6] = 2    # quad 0, pair 3 lo; token 57 = (g 1, m 7): lane 7 -> word 7, bits 28-29
+    enc["k_codes"][1, 64] = 1    # rate-1 quad at 1024, pair 0 lo; token 1 = (g 1, m 0): lane 4 -> halfword 4, bit 0
+    enc["k_codes"][0, 127] = 1   # rate-1 quad at 1472, pair 3 hi; token 0: lane 3 -> halfword 3, bit 8
+    enc["v_codes"][1, 7] = 5     # chunk 0, dim 7 = (g 0, mt 3, k odd), token 1 = hi of (0, 1): lane 0, field 13
+    enc["v_codes"][2, 0] = 6     # dim 0, token 2 = lo of (2, 3): t 1, k 0 -> lane 1, field 0
+    enc["v_codes"][9, 127] = 7   # dim 127 = (g 7, mt 7, k odd), token 9 = hi of (8, 9): t 0, k 3 -> lane 28, field 31
+    enc["v_codes"][17, 0] = 4    # chunk 1 (tokens 16..31), token 1 of the chunk, dim 0: lane 0, field 0 hi
     enc["k_norms"][1] = [1.5, -2.0]
     enc["v_norm"][2] = 0.25
     buf = O.pack(lay, enc, 64)
-    kb = lay.k_record_bytes
-    assert kb == 24 and lay.tile_bytes == 64 * (24 + 48 + 12) and buf.size == lay.tile_bytes
-    assert buf[9] == 0b00001100
-    assert buf[1024 + 2] == 1
-    assert buf[1408 + 1] == 0b10000000
-    vbase = 64 * kb
-    bit = (16 * 7 + 1) * 3
-    assert (int.from_bytes(buf[vbase:vbase + 8 * 48].tobytes(), "little") >> bit) & 7 == 5
-    assert (int.from_bytes(buf[vbase:vbase + 8 * 48].tobytes(), "little") >> 12) & 7 == 6
+    assert lay.k_record_bytes == 24 and lay.tile_bytes == 64 * (24 + 48 + 12) and buf.size == lay.tile_bytes
+    assert buf[40] == 0b00001100
+    assert buf[31] == 0b00100000
+    assert buf[1024 + 8] == 1
+    assert buf[1472 + 7] == 1
+    vbase = 64 * 24
+    lane0 = int.from_bytes(buf[vbase:vbase + 16].tobytes(), "little")
+    assert (lane0 >> (6 * 13 + 3)) & 7 == 5
+    assert buf[vbase + 16] & 7 == 6
+    assert buf[vbase + 512 + 8 * 28 + 7] == 0b11100000        # bits 189-191 of lane 28: its second plane
+    assert (buf[vbase + 768] >> 3) & 7 == 4
     nbase = vbase + 64 * 48
     kn = buf[nbase:nbase + 4 * 128].view(np.float32)
     assert kn[1] == 1.5 and kn[64 + 1] == -2.0
     assert buf[nbase + 512:nbase + 768].view(np.float32)[2] == 0.25
     # nothing else written: one byte per code, and 1.5 / -2.0 / 0.25 have 2 / 1 / 2 nonzero bytes
-    assert int(np.count_nonzero(buf)) == 5 + 2 + 1 + 2
-    u = O.unpack(lay, buf, 3)
+    assert int(np.count_nonzero(buf)) == 8 + 2 + 1 + 2
+    u = O.unpack(lay, buf, n)
     np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
     np.testing.assert_array_equal(u["v_codes"], enc["v_codes"])
 
 
-def test_partial_chunks_are_packed_densely():
+def test_partial_quads_are_packed_densely():
     rates = np.array([4] * 3 + [3] * 5 + [2] * 9 + [1] * 47)     # group dims 6, 10, 18, 94
     assert rates.sum() % 4 == 0
     lay = O.make_layout(rates, 2, 1)
-    ch = lay.k_chunks()
-    assert [(nd, r) for _, nd, r, _ in ch] == [(6, 4), (10, 3), (16, 2), (2, 2), (16, 1), (16, 1), (16, 1),
-                                               (16, 1), (16, 1), (14, 1)]
-    end = ch[-1][3] + 64 * ch[-1][1] * ch[-1][2] // 8
+    qs = lay.k_quads()
+    assert [(npairs, r) for _, npairs, r, _ in qs] == ([(3, 4), (4, 3), (1, 3), (4, 2), (4, 2), (1, 2)]
+                                                       + [(4, 1)] * 11 + [(3, 1)])
+    end = qs[-1][3] + 16 * qs[-1][1] * qs[-1][2]
     assert end == 64 * lay.k_record_bytes                      # no padding
-    assert all(off % 16 == 0 for *_, off in ch)                # every block starts 16-byte aligned
+    assert all(off % 16 == 0 for *_, off in qs)                # every block starts 16-byte aligned
+    assert [p0 for p0, *_ in qs][:4] == [0, 6, 14, 16]
 
 
-def test_chunk_slot_is_a_permutation():
-    assert sorted(O.chunk_slot(j) for j in range(16)) == list(range(16))
-    assert [O.chunk_slot(j) for j in (0, 1, 8, 9, 2, 3)] == [0, 1, 2, 3, 4, 5]
+def test_every_code_has_exactly_one_place():
+    """Pack codes that name their own (token, dim): a one-to-one format unpacks them back,
+    and every code bit of the tile is used (the area sizes are exact)."""
+    for rates, vr in ((np.array([4] * 3 + [3] * 5 + [2] * 9 + [1] * 47), 3), (np.full(64, 1), 1),
+                      (np.full(64, 4), 4), (np.array([2] * 40 + [1] * 24), 2)):
+        lay = O.make_layout(rates, vr, 0)
+        rng = np.random.default_rng(int(rates.sum()) + vr)
+        prates = lay.packed_rates()
+        kc = rng.integers(0, 1 << prates, size=(64, 128))
+        vc = rng.integers(0, 1 << vr, size=(64, 128))
+        enc = {"k_codes": kc, "v_codes": vc, "k_norms": np.zeros((64, lay.n_kgroups)), "v_norm": np.zeros(64)}
+        u = O.unpack(lay, O.pack(lay, enc, 64), 64)
+        np.testing.assert_array_equal(u["k_codes"], kc)
+        np.testing.assert_array_equal(u["v_codes"], vc)
+        full = {"k_codes": (1 << prates)[None, :].repeat(64, 0) - 1, "v_codes": np.full((64, 128), (1 << vr) - 1),
+                "k_norms": np.zeros((64, lay.n_kgroups)), "v_norm": np.zeros(64)}
+        codes = O.pack(lay, full, 64)[:64 * (lay.k_record_bytes + lay.v_record_bytes)]
+        assert np.all(codes == 255)
 
 
 def test_pack_unpack_round_trip():
