@@ -38,6 +38,23 @@ METRIC = "packed-KV decode attention: cached keys/s (HBM GB/s as % of B200 peak 
 UNIT = "keys/s"
 
 
+def _profiled_traffic():
+    """DRAM bytes per launch of the split kernel from the committed ncu summary, or None
+    when the kernel source has changed since that capture."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "split_kernel_llama8b_32k_k2v2.txt")
+    src = os.path.join(ROOT, "packed_cache_decode_b200", "csrc", "decode_mma.cu")
+    try:
+        fields = dict(ln.split(":", 1) for ln in open(prof) if ln.startswith(("source_sha256_16:", "dram_bytes")))
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if fields["source_sha256_16"].split()[0] != sha:
+            return None
+        return int(fields["dram_bytes_per_launch"].split()[0])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -496,7 +513,8 @@ def main():
                        "parallelism": f"replicas x{world} (independent sequences per GPU)"},
             "gbs": model.bytes_per_step / (step_ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak,
+                         "traffic": _profiled_traffic() if wl.name == synth.WORKLOADS["llama8b"].name else None,
                          "kernel": "decode attention call per layer (split -> combine, PDL-chained)",
                          "peak_kind": peak_kind},
             "clocks": clocks,

@@ -39,14 +39,15 @@ unsigned short fp16_bits(double v) {
 
 // Scale kappa_r such that fp16(kappa_r * c) represents the rate-r codebook as exactly as
 // possible: +-1 for rate 1; otherwise the best of the 1024 scales that map the outer
-// magnitude to an integer in [1024, 2048) (max relative error 2.3e-7 at rate 2, 1.8e-5
-// at rate 3, 9.3e-5 at rate 4).
+// magnitude to [1, 2) (fp16 values with 10 fraction bits: max relative error 2.3e-7 at
+// rate 2, 1.8e-5 at rate 3, 9.3e-5 at rate 4). Scaled values stay near 1, so 1/kappa can
+// be folded into fp16 operands without leaving the normal range.
 double codebook_kappa(const double* c, int r) {
   const int m = 1 << (r - 1);
   if (r == 1) return 1.0 / c[m];
   double best = 1.0, best_err = INFINITY;
   for (int A = 1024; A < 2048; ++A) {
-    const double k = A / c[2 * m - 1];
+    const double k = (A / 1024.0) / c[2 * m - 1];
     double err = 0.0;
     for (int i = m; i < 2 * m; ++i) {
       const double v = k * c[i];

@@ -58,11 +58,20 @@ __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier
 __device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_addr(dst)),
-               "l"(src), "r"(bytes), "r"(smem_addr(bar))
-               : "memory");
+// L2 policy for data read once per step (the packed tiles): evicted first, so that the
+// small per-layer constants (rotations) stay in L2 from one step to the next.
+__device__ __forceinline__ unsigned long long evict_first_policy() {
+  unsigned long long pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar,
+                                          unsigned long long policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
   unsigned ok;
@@ -173,74 +182,102 @@ struct Luts {
   unsigned v[kV];        // value pairs: rates 2-3 lane-private, rate 4 shared
 };
 
-// Scores of one key group with compile-time rate R over the quads [q0, q1) of a tile: for
-// each quad, the lane's codes (pair t of the quad, tokens g + 8 m) come in with one load;
-// slots m = 2 rt and 2 rt + 1 give the A fragment of row block rt of an m16n8k8 product
-// with the quad's q' fragment(s). Lanes whose pair is missing (t >= P) multiply whatever
-// they hold with zero B rows.
+// The lane's codes of one quad: Kq<R>::load reads them (rate 3: two planes) at the lane's
+// precomputed byte offsets, a(m) gives the fp16 pair (hi part for rates 3-4) of slot m
+// (token g + 8 m of the tile, dims 2t and 2t+1 of the quad), lo(m) the low parts.
+template <int R, int VR>
+struct Kq;
+template <int VR>
+struct Kq<1, VR> {
+  unsigned w;  // lo codes in bits 8-15, hi codes in bits 24-31
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+    w = prmt(*reinterpret_cast<const unsigned short*>(tb + (off & 0xffffu)), 0u, 0x1404u);
+  }
+  __device__ __forceinline__ unsigned a(int m, const Luts<VR>&, unsigned) const { return sign_pair(w << (7 - m)); }
+  __device__ __forceinline__ unsigned lo(int, const Luts<VR>&) const { return 0u; }
+};
+template <int VR>
+struct Kq<2, VR> {
+  unsigned w;  // nibble m = lo | hi << 2
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+    w = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
+  }
+  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned lane4) const {
+    return lds_u32(T.k2, (shr(w, 4 * m - 7) & 0x780u) | lane4);  // entry at 128 nibble + 4 lane
+  }
+  __device__ __forceinline__ unsigned lo(int, const Luts<VR>&) const { return 0u; }
+};
+template <int VR>
+struct Kq<3, VR> {
+  unsigned f[8];  // byte offsets (8 x field) of the eight 6-bit fields in the pair table
+  uint2 e[8];
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+    const unsigned wa = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
+    const unsigned wb = *reinterpret_cast<const unsigned short*>(tb + (off >> 16));
+    f[0] = (wa << 3) & 0x1f8u;
+    f[1] = (wa >> 3) & 0x1f8u;
+    f[2] = (wa >> 9) & 0x1f8u;
+    f[3] = (wa >> 15) & 0x1f8u;
+    f[4] = (wa >> 21) & 0x1f8u;
+    f[5] = (__funnelshift_r(wa, wb, 30) << 3) & 0x1f8u;
+    f[6] = (wb >> 1) & 0x1f8u;
+    f[7] = (wb >> 7) & 0x1f8u;
+  }
+  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned) { e[m] = lds_u64(T.k3, f[m]); return e[m].x; }
+  __device__ __forceinline__ unsigned lo(int m, const Luts<VR>&) const { return e[m].y; }
+};
+template <int VR>
+struct Kq<4, VR> {
+  uint2 w;  // byte m = lo | hi << 4
+  uint2 e[8];
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+    w = *reinterpret_cast<const uint2*>(tb + (off & 0xffffu));
+  }
+  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned) {
+    const unsigned x = m < 4 ? w.x : w.y;
+    e[m] = lds_u64(T.k4, shr(x, 8 * (m & 3) - 3) & 0x7f8u);
+    return e[m].x;
+  }
+  __device__ __forceinline__ unsigned lo(int m, const Luts<VR>&) const { return e[m].y; }
+};
+
+// Scores of one key group with compile-time rate R over its quads [q0, q1) of a tile.
+// Quads go in pairs into m16n8k16 products (quad q: k columns 0-7, quad q+1: 8-15); a
+// group's odd last quad takes an m16n8k8 product. Row block rt of the tile: rows g and
+// g+8 are slots m = 2 rt and 2 rt + 1. loff[q][lane] = byte offset of the lane's codes in
+// the tile (for a lane without a pair of that quad: any code, its q' rows are zero).
 template <int R, bool NP, int VR>
-__device__ __forceinline__ void key_group(float (&acc)[4][4], const unsigned char* tb, const unsigned* qdesc,
+__device__ __forceinline__ void key_group(float (&acc)[4][4], const unsigned char* tb, const unsigned* loff,
                                           const unsigned* qf, int q0, int q1, int lane, const Luts<VR>& T) {
-  const int g = lane >> 2, t = lane & 3;
   const unsigned lane4 = unsigned(lane) << 2;
-  for (int q = q0; q < q1; ++q) {
-    const unsigned desc = qdesc[q];
-    const int off = int(desc & 0xffffu), P = int(desc >> 16);
-    const int li = t < P ? g * P + t : 0;
-    const unsigned char* blk = tb + off;
-    const unsigned bh = qf[q * 64 + lane];
-    const unsigned bl = NP ? 0u : qf[q * 64 + 32 + lane];
-    if constexpr (R == 1) {
-      // lo codes in bits 0-7, hi codes in bits 8-15: spread to bits 8-15 and 24-31
-      const unsigned h = reinterpret_cast<const unsigned short*>(blk)[li];
-      const unsigned w = prmt(h, 0u, 0x1404u);
+  int q = q0;
+#pragma unroll 1
+  for (; q + 1 < q1; q += 2) {
+    Kq<R, VR> c0, c1;
+    c0.load(tb, loff[q * 32 + lane]);
+    c1.load(tb, loff[(q + 1) * 32 + lane]);
+    const unsigned bh0 = qf[q * 64 + lane], bh1 = qf[(q + 1) * 64 + lane];
+    const unsigned bl0 = NP ? 0u : qf[q * 64 + 32 + lane], bl1 = NP ? 0u : qf[(q + 1) * 64 + 32 + lane];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        const unsigned a0 = sign_pair(w << (7 - 2 * rt)), a1 = sign_pair(w << (6 - 2 * rt));
-        mma1688(acc[rt], a0, a1, bh);
-        if constexpr (!NP) mma1688(acc[rt], a0, a1, bl);
-      }
-    } else if constexpr (R == 2) {
-      const unsigned w = reinterpret_cast<const unsigned*>(blk)[li];
+    for (int rt = 0; rt < 4; ++rt) {
+      const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
+      const unsigned a2 = c1.a(2 * rt, T, lane4), a3 = c1.a(2 * rt + 1, T, lane4);
+      mma16816(acc[rt], a0, a1, a2, a3, bh0, bh1);
+      if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, bl0, bl1);
+      if constexpr (R >= 3)
+        mma16816(acc[rt], c0.lo(2 * rt, T), c0.lo(2 * rt + 1, T), c1.lo(2 * rt, T), c1.lo(2 * rt + 1, T), bh0, bh1);
+    }
+  }
+  if (q < q1) {
+    Kq<R, VR> c0;
+    c0.load(tb, loff[q * 32 + lane]);
+    const unsigned bh = qf[q * 64 + lane], bl = NP ? 0u : qf[q * 64 + 32 + lane];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        // nibble m -> entry m at byte ((w >> 4m) & 15) * 128 + 4 lane
-        const unsigned a0 = lds_u32(T.k2, (shr(w, 8 * rt - 7) & 0x780u) | lane4);
-        const unsigned a1 = lds_u32(T.k2, (shr(w, 8 * rt - 3) & 0x780u) | lane4);
-        mma1688(acc[rt], a0, a1, bh);
-        if constexpr (!NP) mma1688(acc[rt], a0, a1, bl);
-      }
-    } else if constexpr (R == 3) {
-      const unsigned wa = reinterpret_cast<const unsigned*>(blk)[li];
-      const unsigned wb = reinterpret_cast<const unsigned short*>(blk + 32 * P)[li];
-      unsigned f[8];  // byte offsets (8 x field) of the eight 6-bit fields
-      f[0] = (wa << 3) & 0x1f8u;
-      f[1] = (wa >> 3) & 0x1f8u;
-      f[2] = (wa >> 9) & 0x1f8u;
-      f[3] = (wa >> 15) & 0x1f8u;
-      f[4] = (wa >> 21) & 0x1f8u;
-      f[5] = (__funnelshift_r(wa, wb, 30) << 3) & 0x1f8u;
-      f[6] = (wb >> 1) & 0x1f8u;
-      f[7] = (wb >> 7) & 0x1f8u;
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        const uint2 e0 = lds_u64(T.k3, f[2 * rt]), e1 = lds_u64(T.k3, f[2 * rt + 1]);
-        mma1688(acc[rt], e0.x, e1.x, bh);
-        if constexpr (!NP) mma1688(acc[rt], e0.x, e1.x, bl);
-        mma1688(acc[rt], e0.y, e1.y, bh);
-      }
-    } else {
-      const uint2 w = reinterpret_cast<const uint2*>(blk)[li];
-#pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
-        const unsigned x = rt < 2 ? w.x : w.y;
-        const int sb = 16 * (rt & 1);  // byte m = 2 rt at bit sb of x, byte 2 rt + 1 at sb + 8
-        const uint2 e0 = lds_u64(T.k4, shr(x, sb - 3) & 0x7f8u);
-        const uint2 e1 = lds_u64(T.k4, (x >> (sb + 5)) & 0x7f8u);
-        mma1688(acc[rt], e0.x, e1.x, bh);
-        if constexpr (!NP) mma1688(acc[rt], e0.x, e1.x, bl);
-        mma1688(acc[rt], e0.y, e1.y, bh);
-      }
+    for (int rt = 0; rt < 4; ++rt) {
+      const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
+      mma1688(acc[rt], a0, a1, bh);
+      if constexpr (!NP) mma1688(acc[rt], a0, a1, bl);
+      if constexpr (R >= 3) mma1688(acc[rt], c0.lo(2 * rt, T), c0.lo(2 * rt + 1, T), bh);
     }
   }
 }
@@ -346,38 +383,51 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   __shared__ float qr[kMaxG * kD];                   // q' in packed order
   const int tid = threadIdx.x, ng = L.n_kgroups;
   const int b = u / h_kv, h = u % h_kv;
+  // this thread's row of R_g: the first 16 float4 are loaded before q arrives
+  const int p = tid & (kD - 1), h0 = (tid >> 7) * 4;
+  int g = 0, pad = 0;
+  while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
+  const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
+  const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld);
+  constexpr int kPre = 16;
+  float4 r[kPre];
+#pragma unroll
+  for (int j4 = 0; j4 < kPre; ++j4) r[j4] = j4 < ld / 4 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < kMaxG * kQsLd; e += kPrepThreads) qs[e] = 0.f;
   __syncthreads();
   for (int e = tid; e < G * kD; e += kPrepThreads) {
-    const int hh = e >> 7, p = e & (kD - 1);
-    int g = 0, pad = 0;
-    while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
-    qs[hh * kQsLd + pad + p - L.group_off[g]] =
-        load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + L.packed_coord[p]);
+    const int hh = e >> 7, pe = e & (kD - 1);
+    int ge = 0, pade = 0;
+    while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
+    qs[hh * kQsLd + pade + pe - L.group_off[ge]] =
+        load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + L.packed_coord[pe]);
   }
   __syncthreads();
-  {
-    const int p = tid & (kD - 1), h0 = (tid >> 7) * 4;
-    int g = 0, pad = 0;
-    while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
-    const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
-    if (h0 < G) {
-      const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld);
-      const float* qg = qs + h0 * kQsLd + pad;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-      for (int j4 = 0; j4 < ld / 4; ++j4) {
-        const float4 r = __ldg(row + j4);
+  if (h0 < G) {
+    const float* qg = qs + h0 * kQsLd + pad;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j4 = 0; j4 < kPre; ++j4) {
+      if (j4 < ld / 4) {  // q columns past the group's padded row are not read
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
-          acc[k] = fmaf(r.x, x.x, fmaf(r.y, x.y, fmaf(r.z, x.z, fmaf(r.w, x.w, acc[k]))));
+          acc[k] = fmaf(r[j4].x, x.x, fmaf(r[j4].y, x.y, fmaf(r[j4].z, x.z, fmaf(r[j4].w, x.w, acc[k]))));
         }
       }
-      const float f = qscale * rsqrtf(float(d));
-#pragma unroll
-      for (int k = 0; k < 4; ++k) qr[(h0 + k) * kD + p] = acc[k] * f;
     }
+#pragma unroll 8
+    for (int j4 = kPre; j4 < ld / 4; ++j4) {
+      const float4 rr = __ldg(row + j4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
+        acc[k] = fmaf(rr.x, x.x, fmaf(rr.y, x.y, fmaf(rr.z, x.z, fmaf(rr.w, x.w, acc[k]))));
+      }
+    }
+    const float f = qscale * rsqrtf(float(d)) * L.inv_kappa_group[g];  // the key tables carry kappa
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qr[(h0 + k) * kD + p] = acc[k] * f;
   }
   __syncthreads();
   for (int e = tid; e < L.n_kquads * 64; e += kPrepThreads) {
@@ -391,8 +441,8 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
       v0 = qr[hh * kD + d0];
       v1 = qr[hh * kD + d0 + 1];
     }
-    const float h0 = __half2float(__float2half_rn(v0)), h1 = __half2float(__float2half_rn(v1));
-    frag[qi * 64 + j] = lo ? pack_h2(v0 - h0, v1 - h1) : pack_h2(h0, h1);
+    const float r0 = __half2float(__float2half_rn(v0)), r1 = __half2float(__float2half_rn(v1));
+    frag[qi * 64 + j] = lo ? pack_h2(v0 - r0, v1 - r1) : pack_h2(r0, r1);
   }
 }
 
@@ -433,9 +483,8 @@ template <int VR, bool NP>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(16) Luts<VR> T;
-  __shared__ unsigned s_qdesc[kMaxQuads];
-  __shared__ int s_group[kMaxGroups][3];  // first quad, end quad, rate
-  __shared__ float s_ik[kMaxGroups];      // 1 / kappa of the group's rate (the fp16 key tables are scaled)
+  __shared__ unsigned s_loff[kMaxQuads * 32];  // [quad][lane]: byte offsets of the lane's codes in a tile
+  __shared__ int s_group[kMaxGroups][3];      // first quad, end quad, rate
   __shared__ int s_timeout;
   __shared__ Segment s_seg[2];
   __shared__ int s_nseg;
@@ -483,13 +532,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
   } else if constexpr (VR == 4) {
     for (int e = tid; e < 256; e += kThreads) T.v[e] = unsigned(L.vc[e & 15]) | (unsigned(L.vc[e >> 4]) << 16);
   }
-  for (int i = tid; i < L.n_kquads; i += kThreads)
-    s_qdesc[i] = unsigned(L.quad_off[i]) | (unsigned(L.quad_np[i]) << 16);
+  for (int gi = 0; gi < L.n_kgroups; ++gi) {
+    const int r = L.group_rate[gi], q0 = L.group_quad0[gi];
+    for (int i = tid; i < L.group_nquads[gi] * 32; i += kThreads) {
+      // lane (g, t) holds pair t of the quad for tokens g + 8m: its 16 r bits are string
+      // li = g P + t of the block (rate 3: plane A word li, plane B halfword li after 8 P words)
+      const int qi = q0 + i / 32, ln = i % 32, P = L.quad_np[qi], t = ln & 3;
+      const int li = t < P ? (ln >> 2) * P + t : 0;
+      const unsigned base = unsigned(L.quad_off[qi]);
+      s_loff[qi * 32 + ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
+    }
+  }
   if (tid < L.n_kgroups) {
     s_group[tid][0] = L.group_quad0[tid];
     s_group[tid][1] = L.group_quad0[tid] + L.group_nquads[tid];
     s_group[tid][2] = L.group_rate[tid];
-    s_ik[tid] = L.inv_kappa_group[tid];
   }
   __syncthreads();
   const int nseg = s_nseg;
@@ -500,6 +557,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
   const int ng = L.n_kgroups;
   const float vscale = rsqrtf(float(kD)) / L.kappa_v;
   const unsigned lane4 = unsigned(lane) << 2;
+  const unsigned long long l2_stream = evict_first_policy();
   unsigned phase = 0;   // bit k&1: parity of the next completion of stage w + 4 (k & 1)
   unsigned pend = 0;    // bit k&1: a copy into stage w + 4 (k & 1) is in flight
   bool waited = !a.wait_new;
@@ -516,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       }
       const int st = warp + kWarps * (k & 1);
       mbar_expect_tx(&full[st], TB);
-      bulk_load(ring + st * TB, src + (size_t)it * TB, TB, &full[st]);
+      bulk_load(ring + st * TB, src + (size_t)it * TB, TB, &full[st], l2_stream);
     };
     if (lane == 0)
       for (int k = 0; k < min(2, mine); ++k) issue(k);
@@ -569,15 +627,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
           for (int j = 0; j < 4; ++j) acc[rt][j] = 0.f;
         const int q0 = s_group[gi][0], q1 = s_group[gi][1];
         switch (s_group[gi][2]) {
-          case 1: key_group<1, NP, VR>(acc, tb, s_qdesc, qf, q0, q1, lane, T); break;
-          case 2: key_group<2, NP, VR>(acc, tb, s_qdesc, qf, q0, q1, lane, T); break;
-          case 3: key_group<3, NP, VR>(acc, tb, s_qdesc, qf, q0, q1, lane, T); break;
-          default: key_group<4, NP, VR>(acc, tb, s_qdesc, qf, q0, q1, lane, T); break;
+          case 1: key_group<1, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
+          case 2: key_group<2, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
+          case 3: key_group<3, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
+          default: key_group<4, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
         }
-        const float ik = s_ik[gi];
 #pragma unroll
         for (int rt = 0; rt < 4; ++rt) {
-          const float n0 = kn[gi * kTile + 16 * rt + g] * ik, n1 = kn[gi * kTile + 16 * rt + g + 8] * ik;
+          const float n0 = kn[gi * kTile + 16 * rt + g], n1 = kn[gi * kTile + 16 * rt + g + 8];
           sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
           sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
           sc[rt][2] = fmaf(acc[rt][2], n1, sc[rt][2]);
@@ -769,6 +826,15 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   const int n = cta_of_tile((long long)(u + 1) * M - 1, total_tiles, n_ctas) - cta_of_tile((long long)u * M, total_tiles, n_ctas) + 1;
   pdl_wait();  // partials come from split_kernel
   const float2* ml = reinterpret_cast<const float2*>(part_ml) + (size_t)u * S * G + hh;  // slot sp at ml[sp * G]
+  const float* po = part_o + ((size_t)u * S * G + hh) * kD + d;                          // slot sp at po[sp * G * kD]
+  // every load of the merge is issued at once: (m, l) of two slots, o' of 16 slots
+  constexpr int kPv = 16;
+  float pv[kPv];
+#pragma unroll
+  for (int k = 0; k < kPv; ++k) {
+    const int sp = qtr + 4 * k;
+    pv[k] = sp < n ? __ldg(po + (size_t)sp * G * kD) : 0.f;
+  }
   float mloc[2], lloc[2];
   float Mx = -INFINITY;
 #pragma unroll
@@ -802,15 +868,14 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
 #pragma unroll
   for (int i = 0; i < kCombThreads / 32; ++i) l += red[1][i];
   {
-    const float* po = part_o + ((size_t)u * S * G + hh) * kD + d;  // slot sp at po[sp * G * kD]
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    int sp = qtr;
-    for (; sp + 12 < n; sp += 16) {
+    float o0 = 0.f, o1 = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) o[k] = fmaf(w[sp + 4 * k], __ldg(po + (size_t)(sp + 4 * k) * G * kD), o[k]);
+    for (int k = 0; k < kPv; k += 2) {
+      if (qtr + 4 * k < n) o0 = fmaf(w[qtr + 4 * k], pv[k], o0);
+      if (qtr + 4 * (k + 1) < n) o1 = fmaf(w[qtr + 4 * (k + 1)], pv[k + 1], o1);
     }
-    for (; sp < n; sp += 4) o[0] = fmaf(w[sp], __ldg(po + (size_t)sp * G * kD), o[0]);
-    part[qtr][d] = (o[0] + o[1]) + (o[2] + o[3]);
+    for (int sp = qtr + 4 * kPv; sp < n; sp += 4) o0 = fmaf(w[sp], __ldg(po + (size_t)sp * G * kD), o0);
+    part[qtr][d] = o0 + o1;
   }
   __syncthreads();
   if (tid < kD) op[tid] = l > 0.f ? ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) / l : 0.f;
