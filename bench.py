@@ -11,6 +11,7 @@ the 126 MB L2). The step is captured in a CUDA graph and replayed.
     python bench.py --impl reference ...      # the CPU oracle, timed on the host cores
     python bench.py --mode sweep              # decode over the 32q/8kv context x batch x rate grid
     python bench.py --mode encode             # tq_encode append throughput, 1 and 64 new tokens
+    python bench.py --mode mae                # K-only logit error: block rates vs uniform rates
 
 Prints one JSON line (rank 0).
 """
@@ -353,6 +354,43 @@ def run_encode(args):
                               "token_heads_per_s": toks * 8 / (ms * 1e-3)}), flush=True)
 
 
+def run_mae(args):
+    """K-only logit error of the block rate allocation against uniform rates at the same
+    bit budget, on the 8B- and 3B-shaped generators (8192 cached tokens, one layer): the
+    logits come from bgtq_decode_scores over each packed cache, the exact ones from the
+    unquantised keys (fp64). Reports the mean absolute logit error of both layouts."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    for name in ("llama8b", "qwen3b"):
+        base = synth.WORKLOADS[name]
+        wl = synth.Workload(**{**base.__dict__, "length": 8192, "batch": 1, "layers": 1})
+        m = synth.make_layer_model(wl.h_q, wl.h_kv, wl.seed)
+        q_cal, k_cal = synth.make_calibration(m, 256, wl.seed + 1, wl.theta)
+        rates = B.plan_layer_rates(q_cal.numpy(), k_cal.numpy(), wl.k_bits)
+        q, k, v = synth.make_cache_inputs(m, 1, wl.length, wl.seed, wl.theta, torch.float32)
+        scale = 1.0 / math.sqrt(128)
+        G = wl.h_q // wl.h_kv
+        exact = torch.einsum("hgd,htd->hgt", q[0].view(wl.h_kv, G, 128).double(), k[0].transpose(0, 1).double())
+        exact = (exact * scale).reshape(wl.h_q, wl.length).to(dev)
+        line = {"mode": "mae", "workload": wl.name, "tokens": wl.length, "k_bits": wl.k_bits,
+                "block_rates": {str(r): int((rates == r).sum()) for r in sorted(set(rates.tolist()))}}
+        for tag, rr in (("block_gtq", rates), ("uniform", np.full(64, wl.k_bits))):
+            lay = B.Layout(rr, wl.v_bits, wl.seed).upload(0)
+            cap = wl.length
+            cache = torch.zeros(lay.cache_bytes(1, wl.h_kv, cap), dtype=torch.uint8, device=dev)
+            lens = torch.zeros(1, dtype=torch.int32, device=dev)
+            B.encode_append(lay, k.to(dev), v.to(dev), lens, cache, cap)
+            lens.fill_(wl.length)
+            ws = torch.empty(B.workspace_bytes(lay, 1, wl.h_q, wl.h_kv, wl.length), dtype=torch.uint8, device=dev)
+            sc = torch.empty(1, wl.h_q, wl.length, dtype=torch.float32, device=dev)
+            B.decode_scores(lay, q.to(dev), cache, lens, cap, wl.length, sc, ws, wl.h_kv)
+            torch.cuda.synchronize()
+            line[f"mae_{tag}"] = float((sc[0].double() - exact).abs().mean())
+            line[f"bytes_per_token_{tag}"] = lay.bytes_per_token
+        line["reduction"] = 1.0 - line["mae_block_gtq"] / line["mae_uniform"]
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -364,12 +402,14 @@ def main():
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="step", choices=["step", "sweep", "encode"])
+    ap.add_argument("--mode", default="step", choices=["step", "sweep", "encode", "mae"])
     args = ap.parse_args()
     if args.mode == "sweep":
         return run_sweep(args)
     if args.mode == "encode":
         return run_encode(args)
+    if args.mode == "mae":
+        return run_mae(args)
     wl = synth.WORKLOADS[args.workload]
     if args.layers:
         wl = synth.Workload(**{**wl.__dict__, "layers": args.layers})

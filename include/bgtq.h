@@ -194,6 +194,19 @@ bgtq_status bgtq_decode_step(const bgtq_layout* layout, const void* k_new, const
                              long long max_seq_len, float softmax_scale, float* out,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Attention logits over the packed cache [BGTQ s5]: scores[(b*h_q + i)*scores_ld + t] =
+ * softmax_scale * q_i . k_hat_t for every cached token t < seq_lens_dev[b] (k_hat decoded
+ * from the packed codes: sum over groups of |k_g|/sqrt(d_g) R_g^T c[codes]), fp32 device
+ * memory owned by the caller; entries at t >= seq_lens_dev[b] are not written.
+ * scores_ld >= max_seq_len. Other arguments and the workspace as for
+ * bgtq_decode_attention. Computed with the same key path as the attention (for
+ * diagnostics such as the logit error of a rate allocation). */
+bgtq_status bgtq_decode_scores(const bgtq_layout* layout, const void* q, int q_dtype, int batch,
+                               int h_q, int h_kv, const void* cache, const int* seq_lens_dev,
+                               long long capacity, long long max_seq_len, float softmax_scale,
+                               float* scores, long long scores_ld, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- no-allocation variant */
 
 /* The pages have no counterpart to this call: it is a library convenience.

@@ -616,3 +616,22 @@ def decode_attention(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int
     u = unpack(layout, buf, length)
     kh, vh = reconstruct(layout, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
     return attention(q, kh, vh, scale)
+
+
+def decode_scores(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int, scale: float) -> np.ndarray:
+    """Logits scale * q . k_hat of the G query heads q [G, 128] against every cached token of
+    one KV head's packed cache [BGTQ sentence 5: scores over the packed codes]; [G, length]."""
+    u = unpack(layout, buf, length)
+    kh, _ = reconstruct(layout, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
+    return (np.asarray(q, dtype=np.float64) @ kh.T) * scale
+
+
+def logit_mae(layout: Layout, q: np.ndarray, k: np.ndarray, scale: float) -> float:
+    """K-only logit error of a layout [BGTQ sentence 6: layer-averaged logit MAE against
+    uniform TQ-MSE]: mean over query heads and tokens of |scale q . k_hat - scale q . k|,
+    where k_hat is the TQ-MSE reconstruction of the keys k [n, 128] (values unused)."""
+    k = np.asarray(k, dtype=np.float64)
+    enc = encode(layout, k, np.zeros_like(k))
+    kh, _ = reconstruct(layout, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+    q = np.asarray(q, dtype=np.float64)
+    return float(np.mean(np.abs((q @ kh.T - q @ k.T) * scale)))

@@ -26,7 +26,7 @@ EXPORTED = [
     "bgtq_layout_create", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
     "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
-    "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step",
+    "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
 ]
 
 
@@ -71,6 +71,7 @@ def load():
         "bgtq_decode_attention_noalloc": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P]),
         "bgtq_noalloc_scratch_capacity": (C.c_size_t, []),
         "bgtq_decode_step": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_scores": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, LL, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -258,6 +259,20 @@ def decode_step(layout: Layout, k_new, v_new, q, cache, seq_lens, capacity: int,
                                    max_seq_len, scale, C.c_void_p(out.data_ptr()),
                                    C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_step")
+
+
+def decode_scores(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, scores, workspace,
+                  h_kv: int, softmax_scale: float | None = None, stream=None):
+    """Logits softmax_scale * q . k_hat over the packed cache: scores [B, h_q, >= max_seq_len]
+    fp32 CUDA (entries past each row's length are left as they are)."""
+    B_, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and scores.is_contiguous() and scores.shape[:2] == (B_, h_q)
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_scores(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q, h_kv,
+                                     C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                     max_seq_len, scale, C.c_void_p(scores.data_ptr()), scores.shape[2],
+                                     C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_scores")
 
 
 def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out,

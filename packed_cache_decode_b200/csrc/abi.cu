@@ -297,6 +297,36 @@ bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void
   return BGTQ_OK;
 }
 
+bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q, int h_kv,
+                               const void* cache, const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                               float softmax_scale, float* scores, long long scores_ld, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_device(L, "decode_scores");
+  if (st != BGTQ_OK) return st;
+  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_scores: bad dtype");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
+    return fail(BGTQ_ERR_INVALID, "decode_scores: need h_q = G * h_kv with G in 1..8");
+  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_scores: batch * h_kv > 65535");
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, "decode_scores: capacity must be a positive multiple of 64");
+  if (max_seq_len < 0 || max_seq_len > capacity)
+    return fail(BGTQ_ERR_CAPACITY, "decode_scores: max_seq_len must be in [0, capacity]");
+  if (scores_ld < max_seq_len) return fail(BGTQ_ERR_INVALID, "decode_scores: scores_ld < max_seq_len");
+  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_scores: bad softmax_scale");
+  if (!q || !cache || !seq_lens_dev || !scores) return fail(BGTQ_ERR_INVALID, "decode_scores: null pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_scores");
+  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  if (!workspace || workspace_bytes < plan.workspace_bytes)
+    return fail(BGTQ_ERR_WORKSPACE, "decode_scores: workspace missing or smaller than bgtq_workspace_bytes()");
+  e = launch_scores(L->dev, plan, q, q_dtype, batch, h_q, h_kv, cache, seq_lens_dev, capacity / kTile, softmax_scale,
+                    scores, scores_ld, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_scores");
+  return BGTQ_OK;
+}
+
 bgtq_status bgtq_device_status(const bgtq_layout* L, unsigned* flags, int clear) {
   bgtq_status st = check_device(L, "device_status");
   if (st != BGTQ_OK) return st;

@@ -133,6 +133,8 @@ struct SplitArgs {
   int h_q, h_kv, G;
   float* part_ml;         // [units][n_parts][G][2]
   float* part_o;          // [units][n_parts][G][128]
+  float* scores;          // scores-only mode: [batch][h_q][scores_ld] logits (softmax_scale q.k_hat)
+  long long scores_ld;
   int len_add;            // tokens appended by the previous kernel: row b attends over seq_lens[b] + len_add
   int wait_new;           // the previous kernel appends at seq_lens[b]: wait for it before copying that tile
 };
@@ -479,7 +481,9 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
   }
 }
 
-template <int VR, bool NP>
+// SC: scores only. The tiles' logits (softmax_scale q . k_hat, natural units) go to
+// a.scores; no softmax, values, partials or merge.
+template <int VR, bool NP, bool SC = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(16) Luts<VR> T;
@@ -654,6 +658,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         if (gt0 + 16 * rt + 8 >= S.len) sc[rt][2] = sc[rt][3] = -INFINITY;
       }
 
+      if constexpr (SC) {
+        // column 2t + c holds head 2t + c (G <= 4: lanes t < 2; t >= 2 hold copies)
+        const int b = S.u / a.h_kv, hkv = S.u % a.h_kv;
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int head = 2 * t + (j & 1);
+            const long long tok = gt0 + 16 * rt + 8 * (j >> 1);
+            if ((!NP || t < 2) && head < a.G && tok < S.len)
+              a.scores[((size_t)b * a.h_q + (size_t)hkv * a.G + head) * a.scores_ld + tok] = sc[rt][j] * (1.f / kLog2e);
+          }
+      } else {
       // ---------------- online softmax over the 64 tokens (heads of columns 2t, 2t+1), base 2
       float x0 = -INFINITY, x1 = -INFINITY;
 #pragma unroll
@@ -709,6 +726,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
           mma16816(O[mt], vl.field(4 * mt, T.v, lane4), vl.field(4 * mt + 1, T.v, lane4),
                    vl.field(4 * mt + 2, T.v, lane4), vl.field(4 * mt + 3, T.v, lane4), pb[rt][0], pb[rt][1]);
       }
+      }  // not scores-only
       __syncwarp();  // every lane is done with the stage before it is refilled
       if (k + 2 < mine) {
         if (lane == 0) issue(k + 2);
@@ -721,6 +739,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
     // with the segment's tiles and has no copy in flight)
     __syncthreads();
     if (*static_cast<volatile int*>(&s_timeout)) break;  // uniform over the CTA
+    if constexpr (SC) continue;  // the q' fragments are reloaded for the next segment
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -774,14 +793,14 @@ size_t split_smem_bytes(int tile_bytes) {
   return 128 + size_t(kRing) * tile_bytes + kMaxQuads * 64 * sizeof(unsigned) + 2 * kWarps * 8 * sizeof(float);
 }
 
-template <int VR, bool NP>
+template <int VR, bool NP, bool SC = false>
 cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, cudaStream_t stream) {
   const size_t smem = split_smem_bytes(L.tile_bytes);
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(split_kernel<VR, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(split_kernel<VR, NP, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(split_smem_bytes(kMaxTileBytes)));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
@@ -796,7 +815,7 @@ cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP>, L, a);
+  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC>, L, a);
 }
 
 // ------------------------------------------------------------------ combine
@@ -891,10 +910,10 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   if (tid < kD) out[((size_t)b * h_q + hq) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
 }
 
-template <int VR, bool NP>
+template <int VR, bool NP, bool SC = false>
 int split_occupancy(const DevLayout& L) {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<VR, NP>, kThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<VR, NP, SC>, kThreads,
                                                     split_smem_bytes(L.tile_bytes)) != cudaSuccess)
     return 1;
   return n < 1 ? 1 : n;
@@ -904,15 +923,19 @@ int split_occupancy(const DevLayout& L) {
 // kernel that wrote the q' fragments (and, after an append, the new tokens).
 cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int batch, int h_q, int h_kv,
                              const void* cache, const int* seq_lens, long long n_tiles, float* out, void* workspace,
-                             int len_add, bool after_append, cudaStream_t stream) {
+                             int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
+                             long long scores_ld = 0) {
   const int G = h_q / h_kv;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
-  const int variant = L.v_rate * 2 + (np ? 1 : 0);
+  // scores only: variants 0 (G > 4) and 1 (G <= 4), no value tables
+  const int variant = scores ? (np ? 1 : 0) : L.v_rate * 2 + (np ? 1 : 0);
   // the workspace was sized for the most CTAs per SM; shared memory may allow fewer
   // (larger slices, fewer partials per unit)
   int occ = 1;
   switch (variant) {
+    case 0: occ = split_occupancy<1, false, true>(L); break;
+    case 1: occ = split_occupancy<1, true, true>(L); break;
     case 2: occ = split_occupancy<1, false>(L); break;
     case 3: occ = split_occupancy<1, true>(L); break;
     case 4: occ = split_occupancy<2, false>(L); break;
@@ -948,10 +971,14 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   ws += qfrag_bytes(units);
   a.part_ml = reinterpret_cast<float*>(ws);
   a.part_o = reinterpret_cast<float*>(ws + align256(size_t(units) * plan.n_parts * G * 2 * sizeof(float)));
+  a.scores = scores;
+  a.scores_ld = scores_ld;
   a.len_add = len_add;
   a.wait_new = after_append ? 1 : 0;
   const unsigned n_ctas = unsigned(plan.n_ctas);
   switch (variant) {
+    case 0: return launch_split<1, false, true>(a, L, n_ctas, stream);
+    case 1: return launch_split<1, true, true>(a, L, n_ctas, stream);
     case 2: e = launch_split<1, false>(a, L, n_ctas, stream); break;
     case 3: e = launch_split<1, true>(a, L, n_ctas, stream); break;
     case 4: e = launch_split<2, false>(a, L, n_ctas, stream); break;
@@ -1009,6 +1036,18 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, n_tiles, out, workspace, 0, false, stream);
+}
+
+cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
+                          int h_kv, const void* cache, const int* seq_lens, long long n_tiles, float softmax_scale,
+                          float* scores, long long scores_ld, void* workspace, cudaStream_t stream) {
+  const int G = h_q / h_kv;
+  qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
+      L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, n_tiles, nullptr, workspace, 0, false, stream,
+                          scores, scores_ld);
 }
 
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,

@@ -39,4 +39,11 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
                                int batch, int h_q, int h_kv, void* cache, long long n_tiles, float softmax_scale, float* out, void* workspace,
                                cudaStream_t stream);
 
+// Logits only: scores[(b h_q + hq) scores_ld + t] = softmax_scale q . k_hat_t for every
+// cached token t < seq_lens[b] (the q-preparation kernel, then the split kernel in its
+// scores-only form).
+cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
+                          int h_kv, const void* cache, const int* seq_lens, long long n_tiles, float softmax_scale,
+                          float* scores, long long scores_ld, void* workspace, cudaStream_t stream);
+
 }  // namespace bgtq

@@ -396,3 +396,57 @@ def test_decode_attention_equals_rotated_space_form():
     cv = lay.codebooks[3][0][u["v_codes"]] * (u["v_norm"] / math.sqrt(128))[:, None]
     out_rot = (p @ cv) @ lay.v_rot
     np.testing.assert_allclose(out, out_rot, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------------------ scores and logit error
+def test_scores_are_the_logits_of_the_attention():
+    """softmax(scores) @ v_hat reproduces the oracle attention: scores are its logits."""
+    rng = np.random.default_rng(21)
+    lay = O.make_layout(_random_rates(rng), 3, 4)
+    k = rng.standard_normal((90, 128)) * 2
+    v = rng.standard_normal((90, 128))
+    q = rng.standard_normal((3, 128))
+    enc = O.encode(lay, k, v)
+    buf = O.pack(lay, enc, 128)
+    s = O.decode_scores(lay, q, buf, 90, 0.1)
+    assert s.shape == (3, 90)
+    u = O.unpack(lay, buf, 90)
+    _, vh = O.reconstruct(lay, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(p @ vh, O.decode_attention(lay, q, buf, 90, 0.1), rtol=1e-12, atol=1e-12)
+
+
+def test_logit_mae_matches_the_distortion_closed_form():
+    """For Gaussian keys and queries (independent of the rotation), E|q . (k_hat - k)|^2 =
+    |q|^2 |k|^2 D(b) / d per coordinate sum, so the mean absolute error of a uniform b-bit
+    layout is close to sqrt(2/pi) * sqrt(sum_i q_i^2 E[(k_hat - k)_i^2]) and shrinks with
+    b as sqrt(D(b))."""
+    rng = np.random.default_rng(22)
+    q = rng.standard_normal((4, 128))
+    k = rng.standard_normal((3000, 128))
+    maes = []
+    for b in (1, 2, 3, 4):
+        lay = O.make_layout(np.full(64, b), 2, 1)
+        maes.append(O.logit_mae(lay, q, k, 1.0))
+    D = O.lloyd_max_mse_table()
+    for b, m in zip((1, 2, 3, 4), maes):
+        # k_hat - k has per-coordinate variance |k|^2 D(b) / d ~ D(b), isotropic after R^T
+        want = math.sqrt(2 / math.pi) * np.mean(np.linalg.norm(q, axis=1)) * math.sqrt(D[b])
+        assert abs(m / want - 1) < 0.08, (b, m, want)
+    assert maes == sorted(maes, reverse=True)
+
+
+def test_block_allocation_beats_uniform_rates_on_skewed_blocks():
+    """The abstract's claim in its simplest form: with energy concentrated in a few RoPE
+    blocks, the largest-marginal-gain allocation at the same bit budget gives a lower
+    K-only logit error than uniform rates."""
+    m = synth.make_layer_model(4, 1, 7)
+    q_cal, k_cal = synth.make_calibration(m, 256, 8, 5e5)
+    rates = O.greedy_rates(O.block_energy(q_cal.double().numpy(), k_cal.double().numpy()),
+                           O.lloyd_max_mse_table(), 1, 4, 64 * 2)
+    k = synth.key_slice(m, 0, 0, 600, 0, 9, 5e5).double().numpy()
+    q = torch.stack([synth.query_slice(m, 0, i, 1, 599, 9, 5e5)[0] for i in range(4)]).double().numpy()
+    gtq = O.logit_mae(O.make_layout(rates, 2, 3), q, k, 1 / math.sqrt(128))
+    uni = O.logit_mae(O.make_layout(np.full(64, 2), 2, 3), q, k, 1 / math.sqrt(128))
+    assert gtq < 0.8 * uni, (gtq, uni)
