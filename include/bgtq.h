@@ -84,6 +84,8 @@ enum { BGTQ_F32 = 0, BGTQ_BF16 = 1, BGTQ_F16 = 2 };
 #define BGTQ_STATUS_DECODE_CLAMPED 2u   /* decode: seq_len > capacity or > max_seq_len; clamped */
 #define BGTQ_STATUS_TIMEOUT 4u          /* decode: a bulk copy did not complete within the kernel's bounded
                                            wait; that call's output is invalid */
+#define BGTQ_STATUS_BAD_PAGE 8u        /* paged calls: a block-table entry outside the pool; the encode
+                                          skips that token, the attention reads nothing for that tile */
 
 typedef struct bgtq_layout bgtq_layout;
 
@@ -206,6 +208,34 @@ bgtq_status bgtq_decode_scores(const bgtq_layout* layout, const void* q, int q_d
                                long long capacity, long long max_seq_len, float softmax_scale,
                                float* scores, long long scores_ld, void* workspace,
                                size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- paged caches */
+
+/* The calls above with a paged cache (sequences of different lengths share one pool,
+ * e.g. in a serving engine). The pool holds num_pages pages of h_kv * tile_bytes bytes:
+ * page p = the h_kv tiles (KV heads in order, each in the tile format above) of one
+ * 64-token span of one batch row. block_table_dev[b * max_pages + i] (int32, device) is
+ * the page of tokens 64 i .. 64 i + 63 of row b; a row holds at most max_pages * 64
+ * tokens (its "capacity"). Entries outside [0, num_pages) set BGTQ_STATUS_BAD_PAGE (the
+ * encode then skips the token, the attention leaves that tile out); the caller keeps
+ * pages of different rows distinct. Results are the same as with a contiguous cache. */
+long long bgtq_paged_pool_bytes(const bgtq_layout* layout, int h_kv, long long num_pages);
+bgtq_status bgtq_encode_append_paged(const bgtq_layout* layout, const void* k, const void* v, int dtype,
+                                     int batch, int n_new, int h_kv, const int* seq_lens_dev, void* pool,
+                                     long long num_pages, const int* block_table_dev, long long max_pages,
+                                     void* stream);
+bgtq_status bgtq_decode_attention_paged(const bgtq_layout* layout, const void* q, int q_dtype, int batch,
+                                        int h_q, int h_kv, const void* pool, long long num_pages,
+                                        const int* block_table_dev, long long max_pages,
+                                        const int* seq_lens_dev, long long max_seq_len,
+                                        float softmax_scale, float* out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+bgtq_status bgtq_decode_step_paged(const bgtq_layout* layout, const void* k_new, const void* v_new,
+                                   int kv_dtype, int n_new, const void* q, int q_dtype, int batch,
+                                   int h_q, int h_kv, void* pool, long long num_pages,
+                                   const int* block_table_dev, long long max_pages,
+                                   const int* seq_lens_dev, long long max_seq_len, float softmax_scale,
+                                   float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------- no-allocation variant */
 

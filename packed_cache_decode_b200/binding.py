@@ -20,6 +20,8 @@ HEAD_DIM = 128
 TILE_TOKENS = 64
 STATUS_ENCODE_OVERFLOW = 1
 STATUS_DECODE_CLAMPED = 2
+STATUS_TIMEOUT = 4
+STATUS_BAD_PAGE = 8
 
 EXPORTED = [
     "bgtq_last_error_string", "bgtq_version", "bgtq_lloyd_max", "bgtq_block_energy", "bgtq_allocate_rates",
@@ -27,6 +29,7 @@ EXPORTED = [
     "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
     "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
+    "bgtq_paged_pool_bytes", "bgtq_encode_append_paged", "bgtq_decode_attention_paged", "bgtq_decode_step_paged",
 ]
 
 
@@ -72,6 +75,10 @@ def load():
         "bgtq_noalloc_scratch_capacity": (C.c_size_t, []),
         "bgtq_decode_step": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
         "bgtq_decode_scores": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, LL, P, C.c_size_t, P]),
+        "bgtq_paged_pool_bytes": (LL, [P, I, LL]),
+        "bgtq_encode_append_paged": (I, [P, P, P, I, I, I, I, P, P, LL, P, LL, P]),
+        "bgtq_decode_attention_paged": (I, [P, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_step_paged": (I, [P, P, P, I, I, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -273,6 +280,73 @@ def decode_scores(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len
                                      max_seq_len, scale, C.c_void_p(scores.data_ptr()), scores.shape[2],
                                      C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_scores")
+
+
+class PagedCache:
+    """A pool of pages (uint8 CUDA tensor) and a block table [batch, max_pages] (int32 CUDA):
+    page p holds the h_kv tiles of one 64-token span of one row."""
+
+    def __init__(self, pool, block_table):
+        import torch
+        assert pool.dtype == torch.uint8 and block_table.dtype == torch.int32
+        assert block_table.is_contiguous() and block_table.dim() == 2
+        self.pool, self.table = pool, block_table
+
+    def num_pages(self, layout: "Layout", h_kv: int) -> int:
+        return self.pool.numel() // (h_kv * layout.tile_bytes)
+
+    @property
+    def max_pages(self) -> int:
+        return self.table.shape[1]
+
+
+def paged_pool_bytes(layout: Layout, h_kv: int, num_pages: int) -> int:
+    n = load().bgtq_paged_pool_bytes(layout.handle, h_kv, num_pages)
+    if n < 0:
+        _check(ERR_INVALID, "paged_pool_bytes")
+    return int(n)
+
+
+def encode_append_paged(layout: Layout, k, v, seq_lens, cache: PagedCache, stream=None):
+    """k, v [B, n_new, h_kv, 128]; tokens go to the pages the block table names."""
+    B_, n_new, h_kv, d = k.shape
+    assert d == HEAD_DIM and k.is_contiguous() and v.is_contiguous() and v.shape == k.shape and v.dtype == k.dtype
+    _check(load().bgtq_encode_append_paged(layout.handle, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()),
+                                           dtype_code(k), B_, n_new, h_kv, C.c_void_p(seq_lens.data_ptr()),
+                                           C.c_void_p(cache.pool.data_ptr()), cache.num_pages(layout, h_kv),
+                                           C.c_void_p(cache.table.data_ptr()), cache.max_pages, _stream_ptr(stream)),
+           "encode_append_paged")
+
+
+def decode_attention_paged(layout: Layout, q, cache: PagedCache, seq_lens, max_seq_len: int, out, workspace,
+                           h_kv: int, softmax_scale: float | None = None, stream=None):
+    B_, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_paged(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q, h_kv,
+                                              C.c_void_p(cache.pool.data_ptr()), cache.num_pages(layout, h_kv),
+                                              C.c_void_p(cache.table.data_ptr()), cache.max_pages,
+                                              C.c_void_p(seq_lens.data_ptr()), max_seq_len, scale,
+                                              C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                              workspace.numel(), _stream_ptr(stream)),
+           "decode_attention_paged")
+
+
+def decode_step_paged(layout: Layout, k_new, v_new, q, cache: PagedCache, seq_lens, max_seq_len: int, out,
+                      workspace, softmax_scale: float | None = None, stream=None):
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and k_new.is_contiguous() and v_new.is_contiguous() and v_new.shape == k_new.shape
+    Bq, h_q, dq = q.shape
+    assert Bq == B_ and dq == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_paged(layout.handle, C.c_void_p(k_new.data_ptr()), C.c_void_p(v_new.data_ptr()),
+                                         dtype_code(k_new), n_new, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q,
+                                         h_kv, C.c_void_p(cache.pool.data_ptr()), cache.num_pages(layout, h_kv),
+                                         C.c_void_p(cache.table.data_ptr()), cache.max_pages,
+                                         C.c_void_p(seq_lens.data_ptr()), max_seq_len, scale,
+                                         C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                         workspace.numel(), _stream_ptr(stream)),
+           "decode_step_paged")
 
 
 def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out,

@@ -204,22 +204,109 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   return BGTQ_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The checks and launches shared by the contiguous and the paged entry points; the
+// caller has checked the cache description and passes it as a CacheRef.
+bgtq_status encode_impl(const bgtq_layout* L, const char* who, const void* k, const void* v, int dtype, int batch,
+                        int n_new, int h_kv, const int* seq_lens_dev, const CacheRef& c, void* stream) {
+  if (!valid_dtype(dtype)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad dtype");
+  if (batch <= 0 || batch > 65535 || h_kv <= 0 || h_kv > 65535 || n_new < 0)
+    return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad batch / h_kv / n_new");
+  if (n_new == 0) return BGTQ_OK;
+  if (!k || !v || !seq_lens_dev) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
+  cudaError_t e = launch_tq_encode(L->dev, k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return BGTQ_OK;
+}
+
+// Shape checks of the attention calls; on success *plan is the launch plan.
+bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype, int batch, int h_q, int h_kv,
+                             long long row_tokens, long long max_seq_len, float softmax_scale, const void* q,
+                             const int* seq_lens_dev, const void* out, void* workspace, size_t workspace_bytes,
+                             DecodePlan* plan) {
+  const std::string w(who);
+  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, w + ": bad dtype");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
+    return fail(BGTQ_ERR_INVALID, w + ": need h_q = G * h_kv with G in 1..8");
+  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, w + ": batch * h_kv > 65535");
+  if (max_seq_len < 0 || max_seq_len > row_tokens)
+    return fail(BGTQ_ERR_CAPACITY, w + ": max_seq_len must be in [0, capacity]");
+  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, w + ": bad softmax_scale");
+  if (!q || !seq_lens_dev || !out) return fail(BGTQ_ERR_INVALID, w + ": null pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  *plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  if (!workspace || workspace_bytes < plan->workspace_bytes)
+    return fail(BGTQ_ERR_WORKSPACE, w + ": workspace missing or smaller than bgtq_workspace_bytes()");
+  return BGTQ_OK;
+}
+
+bgtq_status decode_impl(const bgtq_layout* L, const char* who, const void* q, int q_dtype, int batch, int h_q,
+                        int h_kv, const CacheRef& c, const int* seq_lens_dev, long long max_seq_len,
+                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  DecodePlan plan;
+  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, c.n_tiles * kTile, max_seq_len, softmax_scale,
+                                    q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
+  if (st != BGTQ_OK) return st;
+  cudaError_t e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, softmax_scale, out,
+                                workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return BGTQ_OK;
+}
+
+bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, const void* v_new, int kv_dtype,
+                      int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, const CacheRef& c,
+                      const int* seq_lens_dev, long long max_seq_len, float softmax_scale, float* out,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(kv_dtype)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad dtype");
+  if (n_new < 0 || (long long)n_new * kEncodeParts * batch * h_kv + (long long)batch * h_kv > 0x7fffffffLL)
+    return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad n_new");
+  if (n_new > 0 && (!k_new || !v_new)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
+  DecodePlan plan;
+  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, c.n_tiles * kTile, max_seq_len, softmax_scale,
+                                    q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
+  if (st != BGTQ_OK) return st;
+  cudaError_t e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch,
+                                     h_q, h_kv, c, softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return BGTQ_OK;
+}
+
+bgtq_status contiguous(const char* who, void* cache, long long capacity, CacheRef* c) {
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, std::string(who) + ": capacity must be a positive multiple of 64");
+  if (!cache) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
+  *c = CacheRef{static_cast<uint8_t*>(cache), nullptr, capacity / kTile, 0};
+  return BGTQ_OK;
+}
+
+bgtq_status paged(const char* who, void* pool, long long num_pages, const int* block_table, long long max_pages,
+                  CacheRef* c) {
+  if (num_pages <= 0 || max_pages <= 0)
+    return fail(BGTQ_ERR_CAPACITY, std::string(who) + ": num_pages and max_pages must be positive");
+  if (!pool || !block_table) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
+  *c = CacheRef{static_cast<uint8_t*>(pool), block_table, max_pages, num_pages};
+  return BGTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 bgtq_status bgtq_encode_append(const bgtq_layout* L, const void* k, const void* v, int dtype, int batch,
                                int n_new, int h_kv, const int* seq_lens_dev, void* cache, long long capacity,
                                void* stream) {
   bgtq_status st = check_device(L, "encode_append");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("encode_append", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
-  if (!valid_dtype(dtype)) return fail(BGTQ_ERR_INVALID, "encode_append: bad dtype");
-  if (batch <= 0 || batch > 65535 || h_kv <= 0 || h_kv > 65535 || n_new < 0)
-    return fail(BGTQ_ERR_INVALID, "encode_append: bad batch / h_kv / n_new");
-  if (capacity <= 0 || capacity % kTile)
-    return fail(BGTQ_ERR_CAPACITY, "encode_append: capacity must be a positive multiple of 64");
-  if (n_new == 0) return BGTQ_OK;
-  if (!k || !v || !seq_lens_dev || !cache) return fail(BGTQ_ERR_INVALID, "encode_append: null pointer");
-  cudaError_t e = launch_tq_encode(L->dev, k, v, dtype, batch, n_new, h_kv, seq_lens_dev, cache,
-                                   capacity / kTile, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "encode_append");
-  return BGTQ_OK;
+  return encode_impl(L, "encode_append", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
 }
 
 size_t bgtq_workspace_bytes(const bgtq_layout* L, int batch, int h_q, int h_kv, long long max_seq_len) {
@@ -240,28 +327,11 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dty
                                   long long max_seq_len, float softmax_scale, float* out, void* workspace,
                                   size_t workspace_bytes, void* stream) {
   bgtq_status st = check_device(L, "decode_attention");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("decode_attention", const_cast<void*>(cache), capacity, &c);
   if (st != BGTQ_OK) return st;
-  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_attention: bad dtype");
-  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
-    return fail(BGTQ_ERR_INVALID, "decode_attention: need h_q = G * h_kv with G in 1..8");
-  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_attention: batch * h_kv > 65535");
-  if (capacity <= 0 || capacity % kTile)
-    return fail(BGTQ_ERR_CAPACITY, "decode_attention: capacity must be a positive multiple of 64");
-  if (max_seq_len < 0 || max_seq_len > capacity)
-    return fail(BGTQ_ERR_CAPACITY, "decode_attention: max_seq_len must be in [0, capacity]");
-  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_attention: bad softmax_scale");
-  if (!q || !cache || !seq_lens_dev || !out) return fail(BGTQ_ERR_INVALID, "decode_attention: null pointer");
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "decode_attention");
-  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
-  if (!workspace || workspace_bytes < plan.workspace_bytes)
-    return fail(BGTQ_ERR_WORKSPACE, "decode_attention: workspace missing or smaller than bgtq_workspace_bytes()");
-  e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, cache, seq_lens_dev, capacity / kTile,
-                    softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode_attention");
-  return BGTQ_OK;
+  return decode_impl(L, "decode_attention", q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, max_seq_len,
+                     softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
 bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype, int n_new,
@@ -270,31 +340,56 @@ bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void
                              float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                              void* stream) {
   bgtq_status st = check_device(L, "decode_step");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("decode_step", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
-  if (!valid_dtype(kv_dtype) || !valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_step: bad dtype");
-  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
-    return fail(BGTQ_ERR_INVALID, "decode_step: need h_q = G * h_kv with G in 1..8");
-  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_step: batch * h_kv > 65535");
-  if (n_new < 0 || (long long)n_new * kEncodeParts * batch * h_kv + (long long)batch * h_kv > 0x7fffffffLL)
-    return fail(BGTQ_ERR_INVALID, "decode_step: bad n_new");
-  if (capacity <= 0 || capacity % kTile)
-    return fail(BGTQ_ERR_CAPACITY, "decode_step: capacity must be a positive multiple of 64");
-  if (max_seq_len < 0 || max_seq_len > capacity)
-    return fail(BGTQ_ERR_CAPACITY, "decode_step: max_seq_len must be in [0, capacity]");
-  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_step: bad softmax_scale");
-  if (!q || !cache || !seq_lens_dev || !out || (n_new > 0 && (!k_new || !v_new)))
-    return fail(BGTQ_ERR_INVALID, "decode_step: null pointer");
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "decode_step");
-  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
-  if (!workspace || workspace_bytes < plan.workspace_bytes)
-    return fail(BGTQ_ERR_WORKSPACE, "decode_step: workspace missing or smaller than bgtq_workspace_bytes()");
-  e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch, h_q, h_kv,
-                         cache, capacity / kTile, softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode_step");
-  return BGTQ_OK;
+  return step_impl(L, "decode_step", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev,
+                   max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+long long bgtq_paged_pool_bytes(const bgtq_layout* L, int h_kv, long long num_pages) {
+  if (!L || h_kv <= 0 || num_pages < 0) {
+    set_error("paged_pool_bytes: bad arguments");
+    return -1;
+  }
+  return num_pages * h_kv * (long long)L->tile_bytes;
+}
+
+bgtq_status bgtq_encode_append_paged(const bgtq_layout* L, const void* k, const void* v, int dtype, int batch,
+                                     int n_new, int h_kv, const int* seq_lens_dev, void* pool, long long num_pages,
+                                     const int* block_table_dev, long long max_pages, void* stream) {
+  bgtq_status st = check_device(L, "encode_append_paged");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = paged("encode_append_paged", pool, num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return encode_impl(L, "encode_append_paged", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
+}
+
+bgtq_status bgtq_decode_attention_paged(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q,
+                                        int h_kv, const void* pool, long long num_pages, const int* block_table_dev,
+                                        long long max_pages, const int* seq_lens_dev, long long max_seq_len,
+                                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  bgtq_status st = check_device(L, "decode_attention_paged");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = paged("decode_attention_paged", const_cast<void*>(pool), num_pages, block_table_dev,
+                                max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(L, "decode_attention_paged", q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, max_seq_len,
+                     softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+bgtq_status bgtq_decode_step_paged(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype,
+                                   int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, void* pool,
+                                   long long num_pages, const int* block_table_dev, long long max_pages,
+                                   const int* seq_lens_dev, long long max_seq_len, float softmax_scale, float* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_device(L, "decode_step_paged");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = paged("decode_step_paged", pool, num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return step_impl(L, "decode_step_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, c,
+                   seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
 bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q, int h_kv,
@@ -321,8 +416,9 @@ bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype,
   const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
   if (!workspace || workspace_bytes < plan.workspace_bytes)
     return fail(BGTQ_ERR_WORKSPACE, "decode_scores: workspace missing or smaller than bgtq_workspace_bytes()");
-  e = launch_scores(L->dev, plan, q, q_dtype, batch, h_q, h_kv, cache, seq_lens_dev, capacity / kTile, softmax_scale,
-                    scores, scores_ld, workspace, static_cast<cudaStream_t>(stream));
+  const CacheRef c{static_cast<uint8_t*>(const_cast<void*>(cache)), nullptr, capacity / kTile, 0};
+  e = launch_scores(L->dev, plan, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, softmax_scale, scores, scores_ld,
+                    workspace, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_scores");
   return BGTQ_OK;
 }

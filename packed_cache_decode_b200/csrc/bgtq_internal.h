@@ -59,6 +59,37 @@ struct DevLayout {
   unsigned short vc[16];
 };
 
+// Where the packed tiles of a call live. Contiguous: [batch][h_kv][n_tiles][tile].
+// Paged: a pool of num_pages pages, page p = [h_kv][tile] (one 64-token span of one row),
+// and table[b * n_tiles + i] = the page of tile i of row b.
+struct CacheRef {
+  uint8_t* base;
+  const int* table;      // paged: [batch][n_tiles] page ids; nullptr: contiguous
+  long long n_tiles;     // tiles a row can hold (contiguous: capacity / 64; paged: table width)
+  long long num_pages;   // paged: pages in the pool
+};
+
+#ifdef __CUDACC__
+// Tile i of row b, KV head h. A page id outside the pool sets BGTQ_STATUS_BAD_PAGE and
+// gives nullptr (the caller skips the tile).
+__device__ __forceinline__ uint8_t* tile_ptr(const CacheRef& c, const DevLayout& L, int b, int h, int h_kv,
+                                             long long i) {
+  if (!c.table) return c.base + (((size_t)b * h_kv + h) * c.n_tiles + i) * (size_t)L.tile_bytes;
+  const long long p = c.table[(size_t)b * c.n_tiles + i];
+  if (p < 0 || p >= c.num_pages) {
+    atomicOr(L.status, BGTQ_STATUS_BAD_PAGE);
+    return nullptr;
+  }
+  return c.base + ((size_t)p * h_kv + h) * (size_t)L.tile_bytes;
+}
+// Whether tile i of row b has a page in the pool (contiguous caches: always).
+__device__ __forceinline__ bool tile_present(const CacheRef& c, int b, long long i) {
+  if (!c.table) return true;
+  const long long p = c.table[(size_t)b * c.n_tiles + i];
+  return p >= 0 && p < c.num_pages;
+}
+#endif
+
 }  // namespace bgtq
 
 struct bgtq_layout {

@@ -122,10 +122,9 @@ inline size_t qfrag_bytes(long long units) { return align256(size_t(units) * kMa
 
 // ------------------------------------------------------------------ split kernel
 struct SplitArgs {
-  const uint8_t* cache;
+  CacheRef cache;
   const int* seq_lens;
   const unsigned* qfrag;  // [units][kMaxQuads][2][32] q' B fragments from the preparation kernel
-  long long n_tiles;      // tiles per unit in the cache (capacity / 64)
   int max_tiles;          // M: tiles per unit covered by the plan
   int n_ctas;             // CTAs; CTA c takes tiles [c T / n_ctas, (c+1) T / n_ctas) of the sequence
   int n_parts;            // partial slots per unit
@@ -351,7 +350,7 @@ __device__ __forceinline__ int cta_segments(const DevLayout& L, const SplitArgs&
     const int b = u / a.h_kv;
     long long len = (long long)a.seq_lens[b] + a.len_add;
     if (len < 0) len = 0;
-    const long long cap_tokens = min(a.n_tiles, M) * kTile;
+    const long long cap_tokens = min(a.cache.n_tiles, M) * kTile;
     const long long a0 = max(g0, (long long)u * M) - (long long)u * M;
     const long long a1 = min(g1, (long long)(u + 1) * M) - (long long)u * M;
     if (len > cap_tokens) {
@@ -460,9 +459,8 @@ __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const 
 // token and KV head), the others prepare q' of one unit each.
 __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
                                                                  const void* __restrict__ v, int kv_dtype, int n_new,
-                                                                 int batch, long long n_tiles,
-                                                                 const int* __restrict__ seq_lens_before,
-                                                                 uint8_t* __restrict__ cache,
+                                                                 int batch, const int* __restrict__ seq_lens_before,
+                                                                 CacheRef cache,
                                                                  const void* __restrict__ q, int q_dtype, int h_q,
                                                                  int h_kv, int G, float qscale,
                                                                  unsigned* __restrict__ qfrag, int n_enc) {
@@ -474,7 +472,7 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
     const int t = rest % n_new;
     rest /= n_new;
     const int b = rest % batch, h = rest / batch;
-    enc::encode_token_part(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, n_tiles, t, part, b, h);
+    enc::encode_token_part(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
   } else {
     const int u = e - n_enc;
     prep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
@@ -567,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
   bool waited = !a.wait_new;
   for (int si = 0; si < nseg; ++si) {
     const Segment S = s_seg[si];
-    const uint8_t* src = a.cache + (size_t)S.u * a.n_tiles * TB;
+    const int srow = S.u / a.h_kv, shead = S.u % a.h_kv;
     const long long first_new = waited ? 0 : a.seq_lens[S.u / a.h_kv];
     const int mine = S.n > warp ? (S.n - warp + kWarps - 1) / kWarps : 0;  // tiles of this warp
     auto issue = [&](int k) {  // lane 0 only
@@ -577,8 +575,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         waited = true;
       }
       const int st = warp + kWarps * (k & 1);
-      mbar_expect_tx(&full[st], TB);
-      bulk_load(ring + st * TB, src + (size_t)it * TB, TB, &full[st], l2_stream);
+      const uint8_t* src = tile_ptr(a.cache, L, srow, shead, a.h_kv, it);
+      if (src) {
+        mbar_expect_tx(&full[st], TB);
+        bulk_load(ring + st * TB, src, TB, &full[st], l2_stream);
+      } else {
+        mbar_expect_tx(&full[st], 0);  // a page outside the pool (flagged): the stage keeps old bytes
+      }
     };
     if (lane == 0)
       for (int k = 0; k < min(2, mine); ++k) issue(k);
@@ -614,6 +617,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       }
       const unsigned char* tb = ring + st * TB;
       const long long gt0 = (long long)(S.lt0 + i) * kTile + g;  // token of row g in row block 0
+      // a paged tile without a page (flagged by the copy) is left out
+      const bool present = tile_present(a.cache, S.u / a.h_kv, S.lt0 + i);
+      if (present) {
 
       // ---------------- scores: per key group (rate as a template parameter), per quad,
       // four row blocks; then times the group norms
@@ -727,6 +733,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
                    vl.field(4 * mt + 2, T.v, lane4), vl.field(4 * mt + 3, T.v, lane4), pb[rt][0], pb[rt][1]);
       }
       }  // not scores-only
+      }  // present
       __syncwarp();  // every lane is done with the stage before it is refilled
       if (k + 2 < mine) {
         if (lane == 0) issue(k + 2);
@@ -922,7 +929,7 @@ int split_occupancy(const DevLayout& L) {
 // Split and combine kernels of one call, launched as programmatic dependents of the
 // kernel that wrote the q' fragments (and, after an append, the new tokens).
 cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int batch, int h_q, int h_kv,
-                             const void* cache, const int* seq_lens, long long n_tiles, float* out, void* workspace,
+                             const CacheRef& cache, const int* seq_lens, float* out, void* workspace,
                              int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
                              long long scores_ld = 0) {
   const int G = h_q / h_kv;
@@ -954,9 +961,8 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   if (plan.n_parts > wplan.n_parts || plan.workspace_bytes > wplan.workspace_bytes) return cudaErrorInvalidValue;
   const long long units = (long long)batch * h_kv;
   SplitArgs a;
-  a.cache = static_cast<const uint8_t*>(cache);
+  a.cache = cache;
   a.seq_lens = seq_lens;
-  a.n_tiles = n_tiles;
   a.max_tiles = plan.max_tiles;
   a.n_ctas = plan.n_ctas;
   a.n_parts = plan.n_parts;
@@ -1028,40 +1034,40 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
 }
 
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                          int h_q, int h_kv, const void* cache, const int* seq_lens, long long n_tiles,
-                          float softmax_scale, float* out, void* workspace, cudaStream_t stream) {
+                          int h_q, int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale,
+                          float* out, void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
   qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
       L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, n_tiles, out, workspace, 0, false, stream);
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, out, workspace, 0, false, stream);
 }
 
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
-                          int h_kv, const void* cache, const int* seq_lens, long long n_tiles, float softmax_scale,
-                          float* scores, long long scores_ld, void* workspace, cudaStream_t stream) {
+                          int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale, float* scores,
+                          long long scores_ld, void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
   qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
       L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, n_tiles, nullptr, workspace, 0, false, stream,
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, nullptr, workspace, 0, false, stream,
                           scores, scores_ld);
 }
 
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
-                               int batch, int h_q, int h_kv, void* cache, long long n_tiles, float softmax_scale,
-                               float* out, void* workspace, cudaStream_t stream) {
+                               int batch, int h_q, int h_kv, const CacheRef& cache, float softmax_scale, float* out,
+                               void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
   const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
   step_prep_kernel<<<unsigned(n_enc + batch * h_kv), kPrepThreads, 0, stream>>>(
-      L, k_new, v_new, kv_dtype, n_new, batch, n_tiles, seq_lens_before, static_cast<uint8_t*>(cache), q, q_dtype,
+      L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype,
       h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens_before, n_tiles, out, workspace, n_new,
+  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens_before, out, workspace, n_new,
                           n_new > 0, stream);
 }
 

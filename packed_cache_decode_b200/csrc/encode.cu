@@ -12,23 +12,20 @@ namespace {
 __global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayout L, const void* __restrict__ k,
                                                                         const void* __restrict__ v, int dtype,
                                                                         int n_new, int h_kv,
-                                                                        const int* __restrict__ seq_lens,
-                                                                        uint8_t* __restrict__ cache, long long n_tiles) {
+                                                                        const int* __restrict__ seq_lens, CacheRef cache) {
   // a split kernel launched as this kernel's programmatic dependent may start streaming
   // the tiles that do not receive the new tokens (it waits before the one that does)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  enc::encode_token_part(L, k, v, dtype, n_new, h_kv, seq_lens, cache, n_tiles, blockIdx.x / kEncodeParts,
+  enc::encode_token_part(L, k, v, dtype, n_new, h_kv, seq_lens, cache, blockIdx.x / kEncodeParts,
                          blockIdx.x % kEncodeParts, blockIdx.y, blockIdx.z);
 }
 
 }  // namespace
 
 cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, int dtype, int batch,
-                             int n_new, int h_kv, const int* seq_lens, void* cache, long long n_tiles,
-                             cudaStream_t stream) {
+                             int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream) {
   dim3 grid(n_new * kEncodeParts, batch, h_kv);
-  tq_encode_kernel<<<grid, enc::kEncodeThreads, 0, stream>>>(L, k, v, dtype, n_new, h_kv, seq_lens,
-                                                             static_cast<uint8_t*>(cache), n_tiles);
+  tq_encode_kernel<<<grid, enc::kEncodeThreads, 0, stream>>>(L, k, v, dtype, n_new, h_kv, seq_lens, cache);
   return cudaGetLastError();
 }
 

@@ -117,11 +117,11 @@ constexpr int kEncodeThreads = 256;
 // `part` (0..3).
 __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void* __restrict__ k,
                                                   const void* __restrict__ v, int dtype, int n_new, int h_kv,
-                                                  const int* __restrict__ seq_lens, uint8_t* __restrict__ cache,
-                                                  long long n_tiles, int t, int part, int b, int h) {
+                                                  const int* __restrict__ seq_lens, const CacheRef& cache, int t,
+                                                  int part, int b, int h) {
   const int tid = threadIdx.x;
   const long long pos = (long long)seq_lens[b] + t;
-  if (pos < 0 || pos >= n_tiles * kTile) {
+  if (pos < 0 || pos >= cache.n_tiles * kTile) {
     if (tid == 0 && part == 0) atomicOr(L.status, BGTQ_STATUS_ENCODE_OVERFLOW);
     return;
   }
@@ -181,7 +181,8 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
 
   const long long tile = pos / kTile;
   const int tt = int(pos % kTile);
-  uint8_t* tp = cache + (((size_t)b * h_kv + h) * n_tiles + tile) * (size_t)L.tile_bytes;
+  uint8_t* tp = tile_ptr(cache, L, b, h, h_kv, tile);
+  if (!tp) return;
   if (is_key) {
     put_key_code(L, tp, g, i, tt, unsigned(code));
     if (part == 0 && p < L.n_kgroups)
