@@ -5,29 +5,31 @@
 //   q . k_hat   = sum_g (|k_g| / sqrt(d_g)) (R_g q_g) . c[codes_g]
 //   o           = R_V^T sum_t p_t (|v_t| / sqrt(128)) c[vcodes_t] / sum_t p_t.
 //
-// Two kernels per call:
+// Three kernels per call, chained by programmatic dependent launch:
+//  * qprep_kernel (one CTA per batch row x KV head; in a decode step, step_prep_kernel also
+//    runs the encode CTAs of the new tokens): q' = R_g q_g for the G query heads (fp32,
+//    scaled by softmax_scale * log2(e) / (sqrt(d_g) kappa_g)), split into fp16 hi + lo
+//    parts and laid out as mma B fragments.
 //  * split_kernel: the (batch row, KV head) caches are laid end to end as one sequence of
 //    64-token tiles and every CTA takes an equal slice of it (one or two units' worth), so
-//    the grid is one balanced wave. 4 consumer warps + 1 producer warp. The producer lane
-//    streams the slice's tiles with 1-D bulk async copies (cp.async.bulk + mbarrier, no
-//    multicast) through a ring of up to 8 stages. Meanwhile the consumers compute
-//    q' = R_g q_g for the unit(s) of the slice (fp32, scaled by softmax_scale * log2(e) /
-//    sqrt(d_g)), split it into fp16 hi + lo parts and lay it out as B fragments.
-//    Consumer warp w takes tiles w, w+4, ... of a unit whole, as four 16-token row blocks.
-//    Keys: per quad of 4 dimension pairs, one load gives the lane its codes of the quad for
-//    its 8 tokens (fragment-major format); rate 1 turns into +-1 pairs with bit operations,
-//    rates 2-4 index pair tables in shared memory (lane-private for rate 2, hi + lo parts for
-//    rates 3-4); mma.m16n8k8 multiplies them with q' (for G <= 4 the hi and lo parts are the
-//    eight columns of one product). fp32 accumulators per group, then times the group norm.
-//    Online softmax in base 2 with warp shuffles. Values: the probabilities times
-//    |v|/sqrt(128) in fp16, transposed with movmatrix, against value-code pair lookups in
-//    m16n8k16 products, accumulated in V's rotated space (fp32). Per unit the four warps
-//    merge and the CTA writes its partial (o', m, l).
+//    the grid is one balanced wave. 4 warps, no producer warp: warp w streams its own tiles
+//    w, w+4, ... through a private pair of ring stages with 1-D bulk async copies
+//    (cp.async.bulk + mbarrier, L2 evict-first, no multicast), contiguous or paged. The
+//    CTA starts (tables, first copies) while q-prep runs and waits only before loading
+//    the q' fragments. Keys: per quad of 4 dimension pairs one load gives the lane its
+//    codes for its 8 tokens (fragment-major format); rate 1 turns into +-1 pairs with bit
+//    operations, rates 2-4 index pair tables in shared memory (lane-private for rate 2, hi
+//    + lo parts for rates 3-4); a group's quads go in pairs into mma.m16n8k16 (for G <= 4
+//    the q' hi and lo parts are the eight columns of one product). fp32 accumulators per
+//    group, then times the group norm. Online softmax in base 2 with warp shuffles.
+//    Values: the probabilities times |v|/sqrt(128) in fp16, transposed with movmatrix,
+//    against value-code pair lookups in m16n8k16 products, accumulated in V's rotated
+//    space (fp32). Per unit the four warps merge and the CTA writes its partial (o', m, l).
+//    A scores-only form writes the logits instead.
 //  * combine_kernel (one CTA per batch row x query head, 512 threads): log-sum-exp merge of
-//    the unit's partials and o = R_V^T o'; chained to split_kernel by programmatic dependent
-//    launch.
-// After an append (bgtq_decode_step) the split kernel is also launched as a dependent of the
-// encode kernel: only the tile that receives the new tokens waits for it.
+//    the unit's partials and o = R_V^T o'.
+// After an append (bgtq_decode_step) only the tile that receives the new tokens waits for
+// the encode before it is copied.
 //
 // Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, waits
 // (bounded) for its own copies in flight and returns.
