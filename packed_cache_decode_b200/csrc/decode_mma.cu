@@ -176,6 +176,12 @@ __device__ __forceinline__ uint2 lds_u64(const uint2* base, unsigned boff) {
 __device__ __forceinline__ unsigned shr(unsigned x, int s) { return s >= 0 ? x >> s : x << -s; }
 
 // Shared-memory tables of one CTA.
+// A compile-time int carried as a value (row blocks per work item).
+template <int N>
+struct IntC {
+  static constexpr int value = N;
+};
+
 template <int VR>
 struct Luts {
   static constexpr int kV = VR == 2 ? 16 * 32 : VR == 3 ? 64 * 32 : VR == 4 ? 256 : 1;
@@ -193,8 +199,9 @@ struct Kq;
 template <int VR>
 struct Kq<1, VR> {
   unsigned w;  // lo codes in bits 8-15, hi codes in bits 24-31
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
     w = prmt(*reinterpret_cast<const unsigned short*>(tb + (off & 0xffffu)), 0u, 0x1404u);
+    if (up) w >>= 4;
   }
   __device__ __forceinline__ unsigned a(int m, const Luts<VR>&, unsigned) const { return sign_pair(w << (7 - m)); }
   __device__ __forceinline__ unsigned lo(int, const Luts<VR>&) const { return 0u; }
@@ -202,8 +209,9 @@ struct Kq<1, VR> {
 template <int VR>
 struct Kq<2, VR> {
   unsigned w;  // nibble m = lo | hi << 2
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
     w = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
+    if (up) w >>= 16;
   }
   __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned lane4) const {
     return lds_u32(T.k2, (shr(w, 4 * m - 7) & 0x780u) | lane4);  // entry at 128 nibble + 4 lane
@@ -214,9 +222,10 @@ template <int VR>
 struct Kq<3, VR> {
   unsigned f[8];  // byte offsets (8 x field) of the eight 6-bit fields in the pair table
   uint2 e[8];
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
-    const unsigned wa = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
+    unsigned wa = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
     const unsigned wb = *reinterpret_cast<const unsigned short*>(tb + (off >> 16));
+    if (up) wa = (wa >> 24) | (wb << 8);  // fields 4..7 to 0..3 (only those are used then)
     f[0] = (wa << 3) & 0x1f8u;
     f[1] = (wa >> 3) & 0x1f8u;
     f[2] = (wa >> 9) & 0x1f8u;
@@ -233,8 +242,9 @@ template <int VR>
 struct Kq<4, VR> {
   uint2 w;  // byte m = lo | hi << 4
   uint2 e[8];
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off) {
+  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
     w = *reinterpret_cast<const uint2*>(tb + (off & 0xffffu));
+    if (up) w.x = w.y;
   }
   __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned) {
     const unsigned x = m < 4 ? w.x : w.y;
@@ -249,20 +259,22 @@ struct Kq<4, VR> {
 // group's odd last quad takes an m16n8k8 product. Row block rt of the tile: rows g and
 // g+8 are slots m = 2 rt and 2 rt + 1. loff[q][lane] = byte offset of the lane's codes in
 // the tile (for a lane without a pair of that quad: any code, its q' rows are zero).
-template <int R, bool NP, int VR>
-__device__ __forceinline__ void key_group(float (&acc)[4][4], const unsigned char* tb, const unsigned* loff,
-                                          const unsigned* qf, int q0, int q1, int lane, const Luts<VR>& T) {
+// NRT = 4: the whole tile; NRT = 2: the half tile of row blocks 0-1 (up = false) or 2-3.
+template <int R, bool NP, int VR, int NRT>
+__device__ __forceinline__ void key_group(float (&acc)[NRT][4], const unsigned char* tb, const unsigned* loff,
+                                          const unsigned* qf, int q0, int q1, int lane, const Luts<VR>& T,
+                                          bool up) {
   const unsigned lane4 = unsigned(lane) << 2;
   int q = q0;
 #pragma unroll 1
   for (; q + 1 < q1; q += 2) {
     Kq<R, VR> c0, c1;
-    c0.load(tb, loff[q * 32 + lane]);
-    c1.load(tb, loff[(q + 1) * 32 + lane]);
+    c0.load(tb, loff[q * 32 + lane], NRT < 4 && up);
+    c1.load(tb, loff[(q + 1) * 32 + lane], NRT < 4 && up);
     const unsigned bh0 = qf[q * 64 + lane], bh1 = qf[(q + 1) * 64 + lane];
     const unsigned bl0 = NP ? 0u : qf[q * 64 + 32 + lane], bl1 = NP ? 0u : qf[(q + 1) * 64 + 32 + lane];
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
+    for (int rt = 0; rt < NRT; ++rt) {
       const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
       const unsigned a2 = c1.a(2 * rt, T, lane4), a3 = c1.a(2 * rt + 1, T, lane4);
       mma16816(acc[rt], a0, a1, a2, a3, bh0, bh1);
@@ -273,10 +285,10 @@ __device__ __forceinline__ void key_group(float (&acc)[4][4], const unsigned cha
   }
   if (q < q1) {
     Kq<R, VR> c0;
-    c0.load(tb, loff[q * 32 + lane]);
+    c0.load(tb, loff[q * 32 + lane], NRT < 4 && up);
     const unsigned bh = qf[q * 64 + lane], bl = NP ? 0u : qf[q * 64 + 32 + lane];
 #pragma unroll
-    for (int rt = 0; rt < 4; ++rt) {
+    for (int rt = 0; rt < NRT; ++rt) {
       const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
       mma1688(acc[rt], a0, a1, bh);
       if constexpr (!NP) mma1688(acc[rt], a0, a1, bl);
@@ -569,9 +581,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
     const Segment S = s_seg[si];
     const int srow = S.u / a.h_kv, shead = S.u % a.h_kv;
     const long long first_new = waited ? 0 : a.seq_lens[S.u / a.h_kv];
-    const int mine = S.n > warp ? (S.n - warp + kWarps - 1) / kWarps : 0;  // tiles of this warp
+    // Work items of this warp: full tiles w, w+4, ... of the first 4 floor(n/4); of the
+    // n % 4 tiles left, one each for warps 0-2 if three are left, else half tiles (row
+    // blocks 0-1 or 2-3), so that no warp runs more than half a tile past the others.
+    // Both warps of a split tile copy all of it into their own stages.
+    const int nfw = S.n >> 2, rem = S.n & 3;
+    const bool extra = rem == 3 ? warp < 3 : rem == 2 ? true : rem == 1 ? warp < 2 : false;
+    const int mine = nfw + (extra ? 1 : 0);
+    auto item_tile = [&](int k) {
+      return (k < nfw || rem == 3) ? warp + kWarps * k : kWarps * nfw + (rem == 2 ? (warp >> 1) : 0);
+    };
     auto issue = [&](int k) {  // lane 0 only
-      const int it = S.lt0 + warp + kWarps * k;
+      const int it = S.lt0 + item_tile(k);
       if (!waited && (long long)(it + 1) * kTile > first_new) {
         pdl_wait();  // this tile receives tokens from the encode kernel
         waited = true;
@@ -602,50 +623,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       for (int j = 0; j < 4; ++j) O[mt][j] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    for (int k = 0; k < mine; ++k) {
-      const int st = warp + kWarps * (k & 1), i = warp + kWarps * k;
-      const bool ok = mbar_wait_bounded(&full[st], (phase >> (k & 1)) & 1u);
-      if (ok) {
-        phase ^= 1u << (k & 1);
-        pend &= ~(1u << (k & 1));
-      }
-      if (!ok) {
-        // stop consuming; this warp waits for its own copies below, no partial is written
-        if (lane == 0) {
-          atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
-          s_timeout = 1;
-        }
-        break;
-      }
-      const unsigned char* tb = ring + st * TB;
-      const long long gt0 = (long long)(S.lt0 + i) * kTile + g;  // token of row g in row block 0
-      // a paged tile without a page (flagged by the copy) is left out
-      const bool present = tile_present(a.cache, S.u / a.h_kv, S.lt0 + i);
-      if (present) {
+    // Row blocks rb0 .. rb0 + NRT - 1 of the tile in stage tb; gt0 = token of row g of
+    // row block rb0.
+    auto rows = [&](auto nrt, const unsigned char* tb, int rb0, long long gt0) {
+      constexpr int NRT = decltype(nrt)::value;
+      const bool up = rb0 != 0;
 
       // ---------------- scores: per key group (rate as a template parameter), per quad,
-      // four row blocks; then times the group norms
-      const float* kn = reinterpret_cast<const float*>(tb + L.knorm_off);
-      float sc[4][4];
+      // NRT row blocks; then times the group norms
+      const float* kn = reinterpret_cast<const float*>(tb + L.knorm_off) + 16 * rb0;
+      float sc[NRT][4];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt)
+      for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) sc[rt][j] = 0.f;
       for (int gi = 0; gi < ng; ++gi) {
-        float acc[4][4];
+        float acc[NRT][4];
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt)
+        for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[rt][j] = 0.f;
         const int q0 = s_group[gi][0], q1 = s_group[gi][1];
         switch (s_group[gi][2]) {
-          case 1: key_group<1, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
-          case 2: key_group<2, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
-          case 3: key_group<3, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
-          default: key_group<4, NP, VR>(acc, tb, s_loff, qf, q0, q1, lane, T); break;
+          case 1: key_group<1, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
+          case 2: key_group<2, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
+          case 3: key_group<3, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
+          default: key_group<4, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
         }
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
+        for (int rt = 0; rt < NRT; ++rt) {
           const float n0 = kn[gi * kTile + 16 * rt + g], n1 = kn[gi * kTile + 16 * rt + g + 8];
           sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
           sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
@@ -656,12 +662,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       if constexpr (NP) {
         // columns 4..7 carried the lo parts of q': add them to the hi parts (lanes t, t^2)
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt)
+        for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) sc[rt][j] += __shfl_xor_sync(0xffffffffu, sc[rt][j], 2);
       }
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
+      for (int rt = 0; rt < NRT; ++rt) {
         if (gt0 + 16 * rt >= S.len) sc[rt][0] = sc[rt][1] = -INFINITY;
         if (gt0 + 16 * rt + 8 >= S.len) sc[rt][2] = sc[rt][3] = -INFINITY;
       }
@@ -670,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         // column 2t + c holds head 2t + c (G <= 4: lanes t < 2; t >= 2 hold copies)
         const int b = S.u / a.h_kv, hkv = S.u % a.h_kv;
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt)
+        for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int head = 2 * t + (j & 1);
@@ -679,10 +685,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
               a.scores[((size_t)b * a.h_q + (size_t)hkv * a.G + head) * a.scores_ld + tok] = sc[rt][j] * (1.f / kLog2e);
           }
       } else {
-      // ---------------- online softmax over the 64 tokens (heads of columns 2t, 2t+1), base 2
+      // ---------------- online softmax over the rows (heads of columns 2t, 2t+1), base 2
       float x0 = -INFINITY, x1 = -INFINITY;
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
+      for (int rt = 0; rt < NRT; ++rt) {
         x0 = fmaxf(x0, fmaxf(sc[rt][0], sc[rt][2]));
         x1 = fmaxf(x1, fmaxf(sc[rt][1], sc[rt][3]));
       }
@@ -709,14 +715,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
           O[mt][3] *= corr1;
         }
       }
-      const float* vn = reinterpret_cast<const float*>(tb + L.vnorm_off);
+      const float* vn = reinterpret_cast<const float*>(tb + L.vnorm_off) + 16 * rb0;
 
-      // ---------------- values: row block rt is value chunk rt of the tile. First the
-      // probabilities (times |v| / sqrt(128)) as transposed fp16 B fragments, then the
-      // m16n8k16 products against the value codes
-      unsigned pb[4][2];
+      // ---------------- values: row block rb0 + rt is value chunk rb0 + rt of the tile.
+      // First the probabilities (times |v| / sqrt(128)) as transposed fp16 B fragments,
+      // then the m16n8k16 products against the value codes
+      unsigned pb[NRT][2];
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
+      for (int rt = 0; rt < NRT; ++rt) {
         const float p0 = fast_exp2(sc[rt][0] - b0m), p1 = fast_exp2(sc[rt][1] - b1m);
         const float p2 = fast_exp2(sc[rt][2] - b0m), p3 = fast_exp2(sc[rt][3] - b1m);
         l0 += p0 + p2;
@@ -726,16 +732,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         pb[rt][1] = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
       }
 #pragma unroll
-      for (int rt = 0; rt < 4; ++rt) {
+      for (int rt = 0; rt < NRT; ++rt) {
         ValueLane<VR> vl;
-        vl.load(tb + L.vcode_off + rt * 256 * VR, lane);
+        vl.load(tb + L.vcode_off + (rb0 + rt) * 256 * VR, lane);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
           mma16816(O[mt], vl.field(4 * mt, T.v, lane4), vl.field(4 * mt + 1, T.v, lane4),
                    vl.field(4 * mt + 2, T.v, lane4), vl.field(4 * mt + 3, T.v, lane4), pb[rt][0], pb[rt][1]);
       }
       }  // not scores-only
-      }  // present
+    };
+
+    for (int k = 0; k < mine; ++k) {
+      const int st = warp + kWarps * (k & 1), i = item_tile(k);
+      const bool ok = mbar_wait_bounded(&full[st], (phase >> (k & 1)) & 1u);
+      if (ok) {
+        phase ^= 1u << (k & 1);
+        pend &= ~(1u << (k & 1));
+      }
+      if (!ok) {
+        // stop consuming; this warp waits for its own copies below, no partial is written
+        if (lane == 0) {
+          atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
+          s_timeout = 1;
+        }
+        break;
+      }
+      const unsigned char* tb = ring + st * TB;
+      const long long gt0 = (long long)(S.lt0 + i) * kTile + g;  // token of row g in row block 0
+      // a paged tile without a page (flagged by the copy) is left out
+      if (tile_present(a.cache, S.u / a.h_kv, S.lt0 + i)) {
+        if (k == nfw && rem != 3) {
+          const int rb0 = 2 * (warp & 1);
+          rows(IntC<2>{}, tb, rb0, gt0 + 16 * rb0);
+        } else {
+          rows(IntC<4>{}, tb, 0, gt0);
+        }
+      }
       __syncwarp();  // every lane is done with the stage before it is refilled
       if (k + 2 < mine) {
         if (lane == 0) issue(k + 2);
