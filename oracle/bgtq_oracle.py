@@ -17,7 +17,9 @@ Sources (cited by page title and passage):
   diagram). Box "input vector x" (a per-head K or V vector); box "random rotation /
   Hadamard" (makes coordinates concentrated and near-independent); box "per-coordinate
   MSE scalar quantisation" (a few centroids approximate the rotated coordinates);
-  exercise box 1 (KV-cache memory for a batch/context/kv-head count).
+  exercise box 1 (KV-cache memory for a batch/context/kv-head count); vLLM column, box
+  "NC" (norm correction: corrects the distortion of the norm by the centroids; the
+  "_nc" presets).
 * [Philox] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3"
   (SC'11): the Philox4x32-10 counter-based generator.
 * [BoxMuller] Box and Muller (1958): two uniforms to two independent N(0,1) draws.
@@ -29,13 +31,18 @@ block j = coordinates {j, j+64} (rotate-half RoPE); groups ordered by descending
 blocks ascending, coordinate j before j+64; dense Haar rotation per group from a
 Philox-seeded Gaussian matrix (QR, positive triangular diagonal); y = sqrt(d) R x/|x|;
 code = number of thresholds <= y; one fp32 norm per (token, group); V coded as one
-128-dim TQ-MSE group at the V rate.
+128-dim TQ-MSE group at the V rate. Optional layout variants: norm correction (NC) stores
+|x| sqrt(d) / |c| instead of |x|, c the vector of the chosen centroids, so the decoded
+group vector has the norm of the input; fp16 norms (round to nearest, saturating at the
+largest finite fp16) halve the norm bytes.
 
 Parity pins (tests/test_oracle_pins.py): Philox known-answer vectors; Lloyd-Max closed
 form at 1 bit, the published per-coordinate MSE figures and Monte Carlo; greedy vs
 exhaustive search; rotation orthogonality / QR definition; encode-decode against the
 closed-form distortion; attention against the rotated-space identity and its special
-cases. No function here is "parity unpinned".
+cases; NC against the norm it must restore and the mean centroid energy 1 - D(b) of a
+Lloyd-Max quantiser; fp16 norms against hand-placed bytes. No function here is "parity
+unpinned".
 """
 from __future__ import annotations
 
@@ -45,6 +52,7 @@ from dataclasses import dataclass
 import numpy as np
 
 HEAD_DIM = 128
+FP16_MAX = 65504.0
 N_BLOCKS = 64
 TILE_TOKENS = 64
 CHUNK_TOKENS = 16
@@ -249,6 +257,12 @@ class Layout:
     k_rot: list                          # R_g, d_g x d_g
     v_rot: np.ndarray                    # 128 x 128
     codebooks: dict                      # rate -> (centroids, thresholds)
+    norm_correct: bool = False           # NC: stored norm |x| sqrt(d) / |c| [TQ, box "NC"]
+    norm_fp16: bool = False              # norms stored as fp16 instead of fp32
+
+    @property
+    def norm_bytes(self):
+        return 2 if self.norm_fp16 else 4
 
     @property
     def n_kgroups(self):
@@ -268,8 +282,8 @@ class Layout:
 
     @property
     def bytes_per_token(self):
-        """Resident bytes per (token, KV head): codes plus one fp32 norm per group."""
-        return self.k_record_bytes + self.v_record_bytes + 4 * (self.n_kgroups + 1)
+        """Resident bytes per (token, KV head): codes plus one norm (fp32, or fp16) per group."""
+        return self.k_record_bytes + self.v_record_bytes + self.norm_bytes * (self.n_kgroups + 1)
 
     @property
     def tile_bytes(self):
@@ -311,7 +325,7 @@ def group_coordinates(k_rates) -> list:
     return out
 
 
-def make_layout(k_rates, v_rate: int, seed: int) -> Layout:
+def make_layout(k_rates, v_rate: int, seed: int, norm_correct: bool = False, norm_fp16: bool = False) -> Layout:
     """K record = a whole number of bytes: the 64 block rates must sum to a multiple of 4."""
     if len(k_rates) != N_BLOCKS or (2 * int(np.sum(k_rates))) % 8 or not 1 <= v_rate <= 4:
         raise ValueError("64 block rates summing to a multiple of 4, and a V rate in 1..4")
@@ -322,13 +336,14 @@ def make_layout(k_rates, v_rate: int, seed: int) -> Layout:
     for r in set([r for r, _ in groups] + [v_rate]):
         c, t, _ = lloyd_max(r)
         books[r] = (c, t)
-    return Layout(np.asarray(k_rates, dtype=np.int64), int(v_rate), int(seed), groups, k_rot, v_rot, books)
+    return Layout(np.asarray(k_rates, dtype=np.int64), int(v_rate), int(seed), groups, k_rot, v_rot, books,
+                  bool(norm_correct), bool(norm_fp16))
 
 
 def cache_bytes(layout: Layout, batch: int, h_kv: int, tokens: int) -> int:
     """Resident bytes of a packed cache [TQ exercise box 1]: per (token, KV head)
-    128 b_K/8 + 128 b_V/8 code bytes plus 4 (n_gK + 1) norm bytes; capacity in whole
-    64-token tiles."""
+    128 b_K/8 + 128 b_V/8 code bytes plus 4 (n_gK + 1) norm bytes (2 (n_gK + 1) with
+    fp16 norms); capacity in whole 64-token tiles."""
     tiles = -(-tokens // TILE_TOKENS)
     return batch * h_kv * tiles * layout.tile_bytes
 
@@ -354,17 +369,33 @@ def _tq_encode_group(x: np.ndarray, rot: np.ndarray, thresholds: np.ndarray):
     return codes.astype(np.int64), norms, margin
 
 
+def _norm_correct(norms: np.ndarray, codes: np.ndarray, centroids: np.ndarray) -> np.ndarray:
+    """Norm correction [TQ, vLLM box "NC"]. The decoded group vector (s / sqrt(d)) R^T c
+    has norm s |c| / sqrt(d), and |c|^2 (the energy of the chosen centroids) is not d in
+    general: the centroids distort the norm. Storing s = |x| sqrt(d) / |c| gives the
+    decoded vector the norm |x| of the input. No Lloyd-Max centroid is 0, so |c| > 0."""
+    d = codes.shape[1]
+    cn = np.sqrt(np.sum(centroids[codes] ** 2, axis=1))
+    return norms * math.sqrt(d) / cn
+
+
 def encode(layout: Layout, k: np.ndarray, v: np.ndarray) -> dict:
-    """k, v [n, 128] (any float; promoted to fp64). Codes are in packed-dimension order."""
+    """k, v [n, 128] (any float; promoted to fp64). Codes are in packed-dimension order.
+    Norms are fp64 (rounded to the stored type by ``pack``); with NC they are the
+    corrected norms."""
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     kc, kn, km = [], [], []
     for (r, coords), rot in zip(layout.groups, layout.k_rot):
         c, nrm, m = _tq_encode_group(k[:, coords], rot, layout.codebooks[r][1])
+        if layout.norm_correct:
+            nrm = _norm_correct(nrm, c, layout.codebooks[r][0])
         kc.append(c)
         kn.append(nrm)
         km.append(m)
     vc, vn, vm = _tq_encode_group(v, layout.v_rot, layout.codebooks[layout.v_rate][1])
+    if layout.norm_correct:
+        vn = _norm_correct(vn, vc, layout.codebooks[layout.v_rate][0])
     return {
         "k_codes": np.concatenate(kc, axis=1), "k_norms": np.stack(kn, axis=1), "k_margin": np.concatenate(km, axis=1),
         "v_codes": vc, "v_norm": vn, "v_margin": vm,
@@ -403,8 +434,8 @@ def attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, scale: float)
 # ----------------------------------------------------------------------------------------
 # Packed tile format (the byte layout both sides implement)
 #
-# Tile of 64 tokens = [K area][V area][K norms fp32, group-major: [group][token]]
-# [V norms fp32 [token]]. Both code areas are "fragment-major": they are cut into per-lane
+# Tile of 64 tokens = [K area][V area][K norms, group-major: [group][token]]
+# [V norms [token]], norms fp32 (fp16 in a layout with fp16 norms). Both code areas are "fragment-major": they are cut into per-lane
 # bit strings, lane l = 4 g + t of a 32-lane warp, holding exactly the codes that lane
 # turns into its tensor-core operand registers, so a lane reads its codes with one or two
 # aligned loads and no two lanes share a word. Words are little-endian; bit b of a bit
@@ -550,19 +581,33 @@ def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
         out[:, base + 256 * br * c:base + 256 * br * (c + 1)] = np.packbits(blk, axis=1, bitorder="little")
     # norms
     base += TILE_TOKENS * vb
-    kn = np.zeros((ntile * TILE_TOKENS, ng), dtype=np.float32)
-    kn[:n] = enc["k_norms"].astype(np.float32)
+    nb, nt = layout.norm_bytes, norm_dtype(layout)
+    kn = np.zeros((ntile * TILE_TOKENS, ng), dtype=nt)
+    kn[:n] = stored_norms(layout, enc["k_norms"])
     kn = kn.reshape(ntile, TILE_TOKENS, ng).transpose(0, 2, 1).reshape(ntile, -1)
-    out[:, base:base + 4 * TILE_TOKENS * ng] = kn.view(np.uint8).reshape(ntile, -1)
-    base += 4 * TILE_TOKENS * ng
-    vn = np.zeros(ntile * TILE_TOKENS, dtype=np.float32)
-    vn[:n] = enc["v_norm"].astype(np.float32)
-    out[:, base:base + 4 * TILE_TOKENS] = vn.reshape(ntile, TILE_TOKENS).view(np.uint8)
+    out[:, base:base + nb * TILE_TOKENS * ng] = kn.view(np.uint8).reshape(ntile, -1)
+    base += nb * TILE_TOKENS * ng
+    vn = np.zeros(ntile * TILE_TOKENS, dtype=nt)
+    vn[:n] = stored_norms(layout, enc["v_norm"])
+    out[:, base:base + nb * TILE_TOKENS] = vn.reshape(ntile, TILE_TOKENS).view(np.uint8)
     return out.reshape(-1)
 
 
+def norm_dtype(layout: Layout):
+    return np.float16 if layout.norm_fp16 else np.float32
+
+
+def stored_norms(layout: Layout, norms) -> np.ndarray:
+    """fp64 norms rounded to the layout's norm type (round to nearest even); fp16 norms
+    above the largest finite fp16 are stored as that value, not as infinity."""
+    x = np.asarray(norms, dtype=np.float64)
+    if layout.norm_fp16:
+        return np.minimum(x, FP16_MAX).astype(np.float16)
+    return x.astype(np.float32)
+
+
 def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
-    """Inverse of ``pack`` for tokens 0..n-1 (codes, fp32 norms promoted to fp64)."""
+    """Inverse of ``pack`` for tokens 0..n-1 (codes, stored norms promoted to fp64)."""
     ntile = len(buf) // layout.tile_bytes
     t = np.asarray(buf, dtype=np.uint8).reshape(ntile, layout.tile_bytes)
     kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
@@ -592,10 +637,11 @@ def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
             vc[:, c, lot, dims] = lo
             vc[:, c, hit, dims] = hi
     base += TILE_TOKENS * vb
-    kn = t[:, base:base + 4 * TILE_TOKENS * ng].copy().view(np.float32).reshape(ntile, ng, TILE_TOKENS)
+    nb, nt = layout.norm_bytes, norm_dtype(layout)
+    kn = t[:, base:base + nb * TILE_TOKENS * ng].copy().view(nt).reshape(ntile, ng, TILE_TOKENS)
     kn = kn.transpose(0, 2, 1).reshape(-1, ng)
-    base += 4 * TILE_TOKENS * ng
-    vn = t[:, base:base + 4 * TILE_TOKENS].copy().view(np.float32).reshape(-1)
+    base += nb * TILE_TOKENS * ng
+    vn = t[:, base:base + nb * TILE_TOKENS].copy().view(nt).reshape(-1)
     return {"k_codes": kc[:n], "k_norms": kn[:n].astype(np.float64),
             "v_codes": vc.reshape(-1, HEAD_DIM)[:n], "v_norm": vn[:n].astype(np.float64)}
 
@@ -632,6 +678,6 @@ def logit_mae(layout: Layout, q: np.ndarray, k: np.ndarray, scale: float) -> flo
     where k_hat is the TQ-MSE reconstruction of the keys k [n, 128] (values unused)."""
     k = np.asarray(k, dtype=np.float64)
     enc = encode(layout, k, np.zeros_like(k))
-    kh, _ = reconstruct(layout, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+    kh, _ = reconstruct(layout, enc["k_codes"], stored_norms(layout, enc["k_norms"]), enc["v_codes"], enc["v_norm"])
     q = np.asarray(q, dtype=np.float64)
     return float(np.mean(np.abs((q @ kh.T - q @ k.T) * scale)))

@@ -450,3 +450,77 @@ def test_block_allocation_beats_uniform_rates_on_skewed_blocks():
     gtq = O.logit_mae(O.make_layout(rates, 2, 3), q, k, 1 / math.sqrt(128))
     uni = O.logit_mae(O.make_layout(np.full(64, 2), 2, 3), q, k, 1 / math.sqrt(128))
     assert gtq < 0.8 * uni, (gtq, uni)
+
+
+# ---------------------------------------------------------------- layout variants ----
+def test_norm_correction_restores_the_input_norm():
+    """NC ("TurboQuant" page, vLLM box "NC"): the decoded group vectors have the norms of the
+    inputs, for every group and for V; the codes are those of the plain layout."""
+    rates = np.array([3] * 16 + [2] * 24 + [1] * 24)
+    plain = O.make_layout(rates, 2, 11)
+    nc = O.make_layout(rates, 2, 11, norm_correct=True)
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal((40, 128)) * rng.uniform(0.1, 10, 128)
+    v = rng.standard_normal((40, 128))
+    k[3] = 0.0                                   # a zero vector keeps a zero norm
+    e0, e1 = O.encode(plain, k, v), O.encode(nc, k, v)
+    np.testing.assert_array_equal(e0["k_codes"], e1["k_codes"])
+    np.testing.assert_array_equal(e0["v_codes"], e1["v_codes"])
+    kh, vh = O.reconstruct(nc, e1["k_codes"], e1["k_norms"], e1["v_codes"], e1["v_norm"])
+    for r, coords in nc.groups:
+        np.testing.assert_allclose(np.linalg.norm(kh[:, coords], axis=1), np.linalg.norm(k[:, coords], axis=1),
+                                   rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(np.linalg.norm(vh, axis=1), np.linalg.norm(v, axis=1), rtol=1e-12)
+    # without NC the decoded norms are off by the centroid energy (the distortion NC removes)
+    kh0, _ = O.reconstruct(plain, e0["k_codes"], e0["k_norms"], e0["v_codes"], e0["v_norm"])
+    r1 = nc.groups[-1][1]
+    assert np.max(np.abs(np.linalg.norm(kh0[:, r1], axis=1) / np.maximum(np.linalg.norm(k[:, r1], axis=1), 1e-300)
+                         - 1)[np.linalg.norm(k[:, r1], axis=1) > 0]) > 1e-3
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_norm_correction_factor_matches_the_centroid_energy(bits):
+    """Centroid condition of a Lloyd-Max quantiser: E[Q(y)^2] = E[y^2] - D(b) = 1 - D(b) for
+    y ~ N(0,1). NC stores |x| sqrt(d) / |c|, so the mean of (|x| / stored)^2 = |c|^2 / d
+    over many vectors approaches 1 - D(b) (a rotated unit vector times sqrt(d) has
+    near-Gaussian coordinates; the sphere's correction is O(1/d))."""
+    lay = O.make_layout(np.full(64, bits), bits, 3, norm_correct=True)
+    rng = np.random.default_rng(bits)
+    x = rng.standard_normal((3000, 128))
+    enc = O.encode(lay, x, x)
+    ratio2 = (np.linalg.norm(x, axis=1) / enc["v_norm"]) ** 2
+    d_b = O.lloyd_max_mse_table()[bits]
+    assert abs(ratio2.mean() - (1 - d_b)) < 0.01 * (1 - d_b)
+    kr = (np.linalg.norm(x, axis=1) / enc["k_norms"][:, 0]) ** 2
+    assert abs(kr.mean() - (1 - d_b)) < 0.01 * (1 - d_b)
+
+
+def test_fp16_norms_are_where_the_format_says():
+    """One rate-2 group and V2: K area 64 x 32 bytes, V area 64 x 32, then the K norms fp16
+    [1 group][64 tokens] at 4096 and the V norms fp16 [64] at 4224; 68 bytes per token.
+    fp16 of 3.0 is 0x4200, of 1.5 0x3e00; 1e6 saturates at 65504 (0x7bff); 0.1 rounds to
+    nearest (0x2e66)."""
+    lay = O.make_layout(np.full(64, 2), 2, 0, norm_fp16=True)
+    assert lay.bytes_per_token == 32 + 32 + 2 * 2 and lay.tile_bytes == 64 * 68
+    n = 4
+    enc = {"k_codes": np.zeros((n, 128), dtype=np.int64), "v_codes": np.zeros((n, 128), dtype=np.int64),
+           "k_norms": np.array([[3.0], [1e6], [0.1], [0.0]]), "v_norm": np.array([0.0, 1.5, 0.0, 65519.0])}
+    buf = O.pack(lay, enc, 64)
+    assert buf.size == 64 * 68
+    assert buf[4096:4104].tolist() == [0x00, 0x42, 0xff, 0x7b, 0x66, 0x2e, 0, 0]
+    assert buf[4224:4232].tolist() == [0, 0, 0x00, 0x3e, 0, 0, 0xff, 0x7b]
+    assert int(np.count_nonzero(buf)) == (1 + 2 + 2) + (1 + 2)   # nonzero bytes of the norms; codes are 0
+    u = O.unpack(lay, buf, n)
+    assert u["k_norms"][:, 0].tolist() == [3.0, 65504.0, float(np.float16(0.1)), 0.0]
+    assert u["v_norm"].tolist() == [0.0, 1.5, 0.0, 65504.0]
+
+
+def test_resident_bytes_with_fp16_norms():
+    """Bytes per (token, KV head) = 128 b_K / 8 + 128 b_V / 8 + 2 (n_gK + 1) with fp16
+    norms: K3V3 in one group 48 + 48 + 4 = 100 (5.12x smaller than a 512-byte fp16 K+V
+    record); K2V2 over rates 1-4 (four groups) 32 + 32 + 10 = 74 (6.92x)."""
+    k3 = O.make_layout(np.full(64, 3), 3, 0, norm_fp16=True)
+    assert k3.bytes_per_token == 100 and O.cache_bytes(k3, 2, 4, 65) == 2 * 4 * 2 * 64 * 100
+    mixed = O.make_layout(np.array([4] * 8 + [3] * 8 + [2] * 24 + [1] * 24), 2, 0, norm_fp16=True)
+    assert mixed.n_kgroups == 4 and mixed.k_record_bytes == 32 and mixed.bytes_per_token == 74
+    assert O.make_layout(np.full(64, 3), 3, 0).bytes_per_token == 104           # fp32 norms: 48 + 48 + 8
