@@ -372,7 +372,10 @@ def run_mae(args):
     """K-only logit error of the block rate allocation against uniform rates at the same
     bit budget, on the 8B- and 3B-shaped generators (8192 cached tokens, one layer): the
     logits come from bgtq_decode_scores over each packed cache, the exact ones from the
-    unquantised keys (fp64). Reports the mean absolute logit error of both layouts."""
+    unquantised keys (fp64). Reports the mean absolute logit error of both layouts, and of
+    the block allocation with norm correction and/or fp16 norms, with each layout's
+    resident bytes per (token, KV head) and its footprint ratio to an fp16 K+V record
+    (512 bytes)."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     for name in ("llama8b", "qwen3b"):
@@ -388,8 +391,12 @@ def run_mae(args):
         exact = (exact * scale).reshape(wl.h_q, wl.length).to(dev)
         line = {"mode": "mae", "workload": wl.name, "tokens": wl.length, "k_bits": wl.k_bits,
                 "block_rates": {str(r): int((rates == r).sum()) for r in sorted(set(rates.tolist()))}}
-        for tag, rr in (("block_gtq", rates), ("uniform", np.full(64, wl.k_bits))):
-            lay = B.Layout(rr, wl.v_bits, wl.seed).upload(0)
+        uni = np.full(64, wl.k_bits)
+        variants = (("block_gtq", rates, False, False), ("uniform", uni, False, False),
+                    ("block_gtq_nc", rates, True, False), ("block_gtq_fp16", rates, False, True),
+                    ("block_gtq_nc_fp16", rates, True, True), ("uniform_nc", uni, True, False))
+        for tag, rr, nc, fp16 in variants:
+            lay = B.Layout(rr, wl.v_bits, wl.seed, nc, fp16).upload(0)
             cap = wl.length
             cache = torch.zeros(lay.cache_bytes(1, wl.h_kv, cap), dtype=torch.uint8, device=dev)
             lens = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -401,6 +408,8 @@ def run_mae(args):
             torch.cuda.synchronize()
             line[f"mae_{tag}"] = float((sc[0].double() - exact).abs().mean())
             line[f"bytes_per_token_{tag}"] = lay.bytes_per_token
+            line[f"footprint_x_{tag}"] = round(2 * 128 * 2 / lay.bytes_per_token, 3)
+            assert lay.status() == 0
         line["reduction"] = 1.0 - line["mae_block_gtq"] / line["mae_uniform"]
         print(json.dumps(line), flush=True)
 

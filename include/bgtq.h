@@ -10,7 +10,9 @@
  *         s8 no fp16 sink or recent-token buffer.
  *  [TQ]   "TurboQuant: paper algorithm and vLLM engineering implementation" (pipeline
  *         diagram): input vector x (per-head K or V) -> random rotation -> per-coordinate
- *         MSE scalar quantisation with a few centroids; exercise 1: KV memory footprint.
+ *         MSE scalar quantisation with a few centroids; exercise 1: KV memory footprint;
+ *         vLLM column, box "NC": norm correction of the distortion of the norm by the
+ *         centroids (the "_nc" presets).
  *
  * Conventions for every call:
  *  - head_dim is 128; RoPE block j (0..63) is the coordinate pair {j, j+64}
@@ -45,9 +47,14 @@
  *              16+f = hi of field 16u+f; b_V = 2..4: field n of 2b_V bits at bit 2b_V*n
  *              = lo | hi << b_V. The string sits at bit 64*b_V*l of the chunk, except
  *              b_V = 3, 4: bits 0..127 at bit 128l, the rest at bit 4096 + (64b_V-128)l.
- *   K norms:   n_kgroups x 64 fp32, group-major: |x_g| of each token's group g.
- *   V norms:   64 fp32.
- *  tile_bytes = 64*(Kb + 16*b_V) + 256*(n_kgroups + 1).
+ *   K norms:   n_kgroups x 64 fp32, group-major: the norm s of each token's group g
+ *              (s = |x_g|; with BGTQ_LAYOUT_NORM_CORRECT s = |x_g| sqrt(d_g) / |c|, c the
+ *              vector of the token's centroids in the group).
+ *   V norms:   64 fp32, likewise.
+ *   With BGTQ_LAYOUT_NORM_FP16 both norm areas hold fp16 (round to nearest even; a norm
+ *   above 65504 is stored as 65504).
+ *  tile_bytes = 64*(Kb + 16*b_V) + 64*nb*(n_kgroups + 1), nb = 4 (fp32 norms) or 2 (fp16).
+ *  A token decodes to x_hat_g = (s / sqrt(d_g)) R_g^T c.
  *  A code c of a group with rate r stands for the Lloyd-Max centroid c of N(0,1) with 2^r
  *  levels (ascending); the coordinate it encodes is y = sqrt(d_g) * (R_g x_g)_i / |x_g|.
  */
@@ -98,10 +105,12 @@ typedef struct {
   int v_rate;
   int k_record_bytes;                 /* Kb */
   int v_record_bytes;                 /* 16 * v_rate */
-  int bytes_per_token;                /* Kb + 16 v_rate + 4 (n_kgroups + 1) */
+  int bytes_per_token;                /* Kb + 16 v_rate + norm_bytes (n_kgroups + 1) */
   int tile_tokens;                    /* 64 */
   int tile_bytes;
   unsigned long long seed;
+  unsigned flags;                     /* BGTQ_LAYOUT_* options of bgtq_layout_create_ex */
+  int norm_bytes;                     /* 4 (fp32 norms) or 2 (fp16) */
 } bgtq_layout_info;
 
 /* Message of the last failing call on this host thread ("" if none). */
@@ -137,6 +146,16 @@ bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate,
  * (stream 0), and builds the Lloyd-Max tables. Host only. */
 bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long long seed,
                                bgtq_layout** out);
+/* Layout options (bit flags of bgtq_layout_create_ex; 0 = the layout of bgtq_layout_create).
+ * NORM_CORRECT [TQ, box "NC"]: the stored norm of a group is |x_g| sqrt(d_g) / |c| instead
+ *   of |x_g|, so the decoded vector (s / sqrt(d_g)) R_g^T c has the norm of the input.
+ *   The codes are unchanged; only the norm the encoder writes differs.
+ * NORM_FP16: norms stored as fp16 (2 bytes per token and group instead of 4). */
+#define BGTQ_LAYOUT_NORM_CORRECT 1u
+#define BGTQ_LAYOUT_NORM_FP16 2u
+/* bgtq_layout_create with options; BGTQ_ERR_INVALID for an unknown flag bit. */
+bgtq_status bgtq_layout_create_ex(const int* k_rates, int v_rate, unsigned long long seed, unsigned flags,
+                                  bgtq_layout** out);
 void bgtq_layout_destroy(bgtq_layout* layout);
 bgtq_status bgtq_layout_get_info(const bgtq_layout* layout, bgtq_layout_info* info);
 /* Rotation of K group g (0..n_kgroups-1) or of V (g = n_kgroups), row-major d x d fp64,

@@ -22,10 +22,12 @@ STATUS_ENCODE_OVERFLOW = 1
 STATUS_DECODE_CLAMPED = 2
 STATUS_TIMEOUT = 4
 STATUS_BAD_PAGE = 8
+LAYOUT_NORM_CORRECT = 1
+LAYOUT_NORM_FP16 = 2
 
 EXPORTED = [
     "bgtq_last_error_string", "bgtq_version", "bgtq_lloyd_max", "bgtq_block_energy", "bgtq_allocate_rates",
-    "bgtq_layout_create", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
+    "bgtq_layout_create", "bgtq_layout_create_ex", "bgtq_layout_destroy", "bgtq_layout_get_info", "bgtq_layout_rotation",
     "bgtq_layout_coords", "bgtq_cache_bytes", "bgtq_layout_upload", "bgtq_encode_append",
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
     "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
@@ -37,7 +39,8 @@ class LayoutInfo(C.Structure):
     _fields_ = [("head_dim", C.c_int), ("n_blocks", C.c_int), ("n_kgroups", C.c_int),
                 ("group_rate", C.c_int * 4), ("group_dim", C.c_int * 4), ("v_rate", C.c_int),
                 ("k_record_bytes", C.c_int), ("v_record_bytes", C.c_int), ("bytes_per_token", C.c_int),
-                ("tile_tokens", C.c_int), ("tile_bytes", C.c_int), ("seed", C.c_ulonglong)]
+                ("tile_tokens", C.c_int), ("tile_bytes", C.c_int), ("seed", C.c_ulonglong),
+                ("flags", C.c_uint), ("norm_bytes", C.c_int)]
 
 
 class BgtqError(RuntimeError):
@@ -61,6 +64,7 @@ def load():
         "bgtq_block_energy": (I, [P, LL, I, P, LL, I, P]),
         "bgtq_allocate_rates": (I, [P, I, I, I, LL, P, P]),
         "bgtq_layout_create": (I, [P, I, U, C.POINTER(P)]),
+        "bgtq_layout_create_ex": (I, [P, I, U, C.c_uint, C.POINTER(P)]),
         "bgtq_layout_destroy": (None, [P]),
         "bgtq_layout_get_info": (I, [P, C.POINTER(LayoutInfo)]),
         "bgtq_layout_rotation": (I, [P, I, P, LL]),
@@ -132,17 +136,21 @@ def allocate_rates(score, min_rate: int, max_rate: int, total_bits: int, distort
 class Layout:
     """A layer's packing layout (owns the C handle)."""
 
-    def __init__(self, k_rates, v_rate: int, seed: int):
+    def __init__(self, k_rates, v_rate: int, seed: int, norm_correct: bool = False, norm_fp16: bool = False):
         lib = load()
         r = np.ascontiguousarray(k_rates, dtype=np.int32)
         if r.shape != (64,):
             raise ValueError("64 block rates expected")
         h = C.c_void_p()
-        _check(lib.bgtq_layout_create(_ptr(r), int(v_rate), C.c_ulonglong(seed), C.byref(h)), "layout_create")
+        flags = (LAYOUT_NORM_CORRECT if norm_correct else 0) | (LAYOUT_NORM_FP16 if norm_fp16 else 0)
+        _check(lib.bgtq_layout_create_ex(_ptr(r), int(v_rate), C.c_ulonglong(seed), flags, C.byref(h)),
+               "layout_create")
         self._h = h
         self.k_rates = r.copy()
         self.v_rate = int(v_rate)
         self.seed = int(seed)
+        self.norm_correct = bool(norm_correct)
+        self.norm_fp16 = bool(norm_fp16)
         info = LayoutInfo()
         _check(lib.bgtq_layout_get_info(h, C.byref(info)), "layout_get_info")
         self.info = info

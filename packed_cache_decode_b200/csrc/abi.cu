@@ -102,7 +102,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256;
+  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256 + 5 * 16 * sizeof(double);
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
   if ((e = cudaMalloc(&dblock, bytes)) != cudaSuccess) {
@@ -139,6 +139,15 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
       D.v_rot32 = p;
     }
     off += size_t(d) * ld * sizeof(float);
+  }
+  {
+    // fp64 centroids (the norm correction sums the squares of a token's centroids)
+    off = (off + 15) / 16 * 16;
+    double* hc = reinterpret_cast<double*>(host.data() + off);
+    for (int r = 0; r < 5; ++r)
+      for (int i = 0; i < 16; ++i) hc[r * 16 + i] = r >= 1 && i < (1 << r) ? L->centroid[r][i] : 0.0;
+    D.centroid64 = reinterpret_cast<const double*>(dptr + off);
+    off += 5 * 16 * sizeof(double);
   }
   {
     // codebooks of the tensor-core decode: keys of rates 1-2 scaled (exact in fp16), rates
@@ -183,7 +192,9 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   D.tile_bytes = L->tile_bytes;
   D.vcode_off = kTile * L->k_record_bytes;
   D.knorm_off = D.vcode_off + kTile * L->v_record_bytes;
-  D.vnorm_off = D.knorm_off + 4 * kTile * ng;
+  D.vnorm_off = D.knorm_off + L->norm_bytes * kTile * ng;
+  D.norm_fp16 = (L->flags & BGTQ_LAYOUT_NORM_FP16) ? 1 : 0;
+  D.norm_correct = (L->flags & BGTQ_LAYOUT_NORM_CORRECT) ? 1 : 0;
   for (int g = 0; g < kMaxGroups; ++g) {
     D.group_rate[g] = L->group_rate[g];
     D.group_dim[g] = L->group_dim[g];

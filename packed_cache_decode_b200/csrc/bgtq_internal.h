@@ -27,17 +27,21 @@ struct DevLayout {
   int vcode_off;        // byte offsets inside a tile
   int knorm_off;
   int vnorm_off;
+  int norm_fp16;        // norms stored as fp16 (else fp32)
+  int norm_correct;     // NC: stored norm |x| sqrt(d) / |c|
   int group_rate[kMaxGroups];
   int group_dim[kMaxGroups];
   int group_off[kMaxGroups];     // first packed dimension of the group
   int group_bitoff[kMaxGroups];  // first bit of the group inside a K record
   short packed_coord[kD];        // packed key dimension -> original coordinate
   double threshold[5][16];       // [rate][k], fp64 (2^rate - 1 used)
+
   const double* k_rot64[kMaxGroups];  // d_g x d_g, TRANSPOSED: element (i, j) of R at j * d + i
   const double* v_rot64;              // 128 x 128, transposed likewise
   const float* k_rot32[kMaxGroups];  // row-major, rows padded to k_rot32_ld[g] floats (a multiple of 4)
   int k_rot32_ld[kMaxGroups];
   const float* v_rot32;
+  const double* centroid64;      // [rate][code] at rate * 16 + code, fp64 (norm correction)
   unsigned* status;
   // Fragment-major K area: each group's packed dims cut into quads of 4 pairs (8 dims),
   // the last quad of a group holding the remaining 1-3 pairs.
@@ -107,6 +111,8 @@ struct bgtq_layout {
   double threshold[5][16];
   double mse[5];
   int k_record_bytes, v_record_bytes, bytes_per_token, tile_bytes;
+  unsigned flags;   // BGTQ_LAYOUT_* options
+  int norm_bytes;   // 4 or 2
   // device copy
   int device = -1;
   void* dev_block = nullptr;

@@ -471,6 +471,7 @@ __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const 
 
 // First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
 // token and KV head), the others prepare q' of one unit each.
+template <bool NC>
 __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
                                                                  const void* __restrict__ v, int kv_dtype, int n_new,
                                                                  int batch, const int* __restrict__ seq_lens_before,
@@ -486,16 +487,23 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
     const int t = rest % n_new;
     rest /= n_new;
     const int b = rest % batch, h = rest / batch;
-    enc::encode_token_part(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
-  } else {
+    enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
+  } else if (e - n_enc < batch * h_kv) {  // (a cluster launch pads the grid)
     const int u = e - n_enc;
     prep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
   }
 }
 
+// Norm i of a tile's norm area, stored as fp16 (NH) or fp32.
+template <bool NH>
+__device__ __forceinline__ float tile_norm(const unsigned char* area, int i) {
+  if constexpr (NH) return __half2float(reinterpret_cast<const __half*>(area)[i]);
+  else return reinterpret_cast<const float*>(area)[i];
+}
+
 // SC: scores only. The tiles' logits (softmax_scale q . k_hat, natural units) go to
-// a.scores; no softmax, values, partials or merge.
-template <int VR, bool NP, bool SC = false>
+// a.scores; no softmax, values, partials or merge. NH: the layout stores fp16 norms.
+template <int VR, bool NP, bool SC, bool NH>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(16) Luts<VR> T;
@@ -512,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
   unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);  // [kRing]
   unsigned char* ring = smem + 128;                                        // stage s at ring + s TB
   unsigned* qf = reinterpret_cast<unsigned*>(ring + kRing * TB);           // [quad][2][32]
-  float* mm = reinterpret_cast<float*>(qf + kMaxQuads * 64);               // [warp][8]
+  float* mm = reinterpret_cast<float*>(qf + L.n_kquads * 64);              // [warp][8]
   float* ml = mm + kWarps * 8;                                             // [warp][8]
   // the warps' [8][128] partials reuse the ring once every tile of the segment is consumed
   float* mo = reinterpret_cast<float*>(ring);
@@ -540,6 +548,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       T.k4[e] = make_uint2(unsigned(L.kc4[0][e & 15]) | (unsigned(L.kc4[0][e >> 4]) << 16),
                            unsigned(L.kc4[1][e & 15]) | (unsigned(L.kc4[1][e >> 4]) << 16));
   if constexpr (VR == 2 || VR == 3) {
+    // lane-private pair tables: entry e of lane l at 32 e + l (no bank conflicts)
     constexpr unsigned vm = (1u << VR) - 1u;
     for (int i = tid; i < Luts<VR>::kV; i += kThreads) {
       const int e = i >> 5;
@@ -631,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
 
       // ---------------- scores: per key group (rate as a template parameter), per quad,
       // NRT row blocks; then times the group norms
-      const float* kn = reinterpret_cast<const float*>(tb + L.knorm_off) + 16 * rb0;
+      const unsigned char* kna = tb + L.knorm_off;
       float sc[NRT][4];
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt)
@@ -652,7 +661,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         }
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt) {
-          const float n0 = kn[gi * kTile + 16 * rt + g], n1 = kn[gi * kTile + 16 * rt + g + 8];
+          const int ni = gi * kTile + 16 * (rb0 + rt) + g;
+          const float n0 = tile_norm<NH>(kna, ni), n1 = tile_norm<NH>(kna, ni + 8);
           sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
           sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
           sc[rt][2] = fmaf(acc[rt][2], n1, sc[rt][2]);
@@ -715,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
           O[mt][3] *= corr1;
         }
       }
-      const float* vn = reinterpret_cast<const float*>(tb + L.vnorm_off) + 16 * rb0;
+      const unsigned char* vna = tb + L.vnorm_off;
 
       // ---------------- values: row block rb0 + rt is value chunk rb0 + rt of the tile.
       // First the probabilities (times |v| / sqrt(128)) as transposed fp16 B fragments,
@@ -727,7 +737,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         const float p2 = fast_exp2(sc[rt][2] - b0m), p3 = fast_exp2(sc[rt][3] - b1m);
         l0 += p0 + p2;
         l1 += p1 + p3;
-        const float av0 = vn[16 * rt + g] * vscale, av1 = vn[16 * rt + g + 8] * vscale;
+        const float av0 = tile_norm<NH>(vna, 16 * (rb0 + rt) + g) * vscale;
+        const float av1 = tile_norm<NH>(vna, 16 * (rb0 + rt) + g + 8) * vscale;
         pb[rt][0] = movmatrix_trans(pack_h2(p0 * av0, p1 * av0));
         pb[rt][1] = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
       }
@@ -831,22 +842,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       if (pend & (1u << h)) mbar_wait_bounded(&full[warp + kWarps * h], (phase >> h) & 1u);
 }
 
-size_t split_smem_bytes(int tile_bytes) {
-  return 128 + size_t(kRing) * tile_bytes + kMaxQuads * 64 * sizeof(unsigned) + 2 * kWarps * 8 * sizeof(float);
+size_t split_smem_bytes(int tile_bytes, int n_kquads) {
+  return 128 + size_t(kRing) * tile_bytes + size_t(n_kquads) * 64 * sizeof(unsigned) + 2 * kWarps * 8 * sizeof(float);
 }
 
-template <int VR, bool NP, bool SC = false>
-cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, cudaStream_t stream) {
-  const size_t smem = split_smem_bytes(L.tile_bytes);
+// Once per device and variant, before the occupancy query and the first launch: the
+// largest dynamic shared memory any layout needs, and the whole unified L1/shared array as
+// shared memory (the occupancy the plan assumes is then the one the launch gets).
+template <int VR, bool NP, bool SC, bool NH>
+cudaError_t configure_split() {
   static bool configured[64] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(split_kernel<VR, NP, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(split_smem_bytes(kMaxTileBytes)));
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev >= 64 || configured[dev]) return e;
+  e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(split_smem_bytes(kMaxTileBytes, kMaxQuads)));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             int(cudaSharedmemCarveoutMaxShared));
+  if (e == cudaSuccess) configured[dev] = true;
+  return e;
+}
+
+template <int VR, bool NP, bool SC, bool NH>
+cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, cudaStream_t stream) {
+  const size_t smem = split_smem_bytes(L.tile_bytes, L.n_kquads);
+  cudaError_t e = configure_split<VR, NP, SC, NH>();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_ctas);
   cfg.blockDim = dim3(kThreads);
@@ -857,7 +879,7 @@ cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC>, L, a);
+  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC, NH>, L, a);
 }
 
 // ------------------------------------------------------------------ combine
@@ -952,13 +974,36 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   if (tid < kD) out[((size_t)b * h_q + hq) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
 }
 
-template <int VR, bool NP, bool SC = false>
+template <int VR, bool NP, bool SC, bool NH>
 int split_occupancy(const DevLayout& L) {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<VR, NP, SC>, kThreads,
-                                                    split_smem_bytes(L.tile_bytes)) != cudaSuccess)
+  if (configure_split<VR, NP, SC, NH>() != cudaSuccess) return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<VR, NP, SC, NH>, kThreads,
+                                                    split_smem_bytes(L.tile_bytes, L.n_kquads)) != cudaSuccess)
     return 1;
   return n < 1 ? 1 : n;
+}
+
+// Calls fn(IntC<VR>, IntC<NP>, IntC<SC>, IntC<NH>) with the split-kernel variant of a
+// call: value rate (scores only: 1, the value tables are not built), q' in one product
+// (G <= 4), scores only, fp16 norms.
+template <int VR, int NP, int SC, typename Fn>
+auto split_nh(bool nh, Fn&& fn) {
+  return nh ? fn(IntC<VR>{}, IntC<NP>{}, IntC<SC>{}, IntC<1>{}) : fn(IntC<VR>{}, IntC<NP>{}, IntC<SC>{}, IntC<0>{});
+}
+template <int VR, int SC, typename Fn>
+auto split_np(bool np, bool nh, Fn&& fn) {
+  return np ? split_nh<VR, 1, SC>(nh, fn) : split_nh<VR, 0, SC>(nh, fn);
+}
+template <typename Fn>
+auto split_variant(int v_rate, bool np, bool sc, bool nh, Fn&& fn) {
+  if (sc) return split_np<1, 1>(np, nh, fn);
+  switch (v_rate) {
+    case 1: return split_np<1, 0>(np, nh, fn);
+    case 2: return split_np<2, 0>(np, nh, fn);
+    case 3: return split_np<3, 0>(np, nh, fn);
+    default: return split_np<4, 0>(np, nh, fn);
+  }
 }
 
 // Split and combine kernels of one call, launched as programmatic dependents of the
@@ -970,24 +1015,14 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   const int G = h_q / h_kv;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
-  // scores only: variants 0 (G > 4) and 1 (G <= 4), no value tables
-  const int variant = scores ? (np ? 1 : 0) : L.v_rate * 2 + (np ? 1 : 0);
   // the workspace was sized for the most CTAs per SM; shared memory may allow fewer
   // (larger slices, fewer partials per unit)
-  int occ = 1;
-  switch (variant) {
-    case 0: occ = split_occupancy<1, false, true>(L); break;
-    case 1: occ = split_occupancy<1, true, true>(L); break;
-    case 2: occ = split_occupancy<1, false>(L); break;
-    case 3: occ = split_occupancy<1, true>(L); break;
-    case 4: occ = split_occupancy<2, false>(L); break;
-    case 5: occ = split_occupancy<2, true>(L); break;
-    case 6: occ = split_occupancy<3, false>(L); break;
-    case 7: occ = split_occupancy<3, true>(L); break;
-    case 8: occ = split_occupancy<4, false>(L); break;
-    case 9: occ = split_occupancy<4, true>(L); break;
-    default: return cudaErrorInvalidValue;
-  }
+  const bool sc = scores != nullptr, nh = L.norm_fp16 != 0;
+  if (!sc && (L.v_rate < 1 || L.v_rate > 4)) return cudaErrorInvalidValue;
+  const int occ = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
+    return split_occupancy<decltype(V)::value, decltype(P)::value != 0, decltype(S)::value != 0,
+                           decltype(H)::value != 0>(L);
+  });
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1017,19 +1052,11 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   a.len_add = len_add;
   a.wait_new = after_append ? 1 : 0;
   const unsigned n_ctas = unsigned(plan.n_ctas);
-  switch (variant) {
-    case 0: return launch_split<1, false, true>(a, L, n_ctas, stream);
-    case 1: return launch_split<1, true, true>(a, L, n_ctas, stream);
-    case 2: e = launch_split<1, false>(a, L, n_ctas, stream); break;
-    case 3: e = launch_split<1, true>(a, L, n_ctas, stream); break;
-    case 4: e = launch_split<2, false>(a, L, n_ctas, stream); break;
-    case 5: e = launch_split<2, true>(a, L, n_ctas, stream); break;
-    case 6: e = launch_split<3, false>(a, L, n_ctas, stream); break;
-    case 7: e = launch_split<3, true>(a, L, n_ctas, stream); break;
-    case 8: e = launch_split<4, false>(a, L, n_ctas, stream); break;
-    case 9: e = launch_split<4, true>(a, L, n_ctas, stream); break;
-    default: e = cudaErrorInvalidValue;
-  }
+  e = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
+    return launch_split<decltype(V)::value, decltype(P)::value != 0, decltype(S)::value != 0,
+                        decltype(H)::value != 0>(a, L, n_ctas, stream);
+  });
+  if (sc) return e;  // scores only: no merge
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(batch * h_q));
@@ -1097,10 +1124,31 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
                                void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
   const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
-  step_prep_kernel<<<unsigned(n_enc + batch * h_kv), kPrepThreads, 0, stream>>>(
-      L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype,
-      h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (!L.norm_correct) {
+    step_prep_kernel<false><<<unsigned(n_enc + batch * h_kv), kPrepThreads, 0, stream>>>(
+        L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype,
+        h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
+    e = cudaGetLastError();
+  } else {
+    // norm correction: clusters of the four encode parts of a token; the q' blocks
+    // follow, padded to a whole cluster (the padding blocks return at once)
+    const long long n_blocks = (n_enc + batch * h_kv + kEncodeParts - 1) / kEncodeParts * kEncodeParts;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(n_blocks));
+    cfg.blockDim = dim3(kPrepThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kEncodeParts;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, step_prep_kernel<true>, L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache,
+                           q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
+                           int(n_enc));
+  }
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens_before, out, workspace, n_new,
                           n_new > 0, stream);

@@ -10,6 +10,7 @@
 // distance of a threshold.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -104,6 +105,13 @@ __device__ __forceinline__ void put_value_code(const DevLayout& L, uint8_t* tile
   }
 }
 
+// Stores norm s of entry i (token-major inside its group's row of 64) of a tile's norm
+// area: fp32, or fp16 rounded to nearest even and saturated at the largest finite fp16.
+__device__ __forceinline__ void store_norm(const DevLayout& L, uint8_t* area, int i, double s) {
+  if (L.norm_fp16) reinterpret_cast<__half*>(area)[i] = __double2half(fmin(s, 65504.0));
+  else reinterpret_cast<float*>(area)[i] = float(s);
+}
+
 // Four CTAs of 256 threads code one (token, KV head); CTA `part` owns packed key
 // dimensions and value dimensions [32 part, 32 part + 32). Each of its 64 outputs is
 // computed by four consecutive threads, each over a quarter of the rotation row (read
@@ -111,22 +119,44 @@ __device__ __forceinline__ void put_value_code(const DevLayout& L, uint8_t* tile
 // loads in flight, summed with two shuffles. Every CTA recomputes the group norms (the
 // inputs are 256 values). Codes are written with atomics: the key fields of a chunk and
 // the value rows are shared with other tokens and other parts.
+//
+// Norm correction ("TurboQuant: paper algorithm and vLLM engineering implementation",
+// vLLM column, box "NC"): the stored norm is |x| sqrt(d) / |c|, c the vector of the
+// centroids the group's coordinates were coded to, so that the decoded vector keeps the
+// input's norm. |c|^2 spans the four parts' codes: the four CTAs of a token run as one
+// thread-block cluster; each sums the squares of its own centroids per group (fixed
+// order), writes the sums into part 0's shared memory, and after the cluster barrier
+// part 0 writes the corrected norms. The launch must then use clusters of 4 along x.
 constexpr int kEncodeThreads = 256;
 
 // Body of one encode CTA (256 threads): token t of batch row b, KV head h, output part
-// `part` (0..3).
+// `part` (0..3). NC: the layout has norm correction (L.norm_correct), and the launch runs
+// the four parts of a token as one cluster.
+template <bool NC>
 __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void* __restrict__ k,
                                                   const void* __restrict__ v, int dtype, int n_new, int h_kv,
                                                   const int* __restrict__ seq_lens, const CacheRef& cache, int t,
                                                   int part, int b, int h) {
   const int tid = threadIdx.x;
   const long long pos = (long long)seq_lens[b] + t;
+  // both early exits are the same for the four parts of a token (with NC, a whole cluster
+  // leaves before its first barrier)
   if (pos < 0 || pos >= cache.n_tiles * kTile) {
     if (tid == 0 && part == 0) atomicOr(L.status, BGTQ_STATUS_ENCODE_OVERFLOW);
     return;
   }
+  uint8_t* tp = nullptr;
+  if constexpr (NC) {
+    tp = tile_ptr(cache, L, b, h, h_kv, pos / kTile);
+    if (!tp) return;
+    // the cluster's CTAs must all have started before one writes into another's shared
+    // memory: arrive now, wait just before that write
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  }
   __shared__ double xp[kD], xv[kD];
   __shared__ double gnorm[kMaxGroups + 1];
+  __shared__ double csq[64];                         // NC: squared centroid of each output
+  __shared__ double part_sq[kEncodeParts][kMaxGroups + 1];  // NC, part 0: the parts' sums
 
   const size_t base = (((size_t)b * n_new + t) * h_kv + h) * kD;
   if (tid < kD) xp[tid] = load_elem(k, dtype, base + L.packed_coord[tid]);  // keys in packed order
@@ -172,24 +202,66 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   double acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-  if (q != 0) return;
 
-  const double nrm = gnorm[is_key ? g : kMaxGroups];
-  const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
-  const int r = is_key ? L.group_rate[g] : L.v_rate;
-  const int code = quantize(y, L.threshold[r], r);
-
-  const long long tile = pos / kTile;
+  if constexpr (!NC) {
+    if (q != 0) return;
+    const double nrm = gnorm[is_key ? g : kMaxGroups];
+    const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
+    const int r = is_key ? L.group_rate[g] : L.v_rate;
+    const int code = quantize(y, L.threshold[r], r);
+    const int tt = int(pos % kTile);
+    tp = tile_ptr(cache, L, b, h, h_kv, pos / kTile);
+    if (!tp) return;
+    if (is_key) {
+      put_key_code(L, tp, g, i, tt, unsigned(code));
+      if (part == 0 && p < L.n_kgroups) store_norm(L, tp + L.knorm_off, p * kTile + tt, gnorm[p]);
+    } else {
+      put_value_code(L, tp, p, tt, unsigned(code));
+      if (p == 0) store_norm(L, tp + L.vnorm_off, tt, gnorm[kMaxGroups]);
+    }
+    return;
+  }
   const int tt = int(pos % kTile);
-  uint8_t* tp = tile_ptr(cache, L, b, h, h_kv, tile);
-  if (!tp) return;
-  if (is_key) {
-    put_key_code(L, tp, g, i, tt, unsigned(code));
-    if (part == 0 && p < L.n_kgroups)
-      reinterpret_cast<float*>(tp + L.knorm_off)[p * kTile + tt] = float(gnorm[p]);
-  } else {
-    put_value_code(L, tp, p, tt, unsigned(code));
-    if (p == 0) reinterpret_cast<float*>(tp + L.vnorm_off)[tt] = float(gnorm[kMaxGroups]);
+  if (q == 0) {
+    const double nrm = gnorm[is_key ? g : kMaxGroups];
+    const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
+    const int r = is_key ? L.group_rate[g] : L.v_rate;
+    const int code = quantize(y, L.threshold[r], r);
+    if (is_key) put_key_code(L, tp, g, i, tt, unsigned(code));
+    else put_value_code(L, tp, p, tt, unsigned(code));
+    const double c = L.centroid64[r * 16 + code];
+    csq[o] = c * c;
+  }
+  uint8_t* kna = tp + L.knorm_off;
+  uint8_t* vna = tp + L.vnorm_off;
+  // ---- norm correction: every thread of the four CTAs reaches every cluster barrier
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (tid <= kMaxGroups) {
+    // entry tid < kMaxGroups: key group tid (outputs 0..31 of this part), entry kMaxGroups:
+    // the value vector (outputs 32..63)
+    double sq = 0.0;
+    if (tid == kMaxGroups) {
+      for (int oo = 32; oo < 64; ++oo) sq += csq[oo];
+    } else if (tid < L.n_kgroups) {
+      const int lo = L.group_off[tid], hi = lo + L.group_dim[tid];
+      for (int oo = 0; oo < 32; ++oo) {
+        const int pp = 32 * part + oo;
+        if (pp >= lo && pp < hi) sq += csq[oo];
+      }
+    }
+    double* dst = cluster.map_shared_rank(&part_sq[0][0], 0);
+    dst[part * (kMaxGroups + 1) + tid] = sq;
+  }
+  cluster.sync();
+  if (part == 0 && tid <= kMaxGroups && (tid < L.n_kgroups || tid == kMaxGroups)) {
+    const double c2 = ((part_sq[0][tid] + part_sq[1][tid]) + (part_sq[2][tid] + part_sq[3][tid]));
+    const double dd = tid == kMaxGroups ? double(kD) : double(L.group_dim[tid]);
+    const double s = c2 > 0.0 ? gnorm[tid] * sqrt(dd) / sqrt(c2) : 0.0;
+    if (tid == kMaxGroups) store_norm(L, vna, tt, s);
+    else store_norm(L, kna, tid * kTile + tt, s);
   }
 }
 

@@ -239,8 +239,15 @@ bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate,
 }
 
 bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long long seed, bgtq_layout** out) {
+  return bgtq_layout_create_ex(k_rates, v_rate, seed, 0u, out);
+}
+
+bgtq_status bgtq_layout_create_ex(const int* k_rates, int v_rate, unsigned long long seed, unsigned flags,
+                                  bgtq_layout** out) {
   if (!k_rates || !out) return fail(BGTQ_ERR_INVALID, "layout_create: null pointer");
   *out = nullptr;
+  if (flags & ~(BGTQ_LAYOUT_NORM_CORRECT | BGTQ_LAYOUT_NORM_FP16))
+    return fail(BGTQ_ERR_INVALID, "layout_create: unknown option flag");
   int sum = 0;
   for (int j = 0; j < kBlocks; ++j) {
     if (!valid_rate(k_rates[j])) return fail(BGTQ_ERR_INVALID, "layout_create: key rates must be 1..4");
@@ -253,6 +260,8 @@ bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long lon
   std::memcpy(L->k_rates, k_rates, sizeof(L->k_rates));
   L->v_rate = v_rate;
   L->seed = seed;
+  L->flags = flags;
+  L->norm_bytes = (flags & BGTQ_LAYOUT_NORM_FP16) ? 2 : 4;
   // Equal-rate blocks form one group; groups by descending rate, blocks ascending,
   // coordinate j before j + 64.
   int ng = 0, pd = 0, bit = 0;
@@ -285,7 +294,7 @@ bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long lon
     for (int i = (1 << r) - 1; i < 16; ++i) L->threshold[r][i] = INFINITY;
   L->k_record_bytes = bit / 8;
   L->v_record_bytes = 16 * v_rate;
-  L->bytes_per_token = L->k_record_bytes + L->v_record_bytes + 4 * (ng + 1);
+  L->bytes_per_token = L->k_record_bytes + L->v_record_bytes + L->norm_bytes * (ng + 1);
   L->tile_bytes = kTile * L->bytes_per_token;
   *out = L;
   return BGTQ_OK;
@@ -307,6 +316,8 @@ bgtq_status bgtq_layout_get_info(const bgtq_layout* L, bgtq_layout_info* info) {
   info->tile_tokens = kTile;
   info->tile_bytes = L->tile_bytes;
   info->seed = L->seed;
+  info->flags = L->flags;
+  info->norm_bytes = L->norm_bytes;
   return BGTQ_OK;
 }
 

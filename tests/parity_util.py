@@ -29,6 +29,8 @@ class Case:
     seed: int = 0
     scale_v: bool = False
     capacity: int | None = None
+    norm_correct: bool = False
+    norm_fp16: bool = False
 
     @property
     def cap(self):
@@ -51,7 +53,7 @@ def build_inputs(case: Case):
 
 def gpu_encode(case: Case, rates, k, v, n_chunks: int = 1, layout=None):
     """Encode-append all tokens on the GPU (in n_chunks appends); returns (layout, cache)."""
-    lay = layout or B.Layout(rates, case.v_bits, case.seed).upload(0)
+    lay = layout or B.Layout(rates, case.v_bits, case.seed, case.norm_correct, case.norm_fp16).upload(0)
     cap = case.cap
     cache = torch.zeros(lay.cache_bytes(case.batch, case.h_kv, cap), dtype=torch.uint8, device="cuda")
     kd, vd = k.cuda(), v.cuda()
@@ -77,7 +79,7 @@ def gpu_decode(lay, case: Case, q, cache, seq_lens=None, max_seq_len=None, scale
 
 
 def oracle_slice(case: Case, rates, k, v, b: int, h: int, n: int | None = None):
-    lay = O.make_layout(rates, case.v_bits, case.seed)
+    lay = O.make_layout(rates, case.v_bits, case.seed, case.norm_correct, case.norm_fp16)
     n = case.length if n is None else n
     enc = O.encode(lay, k[b, :n, h].double().numpy(), v[b, :n, h].double().numpy())
     buf = O.pack(lay, enc, case.cap)
@@ -92,7 +94,9 @@ def slice_bytes(case: Case, lay_bytes_per_tile: int, cache_cpu: np.ndarray, b: i
 
 
 def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, capacity: int):
-    """Codes bit-exact except near-threshold coordinates; norms to 1 fp32 ulp.
+    """Codes bit-exact except near-threshold coordinates; norms to 1 ulp of their stored
+    type. With norm correction a norm depends on every code of its token, so tokens with
+    a differing (near-threshold) code are left out of the norm comparison.
     Returns (near-boundary count, how many of those differ)."""
     mask, n_near = O.boundary_mask(lay, enc, capacity, CODE_EPS)
     nt = capacity // 64
@@ -104,9 +108,17 @@ def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, 
     diff = (w[:, :code_bytes] ^ g[:, :code_bytes]) & ~m[:, :code_bytes]
     bad = np.argwhere(diff != 0)
     assert bad.size == 0, f"{len(bad)} code bytes differ away from thresholds, first at tile/byte {bad[:5].tolist()}"
-    wn = w[:, code_bytes:].copy().view(np.float32)
-    gn = g[:, code_bytes:].copy().view(np.float32)
-    ulp = np.abs(wn.view(np.int32).astype(np.int64) - gn.view(np.int32).astype(np.int64))
+    it = np.int16 if lay.norm_fp16 else np.int32
+    wn = w[:, code_bytes:].copy().view(it).astype(np.int64)
+    gn = g[:, code_bytes:].copy().view(it).astype(np.int64)
+    ulp = np.abs(wn - gn)                         # norms are >= 0: integer order is float order
+    if lay.norm_correct:
+        n = enc["k_codes"].shape[0]
+        uw, ug = O.unpack(lay, want, n), O.unpack(lay, got, n)
+        differs = np.zeros(nt * 64, dtype=bool)
+        differs[:n] = np.any(uw["k_codes"] != ug["k_codes"], axis=1) | np.any(uw["v_codes"] != ug["v_codes"], axis=1)
+        per_tile = differs.reshape(nt, 1, 64)     # norm entry j of a tile belongs to token j % 64
+        ulp = np.where(np.broadcast_to(per_tile, (nt, lay.n_kgroups + 1, 64)).reshape(nt, -1), 0, ulp)
     assert ulp.max() <= 1, f"norm differs by {ulp.max()} ulp"
     near_diff = int(np.count_nonzero((w[:, :code_bytes] ^ g[:, :code_bytes]) & m[:, :code_bytes]))
     return n_near, near_diff

@@ -31,12 +31,13 @@ def _tile(pc, lay, h_kv, b, h, i):
     return pc.pool[(p * h_kv + h) * tb:(p * h_kv + h + 1) * tb]
 
 
+@pytest.mark.parametrize("options", [(False, False), (True, True)], ids=["plain", "nc_fp16"])
 @pytest.mark.parametrize("shape", [(16, 4, 3, 700, 2, 2), (16, 2, 2, 333, 3, 3)])
-def test_paged_equals_contiguous(shape):
+def test_paged_equals_contiguous(shape, options):
     h_q, h_kv, batch, length, kb, vb = shape
     case = Case(h_q, h_kv, batch, length, kb, vb, torch.bfloat16, 5e5, 41)
     model, rates, q, k, v = build_inputs(case)
-    lay = B.Layout(rates, case.v_bits, case.seed).upload(0)
+    lay = B.Layout(rates, case.v_bits, case.seed, *options).upload(0)
     cap = case.cap
     max_pages = cap // 64
     lens = torch.tensor([length - 211 * b for b in range(batch)], dtype=torch.int32)

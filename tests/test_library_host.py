@@ -133,3 +133,20 @@ def test_host_validation_without_device(lib):
                                      None) == B.ERR_DEVICE
     if not torch.cuda.is_available():
         assert lib.bgtq_layout_upload(lay.handle, 0) in (B.ERR_CUDA, B.ERR_INVALID)
+
+
+@pytest.mark.parametrize("flags", [0, 1, 2, 3])
+def test_layout_options_match_oracle_bytes(lib, flags):
+    """bgtq_layout_create_ex: the norm options change the bytes per token as the oracle's
+    layout does (2-byte norms with BGTQ_LAYOUT_NORM_FP16); an unknown flag is refused."""
+    rates = np.array([4] * 8 + [3] * 8 + [2] * 24 + [1] * 24)
+    lay = B.Layout(rates, 3, 9, bool(flags & 1), bool(flags & 2))
+    olay = O.make_layout(rates, 3, 9, bool(flags & 1), bool(flags & 2))
+    assert lay.info.flags == flags
+    assert lay.info.bytes_per_token == olay.bytes_per_token
+    assert lay.info.tile_bytes == olay.tile_bytes
+    assert lay.cache_bytes(2, 8, 4097) == O.cache_bytes(olay, 2, 8, 4097)
+    r = np.ascontiguousarray(rates, dtype=np.int32)
+    h = C.c_void_p()
+    assert lib.bgtq_layout_create_ex(r.ctypes.data_as(C.c_void_p), 3, 9, 4, C.byref(h)) == B.ERR_INVALID
+    assert not h.value
