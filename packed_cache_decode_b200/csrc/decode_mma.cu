@@ -384,8 +384,10 @@ __device__ __forceinline__ int cta_segments(const DevLayout& L, const SplitArgs&
 // q' B fragments of unit u (batch row b, KV head h) into frag[kMaxQuads][2][32] (global),
 // by one CTA of kPrepThreads: thread (p = tid % 128, half = tid / 128) computes
 // q'[hh][p] = f_g sum_j R_g[i][j] q[hh][off_g + j] for the heads hh = 4 half .. 4 half + 3
-// (16-byte rows of R_g from global memory, q staged in shared memory), then every
-// fragment word is written once. With G <= 4 the eight B columns are heads 0..3 (hi
+// (16-byte rows of R_g from global memory, q staged in shared memory); with G <= 4 the
+// two halves take heads 0..3 over the two halves of the row instead (all of a thread's
+// row is then loaded before q arrives) and add up in shared memory. Then every fragment
+// word is written once. With G <= 4 the eight B columns are heads 0..3 (hi
 // parts) and heads 0..3 again (lo parts) in the first array; otherwise the first array
 // holds the hi parts of heads 0..7 and the second the lo parts. Missing pairs and heads
 // are zero.
@@ -398,16 +400,21 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   __shared__ float qr[kMaxG * kD];                   // q' in packed order
   const int tid = threadIdx.x, ng = L.n_kgroups;
   const int b = u / h_kv, h = u % h_kv;
-  // this thread's row of R_g: the first 16 float4 are loaded before q arrives
-  const int p = tid & (kD - 1), h0 = (tid >> 7) * 4;
+  __shared__ float red[4 * kD];                      // the k-split halves' partial sums
+  // this thread's row of R_g (columns [4 c0, 4 c1)): the first 16 float4 are loaded
+  // before q arrives
+  const int p = tid & (kD - 1), half = tid >> 7;
+  const bool ksplit = G <= 4;
+  const int h0 = ksplit ? 0 : half * 4;
   int g = 0, pad = 0;
   while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
   const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
-  const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld);
+  const int n4 = ld / 4, c0 = ksplit ? half * ((n4 + 1) / 2) : 0, c1 = ksplit ? min(n4, c0 + (n4 + 1) / 2) : n4;
+  const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld) + c0;
   constexpr int kPre = 16;
   float4 r[kPre];
 #pragma unroll
-  for (int j4 = 0; j4 < kPre; ++j4) r[j4] = j4 < ld / 4 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j4 = 0; j4 < kPre; ++j4) r[j4] = c0 + j4 < c1 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < kMaxG * kQsLd; e += kPrepThreads) qs[e] = 0.f;
   __syncthreads();
   for (int e = tid; e < G * kD; e += kPrepThreads) {
@@ -418,12 +425,12 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
         load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + L.packed_coord[pe]);
   }
   __syncthreads();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   if (h0 < G) {
-    const float* qg = qs + h0 * kQsLd + pad;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* qg = qs + h0 * kQsLd + pad + 4 * c0;
 #pragma unroll
     for (int j4 = 0; j4 < kPre; ++j4) {
-      if (j4 < ld / 4) {  // q columns past the group's padded row are not read
+      if (c0 + j4 < c1) {  // q columns past the group's padded row are not read
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
@@ -432,7 +439,7 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
       }
     }
 #pragma unroll 8
-    for (int j4 = kPre; j4 < ld / 4; ++j4) {
+    for (int j4 = kPre; c0 + j4 < c1; ++j4) {
       const float4 rr = __ldg(row + j4);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -440,6 +447,17 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
         acc[k] = fmaf(rr.x, x.x, fmaf(rr.y, x.y, fmaf(rr.z, x.z, fmaf(rr.w, x.w, acc[k]))));
       }
     }
+  }
+  if (ksplit) {  // uniform over the CTA
+    if (half == 1)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) red[k * kD + p] = acc[k];
+    __syncthreads();
+    if (half == 0)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += red[k * kD + p];
+  }
+  if (h0 < G && (!ksplit || half == 0)) {
     const float f = qscale * rsqrtf(float(d)) * L.inv_kappa_group[g];  // the key tables carry kappa
 #pragma unroll
     for (int k = 0; k < 4; ++k) qr[(h0 + k) * kD + p] = acc[k] * f;
