@@ -664,6 +664,24 @@ def decode_attention(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int
     return attention(q, kh, vh, scale)
 
 
+def decode_attention_multi(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int, scale: float) -> np.ndarray:
+    """Attention of n_q consecutive query tokens q [n_q, G, 128] of one KV head over its
+    packed cache of ``length`` tokens, the last n_q of which are the query tokens' own
+    keys and values (multi-token decode: speculative verification, a prefill chunk).
+    Causal among the new tokens: query j sits at position length - n_q + j and attends to
+    tokens 0 .. length - n_q + j [BGTQ sentence 5: attention over the packed cache; the
+    causal rule is the one of autoregressive attention]. Returns [n_q, G, 128]."""
+    q = np.asarray(q, dtype=np.float64)
+    n_q = q.shape[0]
+    u = unpack(layout, buf, length)
+    kh, vh = reconstruct(layout, u["k_codes"], u["k_norms"], u["v_codes"], u["v_norm"])
+    out = np.zeros_like(q)
+    for j in range(n_q):
+        n = max(0, length - n_q + j + 1)
+        out[j] = attention(q[j], kh[:n], vh[:n], scale)
+    return out
+
+
 def decode_scores(layout: Layout, q: np.ndarray, buf: np.ndarray, length: int, scale: float) -> np.ndarray:
     """Logits scale * q . k_hat of the G query heads q [G, 128] against every cached token of
     one KV head's packed cache [BGTQ sentence 5: scores over the packed codes]; [G, length]."""

@@ -524,3 +524,48 @@ def test_resident_bytes_with_fp16_norms():
     mixed = O.make_layout(np.array([4] * 8 + [3] * 8 + [2] * 24 + [1] * 24), 2, 0, norm_fp16=True)
     assert mixed.n_kgroups == 4 and mixed.k_record_bytes == 32 and mixed.bytes_per_token == 74
     assert O.make_layout(np.full(64, 3), 3, 0).bytes_per_token == 104           # fp32 norms: 48 + 48 + 8
+
+
+# ------------------------------------------------------------ multi-token queries ----
+def _packed_slice(seed, n, rates=None, v_rate=2):
+    rng = np.random.default_rng(seed)
+    lay = O.make_layout(np.full(64, 2) if rates is None else rates, v_rate, seed)
+    k = rng.standard_normal((n, 128)) * rng.uniform(0.2, 4, 128)
+    v = rng.standard_normal((n, 128))
+    enc = O.encode(lay, k, v)
+    return lay, enc, O.pack(lay, enc, 64 * -(-n // 64))
+
+
+def test_multi_token_attention_matches_masked_sdpa():
+    """Query j of n_q new tokens sits at position L - n_q + j: the result equals PyTorch's
+    scaled_dot_product_attention over the decoded cache with the explicit mask
+    key <= L - n_q + j (a library routine, not this oracle's attention)."""
+    lay, enc, buf = _packed_slice(3, 150)
+    L, n_q, G = 150, 5, 3
+    q = np.random.default_rng(4).standard_normal((n_q, G, 128))
+    got = O.decode_attention_multi(lay, q, buf, L, 0.09)
+    kh, vh = O.reconstruct(lay, enc["k_codes"], O.stored_norms(lay, enc["k_norms"]).astype(np.float64),
+                           enc["v_codes"], O.stored_norms(lay, enc["v_norm"]).astype(np.float64))
+    mask = torch.arange(L)[None, :] <= (L - n_q + torch.arange(n_q))[:, None]       # [n_q, L]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q).permute(1, 0, 2)[None], torch.tensor(kh)[None, None].expand(1, G, L, 128),
+        torch.tensor(vh)[None, None].expand(1, G, L, 128), attn_mask=mask[None, None], scale=0.09)
+    np.testing.assert_allclose(got, ref[0].permute(1, 0, 2).numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_multi_token_attention_is_causal_and_reduces_to_one_query():
+    lay, enc, buf = _packed_slice(5, 130)
+    L, n_q = 130, 4
+    q = np.random.default_rng(6).standard_normal((n_q, 2, 128))
+    out = O.decode_attention_multi(lay, q, buf, L, 0.1)
+    # the last query sees the whole cache: single-token decode attention
+    np.testing.assert_allclose(out[-1], O.decode_attention(lay, q[-1], buf, L, 0.1), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(O.decode_attention_multi(lay, q[-1:], buf, L, 0.1)[0], out[-1], rtol=1e-13)
+    # changing the keys and values after query j's position leaves query j alone, and
+    # changes the later queries
+    enc2 = {kk: vv.copy() for kk, vv in enc.items()}
+    enc2["k_codes"][L - 2:] = (enc2["k_codes"][L - 2:] + 1) % 4
+    enc2["v_norm"][L - 2:] *= 3.0
+    out2 = O.decode_attention_multi(lay, q, O.pack(lay, enc2, 192), L, 0.1)
+    np.testing.assert_array_equal(out2[:2], out[:2])
+    assert np.all(np.abs(out2[2:] - out[2:]).max(axis=(1, 2)) > 1e-6)
