@@ -256,6 +256,42 @@ bgtq_status bgtq_decode_step_paged(const bgtq_layout* layout, const void* k_new,
                                    const int* seq_lens_dev, long long max_seq_len, float softmax_scale,
                                    float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Multi-token decode attention ([BGTQ s5]: attention over the packed cache; causal as in
+ * autoregressive attention): n_q consecutive query tokens per row whose keys and values
+ * are already in the cache, as its last n_q tokens. q [batch, n_q, h_q, 128] device
+ * (q_dtype), out [batch, n_q, h_q, 128] fp32 device; query j of row b sits at position
+ * seq_len_b - n_q + j and attends to tokens 0 .. seq_len_b - n_q + j (a row with
+ * seq_len_b < n_q gives zeros for the queries that see no token). The query columns of
+ * a KV head share one tensor-core tile: (h_q / h_kv) * n_q must be <= 8
+ * (BGTQ_ERR_INVALID otherwise). Workspace: bgtq_workspace_bytes(layout, batch,
+ * h_q * n_q, h_kv, max_seq_len). n_q = 1 is bgtq_decode_attention. Other arguments,
+ * ownership and errors as bgtq_decode_attention. */
+bgtq_status bgtq_decode_attention_multi(const bgtq_layout* layout, const void* q, int q_dtype, int batch,
+                                        int n_q, int h_q, int h_kv, const void* cache,
+                                        const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                                        float softmax_scale, float* out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+/* Multi-token decode step (speculative verification, a prefill chunk): append n_new >= 1
+ * tokens per row at seq_lens_dev[b] (k_new, v_new [batch, n_new, h_kv, 128]) and attend
+ * with their own queries q [batch, n_new, h_q, 128], causal among them, in one kernel
+ * chain; out [batch, n_new, h_q, 128] fp32. seq_lens_dev holds the lengths BEFORE the
+ * call and is not modified. (h_q / h_kv) * n_new <= 8; workspace as
+ * bgtq_decode_attention_multi with n_q = n_new. Errors as bgtq_decode_step. */
+bgtq_status bgtq_decode_step_multi(const bgtq_layout* layout, const void* k_new, const void* v_new,
+                                   int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,
+                                   int h_kv, void* cache, const int* seq_lens_dev, long long capacity,
+                                   long long max_seq_len, float softmax_scale, float* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+/* bgtq_decode_step_multi on a paged cache (pool, num_pages, block table as
+ * bgtq_decode_step_paged). */
+bgtq_status bgtq_decode_step_multi_paged(const bgtq_layout* layout, const void* k_new, const void* v_new,
+                                         int kv_dtype, int n_new, const void* q, int q_dtype, int batch,
+                                         int h_q, int h_kv, void* pool, long long num_pages,
+                                         const int* block_table_dev, long long max_pages,
+                                         const int* seq_lens_dev, long long max_seq_len,
+                                         float softmax_scale, float* out, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- no-allocation variant */
 
 /* The pages have no counterpart to this call: it is a library convenience.

@@ -32,6 +32,7 @@ EXPORTED = [
     "bgtq_workspace_bytes", "bgtq_decode_attention", "bgtq_device_status",
     "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
     "bgtq_paged_pool_bytes", "bgtq_encode_append_paged", "bgtq_decode_attention_paged", "bgtq_decode_step_paged",
+    "bgtq_decode_attention_multi", "bgtq_decode_step_multi", "bgtq_decode_step_multi_paged",
 ]
 
 
@@ -83,6 +84,10 @@ def load():
         "bgtq_encode_append_paged": (I, [P, P, P, I, I, I, I, P, P, LL, P, LL, P]),
         "bgtq_decode_attention_paged": (I, [P, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
         "bgtq_decode_step_paged": (I, [P, P, P, I, I, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_attention_multi": (I, [P, P, I, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_step_multi": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_step_multi_paged": (I, [P, P, P, I, I, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t,
+                                             P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -355,6 +360,56 @@ def decode_step_paged(layout: Layout, k_new, v_new, q, cache: PagedCache, seq_le
                                          C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
                                          workspace.numel(), _stream_ptr(stream)),
            "decode_step_paged")
+
+
+def decode_attention_multi(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out, workspace,
+                           h_kv: int, softmax_scale: float | None = None, stream=None):
+    """n_q query tokens per row, causal among them: q [B, n_q, h_q, 128] CUDA (the last n_q
+    of each row's seq_lens[b] cached tokens); out [B, n_q, h_q, 128] fp32. The workspace is
+    sized by workspace_bytes(layout, B, h_q * n_q, h_kv, max_seq_len)."""
+    B_, n_q, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_multi(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, n_q, h_q,
+                                              h_kv, C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()),
+                                              capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                              C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_attention_multi")
+
+
+def decode_step_multi(layout: Layout, k_new, v_new, q, cache, seq_lens, capacity: int, max_seq_len: int, out,
+                      workspace, softmax_scale: float | None = None, stream=None):
+    """Append k_new, v_new [B, n_new, h_kv, 128] at seq_lens[b] (not advanced) and attend with
+    the new tokens' queries q [B, n_new, h_q, 128], causal among them; out [B, n_new, h_q, 128]."""
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and k_new.is_contiguous() and v_new.is_contiguous() and v_new.shape == k_new.shape
+    Bq, nq, h_q, dq = q.shape
+    assert Bq == B_ and nq == n_new and dq == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_multi(layout.handle, C.c_void_p(k_new.data_ptr()), C.c_void_p(v_new.data_ptr()),
+                                         dtype_code(k_new), n_new, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q,
+                                         h_kv, C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                         max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                         C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_step_multi")
+
+
+def decode_step_multi_paged(layout: Layout, k_new, v_new, q, cache: PagedCache, seq_lens, max_seq_len: int, out,
+                            workspace, softmax_scale: float | None = None, stream=None):
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and k_new.is_contiguous() and v_new.is_contiguous() and v_new.shape == k_new.shape
+    Bq, nq, h_q, dq = q.shape
+    assert Bq == B_ and nq == n_new and dq == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_multi_paged(layout.handle, C.c_void_p(k_new.data_ptr()),
+                                               C.c_void_p(v_new.data_ptr()), dtype_code(k_new), n_new,
+                                               C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q, h_kv,
+                                               C.c_void_p(cache.pool.data_ptr()), cache.num_pages(layout, h_kv),
+                                               C.c_void_p(cache.table.data_ptr()), cache.max_pages,
+                                               C.c_void_p(seq_lens.data_ptr()), max_seq_len, scale,
+                                               C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                               workspace.numel(), _stream_ptr(stream)),
+           "decode_step_multi_paged")
 
 
 def decode_attention_noalloc(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, out,

@@ -236,13 +236,15 @@ bgtq_status encode_impl(const bgtq_layout* L, const char* who, const void* k, co
 
 // Shape checks of the attention calls; on success *plan is the launch plan.
 bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype, int batch, int h_q, int h_kv,
-                             long long row_tokens, long long max_seq_len, float softmax_scale, const void* q,
+                             int n_q, long long row_tokens, long long max_seq_len, float softmax_scale, const void* q,
                              const int* seq_lens_dev, const void* out, void* workspace, size_t workspace_bytes,
                              DecodePlan* plan) {
   const std::string w(who);
   if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, w + ": bad dtype");
   if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
     return fail(BGTQ_ERR_INVALID, w + ": need h_q = G * h_kv with G in 1..8");
+  if (n_q < 1 || (h_q / h_kv) * n_q > kMaxG)
+    return fail(BGTQ_ERR_INVALID, w + ": need (h_q / h_kv) * n_q in 1..8");
   if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, w + ": batch * h_kv > 65535");
   if (max_seq_len < 0 || max_seq_len > row_tokens)
     return fail(BGTQ_ERR_CAPACITY, w + ": max_seq_len must be in [0, capacity]");
@@ -252,27 +254,28 @@ bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype,
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, who);
-  *plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  *plan = plan_decode(batch, h_q * n_q, h_kv, max_seq_len, sms);
   if (!workspace || workspace_bytes < plan->workspace_bytes)
     return fail(BGTQ_ERR_WORKSPACE, w + ": workspace missing or smaller than bgtq_workspace_bytes()");
   return BGTQ_OK;
 }
 
 bgtq_status decode_impl(const bgtq_layout* L, const char* who, const void* q, int q_dtype, int batch, int h_q,
-                        int h_kv, const CacheRef& c, const int* seq_lens_dev, long long max_seq_len,
+                        int h_kv, int n_q, const CacheRef& c, const int* seq_lens_dev, long long max_seq_len,
                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
   DecodePlan plan;
-  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, c.n_tiles * kTile, max_seq_len, softmax_scale,
-                                    q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
+  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
+                                    softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
-  cudaError_t e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, softmax_scale, out,
+  cudaError_t e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, softmax_scale, out,
                                 workspace, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
 
+// n_q = 1: one query per row at the newest position; n_q = n_new: the new tokens' queries.
 bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, const void* v_new, int kv_dtype,
-                      int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, const CacheRef& c,
+                      int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, int n_q, const CacheRef& c,
                       const int* seq_lens_dev, long long max_seq_len, float softmax_scale, float* out,
                       void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(kv_dtype)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad dtype");
@@ -280,11 +283,12 @@ bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, 
     return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad n_new");
   if (n_new > 0 && (!k_new || !v_new)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
   DecodePlan plan;
-  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, c.n_tiles * kTile, max_seq_len, softmax_scale,
-                                    q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
+  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
+                                    softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
   cudaError_t e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch,
-                                     h_q, h_kv, c, softmax_scale, out, workspace, static_cast<cudaStream_t>(stream));
+                                     h_q, h_kv, n_q, c, softmax_scale, out, workspace,
+                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
@@ -341,7 +345,7 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dty
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_attention", const_cast<void*>(cache), capacity, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention", q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L, "decode_attention", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -354,7 +358,7 @@ bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_step", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
-  return step_impl(L, "decode_step", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev,
+  return step_impl(L, "decode_step", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev,
                    max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -386,7 +390,7 @@ bgtq_status bgtq_decode_attention_paged(const bgtq_layout* L, const void* q, int
   if (st == BGTQ_OK) st = paged("decode_attention_paged", const_cast<void*>(pool), num_pages, block_table_dev,
                                 max_pages, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention_paged", q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L, "decode_attention_paged", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -399,8 +403,49 @@ bgtq_status bgtq_decode_step_paged(const bgtq_layout* L, const void* k_new, cons
   CacheRef c{};
   if (st == BGTQ_OK) st = paged("decode_step_paged", pool, num_pages, block_table_dev, max_pages, &c);
   if (st != BGTQ_OK) return st;
-  return step_impl(L, "decode_step_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, c,
+  return step_impl(L, "decode_step_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c,
                    seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+bgtq_status bgtq_decode_attention_multi(const bgtq_layout* L, const void* q, int q_dtype, int batch, int n_q,
+                                        int h_q, int h_kv, const void* cache, const int* seq_lens_dev,
+                                        long long capacity, long long max_seq_len, float softmax_scale, float* out,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_device(L, "decode_attention_multi");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("decode_attention_multi", const_cast<void*>(cache), capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(L, "decode_attention_multi", q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, max_seq_len,
+                     softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+bgtq_status bgtq_decode_step_multi(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype,
+                                   int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, void* cache,
+                                   const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                                   float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  bgtq_status st = check_device(L, "decode_step_multi");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("decode_step_multi", cache, capacity, &c);
+  if (st != BGTQ_OK) return st;
+  if (n_new < 1) return fail(BGTQ_ERR_INVALID, "decode_step_multi: n_new must be >= 1");
+  return step_impl(L, "decode_step_multi", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new, c,
+                   seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+bgtq_status bgtq_decode_step_multi_paged(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype,
+                                         int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv,
+                                         void* pool, long long num_pages, const int* block_table_dev,
+                                         long long max_pages, const int* seq_lens_dev, long long max_seq_len,
+                                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  bgtq_status st = check_device(L, "decode_step_multi_paged");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = paged("decode_step_multi_paged", pool, num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  if (n_new < 1) return fail(BGTQ_ERR_INVALID, "decode_step_multi_paged: n_new must be >= 1");
+  return step_impl(L, "decode_step_multi_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new,
+                   c, seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
 bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q, int h_kv,

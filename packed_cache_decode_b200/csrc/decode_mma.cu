@@ -131,7 +131,8 @@ struct SplitArgs {
   int n_ctas;             // CTAs; CTA c takes tiles [c T / n_ctas, (c+1) T / n_ctas) of the sequence
   int n_parts;            // partial slots per unit
   long long total_tiles;  // units x M
-  int h_q, h_kv, G;
+  int h_q, h_kv, G;       // G: query columns per KV head (query heads per KV head x n_q)
+  int n_q;                // query tokens per row; column n is query token n % n_q
   float* part_ml;         // [units][n_parts][G][2]
   float* part_o;          // [units][n_parts][G][128]
   float* scores;          // scores-only mode: [batch][h_q][scores_ld] logits (softmax_scale q.k_hat)
@@ -395,7 +396,7 @@ constexpr int kPrepThreads = 256;
 static_assert(kPrepThreads == enc::kEncodeThreads, "the step kernel runs both bodies");
 
 __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __restrict__ q, int q_dtype, int h_q,
-                                          int h_kv, int G, float qscale, int u, unsigned* __restrict__ frag) {
+                                          int h_kv, int G, int n_q, float qscale, int u, unsigned* __restrict__ frag) {
   __shared__ __align__(16) float qs[kMaxG * kQsLd];  // q per group at 16-byte aligned columns
   __shared__ float qr[kMaxG * kD];                   // q' in packed order
   const int tid = threadIdx.x, ng = L.n_kgroups;
@@ -421,8 +422,9 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
     const int hh = e >> 7, pe = e & (kD - 1);
     int ge = 0, pade = 0;
     while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
-    qs[hh * kQsLd + pade + pe - L.group_off[ge]] =
-        load_q(q, q_dtype, ((size_t)b * h_q + (size_t)h * G + hh) * kD + L.packed_coord[pe]);
+    // column hh: query head h G / n_q + hh / n_q at query token hh % n_q of q [b][token][head]
+    const size_t qrow = ((size_t)b * n_q + hh % n_q) * h_q + (size_t)h * (G / n_q) + hh / n_q;
+    qs[hh * kQsLd + pade + pe - L.group_off[ge]] = load_q(q, q_dtype, qrow * kD + L.packed_coord[pe]);
   }
   __syncthreads();
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -480,11 +482,11 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
 }
 
 __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
-                                                             int h_q, int h_kv, int G, float qscale,
+                                                             int h_q, int h_kv, int G, int n_q, float qscale,
                                                              unsigned* __restrict__ qfrag) {
   pdl_trigger();
   const int u = blockIdx.x;
-  prep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
+  prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
 }
 
 // First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
                                                                  int batch, const int* __restrict__ seq_lens_before,
                                                                  CacheRef cache,
                                                                  const void* __restrict__ q, int q_dtype, int h_q,
-                                                                 int h_kv, int G, float qscale,
+                                                                 int h_kv, int G, int n_q, float qscale,
                                                                  unsigned* __restrict__ qfrag, int n_enc) {
   pdl_trigger();
   const int e = blockIdx.x;
@@ -508,7 +510,7 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
     enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
   } else if (e - n_enc < batch * h_kv) {  // (a cluster launch pads the grid)
     const int u = e - n_enc;
-    prep_unit(L, q, q_dtype, h_q, h_kv, G, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
+    prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
   }
 }
 
@@ -694,10 +696,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
 #pragma unroll
           for (int j = 0; j < 4; ++j) sc[rt][j] += __shfl_xor_sync(0xffffffffu, sc[rt][j], 2);
       }
+      // Rows past a column's last visible token get -inf. The row's n_q query tokens are
+      // its last n_q cached tokens: column n (query token n % n_q) sees the tokens before
+      // S.len - (n_q - 1 - n % n_q). Warp-uniform test: only rows from the first token
+      // some column cannot see need the masks (n_q = 1: the end of the row).
+      if (gt0 - g + 16 * NRT > S.len - (a.n_q - 1)) {
+        const int c0 = NP ? 2 * (t & 1) : 2 * t;  // this lane's columns c0, c0 + 1
+        const long long vis0 = S.len - (a.n_q - 1 - c0 % a.n_q), vis1 = S.len - (a.n_q - 1 - (c0 + 1) % a.n_q);
 #pragma unroll
-      for (int rt = 0; rt < NRT; ++rt) {
-        if (gt0 + 16 * rt >= S.len) sc[rt][0] = sc[rt][1] = -INFINITY;
-        if (gt0 + 16 * rt + 8 >= S.len) sc[rt][2] = sc[rt][3] = -INFINITY;
+        for (int rt = 0; rt < NRT; ++rt) {
+          const long long r0 = gt0 + 16 * rt, r1 = r0 + 8;
+          if (r0 >= vis0) sc[rt][0] = -INFINITY;
+          if (r0 >= vis1) sc[rt][1] = -INFINITY;
+          if (r1 >= vis0) sc[rt][2] = -INFINITY;
+          if (r1 >= vis1) sc[rt][3] = -INFINITY;
+        }
       }
 
       if constexpr (SC) {
@@ -903,13 +916,15 @@ cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas
 // ------------------------------------------------------------------ combine
 constexpr int kCombThreads = 512;
 
-// One CTA per (batch row, query head): log-sum-exp merge of the unit's partials, then
+// One CTA per (batch row, query column): log-sum-exp merge of the unit's partials, then
 // o = R_V^T o'. Four threads per output dimension. R_V (not written by the split kernel)
-// is read into registers before waiting for the split kernel to finish.
+// is read into registers before waiting for the split kernel to finish. h_q counts query
+// columns (query heads x n_q); column hh of KV head h is query head h G / n_q + hh / n_q
+// at query token hh % n_q, written to out[b][token][head].
 __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* __restrict__ part_ml,
                                                               const float* __restrict__ part_o, int S,
                                                               int max_tiles, long long total_tiles, int n_ctas, int G, int h_q,
-                                                              int h_kv, const float* __restrict__ v_rot,
+                                                              int h_kv, int n_q, const float* __restrict__ v_rot,
                                                               float* __restrict__ out) {
   const int bq = blockIdx.x, b = bq / h_q, hq = bq % h_q;
   const int u = b * h_kv + hq / G, hh = hq % G;
@@ -989,7 +1004,9 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   }
   part[qtr][d] = r0 + r1;
   __syncthreads();
-  if (tid < kD) out[((size_t)b * h_q + hq) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
+  const int heads = h_q / n_q, head = (hq / G) * (G / n_q) + hh / n_q, tok = hh % n_q;
+  if (tid < kD)
+    out[(((size_t)b * n_q + tok) * heads + head) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
 }
 
 template <int VR, bool NP, bool SC, bool NH>
@@ -1026,11 +1043,13 @@ auto split_variant(int v_rate, bool np, bool sc, bool nh, Fn&& fn) {
 
 // Split and combine kernels of one call, launched as programmatic dependents of the
 // kernel that wrote the q' fragments (and, after an append, the new tokens).
-cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int batch, int h_q, int h_kv,
+// n_q query tokens per row: the split and combine kernels see h_q n_q query columns,
+// G = h_q n_q / h_kv per KV head.
+cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int batch, int h_q, int h_kv, int n_q,
                              const CacheRef& cache, const int* seq_lens, float* out, void* workspace,
                              int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
                              long long scores_ld = 0) {
-  const int G = h_q / h_kv;
+  const int hc = h_q * n_q, G = hc / h_kv;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
   // the workspace was sized for the most CTAs per SM; shared memory may allow fewer
@@ -1045,7 +1064,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const DecodePlan plan = plan_decode(batch, h_q, h_kv, (long long)wplan.max_tiles * kTile, sms, occ);
+  const DecodePlan plan = plan_decode(batch, hc, h_kv, (long long)wplan.max_tiles * kTile, sms, occ);
   if (plan.n_parts > wplan.n_parts || plan.workspace_bytes > wplan.workspace_bytes) return cudaErrorInvalidValue;
   const long long units = (long long)batch * h_kv;
   SplitArgs a;
@@ -1055,9 +1074,10 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   a.n_ctas = plan.n_ctas;
   a.n_parts = plan.n_parts;
   a.total_tiles = units * plan.max_tiles;
-  a.h_q = h_q;
+  a.h_q = hc;
   a.h_kv = h_kv;
   a.G = G;
+  a.n_q = n_q;
   // q' fragments first, then the partials in the launch plan's layout (never larger than
   // the workspace plan's)
   char* ws = static_cast<char*>(workspace);
@@ -1077,7 +1097,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   if (sc) return e;  // scores only: no merge
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(batch * h_q));
+  cfg.gridDim = dim3(unsigned(batch * hc));
   cfg.blockDim = dim3(kCombThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1086,7 +1106,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)a.part_ml, (const float*)a.part_o, plan.n_parts,
-                            plan.max_tiles, a.total_tiles, plan.n_ctas, G, h_q, h_kv, L.v_rot32, out);
+                            plan.max_tiles, a.total_tiles, plan.n_ctas, G, hc, h_kv, n_q, L.v_rot32, out);
 }
 
 }  // namespace
@@ -1114,14 +1134,14 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
 }
 
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                          int h_q, int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale,
+                          int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
                           float* out, void* workspace, cudaStream_t stream) {
-  const int G = h_q / h_kv;
+  const int G = h_q * n_q / h_kv;
   qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+      L, q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, out, workspace, 0, false, stream);
+  return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens, out, workspace, 0, false, stream);
 }
 
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
@@ -1129,24 +1149,24 @@ cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void
                           long long scores_ld, void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
   qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+      L, q, q_dtype, h_q, h_kv, G, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens, nullptr, workspace, 0, false, stream,
+  return launch_attention(L, plan, batch, h_q, h_kv, 1, cache, seq_lens, nullptr, workspace, 0, false, stream,
                           scores, scores_ld);
 }
 
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
-                               int batch, int h_q, int h_kv, const CacheRef& cache, float softmax_scale, float* out,
-                               void* workspace, cudaStream_t stream) {
-  const int G = h_q / h_kv;
+                               int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
+                               float* out, void* workspace, cudaStream_t stream) {
+  const int G = h_q * n_q / h_kv;
   const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
   cudaError_t e;
   if (!L.norm_correct) {
     step_prep_kernel<false><<<unsigned(n_enc + batch * h_kv), kPrepThreads, 0, stream>>>(
         L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype,
-        h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
+        h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
     e = cudaGetLastError();
   } else {
     // norm correction: clusters of the four encode parts of a token; the q' blocks
@@ -1164,11 +1184,11 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, step_prep_kernel<true>, L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache,
-                           q, q_dtype, h_q, h_kv, G, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
+                           q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
                            int(n_enc));
   }
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, cache, seq_lens_before, out, workspace, n_new,
+  return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens_before, out, workspace, n_new,
                           n_new > 0, stream);
 }
 

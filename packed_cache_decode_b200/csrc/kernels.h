@@ -26,17 +26,20 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
 cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, int dtype, int batch,
                              int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream);
 
+// n_q query tokens per row (q [batch][n_q][h_q][128], out likewise), causal among them;
+// the plan is made for h_q n_q query columns.
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
-                          int h_q, int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale,
+                          int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
                           float* out, void* workspace, cudaStream_t stream);
 
 // Append n_new tokens at seq_lens_before[b] and attend over seq_lens_before[b] + n_new
 // tokens: the encode kernel, then the split kernel as its programmatic dependent (only the
-// tile receiving the new tokens waits for the encode), then the combine.
+// tile receiving the new tokens waits for the encode), then the combine. n_q = 1: one
+// query per row at the newest position; n_q = n_new: the new tokens' own queries.
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
-                               int batch, int h_q, int h_kv, const CacheRef& cache, float softmax_scale, float* out,
-                               void* workspace, cudaStream_t stream);
+                               int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
+                               float* out, void* workspace, cudaStream_t stream);
 
 // Logits only: scores[(b h_q + hq) scores_ld + t] = softmax_scale q . k_hat_t for every
 // cached token t < seq_lens[b] (the q-preparation kernel, then the split kernel in its
