@@ -174,7 +174,9 @@ def lloyd_max(bits: int, tol: float = 1e-15, max_iter: int = 200000):
 
 
 def lloyd_max_mse_table(max_bits: int = 4) -> dict:
-    return {b: lloyd_max(b)[2] for b in range(1, max_bits + 1)}
+    """D(b) for b = 0..max_bits. D(0) = 1: a block given no bits is not stored and decodes
+    to 0, the error of predicting 0 for an N(0,1) coordinate is its variance."""
+    return {0: 1.0, **{b: lloyd_max(b)[2] for b in range(1, max_bits + 1)}}
 
 
 # ----------------------------------------------------------------------------------------
@@ -306,6 +308,11 @@ class Layout:
             p += d
         return out
 
+    @property
+    def n_packed(self):
+        """Stored key dimensions (128 minus two per rate-0 block)."""
+        return int(sum(len(c) for _, c in self.groups))
+
     def packed_rates(self):
         return np.concatenate([np.full(len(c), r) for r, c in self.groups])
 
@@ -315,10 +322,10 @@ class Layout:
 
 def group_coordinates(k_rates) -> list:
     """Equal-rate blocks form one group [BGTQ sentence 5]; descending rate, blocks ascending,
-    coordinate j before j+64 inside block j."""
+    coordinate j before j+64 inside block j. Rate-0 blocks are in no group (not stored)."""
     rates = np.asarray(k_rates)
     out = []
-    for r in sorted(set(int(x) for x in rates), reverse=True):
+    for r in sorted(set(int(x) for x in rates if x > 0), reverse=True):
         blocks = [j for j in range(N_BLOCKS) if rates[j] == r]
         coords = np.array([c for j in blocks for c in (j, j + N_BLOCKS)], dtype=np.int64)
         out.append((r, coords))
@@ -326,9 +333,12 @@ def group_coordinates(k_rates) -> list:
 
 
 def make_layout(k_rates, v_rate: int, seed: int, norm_correct: bool = False, norm_fp16: bool = False) -> Layout:
-    """K record = a whole number of bytes: the 64 block rates must sum to a multiple of 4."""
-    if len(k_rates) != N_BLOCKS or (2 * int(np.sum(k_rates))) % 8 or not 1 <= v_rate <= 4:
-        raise ValueError("64 block rates summing to a multiple of 4, and a V rate in 1..4")
+    """K record = a whole number of bytes: the 64 block rates (0..4, at least one block
+    coded) must sum to a multiple of 4."""
+    r = np.asarray(k_rates)
+    if (len(r) != N_BLOCKS or (2 * int(np.sum(r))) % 8 or not 1 <= v_rate <= 4 or r.min() < 0 or r.max() > 4
+            or r.max() < 1):
+        raise ValueError("64 block rates in 0..4, not all 0, summing to a multiple of 4, and a V rate in 1..4")
     groups = group_coordinates(k_rates)
     k_rot = [haar_rotation(seed, r, len(c)) for r, c in groups]
     v_rot = haar_rotation(seed, 0, HEAD_DIM)
@@ -555,7 +565,7 @@ def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
     kb, vb, ng, br = layout.k_record_bytes, layout.v_record_bytes, layout.n_kgroups, layout.v_rate
     # K area
     kcodes = np.zeros((ntile * TILE_TOKENS, HEAD_DIM), dtype=np.int64)
-    kcodes[:n] = enc["k_codes"]
+    kcodes[:n, :layout.n_packed] = enc["k_codes"]
     kcodes = kcodes.reshape(ntile, 8, 8, HEAD_DIM)          # [tile, m, g, dim]: token g + 8 m
     for p0, npairs, r, off in layout.k_quads():
         blk = np.zeros((ntile, 128 * npairs * r), dtype=np.uint8)
@@ -642,7 +652,7 @@ def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
     kn = kn.transpose(0, 2, 1).reshape(-1, ng)
     base += nb * TILE_TOKENS * ng
     vn = t[:, base:base + nb * TILE_TOKENS].copy().view(nt).reshape(-1)
-    return {"k_codes": kc[:n], "k_norms": kn[:n].astype(np.float64),
+    return {"k_codes": kc[:n, :layout.n_packed], "k_norms": kn[:n].astype(np.float64),
             "v_codes": vc.reshape(-1, HEAD_DIM)[:n], "v_norm": vn[:n].astype(np.float64)}
 
 

@@ -569,3 +569,52 @@ def test_multi_token_attention_is_causal_and_reduces_to_one_query():
     out2 = O.decode_attention_multi(lay, q, O.pack(lay, enc2, 192), L, 0.1)
     np.testing.assert_array_equal(out2[:2], out[:2])
     assert np.all(np.abs(out2[2:] - out[2:]).max(axis=(1, 2)) > 1e-6)
+
+
+# -------------------------------------------------------------------- rate-0 blocks ----
+def test_greedy_with_rate_zero_equals_exhaustive_optimum():
+    """With D(0) = 1 (an uncoded N(0,1) coordinate decodes to 0) the gains still diminish
+    (1 - D(1) > D(1) - D(2) > ...), so largest-marginal-gain allocation from rate 0 is the
+    exhaustive optimum of the proxy [BGTQ sentence 4]."""
+    D = O.lloyd_max_mse_table()
+    assert D[0] == 1.0 and D[0] - D[1] > D[1] - D[2] > D[2] - D[3] > D[3] - D[4] > 0
+    rng = np.random.default_rng(2)
+    cases = 0
+    for n in (1, 2, 3, 4, 5):
+        s = rng.exponential(size=n) * rng.choice([1, 10, 100], size=n)
+        for budget in range(0, 4 * n + 1):
+            g = O.greedy_rates(s, D, 0, 4, budget)
+            best, args = O.brute_force_rates(s, D, 0, 4, budget)
+            assert O.proxy_objective(s, g, D) == pytest.approx(best, rel=1e-12, abs=1e-15)
+            if len(args) == 1:
+                assert tuple(g) == args[0]
+            cases += 1
+    assert cases > 40
+
+
+def test_rate_zero_blocks_are_not_stored_and_decode_to_zero():
+    """A rate-0 block is in no group: its two coordinates take no code bits, the group
+    norms cover the coded coordinates only, and they decode to exactly 0; the coded
+    groups keep the Lloyd-Max distortion of their rate."""
+    rates = np.array([0] * 8 + [1] * 16 + [2] * 16 + [3] * 16 + [4] * 8)    # sum 128: K2
+    lay = O.make_layout(rates, 2, 9)
+    assert [r for r, _ in lay.groups] == [4, 3, 2, 1] and lay.n_packed == 128 - 16
+    zero = np.r_[0:8, 64:72]
+    assert not set(zero) & set(np.concatenate([c for _, c in lay.groups]))
+    assert lay.k_record_bytes == (16 * 2 * 1 + 16 * 2 * 2 + 16 * 2 * 3 + 8 * 2 * 4) // 8 == 32
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((3000, 128))
+    enc = O.encode(lay, x, x)
+    assert enc["k_codes"].shape == (3000, 112)
+    c1 = lay.groups[-1][1]
+    np.testing.assert_allclose(enc["k_norms"][:, -1], np.linalg.norm(x[:, c1], axis=1), rtol=1e-14)
+    kh, _ = O.reconstruct(lay, enc["k_codes"], enc["k_norms"], enc["v_codes"], enc["v_norm"])
+    assert np.all(kh[:, zero] == 0.0)
+    for r, coords in lay.groups:
+        rel = np.sum((kh[:, coords] - x[:, coords]) ** 2) / np.sum(x[:, coords] ** 2)
+        assert rel == pytest.approx(O.lloyd_max(r)[2], rel=0.15)
+    buf = O.pack(lay, enc, 3008)
+    u = O.unpack(lay, buf, 3000)
+    np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
+    with pytest.raises(ValueError):
+        O.make_layout(np.zeros(64, dtype=int), 2, 0)
