@@ -373,7 +373,8 @@ def run_mae(args):
     bit budget, on the 8B- and 3B-shaped generators (8192 cached tokens, one layer): the
     logits come from bgtq_decode_scores over each packed cache, the exact ones from the
     unquantised keys (fp64). Reports the mean absolute logit error of both layouts, and of
-    the block allocation with norm correction and/or fp16 norms, with each layout's
+    the block allocation with norm correction and/or fp16 norms and of the allocation that
+    may leave blocks uncoded (rates from 0), with each layout's
     resident bytes per (token, KV head) and its footprint ratio to an fp16 K+V record
     (512 bytes)."""
     dev = torch.device("cuda", 0)
@@ -392,7 +393,10 @@ def run_mae(args):
         line = {"mode": "mae", "workload": wl.name, "tokens": wl.length, "k_bits": wl.k_bits,
                 "block_rates": {str(r): int((rates == r).sum()) for r in sorted(set(rates.tolist()))}}
         uni = np.full(64, wl.k_bits)
+        rates0 = B.plan_layer_rates(q_cal.numpy(), k_cal.numpy(), wl.k_bits, min_rate=0)
+        line["block_rates_from_0"] = {str(r): int((rates0 == r).sum()) for r in sorted(set(rates0.tolist()))}
         variants = (("block_gtq", rates, False, False), ("uniform", uni, False, False),
+                    ("block_gtq_rate0", rates0, False, False),
                     ("block_gtq_nc", rates, True, False), ("block_gtq_fp16", rates, False, True),
                     ("block_gtq_nc_fp16", rates, True, True), ("uniform_nc", uni, True, False))
         for tag, rr, nc, fp16 in variants:

@@ -111,6 +111,7 @@ typedef struct {
   unsigned long long seed;
   unsigned flags;                     /* BGTQ_LAYOUT_* options of bgtq_layout_create_ex */
   int norm_bytes;                     /* 4 (fp32 norms) or 2 (fp16) */
+  int n_packed;                       /* stored key dimensions: 128 - 2 x (rate-0 blocks) */
 } bgtq_layout_info;
 
 /* Message of the last failing call on this host thread ("" if none). */
@@ -135,13 +136,16 @@ bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q,
  * adds one bit to the block with the largest score[j] * (D[b_j] - D[b_j + 1]) among
  * blocks below max_rate (ties: lowest j) until the rates sum to total_bits.
  * distortion: array indexed by rate (entries min_rate..max_rate used), or NULL for the
- * Gaussian Lloyd-Max MSE. 1 <= min_rate <= max_rate <= 4. BGTQ_ERR_INFEASIBLE if
+ * Gaussian Lloyd-Max MSE with D(0) = 1 (a rate-0 block is not stored and decodes to 0).
+ * 0 <= min_rate <= max_rate <= 4, max_rate >= 1. BGTQ_ERR_INFEASIBLE if
  * total_bits is outside [n_blocks*min_rate, n_blocks*max_rate]. rates_out[n_blocks]. */
 bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate, int max_rate,
                                 long long total_bits, const double* distortion, int* rates_out);
 
-/* Layout of one layer [BGTQ s5]: k_rates[64] in 1..4 summing to a multiple of 4 (so a K
- * record is whole bytes), v_rate in 1..4, seed of the rotations. Groups equal-rate blocks,
+/* Layout of one layer [BGTQ s5]: k_rates[64] in 0..4 summing to a multiple of 4 (so a K
+ * record is whole bytes) with at least one block coded, v_rate in 1..4, seed of the
+ * rotations. A rate-0 block is not stored: it joins no group and its two coordinates
+ * decode to 0 (they take no part in the scores). Groups equal-rate blocks,
  * draws one seeded Haar rotation per K group (Philox4x32-10 stream = rate) and one for V
  * (stream 0), and builds the Lloyd-Max tables. Host only. */
 bgtq_status bgtq_layout_create(const int* k_rates, int v_rate, unsigned long long seed,

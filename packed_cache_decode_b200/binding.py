@@ -41,7 +41,7 @@ class LayoutInfo(C.Structure):
                 ("group_rate", C.c_int * 4), ("group_dim", C.c_int * 4), ("v_rate", C.c_int),
                 ("k_record_bytes", C.c_int), ("v_record_bytes", C.c_int), ("bytes_per_token", C.c_int),
                 ("tile_tokens", C.c_int), ("tile_bytes", C.c_int), ("seed", C.c_ulonglong),
-                ("flags", C.c_uint), ("norm_bytes", C.c_int)]
+                ("flags", C.c_uint), ("norm_bytes", C.c_int), ("n_packed", C.c_int)]
 
 
 class BgtqError(RuntimeError):

@@ -187,6 +187,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     D.n_kquads = qi;
   }
   D.n_kgroups = ng;
+  D.n_packed = L->n_packed;
   D.v_rate = L->v_rate;
   D.k_record_bytes = L->k_record_bytes;
   D.tile_bytes = L->tile_bytes;

@@ -21,6 +21,7 @@ constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32
 // Everything a kernel needs about one layer's packing, passed by value.
 struct DevLayout {
   int n_kgroups;
+  int n_packed;         // stored key dimensions (packed dims n_packed..127 do not exist)
   int v_rate;
   int k_record_bytes;   // Kb
   int tile_bytes;
@@ -113,6 +114,7 @@ struct bgtq_layout {
   int k_record_bytes, v_record_bytes, bytes_per_token, tile_bytes;
   unsigned flags;   // BGTQ_LAYOUT_* options
   int norm_bytes;   // 4 or 2
+  int n_packed;     // stored key dimensions: 128 minus two per rate-0 block
   // device copy
   int device = -1;
   void* dev_block = nullptr;

@@ -410,7 +410,8 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   int g = 0, pad = 0;
   while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
   const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
-  const int n4 = ld / 4, c0 = ksplit ? half * ((n4 + 1) / 2) : 0, c1 = ksplit ? min(n4, c0 + (n4 + 1) / 2) : n4;
+  // packed dims past n_packed (rate-0 blocks) have no row: no loads, q' = 0
+  const int n4 = p < L.n_packed ? ld / 4 : 0, c0 = ksplit ? half * ((n4 + 1) / 2) : 0, c1 = ksplit ? min(n4, c0 + (n4 + 1) / 2) : n4;
   const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld) + c0;
   constexpr int kPre = 16;
   float4 r[kPre];
@@ -420,6 +421,7 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   __syncthreads();
   for (int e = tid; e < G * kD; e += kPrepThreads) {
     const int hh = e >> 7, pe = e & (kD - 1);
+    if (pe >= L.n_packed) continue;
     int ge = 0, pade = 0;
     while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
     // column hh: query head h G / n_q + hh / n_q at query token hh % n_q of q [b][token][head]

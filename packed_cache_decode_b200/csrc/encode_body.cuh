@@ -159,7 +159,8 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   __shared__ double part_sq[kEncodeParts][kMaxGroups + 1];  // NC, part 0: the parts' sums
 
   const size_t base = (((size_t)b * n_new + t) * h_kv + h) * kD;
-  if (tid < kD) xp[tid] = load_elem(k, dtype, base + L.packed_coord[tid]);  // keys in packed order
+  // keys in packed order (packed dims past n_packed belong to rate-0 blocks: not stored)
+  if (tid < kD) xp[tid] = tid < L.n_packed ? load_elem(k, dtype, base + L.packed_coord[tid]) : 0.0;
   else xv[tid - kD] = load_elem(v, dtype, base + tid - kD);
   __syncthreads();
 
@@ -183,6 +184,7 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   const int o = tid >> 2, q = tid & 3;
   const bool is_key = o < 32;
   const int p = 32 * part + (o & 31);
+  const bool live = !is_key || p < L.n_packed;  // a key output past n_packed does not exist
   int g = 0;
   if (is_key)
     while (g + 1 < L.n_kgroups && p >= L.group_off[g + 1]) ++g;
@@ -191,7 +193,7 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   const int i = p - off;
   const double* col = (is_key ? L.k_rot64[g] : L.v_rot64) + i;  // element (i, j) at j * d + i
   const double* x = is_key ? xp + off : xv;
-  const int j0 = (q * d) / 4, j1 = ((q + 1) * d) / 4;
+  const int j0 = live ? (q * d) / 4 : 0, j1 = live ? ((q + 1) * d) / 4 : 0;
   double a[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
   int j = j0;
   for (; j + 8 <= j1; j += 8) {
@@ -204,7 +206,7 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
 
   if constexpr (!NC) {
-    if (q != 0) return;
+    if (q != 0 || !live) return;
     const double nrm = gnorm[is_key ? g : kMaxGroups];
     const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
     const int r = is_key ? L.group_rate[g] : L.v_rate;
@@ -222,7 +224,8 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
     return;
   }
   const int tt = int(pos % kTile);
-  if (q == 0) {
+  if (q == 0 && !live) csq[o] = 0.0;
+  if (q == 0 && live) {
     const double nrm = gnorm[is_key ? g : kMaxGroups];
     const double y = nrm > 0.0 ? sqrt(double(d)) * acc / nrm : 0.0;
     const int r = is_key ? L.group_rate[g] : L.v_rate;

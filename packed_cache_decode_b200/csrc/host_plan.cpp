@@ -209,13 +209,14 @@ bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q, const 
 bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate, int max_rate,
                                 long long total_bits, const double* distortion, int* rates_out) {
   if (!score || !rates_out || n_blocks <= 0) return fail(BGTQ_ERR_INVALID, "allocate_rates: bad arguments");
-  if (!valid_rate(min_rate) || !valid_rate(max_rate) || min_rate > max_rate)
-    return fail(BGTQ_ERR_INVALID, "allocate_rates: need 1 <= min_rate <= max_rate <= 4");
+  if (min_rate < 0 || !valid_rate(max_rate) || min_rate > max_rate)
+    return fail(BGTQ_ERR_INVALID, "allocate_rates: need 0 <= min_rate <= max_rate <= 4, max_rate >= 1");
   if (total_bits < (long long)n_blocks * min_rate || total_bits > (long long)n_blocks * max_rate)
     return fail(BGTQ_ERR_INFEASIBLE, "allocate_rates: budget outside [n*min_rate, n*max_rate]");
   double D[6] = {0, 0, 0, 0, 0, 0};
   for (int r = min_rate; r <= max_rate; ++r) {
     if (distortion) D[r] = distortion[r];
+    else if (r == 0) D[r] = 1.0;  // an uncoded N(0,1) coordinate decodes to 0: its variance
     else lloyd_max_host(r, nullptr, nullptr, &D[r]);
   }
   for (int j = 0; j < n_blocks; ++j) {
@@ -250,10 +251,11 @@ bgtq_status bgtq_layout_create_ex(const int* k_rates, int v_rate, unsigned long 
     return fail(BGTQ_ERR_INVALID, "layout_create: unknown option flag");
   int sum = 0;
   for (int j = 0; j < kBlocks; ++j) {
-    if (!valid_rate(k_rates[j])) return fail(BGTQ_ERR_INVALID, "layout_create: key rates must be 1..4");
+    if (k_rates[j] < 0 || k_rates[j] > 4) return fail(BGTQ_ERR_INVALID, "layout_create: key rates must be 0..4");
     sum += k_rates[j];
   }
   if ((2 * sum) % 8) return fail(BGTQ_ERR_INVALID, "layout_create: key rates must sum to a multiple of 4");
+  if (sum == 0) return fail(BGTQ_ERR_INVALID, "layout_create: at least one key block must be coded");
   if (!valid_rate(v_rate)) return fail(BGTQ_ERR_INVALID, "layout_create: v_rate must be 1..4");
   bgtq_layout* L = new (std::nothrow) bgtq_layout();
   if (!L) return fail(BGTQ_ERR_NOMEM, "layout_create: out of host memory");
@@ -283,6 +285,8 @@ bgtq_status bgtq_layout_create_ex(const int* k_rates, int v_rate, unsigned long 
     ++ng;
   }
   L->n_kgroups = ng;
+  L->n_packed = pd;  // rate-0 blocks are in no group: their coordinates are not stored
+  for (int p = pd; p < kD; ++p) L->packed_coord[p] = 0;
   for (int g = ng; g < kMaxGroups; ++g) L->group_rate[g] = L->group_dim[g] = L->group_off[g] = L->group_bitoff[g] = 0;
   for (int g = 0; g < ng; ++g) haar_rotation(seed, uint32_t(L->group_rate[g]), L->group_dim[g], L->rot[g]);
   haar_rotation(seed, 0u, kD, L->rot[ng]);
@@ -318,6 +322,7 @@ bgtq_status bgtq_layout_get_info(const bgtq_layout* L, bgtq_layout_info* info) {
   info->seed = L->seed;
   info->flags = L->flags;
   info->norm_bytes = L->norm_bytes;
+  info->n_packed = L->n_packed;
   return BGTQ_OK;
 }
 

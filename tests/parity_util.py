@@ -31,6 +31,7 @@ class Case:
     capacity: int | None = None
     norm_correct: bool = False
     norm_fp16: bool = False
+    min_rate: int = 1            # 0: the allocation may leave blocks uncoded
 
     @property
     def cap(self):
@@ -41,7 +42,7 @@ def oracle_rates(model, case: Case) -> np.ndarray:
     """Per-layer rates from 256 calibration tokens (seed + 1), computed by the oracle."""
     q_cal, k_cal = synth.make_calibration(model, 256, case.seed + 1, case.theta)
     s = O.block_energy(q_cal.double().numpy(), k_cal.double().numpy())
-    return O.greedy_rates(s, O.lloyd_max_mse_table(), 1, 4, 64 * case.k_bits)
+    return O.greedy_rates(s, O.lloyd_max_mse_table(), case.min_rate, 4, 64 * case.k_bits)
 
 
 def build_inputs(case: Case):

@@ -32,6 +32,9 @@ CASES = {
     "gqa2_len1": Case(2, 1, 1, 1, 2, 2, torch.float32, 5e5, 7),
     "gqa1_len64": Case(1, 1, 2, 64, 2, 3, torch.float32, 5e5, 8),
     "gqa1_len65": Case(3, 3, 1, 65, 2, 1, torch.float32, 5e5, 9),
+    # allocations from rate 0: some blocks are not stored
+    "gqa4_k2v2_rate0": Case(16, 4, 2, 700, 2, 2, torch.bfloat16, 5e5, 10, min_rate=0),
+    "gqa8_k1v2_rate0": Case(16, 2, 1, 300, 1, 2, torch.bfloat16, 1e6, 11, min_rate=0),
 }
 
 

@@ -150,3 +150,26 @@ def test_layout_options_match_oracle_bytes(lib, flags):
     h = C.c_void_p()
     assert lib.bgtq_layout_create_ex(r.ctypes.data_as(C.c_void_p), 3, 9, 4, C.byref(h)) == B.ERR_INVALID
     assert not h.value
+
+
+def test_rate_zero_layout_and_allocation_match_oracle(lib):
+    """Rate-0 blocks: the allocation from rate 0 equals the oracle's greedy (D(0) = 1), the
+    layout stores 128 - 2 x (rate-0 blocks) key dimensions in the oracle's byte count, and
+    an all-zero rate vector is refused."""
+    rng = np.random.default_rng(12)
+    s = rng.exponential(size=64) * rng.choice([0.01, 1, 100], size=64)
+    for bits in (1, 2, 3):
+        got = B.allocate_rates(s, 0, 4, 64 * bits)
+        want = O.greedy_rates(s, O.lloyd_max_mse_table(), 0, 4, 64 * bits)
+        np.testing.assert_array_equal(got, want)
+        assert (got == 0).any()
+        lay, olay = B.Layout(got, 2, 5), O.make_layout(got, 2, 5)
+        assert lay.info.n_packed == olay.n_packed == 128 - 2 * int((got == 0).sum())
+        assert lay.info.bytes_per_token == olay.bytes_per_token
+        assert lay.info.n_kgroups == olay.n_kgroups
+        coords = np.zeros(128, dtype=np.int32)
+        assert lib.bgtq_layout_coords(lay.handle, coords.ctypes.data_as(C.c_void_p)) == B.OK
+        np.testing.assert_array_equal(coords[:olay.n_packed], olay.packed_coords())
+    h = C.c_void_p()
+    zero = np.zeros(64, dtype=np.int32)
+    assert lib.bgtq_layout_create(zero.ctypes.data_as(C.c_void_p), 2, 0, C.byref(h)) == B.ERR_INVALID
