@@ -203,6 +203,21 @@ def block_energy(q_cal: np.ndarray, k_cal: np.ndarray) -> np.ndarray:
     return s
 
 
+def block_energy_heads(q_cal: np.ndarray, k_cal: np.ndarray) -> np.ndarray:
+    """The energy score of each KV head on its own, [h_kv, 64]: the terms that
+    ``block_energy`` sums over KV heads [BGTQ sentence 3], for an allocation per KV head."""
+    q = np.asarray(q_cal, dtype=np.float64)
+    k = np.asarray(k_cal, dtype=np.float64)
+    h_q, h_kv = q.shape[1], k.shape[1]
+    g = h_q // h_kv
+    out = np.zeros((h_kv, N_BLOCKS))
+    for h in range(h_kv):
+        qh, kh = q[:, h * g:(h + 1) * g, :], k[:, h, :]
+        out[h] = ((qh[..., :N_BLOCKS] ** 2 + qh[..., N_BLOCKS:] ** 2).mean(axis=(0, 1))
+                  * (kh[..., :N_BLOCKS] ** 2 + kh[..., N_BLOCKS:] ** 2).mean(axis=0))
+    return out
+
+
 def proxy_objective(score, rates, distortion) -> float:
     """Separable integer proxy sum_j s_j D(b_j) [BGTQ sentence 4]."""
     return float(sum(score[j] * distortion[rates[j]] for j in range(len(rates))))

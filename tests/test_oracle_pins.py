@@ -618,3 +618,21 @@ def test_rate_zero_blocks_are_not_stored_and_decode_to_zero():
     np.testing.assert_array_equal(u["k_codes"], enc["k_codes"])
     with pytest.raises(ValueError):
         O.make_layout(np.zeros(64, dtype=int), 2, 0)
+
+
+# ------------------------------------------------------------ per-KV-head allocation ----
+def test_per_head_energy_sums_to_the_layer_score_and_follows_each_head():
+    """The per-KV-head scores add up to the layer score, and a head whose keys (and only
+    its keys) are scaled by c in block j has its own score for j multiplied by c^2 while
+    the other heads' scores stay put."""
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((40, 8, 128))
+    k = rng.standard_normal((30, 4, 128))
+    per = O.block_energy_heads(q, k)
+    np.testing.assert_allclose(per.sum(axis=0), O.block_energy(q, k), rtol=1e-13)
+    k2 = k.copy()
+    k2[:, 2, [5, 69]] *= 3.0
+    per2 = O.block_energy_heads(q, k2)
+    assert per2[2, 5] == pytest.approx(9.0 * per[2, 5], rel=1e-12)
+    np.testing.assert_allclose(np.delete(per2, 2, axis=0), np.delete(per, 2, axis=0), rtol=0, atol=0)
+    np.testing.assert_allclose(np.delete(per2[2], 5), np.delete(per[2], 5), rtol=0, atol=0)
