@@ -131,6 +131,12 @@ bgtq_status bgtq_lloyd_max(int bits, double* centroids, double* thresholds, doub
  * heads of |q_j|^2) x (mean over calibration keys of |k_j|^2). */
 bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q,
                               const float* k_cal, long long n_k, int h_kv, double* score_out);
+/* The same energy score per KV head, for a rate allocation per KV head: score_out
+ * [h_kv * 64], score_out[h * 64 + j] = the term of KV head h in bgtq_block_energy (whose
+ * score is their sum). A per-head allocation gives each KV head its own layout; such
+ * heads are cached and decoded with one call per KV head (h_kv = 1). */
+bgtq_status bgtq_block_energy_heads(const float* q_cal, long long n_q, int h_q,
+                                    const float* k_cal, long long n_k, int h_kv, double* score_out);
 
 /* Largest-marginal-gain rate allocation [BGTQ s4]. Rates start at min_rate; each step
  * adds one bit to the block with the largest score[j] * (D[b_j] - D[b_j + 1]) among

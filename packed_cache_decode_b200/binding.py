@@ -33,6 +33,7 @@ EXPORTED = [
     "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
     "bgtq_paged_pool_bytes", "bgtq_encode_append_paged", "bgtq_decode_attention_paged", "bgtq_decode_step_paged",
     "bgtq_decode_attention_multi", "bgtq_decode_step_multi", "bgtq_decode_step_multi_paged",
+    "bgtq_block_energy_heads",
 ]
 
 
@@ -63,6 +64,7 @@ def load():
         "bgtq_version": (I, []),
         "bgtq_lloyd_max": (I, [I, P, P, P]),
         "bgtq_block_energy": (I, [P, LL, I, P, LL, I, P]),
+        "bgtq_block_energy_heads": (I, [P, LL, I, P, LL, I, P]),
         "bgtq_allocate_rates": (I, [P, I, I, I, LL, P, P]),
         "bgtq_layout_create": (I, [P, I, U, C.POINTER(P)]),
         "bgtq_layout_create_ex": (I, [P, I, U, C.c_uint, C.POINTER(P)]),
@@ -121,6 +123,16 @@ def block_energy(q_cal, k_cal) -> np.ndarray:
     s = np.zeros(64)
     _check(load().bgtq_block_energy(_ptr(q), q.shape[0], q.shape[1], _ptr(k), k.shape[0], k.shape[1], _ptr(s)),
            "block_energy")
+    return s
+
+
+def block_energy_heads(q_cal, k_cal) -> np.ndarray:
+    """Energy score per KV head, [h_kv, 64] (their sum is block_energy)."""
+    q = np.ascontiguousarray(q_cal, dtype=np.float32)
+    k = np.ascontiguousarray(k_cal, dtype=np.float32)
+    s = np.zeros((k.shape[1], 64))
+    _check(load().bgtq_block_energy_heads(_ptr(q), q.shape[0], q.shape[1], _ptr(k), k.shape[0], k.shape[1], _ptr(s)),
+           "block_energy_heads")
     return s
 
 
@@ -431,3 +443,10 @@ def plan_layer_rates(q_cal, k_cal, avg_bits: int, min_rate: int = 1, max_rate: i
     """Energy score + largest-marginal-gain allocation for one layer (library calls)."""
     s = block_energy(q_cal, k_cal)
     return allocate_rates(s, min_rate, max_rate, 64 * avg_bits)
+
+
+def plan_head_rates(q_cal, k_cal, avg_bits: int, min_rate: int = 1, max_rate: int = 4) -> np.ndarray:
+    """Rates per KV head, [h_kv, 64]: each head's own energy score and allocation (each row
+    is the rate vector of that head's own layout)."""
+    s = block_energy_heads(q_cal, k_cal)
+    return np.stack([allocate_rates(s[h], min_rate, max_rate, 64 * avg_bits) for h in range(s.shape[0])])

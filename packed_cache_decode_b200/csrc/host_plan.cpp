@@ -178,13 +178,14 @@ bgtq_status bgtq_lloyd_max(int bits, double* centroids, double* thresholds, doub
   return BGTQ_OK;
 }
 
-bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q, const float* k_cal,
-                              long long n_k, int h_kv, double* score_out) {
-  if (!q_cal || !k_cal || !score_out) return fail(BGTQ_ERR_INVALID, "block_energy: null pointer");
+namespace {
+// Energy score of every KV head [BGTQ s3]: per_head[h * 64 + j].
+bgtq_status energy_per_head(const char* who, const float* q_cal, long long n_q, int h_q, const float* k_cal,
+                            long long n_k, int h_kv, double* per_head) {
+  if (!q_cal || !k_cal || !per_head) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
   if (n_q <= 0 || n_k <= 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv)
-    return fail(BGTQ_ERR_INVALID, "block_energy: need n_q, n_k > 0 and h_q a multiple of h_kv");
+    return fail(BGTQ_ERR_INVALID, std::string(who) + ": need n_q, n_k > 0 and h_q a multiple of h_kv");
   const int grp = h_q / h_kv;
-  for (int j = 0; j < kBlocks; ++j) score_out[j] = 0.0;
   std::vector<double> qe(kBlocks), ke(kBlocks);
   for (int h = 0; h < h_kv; ++h) {
     std::fill(qe.begin(), qe.end(), 0.0);
@@ -201,9 +202,28 @@ bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q, const 
         ke[j] += double(x[j]) * x[j] + double(x[j + kBlocks]) * x[j + kBlocks];
     }
     for (int j = 0; j < kBlocks; ++j)
-      score_out[j] += (qe[j] / (double(n_q) * grp)) * (ke[j] / double(n_k));
+      per_head[size_t(h) * kBlocks + j] = (qe[j] / (double(n_q) * grp)) * (ke[j] / double(n_k));
   }
   return BGTQ_OK;
+}
+}  // namespace
+
+bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q, const float* k_cal,
+                              long long n_k, int h_kv, double* score_out) {
+  if (!score_out) return fail(BGTQ_ERR_INVALID, "block_energy: null pointer");
+  std::vector<double> per(size_t(h_kv > 0 ? h_kv : 0) * kBlocks);
+  const bgtq_status st = energy_per_head("block_energy", q_cal, n_q, h_q, k_cal, n_k, h_kv, per.data());
+  if (st != BGTQ_OK) return st;
+  for (int j = 0; j < kBlocks; ++j) {
+    score_out[j] = 0.0;
+    for (int h = 0; h < h_kv; ++h) score_out[j] += per[size_t(h) * kBlocks + j];
+  }
+  return BGTQ_OK;
+}
+
+bgtq_status bgtq_block_energy_heads(const float* q_cal, long long n_q, int h_q, const float* k_cal,
+                                    long long n_k, int h_kv, double* score_out) {
+  return energy_per_head("block_energy_heads", q_cal, n_q, h_q, k_cal, n_k, h_kv, score_out);
 }
 
 bgtq_status bgtq_allocate_rates(const double* score, int n_blocks, int min_rate, int max_rate,

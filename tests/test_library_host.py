@@ -173,3 +173,15 @@ def test_rate_zero_layout_and_allocation_match_oracle(lib):
     h = C.c_void_p()
     zero = np.zeros(64, dtype=np.int32)
     assert lib.bgtq_layout_create(zero.ctypes.data_as(C.c_void_p), 2, 0, C.byref(h)) == B.ERR_INVALID
+
+
+def test_per_head_energy_matches_oracle_and_sums_to_layer_score(lib):
+    m = synth.make_layer_model(16, 4, 3)
+    q_cal, k_cal = synth.make_calibration(m, 64, 4, 5e5)
+    per = B.block_energy_heads(q_cal.numpy(), k_cal.numpy())
+    np.testing.assert_allclose(per, O.block_energy_heads(q_cal.double().numpy(), k_cal.double().numpy()),
+                               rtol=1e-12)
+    np.testing.assert_allclose(per.sum(axis=0), B.block_energy(q_cal.numpy(), k_cal.numpy()), rtol=1e-12)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2)
+    assert rates.shape == (4, 64) and np.all(rates.sum(axis=1) == 128)
+    assert len({tuple(r) for r in rates}) > 1            # the heads' allocations differ
