@@ -7,29 +7,35 @@
 //
 // Three kernels per call, chained by programmatic dependent launch:
 //  * qprep_kernel (one CTA per batch row x KV head; in a decode step, step_prep_kernel also
-//    runs the encode CTAs of the new tokens): q' = R_g q_g for the G query heads (fp32,
-//    scaled by softmax_scale * log2(e) / (sqrt(d_g) kappa_g)), split into fp16 hi + lo
-//    parts and laid out as mma B fragments.
+//    runs the encode CTAs of the new tokens): q' = R_g q_g for the G query columns of the
+//    KV head (fp32, scaled by softmax_scale * log2(e) / (sqrt(d_g) kappa_g)), split into
+//    fp16 hi + lo parts and laid out as mma B fragments. A column is one query head at
+//    one query token: G = query heads per KV head x n_q query tokens (n_q = 1 except in
+//    multi-token calls).
 //  * split_kernel: the (batch row, KV head) caches are laid end to end as one sequence of
 //    64-token tiles and every CTA takes an equal slice of it (one or two units' worth), so
 //    the grid is one balanced wave. 4 warps, no producer warp: warp w streams its own tiles
 //    w, w+4, ... through a private pair of ring stages with 1-D bulk async copies
-//    (cp.async.bulk + mbarrier, L2 evict-first, no multicast), contiguous or paged. The
-//    CTA starts (tables, first copies) while q-prep runs and waits only before loading
-//    the q' fragments. Keys: per quad of 4 dimension pairs one load gives the lane its
-//    codes for its 8 tokens (fragment-major format); rate 1 turns into +-1 pairs with bit
-//    operations, rates 2-4 index pair tables in shared memory (lane-private for rate 2, hi
-//    + lo parts for rates 3-4); a group's quads go in pairs into mma.m16n8k16 (for G <= 4
-//    the q' hi and lo parts are the eight columns of one product). fp32 accumulators per
-//    group, then times the group norm. Online softmax in base 2 with warp shuffles.
-//    Values: the probabilities times |v|/sqrt(128) in fp16, transposed with movmatrix,
-//    against value-code pair lookups in m16n8k16 products, accumulated in V's rotated
-//    space (fp32). Per unit the four warps merge and the CTA writes its partial (o', m, l).
-//    A scores-only form writes the logits instead.
-//  * combine_kernel (one CTA per batch row x query head, 512 threads): log-sum-exp merge of
-//    the unit's partials and o = R_V^T o'.
+//    (cp.async.bulk + mbarrier, L2 evict-first, no multicast), contiguous or paged; one or
+//    two tiles left over after a multiple of four go out as half tiles (row blocks 0-1 and
+//    2-3 to two warps). The CTA starts (tables, first copies) while q-prep runs and waits
+//    only before loading the q' fragments. Keys: per quad of 4 dimension pairs one load
+//    gives the lane its codes for its 8 tokens (fragment-major format); rate 1 turns into
+//    +-1 pairs with bit operations, rates 2-4 index pair tables in shared memory
+//    (lane-private for rate 2, hi + lo parts for rates 3-4); a group's quads go in pairs
+//    into mma.m16n8k16 (for G <= 4 the q' hi and lo parts are the eight columns of one
+//    product). fp32 accumulators per group, then times the group norm (fp32 or fp16, a
+//    template variant). Each column masks the tokens past its own position (the row's
+//    last tiles only). Online softmax in base 2 with warp shuffles. Values: the
+//    probabilities times |v|/sqrt(128) in fp16, transposed with movmatrix, against
+//    value-code pair lookups in m16n8k16 products, accumulated in V's rotated space
+//    (fp32). Per unit the four warps merge and the CTA writes its partial (o', m, l). A
+//    scores-only form writes the logits instead.
+//  * combine_kernel (one CTA per batch row x query column, 512 threads): log-sum-exp merge
+//    of the unit's partials and o = R_V^T o', written to out[b][token][head].
 // After an append (bgtq_decode_step) only the tile that receives the new tokens waits for
-// the encode before it is copied.
+// the encode before it is copied. With norm correction the step's encode CTAs run as
+// clusters of four (their launch pads the grid to whole clusters).
 //
 // Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, waits
 // (bounded) for its own copies in flight and returns.
