@@ -531,6 +531,8 @@ __device__ __forceinline__ float tile_norm(const unsigned char* area, int i) {
 
 // SC: scores only. The tiles' logits (softmax_scale q . k_hat, natural units) go to
 // a.scores; no softmax, values, partials or merge. NH: the layout stores fp16 norms.
+// (the scores-only instantiation discards the softmax and value code of the tile body)
+#pragma nv_diag_suppress 128
 template <int VR, bool NP, bool SC, bool NH>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -880,6 +882,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
     for (int h = 0; h < 2; ++h)
       if (pend & (1u << h)) mbar_wait_bounded(&full[warp + kWarps * h], (phase >> h) & 1u);
 }
+#pragma nv_diag_default 128
 
 size_t split_smem_bytes(int tile_bytes, int n_kquads) {
   return 128 + size_t(kRing) * tile_bytes + size_t(n_kquads) * 64 * sizeof(unsigned) + 2 * kWarps * 8 * sizeof(float);
