@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <utility>
 
 #include "bgtq_internal.h"
 #include "encode_body.cuh"
@@ -425,6 +426,12 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   for (int j4 = 0; j4 < kPre; ++j4) r[j4] = c0 + j4 < c1 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < kMaxG * kQsLd; e += kPrepThreads) qs[e] = 0.f;
   __syncthreads();
+  // in a decode step (launched as a programmatic dependent) the CTA got here, rows of R in
+  // flight, while the kernel before it ran; q is the caller's: wait for that kernel before
+  // reading it. Only then may the split kernel launch: it reads the cache, which that
+  // kernel may write. (q-prep alone is a plain launch: both are no-ops there.)
+  pdl_wait();
+  pdl_trigger();
   for (int e = tid; e < G * kD; e += kPrepThreads) {
     const int hh = e >> 7, pe = e & (kD - 1);
     if (pe >= L.n_packed) continue;
@@ -492,6 +499,7 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
 __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
                                                              int h_q, int h_kv, int G, int n_q, float qscale,
                                                              unsigned* __restrict__ qfrag) {
+  // launched after the kernel before it has completed: the split kernel may start now
   pdl_trigger();
   const int u = blockIdx.x;
   prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
@@ -507,7 +515,8 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
                                                                  const void* __restrict__ q, int q_dtype, int h_q,
                                                                  int h_kv, int G, int n_q, float qscale,
                                                                  unsigned* __restrict__ qfrag, int n_enc) {
-  pdl_trigger();
+  // every block triggers its dependent (the split kernel) after its own wait for the
+  // kernel before it (in the encode and q-prep bodies; padding blocks by exiting)
   const int e = blockIdx.x;
   if (e < n_enc) {
     const int part = e % kEncodeParts;
@@ -937,6 +946,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
                                                               int max_tiles, long long total_tiles, int n_ctas, int G, int h_q,
                                                               int h_kv, int n_q, const float* __restrict__ v_rot,
                                                               float* __restrict__ out) {
+  pdl_trigger();  // the next call's first kernel may start its prologue now
   const int bq = blockIdx.x, b = bq / h_q, hq = bq % h_q;
   const int u = b * h_kv + hq / G, hh = hq % G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1028,6 +1038,23 @@ int split_occupancy(const DevLayout& L) {
                                                     split_smem_bytes(L.tile_bytes, L.n_kquads)) != cudaSuccess)
     return 1;
   return n < 1 ? 1 : n;
+}
+
+// Launch as a programmatic dependent of the kernel before it on the stream: the CTAs may
+// start while that kernel runs and wait (griddepcontrol.wait) before reading its results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t stream,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Calls fn(IntC<VR>, IntC<NP>, IntC<SC>, IntC<NH>) with the split-kernel variant of a
@@ -1148,6 +1175,8 @@ cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
                           float* out, void* workspace, cudaStream_t stream) {
   const int G = h_q * n_q / h_kv;
+  // a plain launch: the split kernel, launched as soon as this kernel starts, reads the
+  // cache, which the kernel before this one may write
   qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
       L, q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
@@ -1175,10 +1204,9 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
   const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
   cudaError_t e;
   if (!L.norm_correct) {
-    step_prep_kernel<false><<<unsigned(n_enc + batch * h_kv), kPrepThreads, 0, stream>>>(
-        L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype,
-        h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
-    e = cudaGetLastError();
+    e = launch_dependent(step_prep_kernel<false>, unsigned(n_enc + batch * h_kv), kPrepThreads, stream, L, k_new,
+                         v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, G, n_q,
+                         softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   } else {
     // norm correction: clusters of the four encode parts of a token; the q' blocks
     // follow, padded to a whole cluster (the padding blocks return at once)

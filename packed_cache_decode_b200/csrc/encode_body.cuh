@@ -138,6 +138,13 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
                                                   const int* __restrict__ seq_lens, const CacheRef& cache, int t,
                                                   int part, int b, int h) {
   const int tid = threadIdx.x;
+  // a decode step may be launched while the kernel before it still runs (programmatic
+  // dependent launch): nothing the caller writes (seq_lens, k, v, the cache, a block
+  // table) is read before that kernel has completed (a no-op for a plain launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // from here on a kernel launched as this one's dependent may start (it waits for this
+  // grid before it reads the tokens written here)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long pos = (long long)seq_lens[b] + t;
   // both early exits are the same for the four parts of a token (with NC, a whole cluster
   // leaves before its first barrier)
