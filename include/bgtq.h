@@ -116,6 +116,8 @@ typedef struct {
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char* bgtq_last_error_string(void);
+/* ABI version: 200 (bgtq_layout_info gained flags, norm_bytes and n_packed; layout
+ * options, rate-0 blocks, per-head scores and multi-token calls were added). */
 int bgtq_version(void);
 
 /* ---------------------------------------------------------------- host planning ---- */

@@ -170,7 +170,8 @@ extern "C" {
 
 const char* bgtq_last_error_string(void) { return bgtq::last_error(); }
 
-int bgtq_version(void) { return 100; }
+// 200: layout options, n_packed and flags in bgtq_layout_info, multi-token calls
+int bgtq_version(void) { return 200; }
 
 bgtq_status bgtq_lloyd_max(int bits, double* centroids, double* thresholds, double* mse) {
   if (!valid_rate(bits)) return fail(BGTQ_ERR_INVALID, "lloyd_max: bits must be 1..4");

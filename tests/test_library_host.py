@@ -185,3 +185,11 @@ def test_per_head_energy_matches_oracle_and_sums_to_layer_score(lib):
     rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2)
     assert rates.shape == (4, 64) and np.all(rates.sum(axis=1) == 128)
     assert len({tuple(r) for r in rates}) > 1            # the heads' allocations differ
+
+
+def test_abi_version_and_info_size_agree_with_the_binding(lib):
+    """The binding's bgtq_layout_info mirrors the header's (the library fills every field)."""
+    assert lib.bgtq_version() == 200
+    lay = B.Layout(np.full(64, 2), 2, 0)
+    assert lay.info.n_packed == 128 and lay.info.norm_bytes == 4 and lay.info.flags == 0
+    assert lay.info.tile_tokens == 64 and lay.info.head_dim == 128
