@@ -193,3 +193,24 @@ def test_abi_version_and_info_size_agree_with_the_binding(lib):
     lay = B.Layout(np.full(64, 2), 2, 0)
     assert lay.info.n_packed == 128 and lay.info.norm_bytes == 4 and lay.info.flags == 0
     assert lay.info.tile_tokens == 64 and lay.info.head_dim == 128
+
+
+def test_new_host_calls_refuse_bad_arguments(lib):
+    q = np.zeros((4, 6, 128), dtype=np.float32)
+    k = np.zeros((4, 4, 128), dtype=np.float32)
+    out = np.zeros(4 * 64)
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    assert lib.bgtq_block_energy_heads(p(q), 4, 6, p(k), 4, 4, p(out)) == B.ERR_INVALID   # 6 % 4 != 0
+    assert lib.bgtq_block_energy_heads(None, 4, 8, p(k), 4, 4, p(out)) == B.ERR_INVALID
+    s = np.ones(64)
+    r = np.zeros(64, dtype=np.int32)
+    assert lib.bgtq_allocate_rates(p(s), 64, -1, 4, 64, None, p(r)) == B.ERR_INVALID
+    assert lib.bgtq_allocate_rates(p(s), 64, 0, 0, 0, None, p(r)) == B.ERR_INVALID      # max_rate must be >= 1
+    assert lib.bgtq_allocate_rates(p(s), 64, 0, 4, 257, None, p(r)) == B.ERR_INFEASIBLE
+    assert lib.bgtq_allocate_rates(p(s), 64, 0, 4, 0, None, p(r)) == B.OK and not r.any()
+    bad = np.full(64, 5, dtype=np.int32)
+    h = C.c_void_p()
+    assert lib.bgtq_layout_create(p(bad), 2, 0, C.byref(h)) == B.ERR_INVALID
+    neg = np.full(64, 2, dtype=np.int32)
+    neg[3] = -1
+    assert lib.bgtq_layout_create(p(neg), 2, 0, C.byref(h)) == B.ERR_INVALID
