@@ -41,8 +41,10 @@ form at 1 bit, the published per-coordinate MSE figures and Monte Carlo; greedy 
 exhaustive search; rotation orthogonality / QR definition; encode-decode against the
 closed-form distortion; attention against the rotated-space identity and its special
 cases; NC against the norm it must restore and the mean centroid energy 1 - D(b) of a
-Lloyd-Max quantiser; fp16 norms against hand-placed bytes. No function here is "parity
-unpinned".
+Lloyd-Max quantiser; fp16 norms against hand-placed bytes; multi-token attention against
+PyTorch's masked scaled_dot_product_attention and causality; rate-0 blocks against
+exhaustive allocation, D(0) by Monte Carlo and exact zeros; per-head scores against the
+layer score and a constructed scaling. No function here is "parity unpinned".
 """
 from __future__ import annotations
 
