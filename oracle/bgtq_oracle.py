@@ -24,7 +24,7 @@ Sources (cited by page title and passage):
   (SC'11): the Philox4x32-10 counter-based generator.
 * [BoxMuller] Box and Muller (1958): two uniforms to two independent N(0,1) draws.
 
-Readings where the pages leave a step open (each one is also listed in the design doc):
+Readings where the pages leave a step open:
 energy score = mean query block energy x mean key block energy (blockwise bound,
 Cauchy-Schwarz per block); rate penalty D(b) = Gaussian Lloyd-Max per-coordinate MSE;
 block j = coordinates {j, j+64} (rotate-half RoPE); groups ordered by descending rate,
@@ -34,7 +34,10 @@ code = number of thresholds <= y; one fp32 norm per (token, group); V coded as o
 128-dim TQ-MSE group at the V rate. Optional layout variants: norm correction (NC) stores
 |x| sqrt(d) / |c| instead of |x|, c the vector of the chosen centroids, so the decoded
 group vector has the norm of the input; fp16 norms (round to nearest, saturating at the
-largest finite fp16) halve the norm bytes.
+largest finite fp16) halve the norm bytes. Beyond the pages: a block may get rate 0 (not
+stored, decodes to 0, D(0) = 1); rates may be allocated per KV head from that head's term
+of the energy score; n_q new query tokens attend causally (token j up to its own
+position).
 
 Parity pins (tests/test_oracle_pins.py): Philox known-answer vectors; Lloyd-Max closed
 form at 1 bit, the published per-coordinate MSE figures and Monte Carlo; greedy vs
