@@ -7,7 +7,6 @@ attention output of every query head that reads them.
 """
 import math
 
-import numpy as np
 import pytest
 import torch
 

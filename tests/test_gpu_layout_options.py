@@ -16,7 +16,7 @@ import torch
 import oracle as O
 from packed_cache_decode_b200 import binding as B
 
-from .parity_util import ATTN_REL_L2, Case, build_inputs, compare_packed, gpu_encode, oracle_slice, rel_l2, slice_bytes
+from .parity_util import Case, build_inputs, compare_packed, gpu_encode, oracle_slice, slice_bytes
 from .test_gpu_parity import _run_case
 
 pytestmark = pytest.mark.gpu

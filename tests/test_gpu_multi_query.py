@@ -15,8 +15,7 @@ import oracle as O
 from packed_cache_decode_b200 import binding as B
 from packed_cache_decode_b200 import synth
 
-from .parity_util import (ATTN_REL_L2, Case, build_inputs, compare_packed, gpu_encode, oracle_slice, rel_l2,
-                          slice_bytes)
+from .parity_util import ATTN_REL_L2, Case, build_inputs, gpu_encode, oracle_slice, rel_l2, slice_bytes
 
 pytestmark = pytest.mark.gpu
 

@@ -13,7 +13,6 @@ import torch
 
 import oracle as O
 from packed_cache_decode_b200 import binding as B
-from packed_cache_decode_b200 import synth
 
 from .parity_util import (ATTN_REL_L2, Case, build_inputs, compare_packed, gpu_decode, gpu_encode, oracle_slice,
                           rel_l2, slice_bytes)

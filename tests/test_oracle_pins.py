@@ -3,7 +3,6 @@
 Each test is chosen so that a plausible slip in the oracle (a dropped term, a wrong
 sign or index, a transposed operand) fails it. No GPU needed.
 """
-import itertools
 import math
 import os
 

@@ -5,7 +5,6 @@ pool, plugins whose framework forbids allocation while they execute), so the lib
 offers bgtq_decode_attention_noalloc, which keeps its split-K scratch in a fixed
 device array instead of a caller workspace. This file is collected last on purpose.
 """
-import ctypes as C
 
 import numpy as np
 import pytest
