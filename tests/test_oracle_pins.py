@@ -638,3 +638,36 @@ def test_per_head_energy_sums_to_the_layer_score_and_follows_each_head():
     assert per2[2, 5] == pytest.approx(9.0 * per[2, 5], rel=1e-12)
     np.testing.assert_allclose(np.delete(per2, 2, axis=0), np.delete(per, 2, axis=0), rtol=0, atol=0)
     np.testing.assert_allclose(np.delete(per2[2], 5), np.delete(per[2], 5), rtol=0, atol=0)
+
+
+def test_random_layouts_with_every_option_pack_one_to_one():
+    """Random rate vectors over 0..4 (some blocks uncoded), every value rate and both norm
+    types: codes and norms round-trip, and codes at their largest value fill the code
+    areas exactly (no bit unused, none shared)."""
+    rng = np.random.default_rng(31)
+    done = 0
+    while done < 12:
+        rates = rng.integers(0, 5, size=64)
+        if rates.sum() % 4 or rates.max() == 0:
+            continue
+        vr = int(rng.integers(1, 5))
+        fp16 = bool(done % 2)
+        lay = O.make_layout(rates, vr, done, norm_fp16=fp16)
+        pr = lay.packed_rates()
+        n = 100
+        kc = rng.integers(0, 1 << pr, size=(n, lay.n_packed))
+        vc = rng.integers(0, 1 << vr, size=(n, 128))
+        kn = rng.uniform(0, 50, size=(n, lay.n_kgroups))
+        vn = rng.uniform(0, 50, size=n)
+        buf = O.pack(lay, {"k_codes": kc, "v_codes": vc, "k_norms": kn, "v_norm": vn}, 128)
+        assert buf.size == 2 * lay.tile_bytes
+        u = O.unpack(lay, buf, n)
+        np.testing.assert_array_equal(u["k_codes"], kc)
+        np.testing.assert_array_equal(u["v_codes"], vc)
+        np.testing.assert_array_equal(u["k_norms"], O.stored_norms(lay, kn).astype(np.float64))
+        np.testing.assert_array_equal(u["v_norm"], O.stored_norms(lay, vn).astype(np.float64))
+        full = {"k_codes": np.repeat((1 << pr)[None, :] - 1, 128, 0), "v_codes": np.full((128, 128), (1 << vr) - 1),
+                "k_norms": np.zeros((128, lay.n_kgroups)), "v_norm": np.zeros(128)}
+        tiles = O.pack(lay, full, 128).reshape(2, lay.tile_bytes)
+        assert np.all(tiles[:, :64 * (lay.k_record_bytes + lay.v_record_bytes)] == 255)
+        done += 1
