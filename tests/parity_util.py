@@ -14,6 +14,12 @@ from packed_cache_decode_b200 import synth
 
 CODE_EPS = 1e-6        # coordinates this close to a threshold may code either way
 ATTN_REL_L2 = 2e-3     # attention output tolerance (relative L2 per query head)
+# Near-threshold coordinates are rare: the density of a rotated coordinate at a threshold
+# is at most that of N(0,1) (0.4), so with up to 15 thresholds a coordinate falls within
+# 1e-6 of one with probability below about 1.2e-5.
+NEAR_FRAC = 1e-4
+NEAR_SLACK = 3
+NEAR_STATS = {"coords": 0, "near": 0, "near_coded_differently": 0}   # running totals of compare_packed
 
 
 @dataclass
@@ -98,7 +104,12 @@ def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, 
     """Codes bit-exact except near-threshold coordinates; norms to 1 ulp of their stored
     type. With norm correction a norm depends on every code of its token, so tokens with
     a differing (near-threshold) code are left out of the norm comparison.
-    Returns (near-boundary count, how many of those differ)."""
+
+    A coordinate is near a threshold when the oracle's rotated value lies within
+    CODE_EPS of a decision threshold; only those may code differently. Asserts that every
+    coordinate that codes differently is one of them and that they stay rare (at most
+    NEAR_FRAC of the coordinates, plus a few). Returns (near-threshold count, how many of
+    those code differently)."""
     mask, n_near = O.boundary_mask(lay, enc, capacity, CODE_EPS)
     nt = capacity // 64
     tb = lay.tile_bytes
@@ -109,20 +120,30 @@ def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, 
     diff = (w[:, :code_bytes] ^ g[:, :code_bytes]) & ~m[:, :code_bytes]
     bad = np.argwhere(diff != 0)
     assert bad.size == 0, f"{len(bad)} code bytes differ away from thresholds, first at tile/byte {bad[:5].tolist()}"
+    n = enc["k_codes"].shape[0]
+    uw, ug = O.unpack(lay, want, n), O.unpack(lay, got, n)
+    kd = uw["k_codes"] != ug["k_codes"]
+    vd = uw["v_codes"] != ug["v_codes"]
+    assert np.all(enc["k_margin"][kd] < CODE_EPS) and np.all(enc["v_margin"][vd] < CODE_EPS), \
+        "a coordinate away from every threshold codes differently"
+    n_diff = int(kd.sum() + vd.sum())
+    coords = enc["k_margin"].size + enc["v_margin"].size
+    assert n_diff <= n_near
+    assert n_near <= NEAR_FRAC * coords + NEAR_SLACK, f"{n_near} of {coords} coordinates near a threshold"
     it = np.int16 if lay.norm_fp16 else np.int32
     wn = w[:, code_bytes:].copy().view(it).astype(np.int64)
     gn = g[:, code_bytes:].copy().view(it).astype(np.int64)
     ulp = np.abs(wn - gn)                         # norms are >= 0: integer order is float order
     if lay.norm_correct:
-        n = enc["k_codes"].shape[0]
-        uw, ug = O.unpack(lay, want, n), O.unpack(lay, got, n)
         differs = np.zeros(nt * 64, dtype=bool)
-        differs[:n] = np.any(uw["k_codes"] != ug["k_codes"], axis=1) | np.any(uw["v_codes"] != ug["v_codes"], axis=1)
+        differs[:n] = np.any(kd, axis=1) | np.any(vd, axis=1)
         per_tile = differs.reshape(nt, 1, 64)     # norm entry j of a tile belongs to token j % 64
         ulp = np.where(np.broadcast_to(per_tile, (nt, lay.n_kgroups + 1, 64)).reshape(nt, -1), 0, ulp)
     assert ulp.max() <= 1, f"norm differs by {ulp.max()} ulp"
-    near_diff = int(np.count_nonzero((w[:, :code_bytes] ^ g[:, :code_bytes]) & m[:, :code_bytes]))
-    return n_near, near_diff
+    NEAR_STATS["coords"] += coords
+    NEAR_STATS["near"] += n_near
+    NEAR_STATS["near_coded_differently"] += n_diff
+    return n_near, n_diff
 
 
 def rel_l2(a: np.ndarray, b: np.ndarray) -> float:

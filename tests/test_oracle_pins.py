@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle as O
+from oracle import bgtq_oracle as OM
 from packed_cache_decode_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -671,3 +672,91 @@ def test_random_layouts_with_every_option_pack_one_to_one():
         tiles = O.pack(lay, full, 128).reshape(2, lay.tile_bytes)
         assert np.all(tiles[:, :64 * (lay.k_record_bytes + lay.v_record_bytes)] == 255)
         done += 1
+
+
+# ------------------------------------------------------------------ near-threshold mask
+def _unit_input_for(y, rot, scale):
+    """x with sqrt(d) R x / |x| = y (|y|^2 = d): x = scale R^T y / sqrt(d), |x| = scale."""
+    d = len(y)
+    return scale * (rot.T @ y) / math.sqrt(d)
+
+
+@pytest.mark.parametrize("rate", [1, 2, 3, 4])
+def test_encode_margin_is_the_distance_to_the_nearest_threshold(rate):
+    # Rotated coordinates placed at known offsets from known thresholds: the margin the
+    # encoder returns is that offset (an absolute distance, to the nearest threshold, not
+    # to a centroid), and the code falls on the side of the threshold the offset says.
+    d = 64
+    rot = O.haar_rotation(5, rate, d)
+    _, t, _ = O.lloyd_max(rate)
+    k_mid = len(t) // 2                          # the middle threshold, exactly 0
+    k_out = len(t) - 1                           # the largest threshold
+    offsets = [(k_out, 0.5e-6), (k_out, -0.5e-6), (k_out, 2e-6), (k_out, -2e-6), (k_mid, 3e-6), (0, -4e-6)]
+    y = np.zeros(d)
+    for i, (k, off) in enumerate(offsets):
+        y[i] = t[k] + off
+    # fill the rest with values midway between thresholds (far from every threshold) and
+    # close the norm |y|^2 = d with the last coordinate
+    inner = 0.5 * (t[k_mid] + t[k_mid + 1]) if len(t) > 1 else 0.8
+    for i in range(len(offsets), d - 1):
+        y[i] = inner if i % 2 else -inner
+    rest = d - np.sum(y[:-1] ** 2)
+    assert rest > 0
+    y[-1] = math.sqrt(rest)
+    x = _unit_input_for(y, rot, 3.7)
+    codes, norms, margin = OM._tq_encode_group(x[None, :], rot, t)
+    np.testing.assert_allclose(norms, [3.7], rtol=1e-14)
+    for i, (k, off) in enumerate(offsets):
+        assert abs(margin[0, i] - abs(off)) < 1e-12, (i, margin[0, i], off)
+        assert codes[0, i] == (k + 1 if off > 0 else k)
+    last = np.min(np.abs(y[-1] - t))
+    assert abs(margin[0, -1] - last) < 1e-12
+    # a coordinate exactly on the middle threshold codes up and has margin 0
+    y0 = np.zeros(d)
+    y0[0] = 0.0
+    y0[1:] = math.sqrt(d / (d - 1))
+    codes0, _, m0 = OM._tq_encode_group(_unit_input_for(y0, rot, 1.0)[None, :], rot, t)
+    assert m0[0, 0] < 1e-14
+    assert codes0[0, 0] in (k_mid, k_mid + 1)
+
+
+def test_boundary_mask_covers_exactly_the_near_threshold_codes():
+    # Margins set by hand on a mixed-rate layout: the mask must hold all of a coordinate's
+    # code bits (1 << rate) - 1 exactly where the margin is below eps (an absolute eps,
+    # compared with <), nothing elsewhere, and count those coordinates.
+    rates = np.array([4] * 3 + [3] * 4 + [2] * 19 + [1] * 38)
+    assert (2 * rates.sum()) % 8 == 0
+    lay = O.make_layout(rates, 3, 2)
+    n, eps = 70, 1e-6
+    rng = np.random.default_rng(3)
+    km = rng.uniform(0.01, 1.0, (n, lay.n_packed))
+    vm = rng.uniform(0.01, 1.0, (n, 128))
+    near_k = [(0, 0), (5, 7), (69, 127), (64, 30), (33, 12)]
+    for i, j in near_k:
+        km[i, j] = 0.5e-6
+    km[1, 1] = 2e-6                       # outside (absolute), inside for a relative eps on |y| ~ 2.4
+    km[2, 2] = eps                        # not below eps
+    near_v = [(3, 4), (63, 64)]
+    for i, j in near_v:
+        vm[i, j] = 0.0
+    enc = {"k_codes": np.zeros((n, lay.n_packed), dtype=np.int64), "v_codes": np.zeros((n, 128), dtype=np.int64),
+           "k_norms": np.ones((n, lay.n_kgroups)), "v_norm": np.ones(n), "k_margin": km, "v_margin": vm}
+    cap = 128
+    mask, count = O.boundary_mask(lay, enc, cap, eps)
+    assert count == len(near_k) + len(near_v)
+    u = O.unpack(lay, mask, n)
+    want_k = np.zeros((n, lay.n_packed), dtype=np.int64)
+    pr = lay.packed_rates()
+    for i, j in near_k:
+        want_k[i, j] = (1 << pr[j]) - 1
+    want_v = np.zeros((n, 128), dtype=np.int64)
+    for i, j in near_v:
+        want_v[i, j] = (1 << 3) - 1
+    np.testing.assert_array_equal(u["k_codes"], want_k)
+    np.testing.assert_array_equal(u["v_codes"], want_v)
+    # the mask touches no norm byte and no token slot past n
+    full = O.unpack(lay, mask, cap)
+    assert not full["k_codes"][n:].any() and not full["v_codes"][n:].any()
+    assert not full["k_norms"].any() and not full["v_norm"].any()
+    # set bits: exactly sum of the masked coordinates' rates
+    assert int(np.unpackbits(mask).sum()) == sum(pr[j] for _, j in near_k) + 3 * len(near_v)
