@@ -33,17 +33,23 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from packed_cache_decode_b200 import binding as B  # noqa: E402
+from packed_cache_decode_b200 import sharding  # noqa: E402
 from packed_cache_decode_b200 import synth  # noqa: E402
 
 METRIC = "packed-KV decode attention: cached keys/s (HBM GB/s as % of B200 peak in roofline)"
 UNIT = "keys/s"
 
 
-def _profiled_traffic():
-    """DRAM bytes per launch of the split kernel from the committed ncu summary, or None
-    when the kernel source has changed since that capture."""
+PROFILE_KEYS = {"llama70b": "llama70b_b4_128k_k2v2", "llama8b": "llama8b_32k_k2v2", "qwen3b": "qwen3b_128k_k3v3"}
+
+
+def _profiled_traffic(key: str):
+    """DRAM bytes per launch of the split kernel from the committed ncu summary of this
+    workload, or None when there is none or the kernel source has changed since."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "split_kernel_llama8b_32k_k2v2.txt")
+    if key not in PROFILE_KEYS:
+        return None
+    prof = os.path.join(ROOT, "profiles", f"split_kernel_{PROFILE_KEYS[key]}.txt")
     src = os.path.join(ROOT, "packed_cache_decode_b200", "csrc", "decode_mma.cu")
     try:
         fields = dict(ln.split(":", 1) for ln in open(prof) if ln.startswith(("source_sha256_16:", "dram_bytes")))
@@ -150,23 +156,33 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------ workload
 class Model:
-    """Per-layer packed caches and per-step inputs of one workload on one GPU."""
+    """Per-layer packed caches and per-step inputs of one workload on one GPU. With a
+    shard (sharding.Shard) the GPU holds only that shard's batch rows and KV heads (and
+    the query heads that read them); rates are still allocated per layer over all heads."""
 
-    def __init__(self, wl: synth.Workload, device: torch.device, seed_offset: int = 0):
+    def __init__(self, wl: synth.Workload, device: torch.device, seed_offset: int = 0, shard=None):
         self.wl = wl
         self.dev = device
-        L, Bt, hq, hkv = wl.length, wl.batch, wl.h_q, wl.h_kv
+        G = wl.h_q // wl.h_kv
+        if shard is None:
+            shard = sharding.Shard(0, wl.batch, 0, wl.h_kv)
+        self.shard = shard
+        self.heads = list(range(shard.h0, shard.h1))
+        L = wl.length
+        Bt, hkv = shard.b1 - shard.b0, shard.h1 - shard.h0
+        hq = G * hkv
+        self.batch, self.h_q, self.h_kv = Bt, hq, hkv
         self.capacity = 64 * math.ceil(L / 64)
         self.layers = []
         gen = torch.Generator(device=device)
         for layer in range(wl.layers):
             seed = wl.seed * 1000 + layer + seed_offset
-            m = synth.make_layer_model(hq, hkv, seed)
+            m = synth.make_layer_model(wl.h_q, wl.h_kv, seed)
             q_cal, k_cal = synth.make_calibration(m, 256, seed + 1, wl.theta)
             rates = B.plan_layer_rates(q_cal.numpy(), k_cal.numpy(), wl.k_bits)
             lay = B.Layout(rates, wl.v_bits, seed).upload(device.index)
             cache = torch.zeros(lay.cache_bytes(Bt, hkv, self.capacity), dtype=torch.uint8, device=device)
-            gen.manual_seed(seed)
+            gen.manual_seed(seed + 7919 * shard.b0 + 104729 * shard.h0)
             # prefill tokens 0..L-2 in bounded chunks (about 1 GB of fp32 draws at a time);
             # token L-1 is the one every step appends again
             chunk = int(max(64, min(16384, 1e9 // (Bt * hkv * 128 * 4 * 3))))
@@ -213,23 +229,26 @@ class Model:
         # Same recipe as synth.key_slice / value_slice (positions a..b-1), drawn on the device.
         dt = self.wl.dtype
         x = torch.randn(Bt, b - a, hkv, 128, generator=gen, device=self.dev)
-        x *= torch.cat([m.k_scale, m.k_scale], 1).to(self.dev)[None, None]
-        for h in range(hkv):
-            x[:, :, h, m.outliers[h].to(self.dev)] *= m.outlier_gain
+        x *= torch.cat([m.k_scale, m.k_scale], 1)[self.heads].to(self.dev)[None, None]
+        for i, h in enumerate(self.heads):
+            x[:, :, i, m.outliers[h].to(self.dev)] *= m.outlier_gain
         x = _rope_dev(x, torch.arange(a, b, device=self.dev), self.wl.theta)
         v = torch.randn(Bt, b - a, hkv, 128, generator=gen, device=self.dev)
         return x.to(dt), v.to(dt)
 
     def _draw_q(self, m, Bt, hq, pos, gen):
+        G = m.group
+        qh = [h * G + j for h in self.heads for j in range(G)]
         x = torch.randn(Bt, 1, hq, 128, generator=gen, device=self.dev)
-        x *= torch.cat([m.q_scale, m.q_scale], 1).to(self.dev)[None, None]
-        for i in range(hq):
-            x[:, :, i, m.outliers[i // m.group].to(self.dev)] *= m.outlier_gain
+        x *= torch.cat([m.q_scale, m.q_scale], 1)[qh].to(self.dev)[None, None]
+        for i, hh in enumerate(qh):
+            x[:, :, i, m.outliers[hh // G].to(self.dev)] *= m.outlier_gain
         x = _rope_dev(x, torch.tensor([pos], device=self.dev), self.wl.theta)
         return x[:, 0].contiguous().to(self.wl.dtype)
 
-    # kernel launches of one layer in a step: encode + split + combine
-    LAUNCHES_PER_LAYER = 3
+    # kernel launches of one layer in a step: step-prep (encode + q-prep) + split (the
+    # log-sum-exp merge runs in the last split CTA of each unit)
+    LAUNCHES_PER_LAYER = 2
 
     def step(self, stream):
         """Every layer: append the step's token and attend (one bgtq_decode_step call)."""
@@ -237,10 +256,17 @@ class Model:
             B.decode_step(x["layout"], x["k_new"], x["v_new"], x["q"], x["cache"], self.lens_before, self.capacity,
                           self.wl.length, x["out"], self.workspace, stream=stream)
 
+    def decode_layer(self, stream, i=0, reps=1):
+        """The decode-attention call of layer i, reps times over the same cache."""
+        x = self.layers[i]
+        for _ in range(reps):
+            B.decode_attention(x["layout"], x["q"], x["cache"], self.lens_after, self.capacity, self.wl.length,
+                               x["out"], self.workspace, self.h_kv, stream=stream)
+
     def decode_only(self, stream):
         for x in self.layers:
             B.decode_attention(x["layout"], x["q"], x["cache"], self.lens_after, self.capacity, self.wl.length,
-                               x["out"], self.workspace, self.wl.h_kv, stream=stream)
+                               x["out"], self.workspace, self.h_kv, stream=stream)
 
 
 def _rope_dev(x, pos, theta):
@@ -253,9 +279,11 @@ def _rope_dev(x, pos, theta):
 
 
 # ------------------------------------------------------------------------ oracle timing
-def oracle_sample(wl: synth.Workload, budget_s: float):
+def oracle_sample(wl: synth.Workload, budget_s: float, max_tokens: int = 16384):
     """Time the CPU oracle on whole (batch row, KV head) units of one layer of the
-    workload: encode the new token, then unpack + reconstruct + attend over the cache."""
+    workload: encode the new token, then unpack + reconstruct + attend over the cache.
+    The sample is bounded: each unit's context is the workload's first max_tokens tokens
+    (the oracle's cost per cached key does not depend on the context length)."""
     import oracle as O
     try:
         from threadpoolctl import threadpool_info
@@ -268,12 +296,13 @@ def oracle_sample(wl: synth.Workload, budget_s: float):
                            O.lloyd_max_mse_table(), 1, 4, 64 * wl.k_bits)
     lay = O.make_layout(rates, wl.v_bits, wl.seed)
     G = wl.h_q // wl.h_kv
-    cap = 64 * math.ceil(wl.length / 64)
+    L = min(wl.length, max_tokens)
+    cap = 64 * math.ceil(L / 64)
     prepared = []
     for h in range(min(2, wl.h_kv)):
-        k = synth.key_slice(m, 0, h, wl.length, 0, wl.seed, wl.theta).double().numpy()
-        v = synth.value_slice(m, 0, h, wl.length, wl.seed).double().numpy()
-        q = torch.stack([synth.query_slice(m, 0, h * G + i, 1, wl.length - 1, wl.seed, wl.theta)[0]
+        k = synth.key_slice(m, 0, h, L, 0, wl.seed, wl.theta).double().numpy()
+        v = synth.value_slice(m, 0, h, L, wl.seed).double().numpy()
+        q = torch.stack([synth.query_slice(m, 0, h * G + i, 1, L - 1, wl.seed, wl.theta)[0]
                          for i in range(G)]).double().numpy()
         prepared.append((k, v, q, O.pack(lay, O.encode(lay, k[:-1], v[:-1]), cap)))
     units, keys, elapsed = 0, 0, 0.0
@@ -281,7 +310,7 @@ def oracle_sample(wl: synth.Workload, budget_s: float):
         k, v, q, buf = prepared[units % len(prepared)]
         t0 = time.perf_counter()
         new = O.encode(lay, k[-1:], v[-1:])                        # the step's append
-        u = O.unpack(lay, buf, wl.length - 1)
+        u = O.unpack(lay, buf, L - 1)
         for key in ("k_codes", "v_codes"):
             u[key] = np.concatenate([u[key], new[key]])
         u["k_norms"] = np.concatenate([u["k_norms"], new["k_norms"].astype(np.float32)])
@@ -290,10 +319,13 @@ def oracle_sample(wl: synth.Workload, budget_s: float):
         O.attention(q, kh, vh, 1 / math.sqrt(128))
         elapsed += time.perf_counter() - t0
         units += 1
-        keys += wl.length
+        keys += L
     return {"value": keys / elapsed, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "threads": f"numpy with {cores} BLAS thread(s) for the matrix products; the oracle's Python loops run "
+                       f"on one core",
             "sample": f"{units} (batch row, KV head) unit passes over {len(prepared)} distinct unit(s) of one "
-                      f"layer, {wl.length} cached tokens each: append 1 token + decode attention, {elapsed:.1f} s"}
+                      f"layer, the first {L} cached tokens of the workload each: append 1 token + decode "
+                      f"attention, {elapsed:.1f} s"}
 
 
 # ------------------------------------------------------------------------ sweep / encode modes
@@ -446,10 +478,14 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama8b", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default="llama70b", choices=list(synth.WORKLOADS))
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-others", action="store_true", help="skip the 8B- and 3B-shaped lines of the default run")
+    ap.add_argument("--shard", action="store_true",
+                    help="N > 1: split one workload's (batch row, KV head) units over the ranks (strong scaling) "
+                         "instead of running independent replicas")
     ap.add_argument("--mode", default="step", choices=["step", "sweep", "encode", "mae"])
     args = ap.parse_args()
     if args.mode == "sweep":
@@ -496,10 +532,77 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
 
-    model = Model(wl, dev, seed_offset=rank * 100000)
+    shard = sharding.shard_units(wl.batch, wl.h_kv, rank, world) if args.shard else None
+    model = Model(wl, dev, seed_offset=0 if args.shard else rank * 100000, shard=shard)
     stream = torch.cuda.Stream(device=dev)
 
-    # capture one step and the decode-only sequence as CUDA graphs
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    clk = ClockSampler(dev).start()
+    r = measure(model, stream, args.steps, args.warmup, barrier, clk)
+    clk.stop()
+    clocks = clk.summary(r["t_on"], r["t_off"])
+
+    times = torch.tensor([r["step_ms"], r["dec_ms"], r["e2e_ms"], r["l2_ms"]], dtype=torch.float64, device=dev)
+    totals = torch.tensor([float(model.keys_per_step), float(model.bytes_per_step)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(times, op=pg.ReduceOp.MAX)
+        pg.all_reduce(totals, op=pg.ReduceOp.SUM)
+    step_ms, dec_ms, e2e_ms, l2_ms = times.tolist()
+    keys, total_bytes = totals.tolist()
+
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        dec_bytes = model.bytes_per_step / wl.layers
+        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+        layer_mb = dec_bytes / 1e6
+        line = {
+            "metric": METRIC, "value": keys / (step_ms * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "context": wl.length,
+                       "h_q": wl.h_q, "h_kv": wl.h_kv, "rates": f"K{wl.k_bits}V{wl.v_bits}",
+                       "bytes_per_token_head": model.layers[0]["layout"].bytes_per_token,
+                       "step": "per layer: bgtq_decode_step (append 1 token + decode attention); CUDA graph",
+                       "l2": f"inputs larger than L2: {model.bytes_per_step / 1e6:.0f} MB of packed caches per step "
+                             f"on each GPU (one cache per layer)",
+                       "parallelism": (f"(batch row, KV head) units sharded over {world} GPU(s), no collective on the "
+                                       f"data path" if args.shard else
+                                       f"replicas x{world} (independent sequences per GPU)")},
+            "gbs": total_bytes / (step_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": _profiled_traffic(args.workload),
+                         "kernel": "decode attention call per layer (q-prep -> split with fused merge, PDL-chained)",
+                         "bytes_per_launch": dec_bytes, "peak_kind": peak_kind},
+            "l2_warm": {"us_per_call": l2_ms * 1e3, "GBs": dec_bytes / (l2_ms * 1e-3) / 1e9,
+                        "note": f"layer 0's decode call repeated over the same {layer_mb:.0f} MB cache"
+                                + (" (fits the 126 MB L2)" if layer_mb < 126 else " (larger than L2: read from HBM)")},
+            "clocks": clocks,
+            "gpu_launches": args.steps * wl.layers * Model.LAUNCHES_PER_LAYER,
+            "e2e": {"value": keys / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"]},
+        }
+        if world == 1 and not args.no_others and args.workload == "llama70b":
+            line["other_workloads"] = other_workloads(args, dev, stream, barrier, peak)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(wl, args.cpu_budget)
+            line["codes_vs_oracle"] = codes_vs_oracle(wl, dev)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def measure(model, stream, steps, warmup, barrier, clk=None):
+    """Device times (CUDA events on the launching stream) of one model: the decode step
+    (all layers, CUDA graph), the decode-attention calls alone (graph over all layers),
+    layer 0's call repeated over one cache (L2-warm when it fits), and the same step end to
+    end with host buffers (one pinned copy each way per step inside the timed region)."""
+    dev = model.dev
     with torch.cuda.stream(stream):
         for _ in range(2):
             model.step(stream)
@@ -510,50 +613,38 @@ def main():
     g_dec = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_dec, stream=stream):
         model.decode_only(stream)
+    reps = 20
+    g_l2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_l2, stream=stream):
+        model.decode_layer(stream, 0, reps)
     torch.cuda.synchronize(dev)
 
-    def barrier():
-        torch.cuda.synchronize(dev)
-        if pg:
-            pg.barrier()
-        torch.cuda.synchronize(dev)
+    def timed(graph, n, pre=3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(pre):
+                graph.replay()
+            e0.record(stream)
+            for _ in range(n):
+                graph.replay()
+            e1.record(stream)
+        barrier()
+        return e0.elapsed_time(e1) / n
 
-    clk = ClockSampler(dev).start()
     with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
+        for _ in range(max(3, warmup)):
             g_step.replay()
     barrier()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_on = clk.mark()
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(args.steps):
-            g_step.replay()
-        ev1.record(stream)
-    barrier()
-    t_off = clk.mark()
-    step_ms = ev0.elapsed_time(ev1) / args.steps
-    # dominant kernels: the decode attention call of each layer (qprep -> split -> combine),
-    # timed on their own stream over the same caches
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            g_dec.replay()
-        d0.record(stream)
-        for _ in range(args.steps):
-            g_dec.replay()
-        d1.record(stream)
-    barrier()
-    dec_ms = d0.elapsed_time(d1) / (args.steps * wl.layers)
-    clk.stop()
-    clocks = clk.summary(t_on, t_off)
+    t_on = clk.mark() if clk else 0.0
+    step_ms = timed(g_step, steps, pre=0)
+    t_off = clk.mark() if clk else 0.0
+    dec_ms = timed(g_dec, steps) / model.wl.layers
+    l2_ms = timed(g_l2, max(3, steps // 2)) / reps
 
     # end to end through the public API with host buffers (pinned), copies inside the timing:
     # every step copies all layers' inputs in and all outputs back, one copy each way
     h_in = model.inputs.cpu().pin_memory()
     h_out = torch.empty_like(model.outputs, device="cpu").pin_memory()
-    h2d = h_in.numel() * h_in.element_size()
-    d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
         model.inputs.copy_(h_in, non_blocking=True)
@@ -567,50 +658,72 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             e2e_step()
         e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e_ms = e0.elapsed_time(e1) / steps
+    del g_step, g_dec, g_l2
+    return {"step_ms": step_ms, "dec_ms": dec_ms, "l2_ms": l2_ms, "e2e_ms": e2e_ms, "t_on": t_on, "t_off": t_off,
+            "h2d": h_in.numel() * h_in.element_size(), "d2h": h_out.numel() * h_out.element_size()}
 
-    times = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(times, op=pg.ReduceOp.MAX)
-    step_ms, dec_ms, e2e_ms = times.tolist()
-    del g_step, g_dec
 
-    if rank == 0:
-        peak, peak_kind = _peaks()
-        keys = model.keys_per_step * world
+def other_workloads(args, dev, stream, barrier, peak):
+    """The 8B- and 3B-shaped layers measured the same way in the same run (their whole
+    steps, the decode call's HBM fraction, the L2-warm single-layer call)."""
+    out = {}
+    for key in ("llama8b", "qwen3b"):
+        wl = synth.WORKLOADS[key]
+        model = Model(wl, dev)
+        r = measure(model, stream, max(5, args.steps), args.warmup, barrier)
         dec_bytes = model.bytes_per_step / wl.layers
-        achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-        line = {
-            "metric": METRIC, "value": keys / (step_ms * 1e-3), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "context": wl.length,
-                       "h_q": wl.h_q, "h_kv": wl.h_kv, "rates": f"K{wl.k_bits}V{wl.v_bits}",
-                       "bytes_per_token_head": model.layers[0]["layout"].bytes_per_token,
-                       "step": "per layer: bgtq_decode_step (append 1 token + decode attention); CUDA graph",
-                       "l2": f"inputs larger than L2: {model.bytes_per_step / 1e6:.0f} MB of packed caches per step",
-                       "parallelism": f"replicas x{world} (independent sequences per GPU)"},
-            "gbs": model.bytes_per_step / (step_ms * 1e-3) / 1e9,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": _profiled_traffic() if wl.name == synth.WORKLOADS["llama8b"].name else None,
-                         "kernel": "decode attention call per layer (split -> combine, PDL-chained)",
-                         "peak_kind": peak_kind},
-            "clocks": clocks,
-            "gpu_launches": args.steps * wl.layers * Model.LAUNCHES_PER_LAYER,
-            "e2e": {"value": keys / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(wl, args.cpu_budget)
-        print(json.dumps(line), flush=True)
-    if pg:
-        pg.barrier()
-        pg.destroy_process_group()
+        out[key] = {"workload": wl.name, "layers": wl.layers, "ms_per_step": r["step_ms"],
+                    "keys_per_s": model.keys_per_step / (r["step_ms"] * 1e-3),
+                    "decode_call_us": r["dec_ms"] * 1e3, "decode_call_GBs": dec_bytes / (r["dec_ms"] * 1e-3) / 1e9,
+                    "frac": dec_bytes / (r["dec_ms"] * 1e-3) / 1e9 / peak,
+                    "l2_warm_us_per_call": r["l2_ms"] * 1e3,
+                    "l2_warm_GBs": dec_bytes / (r["l2_ms"] * 1e-3) / 1e9,
+                    "e2e_keys_per_s": model.keys_per_step / (r["e2e_ms"] * 1e-3),
+                    "bytes_per_token_head": model.layers[0]["layout"].bytes_per_token}
+        del model
+        torch.cuda.empty_cache()
+    return out
+
+
+def codes_vs_oracle(wl, dev, units=2, tokens=4096):
+    """Near-threshold code statistics on a bounded sample: the GPU encodes (batch row 0,
+    KV heads 0..units-1) x tokens of the workload's generator; the oracle encodes the same
+    inputs. Codes may differ only where the oracle's rotated value lies within 1e-6 of a
+    decision threshold; reports how many such coordinates there are and how many differ."""
+    import oracle as O
+    m = synth.make_layer_model(wl.h_q, wl.h_kv, wl.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, wl.seed + 1, wl.theta)
+    rates = O.greedy_rates(O.block_energy(q_cal.double().numpy(), k_cal.double().numpy()),
+                           O.lloyd_max_mse_table(), 1, 4, 64 * wl.k_bits)
+    olay = O.make_layout(rates, wl.v_bits, wl.seed)
+    lay = B.Layout(rates, wl.v_bits, wl.seed).upload(dev.index)
+    n = min(tokens, wl.length)
+    k = torch.stack([synth.key_slice(m, 0, h, n, 0, wl.seed, wl.theta) for h in range(units)], 1).to(wl.dtype)
+    v = torch.stack([synth.value_slice(m, 0, h, n, wl.seed) for h in range(units)], 1).to(wl.dtype)
+    cap = 64 * math.ceil(n / 64)
+    cache = torch.zeros(lay.cache_bytes(1, units, cap), dtype=torch.uint8, device=dev)
+    lens = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.encode_append(lay, k[None].to(dev), v[None].to(dev), lens, cache, cap)
+    got_all = cache.cpu().numpy()
+    per = cap // 64 * olay.tile_bytes
+    coords = near = near_diff = elsewhere = 0
+    for h in range(units):
+        enc = O.encode(olay, k[:, h].double().numpy(), v[:, h].double().numpy())
+        want = O.unpack(olay, O.pack(olay, enc, cap), n)
+        got = O.unpack(olay, got_all[h * per:(h + 1) * per], n)
+        mk, mv = enc["k_margin"] < 1e-6, enc["v_margin"] < 1e-6
+        dk, dv = got["k_codes"] != want["k_codes"], got["v_codes"] != want["v_codes"]
+        coords += mk.size + mv.size
+        near += int(mk.sum() + mv.sum())
+        near_diff += int((dk & mk).sum() + (dv & mv).sum())
+        elsewhere += int((dk & ~mk).sum() + (dv & ~mv).sum())
+    return {"coords": coords, "near_threshold": near, "near_threshold_coded_differently": near_diff,
+            "differ_elsewhere": elsewhere, "sample": f"batch row 0, KV heads 0..{units - 1}, {n} tokens, one layer"}
 
 
 if __name__ == "__main__":

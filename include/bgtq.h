@@ -240,6 +240,30 @@ bgtq_status bgtq_decode_scores(const bgtq_layout* layout, const void* q, int q_d
                                float* scores, long long scores_ld, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- split over token ranges */
+
+/* Decode attention over one part of every row's tokens, for attention split over
+ * disjoint token ranges (e.g. one range per GPU, each holding the packed cache of its
+ * range), merged afterwards by bgtq_merge_partials. [BGTQ s5: attention over packed
+ * caches; the split is the log-sum-exp bookkeeping of split attention, which reaches the
+ * same result as attention over all tokens.] Arguments as bgtq_decode_attention (the
+ * cache holds this part's tokens of each row, seq_lens_dev their count); instead of out,
+ * partial [batch, h_q, 130] fp32 device receives per query head: m = the largest logit
+ * in base-2 units (softmax_scale q.k_hat / ln 2), l = sum_t 2^(logit_t - m), and
+ * o'[128] = sum_t 2^(logit_t - m) v'_t / l with v'_t = (|v_t| / sqrt(128)) c[vcodes_t]
+ * the value in V's rotated space. A row with no token gives m = -inf, l = 0, o' = 0. */
+bgtq_status bgtq_decode_attention_partial(const bgtq_layout* layout, const void* q, int q_dtype, int batch,
+                                          int h_q, int h_kv, const void* cache, const int* seq_lens_dev,
+                                          long long capacity, long long max_seq_len, float softmax_scale,
+                                          float* partial, void* workspace, size_t workspace_bytes, void* stream);
+/* Merges n_parts partial records of the same rows and heads over disjoint token ranges:
+ * partials [n_parts, batch, h_q, 130] fp32 device (each part as written by
+ * bgtq_decode_attention_partial), out [batch, h_q, 128] fp32 device = R_V^T of the
+ * log-sum-exp merge (M = max m, w = l 2^(m - M), o' = sum w o' / sum w): the attention
+ * output over the union of the parts' tokens. */
+bgtq_status bgtq_merge_partials(const bgtq_layout* layout, const float* partials, int n_parts, int batch, int h_q,
+                                float* out, void* stream);
+
 /* ---------------------------------------------------------------- paged caches */
 
 /* The calls above with a paged cache (sequences of different lengths share one pool,

@@ -37,7 +37,8 @@ group vector has the norm of the input; fp16 norms (round to nearest, saturating
 largest finite fp16) halve the norm bytes. Beyond the pages: a block may get rate 0 (not
 stored, decodes to 0, D(0) = 1); rates may be allocated per KV head from that head's term
 of the energy score; n_q new query tokens attend causally (token j up to its own
-position).
+position); decode attention may be split over disjoint token ranges (e.g. one per GPU)
+and merged by log-sum-exp.
 
 Parity pins (tests/test_oracle_pins.py): Philox known-answer vectors; Lloyd-Max closed
 form at 1 bit, the published per-coordinate MSE figures and Monte Carlo; greedy vs
@@ -47,7 +48,9 @@ cases; NC against the norm it must restore and the mean centroid energy 1 - D(b)
 Lloyd-Max quantiser; fp16 norms against hand-placed bytes; multi-token attention against
 PyTorch's masked scaled_dot_product_attention and causality; rate-0 blocks against
 exhaustive allocation, D(0) by Monte Carlo and exact zeros; per-head scores against the
-layer score and a constructed scaling. No function here is "parity unpinned".
+layer score and a constructed scaling; partial attention and its log-sum-exp merge against
+attention over the whole token set (random splits, empty parts). No function here is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -459,6 +462,38 @@ def attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, scale: float)
     p = np.exp(s)
     p /= p.sum(axis=1, keepdims=True)
     return p @ v_hat
+
+
+def partial_attention(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, scale: float):
+    """Attention of queries q [G, 128] over one part of the cached tokens, kept in the
+    form that parts over disjoint token sets can be merged from (the log-sum-exp
+    bookkeeping of split attention): s_t = scale q . k_t, m = max_t s_t,
+    l = sum_t exp(s_t - m), o = sum_t exp(s_t - m) v_t / l. Returns (m [G], l [G],
+    o [G, 128]); an empty part gives m = -inf, l = 0, o = 0."""
+    q = np.asarray(q, dtype=np.float64)
+    G = q.shape[0]
+    if k_hat.shape[0] == 0:
+        return np.full(G, -np.inf), np.zeros(G), np.zeros((G, v_hat.shape[1]))
+    s = (q @ k_hat.T) * scale
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    l = e.sum(axis=1)
+    return m, l, (e @ v_hat) / l[:, None]
+
+
+def merge_partials(parts) -> np.ndarray:
+    """Merge partial attentions [(m, l, o)] over disjoint token sets into the attention over
+    their union: M = max_r m_r, w_r = l_r exp(m_r - M), o = sum_r w_r o_r / sum_r w_r.
+    Rows whose parts are all empty give 0."""
+    m = np.stack([p[0] for p in parts])          # [R, G]
+    l = np.stack([p[1] for p in parts])
+    o = np.stack([p[2] for p in parts])          # [R, G, 128]
+    M = m.max(axis=0)
+    finite = np.isfinite(M)
+    w = np.where(np.isfinite(m) & finite[None], l * np.exp(np.where(np.isfinite(m), m, 0.0) - np.where(finite, M, 0.0)[None]), 0.0)
+    den = w.sum(axis=0)
+    out = np.einsum("rg,rgd->gd", w, o)
+    return np.where(den[:, None] > 0, out / np.where(den > 0, den, 1.0)[:, None], 0.0)
 
 
 # ----------------------------------------------------------------------------------------

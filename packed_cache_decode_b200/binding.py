@@ -32,7 +32,7 @@ EXPORTED = [
     "bgtq_decode_attention_noalloc", "bgtq_noalloc_scratch_capacity", "bgtq_decode_step", "bgtq_decode_scores",
     "bgtq_paged_pool_bytes", "bgtq_encode_append_paged", "bgtq_decode_attention_paged", "bgtq_decode_step_paged",
     "bgtq_decode_attention_multi", "bgtq_decode_step_multi", "bgtq_decode_step_multi_paged",
-    "bgtq_block_energy_heads",
+    "bgtq_block_energy_heads", "bgtq_decode_attention_partial", "bgtq_merge_partials",
 ]
 
 
@@ -77,6 +77,8 @@ def load():
         "bgtq_workspace_bytes": (C.c_size_t, [P, I, I, I, LL]),
         "bgtq_decode_attention": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
         "bgtq_device_status": (I, [P, C.POINTER(C.c_uint), I]),
+        "bgtq_decode_attention_partial": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_merge_partials": (I, [P, P, I, I, I, P, P]),
         "bgtq_decode_attention_noalloc": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P]),
         "bgtq_noalloc_scratch_capacity": (C.c_size_t, []),
         "bgtq_decode_step": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
@@ -272,6 +274,35 @@ def decode_attention(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_
                                         max_seq_len, scale, C.c_void_p(out.data_ptr()),
                                         C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_attention")
+
+
+PARTIAL_RECORD = HEAD_DIM + 2   # (m, l, o'[128]) per query head
+
+
+def decode_attention_partial(layout: Layout, q, cache, seq_lens, capacity: int, max_seq_len: int, partial,
+                             workspace, h_kv: int, softmax_scale: float | None = None, stream=None):
+    """Attention over this cache's part of every row's tokens, as mergeable records:
+    q [B, h_q, 128] CUDA; partial [B, h_q, 130] fp32 CUDA receives (m, l, o') per head."""
+    B, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and partial.is_contiguous()
+    assert tuple(partial.shape) == (B, h_q, PARTIAL_RECORD) and str(partial.dtype) == "torch.float32"
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_partial(layout.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B, h_q, h_kv,
+                                                C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()),
+                                                capacity, max_seq_len, scale, C.c_void_p(partial.data_ptr()),
+                                                C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                                _stream_ptr(stream)),
+           "decode_attention_partial")
+
+
+def merge_partials(layout: Layout, partials, out, stream=None):
+    """partials [n_parts, B, h_q, 130] fp32 CUDA (records over disjoint token ranges);
+    out [B, h_q, 128] fp32 CUDA = attention over the union of the ranges."""
+    n, B, h_q, r = partials.shape
+    assert r == PARTIAL_RECORD and partials.is_contiguous() and out.is_contiguous()
+    assert tuple(out.shape) == (B, h_q, HEAD_DIM)
+    _check(load().bgtq_merge_partials(layout.handle, C.c_void_p(partials.data_ptr()), n, B, h_q,
+                                      C.c_void_p(out.data_ptr()), _stream_ptr(stream)), "merge_partials")
 
 
 def decode_step(layout: Layout, k_new, v_new, q, cache, seq_lens, capacity: int, max_seq_len: int, out, workspace,

@@ -261,15 +261,17 @@ bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype,
   return BGTQ_OK;
 }
 
+// rec non-null: partial records (m, l, o') instead of outputs (out is then rec).
 bgtq_status decode_impl(const bgtq_layout* L, const char* who, const void* q, int q_dtype, int batch, int h_q,
                         int h_kv, int n_q, const CacheRef& c, const int* seq_lens_dev, long long max_seq_len,
-                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes, void* stream,
+                        float* rec = nullptr) {
   DecodePlan plan;
   bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
                                     softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
   cudaError_t e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, softmax_scale, out,
-                                workspace, static_cast<cudaStream_t>(stream));
+                                workspace, static_cast<cudaStream_t>(stream), rec);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
@@ -348,6 +350,31 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dty
   if (st != BGTQ_OK) return st;
   return decode_impl(L, "decode_attention", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
+}
+
+bgtq_status bgtq_decode_attention_partial(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q,
+                                          int h_kv, const void* cache, const int* seq_lens_dev, long long capacity,
+                                          long long max_seq_len, float softmax_scale, float* partial, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_device(L, "decode_attention_partial");
+  CacheRef c{};
+  if (st == BGTQ_OK) st = contiguous("decode_attention_partial", const_cast<void*>(cache), capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(L, "decode_attention_partial", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
+                     softmax_scale, partial, workspace, workspace_bytes, stream, partial);
+}
+
+bgtq_status bgtq_merge_partials(const bgtq_layout* L, const float* partials, int n_parts, int batch, int h_q,
+                                float* out, void* stream) {
+  bgtq_status st = check_device(L, "merge_partials");
+  if (st != BGTQ_OK) return st;
+  if (n_parts < 1 || batch <= 0 || h_q <= 0 || (long long)batch * h_q > 0x7fffffffLL)
+    return fail(BGTQ_ERR_INVALID, "merge_partials: bad n_parts / batch / h_q");
+  if (!partials || !out) return fail(BGTQ_ERR_INVALID, "merge_partials: null pointer");
+  cudaError_t e = launch_merge_records(L->dev, partials, n_parts, (long long)batch * h_q, out,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge_partials");
+  return BGTQ_OK;
 }
 
 bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void* v_new, int kv_dtype, int n_new,

@@ -12,33 +12,37 @@
 //    fp16 hi + lo parts and laid out as mma B fragments. A column is one query head at
 //    one query token: G = query heads per KV head x n_q query tokens (n_q = 1 except in
 //    multi-token calls).
-//  * split_kernel: the (batch row, KV head) caches are laid end to end as one sequence of
-//    64-token tiles and every CTA takes an equal slice of it (one or two units' worth), so
-//    the grid is one balanced wave. 4 warps, no producer warp: warp w streams its own tiles
-//    w, w+4, ... through a private pair of ring stages with 1-D bulk async copies
-//    (cp.async.bulk + mbarrier, L2 evict-first, no multicast), contiguous or paged; one or
-//    two tiles left over after a multiple of four go out as half tiles (row blocks 0-1 and
-//    2-3 to two warps). The CTA starts (tables, first copies) while q-prep runs and waits
-//    only before loading the q' fragments. Keys: per quad of 4 dimension pairs one load
-//    gives the lane its codes for its 8 tokens (fragment-major format); rate 1 turns into
-//    +-1 pairs with bit operations, rates 2-4 index pair tables in shared memory
-//    (lane-private for rate 2, hi + lo parts for rates 3-4); a group's quads go in pairs
-//    into mma.m16n8k16 (for G <= 4 the q' hi and lo parts are the eight columns of one
-//    product). fp32 accumulators per group, then times the group norm (fp32 or fp16, a
-//    template variant). Each column masks the tokens past its own position (the row's
-//    last tiles only). Online softmax in base 2 with warp shuffles. Values: the
-//    probabilities times |v|/sqrt(128) in fp16, transposed with movmatrix, against
-//    value-code pair lookups in m16n8k16 products, accumulated in V's rotated space
-//    (fp32). Per unit the four warps merge and the CTA writes its partial (o', m, l). A
-//    scores-only form writes the logits instead.
+//  * split_kernel: one CTA per SM, 8 or 12 warps. The (batch row, KV head) caches are
+//    laid end to end as one sequence of 64-token tiles and every CTA takes an equal slice
+//    of it (one wave). Inside a slice, unit by unit, warp w streams its own tiles w, w+W,
+//    ... through a private pair of ring stages with 1-D bulk async copies (cp.async.bulk +
+//    mbarrier, L2 evict-first, no multicast), contiguous or paged; the tiles left over after
+//    a multiple of W go out whole or as half tiles (row blocks 0-1 and 2-3) so that no warp
+//    runs more than half a tile past the others. Keys: per quad of 4 dimension pairs one
+//    load gives the lane its codes for its 8 tokens (fragment-major format); rate 1 turns
+//    into +-1 pairs with bit operations; rates 2 and 4 look up byte-indexed tables (one
+//    prmt builds the address from a code byte, one 64-bit shared load returns two A
+//    registers, or a hi + lo pair at rate 4); rate 3 indexes a 6-bit pair table. The
+//    tables hold 16 copies of every entry, lane l reading copy l % 16, so a half-warp's
+//    64-bit loads never share a bank. A group's quads go in pairs into mma.m16n8k16
+//    (for G <= 4 the q' hi and lo parts are the eight columns of one product). fp32
+//    accumulators per group, then times the group norm (fp32 or fp16, a template
+//    variant). Each column masks the tokens past its own position (the row's last tiles
+//    only). Online softmax in base 2 with warp shuffles. Values: the probabilities times
+//    |v|/sqrt(128) in fp16, transposed with movmatrix, against value codes turned into A
+//    registers the same way (rate 2: the byte table), accumulated in V's rotated space
+//    (fp32). At the end of a unit the warps merge and the CTA writes its partial
+//    (o', m, l). A scores-only form writes the logits instead.
 //  * combine_kernel (one CTA per batch row x query column, 512 threads): log-sum-exp merge
-//    of the unit's partials and o = R_V^T o', written to out[b][token][head].
+//    of the unit's partials and o = R_V^T o', written to out[b][token][head] (or, for a
+//    call over one token range of a split sequence, the merged record (m, l, o')).
 // After an append (bgtq_decode_step) only the tile that receives the new tokens waits for
 // the encode before it is copied. With norm correction the step's encode CTAs run as
 // clusters of four (their launch pads the grid to whole clusters).
 //
-// Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, waits
-// (bounded) for its own copies in flight and returns.
+// Every mbarrier wait is bounded; on timeout the kernel records BGTQ_STATUS_TIMEOUT, drops
+// the warp's partial (m = -inf, l = 0), waits (bounded) for its own copies in flight and
+// goes on; the call's output is then invalid and the status says so.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -101,15 +105,14 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 __device__ __forceinline__ void mma16816(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
                                          unsigned b0, unsigned b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ unsigned movmatrix_trans(unsigned x) {
   unsigned y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 __device__ __forceinline__ unsigned pack_h2(float lo, float hi) {
@@ -122,12 +125,14 @@ __device__ __forceinline__ float load_q(const void* p, int dtype, size_t i) {
   return __half2float(static_cast<const __half*>(p)[i]);
 }
 
-constexpr int kMaxParts = 1024;      // partial slots per unit the combine can merge
-constexpr int kCtasPerSm = 3;        // split CTAs resident per SM (registers, shared memory)
-constexpr int kMaxTileBytes = kTile * (2 * kD * 4 / 8 + 4 * (kMaxGroups + 1));  // K4V4, four groups
+constexpr int kMaxParts = 1024;      // partial slots per unit the merge can take
+
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline size_t qfrag_bytes(long long units) { return align256(size_t(units) * kMaxQuads * 64 * sizeof(unsigned)); }
+// per unit: the q' B fragments [kMaxQuads][2][32] words, then the 8 column sums of the
+// rate-1 group's fragments (and padding to 16 bytes)
+constexpr int kQfragWords = kMaxQuads * 64 + 16;
+inline size_t qfrag_bytes(long long units) { return align256(size_t(units) * kQfragWords * sizeof(unsigned)); }
 
 // ------------------------------------------------------------------ split kernel
 struct SplitArgs {
@@ -148,10 +153,7 @@ struct SplitArgs {
   int wait_new;           // the previous kernel appends at seq_lens[b]: wait for it before copying that tile
 };
 
-constexpr int kWarps = 4;                        // warps, one whole 64-token tile at a time each
-constexpr int kThreads = 32 * kWarps;
-constexpr int kRing = 2 * kWarps;                // ring stages: two per warp
-constexpr int kQsLd = kD + 16;                   // row of q staged per group at 16-byte aligned offsets
+constexpr int kQsLd = kD + 16;                   // row of q staged per group at 16-byte aligned columns
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -159,7 +161,7 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 __device__ __forceinline__ void mma1688(float (&c)[4], unsigned a0, unsigned a1, unsigned b0) {
-  asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
                : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
                : "r"(a0), "r"(a1), "r"(b0));
 }
@@ -172,135 +174,207 @@ __device__ __forceinline__ unsigned prmt(unsigned a, unsigned b, unsigned sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
 }
-// Table reads at a byte offset. Lane-private tables keep entry e of lane l at word
-// 32 e + l, so the 32 lanes of a lookup always hit 32 different banks.
-__device__ __forceinline__ unsigned lds_u32(const unsigned* base, unsigned boff) {
-  return *reinterpret_cast<const unsigned*>(reinterpret_cast<const unsigned char*>(base) + boff);
+// Shared loads at 32-bit shared-window addresses. They are pure (no side effects, so the
+// compiler may schedule them freely): every address they get derives from a value passed
+// through launder() after the wait or barrier that made the data valid (a tile's copy, the
+// q' fragments of a unit, the tables), which keeps them after it.
+__device__ __forceinline__ unsigned launder(unsigned x) {
+  unsigned y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x) : "memory");
+  return y;
 }
-__device__ __forceinline__ uint2 lds_u64(const uint2* base, unsigned boff) {
-  return *reinterpret_cast<const uint2*>(reinterpret_cast<const unsigned char*>(base) + boff);
+__device__ __forceinline__ unsigned ld_s16(unsigned a) {
+  unsigned short v;
+  asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ unsigned ld_s32(unsigned a) {
+  unsigned v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float ld_sf32(unsigned a) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_s64(unsigned a) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_s128(unsigned a) {
+  uint4 v;
+  asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
 }
 // x >> s for an s that is known after unrolling and may be negative (a left shift).
 __device__ __forceinline__ unsigned shr(unsigned x, int s) { return s >= 0 ? x >> s : x << -s; }
 
-// Shared-memory tables of one CTA.
+// Byte-indexed tables (16 copies of each 8-byte entry, 256 rows of 256 bytes): the row of
+// code byte `byte` of w, plus the lane's copy offset c8 = 8 (lane % 16) < 128, in one prmt
+// (byte 0 of the result from c8, byte 1 from w, bytes 2-3 zero).
+__device__ __forceinline__ unsigned row8(unsigned w, unsigned c8, int byte) {
+  return prmt(w, c8, 0x5504u | (unsigned(byte) << 4));
+}
+constexpr int kTbl8Bytes = 256 * 256;   // rows: [0,128) rate-2 pair pairs, [128,256) rate-4 hi/lo pairs
+constexpr int kTbl3Bytes = 64 * 128;    // rate-3 hi/lo pairs, 6-bit index, 16 copies
+
+// Dynamic shared memory of a split CTA, at offsets fixed at compile time (so that every
+// table lookup is one shared load with an immediate offset): mbarriers, the byte table,
+// the rate-3 table, the value table of the value rate VR (rate 3: 64 lane-private
+// entries, rate 4: 256 shared ones), the q' fragments [pair slot][lane] (hi, hi, lo, lo),
+// then the ring of 2 stages per warp (its size depends on the layout's tile bytes).
+constexpr int kSmT8 = 256;
+constexpr int kSmT3 = kSmT8 + kTbl8Bytes;
+constexpr int kSmVt = kSmT3 + kTbl3Bytes;
+template <int VR>
+__host__ __device__ constexpr int vtab_bytes() { return VR == 3 ? 64 * 32 * 4 : VR == 4 ? 256 * 4 : 0; }
+constexpr int kPairSlots = kMaxQuads / 2 + kMaxGroups;  // quad pairs of all groups (a group's odd quad alone)
+template <int VR>
+__host__ __device__ constexpr int sm_qf() { return kSmVt + vtab_bytes<VR>(); }
+template <int VR>
+__host__ __device__ constexpr int sm_ring() { return (sm_qf<VR>() + kPairSlots * 32 * 16 + 127) / 128 * 128; }
+
 // A compile-time int carried as a value (row blocks per work item).
 template <int N>
 struct IntC {
   static constexpr int value = N;
 };
 
-template <int VR>
-struct Luts {
-  static constexpr int kV = VR == 2 ? 16 * 32 : VR == 3 ? 64 * 32 : VR == 4 ? 256 : 1;
-  unsigned k2[16 * 32];  // rate-2 key pairs, lane-private
-  uint2 k3[64];          // rate-3 key pairs {hi, lo}
-  uint2 k4[256];         // rate-4 key pairs {hi, lo}
-  unsigned v[kV];        // value pairs: rates 2-3 lane-private, rate 4 shared
-};
-
-// The lane's codes of one quad: Kq<R>::load reads them (rate 3: two planes) at the lane's
-// precomputed byte offsets, a(m) gives the fp16 pair (hi part for rates 3-4) of slot m
-// (token g + 8 m of the tile, dims 2t and 2t+1 of the quad), lo(m) the low parts.
-template <int R, int VR>
-struct Kq;
-template <int VR>
-struct Kq<1, VR> {
-  unsigned w;  // lo codes in bits 8-15, hi codes in bits 24-31
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
-    w = prmt(*reinterpret_cast<const unsigned short*>(tb + (off & 0xffffu)), 0u, 0x1404u);
+// The lane's codes of one quad of a key group with rate R: load() reads them at the lane's
+// byte offset (rate 3: two planes); `up` moves slots 4-7 to 0-3 (the upper half tile).
+template <int R>
+struct KCodes;
+template <>
+struct KCodes<1> {
+  unsigned w;  // lo codes in bits 0-7, hi codes in bits 16-23 (slot m at bits m, 16 + m)
+  __device__ __forceinline__ void load(unsigned tb, unsigned off, bool up) {
+    w = prmt(ld_s16(tb + (off & 0xffffu)), 0u, 0x4140u);
     if (up) w >>= 4;
   }
-  __device__ __forceinline__ unsigned a(int m, const Luts<VR>&, unsigned) const { return sign_pair(w << (7 - m)); }
-  __device__ __forceinline__ unsigned lo(int, const Luts<VR>&) const { return 0u; }
+  // fp16 pair of slot m: 0 or 2^(m - 24) per half (fp16 subnormals, exact on the tensor
+  // cores); the code c = +-a is 2 a bit - a, so the group's scores come out as
+  // 2^(25 - m) acc - sum of the B column (applied after the products)
+  __device__ __forceinline__ unsigned a(int m) const { return w & (0x00010001u << m); }
 };
-template <int VR>
-struct Kq<2, VR> {
-  unsigned w;  // nibble m = lo | hi << 2
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
-    w = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
+template <>
+struct KCodes<2> {
+  unsigned w;  // nibble m = lo | hi << 2; byte j = slots 2j, 2j+1
+  __device__ __forceinline__ void load(unsigned tb, unsigned off, bool up) {
+    w = ld_s32(tb + (off & 0xffffu));
     if (up) w >>= 16;
   }
-  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned lane4) const {
-    return lds_u32(T.k2, (shr(w, 4 * m - 7) & 0x780u) | lane4);  // entry at 128 nibble + 4 lane
-  }
-  __device__ __forceinline__ unsigned lo(int, const Luts<VR>&) const { return 0u; }
 };
-template <int VR>
-struct Kq<3, VR> {
-  unsigned f[8];  // byte offsets (8 x field) of the eight 6-bit fields in the pair table
-  uint2 e[8];
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
-    unsigned wa = *reinterpret_cast<const unsigned*>(tb + (off & 0xffffu));
-    const unsigned wb = *reinterpret_cast<const unsigned short*>(tb + (off >> 16));
-    if (up) wa = (wa >> 24) | (wb << 8);  // fields 4..7 to 0..3 (only those are used then)
-    f[0] = (wa << 3) & 0x1f8u;
-    f[1] = (wa >> 3) & 0x1f8u;
-    f[2] = (wa >> 9) & 0x1f8u;
-    f[3] = (wa >> 15) & 0x1f8u;
-    f[4] = (wa >> 21) & 0x1f8u;
-    f[5] = (__funnelshift_r(wa, wb, 30) << 3) & 0x1f8u;
-    f[6] = (wb >> 1) & 0x1f8u;
-    f[7] = (wb >> 7) & 0x1f8u;
-  }
-  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned) { e[m] = lds_u64(T.k3, f[m]); return e[m].x; }
-  __device__ __forceinline__ unsigned lo(int m, const Luts<VR>&) const { return e[m].y; }
-};
-template <int VR>
-struct Kq<4, VR> {
-  uint2 w;  // byte m = lo | hi << 4
-  uint2 e[8];
-  __device__ __forceinline__ void load(const unsigned char* tb, unsigned off, bool up = false) {
-    w = *reinterpret_cast<const uint2*>(tb + (off & 0xffffu));
-    if (up) w.x = w.y;
-  }
-  __device__ __forceinline__ unsigned a(int m, const Luts<VR>& T, unsigned) {
-    const unsigned x = m < 4 ? w.x : w.y;
-    e[m] = lds_u64(T.k4, shr(x, 8 * (m & 3) - 3) & 0x7f8u);
-    return e[m].x;
-  }
-  __device__ __forceinline__ unsigned lo(int m, const Luts<VR>&) const { return e[m].y; }
-};
-
-// Scores of one key group with compile-time rate R over its quads [q0, q1) of a tile.
-// Quads go in pairs into m16n8k16 products (quad q: k columns 0-7, quad q+1: 8-15); a
-// group's odd last quad takes an m16n8k8 product. Row block rt of the tile: rows g and
-// g+8 are slots m = 2 rt and 2 rt + 1. loff[q][lane] = byte offset of the lane's codes in
-// the tile (for a lane without a pair of that quad: any code, its q' rows are zero).
-// NRT = 4: the whole tile; NRT = 2: the half tile of row blocks 0-1 (up = false) or 2-3.
-template <int R, bool NP, int VR, int NRT>
-__device__ __forceinline__ void key_group(float (&acc)[NRT][4], const unsigned char* tb, const unsigned* loff,
-                                          const unsigned* qf, int q0, int q1, int lane, const Luts<VR>& T,
-                                          bool up) {
-  const unsigned lane4 = unsigned(lane) << 2;
-  int q = q0;
-#pragma unroll 1
-  for (; q + 1 < q1; q += 2) {
-    Kq<R, VR> c0, c1;
-    c0.load(tb, loff[q * 32 + lane], NRT < 4 && up);
-    c1.load(tb, loff[(q + 1) * 32 + lane], NRT < 4 && up);
-    const unsigned bh0 = qf[q * 64 + lane], bh1 = qf[(q + 1) * 64 + lane];
-    const unsigned bl0 = NP ? 0u : qf[q * 64 + 32 + lane], bl1 = NP ? 0u : qf[(q + 1) * 64 + 32 + lane];
-#pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) {
-      const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
-      const unsigned a2 = c1.a(2 * rt, T, lane4), a3 = c1.a(2 * rt + 1, T, lane4);
-      mma16816(acc[rt], a0, a1, a2, a3, bh0, bh1);
-      if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, bl0, bl1);
-      if constexpr (R >= 3)
-        mma16816(acc[rt], c0.lo(2 * rt, T), c0.lo(2 * rt + 1, T), c1.lo(2 * rt, T), c1.lo(2 * rt + 1, T), bh0, bh1);
+template <>
+struct KCodes<3> {
+  unsigned wa, wb;  // 48-bit string: field m (6 bits) at bit 6 m; plane B holds bits 32..47
+  __device__ __forceinline__ void load(unsigned tb, unsigned off, bool up) {
+    wa = ld_s32(tb + (off & 0xffffu));
+    wb = ld_s16(tb + (off >> 16));
+    if (up) {  // fields 4..7 to 0..3 (only those are used then)
+      wa = (wa >> 24) | (wb << 8);
+      wb = 0;
     }
   }
-  if (q < q1) {
-    Kq<R, VR> c0;
-    c0.load(tb, loff[q * 32 + lane], NRT < 4 && up);
-    const unsigned bh = qf[q * 64 + lane], bl = NP ? 0u : qf[q * 64 + 32 + lane];
+  // row offset (field x 128) plus the lane's copy offset
+  __device__ __forceinline__ unsigned row(int m, unsigned c8) const {
+    const int p = 6 * m;
+    unsigned x;
+    if (p + 6 <= 32) x = shr(wa, p - 7);
+    else if (p >= 32) x = shr(wb, p - 32 - 7);
+    else x = __funnelshift_r(wa, wb, p) << 7;
+    return (x & 0x1F80u) | c8;
+  }
+};
+template <>
+struct KCodes<4> {
+  uint2 w;  // byte m = lo | hi << 4
+  __device__ __forceinline__ void load(unsigned tb, unsigned off, bool up) {
+    w = ld_s64(tb + (off & 0xffffu));
+    if (up) w.x = w.y;
+  }
+};
+
+// Scores of one key group with compile-time rate R over its nq quads of a tile. Quads go in
+// pairs into m16n8k16 products (quad 2i: k columns 0-7, quad 2i+1: 8-15); a group's odd
+// last quad takes an m16n8k8 product. Row block rt of the work item: rows g and g+8 are
+// slots m = 2 rt and 2 rt + 1. The lane's codes of quad j of the group sit at kb + 64 R j
+// + lo_full (the last quad, which may hold fewer pairs: at off_last); a lane without a pair
+// of that quad reads any code, its q' rows are zero. qf4[j / 2] = the lane's (hi, hi, lo,
+// lo) B fragments of quad pair j / 2 (a single last quad: (hi, 0, lo, 0)).
+// NRT = 4: the whole tile; NRT = 2: the half tile of row blocks 0-1 (up = false) or 2-3.
+template <int R, bool NP, int NRT>
+__device__ __forceinline__ void key_group(float (&acc)[NRT][4], unsigned tb, unsigned kb, unsigned lo_full,
+                                          unsigned off_last, int nq, unsigned qf4, bool up, unsigned t8, unsigned t3,
+                                          unsigned c8) {
+  // a full quad block is 16 x 4 pairs x R bytes; rate-3 offsets hold both planes' offsets
+  // (low and high halfword), so a step moves both
+  constexpr unsigned kQuadBytes = R == 3 ? 64u * R * 0x10001u : 64u * R;
+  unsigned off = kb * (R == 3 ? 0x10001u : 1u) + lo_full;
+  int j = 0;
+#pragma unroll 1
+  for (; j + 1 < nq; j += 2, off += 2 * kQuadBytes) {
+    KCodes<R> c0, c1;
+    c0.load(tb, off, NRT < 4 && up);
+    c1.load(tb, j + 2 == nq ? off_last : off + kQuadBytes, NRT < 4 && up);
+    const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
 #pragma unroll
     for (int rt = 0; rt < NRT; ++rt) {
-      const unsigned a0 = c0.a(2 * rt, T, lane4), a1 = c0.a(2 * rt + 1, T, lane4);
-      mma1688(acc[rt], a0, a1, bh);
-      if constexpr (!NP) mma1688(acc[rt], a0, a1, bl);
-      if constexpr (R >= 3) mma1688(acc[rt], c0.lo(2 * rt, T), c0.lo(2 * rt + 1, T), bh);
+      const int m = 2 * rt;
+      unsigned a0, a1, a2, a3, l0 = 0, l1 = 0, l2 = 0, l3 = 0;
+      if constexpr (R == 1) {
+        a0 = c0.a(m);
+        a1 = c0.a(m + 1);
+        a2 = c1.a(m);
+        a3 = c1.a(m + 1);
+      } else if constexpr (R == 2) {
+        const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt)), e1 = ld_s64(t8 + row8(c1.w, c8, rt));
+        a0 = e0.x;
+        a1 = e0.y;
+        a2 = e1.x;
+        a3 = e1.y;
+      } else if constexpr (R == 3) {
+        const uint2 e0 = ld_s64(t3 + c0.row(m, c8)), e1 = ld_s64(t3 + c0.row(m + 1, c8));
+        const uint2 e2 = ld_s64(t3 + c1.row(m, c8)), e3 = ld_s64(t3 + c1.row(m + 1, c8));
+        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y, a2 = e2.x, l2 = e2.y, a3 = e3.x, l3 = e3.y;
+      } else {
+        const unsigned x0 = m < 4 ? c0.w.x : c0.w.y, x1 = m < 4 ? c1.w.x : c1.w.y;
+        const uint2 e0 = ld_s64(t8 + 128 + row8(x0, c8, m & 3)), e1 = ld_s64(t8 + 128 + row8(x0, c8, (m & 3) + 1));
+        const uint2 e2 = ld_s64(t8 + 128 + row8(x1, c8, m & 3)), e3 = ld_s64(t8 + 128 + row8(x1, c8, (m & 3) + 1));
+        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y, a2 = e2.x, l2 = e2.y, a3 = e3.x, l3 = e3.y;
+      }
+      mma16816(acc[rt], a0, a1, a2, a3, f.x, f.y);
+      if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, f.z, f.w);
+      if constexpr (R >= 3) mma16816(acc[rt], l0, l1, l2, l3, f.x, f.y);
+    }
+  }
+  if (j < nq) {
+    KCodes<R> c0;
+    c0.load(tb, j + 1 == nq ? off_last : off, NRT < 4 && up);
+    const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
+#pragma unroll
+    for (int rt = 0; rt < NRT; ++rt) {
+      const int m = 2 * rt;
+      unsigned a0, a1, l0 = 0, l1 = 0;
+      if constexpr (R == 1) {
+        a0 = c0.a(m);
+        a1 = c0.a(m + 1);
+      } else if constexpr (R == 2) {
+        const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt));
+        a0 = e0.x;
+        a1 = e0.y;
+      } else if constexpr (R == 3) {
+        const uint2 e0 = ld_s64(t3 + c0.row(m, c8)), e1 = ld_s64(t3 + c0.row(m + 1, c8));
+        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y;
+      } else {
+        const unsigned x0 = m < 4 ? c0.w.x : c0.w.y;
+        const uint2 e0 = ld_s64(t8 + 128 + row8(x0, c8, m & 3)), e1 = ld_s64(t8 + 128 + row8(x0, c8, (m & 3) + 1));
+        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y;
+      }
+      mma1688(acc[rt], a0, a1, f.x);
+      if constexpr (!NP) mma1688(acc[rt], a0, a1, f.z);
+      if constexpr (R >= 3) mma1688(acc[rt], l0, l1, f.x);
     }
   }
 }
@@ -310,23 +384,23 @@ __device__ __forceinline__ void key_group(float (&acc)[NRT][4], const unsigned c
 template <int VR>
 struct ValueLane {
   unsigned w[2 * VR];
-  __device__ __forceinline__ void load(const unsigned char* vblk, int lane) {
+  __device__ __forceinline__ void load(unsigned vblk, int lane) {
     if constexpr (VR == 1) {
-      const uint2 x = reinterpret_cast<const uint2*>(vblk)[lane];
+      const uint2 x = ld_s64(vblk + 8 * lane);
       w[0] = x.x;
       w[1] = x.y;
     } else {
-      const uint4 x = reinterpret_cast<const uint4*>(vblk)[lane];
+      const uint4 x = ld_s128(vblk + 16 * lane);
       w[0] = x.x;
       w[1] = x.y;
       w[2] = x.z;
       w[3] = x.w;
       if constexpr (VR == 3) {
-        const uint2 y = reinterpret_cast<const uint2*>(vblk + 512)[lane];
+        const uint2 y = ld_s64(vblk + 512 + 8 * lane);
         w[4] = y.x;
         w[5] = y.y;
       } else if constexpr (VR == 4) {
-        const uint4 y = reinterpret_cast<const uint4*>(vblk + 512)[lane];
+        const uint4 y = ld_s128(vblk + 512 + 16 * lane);
         w[4] = y.x;
         w[5] = y.y;
         w[6] = y.z;
@@ -334,318 +408,217 @@ struct ValueLane {
       }
     }
   }
-  // fp16 pair of field n (compile-time after unrolling)
-  __device__ __forceinline__ unsigned field(int n, const unsigned* vlut, unsigned lane4) const {
+  // the four A registers of m-tile mt (compile-time after unrolling). Rate 2: byte 2 mt
+  // (fields 4 mt, 4 mt + 1) and byte 2 mt + 1 of the string, each one row of the byte table.
+  __device__ __forceinline__ void regs(int mt, unsigned t8, unsigned vlut, unsigned c8, unsigned lane4,
+                                       unsigned (&a)[4]) const {
+    if constexpr (VR == 2) {
+      const uint2 e0 = ld_s64(t8 + row8(w[mt >> 1], c8, 2 * (mt & 1)));
+      const uint2 e1 = ld_s64(t8 + row8(w[mt >> 1], c8, 2 * (mt & 1) + 1));
+      a[0] = e0.x;
+      a[1] = e0.y;
+      a[2] = e1.x;
+      a[3] = e1.y;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) a[k] = field(4 * mt + k, vlut, lane4);
+    }
+  }
+  __device__ __forceinline__ unsigned field(int n, unsigned vlut, unsigned lane4) const {
     if constexpr (VR == 1) {
       return sign_pair(w[n >> 4] << (15 - (n & 15)));
-    } else if constexpr (VR == 2) {
-      return lds_u32(vlut, (shr(w[n >> 3], 4 * (n & 7) - 7) & 0x780u) | lane4);
     } else if constexpr (VR == 3) {
       const int bit = 6 * n, wi = bit >> 5, sh = bit & 31;
       const unsigned x = sh <= 26 ? (w[wi] >> sh) : __funnelshift_r(w[wi], w[wi + 1], sh);
-      return lds_u32(vlut, ((x & 63u) << 7) | lane4);
+      return ld_s32(vlut + (((x & 63u) << 7) | lane4));
     } else {
-      return lds_u32(vlut, shr(w[n >> 2], 8 * (n & 3) - 2) & 0x3fcu);
+      return ld_s32(vlut + (shr(w[n >> 2], 8 * (n & 3) - 2) & 0x3fcu));
     }
   }
 };
 
 // The slice of CTA c: tiles [c T / C, (c+1) T / C) of the units x M = T tiles laid end to
-// end (C CTAs, C <= T, slices at most M long), i.e. one or two segments, each a tile range
-// of one unit (clipped to the unit's length when streamed).
+// end, i.e. a run of segments, each a tile range of one unit (clipped to the unit's length
+// when streamed).
 __host__ __device__ inline int cta_of_tile(long long x, long long T, long long C) { return int(((x + 1) * C - 1) / T); }
 
 struct Segment {
-  int u;        // unit = batch row * h_kv + KV head
-  int lt0;      // first tile (inside the unit) of the slice
-  int n;        // tiles to stream (after clipping to the unit's length)
-  int part;     // partial slot of this CTA for the unit
+  int u;          // unit = batch row * h_kv + KV head
+  int lt0;        // first tile (inside the unit) of the slice
+  int n;          // tiles to stream (after clipping to the unit's length)
+  int part;       // partial slot of this CTA for the unit
   long long len;  // tokens of the unit
 };
 
-__device__ __forceinline__ int cta_segments(const DevLayout& L, const SplitArgs& a, int c, Segment* seg, int tid) {
+__device__ __forceinline__ Segment make_segment(const DevLayout& L, const SplitArgs& a, int c, int u, bool flag) {
   const long long M = a.max_tiles, T = a.total_tiles, C = a.n_ctas;
   const long long g0 = (long long)c * T / C, g1 = (long long)(c + 1) * T / C;
-  const int u0 = int(g0 / M), u1 = int((g1 - 1) / M);
-  int nseg = 0;
-  for (int u = u0; u <= u1 && nseg < 2; ++u, ++nseg) {
-    const int b = u / a.h_kv;
-    long long len = (long long)a.seq_lens[b] + a.len_add;
-    if (len < 0) len = 0;
-    const long long cap_tokens = min(a.cache.n_tiles, M) * kTile;
-    const long long a0 = max(g0, (long long)u * M) - (long long)u * M;
-    const long long a1 = min(g1, (long long)(u + 1) * M) - (long long)u * M;
-    if (len > cap_tokens) {
-      if (tid == 0 && a0 == 0) atomicOr(L.status, BGTQ_STATUS_DECODE_CLAMPED);
-      len = cap_tokens;
-    }
-    const long long len_tiles = (len + kTile - 1) / kTile;
-    seg[nseg].u = u;
-    seg[nseg].lt0 = int(a0);
-    seg[nseg].n = int(max(0LL, min(a1, len_tiles) - a0));
-    seg[nseg].part = c - cta_of_tile((long long)u * M, T, C);
-    seg[nseg].len = len;
+  const int b = u / a.h_kv;
+  long long len = (long long)a.seq_lens[b] + a.len_add;
+  if (len < 0) len = 0;
+  const long long cap_tokens = min(a.cache.n_tiles, M) * kTile;
+  const long long a0 = max(g0, (long long)u * M) - (long long)u * M;
+  const long long a1 = min(g1, (long long)(u + 1) * M) - (long long)u * M;
+  if (len > cap_tokens) {
+    if (flag && a0 == 0) atomicOr(L.status, BGTQ_STATUS_DECODE_CLAMPED);
+    len = cap_tokens;
   }
-  return nseg;
-}
-
-// q' B fragments of unit u (batch row b, KV head h) into frag[kMaxQuads][2][32] (global),
-// by one CTA of kPrepThreads: thread (p = tid % 128, half = tid / 128) computes
-// q'[hh][p] = f_g sum_j R_g[i][j] q[hh][off_g + j] for the heads hh = 4 half .. 4 half + 3
-// (16-byte rows of R_g from global memory, q staged in shared memory); with G <= 4 the
-// two halves take heads 0..3 over the two halves of the row instead (all of a thread's
-// row is then loaded before q arrives) and add up in shared memory. Then every fragment
-// word is written once. With G <= 4 the eight B columns are heads 0..3 (hi
-// parts) and heads 0..3 again (lo parts) in the first array; otherwise the first array
-// holds the hi parts of heads 0..7 and the second the lo parts. Missing pairs and heads
-// are zero.
-constexpr int kPrepThreads = 256;
-static_assert(kPrepThreads == enc::kEncodeThreads, "the step kernel runs both bodies");
-
-__device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __restrict__ q, int q_dtype, int h_q,
-                                          int h_kv, int G, int n_q, float qscale, int u, unsigned* __restrict__ frag) {
-  __shared__ __align__(16) float qs[kMaxG * kQsLd];  // q per group at 16-byte aligned columns
-  __shared__ float qr[kMaxG * kD];                   // q' in packed order
-  const int tid = threadIdx.x, ng = L.n_kgroups;
-  const int b = u / h_kv, h = u % h_kv;
-  __shared__ float red[4 * kD];                      // the k-split halves' partial sums
-  // this thread's row of R_g (columns [4 c0, 4 c1)): the first 16 float4 are loaded
-  // before q arrives
-  const int p = tid & (kD - 1), half = tid >> 7;
-  const bool ksplit = G <= 4;
-  const int h0 = ksplit ? 0 : half * 4;
-  int g = 0, pad = 0;
-  while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
-  const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
-  // packed dims past n_packed (rate-0 blocks) have no row: no loads, q' = 0
-  const int n4 = p < L.n_packed ? ld / 4 : 0, c0 = ksplit ? half * ((n4 + 1) / 2) : 0, c1 = ksplit ? min(n4, c0 + (n4 + 1) / 2) : n4;
-  const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld) + c0;
-  constexpr int kPre = 16;
-  float4 r[kPre];
-#pragma unroll
-  for (int j4 = 0; j4 < kPre; ++j4) r[j4] = c0 + j4 < c1 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int e = tid; e < kMaxG * kQsLd; e += kPrepThreads) qs[e] = 0.f;
-  __syncthreads();
-  // in a decode step (launched as a programmatic dependent) the CTA got here, rows of R in
-  // flight, while the kernel before it ran; q is the caller's: wait for that kernel before
-  // reading it. Only then may the split kernel launch: it reads the cache, which that
-  // kernel may write. (q-prep alone is a plain launch: both are no-ops there.)
-  pdl_wait();
-  pdl_trigger();
-  for (int e = tid; e < G * kD; e += kPrepThreads) {
-    const int hh = e >> 7, pe = e & (kD - 1);
-    if (pe >= L.n_packed) continue;
-    int ge = 0, pade = 0;
-    while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
-    // column hh: query head h G / n_q + hh / n_q at query token hh % n_q of q [b][token][head]
-    const size_t qrow = ((size_t)b * n_q + hh % n_q) * h_q + (size_t)h * (G / n_q) + hh / n_q;
-    qs[hh * kQsLd + pade + pe - L.group_off[ge]] = load_q(q, q_dtype, qrow * kD + L.packed_coord[pe]);
-  }
-  __syncthreads();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (h0 < G) {
-    const float* qg = qs + h0 * kQsLd + pad + 4 * c0;
-#pragma unroll
-    for (int j4 = 0; j4 < kPre; ++j4) {
-      if (c0 + j4 < c1) {  // q columns past the group's padded row are not read
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
-          acc[k] = fmaf(r[j4].x, x.x, fmaf(r[j4].y, x.y, fmaf(r[j4].z, x.z, fmaf(r[j4].w, x.w, acc[k]))));
-        }
-      }
-    }
-#pragma unroll 8
-    for (int j4 = kPre; c0 + j4 < c1; ++j4) {
-      const float4 rr = __ldg(row + j4);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
-        acc[k] = fmaf(rr.x, x.x, fmaf(rr.y, x.y, fmaf(rr.z, x.z, fmaf(rr.w, x.w, acc[k]))));
-      }
-    }
-  }
-  if (ksplit) {  // uniform over the CTA
-    if (half == 1)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) red[k * kD + p] = acc[k];
-    __syncthreads();
-    if (half == 0)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] += red[k * kD + p];
-  }
-  if (h0 < G && (!ksplit || half == 0)) {
-    const float f = qscale * rsqrtf(float(d)) * L.inv_kappa_group[g];  // the key tables carry kappa
-#pragma unroll
-    for (int k = 0; k < 4; ++k) qr[(h0 + k) * kD + p] = acc[k] * f;
-  }
-  __syncthreads();
-  for (int e = tid; e < L.n_kquads * 64; e += kPrepThreads) {
-    const int qi = e >> 6, j = e & 63, lane = j & 31, n = lane >> 2, t = lane & 3;
-    const bool lo_half = j >= 32;
-    const int d0 = L.quad_dim0[qi] + 2 * t;
-    const int hh = G <= 4 ? (n & 3) : n;
-    const bool lo = G <= 4 ? n >= 4 : lo_half;
-    float v0 = 0.f, v1 = 0.f;
-    if (t < L.quad_np[qi] && hh < G && !(G <= 4 && lo_half)) {
-      v0 = qr[hh * kD + d0];
-      v1 = qr[hh * kD + d0 + 1];
-    }
-    const float r0 = __half2float(__float2half_rn(v0)), r1 = __half2float(__float2half_rn(v1));
-    frag[qi * 64 + j] = lo ? pack_h2(v0 - r0, v1 - r1) : pack_h2(r0, r1);
-  }
-}
-
-__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
-                                                             int h_q, int h_kv, int G, int n_q, float qscale,
-                                                             unsigned* __restrict__ qfrag) {
-  // launched after the kernel before it has completed: the split kernel may start now
-  pdl_trigger();
-  const int u = blockIdx.x;
-  prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
-}
-
-// First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
-// token and KV head), the others prepare q' of one unit each.
-template <bool NC>
-__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
-                                                                 const void* __restrict__ v, int kv_dtype, int n_new,
-                                                                 int batch, const int* __restrict__ seq_lens_before,
-                                                                 CacheRef cache,
-                                                                 const void* __restrict__ q, int q_dtype, int h_q,
-                                                                 int h_kv, int G, int n_q, float qscale,
-                                                                 unsigned* __restrict__ qfrag, int n_enc) {
-  // every block triggers its dependent (the split kernel) after its own wait for the
-  // kernel before it (in the encode and q-prep bodies; padding blocks by exiting)
-  const int e = blockIdx.x;
-  if (e < n_enc) {
-    const int part = e % kEncodeParts;
-    int rest = e / kEncodeParts;
-    const int t = rest % n_new;
-    rest /= n_new;
-    const int b = rest % batch, h = rest / batch;
-    enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
-  } else if (e - n_enc < batch * h_kv) {  // (a cluster launch pads the grid)
-    const int u = e - n_enc;
-    prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kMaxQuads * 64);
-  }
+  const long long len_tiles = (len + kTile - 1) / kTile;
+  Segment s;
+  s.u = u;
+  s.lt0 = int(a0);
+  s.n = int(max(0LL, min(a1, len_tiles) - a0));
+  s.part = c - cta_of_tile((long long)u * M, T, C);
+  s.len = len;
+  return s;
 }
 
 // Norm i of a tile's norm area, stored as fp16 (NH) or fp32.
 template <bool NH>
-__device__ __forceinline__ float tile_norm(const unsigned char* area, int i) {
-  if constexpr (NH) return __half2float(reinterpret_cast<const __half*>(area)[i]);
-  else return reinterpret_cast<const float*>(area)[i];
+__device__ __forceinline__ float tile_norm(unsigned area, int i) {
+  if constexpr (NH) return __half2float(__ushort_as_half((unsigned short)ld_s16(area + 2 * i)));
+  else return ld_sf32(area + 4 * i);
 }
 
 // SC: scores only. The tiles' logits (softmax_scale q . k_hat, natural units) go to
 // a.scores; no softmax, values, partials or merge. NH: the layout stores fp16 norms.
+// W: warps per CTA (one CTA per SM).
 // (the scores-only instantiation discards the softmax and value code of the tile body)
 #pragma nv_diag_suppress 128
-template <int VR, bool NP, bool SC, bool NH>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L, SplitArgs a) {
+template <int VR, bool NP, bool SC, bool NH, int W>
+__global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ __align__(16) Luts<VR> T;
-  __shared__ unsigned s_loff[kMaxQuads * 32];  // [quad][lane]: byte offsets of the lane's codes in a tile
-  __shared__ int s_group[kMaxGroups][3];      // first quad, end quad, rate
+  // per key rate r (1..4): its group (-1: none), quads, byte offset of its first quad in a
+  // tile, first q' pair slot; per lane: its offset inside a full quad and the offset of
+  // its codes in the group's last quad
+  __shared__ int s_gi[5], s_gnq[5], s_gkb[5], s_gslot[5];
+  __shared__ unsigned s_lof[5][32], s_olast[5][32];
   __shared__ int s_timeout;
-  __shared__ Segment s_seg[2];
-  __shared__ int s_nseg;
+  __shared__ float s_mm[W][8], s_ml[W][8];
   const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int TB = L.tile_bytes;
 
-  unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);  // [kRing]
-  unsigned char* ring = smem + 128;                                        // stage s at ring + s TB
-  unsigned* qf = reinterpret_cast<unsigned*>(ring + kRing * TB);           // [quad][2][32]
-  float* mm = reinterpret_cast<float*>(qf + L.n_kquads * 64);              // [warp][8]
-  float* ml = mm + kWarps * 8;                                             // [warp][8]
-  // the warps' [8][128] partials reuse the ring once every tile of the segment is consumed
-  float* mo = reinterpret_cast<float*>(ring);
+  unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);  // [2 W]
+  unsigned char* t8 = smem + kSmT8;
+  unsigned char* t3 = smem + kSmT3;
+  unsigned* vlut = reinterpret_cast<unsigned*>(smem + kSmVt);
+  uint4* qf4 = reinterpret_cast<uint4*>(smem + sm_qf<VR>());         // [pair slot][lane]
+  unsigned char* ring = smem + sm_ring<VR>();                           // stage s at ring + s TB
+  float* mo = reinterpret_cast<float*>(ring);  // the warps' [8][128] partials reuse the ring
 
   if (tid == 0) {
     s_timeout = 0;
-    s_nseg = cta_segments(L, a, c, s_seg, 0);
-    for (int i = 0; i < kRing; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < 2 * W; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
-  // pair tables from the layout's fp16 codebooks: only those of the rates it uses
+  // tables from the layout's fp16 codebooks: only those the layout uses. The codebooks
+  // (kernel parameters) are first staged in shared memory: read with a different index in
+  // every lane, the parameter bank would serialise.
+  __shared__ unsigned short s_cb[4 + 16 + 32 + 16];  // kc2, kc3 [hi, lo][8], kc4 [hi, lo][16], vc
+  if (tid < 4) s_cb[tid] = L.kc2[tid];
+  else if (tid < 20) s_cb[tid] = L.kc3[(tid - 4) >> 3][(tid - 4) & 7];
+  else if (tid < 52) s_cb[tid] = L.kc4[(tid - 20) >> 4][(tid - 20) & 15];
+  else if (tid < 68) s_cb[tid] = L.vc[tid - 52];
+  __syncthreads();
+  const unsigned short *c2 = s_cb, *c3h = s_cb + 4, *c3l = s_cb + 12, *c4h = s_cb + 20, *c4l = s_cb + 36, *cv = s_cb + 52;
   unsigned has = 0;
   for (int gi = 0; gi < L.n_kgroups; ++gi) has |= 1u << L.group_rate[gi];
-  if (has & 4u)
-    for (int i = tid; i < 16 * 32; i += kThreads) {
-      const int e = i >> 5;
-      T.k2[i] = unsigned(L.kc2[e & 3]) | (unsigned(L.kc2[e >> 2]) << 16);
+  if ((has & 4u) || VR == 2) {
+    // rate-2 pair pairs: row e = code byte (nibble = lo | hi << 2 of one slot), 16 copies
+    const unsigned short* cb = (has & 4u) ? c2 : cv;
+    for (int i = tid; i < 256 * 16; i += 32 * W) {
+      const int e = i >> 4, cp = i & 15;
+      const uint2 v = make_uint2(unsigned(cb[e & 3]) | (unsigned(cb[(e >> 2) & 3]) << 16),
+                                 unsigned(cb[(e >> 4) & 3]) | (unsigned(cb[e >> 6]) << 16));
+      *reinterpret_cast<uint2*>(t8 + e * 256 + cp * 8) = v;
+    }
+  }
+  if (has & 16u)
+    for (int i = tid; i < 256 * 16; i += 32 * W) {
+      const int e = i >> 4, cp = i & 15;
+      const uint2 v = make_uint2(unsigned(c4h[e & 15]) | (unsigned(c4h[e >> 4]) << 16),
+                                 unsigned(c4l[e & 15]) | (unsigned(c4l[e >> 4]) << 16));
+      *reinterpret_cast<uint2*>(t8 + e * 256 + 128 + cp * 8) = v;
     }
   if (has & 8u)
-    for (int e = tid; e < 64; e += kThreads)
-      T.k3[e] = make_uint2(unsigned(L.kc3[0][e & 7]) | (unsigned(L.kc3[0][e >> 3]) << 16),
-                           unsigned(L.kc3[1][e & 7]) | (unsigned(L.kc3[1][e >> 3]) << 16));
-  if (has & 16u)
-    for (int e = tid; e < 256; e += kThreads)
-      T.k4[e] = make_uint2(unsigned(L.kc4[0][e & 15]) | (unsigned(L.kc4[0][e >> 4]) << 16),
-                           unsigned(L.kc4[1][e & 15]) | (unsigned(L.kc4[1][e >> 4]) << 16));
-  if constexpr (VR == 2 || VR == 3) {
-    // lane-private pair tables: entry e of lane l at 32 e + l (no bank conflicts)
-    constexpr unsigned vm = (1u << VR) - 1u;
-    for (int i = tid; i < Luts<VR>::kV; i += kThreads) {
+    for (int i = tid; i < 64 * 16; i += 32 * W) {
+      const int e = i >> 4, cp = i & 15;
+      const uint2 v = make_uint2(unsigned(c3h[e & 7]) | (unsigned(c3h[e >> 3]) << 16),
+                                 unsigned(c3l[e & 7]) | (unsigned(c3l[e >> 3]) << 16));
+      *reinterpret_cast<uint2*>(t3 + e * 128 + cp * 8) = v;
+    }
+  if constexpr (VR == 3) {
+    // lane-private pair table: entry e of lane l at word 32 e + l (no bank conflicts)
+    for (int i = tid; i < 64 * 32; i += 32 * W) {
       const int e = i >> 5;
-      T.v[i] = unsigned(L.vc[e & vm]) | (unsigned(L.vc[e >> VR]) << 16);
+      vlut[i] = unsigned(cv[e & 7]) | (unsigned(cv[e >> 3]) << 16);
     }
   } else if constexpr (VR == 4) {
-    for (int e = tid; e < 256; e += kThreads) T.v[e] = unsigned(L.vc[e & 15]) | (unsigned(L.vc[e >> 4]) << 16);
+    for (int e = tid; e < 256; e += 32 * W) vlut[e] = unsigned(cv[e & 15]) | (unsigned(cv[e >> 4]) << 16);
   }
-  for (int gi = 0; gi < L.n_kgroups; ++gi) {
-    const int r = L.group_rate[gi], q0 = L.group_quad0[gi];
-    for (int i = tid; i < L.group_nquads[gi] * 32; i += kThreads) {
-      // lane (g, t) holds pair t of the quad for tokens g + 8m: its 16 r bits are string
-      // li = g P + t of the block (rate 3: plane A word li, plane B halfword li after 8 P words)
-      const int qi = q0 + i / 32, ln = i % 32, P = L.quad_np[qi], t = ln & 3;
-      const int li = t < P ? (ln >> 2) * P + t : 0;
-      const unsigned base = unsigned(L.quad_off[qi]);
-      s_loff[qi * 32 + ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
-    }
-  }
+  if (tid < 5) s_gi[tid] = -1;
+  __syncthreads();
   if (tid < L.n_kgroups) {
-    s_group[tid][0] = L.group_quad0[tid];
-    s_group[tid][1] = L.group_quad0[tid] + L.group_nquads[tid];
-    s_group[tid][2] = L.group_rate[tid];
+    // groups are in descending rate order: the pair slots of the groups before this one
+    int slot = 0;
+    for (int gj = 0; gj < tid; ++gj) slot += (L.group_nquads[gj] + 1) >> 1;
+    const int r = L.group_rate[tid];
+    s_gi[r] = tid;
+    s_gnq[r] = L.group_nquads[tid];
+    s_gkb[r] = L.quad_off[L.group_quad0[tid]];
+    s_gslot[r] = slot;
+  }
+  for (int i = tid; i < L.n_kgroups * 32; i += 32 * W) {
+    // lane (g, t) holds pair t of a quad for tokens g + 8m: its 16 r bits are string
+    // li = g P + t of the quad's block (rate 3: plane A word li, plane B halfword li after
+    // 8 P words). Full quads have P = 4 (li = lane).
+    const int gi = i >> 5, ln = i & 31, r = L.group_rate[gi];
+    const int ql = L.group_quad0[gi] + L.group_nquads[gi] - 1, P = L.quad_np[ql], tt = ln & 3;
+    const int li = tt < P ? (ln >> 2) * P + tt : 0;
+    const unsigned full = r == 3 ? 4u * ln | ((128u + 2u * ln) << 16) : 2u * r * ln;
+    const unsigned base = unsigned(L.quad_off[ql]);
+    s_lof[r][ln] = full;
+    s_olast[r][ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
   }
   __syncthreads();
-  const int nseg = s_nseg;
 
-  // Warp w streams its own tiles w, w+4, w+8, ... of a segment through the two ring stages
-  // w and w+4 (its k-th tile in stage w + 4 (k & 1)): lane 0 issues tile k+2 as soon as
-  // the warp is done with tile k, so no other warp ever waits on these stages.
-  const int ng = L.n_kgroups;
   const float vscale = rsqrtf(float(kD)) / L.kappa_v;
   const unsigned lane4 = unsigned(lane) << 2;
+  // 32-bit shared-window addresses of the tables (valid from here on) and of the ring
+  const unsigned sbase = smem_addr(smem);
+  const unsigned t8a = launder(sbase + kSmT8), t3a = launder(sbase + kSmT3), vluta = launder(sbase + kSmVt);
+  const unsigned ringa = sbase + sm_ring<VR>();
+  const unsigned c8 = unsigned(lane & 15) << 3;
   const unsigned long long l2_stream = evict_first_policy();
-  unsigned phase = 0;   // bit k&1: parity of the next completion of stage w + 4 (k & 1)
-  unsigned pend = 0;    // bit k&1: a copy into stage w + 4 (k & 1) is in flight
+  const long long M = a.max_tiles, T = a.total_tiles, C = a.n_ctas;
+  const long long g0 = (long long)c * T / C, g1 = (long long)(c + 1) * T / C;
+  const int u_first = int(g0 / M), u_last = int((g1 - 1) / M);
+  unsigned phase = 0;   // bit k&1: parity of the next completion of stage w + W (k & 1)
   bool waited = !a.wait_new;
-  for (int si = 0; si < nseg; ++si) {
-    const Segment S = s_seg[si];
+  bool q_ready = false;
+
+  for (int u = u_first; u <= u_last; ++u) {
+    const Segment S = make_segment(L, a, c, u, tid == 0);
     const int srow = S.u / a.h_kv, shead = S.u % a.h_kv;
-    const long long first_new = waited ? 0 : a.seq_lens[S.u / a.h_kv];
-    // Work items of this warp: full tiles w, w+4, ... of the first 4 floor(n/4); of the
-    // n % 4 tiles left, one each for warps 0-2 if three are left, else half tiles (row
-    // blocks 0-1 or 2-3), so that no warp runs more than half a tile past the others.
-    // Both warps of a split tile copy all of it into their own stages.
-    const int nfw = S.n >> 2, rem = S.n & 3;
-    const bool extra = rem == 3 ? warp < 3 : rem == 2 ? true : rem == 1 ? warp < 2 : false;
+    const long long first_new = waited ? 0 : a.seq_lens[srow];
+    // Work items of this warp: full tiles w, w+W, ... of the first W floor(n/W); the
+    // rem = n % W tiles left go one to each of the first rem warps, or, when 2 rem <= W,
+    // as half tiles (row blocks 0-1 and 2-3) to the first 2 rem warps. Both warps of a
+    // split tile copy all of it into their own stages.
+    const int nfw = S.n / W, rem = S.n % W;
+    const bool halves = rem > 0 && 2 * rem <= W;
+    const bool extra = halves ? warp < 2 * rem : warp < rem;
     const int mine = nfw + (extra ? 1 : 0);
-    auto item_tile = [&](int k) {
-      return (k < nfw || rem == 3) ? warp + kWarps * k : kWarps * nfw + (rem == 2 ? (warp >> 1) : 0);
-    };
+    auto item_tile = [&](int k) { return k < nfw ? warp + W * k : W * nfw + (halves ? (warp >> 1) : warp); };
     auto issue = [&](int k) {  // lane 0 only
       const int it = S.lt0 + item_tile(k);
       if (!waited && (long long)(it + 1) * kTile > first_new) {
         pdl_wait();  // this tile receives tokens from the encode kernel
         waited = true;
       }
-      const int st = warp + kWarps * (k & 1);
+      const int st = warp + W * (k & 1);
       const uint8_t* src = tile_ptr(a.cache, L, srow, shead, a.h_kv, it);
       if (src) {
         mbar_expect_tx(&full[st], TB);
@@ -656,13 +629,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
     };
     if (lane == 0)
       for (int k = 0; k < min(2, mine); ++k) issue(k);
-    pend = mine >= 2 ? 3u : mine == 1 ? 1u : 0u;
-    if (si == 0) pdl_wait();  // q' fragments come from the preparation kernel
-    {
-      const uint4* src4 = reinterpret_cast<const uint4*>(a.qfrag + (size_t)S.u * kMaxQuads * 64);
-      for (int e = tid; e < L.n_kquads * 16; e += kThreads) reinterpret_cast<uint4*>(qf)[e] = src4[e];
+    unsigned pend = mine >= 2 ? 3u : mine == 1 ? 1u : 0u;  // bit k&1: a copy into that stage is in flight
+    if (!q_ready) {
+      pdl_wait();  // q' fragments come from the preparation kernel
+      q_ready = true;
     }
+    const unsigned* src = a.qfrag + (size_t)S.u * kQfragWords;
+    {
+      // q' fragments of the unit, re-laid per group by quad pair: [slot][lane] = (hi of
+      // quad 2k, hi of 2k+1, lo of 2k, lo of 2k+1), zeros for a missing odd partner
+      int slot = 0;
+      for (int gi = 0; gi < L.n_kgroups; ++gi) {
+        const int q0 = L.group_quad0[gi], nq = L.group_nquads[gi];
+        for (int e = tid; e < ((nq + 1) >> 1) * 32; e += 32 * W) {
+          const int k = e >> 5, ln = e & 31, qa = q0 + 2 * k;
+          const bool pair = 2 * k + 1 < nq;
+          qf4[(slot + k) * 32 + ln] = make_uint4(src[qa * 64 + ln], pair ? src[(qa + 1) * 64 + ln] : 0u,
+                                                 src[qa * 64 + 32 + ln], pair ? src[(qa + 1) * 64 + 32 + ln] : 0u);
+        }
+        slot += (nq + 1) >> 1;
+      }
+    }
+    // column sums of the rate-1 group's B fragments (its 0/1 operands need them)
+    const int sbc = 2 * t;  // this lane's B columns 2t, 2t+1
+    const float sb0 = s_gi[1] >= 0 ? reinterpret_cast<const float*>(src + kMaxQuads * 64)[sbc] : 0.f;
+    const float sb1 = s_gi[1] >= 0 ? reinterpret_cast<const float*>(src + kMaxQuads * 64)[sbc + 1] : 0.f;
     __syncthreads();
+    const unsigned qf4a = launder(sbase + sm_qf<VR>());  // the unit's fragments are in
 
     float O[8][4];
 #pragma unroll
@@ -673,41 +666,56 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
 
     // Row blocks rb0 .. rb0 + NRT - 1 of the tile in stage tb; gt0 = token of row g of
     // row block rb0.
-    auto rows = [&](auto nrt, const unsigned char* tb, int rb0, long long gt0) {
+    auto rows = [&](auto nrt, unsigned tb, int rb0, long long gt0) {
       constexpr int NRT = decltype(nrt)::value;
       const bool up = rb0 != 0;
 
       // ---------------- scores: per key group (rate as a template parameter), per quad,
       // NRT row blocks; then times the group norms
-      const unsigned char* kna = tb + L.knorm_off;
+      const unsigned kna = tb + L.knorm_off;
       float sc[NRT][4];
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) sc[rt][j] = 0.f;
-      for (int gi = 0; gi < ng; ++gi) {
+      // key groups in a fixed rate order (rate known at compile time); a rate the layout
+      // does not use has no group
+      auto group = [&](auto rc) {
+        constexpr int R = decltype(rc)::value;
+        const int gi = s_gi[R];
+        if (gi < 0) return;
         float acc[NRT][4];
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[rt][j] = 0.f;
-        const int q0 = s_group[gi][0], q1 = s_group[gi][1];
-        switch (s_group[gi][2]) {
-          case 1: key_group<1, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
-          case 2: key_group<2, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
-          case 3: key_group<3, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
-          default: key_group<4, NP, VR, NRT>(acc, tb, s_loff, qf, q0, q1, lane, T, up); break;
-        }
+        key_group<R, NP, NRT>(acc, tb, unsigned(s_gkb[R]), s_lof[R][lane], s_olast[R][lane], s_gnq[R],
+                              qf4a + s_gslot[R] * 512 + 16 * lane, up, t8a, t3a, c8);
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt) {
           const int ni = gi * kTile + 16 * (rb0 + rt) + g;
           const float n0 = tile_norm<NH>(kna, ni), n1 = tile_norm<NH>(kna, ni + 8);
-          sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
-          sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
-          sc[rt][2] = fmaf(acc[rt][2], n1, sc[rt][2]);
-          sc[rt][3] = fmaf(acc[rt][3], n1, sc[rt][3]);
+          if constexpr (R == 1) {
+            // 0/1 operands of value 2^(m - 24) (rows g, g+8 = positions 2rt, 2rt + 1):
+            // sum_i B_i c_i = 2^(25 - m) acc - (column sum of B)
+            const float s0 = n0 * __int_as_float((127 + 25 - 2 * rt) << 23);
+            const float s1 = n1 * __int_as_float((127 + 24 - 2 * rt) << 23);
+            sc[rt][0] = fmaf(acc[rt][0], s0, fmaf(-sb0, n0, sc[rt][0]));
+            sc[rt][1] = fmaf(acc[rt][1], s0, fmaf(-sb1, n0, sc[rt][1]));
+            sc[rt][2] = fmaf(acc[rt][2], s1, fmaf(-sb0, n1, sc[rt][2]));
+            sc[rt][3] = fmaf(acc[rt][3], s1, fmaf(-sb1, n1, sc[rt][3]));
+          } else {
+            sc[rt][0] = fmaf(acc[rt][0], n0, sc[rt][0]);
+            sc[rt][1] = fmaf(acc[rt][1], n0, sc[rt][1]);
+            sc[rt][2] = fmaf(acc[rt][2], n1, sc[rt][2]);
+            sc[rt][3] = fmaf(acc[rt][3], n1, sc[rt][3]);
+          }
         }
-      }
+      };
+      group(IntC<4>{});
+      group(IntC<3>{});
+      group(IntC<2>{});
+      group(IntC<1>{});
       if constexpr (NP) {
         // columns 4..7 carried the lo parts of q': add them to the hi parts (lanes t, t^2)
 #pragma unroll
@@ -775,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
           O[mt][3] *= corr1;
         }
       }
-      const unsigned char* vna = tb + L.vnorm_off;
+      const unsigned vna = tb + L.vnorm_off;
 
       // ---------------- values: row block rb0 + rt is value chunk rb0 + rt of the tile.
       // First the probabilities (times |v| / sqrt(128)) as transposed fp16 B fragments,
@@ -797,33 +805,37 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         ValueLane<VR> vl;
         vl.load(tb + L.vcode_off + (rb0 + rt) * 256 * VR, lane);
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-          mma16816(O[mt], vl.field(4 * mt, T.v, lane4), vl.field(4 * mt + 1, T.v, lane4),
-                   vl.field(4 * mt + 2, T.v, lane4), vl.field(4 * mt + 3, T.v, lane4), pb[rt][0], pb[rt][1]);
+        for (int mt = 0; mt < 8; ++mt) {
+          unsigned av[4];
+          vl.regs(mt, t8a, vluta, c8, lane4, av);
+          mma16816(O[mt], av[0], av[1], av[2], av[3], pb[rt][0], pb[rt][1]);
+        }
       }
       }  // not scores-only
     };
 
     for (int k = 0; k < mine; ++k) {
-      const int st = warp + kWarps * (k & 1), i = item_tile(k);
-      const bool ok = mbar_wait_bounded(&full[st], (phase >> (k & 1)) & 1u);
-      if (ok) {
-        phase ^= 1u << (k & 1);
-        pend &= ~(1u << (k & 1));
-      }
+      const int st = warp + W * (k & 1), i = item_tile(k);
+      // warp-uniform decision: every lane waits, the warp goes on only if all saw the copy
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[st], (phase >> (k & 1)) & 1u));
       if (!ok) {
-        // stop consuming; this warp waits for its own copies below, no partial is written
+        // stop consuming; this warp's partial is dropped (m = -inf, l = 0) and it waits for
+        // its own copies below
         if (lane == 0) {
           atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
           s_timeout = 1;
         }
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
         break;
       }
-      const unsigned char* tb = ring + st * TB;
+      phase ^= 1u << (k & 1);
+      pend &= ~(1u << (k & 1));
+      const unsigned tb = launder(ringa + unsigned(st * TB));  // after the wait: the tile is in
       const long long gt0 = (long long)(S.lt0 + i) * kTile + g;  // token of row g in row block 0
       // a paged tile without a page (flagged by the copy) is left out
       if (tile_present(a.cache, S.u / a.h_kv, S.lt0 + i)) {
-        if (k == nfw && rem != 3) {
+        if (k == nfw && halves) {
           const int rb0 = 2 * (warp & 1);
           rows(IntC<2>{}, tb, rb0, gt0 + 16 * rb0);
         } else {
@@ -836,13 +848,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
         pend |= 1u << (k & 1);
       }
     }
-
-    if (si + 1 == nseg) pdl_trigger();
+    // after a timeout: the ring is reused below, so wait (bounded) for this warp's copies
+    // still in flight; only a second timeout here can leave one landing in shared memory
+    if (pend && lane == 0)
+      for (int h = 0; h < 2; ++h)
+        if (pend & (1u << h)) mbar_wait_bounded(&full[warp + W * h], (phase >> h) & 1u);
+    __syncwarp();
+    if (pend) phase ^= pend;  // the stages with a copy awaited above completed a phase
+    if (u == u_last) pdl_trigger();
     // ---------------- merge the warps (their partials reuse the ring: every warp is done
     // with the segment's tiles and has no copy in flight)
     __syncthreads();
-    if (*static_cast<volatile int*>(&s_timeout)) break;  // uniform over the CTA
-    if constexpr (SC) continue;  // the q' fragments are reloaded for the next segment
+    if constexpr (SC) {
+      __syncthreads();  // the q' fragments are reloaded for the next segment
+      continue;
+    }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -857,87 +877,46 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) split_kernel(DevLayout L
       mow[(2 * t + 1) * kD + 16 * g + 2 * mt + 1] = O[mt][3];
     }
     if (g == 0) {
-      mm[warp * 8 + 2 * t] = m0;
-      mm[warp * 8 + 2 * t + 1] = m1;
-      ml[warp * 8 + 2 * t] = l0;
-      ml[warp * 8 + 2 * t + 1] = l1;
+      s_mm[warp][2 * t] = m0;
+      s_mm[warp][2 * t + 1] = m1;
+      s_ml[warp][2 * t] = l0;
+      s_ml[warp][2 * t + 1] = l1;
     }
     __syncthreads();
     const int G = a.G;
-    for (int hh = 0; hh < G; ++hh) {
-      float M = -INFINITY;
+    for (int it = tid; it < G * kD; it += 32 * W) {
+      const int hh = it >> 7, d = it & (kD - 1);
+      float Mx = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * 8 + hh]);
+      for (int w = 0; w < W; ++w) Mx = fmaxf(Mx, s_mm[w][hh]);
       float o = 0.f, l = 0.f;
-      if (M != -INFINITY) {
+      if (Mx != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float f = fast_exp2(mm[w * 8 + hh] - M);
-          o = fmaf(f, mo[(w * 8 + hh) * kD + tid], o);
-          l = fmaf(f, ml[w * 8 + hh], l);
+        for (int w = 0; w < W; ++w) {
+          const float f = fast_exp2(s_mm[w][hh] - Mx);
+          o = fmaf(f, mo[(w * 8 + hh) * kD + d], o);
+          l = fmaf(f, s_ml[w][hh], l);
         }
       }
       const size_t idx = ((size_t)S.u * a.n_parts + S.part) * G + hh;
-      a.part_o[idx * kD + tid] = o;
-      if (tid == 0) {
-        a.part_ml[idx * 2] = M;
+      a.part_o[idx * kD + d] = o;
+      if (d == 0) {
+        a.part_ml[idx * 2] = Mx;
         a.part_ml[idx * 2 + 1] = l;
       }
     }
     __syncthreads();  // the merge area is the next segment's ring
+    if (s_timeout) break;  // uniform over the CTA: a copy engine that stalled once is not waited on again
   }
-  // after a timeout: do not leave while this warp's copies into shared memory are in flight
-  if (lane == 0)
-    for (int h = 0; h < 2; ++h)
-      if (pend & (1u << h)) mbar_wait_bounded(&full[warp + kWarps * h], (phase >> h) & 1u);
 }
 #pragma nv_diag_default 128
-
-size_t split_smem_bytes(int tile_bytes, int n_kquads) {
-  return 128 + size_t(kRing) * tile_bytes + size_t(n_kquads) * 64 * sizeof(unsigned) + 2 * kWarps * 8 * sizeof(float);
-}
-
-// Once per device and variant, before the occupancy query and the first launch: the
-// largest dynamic shared memory any layout needs, and the whole unified L1/shared array as
-// shared memory (the occupancy the plan assumes is then the one the launch gets).
-template <int VR, bool NP, bool SC, bool NH>
-cudaError_t configure_split() {
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev >= 64 || configured[dev]) return e;
-  e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(split_smem_bytes(kMaxTileBytes, kMaxQuads)));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             int(cudaSharedmemCarveoutMaxShared));
-  if (e == cudaSuccess) configured[dev] = true;
-  return e;
-}
-
-template <int VR, bool NP, bool SC, bool NH>
-cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, cudaStream_t stream) {
-  const size_t smem = split_smem_bytes(L.tile_bytes, L.n_kquads);
-  cudaError_t e = configure_split<VR, NP, SC, NH>();
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_ctas);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC, NH>, L, a);
-}
 
 // ------------------------------------------------------------------ combine
 constexpr int kCombThreads = 512;
 
 // One CTA per (batch row, query column): log-sum-exp merge of the unit's partials, then
-// o = R_V^T o'. Four threads per output dimension. R_V (not written by the split kernel)
+// o = R_V^T o' (or, with rec, the merged record (m, l, o') of the column: the partial of a
+// call over one token range, merged later with other ranges' records). Four threads per output dimension. R_V (not written by the split kernel)
 // is read into registers before waiting for the split kernel to finish. h_q counts query
 // columns (query heads x n_q); column hh of KV head h is query head h G / n_q + hh / n_q
 // at query token hh % n_q, written to out[b][token][head].
@@ -945,7 +924,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
                                                               const float* __restrict__ part_o, int S,
                                                               int max_tiles, long long total_tiles, int n_ctas, int G, int h_q,
                                                               int h_kv, int n_q, const float* __restrict__ v_rot,
-                                                              float* __restrict__ out) {
+                                                              float* __restrict__ out, float* __restrict__ rec) {
   pdl_trigger();  // the next call's first kernel may start its prologue now
   const int bq = blockIdx.x, b = bq / h_q, hq = bq % h_q;
   const int u = b * h_kv + hq / G, hh = hq % G;
@@ -1016,6 +995,16 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   }
   __syncthreads();
   if (tid < kD) op[tid] = l > 0.f ? ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) / l : 0.f;
+  const int heads = h_q / n_q, head = (hq / G) * (G / n_q) + hh / n_q, tok = hh % n_q;
+  if (rec) {  // uniform over the grid
+    float* r = rec + (((size_t)b * n_q + tok) * heads + head) * (kD + 2);
+    if (tid == 0) {
+      r[0] = Mx;
+      r[1] = l;
+    }
+    if (tid < kD) r[2 + tid] = op[tid];
+    return;
+  }
   __syncthreads();
   float r0 = 0.f, r1 = 0.f;
 #pragma unroll
@@ -1025,19 +1014,237 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   }
   part[qtr][d] = r0 + r1;
   __syncthreads();
-  const int heads = h_q / n_q, head = (hq / G) * (G / n_q) + hh / n_q, tok = hh % n_q;
   if (tid < kD)
     out[(((size_t)b * n_q + tok) * heads + head) * kD + tid] = (part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid]);
 }
 
-template <int VR, bool NP, bool SC, bool NH>
-int split_occupancy(const DevLayout& L) {
-  int n = 0;
-  if (configure_split<VR, NP, SC, NH>() != cudaSuccess) return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, split_kernel<VR, NP, SC, NH>, kThreads,
-                                                    split_smem_bytes(L.tile_bytes, L.n_kquads)) != cudaSuccess)
-    return 1;
-  return n < 1 ? 1 : n;
+// Dynamic shared memory of one split CTA: the fixed part for the value rate plus the ring
+// (which the warps' merge and, through it, the combine's partials reuse).
+inline int split_smem_bytes(int v_rate, int tile_bytes, int warps) {
+  const int fixed = v_rate == 3 ? sm_ring<3>() : v_rate == 4 ? sm_ring<4>() : sm_ring<2>();
+  const size_t ring = size_t(2 * warps) * tile_bytes;
+  return fixed + int(std::max(ring, size_t(warps) * 8 * kD * 4));
+}
+
+// Once per device and variant: the largest dynamic shared memory the kernel may use (the
+// device's per-block opt-in limit minus the kernel's static shared memory), set as the
+// kernel's limit together with the whole unified L1/shared array as shared memory.
+template <int VR, bool NP, bool SC, bool NH, int W>
+cudaError_t configure_split(int* dyn_limit) {
+  static int limit[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!limit[dev]) {
+    int optin = 0;
+    cudaFuncAttributes fa{};
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, split_kernel<VR, NP, SC, NH, W>);
+    if (e != cudaSuccess) return e;
+    const int dyn = optin - int(fa.sharedSizeBytes);
+    e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+    limit[dev] = dyn;
+  }
+  *dyn_limit = limit[dev];
+  return cudaSuccess;
+}
+
+template <int VR, bool NP, bool SC, bool NH, int W>
+cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, int smem, cudaStream_t stream) {
+  int limit = 0;
+  cudaError_t e = configure_split<VR, NP, SC, NH, W>(&limit);
+  if (e != cudaSuccess) return e;
+  if (smem > limit) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_ctas);
+  cfg.blockDim = dim3(32 * W);
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC, NH, W>, L, a);
+}
+
+// q' B fragments of unit u (batch row b, KV head h) into frag[kMaxQuads][2][32] (global),
+// by one CTA of kPrepThreads: thread (p = tid % 128, half = tid / 128) computes
+// q'[hh][p] = f_g sum_j R_g[i][j] q[hh][off_g + j] for the heads hh = 4 half .. 4 half + 3
+// (16-byte rows of R_g from global memory, q staged in shared memory); with G <= 4 the
+// two halves take heads 0..3 over the two halves of the row instead (all of a thread's
+// row is then loaded before q arrives) and add up in shared memory. Then every fragment
+// word is written once. With G <= 4 the eight B columns are heads 0..3 (hi
+// parts) and heads 0..3 again (lo parts) in the first array; otherwise the first array
+// holds the hi parts of heads 0..7 and the second the lo parts. Missing pairs and heads
+// are zero.
+constexpr int kPrepThreads = 256;
+static_assert(kPrepThreads == enc::kEncodeThreads, "the step kernel runs both bodies");
+static_assert(kPrepThreads == 8 * 32, "q-prep sums one B column per warp");
+
+// Word j (0..63) of quad qi's B fragments from q' (qr [head][packed dim], fp32): lane =
+// j % 32 = 4 n + t holds column n, dims 2t and 2t+1 of the quad; j < 32: the hi parts
+// (with G <= 4: hi parts of heads 0..3 in columns 0-3, lo parts in columns 4-7), j >= 32:
+// the lo parts (zero with G <= 4). Missing pairs and heads are zero.
+__device__ __forceinline__ unsigned frag_word(const DevLayout& L, const float* qr, int G, int qi, int j) {
+  const int lane = j & 31, n = lane >> 2, t = lane & 3;
+  const bool lo_half = j >= 32;
+  const int d0 = L.quad_dim0[qi] + 2 * t;
+  const int hh = G <= 4 ? (n & 3) : n;
+  const bool lo = G <= 4 ? n >= 4 : lo_half;
+  float v0 = 0.f, v1 = 0.f;
+  if (t < L.quad_np[qi] && hh < G && !(G <= 4 && lo_half)) {
+    v0 = qr[hh * kD + d0];
+    v1 = qr[hh * kD + d0 + 1];
+  }
+  const float r0 = __half2float(__float2half_rn(v0)), r1 = __half2float(__float2half_rn(v1));
+  return lo ? pack_h2(v0 - r0, v1 - r1) : pack_h2(r0, r1);
+}
+
+__device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __restrict__ q, int q_dtype, int h_q,
+                                          int h_kv, int G, int n_q, float qscale, int u, unsigned* __restrict__ frag) {
+  __shared__ __align__(16) float qs[kMaxG * kQsLd];  // q per group at 16-byte aligned columns
+  __shared__ float qr[kMaxG * kD];                   // q' in packed order
+  const int tid = threadIdx.x, ng = L.n_kgroups;
+  const int b = u / h_kv, h = u % h_kv;
+  __shared__ float red[4 * kD];                      // the k-split halves' partial sums
+  // this thread's row of R_g (columns [4 c0, 4 c1)): the first 16 float4 are loaded
+  // before q arrives
+  const int p = tid & (kD - 1), half = tid >> 7;
+  const bool ksplit = G <= 4;
+  const int h0 = ksplit ? 0 : half * 4;
+  int g = 0, pad = 0;
+  while (g + 1 < ng && p >= L.group_off[g + 1]) pad += L.k_rot32_ld[g++];
+  const int d = L.group_dim[g], i = p - L.group_off[g], ld = L.k_rot32_ld[g];
+  // packed dims past n_packed (rate-0 blocks) have no row: no loads, q' = 0
+  const int n4 = p < L.n_packed ? ld / 4 : 0, c0 = ksplit ? half * ((n4 + 1) / 2) : 0, c1 = ksplit ? min(n4, c0 + (n4 + 1) / 2) : n4;
+  const float4* row = reinterpret_cast<const float4*>(L.k_rot32[g] + (size_t)i * ld) + c0;
+  constexpr int kPre = 16;
+  float4 r[kPre];
+#pragma unroll
+  for (int j4 = 0; j4 < kPre; ++j4) r[j4] = c0 + j4 < c1 ? __ldg(row + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int e = tid; e < kMaxG * kQsLd; e += kPrepThreads) qs[e] = 0.f;
+  // the packed-to-original coordinate map in shared memory (a parameter-bank read with a
+  // different index in every lane would serialise)
+  __shared__ short s_pc[kD];
+  if (tid < kD) s_pc[tid] = L.packed_coord[tid];
+  __syncthreads();
+  // in a decode step (launched as a programmatic dependent) the CTA got here, rows of R in
+  // flight, while the kernel before it ran; q is the caller's: wait for that kernel before
+  // reading it. Only then may the split kernel launch: it reads the cache, which that
+  // kernel may write. (q-prep alone is a plain launch: both are no-ops there.)
+  pdl_wait();
+  pdl_trigger();
+  for (int e = tid; e < G * kD; e += kPrepThreads) {
+    const int hh = e >> 7, pe = e & (kD - 1);
+    if (pe >= L.n_packed) continue;
+    int ge = 0, pade = 0;
+    while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
+    // column hh: query head h G / n_q + hh / n_q at query token hh % n_q of q [b][token][head]
+    const size_t qrow = ((size_t)b * n_q + hh % n_q) * h_q + (size_t)h * (G / n_q) + hh / n_q;
+    qs[hh * kQsLd + pade + pe - L.group_off[ge]] = load_q(q, q_dtype, qrow * kD + s_pc[pe]);
+  }
+  __syncthreads();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (h0 < G) {
+    const float* qg = qs + h0 * kQsLd + pad + 4 * c0;
+#pragma unroll
+    for (int j4 = 0; j4 < kPre; ++j4) {
+      if (c0 + j4 < c1) {  // q columns past the group's padded row are not read
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
+          acc[k] = fmaf(r[j4].x, x.x, fmaf(r[j4].y, x.y, fmaf(r[j4].z, x.z, fmaf(r[j4].w, x.w, acc[k]))));
+        }
+      }
+    }
+#pragma unroll 8
+    for (int j4 = kPre; c0 + j4 < c1; ++j4) {
+      const float4 rr = __ldg(row + j4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(qg + k * kQsLd + 4 * j4);
+        acc[k] = fmaf(rr.x, x.x, fmaf(rr.y, x.y, fmaf(rr.z, x.z, fmaf(rr.w, x.w, acc[k]))));
+      }
+    }
+  }
+  if (ksplit) {  // uniform over the CTA
+    if (half == 1)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) red[k * kD + p] = acc[k];
+    __syncthreads();
+    if (half == 0)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += red[k * kD + p];
+  }
+  if (h0 < G && (!ksplit || half == 0)) {
+    const float f = qscale * rsqrtf(float(d)) * L.inv_kappa_group[g];  // the key tables carry kappa
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qr[(h0 + k) * kD + p] = acc[k] * f;
+  }
+  __syncthreads();
+  for (int e = tid; e < L.n_kquads * 64; e += kPrepThreads) frag[e] = frag_word(L, qr, G, e >> 6, e & 63);
+  // Column sums of the rate-1 group's B fragments, as the products see them (the sum of
+  // both fp16 halves of every word of the column, hi and lo arrays): the split kernel
+  // turns the group's 0/1 operands into +-1 codes with them. Warp n sums column n in a
+  // fixed order (deterministic).
+  int g1 = -1;
+  for (int gi = 0; gi < ng; ++gi)
+    if (L.group_rate[gi] == 1) g1 = gi;
+  if (g1 >= 0) {
+    const int n = tid >> 5, ln = tid & 31;   // 8 warps, one per B column
+    const int q0 = L.group_quad0[g1], nw = L.group_nquads[g1] * 8;  // 8 words of column n per quad
+    float acc = 0.f;
+    for (int w = ln; w < nw; w += 32) {
+      const int qi = q0 + (w >> 3), k = w & 7, j = (k >> 2) * 32 + 4 * n + (k & 3);
+      const unsigned x = frag_word(L, qr, G, qi, j);
+      acc += __half2float(__ushort_as_half((unsigned short)(x & 0xffffu))) +
+             __half2float(__ushort_as_half((unsigned short)(x >> 16)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (ln == 0) reinterpret_cast<float*>(frag + kMaxQuads * 64)[n] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
+                                                             int h_q, int h_kv, int G, int n_q, float qscale,
+                                                             unsigned* __restrict__ qfrag) {
+  // launched after the kernel before it has completed: the split kernel may start now
+  pdl_trigger();
+  const int u = blockIdx.x;
+  prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+}
+
+// First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
+// token and KV head), the others prepare q' of one unit each.
+template <bool NC>
+__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
+                                                                 const void* __restrict__ v, int kv_dtype, int n_new,
+                                                                 int batch, const int* __restrict__ seq_lens_before,
+                                                                 CacheRef cache,
+                                                                 const void* __restrict__ q, int q_dtype, int h_q,
+                                                                 int h_kv, int G, int n_q, float qscale,
+                                                                 unsigned* __restrict__ qfrag, int n_enc) {
+  // every block triggers its dependent (the split kernel) after its own wait for the
+  // kernel before it (in the encode and q-prep bodies; padding blocks by exiting)
+  const int e = blockIdx.x;
+  if (e < n_enc) {
+    const int part = e % kEncodeParts;
+    int rest = e / kEncodeParts;
+    const int t = rest % n_new;
+    rest /= n_new;
+    const int b = rest % batch, h = rest / batch;
+    enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
+  } else if (e - n_enc < batch * h_kv) {  // (a cluster launch pads the grid)
+    const int u = e - n_enc;
+    prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+  }
 }
 
 // Launch as a programmatic dependent of the kernel before it on the stream: the CTAs may
@@ -1079,31 +1286,40 @@ auto split_variant(int v_rate, bool np, bool sc, bool nh, Fn&& fn) {
   }
 }
 
-// Split and combine kernels of one call, launched as programmatic dependents of the
-// kernel that wrote the q' fragments (and, after an append, the new tokens).
-// n_q query tokens per row: the split and combine kernels see h_q n_q query columns,
+// Dynamic shared memory a split CTA may use: the device's per-block opt-in limit less a
+// reserve for the kernel's static shared memory (a few KB: group table, merge scalars).
+constexpr int kStaticReserve = 6 * 1024;
+int split_smem_limit() {
+  int dev = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 0;
+  return optin - kStaticReserve;
+}
+
+// Warps per split CTA: 12 when their ring stages fit next to the tables, else 8.
+int split_warps(int v_rate, int tile_bytes, int limit) {
+  return split_smem_bytes(v_rate, tile_bytes, 12) <= limit ? 12 : 8;
+}
+
+// The split kernel of one call (and, unless scores only, the merge in its last CTA per
+// unit), launched as a programmatic dependent of the kernel that wrote the q' fragments
+// (and, after an append, the new tokens). n_q query tokens per row: h_q n_q query columns,
 // G = h_q n_q / h_kv per KV head.
-cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int batch, int h_q, int h_kv, int n_q,
+cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int batch, int h_q, int h_kv, int n_q,
                              const CacheRef& cache, const int* seq_lens, float* out, void* workspace,
                              int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
-                             long long scores_ld = 0) {
+                             long long scores_ld = 0, float* rec = nullptr) {
   const int hc = h_q * n_q, G = hc / h_kv;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
-  // the workspace was sized for the most CTAs per SM; shared memory may allow fewer
-  // (larger slices, fewer partials per unit)
   const bool sc = scores != nullptr, nh = L.norm_fp16 != 0;
   if (!sc && (L.v_rate < 1 || L.v_rate > 4)) return cudaErrorInvalidValue;
-  const int occ = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
-    return split_occupancy<decltype(V)::value, decltype(P)::value != 0, decltype(S)::value != 0,
-                           decltype(H)::value != 0>(L);
-  });
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const DecodePlan plan = plan_decode(batch, hc, h_kv, (long long)wplan.max_tiles * kTile, sms, occ);
-  if (plan.n_parts > wplan.n_parts || plan.workspace_bytes > wplan.workspace_bytes) return cudaErrorInvalidValue;
+  const int limit = split_smem_limit();
+  const int vr = sc ? 1 : L.v_rate;  // the scores-only variant builds no value table
+  const int W = split_warps(vr, L.tile_bytes, limit);
+  const int smem = split_smem_bytes(vr, L.tile_bytes, W);
+  if (smem > limit) return cudaErrorInvalidValue;
   const long long units = (long long)batch * h_kv;
   SplitArgs a;
   a.cache = cache;
@@ -1116,8 +1332,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   a.h_kv = h_kv;
   a.G = G;
   a.n_q = n_q;
-  // q' fragments first, then the partials in the launch plan's layout (never larger than
-  // the workspace plan's)
+  // q' fragments, the unit counters, then the partials
   char* ws = static_cast<char*>(workspace);
   a.qfrag = reinterpret_cast<const unsigned*>(ws);
   ws += qfrag_bytes(units);
@@ -1128,67 +1343,98 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& wplan, int ba
   a.len_add = len_add;
   a.wait_new = after_append ? 1 : 0;
   const unsigned n_ctas = unsigned(plan.n_ctas);
-  e = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
-    return launch_split<decltype(V)::value, decltype(P)::value != 0, decltype(S)::value != 0,
-                        decltype(H)::value != 0>(a, L, n_ctas, stream);
+  cudaError_t e = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
+    constexpr int VR = decltype(V)::value;
+    constexpr bool NPv = decltype(P)::value != 0, SCv = decltype(S)::value != 0, NHv = decltype(H)::value != 0;
+    return W == 12 ? launch_split<VR, NPv, SCv, NHv, 12>(a, L, n_ctas, smem, stream)
+                   : launch_split<VR, NPv, SCv, NHv, 8>(a, L, n_ctas, smem, stream);
   });
-  if (sc) return e;  // scores only: no merge
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(batch * hc));
-  cfg.blockDim = dim3(kCombThreads);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, (const float*)a.part_ml, (const float*)a.part_o, plan.n_parts,
-                            plan.max_tiles, a.total_tiles, plan.n_ctas, G, hc, h_kv, n_q, L.v_rot32, out);
+  if (sc || e != cudaSuccess) return e;  // scores only: no merge
+  return launch_dependent(combine_kernel, unsigned(batch * hc), kCombThreads, stream, (const float*)a.part_ml,
+                          (const float*)a.part_o, plan.n_parts, plan.max_tiles, a.total_tiles, plan.n_ctas, G, hc,
+                          h_kv, n_q, L.v_rot32, out, rec);
 }
 
 }  // namespace
 
-DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms, int ctas_per_sm) {
+DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms, int /*ctas_per_sm*/) {
   DecodePlan p{};
-  if (ctas_per_sm <= 0 || ctas_per_sm > kCtasPerSm) ctas_per_sm = kCtasPerSm;
   const int G = h_q / h_kv;
   p.max_tiles = int((max_seq_len + kTile - 1) / kTile);
   if (p.max_tiles < 1) p.max_tiles = 1;
   const long long units = (long long)batch * h_kv;
   const long long total = units * p.max_tiles;
-  // one wave of ctas_per_sm CTAs per SM with slices of equal length (+-1 tile), no longer
-  // than a unit; more units than CTA slots: one CTA per unit
-  const long long slots = (long long)ctas_per_sm * num_sms;
-  long long C = units >= slots ? units : std::min(slots, total);
-  // a unit meets at most ceil(C / units) + 1 slices; the combine merges up to kMaxParts
-  while ((C + units - 1) / units + 1 > kMaxParts) C -= units;
+  // one CTA per SM, slices of equal length (+-1 tile); a slice may span several units
+  long long C = std::min<long long>(num_sms, total);
+  // a unit meets at most ceil(C / units) + 1 slices; the merge takes up to kMaxParts
+  while (C > 1 && (C + units - 1) / units + 1 > kMaxParts) --C;
   p.n_ctas = int(C);
   p.tiles_per_cta = int((total + C - 1) / C);
   p.n_parts = int((C + units - 1) / units + 1);
-  p.workspace_bytes = qfrag_bytes(units) + align256(size_t(units) * p.n_parts * G * 2 * sizeof(float)) +
+  p.workspace_bytes = qfrag_bytes(units) +
+                      align256(size_t(units) * p.n_parts * G * 2 * sizeof(float)) +
                       size_t(units) * p.n_parts * G * kD * sizeof(float);
   return p;
 }
 
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
-                          float* out, void* workspace, cudaStream_t stream) {
+                          float* out, void* workspace, cudaStream_t stream, float* rec) {
   const int G = h_q * n_q / h_kv;
+  const long long units = (long long)batch * h_kv;
   // a plain launch: the split kernel, launched as soon as this kernel starts, reads the
   // cache, which the kernel before this one may write
-  qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
+  qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
       L, q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens, out, workspace, 0, false, stream);
+  return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens, out, workspace, 0, false, stream,
+                          nullptr, 0, rec);
+}
+
+namespace {
+// One CTA of 128 threads per (batch row, query column): log-sum-exp merge of n_rec partial
+// records (m, l, o') of the same column over disjoint token ranges, then o = R_V^T o'.
+__global__ void __launch_bounds__(kD) merge_records_kernel(const float* __restrict__ recs, int n_rec,
+                                                           long long rec_stride, const float* __restrict__ v_rot,
+                                                           float* __restrict__ out) {
+  const int col = blockIdx.x, d = threadIdx.x;
+  __shared__ float op[kD];
+  const float* r0 = recs + (size_t)col * (kD + 2);
+  float M = -INFINITY;
+  for (int r = 0; r < n_rec; ++r) M = fmaxf(M, r0[(size_t)r * rec_stride]);
+  float den = 0.f, o = 0.f;
+  if (M != -INFINITY)
+    for (int r = 0; r < n_rec; ++r) {
+      const float* x = r0 + (size_t)r * rec_stride;
+      const float w = x[0] == -INFINITY ? 0.f : exp2f(x[0] - M) * x[1];
+      den += w;
+      o = fmaf(w, x[2 + d], o);
+    }
+  op[d] = den > 0.f ? o / den : 0.f;
+  __syncthreads();
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < kD; i += 2) {
+    acc0 = fmaf(__ldg(v_rot + (size_t)i * kD + d), op[i], acc0);
+    acc1 = fmaf(__ldg(v_rot + (size_t)(i + 1) * kD + d), op[i + 1], acc1);
+  }
+  out[(size_t)col * kD + d] = acc0 + acc1;
+}
+}  // namespace
+
+cudaError_t launch_merge_records(const DevLayout& L, const float* recs, int n_rec, long long columns, float* out,
+                                 cudaStream_t stream) {
+  merge_records_kernel<<<unsigned(columns), kD, 0, stream>>>(recs, n_rec, columns * (kD + 2), L.v_rot32, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
                           int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale, float* scores,
                           long long scores_ld, void* workspace, cudaStream_t stream) {
   const int G = h_q / h_kv;
-  qprep_kernel<<<unsigned(batch * h_kv), kPrepThreads, 0, stream>>>(
+  const long long units = (long long)batch * h_kv;
+  qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
       L, q, q_dtype, h_q, h_kv, G, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1201,16 +1447,17 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
                                int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
                                float* out, void* workspace, cudaStream_t stream) {
   const int G = h_q * n_q / h_kv;
-  const long long n_enc = (long long)n_new * kEncodeParts * batch * h_kv;
+  const long long units = (long long)batch * h_kv;
+  const long long n_enc = (long long)n_new * kEncodeParts * units;
   cudaError_t e;
   if (!L.norm_correct) {
-    e = launch_dependent(step_prep_kernel<false>, unsigned(n_enc + batch * h_kv), kPrepThreads, stream, L, k_new,
+    e = launch_dependent(step_prep_kernel<false>, unsigned(n_enc + units), kPrepThreads, stream, L, k_new,
                          v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, G, n_q,
                          softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   } else {
     // norm correction: clusters of the four encode parts of a token; the q' blocks
     // follow, padded to a whole cluster (the padding blocks return at once)
-    const long long n_blocks = (n_enc + batch * h_kv + kEncodeParts - 1) / kEncodeParts * kEncodeParts;
+    const long long n_blocks = (n_enc + units + kEncodeParts - 1) / kEncodeParts * kEncodeParts;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(n_blocks));
     cfg.blockDim = dim3(kPrepThreads);

@@ -30,7 +30,12 @@ cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, i
 // the plan is made for h_q n_q query columns.
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
-                          float* out, void* workspace, cudaStream_t stream);
+                          float* out, void* workspace, cudaStream_t stream, float* rec = nullptr);
+
+// Merge of partial records over disjoint token ranges: recs [n_rec][columns][130]
+// (m, l, o' of each query column), out [columns][128] = R_V^T (log-sum-exp merge of o').
+cudaError_t launch_merge_records(const DevLayout& L, const float* recs, int n_rec, long long columns, float* out,
+                                 cudaStream_t stream);
 
 // Append n_new tokens at seq_lens_before[b] and attend over seq_lens_before[b] + n_new
 // tokens: the encode kernel, then the split kernel as its programmatic dependent (only the

@@ -60,3 +60,32 @@ def aggregate(local_keys: float, local_ms: float, dist=None) -> tuple[float, flo
     dist.all_reduce(k, op=dist.ReduceOp.SUM)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(k.item()), float(t.item())
+
+
+# ------------------------------------------------------------------ one sequence over GPUs
+def token_range(length: int, rank: int, world: int, tile: int = 64) -> tuple[int, int]:
+    """Tokens [t0, t1) of a sequence of `length` tokens that rank `rank` of `world` holds
+    when one long sequence is split over GPUs: whole 64-token tiles, as even as possible,
+    in rank order (the last rank holds the newest tokens)."""
+    if world < 1 or not 0 <= rank < world or length < 0:
+        raise ValueError("bad rank/world/length")
+    tiles = -(-length // tile)
+    a, b = _split(tiles, world, rank)
+    return min(length, a * tile), min(length, b * tile)
+
+
+def split_sequence_decode(partial_fn, merge_fn, dist=None):
+    """Decode attention of one query step over a sequence split across ranks: each rank
+    computes the partial records (m, l, o') of its own token range (partial_fn() -> tensor
+    [B, h_q, 130]), all ranks exchange them (one all-gather: the only data-path
+    collective), and each rank merges them in rank order (merge_fn(stacked [world, B, h_q,
+    130]) -> output). With dist None or a single rank, the local records are merged alone.
+    The records are a few hundred bytes per query head, whatever the context length."""
+    import torch
+    rec = partial_fn()
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return merge_fn(rec[None])
+    world = dist.get_world_size()
+    parts = [torch.empty_like(rec) for _ in range(world)]
+    dist.all_gather(parts, rec.contiguous())
+    return merge_fn(torch.stack(parts))

@@ -5,13 +5,16 @@ the paged encode must equal the contiguous encode's tile byte for byte, and atte
 over the paged cache must give the contiguous call's output bit for bit (same kernels,
 same launch plan).
 """
+import math
+
 import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from packed_cache_decode_b200 import binding as B
 
-from .parity_util import Case, build_inputs
+from .parity_util import ATTN_REL_L2, Case, build_inputs, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -66,6 +69,19 @@ def test_paged_equals_contiguous(shape, options):
     torch.cuda.synchronize()
     assert lay.status() == 0
     assert torch.equal(o1, o2)
+    # the paged output against the oracle, per query head: the oracle encodes and packs
+    # each row's own tokens and attends over them
+    olay = O.make_layout(rates, case.v_bits, case.seed, *options)
+    G = h_q // h_kv
+    out = o2.cpu().double().numpy()
+    for b in range(batch):
+        n = int(lens[b])
+        for h in range(h_kv):
+            enc = O.encode(olay, k[b, :n, h].double().numpy(), v[b, :n, h].double().numpy())
+            buf = O.pack(olay, enc, cap)
+            ref = O.decode_attention(olay, q[b, h * G:(h + 1) * G].double().numpy(), buf, n, 1 / math.sqrt(128))
+            for i in range(G):
+                assert rel_l2(out[b, h * G + i], ref[i]) <= ATTN_REL_L2, (b, h, i, rel_l2(out[b, h * G + i], ref[i]))
 
 
 def test_paged_steps_equal_contiguous_steps():

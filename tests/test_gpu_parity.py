@@ -131,7 +131,8 @@ def test_zero_vectors_code_to_middle_and_zero_norm():
     for h in range(2):
         olay, enc, want = oracle_slice(case, rates, k, v, 0, h)
         assert np.all(enc["k_norms"][5] == 0) and enc["v_norm"][9] == 0
-        compare_packed(olay, enc, want, slice_bytes(case, olay.tile_bytes, cache_cpu, 0, h), case.cap)
+        compare_packed(olay, enc, want, slice_bytes(case, olay.tile_bytes, cache_cpu, 0, h), case.cap,
+                       near_rare=False)
     out = gpu_decode(lay, case, q, cache)
     assert np.all(np.isfinite(out))
 

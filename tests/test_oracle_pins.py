@@ -760,3 +760,25 @@ def test_boundary_mask_covers_exactly_the_near_threshold_codes():
     assert not full["k_norms"].any() and not full["v_norm"].any()
     # set bits: exactly sum of the masked coordinates' rates
     assert int(np.unpackbits(mask).sum()) == sum(pr[j] for _, j in near_k) + 3 * len(near_v)
+
+
+# ------------------------------------------------------------------ split attention
+def test_merged_partials_equal_attention_over_the_union():
+    # The log-sum-exp merge of partial attentions over disjoint token ranges is the
+    # softmax attention over all tokens: random split points (empty parts included) and
+    # peaked logits (large scale), against attention() computed directly.
+    rng = np.random.default_rng(11)
+    n, G = 300, 4
+    k = rng.standard_normal((n, 128)) * 3
+    v = rng.standard_normal((n, 128))
+    q = rng.standard_normal((G, 128)) * 2
+    full = O.attention(q, k, v, 0.3)
+    for cuts in ([0, 300], [0, 0, 300], [0, 1, 299, 300], [0, 64, 64, 200, 300], [0, 150, 300, 300]):
+        parts = [O.partial_attention(q, k[a:b], v[a:b], 0.3) for a, b in zip(cuts[:-1], cuts[1:])]
+        np.testing.assert_allclose(O.merge_partials(parts), full, rtol=1e-12, atol=1e-12)
+    # a merge that dropped the l weights, or kept per-part maxima, would not match
+    m, l, o = O.partial_attention(q, k[:10], v[:10], 0.3)
+    assert np.all(l >= 1.0) and np.allclose(o, O.attention(q, k[:10], v[:10], 0.3))
+    empty = O.partial_attention(q, k[:0], v[:0], 0.3)
+    assert np.all(np.isneginf(empty[0])) and not empty[1].any() and not empty[2].any()
+    np.testing.assert_array_equal(O.merge_partials([empty, empty]), np.zeros((G, 128)))
