@@ -499,8 +499,10 @@ def merge_partials(parts) -> np.ndarray:
 # ----------------------------------------------------------------------------------------
 # Packed tile format (the byte layout both sides implement)
 #
-# Tile of 64 tokens = [K area][V area][K norms, group-major: [group][token]]
-# [V norms [token]], norms fp32 (fp16 in a layout with fp16 norms). Both code areas are "fragment-major": they are cut into per-lane
+# Tile of 64 tokens = [K area][V area][K norms [group][g][m]][V norms [g][m]], the norm of
+# token g + 8 m of the tile (g, m = 0..7) at entry 8 g + m of its row of 64 (so the eight
+# tokens a lane's tensor-core rows cover are consecutive), norms fp32 (fp16 in a layout
+# with fp16 norms). Both code areas are "fragment-major": they are cut into per-lane
 # bit strings, lane l = 4 g + t of a 32-lane warp, holding exactly the codes that lane
 # turns into its tensor-core operand registers, so a lane reads its codes with one or two
 # aligned loads and no two lanes share a word. Words are little-endian; bit b of a bit
@@ -649,12 +651,14 @@ def pack(layout: Layout, enc: dict, capacity: int) -> np.ndarray:
     nb, nt = layout.norm_bytes, norm_dtype(layout)
     kn = np.zeros((ntile * TILE_TOKENS, ng), dtype=nt)
     kn[:n] = stored_norms(layout, enc["k_norms"])
-    kn = kn.reshape(ntile, TILE_TOKENS, ng).transpose(0, 2, 1).reshape(ntile, -1)
+    # [tile, token, group] -> [tile, group, row g, slot m] (token g + 8 m)
+    kn = kn.reshape(ntile, 8, 8, ng).transpose(0, 3, 2, 1).reshape(ntile, -1)
     out[:, base:base + nb * TILE_TOKENS * ng] = kn.view(np.uint8).reshape(ntile, -1)
     base += nb * TILE_TOKENS * ng
     vn = np.zeros(ntile * TILE_TOKENS, dtype=nt)
     vn[:n] = stored_norms(layout, enc["v_norm"])
-    out[:, base:base + nb * TILE_TOKENS] = vn.reshape(ntile, TILE_TOKENS).view(np.uint8)
+    vn = vn.reshape(ntile, 8, 8).transpose(0, 2, 1).reshape(ntile, TILE_TOKENS)
+    out[:, base:base + nb * TILE_TOKENS] = vn.view(np.uint8)
     return out.reshape(-1)
 
 
@@ -703,10 +707,10 @@ def unpack(layout: Layout, buf: np.ndarray, n: int) -> dict:
             vc[:, c, hit, dims] = hi
     base += TILE_TOKENS * vb
     nb, nt = layout.norm_bytes, norm_dtype(layout)
-    kn = t[:, base:base + nb * TILE_TOKENS * ng].copy().view(nt).reshape(ntile, ng, TILE_TOKENS)
-    kn = kn.transpose(0, 2, 1).reshape(-1, ng)
+    kn = t[:, base:base + nb * TILE_TOKENS * ng].copy().view(nt).reshape(ntile, ng, 8, 8)  # [group][g][m]
+    kn = kn.transpose(0, 3, 2, 1).reshape(-1, ng)                                          # token g + 8 m
     base += nb * TILE_TOKENS * ng
-    vn = t[:, base:base + nb * TILE_TOKENS].copy().view(nt).reshape(-1)
+    vn = t[:, base:base + nb * TILE_TOKENS].copy().view(nt).reshape(ntile, 8, 8).transpose(0, 2, 1).reshape(-1)
     return {"k_codes": kc[:n, :layout.n_packed], "k_norms": kn[:n].astype(np.float64),
             "v_codes": vc.reshape(-1, HEAD_DIM)[:n], "v_norm": vn[:n].astype(np.float64)}
 

@@ -102,7 +102,8 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256 + 5 * 16 * sizeof(double);
+  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256 + 5 * 16 * sizeof(double) +
+                       kTablesBytes + 16;
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
   if ((e = cudaMalloc(&dblock, bytes)) != cudaSuccess) {
@@ -169,6 +170,38 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
     for (int r = 0; r < 5; ++r) D.kappa[r] = float(kap[r]);
     D.kappa_v = float(kap_v);
     for (int g = 0; g < ng; ++g) D.inv_kappa_group[g] = float(1.0 / kap[L->group_rate[g]]);
+  }
+  {
+    // the decode lookup tables, in the split kernel's shared-memory order (16 copies of
+    // every entry so that the lanes of a half-warp never share a bank)
+    off = (off + 15) / 16 * 16;
+    unsigned char* tb = host.data() + off;
+    bool has[5] = {false, false, false, false, false};
+    for (int g = 0; g < ng; ++g) has[L->group_rate[g]] = true;
+    const unsigned short* c2 = has[2] ? D.kc2 : D.vc;  // equal when both are used (same rate, same kappa)
+    auto put2 = [&](size_t at, unsigned x, unsigned y) {
+      std::memcpy(tb + at, &x, 4);
+      std::memcpy(tb + at + 4, &y, 4);
+    };
+    for (int e = 0; e < 256; ++e)
+      for (int cp = 0; cp < 16; ++cp) {
+        if (has[2] || L->v_rate == 2)
+          put2(size_t(e) * 256 + cp * 8, c2[e & 3] | (unsigned(c2[(e >> 2) & 3]) << 16),
+               c2[(e >> 4) & 3] | (unsigned(c2[e >> 6]) << 16));
+        put2(size_t(e) * 256 + 128 + cp * 8, D.kc4[0][e & 15] | (unsigned(D.kc4[0][e >> 4]) << 16),
+             D.kc4[1][e & 15] | (unsigned(D.kc4[1][e >> 4]) << 16));
+      }
+    for (int e = 0; e < 64; ++e)
+      for (int cp = 0; cp < 16; ++cp)
+        put2(size_t(kTbl8Bytes) + size_t(e) * 128 + cp * 8, D.kc3[0][e & 7] | (unsigned(D.kc3[0][e >> 3]) << 16),
+             D.kc3[1][e & 7] | (unsigned(D.kc3[1][e >> 3]) << 16));
+    unsigned* vt = reinterpret_cast<unsigned*>(tb + kTbl8Bytes + kTbl3Bytes);
+    if (L->v_rate == 3)  // lane-private: entry e of lane l at word 32 e + l
+      for (int i = 0; i < 64 * 32; ++i) vt[i] = D.vc[(i >> 5) & 7] | (unsigned(D.vc[(i >> 5) >> 3]) << 16);
+    else if (L->v_rate == 4)
+      for (int e = 0; e < 256; ++e) vt[e] = D.vc[e & 15] | (unsigned(D.vc[e >> 4]) << 16);
+    D.tables = dptr + off;
+    off += kTablesBytes;
   }
   {
     int qi = 0, koff = 0;

@@ -18,6 +18,17 @@ constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
 constexpr int kMaxQuads = 20;            // sum over groups of ceil(d_g / 8) <= 128/8 + 3
 constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32 outputs each
 
+// Decode lookup tables, built once per layout (host, at upload) in the order the split
+// kernel keeps them in shared memory: 256 rows of 256 bytes (bytes 0-127: 16 copies of the
+// rate-2 entry of a code byte, two slots' fp16 pairs; bytes 128-255: 16 copies of the rate-4
+// entry, the hi and lo fp16 pairs of one slot), then 64 rows of 128 bytes (16 copies of the
+// rate-3 hi and lo pairs of a 6-bit field), then the value table (rate 3: 64 entries x 32
+// lanes, rate 4: 256 shared entries; 4 bytes each).
+constexpr int kTbl8Bytes = 256 * 256;
+constexpr int kTbl3Bytes = 64 * 128;
+constexpr int kTblVBytes = 64 * 32 * 4;
+constexpr int kTablesBytes = kTbl8Bytes + kTbl3Bytes + kTblVBytes;
+
 // Everything a kernel needs about one layer's packing, passed by value.
 struct DevLayout {
   int n_kgroups;
@@ -62,6 +73,7 @@ struct DevLayout {
   unsigned short kc3[2][8];      // [hi, lo][code]
   unsigned short kc4[2][16];
   unsigned short vc[16];
+  const unsigned char* tables;   // the decode lookup tables (kTablesBytes, 16-byte aligned)
 };
 
 // Where the packed tiles of a call live. Contiguous: [batch][h_kv][n_tiles][tile].

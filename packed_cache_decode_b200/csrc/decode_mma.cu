@@ -78,6 +78,12 @@ __device__ __forceinline__ unsigned long long evict_first_policy() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+// L2 policy for small per-layer constants read by every CTA (the decode tables): kept.
+__device__ __forceinline__ unsigned long long evict_last_policy() {
+  unsigned long long pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar,
                                           unsigned long long policy) {
   asm volatile(
@@ -193,11 +199,6 @@ __device__ __forceinline__ unsigned ld_s32(unsigned a) {
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
-__device__ __forceinline__ float ld_sf32(unsigned a) {
-  float v;
-  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-  return v;
-}
 __device__ __forceinline__ uint2 ld_s64(unsigned a) {
   uint2 v;
   asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
@@ -217,8 +218,6 @@ __device__ __forceinline__ unsigned shr(unsigned x, int s) { return s >= 0 ? x >
 __device__ __forceinline__ unsigned row8(unsigned w, unsigned c8, int byte) {
   return prmt(w, c8, 0x5504u | (unsigned(byte) << 4));
 }
-constexpr int kTbl8Bytes = 256 * 256;   // rows: [0,128) rate-2 pair pairs, [128,256) rate-4 hi/lo pairs
-constexpr int kTbl3Bytes = 64 * 128;    // rate-3 hi/lo pairs, 6-bit index, 16 copies
 
 // Dynamic shared memory of a split CTA, at offsets fixed at compile time (so that every
 // table lookup is one shared load with an immediate offset): mbarriers, the byte table,
@@ -298,20 +297,29 @@ struct KCodes<4> {
 
 // Scores of one key group with compile-time rate R over its nq quads of a tile. Quads go in
 // pairs into m16n8k16 products (quad 2i: k columns 0-7, quad 2i+1: 8-15); a group's odd
-// last quad takes an m16n8k8 product. Row block rt of the work item: rows g and g+8 are
-// slots m = 2 rt and 2 rt + 1. The lane's codes of quad j of the group sit at kb + 64 R j
-// + lo_full (the last quad, which may hold fewer pairs: at off_last); a lane without a pair
-// of that quad reads any code, its q' rows are zero. qf4[j / 2] = the lane's (hi, hi, lo,
-// lo) B fragments of quad pair j / 2 (a single last quad: (hi, 0, lo, 0)).
+// last quad takes an m16n8k8 product. The lane's codes of quad j of the group sit at kb +
+// 64 R j + lo_full (the last quad, which may hold fewer pairs: at off_last); a lane without
+// a pair of that quad reads any code, its q' rows are zero. qf4 + 512 (j / 2) = the lane's
+// (hi, hi, lo, lo) B fragments of quad pair j / 2 (a single last quad: (hi, 0, lo, 0)).
+// Rates 1-2: row block rt of the work item: rows g and g+8 are slots m = 2 rt and 2 rt + 1;
+// acc[rt] holds them. Rates 3-4 (centroids as fp16 hi + lo parts): one product per slot m,
+// its hi parts in row g and its lo parts in row g+8 (one 64-bit table load gives the lane
+// both, in operand order); acc[m] then holds the slot's two halves, summed afterwards.
 // NRT = 4: the whole tile; NRT = 2: the half tile of row blocks 0-1 (up = false) or 2-3.
 template <int R, bool NP, int NRT>
-__device__ __forceinline__ void key_group(float (&acc)[NRT][4], unsigned tb, unsigned kb, unsigned lo_full,
-                                          unsigned off_last, int nq, unsigned qf4, bool up, unsigned t8, unsigned t3,
-                                          unsigned c8) {
+__device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4], unsigned tb, unsigned kb,
+                                          unsigned lo_full, unsigned off_last, int nq, unsigned qf4, bool up,
+                                          unsigned t8, unsigned t3, unsigned c8) {
   // a full quad block is 16 x 4 pairs x R bytes; rate-3 offsets hold both planes' offsets
   // (low and high halfword), so a step moves both
   constexpr unsigned kQuadBytes = R == 3 ? 64u * R * 0x10001u : 64u * R;
   unsigned off = kb * (R == 3 ? 0x10001u : 1u) + lo_full;
+  // (hi, lo) table entry of slot m of a quad's codes
+  auto entry = [&](const KCodes<R>& c, int m) -> uint2 {
+    if constexpr (R == 3) return ld_s64(t3 + c.row(m, c8));
+    else if constexpr (R == 4) return ld_s64(t8 + 128 + row8(m < 4 ? c.w.x : c.w.y, c8, m & 3));
+    else return make_uint2(0u, 0u);
+  };
   int j = 0;
 #pragma unroll 1
   for (; j + 1 < nq; j += 2, off += 2 * kQuadBytes) {
@@ -319,62 +327,62 @@ __device__ __forceinline__ void key_group(float (&acc)[NRT][4], unsigned tb, uns
     c0.load(tb, off, NRT < 4 && up);
     c1.load(tb, j + 2 == nq ? off_last : off + kQuadBytes, NRT < 4 && up);
     const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
+    if constexpr (R <= 2) {
 #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) {
-      const int m = 2 * rt;
-      unsigned a0, a1, a2, a3, l0 = 0, l1 = 0, l2 = 0, l3 = 0;
-      if constexpr (R == 1) {
-        a0 = c0.a(m);
-        a1 = c0.a(m + 1);
-        a2 = c1.a(m);
-        a3 = c1.a(m + 1);
-      } else if constexpr (R == 2) {
-        const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt)), e1 = ld_s64(t8 + row8(c1.w, c8, rt));
-        a0 = e0.x;
-        a1 = e0.y;
-        a2 = e1.x;
-        a3 = e1.y;
-      } else if constexpr (R == 3) {
-        const uint2 e0 = ld_s64(t3 + c0.row(m, c8)), e1 = ld_s64(t3 + c0.row(m + 1, c8));
-        const uint2 e2 = ld_s64(t3 + c1.row(m, c8)), e3 = ld_s64(t3 + c1.row(m + 1, c8));
-        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y, a2 = e2.x, l2 = e2.y, a3 = e3.x, l3 = e3.y;
-      } else {
-        const unsigned x0 = m < 4 ? c0.w.x : c0.w.y, x1 = m < 4 ? c1.w.x : c1.w.y;
-        const uint2 e0 = ld_s64(t8 + 128 + row8(x0, c8, m & 3)), e1 = ld_s64(t8 + 128 + row8(x0, c8, (m & 3) + 1));
-        const uint2 e2 = ld_s64(t8 + 128 + row8(x1, c8, m & 3)), e3 = ld_s64(t8 + 128 + row8(x1, c8, (m & 3) + 1));
-        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y, a2 = e2.x, l2 = e2.y, a3 = e3.x, l3 = e3.y;
+      for (int rt = 0; rt < NRT; ++rt) {
+        const int m = 2 * rt;
+        unsigned a0, a1, a2, a3;
+        if constexpr (R == 1) {
+          a0 = c0.a(m);
+          a1 = c0.a(m + 1);
+          a2 = c1.a(m);
+          a3 = c1.a(m + 1);
+        } else {
+          const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt)), e1 = ld_s64(t8 + row8(c1.w, c8, rt));
+          a0 = e0.x;
+          a1 = e0.y;
+          a2 = e1.x;
+          a3 = e1.y;
+        }
+        mma16816(acc[rt], a0, a1, a2, a3, f.x, f.y);
+        if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, f.z, f.w);
       }
-      mma16816(acc[rt], a0, a1, a2, a3, f.x, f.y);
-      if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, f.z, f.w);
-      if constexpr (R >= 3) mma16816(acc[rt], l0, l1, l2, l3, f.x, f.y);
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2 * NRT; ++m) {
+        const uint2 e0 = entry(c0, m), e1 = entry(c1, m);
+        mma16816(acc[m], e0.x, e0.y, e1.x, e1.y, f.x, f.y);
+        if constexpr (!NP) mma16816(acc[m], e0.x, e0.y, e1.x, e1.y, f.z, f.w);
+      }
     }
   }
   if (j < nq) {
     KCodes<R> c0;
     c0.load(tb, j + 1 == nq ? off_last : off, NRT < 4 && up);
     const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
+    if constexpr (R <= 2) {
 #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) {
-      const int m = 2 * rt;
-      unsigned a0, a1, l0 = 0, l1 = 0;
-      if constexpr (R == 1) {
-        a0 = c0.a(m);
-        a1 = c0.a(m + 1);
-      } else if constexpr (R == 2) {
-        const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt));
-        a0 = e0.x;
-        a1 = e0.y;
-      } else if constexpr (R == 3) {
-        const uint2 e0 = ld_s64(t3 + c0.row(m, c8)), e1 = ld_s64(t3 + c0.row(m + 1, c8));
-        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y;
-      } else {
-        const unsigned x0 = m < 4 ? c0.w.x : c0.w.y;
-        const uint2 e0 = ld_s64(t8 + 128 + row8(x0, c8, m & 3)), e1 = ld_s64(t8 + 128 + row8(x0, c8, (m & 3) + 1));
-        a0 = e0.x, l0 = e0.y, a1 = e1.x, l1 = e1.y;
+      for (int rt = 0; rt < NRT; ++rt) {
+        const int m = 2 * rt;
+        unsigned a0, a1;
+        if constexpr (R == 1) {
+          a0 = c0.a(m);
+          a1 = c0.a(m + 1);
+        } else {
+          const uint2 e0 = ld_s64(t8 + row8(c0.w, c8, rt));
+          a0 = e0.x;
+          a1 = e0.y;
+        }
+        mma1688(acc[rt], a0, a1, f.x);
+        if constexpr (!NP) mma1688(acc[rt], a0, a1, f.z);
       }
-      mma1688(acc[rt], a0, a1, f.x);
-      if constexpr (!NP) mma1688(acc[rt], a0, a1, f.z);
-      if constexpr (R >= 3) mma1688(acc[rt], l0, l1, f.x);
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2 * NRT; ++m) {
+        const uint2 e0 = entry(c0, m);
+        mma1688(acc[m], e0.x, e0.y, f.x);
+        if constexpr (!NP) mma1688(acc[m], e0.x, e0.y, f.z);
+      }
     }
   }
 }
@@ -473,11 +481,29 @@ __device__ __forceinline__ Segment make_segment(const DevLayout& L, const SplitA
   return s;
 }
 
-// Norm i of a tile's norm area, stored as fp16 (NH) or fp32.
-template <bool NH>
-__device__ __forceinline__ float tile_norm(unsigned area, int i) {
-  if constexpr (NH) return __half2float(__ushort_as_half((unsigned short)ld_s16(area + 2 * i)));
-  else return ld_sf32(area + 4 * i);
+// The norms of slots s0 .. s0 + 2 NRT - 1 of row g (tokens g + 8 s) from the row's 8
+// consecutive entries at `row` (entry 8 g + m holds token g + 8 m): 128-bit loads.
+template <bool NH, int NRT>
+__device__ __forceinline__ void row_norms(unsigned row, int s0, float (&n)[2 * NRT]) {
+  if constexpr (NH) {
+    const uint4 x = ld_s128(row);  // all 8 fp16 entries
+    const unsigned w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 2 * NRT; i += 2) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[(s0 + i) >> 1]));
+      n[i] = f.x;
+      n[i + 1] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2 * NRT; i += 4) {
+      const uint4 x = ld_s128(row + 4 * (s0 + i));
+      n[i] = __uint_as_float(x.x);
+      n[i + 1] = __uint_as_float(x.y);
+      n[i + 2] = __uint_as_float(x.z);
+      n[i + 3] = __uint_as_float(x.w);
+    }
+  }
 }
 
 // SC: scores only. The tiles' logits (softmax_scale q . k_hat, natural units) go to
@@ -502,8 +528,6 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
 
   unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);  // [2 W]
   unsigned char* t8 = smem + kSmT8;
-  unsigned char* t3 = smem + kSmT3;
-  unsigned* vlut = reinterpret_cast<unsigned*>(smem + kSmVt);
   uint4* qf4 = reinterpret_cast<uint4*>(smem + sm_qf<VR>());         // [pair slot][lane]
   unsigned char* ring = smem + sm_ring<VR>();                           // stage s at ring + s TB
   float* mo = reinterpret_cast<float*>(ring);  // the warps' [8][128] partials reuse the ring
@@ -513,50 +537,15 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
     for (int i = 0; i < 2 * W; ++i) mbar_init(&full[i], 1);
     fence_mbar_init();
   }
-  // tables from the layout's fp16 codebooks: only those the layout uses. The codebooks
-  // (kernel parameters) are first staged in shared memory: read with a different index in
-  // every lane, the parameter bank would serialise.
-  __shared__ unsigned short s_cb[4 + 16 + 32 + 16];  // kc2, kc3 [hi, lo][8], kc4 [hi, lo][16], vc
-  if (tid < 4) s_cb[tid] = L.kc2[tid];
-  else if (tid < 20) s_cb[tid] = L.kc3[(tid - 4) >> 3][(tid - 4) & 7];
-  else if (tid < 52) s_cb[tid] = L.kc4[(tid - 20) >> 4][(tid - 20) & 15];
-  else if (tid < 68) s_cb[tid] = L.vc[tid - 52];
-  __syncthreads();
-  const unsigned short *c2 = s_cb, *c3h = s_cb + 4, *c3l = s_cb + 12, *c4h = s_cb + 20, *c4l = s_cb + 36, *cv = s_cb + 52;
-  unsigned has = 0;
-  for (int gi = 0; gi < L.n_kgroups; ++gi) has |= 1u << L.group_rate[gi];
-  if ((has & 4u) || VR == 2) {
-    // rate-2 pair pairs: row e = code byte (nibble = lo | hi << 2 of one slot), 16 copies
-    const unsigned short* cb = (has & 4u) ? c2 : cv;
-    for (int i = tid; i < 256 * 16; i += 32 * W) {
-      const int e = i >> 4, cp = i & 15;
-      const uint2 v = make_uint2(unsigned(cb[e & 3]) | (unsigned(cb[(e >> 2) & 3]) << 16),
-                                 unsigned(cb[(e >> 4) & 3]) | (unsigned(cb[e >> 6]) << 16));
-      *reinterpret_cast<uint2*>(t8 + e * 256 + cp * 8) = v;
-    }
-  }
-  if (has & 16u)
-    for (int i = tid; i < 256 * 16; i += 32 * W) {
-      const int e = i >> 4, cp = i & 15;
-      const uint2 v = make_uint2(unsigned(c4h[e & 15]) | (unsigned(c4h[e >> 4]) << 16),
-                                 unsigned(c4l[e & 15]) | (unsigned(c4l[e >> 4]) << 16));
-      *reinterpret_cast<uint2*>(t8 + e * 256 + 128 + cp * 8) = v;
-    }
-  if (has & 8u)
-    for (int i = tid; i < 64 * 16; i += 32 * W) {
-      const int e = i >> 4, cp = i & 15;
-      const uint2 v = make_uint2(unsigned(c3h[e & 7]) | (unsigned(c3h[e >> 3]) << 16),
-                                 unsigned(c3l[e & 7]) | (unsigned(c3l[e >> 3]) << 16));
-      *reinterpret_cast<uint2*>(t3 + e * 128 + cp * 8) = v;
-    }
-  if constexpr (VR == 3) {
-    // lane-private pair table: entry e of lane l at word 32 e + l (no bank conflicts)
-    for (int i = tid; i < 64 * 32; i += 32 * W) {
-      const int e = i >> 5;
-      vlut[i] = unsigned(cv[e & 7]) | (unsigned(cv[e >> 3]) << 16);
-    }
-  } else if constexpr (VR == 4) {
-    for (int e = tid; e < 256; e += 32 * W) vlut[e] = unsigned(cv[e & 15]) | (unsigned(cv[e >> 4]) << 16);
+  // the decode tables: one bulk copy of the layout's prebuilt tables (value table of this
+  // variant's value rate included), waited for below, after the other set-up
+  __shared__ __align__(8) unsigned long long s_tbar;
+  constexpr unsigned kTblCopy = unsigned(sm_qf<VR>() - kSmT8);
+  if (tid == 0) {
+    mbar_init(&s_tbar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(&s_tbar, kTblCopy);
+    bulk_load(t8, L.tables, kTblCopy, &s_tbar, evict_last_policy());
   }
   if (tid < 5) s_gi[tid] = -1;
   __syncthreads();
@@ -582,6 +571,9 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
     s_lof[r][ln] = full;
     s_olast[r][ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
   }
+  // every thread waits (bounded) for the tables; on a timeout the status says so and the
+  // decode goes on with whatever the tables hold (the call's output is then invalid)
+  if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_tbar, 0)) && lane == 0) atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
   __syncthreads();
 
   const float vscale = rsqrtf(float(kD)) / L.kappa_v;
@@ -684,17 +676,31 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
         constexpr int R = decltype(rc)::value;
         const int gi = s_gi[R];
         if (gi < 0) return;
-        float acc[NRT][4];
+        constexpr int NA = R >= 3 ? 2 * NRT : NRT;
+        float acc[NA][4];
 #pragma unroll
-        for (int rt = 0; rt < NRT; ++rt)
+        for (int i = 0; i < NA; ++i)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[rt][j] = 0.f;
+          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
         key_group<R, NP, NRT>(acc, tb, unsigned(s_gkb[R]), s_lof[R][lane], s_olast[R][lane], s_gnq[R],
                               qf4a + s_gslot[R] * 512 + 16 * lane, up, t8a, t3a, c8);
+        if constexpr (R >= 3) {
+          // slot 2rt + i: rows g (hi parts) + g+8 (lo parts) of acc[2rt + i] -> row g + 8i of rt
+#pragma unroll
+          for (int rt = 0; rt < NRT; ++rt) {
+            const float h00 = acc[2 * rt][0] + acc[2 * rt][2], h01 = acc[2 * rt][1] + acc[2 * rt][3];
+            const float h10 = acc[2 * rt + 1][0] + acc[2 * rt + 1][2], h11 = acc[2 * rt + 1][1] + acc[2 * rt + 1][3];
+            acc[rt][0] = h00;
+            acc[rt][1] = h01;
+            acc[rt][2] = h10;
+            acc[rt][3] = h11;
+          }
+        }
+        float nrm[2 * NRT];
+        row_norms<NH, NRT>(kna + (NH ? 2 : 4) * (gi * kTile + 8 * g), 2 * rb0, nrm);
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt) {
-          const int ni = gi * kTile + 16 * (rb0 + rt) + g;
-          const float n0 = tile_norm<NH>(kna, ni), n1 = tile_norm<NH>(kna, ni + 8);
+          const float n0 = nrm[2 * rt], n1 = nrm[2 * rt + 1];
           if constexpr (R == 1) {
             // 0/1 operands of value 2^(m - 24) (rows g, g+8 = positions 2rt, 2rt + 1):
             // sum_i B_i c_i = 2^(25 - m) acc - (column sum of B)
@@ -789,14 +795,15 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
       // First the probabilities (times |v| / sqrt(128)) as transposed fp16 B fragments,
       // then the m16n8k16 products against the value codes
       unsigned pb[NRT][2];
+      float vnr[2 * NRT];
+      row_norms<NH, NRT>(vna + (NH ? 2 : 4) * 8 * g, 2 * rb0, vnr);
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt) {
         const float p0 = fast_exp2(sc[rt][0] - b0m), p1 = fast_exp2(sc[rt][1] - b1m);
         const float p2 = fast_exp2(sc[rt][2] - b0m), p3 = fast_exp2(sc[rt][3] - b1m);
         l0 += p0 + p2;
         l1 += p1 + p3;
-        const float av0 = tile_norm<NH>(vna, 16 * (rb0 + rt) + g) * vscale;
-        const float av1 = tile_norm<NH>(vna, 16 * (rb0 + rt) + g + 8) * vscale;
+        const float av0 = vnr[2 * rt] * vscale, av1 = vnr[2 * rt + 1] * vscale;
         pb[rt][0] = movmatrix_trans(pack_h2(p0 * av0, p1 * av0));
         pb[rt][1] = movmatrix_trans(pack_h2(p2 * av1, p3 * av1));
       }

@@ -105,8 +105,12 @@ __device__ __forceinline__ void put_value_code(const DevLayout& L, uint8_t* tile
   }
 }
 
-// Stores norm s of entry i (token-major inside its group's row of 64) of a tile's norm
-// area: fp32, or fp16 rounded to nearest even and saturated at the largest finite fp16.
+// Entry of token tt (0..63 in its tile) in a row of 64 norms: token g + 8 m at 8 g + m, so
+// the eight tokens of a lane's tensor-core rows are consecutive.
+__device__ __forceinline__ int norm_entry(int tt) { return (tt & 7) * 8 + (tt >> 3); }
+
+// Stores norm s of entry i of a tile's norm area: fp32, or fp16 rounded to nearest even
+// and saturated at the largest finite fp16.
 __device__ __forceinline__ void store_norm(const DevLayout& L, uint8_t* area, int i, double s) {
   if (L.norm_fp16) reinterpret_cast<__half*>(area)[i] = __double2half(fmin(s, 65504.0));
   else reinterpret_cast<float*>(area)[i] = float(s);
@@ -223,10 +227,10 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
     if (!tp) return;
     if (is_key) {
       put_key_code(L, tp, g, i, tt, unsigned(code));
-      if (part == 0 && p < L.n_kgroups) store_norm(L, tp + L.knorm_off, p * kTile + tt, gnorm[p]);
+      if (part == 0 && p < L.n_kgroups) store_norm(L, tp + L.knorm_off, p * kTile + norm_entry(tt), gnorm[p]);
     } else {
       put_value_code(L, tp, p, tt, unsigned(code));
-      if (p == 0) store_norm(L, tp + L.vnorm_off, tt, gnorm[kMaxGroups]);
+      if (p == 0) store_norm(L, tp + L.vnorm_off, norm_entry(tt), gnorm[kMaxGroups]);
     }
     return;
   }
@@ -270,8 +274,8 @@ __device__ __forceinline__ void encode_token_part(const DevLayout& L, const void
     const double c2 = ((part_sq[0][tid] + part_sq[1][tid]) + (part_sq[2][tid] + part_sq[3][tid]));
     const double dd = tid == kMaxGroups ? double(kD) : double(L.group_dim[tid]);
     const double s = c2 > 0.0 ? gnorm[tid] * sqrt(dd) / sqrt(c2) : 0.0;
-    if (tid == kMaxGroups) store_norm(L, vna, tt, s);
-    else store_norm(L, kna, tid * kTile + tt, s);
+    if (tid == kMaxGroups) store_norm(L, vna, norm_entry(tt), s);
+    else store_norm(L, kna, tid * kTile + norm_entry(tt), s);
   }
 }
 

@@ -240,8 +240,9 @@ def test_pack_places_bits_where_the_format_says():
     assert (buf[vbase + 768] >> 3) & 7 == 4
     nbase = vbase + 64 * 48
     kn = buf[nbase:nbase + 4 * 128].view(np.float32)
-    assert kn[1] == 1.5 and kn[64 + 1] == -2.0
-    assert buf[nbase + 512:nbase + 768].view(np.float32)[2] == 0.25
+    # norms: token t = g + 8 m at entry 8 g + m: token 1 -> entry 8, token 2 -> entry 16
+    assert kn[8] == 1.5 and kn[64 + 8] == -2.0
+    assert buf[nbase + 512:nbase + 768].view(np.float32)[16] == 0.25
     # nothing else written: one byte per code, and 1.5 / -2.0 / 0.25 have 2 / 1 / 2 nonzero bytes
     assert int(np.count_nonzero(buf)) == 8 + 2 + 1 + 2
     u = O.unpack(lay, buf, n)
@@ -497,7 +498,8 @@ def test_norm_correction_factor_matches_the_centroid_energy(bits):
 
 def test_fp16_norms_are_where_the_format_says():
     """One rate-2 group and V2: K area 64 x 32 bytes, V area 64 x 32, then the K norms fp16
-    [1 group][64 tokens] at 4096 and the V norms fp16 [64] at 4224; 68 bytes per token.
+    [1 group][64 entries] at 4096 and the V norms fp16 [64] at 4224; 68 bytes per token.
+    Token t = g + 8 m sits at entry 8 g + m: tokens 0, 1, 2, 3 at entries 0, 8, 16, 24.
     fp16 of 3.0 is 0x4200, of 1.5 0x3e00; 1e6 saturates at 65504 (0x7bff); 0.1 rounds to
     nearest (0x2e66)."""
     lay = O.make_layout(np.full(64, 2), 2, 0, norm_fp16=True)
@@ -507,8 +509,9 @@ def test_fp16_norms_are_where_the_format_says():
            "k_norms": np.array([[3.0], [1e6], [0.1], [0.0]]), "v_norm": np.array([0.0, 1.5, 0.0, 65519.0])}
     buf = O.pack(lay, enc, 64)
     assert buf.size == 64 * 68
-    assert buf[4096:4104].tolist() == [0x00, 0x42, 0xff, 0x7b, 0x66, 0x2e, 0, 0]
-    assert buf[4224:4232].tolist() == [0, 0, 0x00, 0x3e, 0, 0, 0xff, 0x7b]
+    assert buf[4096:4098].tolist() == [0x00, 0x42] and buf[4112:4114].tolist() == [0xff, 0x7b]
+    assert buf[4128:4130].tolist() == [0x66, 0x2e] and buf[4144:4146].tolist() == [0, 0]
+    assert buf[4240:4242].tolist() == [0x00, 0x3e] and buf[4272:4274].tolist() == [0xff, 0x7b]
     assert int(np.count_nonzero(buf)) == (1 + 2 + 2) + (1 + 2)   # nonzero bytes of the norms; codes are 0
     u = O.unpack(lay, buf, n)
     assert u["k_norms"][:, 0].tolist() == [3.0, 65504.0, float(np.float16(0.1)), 0.0]
