@@ -246,9 +246,9 @@ class Model:
         x = _rope_dev(x, torch.tensor([pos], device=self.dev), self.wl.theta)
         return x[:, 0].contiguous().to(self.wl.dtype)
 
-    # kernel launches of one layer in a step: step-prep (encode + q-prep) + split (the
-    # log-sum-exp merge runs in the last split CTA of each unit)
-    LAUNCHES_PER_LAYER = 2
+    # kernel launches of one layer in a step: step-prep (encode + q-prep), the split kernel
+    # and the log-sum-exp combine
+    LAUNCHES_PER_LAYER = 3
 
     def step(self, stream):
         """Every layer: append the step's token and attend (one bgtq_decode_step call)."""
@@ -576,7 +576,7 @@ def main():
             "gbs": total_bytes / (step_ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": _profiled_traffic(args.workload),
-                         "kernel": "decode attention call per layer (q-prep -> split with fused merge, PDL-chained)",
+                         "kernel": "decode attention call per layer (q-prep -> split -> combine, PDL-chained)",
                          "bytes_per_launch": dec_bytes, "peak_kind": peak_kind},
             "l2_warm": {"us_per_call": l2_ms * 1e3, "GBs": dec_bytes / (l2_ms * 1e-3) / 1e9,
                         "note": f"layer 0's decode call repeated over the same {layer_mb:.0f} MB cache"

@@ -83,7 +83,7 @@ enum { BGTQ_F32 = 0, BGTQ_BF16 = 1, BGTQ_F16 = 2 };
 #define BGTQ_HEAD_DIM 128
 #define BGTQ_N_BLOCKS 64
 #define BGTQ_TILE_TOKENS 64
-#define BGTQ_MAX_GQA 8
+#define BGTQ_MAX_GQA 32  /* query columns per KV head: (h_q / h_kv) x query tokens */
 #define BGTQ_MAX_KGROUPS 4
 
 /* Device status bits reported by bgtq_device_status. */
@@ -207,7 +207,8 @@ size_t bgtq_workspace_bytes(const bgtq_layout* layout, int batch, int h_q, int h
  * row (0 gives a zero output row), max_seq_len >= every seq_len (plans the split-K grid;
  * larger lengths are clamped and flagged), softmax_scale (e.g. 1/sqrt(128)).
  * out [batch, h_q, 128] fp32 device. workspace: device buffer of at least
- * bgtq_workspace_bytes(...). h_q/h_kv must be 1..8. */
+ * bgtq_workspace_bytes(...). h_q/h_kv must be 1..32; a KV head's query heads are taken 8 at
+ * a time (each group of 8 reads the head's cache once). */
 bgtq_status bgtq_decode_attention(const bgtq_layout* layout, const void* q, int q_dtype,
                                   int batch, int h_q, int h_kv, const void* cache,
                                   const int* seq_lens_dev, long long capacity, long long max_seq_len,
@@ -298,8 +299,8 @@ bgtq_status bgtq_decode_step_paged(const bgtq_layout* layout, const void* k_new,
  * (q_dtype), out [batch, n_q, h_q, 128] fp32 device; query j of row b sits at position
  * seq_len_b - n_q + j and attends to tokens 0 .. seq_len_b - n_q + j (a row with
  * seq_len_b < n_q gives zeros for the queries that see no token). The query columns of
- * a KV head share one tensor-core tile: (h_q / h_kv) * n_q must be <= 8
- * (BGTQ_ERR_INVALID otherwise). Workspace: bgtq_workspace_bytes(layout, batch,
+ * a KV head share a tensor-core tile, 8 at a time: (h_q / h_kv) * n_q must be <= 32
+ * (BGTQ_ERR_INVALID otherwise; each tile of 8 columns reads the head's cache once). Workspace: bgtq_workspace_bytes(layout, batch,
  * h_q * n_q, h_kv, max_seq_len). n_q = 1 is bgtq_decode_attention. Other arguments,
  * ownership and errors as bgtq_decode_attention. */
 bgtq_status bgtq_decode_attention_multi(const bgtq_layout* layout, const void* q, int q_dtype, int batch,
@@ -311,7 +312,7 @@ bgtq_status bgtq_decode_attention_multi(const bgtq_layout* layout, const void* q
  * tokens per row at seq_lens_dev[b] (k_new, v_new [batch, n_new, h_kv, 128]) and attend
  * with their own queries q [batch, n_new, h_q, 128], causal among them, in one kernel
  * chain; out [batch, n_new, h_q, 128] fp32. seq_lens_dev holds the lengths BEFORE the
- * call and is not modified. (h_q / h_kv) * n_new <= 8; workspace as
+ * call and is not modified. (h_q / h_kv) * n_new <= 32; workspace as
  * bgtq_decode_attention_multi with n_q = n_new. Errors as bgtq_decode_step. */
 bgtq_status bgtq_decode_step_multi(const bgtq_layout* layout, const void* k_new, const void* v_new,
                                    int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,

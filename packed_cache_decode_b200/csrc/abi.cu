@@ -102,7 +102,7 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
   const int ng = L->n_kgroups;
   size_t n64 = 0;
   for (int g = 0; g <= ng; ++g) n64 += L->rot[g].size();
-  const size_t bytes = 256 + n64 * sizeof(double) + (n64 + 3 * kD) * sizeof(float) + 256 + 5 * 16 * sizeof(double) +
+  const size_t bytes = 256 + n64 * sizeof(double) + (2 * n64 + 3 * kD) * sizeof(float) + 256 + 5 * 16 * sizeof(double) +
                        kTablesBytes + 16;
   std::vector<unsigned char> host(bytes, 0);
   void* dblock = nullptr;
@@ -140,6 +140,18 @@ bgtq_status bgtq_layout_upload(bgtq_layout* L, int device) {
       D.v_rot32 = p;
     }
     off += size_t(d) * ld * sizeof(float);
+  }
+  off = (off + 15) / 16 * 16;  // 16-byte aligned: the bulk encoder fetches them with bulk copies
+  for (int g = 0; g <= ng; ++g) {
+    // fp32 copies transposed like the fp64 ones (element (i, j) at j * d + i); d is even, so
+    // every copy is a multiple of 16 bytes and the next one stays aligned
+    const int d = int(std::lround(std::sqrt(double(L->rot[g].size()))));
+    float* h32 = reinterpret_cast<float*>(host.data() + off);
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) h32[size_t(j) * d + i] = float(L->rot[g][size_t(i) * d + j]);
+    const float* p = reinterpret_cast<const float*>(dptr + off);
+    if (g < ng) D.k_rot32t[g] = p; else D.v_rot32t = p;
+    off += size_t(d) * d * sizeof(float);
   }
   {
     // fp64 centroids (the norm correction sums the squares of a token's centroids)
@@ -275,11 +287,12 @@ bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype,
                              DecodePlan* plan) {
   const std::string w(who);
   if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, w + ": bad dtype");
-  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
-    return fail(BGTQ_ERR_INVALID, w + ": need h_q = G * h_kv with G in 1..8");
-  if (n_q < 1 || (h_q / h_kv) * n_q > kMaxG)
-    return fail(BGTQ_ERR_INVALID, w + ": need (h_q / h_kv) * n_q in 1..8");
-  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, w + ": batch * h_kv > 65535");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxCols)
+    return fail(BGTQ_ERR_INVALID, w + ": need h_q = G * h_kv with G in 1..32");
+  if (n_q < 1 || (h_q / h_kv) * n_q > kMaxCols)
+    return fail(BGTQ_ERR_INVALID, w + ": need (h_q / h_kv) * n_q in 1..32");
+  const int ct = ((h_q / h_kv) * n_q + kMaxG - 1) / kMaxG;
+  if ((long long)batch * h_kv * ct > 65535) return fail(BGTQ_ERR_INVALID, w + ": too many units (batch * h_kv * column tiles > 65535)");
   if (max_seq_len < 0 || max_seq_len > row_tokens)
     return fail(BGTQ_ERR_CAPACITY, w + ": max_seq_len must be in [0, capacity]");
   if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, w + ": bad softmax_scale");
@@ -361,7 +374,7 @@ bgtq_status bgtq_encode_append(const bgtq_layout* L, const void* k, const void* 
 }
 
 size_t bgtq_workspace_bytes(const bgtq_layout* L, int batch, int h_q, int h_kv, long long max_seq_len) {
-  if (!L || batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG || max_seq_len < 0) {
+  if (!L || batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxCols || max_seq_len < 0) {
     set_error("workspace_bytes: bad arguments");
     return 0;
   }
@@ -516,9 +529,10 @@ bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype,
   bgtq_status st = check_device(L, "decode_scores");
   if (st != BGTQ_OK) return st;
   if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_scores: bad dtype");
-  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxG)
-    return fail(BGTQ_ERR_INVALID, "decode_scores: need h_q = G * h_kv with G in 1..8");
-  if ((long long)batch * h_kv > 65535) return fail(BGTQ_ERR_INVALID, "decode_scores: batch * h_kv > 65535");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxCols)
+    return fail(BGTQ_ERR_INVALID, "decode_scores: need h_q = G * h_kv with G in 1..32");
+  if ((long long)batch * h_kv * ((h_q / h_kv + kMaxG - 1) / kMaxG) > 65535)
+    return fail(BGTQ_ERR_INVALID, "decode_scores: too many units (batch * h_kv * column tiles > 65535)");
   if (capacity <= 0 || capacity % kTile)
     return fail(BGTQ_ERR_CAPACITY, "decode_scores: capacity must be a positive multiple of 64");
   if (max_seq_len < 0 || max_seq_len > capacity)

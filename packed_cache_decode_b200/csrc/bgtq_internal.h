@@ -13,10 +13,12 @@ constexpr int kD = BGTQ_HEAD_DIM;        // 128
 constexpr int kBlocks = BGTQ_N_BLOCKS;   // 64
 constexpr int kTile = BGTQ_TILE_TOKENS;  // 64 tokens per tile
 constexpr int kChunk = 16;               // tokens per V-code chunk
-constexpr int kMaxG = BGTQ_MAX_GQA;
+constexpr int kMaxG = 8;                 // query columns of one unit's tensor-core tile
+constexpr int kMaxCols = BGTQ_MAX_GQA;   // query columns per KV head: column tiles of 8
 constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
 constexpr int kMaxQuads = 20;            // sum over groups of ceil(d_g / 8) <= 128/8 + 3
 constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32 outputs each
+constexpr int kBulkMinTokens = 8;        // appends of this many tokens per row or more: one CTA per tile
 
 // Decode lookup tables, built once per layout (host, at upload) in the order the split
 // kernel keeps them in shared memory: 256 rows of 256 bytes (bytes 0-127: 16 copies of the
@@ -51,6 +53,8 @@ struct DevLayout {
   const double* k_rot64[kMaxGroups];  // d_g x d_g, TRANSPOSED: element (i, j) of R at j * d + i
   const double* v_rot64;              // 128 x 128, transposed likewise
   const float* k_rot32[kMaxGroups];  // row-major, rows padded to k_rot32_ld[g] floats (a multiple of 4)
+  const float* k_rot32t[kMaxGroups]; // d_g x d_g fp32, transposed like k_rot64 (the bulk encoder)
+  const float* v_rot32t;             // 128 x 128 fp32, transposed
   int k_rot32_ld[kMaxGroups];
   const float* v_rot32;
   const double* centroid64;      // [rate][code] at rate * 16 + code, fp64 (norm correction)

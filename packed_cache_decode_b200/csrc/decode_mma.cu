@@ -52,6 +52,7 @@
 
 #include "bgtq_internal.h"
 #include "encode_body.cuh"
+#include "async_copy.cuh"
 #include "kernels.h"
 
 namespace bgtq {
@@ -59,55 +60,6 @@ namespace bgtq {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr unsigned kWaitLimit = 1u << 22;
-
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ unsigned smem_addr(const void* p) { return unsigned(__cvta_generic_to_shared(p)); }
-
-__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-// L2 policy for data read once per step (the packed tiles): evicted first, so that the
-// small per-layer constants (rotations) stay in L2 from one step to the next.
-__device__ __forceinline__ unsigned long long evict_first_policy() {
-  unsigned long long pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-// L2 policy for small per-layer constants read by every CTA (the decode tables): kept.
-__device__ __forceinline__ unsigned long long evict_last_policy() {
-  unsigned long long pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar,
-                                          unsigned long long policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, unsigned parity) {
-  for (unsigned i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void mma16816(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
                                          unsigned b0, unsigned b1) {
@@ -149,8 +101,10 @@ struct SplitArgs {
   int n_ctas;             // CTAs; CTA c takes tiles [c T / n_ctas, (c+1) T / n_ctas) of the sequence
   int n_parts;            // partial slots per unit
   long long total_tiles;  // units x M
-  int h_q, h_kv, G;       // G: query columns per KV head (query heads per KV head x n_q)
-  int n_q;                // query tokens per row; column n is query token n % n_q
+  int h_q, h_kv, Gt;      // Gt: query columns per KV head (query heads per KV head x n_q)
+  int G;                  // columns of a unit's tile: Gt when CT = 1, else 8 (the last tile may hold fewer)
+  int n_q;                // query tokens per row; column n of KV head h is query token n % n_q
+  int CT;                 // column tiles per (batch row, KV head): unit u = cache unit u / CT, tile u % CT
   float* part_ml;         // [units][n_parts][G][2]
   float* part_o;          // [units][n_parts][G][128]
   float* scores;          // scores-only mode: [batch][h_q][scores_ld] logits (softmax_scale q.k_hat)
@@ -461,7 +415,7 @@ struct Segment {
 __device__ __forceinline__ Segment make_segment(const DevLayout& L, const SplitArgs& a, int c, int u, bool flag) {
   const long long M = a.max_tiles, T = a.total_tiles, C = a.n_ctas;
   const long long g0 = (long long)c * T / C, g1 = (long long)(c + 1) * T / C;
-  const int b = u / a.h_kv;
+  const int b = u / a.CT / a.h_kv;
   long long len = (long long)a.seq_lens[b] + a.len_add;
   if (len < 0) len = 0;
   const long long cap_tokens = min(a.cache.n_tiles, M) * kTile;
@@ -593,7 +547,8 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
 
   for (int u = u_first; u <= u_last; ++u) {
     const Segment S = make_segment(L, a, c, u, tid == 0);
-    const int srow = S.u / a.h_kv, shead = S.u % a.h_kv;
+    const int srow = S.u / a.CT / a.h_kv, shead = S.u / a.CT % a.h_kv;
+    const int col0 = S.u % a.CT * kMaxG;  // first column of this unit's tile in its KV head
     const long long first_new = waited ? 0 : a.seq_lens[srow];
     // Work items of this warp: full tiles w, w+W, ... of the first W floor(n/W); the
     // rem = n % W tiles left go one to each of the first rem warps, or, when 2 rem <= W,
@@ -735,7 +690,8 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
       // some column cannot see need the masks (n_q = 1: the end of the row).
       if (gt0 - g + 16 * NRT > S.len - (a.n_q - 1)) {
         const int c0 = NP ? 2 * (t & 1) : 2 * t;  // this lane's columns c0, c0 + 1
-        const long long vis0 = S.len - (a.n_q - 1 - c0 % a.n_q), vis1 = S.len - (a.n_q - 1 - (c0 + 1) % a.n_q);
+        const long long vis0 = S.len - (a.n_q - 1 - (col0 + c0) % a.n_q);
+        const long long vis1 = S.len - (a.n_q - 1 - (col0 + c0 + 1) % a.n_q);
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt) {
           const long long r0 = gt0 + 16 * rt, r1 = r0 + 8;
@@ -747,16 +703,16 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
       }
 
       if constexpr (SC) {
-        // column 2t + c holds head 2t + c (G <= 4: lanes t < 2; t >= 2 hold copies)
-        const int b = S.u / a.h_kv, hkv = S.u % a.h_kv;
+        // column 2t + c holds head col0 + 2t + c of the KV head (G <= 4: lanes t < 2; t >= 2 hold copies)
+        const int b = srow, hkv = shead;
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int head = 2 * t + (j & 1);
+            const int head = col0 + 2 * t + (j & 1);
             const long long tok = gt0 + 16 * rt + 8 * (j >> 1);
-            if ((!NP || t < 2) && head < a.G && tok < S.len)
-              a.scores[((size_t)b * a.h_q + (size_t)hkv * a.G + head) * a.scores_ld + tok] = sc[rt][j] * (1.f / kLog2e);
+            if ((!NP || t < 2) && head < a.Gt && tok < S.len)
+              a.scores[((size_t)b * a.h_q + (size_t)hkv * a.Gt + head) * a.scores_ld + tok] = sc[rt][j] * (1.f / kLog2e);
           }
       } else {
       // ---------------- online softmax over the rows (heads of columns 2t, 2t+1), base 2
@@ -841,7 +797,7 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
       const unsigned tb = launder(ringa + unsigned(st * TB));  // after the wait: the tile is in
       const long long gt0 = (long long)(S.lt0 + i) * kTile + g;  // token of row g in row block 0
       // a paged tile without a page (flagged by the copy) is left out
-      if (tile_present(a.cache, S.u / a.h_kv, S.lt0 + i)) {
+      if (tile_present(a.cache, srow, S.lt0 + i)) {
         if (k == nfw && halves) {
           const int rb0 = 2 * (warp & 1);
           rows(IntC<2>{}, tb, rb0, gt0 + 16 * rb0);
@@ -925,16 +881,19 @@ constexpr int kCombThreads = 512;
 // o = R_V^T o' (or, with rec, the merged record (m, l, o') of the column: the partial of a
 // call over one token range, merged later with other ranges' records). Four threads per output dimension. R_V (not written by the split kernel)
 // is read into registers before waiting for the split kernel to finish. h_q counts query
-// columns (query heads x n_q); column hh of KV head h is query head h G / n_q + hh / n_q
-// at query token hh % n_q, written to out[b][token][head].
+// columns (query heads x n_q); column gc of KV head h is query head h Gt / n_q + gc / n_q
+// at query token gc % n_q, written to out[b][token][head]. G: columns per unit tile.
 __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* __restrict__ part_ml,
                                                               const float* __restrict__ part_o, int S,
                                                               int max_tiles, long long total_tiles, int n_ctas, int G, int h_q,
                                                               int h_kv, int n_q, const float* __restrict__ v_rot,
                                                               float* __restrict__ out, float* __restrict__ rec) {
   pdl_trigger();  // the next call's first kernel may start its prologue now
+  // column hq of row b: KV head h = hq / Gt, column gc = hq % Gt of the head, in column tile
+  // gc / 8 (unit (b h_kv + h) CT + gc / 8) as its column gc % 8 (G columns per unit)
   const int bq = blockIdx.x, b = bq / h_q, hq = bq % h_q;
-  const int u = b * h_kv + hq / G, hh = hq % G;
+  const int Gt = h_q / h_kv, CT = (Gt + kMaxG - 1) / kMaxG, gc = hq % Gt;
+  const int u = (b * h_kv + hq / Gt) * CT + gc / kMaxG, hh = gc % kMaxG;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int d = tid & (kD - 1), qtr = tid >> 7;
   __shared__ float w[kMaxParts];
@@ -1002,7 +961,7 @@ __global__ void __launch_bounds__(kCombThreads, 1) combine_kernel(const float* _
   }
   __syncthreads();
   if (tid < kD) op[tid] = l > 0.f ? ((part[0][tid] + part[1][tid]) + (part[2][tid] + part[3][tid])) / l : 0.f;
-  const int heads = h_q / n_q, head = (hq / G) * (G / n_q) + hh / n_q, tok = hh % n_q;
+  const int heads = h_q / n_q, head = (hq / Gt) * (Gt / n_q) + gc / n_q, tok = gc % n_q;
   if (rec) {  // uniform over the grid
     float* r = rec + (((size_t)b * n_q + tok) * heads + head) * (kD + 2);
     if (tid == 0) {
@@ -1113,12 +1072,17 @@ __device__ __forceinline__ unsigned frag_word(const DevLayout& L, const float* q
   return lo ? pack_h2(v0 - r0, v1 - r1) : pack_h2(r0, r1);
 }
 
+// Gt: query columns of a KV head (query heads per KV head x n_q); a unit holds at most 8 of
+// them (column tile ct = u % CT of cache unit u / CT, CT = ceil(Gt / 8)); G: the unit's
+// fragment columns (Gt when CT = 1, else 8; columns past Gt stay zero).
 __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __restrict__ q, int q_dtype, int h_q,
-                                          int h_kv, int G, int n_q, float qscale, int u, unsigned* __restrict__ frag) {
+                                          int h_kv, int Gt, int n_q, float qscale, int u, unsigned* __restrict__ frag) {
   __shared__ __align__(16) float qs[kMaxG * kQsLd];  // q per group at 16-byte aligned columns
   __shared__ float qr[kMaxG * kD];                   // q' in packed order
   const int tid = threadIdx.x, ng = L.n_kgroups;
-  const int b = u / h_kv, h = u % h_kv;
+  const int CT = (Gt + kMaxG - 1) / kMaxG, G = CT == 1 ? Gt : kMaxG;
+  const int cu = u / CT, ct = u % CT;
+  const int b = cu / h_kv, h = cu % h_kv;
   __shared__ float red[4 * kD];                      // the k-split halves' partial sums
   // this thread's row of R_g (columns [4 c0, 4 c1)): the first 16 float4 are loaded
   // before q arrives
@@ -1152,8 +1116,11 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
     if (pe >= L.n_packed) continue;
     int ge = 0, pade = 0;
     while (ge + 1 < ng && pe >= L.group_off[ge + 1]) pade += L.k_rot32_ld[ge++];
-    // column hh: query head h G / n_q + hh / n_q at query token hh % n_q of q [b][token][head]
-    const size_t qrow = ((size_t)b * n_q + hh % n_q) * h_q + (size_t)h * (G / n_q) + hh / n_q;
+    // column hh of the tile = column gc of the KV head: query head h Gt / n_q + gc / n_q at
+    // query token gc % n_q of q [b][token][head]
+    const int gc = ct * kMaxG + hh;
+    if (gc >= Gt) continue;
+    const size_t qrow = ((size_t)b * n_q + gc % n_q) * h_q + (size_t)h * (Gt / n_q) + gc / n_q;
     qs[hh * kQsLd + pade + pe - L.group_off[ge]] = load_q(q, q_dtype, qrow * kD + s_pc[pe]);
   }
   __syncthreads();
@@ -1220,12 +1187,12 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
 }
 
 __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
-                                                             int h_q, int h_kv, int G, int n_q, float qscale,
+                                                             int h_q, int h_kv, int Gt, int n_q, float qscale,
                                                              unsigned* __restrict__ qfrag) {
   // launched after the kernel before it has completed: the split kernel may start now
   pdl_trigger();
   const int u = blockIdx.x;
-  prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+  prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
 }
 
 // First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
@@ -1236,7 +1203,7 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
                                                                  int batch, const int* __restrict__ seq_lens_before,
                                                                  CacheRef cache,
                                                                  const void* __restrict__ q, int q_dtype, int h_q,
-                                                                 int h_kv, int G, int n_q, float qscale,
+                                                                 int h_kv, int Gt, int n_q, float qscale,
                                                                  unsigned* __restrict__ qfrag, int n_enc) {
   // every block triggers its dependent (the split kernel) after its own wait for the
   // kernel before it (in the encode and q-prep bodies; padding blocks by exiting)
@@ -1248,9 +1215,9 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
     rest /= n_new;
     const int b = rest % batch, h = rest / batch;
     enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
-  } else if (e - n_enc < batch * h_kv) {  // (a cluster launch pads the grid)
+  } else if (e - n_enc < batch * h_kv * ((Gt + kMaxG - 1) / kMaxG)) {  // (a cluster launch pads the grid)
     const int u = e - n_enc;
-    prep_unit(L, q, q_dtype, h_q, h_kv, G, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+    prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
   }
 }
 
@@ -1317,7 +1284,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
                              const CacheRef& cache, const int* seq_lens, float* out, void* workspace,
                              int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
                              long long scores_ld = 0, float* rec = nullptr) {
-  const int hc = h_q * n_q, G = hc / h_kv;
+  const int hc = h_q * n_q, Gt = hc / h_kv, CT = (Gt + kMaxG - 1) / kMaxG, G = CT == 1 ? Gt : kMaxG;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
   const bool sc = scores != nullptr, nh = L.norm_fp16 != 0;
@@ -1327,7 +1294,7 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
   const int W = split_warps(vr, L.tile_bytes, limit);
   const int smem = split_smem_bytes(vr, L.tile_bytes, W);
   if (smem > limit) return cudaErrorInvalidValue;
-  const long long units = (long long)batch * h_kv;
+  const long long units = (long long)batch * h_kv * CT;
   SplitArgs a;
   a.cache = cache;
   a.seq_lens = seq_lens;
@@ -1337,8 +1304,10 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
   a.total_tiles = units * plan.max_tiles;
   a.h_q = hc;
   a.h_kv = h_kv;
+  a.Gt = Gt;
   a.G = G;
   a.n_q = n_q;
+  a.CT = CT;
   // q' fragments, the unit counters, then the partials
   char* ws = static_cast<char*>(workspace);
   a.qfrag = reinterpret_cast<const unsigned*>(ws);
@@ -1366,10 +1335,11 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
 
 DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms, int /*ctas_per_sm*/) {
   DecodePlan p{};
-  const int G = h_q / h_kv;
+  // h_q counts query columns; more than 8 per KV head are split into column tiles
+  const int Gt = h_q / h_kv, CT = (Gt + kMaxG - 1) / kMaxG, G = CT == 1 ? Gt : kMaxG;
   p.max_tiles = int((max_seq_len + kTile - 1) / kTile);
   if (p.max_tiles < 1) p.max_tiles = 1;
-  const long long units = (long long)batch * h_kv;
+  const long long units = (long long)batch * h_kv * CT;
   const long long total = units * p.max_tiles;
   // one CTA per SM, slices of equal length (+-1 tile); a slice may span several units
   long long C = std::min<long long>(num_sms, total);
@@ -1387,12 +1357,12 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
                           float* out, void* workspace, cudaStream_t stream, float* rec) {
-  const int G = h_q * n_q / h_kv;
-  const long long units = (long long)batch * h_kv;
+  const int Gt = h_q * n_q / h_kv;
+  const long long units = (long long)batch * h_kv * ((Gt + kMaxG - 1) / kMaxG);
   // a plain launch: the split kernel, launched as soon as this kernel starts, reads the
   // cache, which the kernel before this one may write
   qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+      L, q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens, out, workspace, 0, false, stream,
@@ -1439,10 +1409,10 @@ cudaError_t launch_merge_records(const DevLayout& L, const float* recs, int n_re
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
                           int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale, float* scores,
                           long long scores_ld, void* workspace, cudaStream_t stream) {
-  const int G = h_q / h_kv;
-  const long long units = (long long)batch * h_kv;
+  const int Gt = h_q / h_kv;
+  const long long units = (long long)batch * h_kv * ((Gt + kMaxG - 1) / kMaxG);
   qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, G, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+      L, q, q_dtype, h_q, h_kv, Gt, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, 1, cache, seq_lens, nullptr, workspace, 0, false, stream,
@@ -1453,13 +1423,14 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
                                int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
                                float* out, void* workspace, cudaStream_t stream) {
-  const int G = h_q * n_q / h_kv;
-  const long long units = (long long)batch * h_kv;
-  const long long n_enc = (long long)n_new * kEncodeParts * units;
+  const int Gt = h_q * n_q / h_kv;
+  const long long cache_units = (long long)batch * h_kv;
+  const long long units = cache_units * ((Gt + kMaxG - 1) / kMaxG);  // q' units (column tiles)
+  const long long n_enc = (long long)n_new * kEncodeParts * cache_units;
   cudaError_t e;
   if (!L.norm_correct) {
     e = launch_dependent(step_prep_kernel<false>, unsigned(n_enc + units), kPrepThreads, stream, L, k_new,
-                         v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, G, n_q,
+                         v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, Gt, n_q,
                          softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   } else {
     // norm correction: clusters of the four encode parts of a token; the q' blocks
@@ -1477,7 +1448,7 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, step_prep_kernel<true>, L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache,
-                           q, q_dtype, h_q, h_kv, G, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
+                           q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
                            int(n_enc));
   }
   if (e != cudaSuccess) return e;

@@ -63,7 +63,7 @@ bgtq_status bgtq_decode_attention_noalloc(const bgtq_layout* L, const void* q, i
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess)
     return bgtq::fail(BGTQ_ERR_CUDA, std::string("decode_attention_noalloc: ") + cudaGetErrorString(e));
-  if (!L || batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > bgtq::kMaxG || max_seq_len < 0)
+  if (!L || batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > bgtq::kMaxCols || max_seq_len < 0)
     return bgtq::fail(BGTQ_ERR_INVALID, "decode_attention_noalloc: bad layout or shape");
   const bgtq::DecodePlan plan = bgtq::plan_decode(batch, h_q, h_kv, max_seq_len, sms);
   if (plan.workspace_bytes > kScratchBytes)

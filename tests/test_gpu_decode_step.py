@@ -141,7 +141,7 @@ def test_step_rejects_bad_arguments():
                                                                  wsb, None)
     assert call(7, 1, 1, 64, 64, ws.numel()) == B.ERR_INVALID       # bad dtype
     assert call(0, -1, 1, 64, 64, ws.numel()) == B.ERR_INVALID      # negative n_new
-    assert call(0, 1, 9, 64, 64, ws.numel()) == B.ERR_INVALID       # G = 9
+    assert call(0, 1, 33, 64, 64, ws.numel()) == B.ERR_INVALID      # G = 33 > 32 (rejected before any launch)
     assert call(0, 1, 1, 65, 64, ws.numel()) == B.ERR_CAPACITY      # capacity not a multiple of 64
     assert call(0, 1, 1, 64, 128, ws.numel()) == B.ERR_CAPACITY     # max_seq_len > capacity
     assert call(0, 1, 1, 64, 64, 0) == B.ERR_WORKSPACE

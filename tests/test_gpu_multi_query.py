@@ -1,8 +1,9 @@
 """Multi-token decode attention through the C ABI against the oracle: n_q query tokens per
 row, the last n_q of the row's cached tokens, causal among themselves (speculative
 verification, a prefill chunk). The G query heads x n_q tokens of a KV head are the
-columns of one tensor-core tile, so the cases cover both q' fragment forms (G n_q <= 4 and
-5..8 columns) and ragged rows.
+columns of tensor-core tiles of 8, so the cases cover both q' fragment forms (G n_q <= 4
+and 5..8 columns), several column tiles per KV head (up to 32 columns, a last tile with a
+single column) and ragged rows.
 """
 import ctypes as C
 import math
@@ -25,6 +26,10 @@ CASES = {   # (case, n_q)
     "gqa1_nq8": (Case(2, 2, 1, 260, 3, 3, torch.bfloat16, 1e6, 53), 8),
     "gqa1_nq3_f32_k1v4": (Case(2, 2, 3, 130, 1, 4, torch.float32, 5e5, 54), 3),
     "gqa8_nq1": (Case(16, 2, 1, 500, 3, 3, torch.bfloat16, 1e6, 55), 1),
+    "gqa8_nq2_16cols": (Case(16, 2, 2, 500, 2, 2, torch.bfloat16, 5e5, 58), 2),
+    "gqa8_nq4_32cols": (Case(16, 2, 1, 300, 3, 3, torch.bfloat16, 1e6, 59), 4),
+    "gqa3_nq3_9cols": (Case(6, 2, 2, 400, 2, 2, torch.float16, 5e5, 60), 3),
+    "gqa16_nq1": (Case(32, 2, 2, 260, 2, 3, torch.bfloat16, 5e5, 61), 1),
 }
 
 
@@ -83,12 +88,14 @@ def test_one_query_token_equals_decode_attention():
     assert torch.equal(o1, o2[:, 0])
 
 
+@pytest.mark.parametrize("h_q", [8, 16], ids=["8cols", "16cols"])
 @pytest.mark.parametrize("paged", [False, True], ids=["contiguous", "paged"])
-def test_step_multi_equals_append_then_attend(paged):
+def test_step_multi_equals_append_then_attend(paged, h_q):
     """decode_step_multi appends the n_new draft tokens and attends with their queries in one
     chain: same cache bytes and outputs as encode_append + decode_attention_multi, and the
-    oracle's multi-token attention over the grown rows."""
-    case = Case(8, 4, 3, 600, 2, 2, torch.bfloat16, 5e5, 57, capacity=640)
+    oracle's multi-token attention over the grown rows (h_q / h_kv x n_new = 8 or 16 query
+    columns per KV head: one or two column tiles)."""
+    case = Case(h_q, 4, 3, 600, 2, 2, torch.bfloat16, 5e5, 57, capacity=640)
     n_new = 4
     model, rates, _, k, v = build_inputs(case)
     lay = B.Layout(rates, case.v_bits, case.seed).upload(0)
@@ -164,9 +171,10 @@ def test_multi_query_rejects_bad_shapes():
     p = lambda t: C.c_void_p(t.data_ptr())
     call = lambda n_q, h_q: lib.bgtq_decode_attention_multi(lay.handle, p(q), 0, 1, n_q, h_q, 1, p(cache), p(lens), 64,
                                                             64, 0.1, p(out), p(ws), ws.numel(), None)
-    assert call(3, 4) == B.ERR_INVALID      # 4 heads x 3 tokens = 12 columns
+    assert call(9, 4) == B.ERR_INVALID      # 4 heads x 9 tokens = 36 columns > 32 (rejected before any launch)
     assert call(0, 1) == B.ERR_INVALID
     assert call(2, 4) == B.OK
+    assert call(3, 4) == B.OK               # 12 columns: two column tiles
     assert lib.bgtq_decode_step_multi(lay.handle, p(q), p(q), 0, 0, p(q), 0, 1, 1, 1, p(cache), p(lens), 64, 64, 0.1,
                                       p(out), p(ws), ws.numel(), None) == B.ERR_INVALID   # n_new = 0
     torch.cuda.synchronize()

@@ -178,10 +178,10 @@ def test_bad_arguments_are_rejected_before_launch():
     p = lambda t: C.c_void_p(t.data_ptr())
     assert lib.bgtq_encode_append(lay.handle, p(k), p(k), 9, 1, 1, 1, p(lens), p(cache), 64, None) == B.ERR_INVALID
     assert lib.bgtq_encode_append(lay.handle, p(k), p(k), 0, 1, 1, 1, p(lens), p(cache), 65, None) == B.ERR_CAPACITY
-    out = torch.zeros(1, 9, 128, device="cuda")
+    out = torch.zeros(1, 33, 128, device="cuda")
     ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    assert lib.bgtq_decode_attention(lay.handle, p(out), 0, 1, 9, 1, p(cache), p(lens), 64, 64, 0.1, p(out), p(ws),
-                                     ws.numel(), None) == B.ERR_INVALID      # G = 9 > 8
+    assert lib.bgtq_decode_attention(lay.handle, p(out), 0, 1, 33, 1, p(cache), p(lens), 64, 64, 0.1, p(out), p(ws),
+                                     ws.numel(), None) == B.ERR_INVALID      # G = 33 > 32
     assert lib.bgtq_decode_attention(lay.handle, p(out), 0, 1, 1, 1, p(cache), p(lens), 64, 128, 0.1, p(out), p(ws),
                                      ws.numel(), None) == B.ERR_CAPACITY     # max_seq_len > capacity
     assert lib.bgtq_decode_attention(lay.handle, p(out), 0, 1, 1, 1, p(cache), p(lens), 64, 64, 0.1, p(out), p(ws),

@@ -23,6 +23,7 @@ CASES = {
     "gqa8_bf16_k3": Case(16, 2, 1, 1000, 3, 3, torch.bfloat16, 1e6, 32),
     "gqa1_f32_k4": Case(2, 2, 1, 129, 4, 1, torch.float32, 5e5, 33),
     "k1_uniform": Case(8, 2, 1, 300, 1, 1, torch.bfloat16, 5e5, 34),
+    "gqa12_two_column_tiles": Case(24, 2, 2, 400, 2, 2, torch.bfloat16, 5e5, 35),
 }
 
 
