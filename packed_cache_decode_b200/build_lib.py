@@ -20,7 +20,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3,-Wall", "-I", os.path.join(ROOT, "include")]
 SOURCES = ["host_plan.cpp", "abi.cu", "encode.cu", "decode_mma.cu", "noalloc.cu"]
-HEADERS = ["bgtq_internal.h", "kernels.h", "encode_body.cuh"]
+HEADERS = ["bgtq_internal.h", "kernels.h", "encode_body.cuh", "async_copy.cuh"]
 
 
 def _newer(target: str, deps: list[str]) -> bool:

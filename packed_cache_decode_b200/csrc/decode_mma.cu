@@ -48,6 +48,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <type_traits>
 #include <utility>
 
 #include "bgtq_internal.h"
@@ -124,6 +125,27 @@ __device__ __forceinline__ void mma1688(float (&c)[4], unsigned a0, unsigned a1,
   asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
                : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
                : "r"(a0), "r"(a1), "r"(b0));
+}
+// The same products with Z: the accumulator starts at zero (C = 0, c not read).
+template <bool Z>
+__device__ __forceinline__ void mma16816s(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
+                                          unsigned b0, unsigned b1) {
+  if constexpr (Z)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+  else
+    mma16816(c, a0, a1, a2, a3, b0, b1);
+}
+template <bool Z>
+__device__ __forceinline__ void mma1688s(float (&c)[4], unsigned a0, unsigned a1, unsigned b0) {
+  if constexpr (Z)
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};\n"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a0), "r"(a1), "r"(b0), "f"(0.f));
+  else
+    mma1688(c, a0, a1, b0);
 }
 
 // +-1 pair from two 1-bit codes sitting at bits 15 and 31 of x (bit 1 -> +1, 0 -> -1):
@@ -274,13 +296,14 @@ __device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4
     else if constexpr (R == 4) return ld_s64(t8 + 128 + row8(m < 4 ? c.w.x : c.w.y, c8, m & 3));
     else return make_uint2(0u, 0u);
   };
-  int j = 0;
-#pragma unroll 1
-  for (; j + 1 < nq; j += 2, off += 2 * kQuadBytes) {
+  // quads 2i, 2i+1 (codes at o0, o1, B fragments of pair i); Z: the group's first
+  // products, which start the accumulators at zero
+  auto pair = [&](auto zc, unsigned o0, unsigned o1, int i) {
+    constexpr bool Z = decltype(zc)::value;
     KCodes<R> c0, c1;
-    c0.load(tb, off, NRT < 4 && up);
-    c1.load(tb, j + 2 == nq ? off_last : off + kQuadBytes, NRT < 4 && up);
-    const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
+    c0.load(tb, o0, NRT < 4 && up);
+    c1.load(tb, o1, NRT < 4 && up);
+    const uint4 f = ld_s128(qf4 + i * 512);
     if constexpr (R <= 2) {
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt) {
@@ -298,21 +321,23 @@ __device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4
           a2 = e1.x;
           a3 = e1.y;
         }
-        mma16816(acc[rt], a0, a1, a2, a3, f.x, f.y);
+        mma16816s<Z>(acc[rt], a0, a1, a2, a3, f.x, f.y);
         if constexpr (!NP) mma16816(acc[rt], a0, a1, a2, a3, f.z, f.w);
       }
     } else {
 #pragma unroll
       for (int m = 0; m < 2 * NRT; ++m) {
         const uint2 e0 = entry(c0, m), e1 = entry(c1, m);
-        mma16816(acc[m], e0.x, e0.y, e1.x, e1.y, f.x, f.y);
+        mma16816s<Z>(acc[m], e0.x, e0.y, e1.x, e1.y, f.x, f.y);
         if constexpr (!NP) mma16816(acc[m], e0.x, e0.y, e1.x, e1.y, f.z, f.w);
       }
     }
-  }
-  if (j < nq) {
+  };
+  // an odd last quad j (codes at o0): m16n8k8 products
+  auto single = [&](auto zc, unsigned o0, int j) {
+    constexpr bool Z = decltype(zc)::value;
     KCodes<R> c0;
-    c0.load(tb, j + 1 == nq ? off_last : off, NRT < 4 && up);
+    c0.load(tb, o0, NRT < 4 && up);
     const uint4 f = ld_s128(qf4 + (j >> 1) * 512);
     if constexpr (R <= 2) {
 #pragma unroll
@@ -327,18 +352,28 @@ __device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4
           a0 = e0.x;
           a1 = e0.y;
         }
-        mma1688(acc[rt], a0, a1, f.x);
+        mma1688s<Z>(acc[rt], a0, a1, f.x);
         if constexpr (!NP) mma1688(acc[rt], a0, a1, f.z);
       }
     } else {
 #pragma unroll
       for (int m = 0; m < 2 * NRT; ++m) {
         const uint2 e0 = entry(c0, m);
-        mma1688(acc[m], e0.x, e0.y, f.x);
+        mma1688s<Z>(acc[m], e0.x, e0.y, f.x);
         if constexpr (!NP) mma1688(acc[m], e0.x, e0.y, f.z);
       }
     }
+  };
+  if (nq == 1) {
+    single(std::true_type{}, off_last, 0);
+    return;
   }
+  pair(std::true_type{}, off, nq == 2 ? off_last : off + kQuadBytes, 0);
+  int j = 2;
+  off += 2 * kQuadBytes;
+#pragma unroll 1
+  for (; j + 1 < nq; j += 2, off += 2 * kQuadBytes) pair(std::false_type{}, off, j + 2 == nq ? off_last : off + kQuadBytes, j >> 1);
+  if (j < nq) single(std::false_type{}, off_last, j);
 }
 
 // Value A fragments of one 16-token chunk: the lane's 64 VR-bit string (one or two
@@ -632,11 +667,7 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
         const int gi = s_gi[R];
         if (gi < 0) return;
         constexpr int NA = R >= 3 ? 2 * NRT : NRT;
-        float acc[NA][4];
-#pragma unroll
-        for (int i = 0; i < NA; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        float acc[NA][4];  // started by the group's first products
         key_group<R, NP, NRT>(acc, tb, unsigned(s_gkb[R]), s_lof[R][lane], s_olast[R][lane], s_gnq[R],
                               qf4a + s_gslot[R] * 512 + 16 * lane, up, t8a, t3a, c8);
         if constexpr (R >= 3) {
