@@ -136,7 +136,8 @@ bgtq_status bgtq_block_energy(const float* q_cal, long long n_q, int h_q,
 /* The same energy score per KV head, for a rate allocation per KV head: score_out
  * [h_kv * 64], score_out[h * 64 + j] = the term of KV head h in bgtq_block_energy (whose
  * score is their sum). A per-head allocation gives each KV head its own layout; such
- * heads are cached and decoded with one call per KV head (h_kv = 1). */
+ * heads are cached and decoded together through a layout set (bgtq_layout_set_create,
+ * below), or with one call per KV head (h_kv = 1). */
 bgtq_status bgtq_block_energy_heads(const float* q_cal, long long n_q, int h_q,
                                     const float* k_cal, long long n_k, int h_kv, double* score_out);
 
@@ -328,6 +329,49 @@ bgtq_status bgtq_decode_step_multi_paged(const bgtq_layout* layout, const void* 
                                          const int* seq_lens_dev, long long max_seq_len,
                                          float softmax_scale, float* out, void* workspace,
                                          size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- one layout per KV head */
+
+/* [BGTQ s3-s5]: the rate allocation may be made per KV head (bgtq_block_energy_heads), each
+ * head then coded with its own layout (its own groups, rotations and codebook tables). A
+ * layout set holds the layouts of the h_kv heads of one attention layer, in head order,
+ * so that one call encodes or decodes every head. The layouts must be uploaded to the
+ * current device and share the value rate, the options (BGTQ_LAYOUT_*) and the seed (the
+ * value rotation); BGTQ_ERR_INVALID otherwise. The set refers to the layouts' device
+ * constants: destroy it before any of its layouts. */
+typedef struct bgtq_layout_set bgtq_layout_set;
+bgtq_status bgtq_layout_set_create(const bgtq_layout* const* layouts, int h_kv, bgtq_layout_set** out);
+void bgtq_layout_set_destroy(bgtq_layout_set* set);
+/* Bytes of one tile of every head in the set's cache: the largest tile of its layouts (a
+ * head with a smaller tile leaves the rest of each tile unused). 0 for a null set. */
+int bgtq_layout_set_tile_bytes(const bgtq_layout_set* set);
+/* Bytes of a contiguous cache [batch][h_kv][capacity/64][tile] of the set (0 on bad
+ * arguments: capacity must be a positive multiple of 64). */
+size_t bgtq_layout_set_cache_bytes(const bgtq_layout_set* set, int batch, long long capacity);
+/* bgtq_encode_append with KV head h coded by layout h of the set: k, v [batch, n_new,
+ * h_kv, 128], h_kv = the set's size, cache of bgtq_layout_set_cache_bytes. Arguments,
+ * ownership and errors otherwise as bgtq_encode_append; status bits go to the set
+ * (bgtq_layout_set_status). */
+bgtq_status bgtq_encode_append_heads(const bgtq_layout_set* set, const void* k, const void* v, int dtype,
+                                     int batch, int n_new, const int* seq_lens_dev, void* cache,
+                                     long long capacity, void* stream);
+/* bgtq_decode_attention over a cache written by bgtq_encode_append_heads: one call for
+ * every KV head (h_kv = the set's size; h_q a multiple of it). Workspace:
+ * bgtq_workspace_bytes(any layout of the set, batch, h_q, h_kv, max_seq_len). Arguments,
+ * ownership and errors otherwise as bgtq_decode_attention. */
+bgtq_status bgtq_decode_attention_heads(const bgtq_layout_set* set, const void* q, int q_dtype, int batch,
+                                        int h_q, const void* cache, const int* seq_lens_dev,
+                                        long long capacity, long long max_seq_len, float softmax_scale,
+                                        float* out, void* workspace, size_t workspace_bytes, void* stream);
+/* bgtq_decode_scores over a cache written by bgtq_encode_append_heads (h_kv = the set's
+ * size). */
+bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* set, const void* q, int q_dtype, int batch,
+                                     int h_q, const void* cache, const int* seq_lens_dev, long long capacity,
+                                     long long max_seq_len, float softmax_scale, float* scores,
+                                     long long scores_ld, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+/* The set's status bits (BGTQ_STATUS_*), as bgtq_device_status. */
+bgtq_status bgtq_layout_set_status(const bgtq_layout_set* set, unsigned* flags, int clear);
 
 /* ---------------------------------------------------------------- no-allocation variant */
 

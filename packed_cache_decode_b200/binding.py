@@ -33,6 +33,8 @@ EXPORTED = [
     "bgtq_paged_pool_bytes", "bgtq_encode_append_paged", "bgtq_decode_attention_paged", "bgtq_decode_step_paged",
     "bgtq_decode_attention_multi", "bgtq_decode_step_multi", "bgtq_decode_step_multi_paged",
     "bgtq_block_energy_heads", "bgtq_decode_attention_partial", "bgtq_merge_partials",
+    "bgtq_layout_set_create", "bgtq_layout_set_destroy", "bgtq_layout_set_tile_bytes", "bgtq_layout_set_cache_bytes",
+    "bgtq_encode_append_heads", "bgtq_decode_attention_heads", "bgtq_decode_scores_heads", "bgtq_layout_set_status",
 ]
 
 
@@ -91,6 +93,14 @@ def load():
         "bgtq_decode_step_multi": (I, [P, P, P, I, I, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
         "bgtq_decode_step_multi_paged": (I, [P, P, P, I, I, P, I, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t,
                                              P]),
+        "bgtq_layout_set_create": (I, [P, I, C.POINTER(P)]),
+        "bgtq_layout_set_destroy": (None, [P]),
+        "bgtq_layout_set_tile_bytes": (I, [P]),
+        "bgtq_layout_set_cache_bytes": (C.c_size_t, [P, I, LL]),
+        "bgtq_encode_append_heads": (I, [P, P, P, I, I, I, P, P, LL, P]),
+        "bgtq_decode_attention_heads": (I, [P, P, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_scores_heads": (I, [P, P, I, I, I, P, P, LL, LL, F, P, LL, P, C.c_size_t, P]),
+        "bgtq_layout_set_status": (I, [P, C.POINTER(C.c_uint), I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -220,6 +230,52 @@ class Layout:
     def close(self):
         if self._h:
             load().bgtq_layout_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class LayoutSet:
+    """The uploaded layouts of the KV heads of one layer, in head order (owns the C handle;
+    keeps the layouts alive)."""
+
+    def __init__(self, layouts):
+        self.layouts = list(layouts)
+        arr = (C.c_void_p * len(self.layouts))(*[lay.handle for lay in self.layouts])
+        h = C.c_void_p()
+        _check(load().bgtq_layout_set_create(arr, len(self.layouts), C.byref(h)), "layout_set_create")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def h_kv(self):
+        return len(self.layouts)
+
+    @property
+    def tile_bytes(self):
+        return int(load().bgtq_layout_set_tile_bytes(self._h))
+
+    def cache_bytes(self, batch: int, capacity: int) -> int:
+        n = load().bgtq_layout_set_cache_bytes(self._h, batch, capacity)
+        if n == 0:
+            _check(ERR_INVALID, "layout_set_cache_bytes")
+        return int(n)
+
+    def status(self, clear: bool = True) -> int:
+        f = C.c_uint(0)
+        _check(load().bgtq_layout_set_status(self._h, C.byref(f), int(clear)), "layout_set_status")
+        return int(f.value)
+
+    def close(self):
+        if self._h:
+            load().bgtq_layout_set_destroy(self._h)
             self._h = None
 
     def __del__(self):
@@ -480,3 +536,41 @@ def plan_head_rates(q_cal, k_cal, avg_bits: int, min_rate: int = 1, max_rate: in
     is the rate vector of that head's own layout)."""
     s = block_energy_heads(q_cal, k_cal)
     return np.stack([allocate_rates(s[h], min_rate, max_rate, 64 * avg_bits) for h in range(s.shape[0])])
+
+
+# ---------------------------------------------------------------- one layout per KV head
+def encode_append_heads(layouts: LayoutSet, k, v, seq_lens, cache, capacity: int, stream=None):
+    """k, v [B, n_new, h_kv, 128] CUDA (h_kv = the set's size); KV head h coded with layout h."""
+    B, n_new, h_kv, d = k.shape
+    assert d == HEAD_DIM and h_kv == layouts.h_kv and k.is_contiguous() and v.is_contiguous()
+    assert v.shape == k.shape and v.dtype == k.dtype
+    _check(load().bgtq_encode_append_heads(layouts.handle, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()),
+                                           dtype_code(k), B, n_new, C.c_void_p(seq_lens.data_ptr()),
+                                           C.c_void_p(cache.data_ptr()), capacity, _stream_ptr(stream)),
+           "encode_append_heads")
+
+
+def decode_attention_heads(layouts: LayoutSet, q, cache, seq_lens, capacity: int, max_seq_len: int, out, workspace,
+                           softmax_scale: float | None = None, stream=None):
+    """One decode-attention call over every KV head of a cache written by encode_append_heads."""
+    B, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_heads(layouts.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B, h_q,
+                                              C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                              max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                              C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_attention_heads")
+
+
+def decode_scores_heads(layouts: LayoutSet, q, cache, seq_lens, capacity: int, max_seq_len: int, scores, workspace,
+                        softmax_scale: float | None = None, stream=None):
+    """Logits of every KV head of a cache written by encode_append_heads: scores [B, h_q, ld]."""
+    B, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and scores.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_scores_heads(layouts.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B, h_q,
+                                           C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()), capacity,
+                                           max_seq_len, scale, C.c_void_p(scores.data_ptr()), scores.shape[-1],
+                                           C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_scores_heads")

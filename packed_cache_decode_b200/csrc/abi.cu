@@ -4,7 +4,9 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
+#include <new>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -267,21 +269,22 @@ namespace {
 
 // The checks and launches shared by the contiguous and the paged entry points; the
 // caller has checked the cache description and passes it as a CacheRef.
-bgtq_status encode_impl(const bgtq_layout* L, const char* who, const void* k, const void* v, int dtype, int batch,
-                        int n_new, int h_kv, const int* seq_lens_dev, const CacheRef& c, void* stream) {
+bgtq_status encode_impl(const DevLayout& D, const char* who, const void* k, const void* v, int dtype, int batch,
+                        int n_new, int h_kv, const int* seq_lens_dev, const CacheRef& c, void* stream,
+                        const DevLayout* heads = nullptr) {
   if (!valid_dtype(dtype)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad dtype");
   if (batch <= 0 || batch > 65535 || h_kv <= 0 || h_kv > 65535 || n_new < 0)
     return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad batch / h_kv / n_new");
   if (n_new == 0) return BGTQ_OK;
   if (!k || !v || !seq_lens_dev) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
-  cudaError_t e = launch_tq_encode(L->dev, k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c,
-                                   static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_tq_encode(D, k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c,
+                                   static_cast<cudaStream_t>(stream), heads);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
 
 // Shape checks of the attention calls; on success *plan is the launch plan.
-bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype, int batch, int h_q, int h_kv,
+bgtq_status attention_checks(const char* who, int q_dtype, int batch, int h_q, int h_kv,
                              int n_q, long long row_tokens, long long max_seq_len, float softmax_scale, const void* q,
                              const int* seq_lens_dev, const void* out, void* workspace, size_t workspace_bytes,
                              DecodePlan* plan) {
@@ -308,16 +311,16 @@ bgtq_status attention_checks(const bgtq_layout* L, const char* who, int q_dtype,
 }
 
 // rec non-null: partial records (m, l, o') instead of outputs (out is then rec).
-bgtq_status decode_impl(const bgtq_layout* L, const char* who, const void* q, int q_dtype, int batch, int h_q,
+bgtq_status decode_impl(const DevLayout& D, const char* who, const void* q, int q_dtype, int batch, int h_q,
                         int h_kv, int n_q, const CacheRef& c, const int* seq_lens_dev, long long max_seq_len,
                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes, void* stream,
-                        float* rec = nullptr) {
+                        float* rec = nullptr, const DevLayout* heads = nullptr) {
   DecodePlan plan;
-  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
+  bgtq_status st = attention_checks(who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
                                     softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
-  cudaError_t e = launch_decode(L->dev, plan, q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, softmax_scale, out,
-                                workspace, static_cast<cudaStream_t>(stream), rec);
+  cudaError_t e = launch_decode(D, plan, q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, softmax_scale, out,
+                                workspace, static_cast<cudaStream_t>(stream), rec, heads);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
@@ -332,7 +335,7 @@ bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, 
     return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad n_new");
   if (n_new > 0 && (!k_new || !v_new)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null pointer");
   DecodePlan plan;
-  bgtq_status st = attention_checks(L, who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
+  bgtq_status st = attention_checks(who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
                                     softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
   cudaError_t e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch,
@@ -370,7 +373,7 @@ bgtq_status bgtq_encode_append(const bgtq_layout* L, const void* k, const void* 
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("encode_append", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
-  return encode_impl(L, "encode_append", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
+  return encode_impl(L->dev, "encode_append", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
 }
 
 size_t bgtq_workspace_bytes(const bgtq_layout* L, int batch, int h_q, int h_kv, long long max_seq_len) {
@@ -394,7 +397,7 @@ bgtq_status bgtq_decode_attention(const bgtq_layout* L, const void* q, int q_dty
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_attention", const_cast<void*>(cache), capacity, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L->dev, "decode_attention", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -406,7 +409,7 @@ bgtq_status bgtq_decode_attention_partial(const bgtq_layout* L, const void* q, i
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_attention_partial", const_cast<void*>(cache), capacity, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention_partial", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L->dev, "decode_attention_partial", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, partial, workspace, workspace_bytes, stream, partial);
 }
 
@@ -451,7 +454,7 @@ bgtq_status bgtq_encode_append_paged(const bgtq_layout* L, const void* k, const 
   CacheRef c{};
   if (st == BGTQ_OK) st = paged("encode_append_paged", pool, num_pages, block_table_dev, max_pages, &c);
   if (st != BGTQ_OK) return st;
-  return encode_impl(L, "encode_append_paged", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
+  return encode_impl(L->dev, "encode_append_paged", k, v, dtype, batch, n_new, h_kv, seq_lens_dev, c, stream);
 }
 
 bgtq_status bgtq_decode_attention_paged(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q,
@@ -464,7 +467,7 @@ bgtq_status bgtq_decode_attention_paged(const bgtq_layout* L, const void* q, int
   if (st == BGTQ_OK) st = paged("decode_attention_paged", const_cast<void*>(pool), num_pages, block_table_dev,
                                 max_pages, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention_paged", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L->dev, "decode_attention_paged", q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -489,7 +492,7 @@ bgtq_status bgtq_decode_attention_multi(const bgtq_layout* L, const void* q, int
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_attention_multi", const_cast<void*>(cache), capacity, &c);
   if (st != BGTQ_OK) return st;
-  return decode_impl(L, "decode_attention_multi", q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, max_seq_len,
+  return decode_impl(L->dev, "decode_attention_multi", q, q_dtype, batch, h_q, h_kv, n_q, c, seq_lens_dev, max_seq_len,
                      softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -522,36 +525,51 @@ bgtq_status bgtq_decode_step_multi_paged(const bgtq_layout* L, const void* k_new
                    c, seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+bgtq_status scores_impl(const DevLayout& D, const char* who, const void* q, int q_dtype, int batch, int h_q,
+                        int h_kv, const void* cache, const int* seq_lens_dev, long long capacity,
+                        long long max_seq_len, float softmax_scale, float* scores, long long scores_ld,
+                        void* workspace, size_t workspace_bytes, void* stream, const DevLayout* heads = nullptr) {
+  const std::string w(who);
+  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, w + ": bad dtype");
+  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxCols)
+    return fail(BGTQ_ERR_INVALID, w + ": need h_q = G * h_kv with G in 1..32");
+  if ((long long)batch * h_kv * ((h_q / h_kv + kMaxG - 1) / kMaxG) > 65535)
+    return fail(BGTQ_ERR_INVALID, w + ": too many units (batch * h_kv * column tiles > 65535)");
+  if (capacity <= 0 || capacity % kTile)
+    return fail(BGTQ_ERR_CAPACITY, w + ": capacity must be a positive multiple of 64");
+  if (max_seq_len < 0 || max_seq_len > capacity)
+    return fail(BGTQ_ERR_CAPACITY, w + ": max_seq_len must be in [0, capacity]");
+  if (scores_ld < max_seq_len) return fail(BGTQ_ERR_INVALID, w + ": scores_ld < max_seq_len");
+  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, w + ": bad softmax_scale");
+  if (!q || !cache || !seq_lens_dev || !scores) return fail(BGTQ_ERR_INVALID, w + ": null pointer");
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
+  if (!workspace || workspace_bytes < plan.workspace_bytes)
+    return fail(BGTQ_ERR_WORKSPACE, w + ": workspace missing or smaller than bgtq_workspace_bytes()");
+  const CacheRef c{static_cast<uint8_t*>(const_cast<void*>(cache)), nullptr, capacity / kTile, 0};
+  e = launch_scores(D, plan, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, softmax_scale, scores, scores_ld,
+                    workspace, static_cast<cudaStream_t>(stream), heads);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return BGTQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
 bgtq_status bgtq_decode_scores(const bgtq_layout* L, const void* q, int q_dtype, int batch, int h_q, int h_kv,
                                const void* cache, const int* seq_lens_dev, long long capacity, long long max_seq_len,
                                float softmax_scale, float* scores, long long scores_ld, void* workspace,
                                size_t workspace_bytes, void* stream) {
   bgtq_status st = check_device(L, "decode_scores");
   if (st != BGTQ_OK) return st;
-  if (!valid_dtype(q_dtype)) return fail(BGTQ_ERR_INVALID, "decode_scores: bad dtype");
-  if (batch <= 0 || h_kv <= 0 || h_q <= 0 || h_q % h_kv || h_q / h_kv > kMaxCols)
-    return fail(BGTQ_ERR_INVALID, "decode_scores: need h_q = G * h_kv with G in 1..32");
-  if ((long long)batch * h_kv * ((h_q / h_kv + kMaxG - 1) / kMaxG) > 65535)
-    return fail(BGTQ_ERR_INVALID, "decode_scores: too many units (batch * h_kv * column tiles > 65535)");
-  if (capacity <= 0 || capacity % kTile)
-    return fail(BGTQ_ERR_CAPACITY, "decode_scores: capacity must be a positive multiple of 64");
-  if (max_seq_len < 0 || max_seq_len > capacity)
-    return fail(BGTQ_ERR_CAPACITY, "decode_scores: max_seq_len must be in [0, capacity]");
-  if (scores_ld < max_seq_len) return fail(BGTQ_ERR_INVALID, "decode_scores: scores_ld < max_seq_len");
-  if (!std::isfinite(softmax_scale)) return fail(BGTQ_ERR_INVALID, "decode_scores: bad softmax_scale");
-  if (!q || !cache || !seq_lens_dev || !scores) return fail(BGTQ_ERR_INVALID, "decode_scores: null pointer");
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return cuda_fail(e, "decode_scores");
-  const DecodePlan plan = plan_decode(batch, h_q, h_kv, max_seq_len, sms);
-  if (!workspace || workspace_bytes < plan.workspace_bytes)
-    return fail(BGTQ_ERR_WORKSPACE, "decode_scores: workspace missing or smaller than bgtq_workspace_bytes()");
-  const CacheRef c{static_cast<uint8_t*>(const_cast<void*>(cache)), nullptr, capacity / kTile, 0};
-  e = launch_scores(L->dev, plan, q, q_dtype, batch, h_q, h_kv, c, seq_lens_dev, softmax_scale, scores, scores_ld,
-                    workspace, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode_scores");
-  return BGTQ_OK;
+  return scores_impl(L->dev, "decode_scores", q, q_dtype, batch, h_q, h_kv, cache, seq_lens_dev, capacity,
+                     max_seq_len, softmax_scale, scores, scores_ld, workspace, workspace_bytes, stream);
 }
 
 bgtq_status bgtq_device_status(const bgtq_layout* L, unsigned* flags, int clear) {
@@ -562,6 +580,127 @@ bgtq_status bgtq_device_status(const bgtq_layout* L, unsigned* flags, int clear)
   if (e == cudaSuccess) e = cudaMemcpy(flags, L->dev.status, sizeof(unsigned), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && clear) e = cudaMemset(L->dev.status, 0, sizeof(unsigned));
   if (e != cudaSuccess) return cuda_fail(e, "device_status");
+  return BGTQ_OK;
+}
+
+// ------------------------------------------------------------------ one layout per KV head
+namespace {
+bgtq_status check_set(const bgtq_layout_set* S, const char* who) {
+  if (!S) return fail(BGTQ_ERR_INVALID, std::string(who) + ": null layout set");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  if (cur != S->device) return fail(BGTQ_ERR_DEVICE, std::string(who) + ": layout set lives on another device");
+  return BGTQ_OK;
+}
+}  // namespace
+
+bgtq_status bgtq_layout_set_create(const bgtq_layout* const* layouts, int n, bgtq_layout_set** out) {
+  if (!out) return fail(BGTQ_ERR_INVALID, "layout_set_create: null output");
+  *out = nullptr;
+  if (!layouts || n < 1 || n > 65535) return fail(BGTQ_ERR_INVALID, "layout_set_create: need 1..65535 layouts");
+  for (int h = 0; h < n; ++h) {
+    bgtq_status st = check_device(layouts[h], "layout_set_create");
+    if (st != BGTQ_OK) return st;
+    const bgtq_layout* a = layouts[0];
+    const bgtq_layout* b = layouts[h];
+    if (b->v_rate != a->v_rate || b->flags != a->flags || b->seed != a->seed)
+      return fail(BGTQ_ERR_INVALID, "layout_set_create: layouts differ in value rate, options or seed");
+  }
+  auto* S = new (std::nothrow) bgtq_layout_set;
+  if (!S) return fail(BGTQ_ERR_NOMEM, "layout_set_create: out of host memory");
+  S->n = n;
+  S->device = layouts[0]->device;
+  for (int h = 0; h < n; ++h) S->tile_stride = std::max(S->tile_stride, layouts[h]->tile_bytes);
+  const size_t bytes = 256 + sizeof(DevLayout) * size_t(n);
+  cudaError_t e = cudaMalloc(&S->dev_block, bytes);
+  if (e != cudaSuccess) {
+    delete S;
+    return cuda_fail(e, "layout_set_create");
+  }
+  unsigned* status = static_cast<unsigned*>(S->dev_block);
+  S->heads = reinterpret_cast<DevLayout*>(static_cast<char*>(S->dev_block) + 256);
+  std::vector<DevLayout> host(static_cast<size_t>(n) + 0);
+  for (int h = 0; h < n; ++h) {
+    host[h] = layouts[h]->dev;     // device pointers of the layout's own tables stay valid
+    host[h].tile_bytes = S->tile_stride;
+    host[h].status = status;
+  }
+  S->head0 = host[0];
+  e = cudaMemset(status, 0, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaMemcpy(S->heads, host.data(), sizeof(DevLayout) * size_t(n), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(S->dev_block);
+    delete S;
+    return cuda_fail(e, "layout_set_create");
+  }
+  *out = S;
+  return BGTQ_OK;
+}
+
+void bgtq_layout_set_destroy(bgtq_layout_set* S) {
+  if (!S) return;
+  if (S->dev_block) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != S->device) cudaSetDevice(S->device);
+    cudaFree(S->dev_block);
+    if (cur >= 0 && cur != S->device) cudaSetDevice(cur);
+  }
+  delete S;
+}
+
+int bgtq_layout_set_tile_bytes(const bgtq_layout_set* S) { return S ? S->tile_stride : 0; }
+
+size_t bgtq_layout_set_cache_bytes(const bgtq_layout_set* S, int batch, long long capacity) {
+  if (!S || batch <= 0 || capacity <= 0 || capacity % kTile) {
+    set_error("layout_set_cache_bytes: bad arguments");
+    return 0;
+  }
+  return size_t(batch) * size_t(S->n) * size_t(capacity / kTile) * size_t(S->tile_stride);
+}
+
+bgtq_status bgtq_encode_append_heads(const bgtq_layout_set* S, const void* k, const void* v, int dtype, int batch,
+                                     int n_new, const int* seq_lens_dev, void* cache, long long capacity,
+                                     void* stream) {
+  CacheRef c;
+  bgtq_status st = check_set(S, "encode_append_heads");
+  if (st == BGTQ_OK) st = contiguous("encode_append_heads", cache, capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return encode_impl(S->head0, "encode_append_heads", k, v, dtype, batch, n_new, S->n, seq_lens_dev, c, stream,
+                     S->heads);
+}
+
+bgtq_status bgtq_decode_attention_heads(const bgtq_layout_set* S, const void* q, int q_dtype, int batch, int h_q,
+                                        const void* cache, const int* seq_lens_dev, long long capacity,
+                                        long long max_seq_len, float softmax_scale, float* out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  CacheRef c;
+  bgtq_status st = check_set(S, "decode_attention_heads");
+  if (st == BGTQ_OK) st = contiguous("decode_attention_heads", const_cast<void*>(cache), capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(S->head0, "decode_attention_heads", q, q_dtype, batch, h_q, S->n, 1, c, seq_lens_dev,
+                     max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, nullptr, S->heads);
+}
+
+bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* S, const void* q, int q_dtype, int batch, int h_q,
+                                     const void* cache, const int* seq_lens_dev, long long capacity,
+                                     long long max_seq_len, float softmax_scale, float* scores, long long scores_ld,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  bgtq_status st = check_set(S, "decode_scores_heads");
+  if (st != BGTQ_OK) return st;
+  return scores_impl(S->head0, "decode_scores_heads", q, q_dtype, batch, h_q, S->n, cache, seq_lens_dev, capacity,
+                     max_seq_len, softmax_scale, scores, scores_ld, workspace, workspace_bytes, stream, S->heads);
+}
+
+bgtq_status bgtq_layout_set_status(const bgtq_layout_set* S, unsigned* flags, int clear) {
+  bgtq_status st = check_set(S, "layout_set_status");
+  if (st != BGTQ_OK) return st;
+  if (!flags) return fail(BGTQ_ERR_INVALID, "layout_set_status: null pointer");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(flags, S->dev_block, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && clear) e = cudaMemset(S->dev_block, 0, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "layout_set_status");
   return BGTQ_OK;
 }
 

@@ -32,7 +32,7 @@ constexpr int kTblVBytes = 64 * 32 * 4;
 constexpr int kTablesBytes = kTbl8Bytes + kTbl3Bytes + kTblVBytes;
 
 // Everything a kernel needs about one layer's packing, passed by value.
-struct DevLayout {
+struct alignas(16) DevLayout {  // (16-byte multiple: copied to shared memory in 16-byte units)
   int n_kgroups;
   int n_packed;         // stored key dimensions (packed dims n_packed..127 do not exist)
   int v_rate;
@@ -135,6 +135,17 @@ struct bgtq_layout {
   int device = -1;
   void* dev_block = nullptr;
   bgtq::DevLayout dev{};
+};
+
+// One layout per KV head (bgtq_layout_set_create): the device array of their DevLayouts,
+// each with the common tile stride and the set's status word.
+struct bgtq_layout_set {
+  int n = 0;                   // KV heads
+  int device = -1;
+  int tile_stride = 0;         // bytes per tile of every head (the largest tile of the layouts)
+  void* dev_block = nullptr;   // status word, then DevLayout[n]
+  bgtq::DevLayout* heads = nullptr;
+  bgtq::DevLayout head0{};     // heads[0] as the host passes it by value
 };
 
 namespace bgtq {

@@ -112,7 +112,16 @@ struct SplitArgs {
   long long scores_ld;
   int len_add;            // tokens appended by the previous kernel: row b attends over seq_lens[b] + len_add
   int wait_new;           // the previous kernel appends at seq_lens[b]: wait for it before copying that tile
+  const DevLayout* heads; // per-KV-head layouts (device array of h_kv), or null: one layout for all heads
 };
+
+// The layout a kernel works with: the by-value kernel parameter, or (PH: one layout per KV
+// head) a copy in shared memory of the current head's layout.
+template <bool PH>
+__device__ __forceinline__ const DevLayout& pick_layout(const DevLayout& param, const unsigned char* copy) {
+  if constexpr (PH) return *reinterpret_cast<const DevLayout*>(copy);
+  else return param;
+}
 
 constexpr int kQsLd = kD + 16;                   // row of q staged per group at 16-byte aligned columns
 
@@ -307,9 +316,9 @@ __device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4
     if constexpr (R <= 2) {
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt) {
-        const int m = 2 * rt;
         unsigned a0, a1, a2, a3;
         if constexpr (R == 1) {
+          const int m = 2 * rt;
           a0 = c0.a(m);
           a1 = c0.a(m + 1);
           a2 = c1.a(m);
@@ -342,9 +351,9 @@ __device__ __forceinline__ void key_group(float (&acc)[R >= 3 ? 2 * NRT : NRT][4
     if constexpr (R <= 2) {
 #pragma unroll
       for (int rt = 0; rt < NRT; ++rt) {
-        const int m = 2 * rt;
         unsigned a0, a1;
         if constexpr (R == 1) {
+          const int m = 2 * rt;
           a0 = c0.a(m);
           a1 = c0.a(m + 1);
         } else {
@@ -500,8 +509,8 @@ __device__ __forceinline__ void row_norms(unsigned row, int s0, float (&n)[2 * N
 // W: warps per CTA (one CTA per SM).
 // (the scores-only instantiation discards the softmax and value code of the tile body)
 #pragma nv_diag_suppress 128
-template <int VR, bool NP, bool SC, bool NH, int W>
-__global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs a) {
+template <int VR, bool NP, bool SC, bool NH, int W, bool PH>
+__global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout Lp, SplitArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // per key rate r (1..4): its group (-1: none), quads, byte offset of its first quad in a
   // tile, first q' pair slot; per lane: its offset inside a full quad and the offset of
@@ -510,10 +519,12 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
   __shared__ unsigned s_lof[5][32], s_olast[5][32];
   __shared__ int s_timeout;
   __shared__ float s_mm[W][8], s_ml[W][8];
+  __shared__ __align__(16) unsigned char s_layout[PH ? sizeof(DevLayout) : 16];
+  const DevLayout& L = pick_layout<PH>(Lp, s_layout);
   const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int TB = L.tile_bytes;
+  const int TB = Lp.tile_bytes;  // (the same for every head's layout)
 
   unsigned long long* full = reinterpret_cast<unsigned long long*>(smem);  // [2 W]
   unsigned char* t8 = smem + kSmT8;
@@ -521,49 +532,63 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
   unsigned char* ring = smem + sm_ring<VR>();                           // stage s at ring + s TB
   float* mo = reinterpret_cast<float*>(ring);  // the warps' [8][128] partials reuse the ring
 
+  __shared__ __align__(8) unsigned long long s_tbar;
   if (tid == 0) {
     s_timeout = 0;
     for (int i = 0; i < 2 * W; ++i) mbar_init(&full[i], 1);
-    fence_mbar_init();
-  }
-  // the decode tables: one bulk copy of the layout's prebuilt tables (value table of this
-  // variant's value rate included), waited for below, after the other set-up
-  __shared__ __align__(8) unsigned long long s_tbar;
-  constexpr unsigned kTblCopy = unsigned(sm_qf<VR>() - kSmT8);
-  if (tid == 0) {
     mbar_init(&s_tbar, 1);
     fence_mbar_init();
-    mbar_expect_tx(&s_tbar, kTblCopy);
-    bulk_load(t8, L.tables, kTblCopy, &s_tbar, evict_last_policy());
   }
-  if (tid < 5) s_gi[tid] = -1;
-  __syncthreads();
-  if (tid < L.n_kgroups) {
-    // groups are in descending rate order: the pair slots of the groups before this one
-    int slot = 0;
-    for (int gj = 0; gj < tid; ++gj) slot += (L.group_nquads[gj] + 1) >> 1;
-    const int r = L.group_rate[tid];
-    s_gi[r] = tid;
-    s_gnq[r] = L.group_nquads[tid];
-    s_gkb[r] = L.quad_off[L.group_quad0[tid]];
-    s_gslot[r] = slot;
-  }
-  for (int i = tid; i < L.n_kgroups * 32; i += 32 * W) {
-    // lane (g, t) holds pair t of a quad for tokens g + 8m: its 16 r bits are string
-    // li = g P + t of the quad's block (rate 3: plane A word li, plane B halfword li after
-    // 8 P words). Full quads have P = 4 (li = lane).
-    const int gi = i >> 5, ln = i & 31, r = L.group_rate[gi];
-    const int ql = L.group_quad0[gi] + L.group_nquads[gi] - 1, P = L.quad_np[ql], tt = ln & 3;
-    const int li = tt < P ? (ln >> 2) * P + tt : 0;
-    const unsigned full = r == 3 ? 4u * ln | ((128u + 2u * ln) << 16) : 2u * r * ln;
-    const unsigned base = unsigned(L.quad_off[ql]);
-    s_lof[r][ln] = full;
-    s_olast[r][ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
-  }
-  // every thread waits (bounded) for the tables; on a timeout the status says so and the
-  // decode goes on with whatever the tables hold (the call's output is then invalid)
-  if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_tbar, 0)) && lane == 0) atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
-  __syncthreads();
+  // The layout's decode state: its prebuilt tables (value table of this variant's value
+  // rate included) by one bulk copy, the group table and the lanes' code offsets. Once per
+  // CTA, and with per-head layouts again whenever a segment's head differs from the last
+  // one (every warp is then past the previous segment's merge: tables and ring are free).
+  constexpr unsigned kTblCopy = unsigned(sm_qf<VR>() - kSmT8);
+  auto load_layout = [&](int head, unsigned tphase) {
+    if constexpr (PH) {
+      static_assert(sizeof(DevLayout) % 16 == 0, "layout copied in 16-byte units");
+      const uint4* src = reinterpret_cast<const uint4*>(a.heads + head);
+      for (int i = tid; i < int(sizeof(DevLayout) / 16); i += 32 * W) reinterpret_cast<uint4*>(s_layout)[i] = src[i];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      mbar_expect_tx(&s_tbar, kTblCopy);
+      bulk_load(t8, L.tables, kTblCopy, &s_tbar, evict_last_policy());
+    }
+    if (tid < 5) s_gi[tid] = -1;
+    __syncthreads();
+    if (tid < L.n_kgroups) {
+      // groups are in descending rate order: the pair slots of the groups before this one
+      int slot = 0;
+      for (int gj = 0; gj < tid; ++gj) slot += (L.group_nquads[gj] + 1) >> 1;
+      const int r = L.group_rate[tid];
+      s_gi[r] = tid;
+      s_gnq[r] = L.group_nquads[tid];
+      s_gkb[r] = L.quad_off[L.group_quad0[tid]];
+      s_gslot[r] = slot;
+    }
+    for (int i = tid; i < L.n_kgroups * 32; i += 32 * W) {
+      // lane (g, t) holds pair t of a quad for tokens g + 8m: its 16 r bits are string
+      // li = g P + t of the quad's block (rate 3: plane A word li, plane B halfword li after
+      // 8 P words). Full quads have P = 4 (li = lane).
+      const int gi = i >> 5, ln = i & 31, r = L.group_rate[gi];
+      const int ql = L.group_quad0[gi] + L.group_nquads[gi] - 1, P = L.quad_np[ql], tt = ln & 3;
+      const int li = tt < P ? (ln >> 2) * P + tt : 0;
+      const unsigned fl = r == 3 ? 4u * ln | ((128u + 2u * ln) << 16) : 2u * r * ln;
+      const unsigned base = unsigned(L.quad_off[ql]);
+      s_lof[r][ln] = fl;
+      s_olast[r][ln] = r == 3 ? (base + 4u * li) | ((base + 32u * P + 2u * li) << 16) : base + 2u * r * li;
+    }
+    // every thread waits (bounded) for the tables; on a timeout the status says so and the
+    // decode goes on with whatever the tables hold (the call's output is then invalid)
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_tbar, tphase)) && lane == 0)
+      atomicOr(L.status, BGTQ_STATUS_TIMEOUT);
+    __syncthreads();
+  };
+  const long long M0 = a.max_tiles, T0 = a.total_tiles, C0 = a.n_ctas;
+  int cur_head = int(((long long)c * T0 / C0) / M0 / a.CT % a.h_kv);
+  unsigned n_loads = 0;  // completed phases of s_tbar
+  load_layout(cur_head, n_loads++ & 1u);
 
   const float vscale = rsqrtf(float(kD)) / L.kappa_v;
   const unsigned lane4 = unsigned(lane) << 2;
@@ -581,6 +606,13 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout L, SplitArgs
   bool q_ready = false;
 
   for (int u = u_first; u <= u_last; ++u) {
+    if constexpr (PH) {
+      const int head = u / a.CT % a.h_kv;  // uniform over the CTA
+      if (head != cur_head) {
+        cur_head = head;
+        load_layout(head, n_loads++ & 1u);
+      }
+    }
     const Segment S = make_segment(L, a, c, u, tid == 0);
     const int srow = S.u / a.CT / a.h_kv, shead = S.u / a.CT % a.h_kv;
     const int col0 = S.u % a.CT * kMaxG;  // first column of this unit's tile in its KV head
@@ -1026,7 +1058,7 @@ inline int split_smem_bytes(int v_rate, int tile_bytes, int warps) {
 // Once per device and variant: the largest dynamic shared memory the kernel may use (the
 // device's per-block opt-in limit minus the kernel's static shared memory), set as the
 // kernel's limit together with the whole unified L1/shared array as shared memory.
-template <int VR, bool NP, bool SC, bool NH, int W>
+template <int VR, bool NP, bool SC, bool NH, int W, bool PH>
 cudaError_t configure_split(int* dyn_limit) {
   static int limit[64] = {};
   int dev = 0;
@@ -1037,12 +1069,12 @@ cudaError_t configure_split(int* dyn_limit) {
     int optin = 0;
     cudaFuncAttributes fa{};
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, split_kernel<VR, NP, SC, NH, W>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, split_kernel<VR, NP, SC, NH, W, PH>);
     if (e != cudaSuccess) return e;
     const int dyn = optin - int(fa.sharedSizeBytes);
-    e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(split_kernel<VR, NP, SC, NH, W, PH>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                int(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) return e;
     limit[dev] = dyn;
@@ -1051,10 +1083,10 @@ cudaError_t configure_split(int* dyn_limit) {
   return cudaSuccess;
 }
 
-template <int VR, bool NP, bool SC, bool NH, int W>
+template <int VR, bool NP, bool SC, bool NH, int W, bool PH>
 cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas, int smem, cudaStream_t stream) {
   int limit = 0;
-  cudaError_t e = configure_split<VR, NP, SC, NH, W>(&limit);
+  cudaError_t e = configure_split<VR, NP, SC, NH, W, PH>(&limit);
   if (e != cudaSuccess) return e;
   if (smem > limit) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
@@ -1067,7 +1099,7 @@ cudaError_t launch_split(const SplitArgs& a, const DevLayout& L, unsigned n_ctas
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC, NH, W>, L, a);
+  return cudaLaunchKernelEx(&cfg, split_kernel<VR, NP, SC, NH, W, PH>, L, a);
 }
 
 // q' B fragments of unit u (batch row b, KV head h) into frag[kMaxQuads][2][32] (global),
@@ -1217,13 +1249,22 @@ __device__ __forceinline__ void prep_unit(const DevLayout& L, const void* __rest
   }
 }
 
-__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const void* __restrict__ q, int q_dtype,
+// The KV head of q' unit u (column tiles of ceil(Gt / 8) per cache unit).
+__device__ __forceinline__ int unit_head(int u, int h_kv, int Gt) { return u / ((Gt + kMaxG - 1) / kMaxG) % h_kv; }
+
+// PH: heads[h] is the layout of KV head h (else L for every head).
+template <bool PH>
+__global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const DevLayout* __restrict__ heads,
+                                                             const void* __restrict__ q, int q_dtype,
                                                              int h_q, int h_kv, int Gt, int n_q, float qscale,
                                                              unsigned* __restrict__ qfrag) {
   // launched after the kernel before it has completed: the split kernel may start now
   pdl_trigger();
   const int u = blockIdx.x;
-  prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+  if constexpr (PH)
+    prep_unit(heads[unit_head(u, h_kv, Gt)], q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+  else
+    prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
 }
 
 // First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
@@ -1314,7 +1355,7 @@ int split_warps(int v_rate, int tile_bytes, int limit) {
 cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int batch, int h_q, int h_kv, int n_q,
                              const CacheRef& cache, const int* seq_lens, float* out, void* workspace,
                              int len_add, bool after_append, cudaStream_t stream, float* scores = nullptr,
-                             long long scores_ld = 0, float* rec = nullptr) {
+                             long long scores_ld = 0, float* rec = nullptr, const DevLayout* heads = nullptr) {
   const int hc = h_q * n_q, Gt = hc / h_kv, CT = (Gt + kMaxG - 1) / kMaxG, G = CT == 1 ? Gt : kMaxG;
   // G <= 4: the q' hi and lo parts share one m16n8k8 product (columns 0-3 and 4-7)
   const bool np = G <= 4;
@@ -1349,12 +1390,17 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
   a.scores_ld = scores_ld;
   a.len_add = len_add;
   a.wait_new = after_append ? 1 : 0;
+  a.heads = heads;
   const unsigned n_ctas = unsigned(plan.n_ctas);
   cudaError_t e = split_variant(L.v_rate, np, sc, nh, [&](auto V, auto P, auto S, auto H) {
     constexpr int VR = decltype(V)::value;
     constexpr bool NPv = decltype(P)::value != 0, SCv = decltype(S)::value != 0, NHv = decltype(H)::value != 0;
-    return W == 12 ? launch_split<VR, NPv, SCv, NHv, 12>(a, L, n_ctas, smem, stream)
-                   : launch_split<VR, NPv, SCv, NHv, 8>(a, L, n_ctas, smem, stream);
+    auto go = [&](auto ph) {
+      constexpr bool PHv = decltype(ph)::value;
+      return W == 12 ? launch_split<VR, NPv, SCv, NHv, 12, PHv>(a, L, n_ctas, smem, stream)
+                     : launch_split<VR, NPv, SCv, NHv, 8, PHv>(a, L, n_ctas, smem, stream);
+    };
+    return heads ? go(std::true_type{}) : go(std::false_type{});
   });
   if (sc || e != cudaSuccess) return e;  // scores only: no merge
   return launch_dependent(combine_kernel, unsigned(batch * hc), kCombThreads, stream, (const float*)a.part_ml,
@@ -1387,17 +1433,21 @@ DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int 
 
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
-                          float* out, void* workspace, cudaStream_t stream, float* rec) {
+                          float* out, void* workspace, cudaStream_t stream, float* rec, const DevLayout* heads) {
   const int Gt = h_q * n_q / h_kv;
   const long long units = (long long)batch * h_kv * ((Gt + kMaxG - 1) / kMaxG);
   // a plain launch: the split kernel, launched as soon as this kernel starts, reads the
   // cache, which the kernel before this one may write
-  qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+  if (heads)
+    qprep_kernel<true><<<unsigned(units), kPrepThreads, 0, stream>>>(
+        L, heads, q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+  else
+    qprep_kernel<false><<<unsigned(units), kPrepThreads, 0, stream>>>(
+        L, nullptr, q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens, out, workspace, 0, false, stream,
-                          nullptr, 0, rec);
+                          nullptr, 0, rec, heads);
 }
 
 namespace {
@@ -1439,15 +1489,19 @@ cudaError_t launch_merge_records(const DevLayout& L, const float* recs, int n_re
 
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
                           int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale, float* scores,
-                          long long scores_ld, void* workspace, cudaStream_t stream) {
+                          long long scores_ld, void* workspace, cudaStream_t stream, const DevLayout* heads) {
   const int Gt = h_q / h_kv;
   const long long units = (long long)batch * h_kv * ((Gt + kMaxG - 1) / kMaxG);
-  qprep_kernel<<<unsigned(units), kPrepThreads, 0, stream>>>(
-      L, q, q_dtype, h_q, h_kv, Gt, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+  if (heads)
+    qprep_kernel<true><<<unsigned(units), kPrepThreads, 0, stream>>>(
+        L, heads, q, q_dtype, h_q, h_kv, Gt, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
+  else
+    qprep_kernel<false><<<unsigned(units), kPrepThreads, 0, stream>>>(
+        L, nullptr, q, q_dtype, h_q, h_kv, Gt, 1, softmax_scale * kLog2e, static_cast<unsigned*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, 1, cache, seq_lens, nullptr, workspace, 0, false, stream,
-                          scores, scores_ld);
+                          scores, scores_ld, nullptr, heads);
 }
 
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,

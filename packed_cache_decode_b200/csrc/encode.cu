@@ -10,13 +10,21 @@ namespace bgtq {
 
 namespace {
 
-template <bool NC>
-__global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayout L, const void* __restrict__ k,
+// The layout of KV head h: the kernel parameter, or (PH) heads[h] in global memory.
+template <bool PH>
+__device__ __forceinline__ const DevLayout& head_layout(const DevLayout& param, const DevLayout* heads, int h) {
+  if constexpr (PH) return heads[h];
+  else return param;
+}
+
+template <bool NC, bool PH>
+__global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayout Lp, const DevLayout* __restrict__ heads,
+                                                                        const void* __restrict__ k,
                                                                         const void* __restrict__ v, int dtype,
                                                                         int n_new, int h_kv,
                                                                         const int* __restrict__ seq_lens, CacheRef cache) {
-  enc::encode_token_part<NC>(L, k, v, dtype, n_new, h_kv, seq_lens, cache, blockIdx.x / kEncodeParts,
-                         blockIdx.x % kEncodeParts, blockIdx.y, blockIdx.z);
+  enc::encode_token_part<NC>(head_layout<PH>(Lp, heads, blockIdx.z), k, v, dtype, n_new, h_kv, seq_lens, cache,
+                             blockIdx.x / kEncodeParts, blockIdx.x % kEncodeParts, blockIdx.y, blockIdx.z);
 }
 
 // ------------------------------------------------------------------ bulk appends
@@ -126,8 +134,9 @@ __device__ __forceinline__ double y_fp64_warp(const double* rt64, const float* x
   return sqrt(double(d)) * dot / n64;
 }
 
-template <bool NC>
-__global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayout L, const void* __restrict__ k,
+template <bool NC, bool PH>
+__global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayout Lp, const DevLayout* __restrict__ heads,
+                                                                                const void* __restrict__ k,
                                                                                 const void* __restrict__ v, int dtype,
                                                                                 int n_new, int h_kv,
                                                                                 const int* __restrict__ seq_lens,
@@ -147,6 +156,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
   __shared__ int s_nnear;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.y, h = blockIdx.z;
+  const DevLayout& L = head_layout<PH>(Lp, heads, h);
   pdl_wait();
   const long long pos0 = seq_lens[b];
   const long long tix = pos0 / kTile + blockIdx.x;
@@ -361,33 +371,32 @@ size_t bulk_smem_bytes(int tile_bytes) {
 }  // namespace
 
 cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, int dtype, int batch,
-                             int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream) {
+                             int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream,
+                             const DevLayout* heads) {
+  const bool ph = heads != nullptr, nc = L.norm_correct != 0;
   if (n_new >= kBulkMinTokens) {
     // bulk appends: one CTA per touched tile (at most ceil(n_new / 64) + 1 per row)
     const size_t smem = bulk_smem_bytes(L.tile_bytes);
-    static bool configured[64][2] = {};
+    static bool configured[64][4] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const int nc = L.norm_correct ? 1 : 0;
-    if (dev < 64 && !configured[dev][nc]) {
-      e = cudaFuncSetAttribute(nc ? tq_encode_tile_kernel<true> : tq_encode_tile_kernel<false>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(bulk_smem_bytes(kMaxTileBytes)));
+    const int vi = (nc ? 1 : 0) + (ph ? 2 : 0);
+    auto kern = nc ? (ph ? tq_encode_tile_kernel<true, true> : tq_encode_tile_kernel<true, false>)
+                   : (ph ? tq_encode_tile_kernel<false, true> : tq_encode_tile_kernel<false, false>);
+    if (dev < 64 && !configured[dev][vi]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bulk_smem_bytes(kMaxTileBytes)));
       if (e != cudaSuccess) return e;
-      configured[dev][nc] = true;
+      configured[dev][vi] = true;
     }
     dim3 grid(unsigned((n_new + kTile - 1) / kTile + 1), batch, h_kv);
-    if (nc)
-      tq_encode_tile_kernel<true><<<grid, kBulkThreads, smem, stream>>>(L, k, v, dtype, n_new, h_kv, seq_lens,
-                                                                               cache);
-    else
-      tq_encode_tile_kernel<false><<<grid, kBulkThreads, smem, stream>>>(L, k, v, dtype, n_new, h_kv, seq_lens,
-                                                                                cache);
+    kern<<<grid, kBulkThreads, smem, stream>>>(L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache);
     return cudaGetLastError();
   }
   dim3 grid(n_new * kEncodeParts, batch, h_kv);
-  if (!L.norm_correct) {
-    tq_encode_kernel<false><<<grid, enc::kEncodeThreads, 0, stream>>>(L, k, v, dtype, n_new, h_kv, seq_lens, cache);
+  if (!nc) {
+    if (ph) tq_encode_kernel<false, true><<<grid, enc::kEncodeThreads, 0, stream>>>(L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache);
+    else tq_encode_kernel<false, false><<<grid, enc::kEncodeThreads, 0, stream>>>(L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache);
     return cudaGetLastError();
   }
   // norm correction: the four parts of a token form one cluster (they exchange sums)
@@ -402,7 +411,8 @@ cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, i
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tq_encode_kernel<true>, L, k, v, dtype, n_new, h_kv, seq_lens, cache);
+  return ph ? cudaLaunchKernelEx(&cfg, tq_encode_kernel<true, true>, L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache)
+            : cudaLaunchKernelEx(&cfg, tq_encode_kernel<true, false>, L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache);
 }
 
 }  // namespace bgtq

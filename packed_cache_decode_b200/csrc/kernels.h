@@ -23,14 +23,19 @@ struct DecodePlan {
 // ctas_per_sm <= 0: the most split CTAs that fit an SM (the workspace of any launch plan).
 DecodePlan plan_decode(int batch, int h_q, int h_kv, long long max_seq_len, int num_sms, int ctas_per_sm = 0);
 
+// heads (device array of h_kv layouts, or null): KV head h is coded with heads[h] (every
+// layout of the array has the same value rate, norm options and tile stride L.tile_bytes;
+// L is heads[0] as the host sees it).
 cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, int dtype, int batch,
-                             int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream);
+                             int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream,
+                             const DevLayout* heads = nullptr);
 
 // n_q query tokens per row (q [batch][n_q][h_q][128], out likewise), causal among them;
 // the plan is made for h_q n_q query columns.
 cudaError_t launch_decode(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch,
                           int h_q, int h_kv, int n_q, const CacheRef& cache, const int* seq_lens, float softmax_scale,
-                          float* out, void* workspace, cudaStream_t stream, float* rec = nullptr);
+                          float* out, void* workspace, cudaStream_t stream, float* rec = nullptr,
+                          const DevLayout* heads = nullptr);
 
 // Merge of partial records over disjoint token ranges: recs [n_rec][columns][130]
 // (m, l, o' of each query column), out [columns][128] = R_V^T (log-sum-exp merge of o').
@@ -51,6 +56,6 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
 // scores-only form).
 cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void* q, int q_dtype, int batch, int h_q,
                           int h_kv, const CacheRef& cache, const int* seq_lens, float softmax_scale, float* scores,
-                          long long scores_ld, void* workspace, cudaStream_t stream);
+                          long long scores_ld, void* workspace, cudaStream_t stream, const DevLayout* heads = nullptr);
 
 }  // namespace bgtq

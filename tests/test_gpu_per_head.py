@@ -1,7 +1,7 @@
 """Rate allocation per KV head through the C ABI: every KV head gets its own energy score,
-rates and layout (its own groups, rotations and tile format), is cached in its own buffer
-and decoded by its own call (h_kv = 1); each head matches the oracle with that head's
-layout."""
+rates and layout (its own groups, rotations and tile format). Each head is cached and
+decoded either by its own calls (h_kv = 1) or, through a layout set, together with the
+other heads in one call; each head matches the oracle with that head's layout."""
 import math
 
 import numpy as np
@@ -50,3 +50,80 @@ def test_per_head_layouts_match_oracle(min_rate):
                                      1 / math.sqrt(128))
             for i in range(G):
                 assert rel_l2(got[b, i], ref[i]) <= ATTN_REL_L2, (h, b, i)
+
+
+def _head_tiles(cache, batch, h_kv, n_tiles, stride, tile_bytes, b, h):
+    """The first tile_bytes of every tile of (row b, head h) in a cache of tile stride `stride`."""
+    return cache.view(batch, h_kv, n_tiles, stride)[b, h, :, :tile_bytes]
+
+
+@pytest.mark.parametrize("shape", [(16, 4, 0), (16, 2, 1)], ids=["gqa4_min0", "gqa8_min1"])
+def test_layout_set_one_call_matches_oracle(shape):
+    """A layout set: one encode and one attention call for every KV head, each head with its
+    own layout. The tiles equal those of the head's own single-layout cache byte for byte,
+    the outputs match the oracle per query head, the logits equal the single-head calls'."""
+    h_q, h_kv, min_rate = shape
+    case = Case(h_q, h_kv, 2, 500, 2, 2, torch.bfloat16, 5e5, 62)
+    m = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, case.seed + 1, case.theta)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2, min_rate=min_rate)
+    assert len({tuple(r) for r in rates}) > 1                      # the heads' layouts differ
+    q, k, v = synth.make_cache_inputs(m, case.batch, case.length, case.seed, case.theta, case.dtype)
+    layouts = [B.Layout(rates[h], case.v_bits, case.seed).upload(0) for h in range(h_kv)]
+    S = B.LayoutSet(layouts)
+    stride, n_tiles = S.tile_bytes, case.cap // 64
+    assert stride == max(lay.tile_bytes for lay in layouts)
+    cache = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    kd, vd = k.cuda(), v.cuda()
+    # bulk appends (>= 8 tokens) and single-token appends
+    for a0, a1 in ((0, 300), (300, 303), (303, 500)):
+        lens0 = torch.full((case.batch,), a0, dtype=torch.int32, device="cuda")
+        B.encode_append_heads(S, kd[:, a0:a1].contiguous(), vd[:, a0:a1].contiguous(), lens0, cache, case.cap)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    G = h_q // h_kv
+    lens = torch.tensor([500, 433], dtype=torch.int32, device="cuda")
+    ws = torch.empty(B.workspace_bytes(layouts[0], case.batch, h_q, h_kv, case.length), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full((case.batch, h_q, 128), float("nan"), device="cuda")
+    B.decode_attention_heads(S, q.cuda(), cache, lens, case.cap, case.length, out, ws)
+    ld = case.length + 5
+    sc = torch.full((case.batch, h_q, ld), float("nan"), device="cuda")
+    B.decode_scores_heads(S, q.cuda(), cache, lens, case.cap, case.length, sc, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    got = out.cpu().double().numpy()
+    for h, lay in enumerate(layouts):
+        # the head's own cache, written and read through the single-layout calls
+        own = torch.zeros(lay.cache_bytes(case.batch, 1, case.cap), dtype=torch.uint8, device="cuda")
+        B.encode_append(lay, kd[:, :, h:h + 1].contiguous(), vd[:, :, h:h + 1].contiguous(),
+                        torch.zeros(case.batch, dtype=torch.int32, device="cuda"), own, case.cap)
+        ws1 = torch.empty(B.workspace_bytes(lay, case.batch, G, 1, case.length), dtype=torch.uint8, device="cuda")
+        sc1 = torch.full((case.batch, G, ld), float("nan"), device="cuda")
+        B.decode_scores(lay, q[:, h * G:(h + 1) * G].contiguous().cuda(), own, lens, case.cap, case.length, sc1, ws1, 1)
+        torch.cuda.synchronize()
+        assert lay.status() == 0
+        for b in range(case.batch):
+            mine = own.view(case.batch, n_tiles, lay.tile_bytes)[b]
+            assert torch.equal(_head_tiles(cache, case.batch, h_kv, n_tiles, stride, lay.tile_bytes, b, h), mine), (h, b)
+        assert torch.equal(sc[:, h * G:(h + 1) * G].isnan(), sc1.isnan())
+        assert torch.equal(sc[:, h * G:(h + 1) * G].nan_to_num(), sc1.nan_to_num()), h
+        olay = O.make_layout(rates[h], case.v_bits, case.seed)
+        for b in range(case.batch):
+            enc = O.encode(olay, k[b, :, h].double().numpy(), v[b, :, h].double().numpy())
+            ref = O.decode_attention(olay, q[b, h * G:(h + 1) * G].double().numpy(), O.pack(olay, enc, case.cap),
+                                     int(lens[b]), 1 / math.sqrt(128))
+            for i in range(G):
+                assert rel_l2(got[b, h * G + i], ref[i]) <= ATTN_REL_L2, (h, b, i)
+
+
+def test_layout_set_rejects_mixed_layouts():
+    a = B.Layout(np.full(64, 2), 2, 0).upload(0)
+    b = B.Layout(np.full(64, 2), 3, 0).upload(0)          # another value rate
+    c = B.Layout(np.full(64, 2), 2, 1).upload(0)          # another seed (value rotation)
+    for pair in ((a, b), (a, c)):
+        with pytest.raises(B.BgtqError) as e:
+            B.LayoutSet(pair)
+        assert e.value.status == B.ERR_INVALID
+    with pytest.raises(B.BgtqError):
+        B.LayoutSet([a, B.Layout(np.full(64, 2), 2, 0)])   # not uploaded
