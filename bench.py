@@ -407,7 +407,7 @@ def run_mae(args):
     unquantised keys (fp64). Reports the mean absolute logit error of both layouts, and of
     the block allocation with norm correction and/or fp16 norms and of the allocation that
     may leave blocks uncoded (rates from 0) and of an allocation per KV head (each head its
-    own layout, one call per head), with each layout's
+    own layout, all heads in one call through a layout set), with each layout's
     resident bytes per (token, KV head) and its footprint ratio to an fp16 K+V record
     (512 bytes)."""
     dev = torch.device("cuda", 0)
@@ -447,24 +447,22 @@ def run_mae(args):
             line[f"bytes_per_token_{tag}"] = lay.bytes_per_token
             line[f"footprint_x_{tag}"] = round(2 * 128 * 2 / lay.bytes_per_token, 3)
             assert lay.status() == 0
-        # an allocation per KV head: every head's own rates and layout, one call per head
+        # an allocation per KV head: every head's own rates and layout, all heads in one
+        # encode and one scores call through a layout set
         per_head = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), wl.k_bits)
-        err, nbytes = 0.0, 0
-        for h in range(wl.h_kv):
-            lay = B.Layout(per_head[h], wl.v_bits, wl.seed).upload(0)
-            cache = torch.zeros(lay.cache_bytes(1, 1, wl.length), dtype=torch.uint8, device=dev)
-            lens = torch.zeros(1, dtype=torch.int32, device=dev)
-            B.encode_append(lay, k[:, :, h:h + 1].contiguous().to(dev), v[:, :, h:h + 1].contiguous().to(dev), lens,
-                            cache, wl.length)
-            lens.fill_(wl.length)
-            ws = torch.empty(B.workspace_bytes(lay, 1, G, 1, wl.length), dtype=torch.uint8, device=dev)
-            sc = torch.empty(1, G, wl.length, dtype=torch.float32, device=dev)
-            B.decode_scores(lay, q[:, h * G:(h + 1) * G].contiguous().to(dev), cache, lens, wl.length, wl.length, sc,
-                            ws, 1)
-            torch.cuda.synchronize()
-            assert lay.status() == 0
-            err += float((sc[0].double() - exact[h * G:(h + 1) * G]).abs().sum())
-            nbytes += lay.bytes_per_token
+        heads = [B.Layout(per_head[h], wl.v_bits, wl.seed).upload(0) for h in range(wl.h_kv)]
+        S = B.LayoutSet(heads)
+        cache = torch.zeros(S.cache_bytes(1, wl.length), dtype=torch.uint8, device=dev)
+        lens = torch.zeros(1, dtype=torch.int32, device=dev)
+        B.encode_append_heads(S, k.to(dev), v.to(dev), lens, cache, wl.length)
+        lens.fill_(wl.length)
+        ws = torch.empty(B.workspace_bytes(heads[0], 1, wl.h_q, wl.h_kv, wl.length), dtype=torch.uint8, device=dev)
+        sc = torch.empty(1, wl.h_q, wl.length, dtype=torch.float32, device=dev)
+        B.decode_scores_heads(S, q.to(dev), cache, lens, wl.length, wl.length, sc, ws)
+        torch.cuda.synchronize()
+        assert S.status() == 0
+        err = float((sc[0].double() - exact).abs().sum())
+        nbytes = sum(lay.bytes_per_token for lay in heads)
         line["mae_block_gtq_per_head"] = err / (wl.h_q * wl.length)
         line["bytes_per_token_block_gtq_per_head"] = nbytes / wl.h_kv
         line["reduction"] = 1.0 - line["mae_block_gtq"] / line["mae_uniform"]

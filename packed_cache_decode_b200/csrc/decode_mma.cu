@@ -606,6 +606,21 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout Lp, SplitArg
   bool q_ready = false;
 
   for (int u = u_first; u <= u_last; ++u) {
+    if (s_timeout) {
+      // a copy engine stalled earlier in this CTA: it is not waited on again, and the CTA's
+      // remaining units get empty partials (m = -inf, l = 0, o' = 0), which the merge ignores
+      const Segment S = make_segment(L, a, c, u, false);
+      for (int it = tid; it < a.G * kD; it += 32 * W) {
+        const int hh = it >> 7, d = it & (kD - 1);
+        const size_t idx = ((size_t)S.u * a.n_parts + S.part) * a.G + hh;
+        a.part_o[idx * kD + d] = 0.f;
+        if (d == 0) {
+          a.part_ml[idx * 2] = -INFINITY;
+          a.part_ml[idx * 2 + 1] = 0.f;
+        }
+      }
+      continue;
+    }
     if constexpr (PH) {
       const int head = u / a.CT % a.h_kv;  // uniform over the CTA
       if (head != cur_head) {
@@ -931,8 +946,7 @@ __global__ void __launch_bounds__(32 * W, 1) split_kernel(DevLayout Lp, SplitArg
         a.part_ml[idx * 2 + 1] = l;
       }
     }
-    __syncthreads();  // the merge area is the next segment's ring
-    if (s_timeout) break;  // uniform over the CTA: a copy engine that stalled once is not waited on again
+    __syncthreads();  // the merge area is the next segment's ring (s_timeout is uniform from here)
   }
 }
 #pragma nv_diag_default 128

@@ -68,14 +68,16 @@ __device__ __forceinline__ void load_column(const T* __restrict__ p, size_t stri
 }
 
 // Half a dot product for N tokens: acc[t] += sum_{jj < n} r[jj ld] x[jj][t], x rows at
-// kXsLd floats.
+// kXsLd floats. The loop runs n_warp >= n steps, the same for the whole warp: steps past
+// the lane's own n read no rotation element and add zero times the lane's last row (its
+// own inputs: a non-finite input elsewhere cannot reach this sum).
 template <int N>
 __device__ __forceinline__ void half_dot(const float* __restrict__ r, int ld, const float* __restrict__ x, int n,
-                                         float (&acc)[N]) {
-#pragma unroll 2
-  for (int jj = 0; jj < n; ++jj) {
-    const float rij = r[jj * ld];
-    const float4* xr = reinterpret_cast<const float4*>(x + jj * kXsLd);
+                                         int n_warp, float (&acc)[N]) {
+#pragma unroll 4
+  for (int jj = 0; jj < n_warp; ++jj, r += ld, x += jj < n ? kXsLd : 0) {
+    const float rij = jj < n ? *r : 0.f;
+    const float4* xr = reinterpret_cast<const float4*>(x);
 #pragma unroll
     for (int q = 0; q < N / 4; ++q) {
       const float4 v = xr[q];
@@ -217,6 +219,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
   const float sdk = sqrtf(float(dk)), sdv = sqrtf(float(kD));
   const float bound_k = 2.f * (sdk * float(dk + 1) + 8.f) * 5.9604645e-8f + 1e-6f;
   const float bound_v = 2.f * (sdv * float(kD + 1) + 8.f) * 5.9604645e-8f + 1e-6f;
+  const int nk_warp = __reduce_max_sync(0xffffffffu, klive ? dk / 2 : 0);  // key steps of the warp
   bool rot_ready = false;
 
   for (long long t0 = t_lo; t0 < t_hi; t0 += kBulkTokens) {
@@ -238,22 +241,32 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
             make_float4(xv[4 * q], xv[4 * q + 1], xv[4 * q + 2], xv[4 * q + 3]);
     }
     __syncthreads();
-    // group norms in fp64: warp w takes tokens w, w + 16; a fixed order of sums
-    for (int tk = warp; tk < nt; tk += kBulkThreads / 32) {
-      for (int gg = 0; gg <= ng; ++gg) {
-        const int a = gg < ng ? L.group_off[gg] : kD, n = gg < ng ? L.group_dim[gg] : kD;
-        double s2 = 0.0;
-        for (int j = lane; j < n; j += 32) {
-          const double x = xs[(a + j) * kXsLd + tk];
-          s2 = fma(x, x, s2);
-        }
+    // group norms in fp64: warp w takes tokens w, w + 16; a fixed order of sums. Lane i
+    // keeps the i-th sum of its warp and takes its square root (in parallel)
+    {
+      double my_s2 = 0.0;
+      int my_e = -1, my_n = 0, slot = 0;
+      for (int tk = warp; tk < nt; tk += kBulkThreads / 32) {
+        for (int gg = 0; gg <= ng; ++gg, ++slot) {
+          const int a = gg < ng ? L.group_off[gg] : kD, n = gg < ng ? L.group_dim[gg] : kD;
+          double s2 = 0.0;
+          for (int j = lane; j < n; j += 32) {
+            const double x = xs[(a + j) * kXsLd + tk];
+            s2 = fma(x, x, s2);
+          }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-        if (lane == 0) {
-          const int e = tk * (kMaxGroups + 1) + (gg < ng ? gg : kMaxGroups);
-          nrm[e] = sqrt(s2);
-          sc[e] = s2 > 0.0 ? float(sqrt(double(n) / s2)) : 0.f;  // sqrt(d) / |x_g|
+          for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+          if (lane == slot) {
+            my_s2 = s2;
+            my_e = tk * (kMaxGroups + 1) + (gg < ng ? gg : kMaxGroups);
+            my_n = n;
+          }
         }
+      }
+      if (my_e >= 0) {
+        const double nr = sqrt(my_s2);
+        nrm[my_e] = nr;
+        sc[my_e] = my_s2 > 0.0 ? sqrtf(float(my_n)) / float(nr) : 0.f;  // sqrt(d) / |x_g|, fp32
       }
     }
     if (!rot_ready) {
@@ -277,7 +290,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
       const float* xh = xs + kHalfTokens * tb;
 #pragma unroll
       for (int t = 0; t < kHalfTokens; ++t) acc[t] = 0.f;
-      half_dot(rs + s_roff[kMaxGroups] + (kD / 2) * hh * kD + p, kD, xh + (kD + (kD / 2) * hh) * kXsLd, kD / 2, acc);
+      half_dot(rs + s_roff[kMaxGroups] + (kD / 2) * hh * kD + p, kD, xh + (kD + (kD / 2) * hh) * kXsLd, kD / 2, kD / 2,
+               acc);
       pair_sum(acc, hh, y);
       unsigned near = decide(y, sc + tk0 * (kMaxGroups + 1) + kMaxGroups, s_thr + L.v_rate * kThrLd, sdv, bound_v,
                              nt - tk0, cw);
@@ -290,7 +304,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
       // packed key dimension p: rows j = dk/2 hh .. of its group's rotation
 #pragma unroll
       for (int t = 0; t < kHalfTokens; ++t) acc[t] = 0.f;
-      if (klive) half_dot(rs + s_roff[g] + (dk / 2) * hh * dk + ki, dk, xh + (koff + (dk / 2) * hh) * kXsLd, dk / 2, acc);
+      half_dot(rs + s_roff[g] + (dk / 2) * hh * dk + ki, dk, xh + (koff + (dk / 2) * hh) * kXsLd, klive ? dk / 2 : 0,
+               nk_warp, acc);
       pair_sum(acc, hh, y);
       if (klive) {
         near = decide(y, sc + tk0 * (kMaxGroups + 1) + g, s_thr + rk * kThrLd, sdk, bound_k, nt - tk0, cw);

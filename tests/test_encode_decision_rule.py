@@ -20,7 +20,7 @@ def _y32(rot32t, x32, i, norm):
     # the kernel's fp32 dot: two halves of the j range, each acc = fma(R[i][j], x_j, acc) in
     # j order, then added (numpy float32 rounds the product and the sum separately, a
     # looser computation than a fused multiply-add); then y = acc f with f = sqrt(d) / |x|
-    # computed in fp64 and rounded to fp32
+    # in fp32 (|x| from fp64, rounded to fp32)
     d = len(x32)
     half = []
     for j0, j1 in ((0, d // 2), (d // 2, d)):
@@ -29,7 +29,7 @@ def _y32(rot32t, x32, i, norm):
             acc = np.float32(acc + np.float32(rot32t[j, i] * x32[j]))
         half.append(acc)
     acc = np.float32(half[0] + half[1])
-    f = np.float32(math.sqrt(d / (norm * norm)))
+    f = np.float32(np.float32(math.sqrt(d)) / np.float32(norm))
     return float(np.float32(acc * f))
 
 
