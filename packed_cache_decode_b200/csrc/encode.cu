@@ -28,9 +28,9 @@ __global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayou
 }
 
 // ------------------------------------------------------------------ bulk appends
-// One CTA of 512 threads per (touched tile, batch row, KV head): the tile is read into
-// shared memory, the new tokens' codes and norms are written there (shared atomics only:
-// no other CTA touches the tile) and the tile is written back. The rotations (transposed
+// One CTA of 512 threads per (pair of touched tiles, batch row, KV head): the tiles are read
+// into shared memory, the new tokens' codes and norms are written there (shared atomics
+// only: no other CTA touches these tiles) and the tiles are written back. The rotations (transposed
 // fp32, every K group's then V's) arrive by bulk copies while the tile and the first
 // tokens load. Tokens go in blocks of 32; threads 0-255 take tokens 0-15 of a block and
 // threads 256-511 tokens 16-31. In each half, lanes l and l + 16 of warp w share packed
@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(enc::kEncodeThreads) tq_encode_kernel(DevLayou
 // are fp64.
 constexpr int kBulkTokens = 32;
 constexpr int kBulkThreads = 512;         // two halves of 256: tokens 0-15 and 16-31 of a block
+constexpr int kCtaTiles = 2;              // most tiles a CTA owns: its blocks of 32 tokens may straddle them
 constexpr int kHalfTokens = kBulkTokens / 2;
 constexpr int kXsLd = kBulkTokens + 4;    // floats per row of the block's inputs (rows 16-byte aligned)
 constexpr int kRotFloats = 2 * kD * kD;   // the K groups' rotations (sum of d_g^2 <= 128^2) and V's
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
                                                                                 const void* __restrict__ v, int dtype,
                                                                                 int n_new, int h_kv,
                                                                                 const int* __restrict__ seq_lens,
-                                                                                CacheRef cache) {
+                                                                                CacheRef cache, int cta_tiles) {
   extern __shared__ __align__(16) unsigned char sm[];
   float* rs = reinterpret_cast<float*>(sm);                                  // rotations (transposed fp32)
   float* xs = rs + kRotFloats;                                               // [256 dims][kXsLd]
@@ -161,8 +162,9 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
   const DevLayout& L = head_layout<PH>(Lp, heads, h);
   pdl_wait();
   const long long pos0 = seq_lens[b];
-  const long long tix = pos0 / kTile + blockIdx.x;
-  long long t_lo = max(pos0, tix * kTile), t_hi = min(pos0 + n_new, (tix + 1) * kTile);
+  // the CTA's tiles: cta_tiles (1 or 2) consecutive tiles from tix0
+  const long long tix0 = pos0 / kTile + (long long)cta_tiles * blockIdx.x;
+  long long t_lo = max(pos0, tix0 * kTile), t_hi = min(pos0 + n_new, (tix0 + cta_tiles) * kTile);
   if (pos0 < 0 || t_lo >= t_hi) return;
   const long long cap = cache.n_tiles * kTile;
   if (t_hi > cap) {
@@ -170,8 +172,15 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
     t_hi = cap;
     if (t_lo >= t_hi) return;
   }
-  uint8_t* gt = tile_ptr(cache, L, b, h, h_kv, tix);
-  if (!gt) return;
+  // the CTA's tiles (a page outside a paged pool is flagged, its tile left out)
+  const int n_t = int((t_hi - 1) / kTile - tix0) + 1;
+  uint8_t* gt[kCtaTiles];
+#pragma unroll
+  for (int i = 0; i < kCtaTiles; ++i) gt[i] = i < n_t ? tile_ptr(cache, L, b, h, h_kv, tix0 + i) : nullptr;
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < kCtaTiles; ++i) any = any || gt[i] != nullptr;
+  if (!any) return;
   const int ng = L.n_kgroups;
   if (tid == 0) {
     // every K group's rotation, then V's: d_g^2 floats each (d_g even: whole 16-byte units)
@@ -191,8 +200,11 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
     bulk_load(rs + o, L.v_rot32t, unsigned(kD * kD) * 4u, &s_bar, keep);
   }
   const int TB = L.tile_bytes;
-  for (int i = tid; i < TB / 16; i += kBulkThreads)
-    reinterpret_cast<uint4*>(tile)[i] = reinterpret_cast<const uint4*>(gt)[i];
+#pragma unroll
+  for (int ti = 0; ti < kCtaTiles; ++ti)
+    if (gt[ti])
+      for (int i = tid; i < TB / 16; i += kBulkThreads)
+        reinterpret_cast<uint4*>(tile + ti * TB)[i] = reinterpret_cast<const uint4*>(gt[ti])[i];
   if (tid < kD) s_pc[tid] = L.packed_coord[tid];
   if (tid < 5 * kThrLd) {
     const int rr = tid / kThrLd, m = tid % kThrLd;
@@ -338,12 +350,15 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
     __syncthreads();
     if (tid == 0) s_nnear = 0;  // next read after the next block's first barrier
     {
-      // the codes of this lane's 8 tokens into the tile (one copy of the packing code)
-      const int tt0 = int(t0 % kTile), t1 = min(nt, tk0 + 8);
+      // the codes of this lane's 8 tokens into their tiles (one copy of the packing code)
+      const int t1 = min(nt, tk0 + 8);
 #pragma unroll 1
       for (int tk = tk0; tk < t1; ++tk) {
-        enc::put_value_code(L, tile, p, tt0 + tk, cd[(kD + p) * kBulkTokens + tk]);
-        if (klive) enc::put_key_code(L, tile, g, ki, tt0 + tk, cd[p * kBulkTokens + tk]);
+        const long long t = t0 + tk;
+        unsigned char* tp = tile + int(t / kTile - tix0) * TB;
+        const int tt = int(t % kTile);
+        enc::put_value_code(L, tp, p, tt, cd[(kD + p) * kBulkTokens + tk]);
+        if (klive) enc::put_key_code(L, tp, g, ki, tt, cd[p * kBulkTokens + tk]);
       }
     }
     // norms (with norm correction: |x| sqrt(d) / |c|, |c|^2 summed in a fixed order)
@@ -364,9 +379,11 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
         s = c2 > 0.0 ? s * sqrt(double(n)) / sqrt(c2) : 0.0;
       }
       if (lane == 0) {
-        const int ent = enc::norm_entry(int((t0 + tk) % kTile));
-        if (gg < ng) enc::store_norm(L, tile + L.knorm_off, gg * kTile + ent, s);
-        else enc::store_norm(L, tile + L.vnorm_off, ent, s);
+        const long long t = t0 + tk;
+        unsigned char* tp = tile + int(t / kTile - tix0) * TB;
+        const int ent = enc::norm_entry(int(t % kTile));
+        if (gg < ng) enc::store_norm(L, tp + L.knorm_off, gg * kTile + ent, s);
+        else enc::store_norm(L, tp + L.vnorm_off, ent, s);
       }
     }
   }
@@ -374,13 +391,16 @@ __global__ void __launch_bounds__(kBulkThreads, 1) tq_encode_tile_kernel(DevLayo
   // a kernel launched as this one's dependent may start (it waits for this grid before it
   // reads the tiles written here)
   pdl_trigger();
-  for (int i2 = tid; i2 < TB / 16; i2 += kBulkThreads)
-    reinterpret_cast<uint4*>(gt)[i2] = reinterpret_cast<const uint4*>(tile)[i2];
+#pragma unroll
+  for (int ti = 0; ti < kCtaTiles; ++ti)
+    if (gt[ti])
+      for (int i2 = tid; i2 < TB / 16; i2 += kBulkThreads)
+        reinterpret_cast<uint4*>(gt[ti])[i2] = reinterpret_cast<const uint4*>(tile + ti * TB)[i2];
 }
 
 size_t bulk_smem_bytes(int tile_bytes) {
   return size_t(kRotFloats) * 4 + size_t(256) * kXsLd * 4 + size_t(kBulkTokens) * (kMaxGroups + 1) * 12 +
-         size_t(kBulkTokens) * 256 * 3 + size_t(tile_bytes);
+         size_t(kBulkTokens) * 256 * 3 + size_t(kCtaTiles) * size_t(tile_bytes);
 }
 
 }  // namespace
@@ -390,7 +410,7 @@ cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, i
                              const DevLayout* heads) {
   const bool ph = heads != nullptr, nc = L.norm_correct != 0;
   if (n_new >= kBulkMinTokens) {
-    // bulk appends: one CTA per touched tile (at most ceil(n_new / 64) + 1 per row)
+    // bulk appends: one CTA per pair of touched tiles
     const size_t smem = bulk_smem_bytes(L.tile_bytes);
     static bool configured[64][4] = {};
     int dev = 0;
@@ -404,8 +424,17 @@ cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, i
       if (e != cudaSuccess) return e;
       configured[dev][vi] = true;
     }
-    dim3 grid(unsigned((n_new + kTile - 1) / kTile + 1), batch, h_kv);
-    kern<<<grid, kBulkThreads, smem, stream>>>(L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache);
+    // a row's new tokens touch at most ceil(n_new / 64) + 1 tiles: two per CTA (a block of
+    // 32 tokens may then straddle them) when that still gives every SM a CTA, else one
+    static int sms[64] = {};
+    if (dev < 64 && !sms[dev]) {
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+    }
+    const long long tiles = (n_new + kTile - 1) / kTile + 1;
+    const int ct = (tiles + 1) / 2 * (long long)batch * h_kv >= (dev < 64 ? sms[dev] : 148) ? kCtaTiles : 1;
+    dim3 grid(unsigned((tiles + ct - 1) / ct), batch, h_kv);
+    kern<<<grid, kBulkThreads, smem, stream>>>(L, heads, k, v, dtype, n_new, h_kv, seq_lens, cache, ct);
     return cudaGetLastError();
   }
   dim3 grid(n_new * kEncodeParts, batch, h_kv);
