@@ -57,7 +57,7 @@ def _head_tiles(cache, batch, h_kv, n_tiles, stride, tile_bytes, b, h):
     return cache.view(batch, h_kv, n_tiles, stride)[b, h, :, :tile_bytes]
 
 
-@pytest.mark.parametrize("shape", [(16, 4, 0), (16, 2, 1)], ids=["gqa4_min0", "gqa8_min1"])
+@pytest.mark.parametrize("shape", [(16, 4, 0), (16, 2, 1), (32, 2, 1)], ids=["gqa4_min0", "gqa8_min1", "gqa16_two_column_tiles"])
 def test_layout_set_one_call_matches_oracle(shape):
     """A layout set: one encode and one attention call for every KV head, each head with its
     own layout. The tiles equal those of the head's own single-layout cache byte for byte,
