@@ -140,7 +140,9 @@ def compare_packed(lay: O.Layout, enc: dict, want: np.ndarray, got: np.ndarray, 
     if lay.norm_correct:
         differs = np.zeros(nt * 64, dtype=bool)
         differs[:n] = np.any(kd, axis=1) | np.any(vd, axis=1)
-        per_tile = differs.reshape(nt, 1, 64)     # norm entry j of a tile belongs to token j % 64
+        # norm entry e of a tile's row of 64 belongs to token 8 (e % 8) + e // 8 (slot-major)
+        e = np.arange(64)
+        per_tile = differs.reshape(nt, 64)[:, 8 * (e % 8) + e // 8].reshape(nt, 1, 64)
         ulp = np.where(np.broadcast_to(per_tile, (nt, lay.n_kgroups + 1, 64)).reshape(nt, -1), 0, ulp)
     assert ulp.max() <= 1, f"norm differs by {ulp.max()} ulp"
     NEAR_STATS["coords"] += coords

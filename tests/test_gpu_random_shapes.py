@@ -1,0 +1,86 @@
+"""Seeded random shapes through the C ABI against the oracle: query heads per KV head,
+query tokens per row (up to 32 columns per KV head), batch, ragged lengths, key and value
+rates, input dtype, norm correction, fp16 norms, rate-0 blocks, and appends split into
+chunks of random sizes (short appends take the per-token encoder, longer ones the bulk
+encoder; a chunk may start anywhere inside a tile). Every packed (row, KV head) slice is
+compared with the oracle's bytes, every query column's output with the oracle's
+attention."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from packed_cache_decode_b200 import binding as B
+from packed_cache_decode_b200 import synth
+
+from .parity_util import ATTN_REL_L2, Case, build_inputs, compare_packed, rel_l2, slice_bytes
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = [torch.float32, torch.bfloat16, torch.float16]
+
+
+def _draw(i):
+    rng = np.random.default_rng(7000 + i)
+    while True:
+        G = int(rng.choice([1, 2, 3, 4, 5, 6, 8, 12, 16]))
+        n_q = int(rng.choice([1, 2, 3, 4]))
+        if G * n_q <= 32:
+            break
+    h_kv = int(rng.integers(1, 4))
+    case = Case(G * h_kv, h_kv, int(rng.integers(1, 4)), int(rng.integers(n_q + 40, 700)), int(rng.choice([2, 3])),
+                int(rng.integers(1, 5)), DTYPES[int(rng.integers(0, 3))], 5e5, 100 + i,
+                norm_correct=bool(rng.integers(0, 2)), norm_fp16=bool(rng.integers(0, 2)),
+                min_rate=int(rng.integers(0, 2)))
+    # append chunks: a long one, a short one (per-token encoder), the rest
+    a = int(rng.integers(1, case.length - 10))
+    b = a + int(rng.integers(1, 8))
+    return case, n_q, [0, a, b, case.length]
+
+
+@pytest.mark.parametrize("i", range(10))
+def test_random_shape_matches_oracle(i):
+    case, n_q, bounds = _draw(i)
+    model, rates, _, k, v = build_inputs(case)
+    lay = B.Layout(rates, case.v_bits, case.seed, case.norm_correct, case.norm_fp16).upload(0)
+    cache = torch.zeros(lay.cache_bytes(case.batch, case.h_kv, case.cap), dtype=torch.uint8, device="cuda")
+    kd, vd = k.cuda(), v.cuda()
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if b > a:
+            lens0 = torch.full((case.batch,), a, dtype=torch.int32, device="cuda")
+            B.encode_append(lay, kd[:, a:b].contiguous(), vd[:, a:b].contiguous(), lens0, cache, case.cap)
+    torch.cuda.synchronize()
+    assert lay.status() == 0
+    olay = O.make_layout(rates, case.v_bits, case.seed, case.norm_correct, case.norm_fp16)
+    cache_cpu = cache.cpu().numpy()
+    bufs = {}
+    for b in range(case.batch):
+        for h in range(case.h_kv):
+            enc = O.encode(olay, k[b, :, h].double().numpy(), v[b, :, h].double().numpy())
+            want = O.pack(olay, enc, case.cap)
+            compare_packed(olay, enc, want, slice_bytes(case, olay.tile_bytes, cache_cpu, b, h), case.cap)
+            bufs[b, h] = want
+    # ragged rows; the last n_q cached tokens of each row carry its queries
+    lens = torch.tensor([max(n_q, case.length - 53 * b) for b in range(case.batch)], dtype=torch.int32)
+    q = torch.empty(case.batch, n_q, case.h_q, 128, dtype=case.dtype)
+    for b in range(case.batch):
+        for hq in range(case.h_q):
+            q[b, :, hq] = synth.query_slice(model, b, hq, n_q, int(lens[b]) - n_q, case.seed, case.theta).to(case.dtype)
+    out = torch.full((case.batch, n_q, case.h_q, 128), float("nan"), device="cuda")
+    ws = torch.empty(B.workspace_bytes(lay, case.batch, case.h_q * n_q, case.h_kv, case.length), dtype=torch.uint8,
+                     device="cuda")
+    B.decode_attention_multi(lay, q.cuda(), cache, lens.cuda(), case.cap, case.length, out, ws, case.h_kv)
+    torch.cuda.synchronize()
+    assert lay.status() == 0
+    got = out.cpu().double().numpy()
+    G = case.h_q // case.h_kv
+    for b in range(case.batch):
+        for h in range(case.h_kv):
+            ref = O.decode_attention_multi(olay, q[b, :, h * G:(h + 1) * G].double().numpy(), bufs[b, h],
+                                           int(lens[b]), 1 / math.sqrt(128))
+            for j in range(n_q):
+                for c in range(G):
+                    err = rel_l2(got[b, j, h * G + c], ref[j, c])
+                    assert err <= ATTN_REL_L2, (case, n_q, b, h, j, c, err)
