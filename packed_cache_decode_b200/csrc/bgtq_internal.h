@@ -18,7 +18,8 @@ constexpr int kMaxCols = BGTQ_MAX_GQA;   // query columns per KV head: column ti
 constexpr int kMaxGroups = BGTQ_MAX_KGROUPS;
 constexpr int kMaxQuads = 20;            // sum over groups of ceil(d_g / 8) <= 128/8 + 3
 constexpr int kEncodeParts = 4;          // encode CTAs per (token, KV head), 32 outputs each
-constexpr int kBulkMinTokens = 8;        // appends of this many tokens per row or more: one CTA per tile
+constexpr int kBulkMinTokens = 4;        // appends of this many tokens per row or more (2 or more when
+                                         // batch x KV heads >= 256): the bulk encoder
 
 // Decode lookup tables, built once per layout (host, at upload) in the order the split
 // kernel keeps them in shared memory: 256 rows of 256 bytes (bytes 0-127: 16 copies of the

@@ -409,7 +409,9 @@ cudaError_t launch_tq_encode(const DevLayout& L, const void* k, const void* v, i
                              int n_new, int h_kv, const int* seq_lens, const CacheRef& cache, cudaStream_t stream,
                              const DevLayout* heads) {
   const bool ph = heads != nullptr, nc = L.norm_correct != 0;
-  if (n_new >= kBulkMinTokens) {
+  // the bulk encoder's cost hardly grows with the tokens a row appends, the per-token
+  // encoder's grows with every token: measured crossover at 4 tokens, 2 for 256 rows x heads
+  if (n_new >= kBulkMinTokens || (n_new >= 2 && (long long)batch * h_kv >= 256)) {
     // bulk appends: one CTA per pair of touched tiles
     const size_t smem = bulk_smem_bytes(L.tile_bytes);
     static bool configured[64][4] = {};

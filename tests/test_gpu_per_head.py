@@ -75,7 +75,7 @@ def test_layout_set_one_call_matches_oracle(shape):
     assert stride == max(lay.tile_bytes for lay in layouts)
     cache = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
     kd, vd = k.cuda(), v.cuda()
-    # bulk appends (>= 8 tokens) and single-token appends
+    # bulk appends (>= 4 tokens) and a 3-token append (the per-token encoder)
     for a0, a1 in ((0, 300), (300, 303), (303, 500)):
         lens0 = torch.full((case.batch,), a0, dtype=torch.int32, device="cuda")
         B.encode_append_heads(S, kd[:, a0:a1].contiguous(), vd[:, a0:a1].contiguous(), lens0, cache, case.cap)
