@@ -214,3 +214,25 @@ def test_new_host_calls_refuse_bad_arguments(lib):
     neg = np.full(64, 2, dtype=np.int32)
     neg[3] = -1
     assert lib.bgtq_layout_create(p(neg), 2, 0, C.byref(h)) == B.ERR_INVALID
+
+
+def test_layout_set_refuses_bad_arguments_without_device(lib):
+    """bgtq_layout_set_create checks its arguments before touching a device: no output
+    pointer, no layouts, and layouts that are not uploaded are refused; the size queries
+    of a null set answer 0."""
+    h = C.c_void_p()
+    assert lib.bgtq_layout_set_create(None, 1, C.byref(h)) == B.ERR_INVALID
+    lay = B.Layout(np.full(64, 2), 2, 0)
+    arr = (C.c_void_p * 1)(lay.handle)
+    assert lib.bgtq_layout_set_create(arr, 0, C.byref(h)) == B.ERR_INVALID
+    assert lib.bgtq_layout_set_create(arr, 1, None) == B.ERR_INVALID
+    assert lib.bgtq_layout_set_create(arr, 1, C.byref(h)) == B.ERR_DEVICE     # not uploaded
+    assert not h.value
+    assert lib.bgtq_layout_set_tile_bytes(None) == 0
+    assert lib.bgtq_layout_set_cache_bytes(None, 1, 64) == 0
+    f = C.c_uint(0)
+    assert lib.bgtq_layout_set_status(None, C.byref(f), 0) == B.ERR_INVALID
+    assert lib.bgtq_encode_append_heads(None, None, None, 0, 1, 1, None, None, 64, None) == B.ERR_INVALID
+    assert lib.bgtq_decode_attention_heads(None, None, 0, 1, 1, None, None, 64, 64, 0.1, None, None, 0,
+                                           None) == B.ERR_INVALID
+    lib.bgtq_layout_set_destroy(None)                                          # a no-op
