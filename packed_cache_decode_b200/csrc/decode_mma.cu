@@ -6,12 +6,13 @@
 //   o           = R_V^T sum_t p_t (|v_t| / sqrt(128)) c[vcodes_t] / sum_t p_t.
 //
 // Three kernels per call, chained by programmatic dependent launch:
-//  * qprep_kernel (one CTA per batch row x KV head; in a decode step, step_prep_kernel also
-//    runs the encode CTAs of the new tokens): q' = R_g q_g for the G query columns of the
-//    KV head (fp32, scaled by softmax_scale * log2(e) / (sqrt(d_g) kappa_g)), split into
-//    fp16 hi + lo parts and laid out as mma B fragments. A column is one query head at
-//    one query token: G = query heads per KV head x n_q query tokens (n_q = 1 except in
-//    multi-token calls).
+//  * qprep_kernel (one CTA per unit; in a decode step, step_prep_kernel also runs the
+//    encode CTAs of the new tokens): q' = R_g q_g for the unit's query columns (fp32,
+//    scaled by softmax_scale * log2(e) / (sqrt(d_g) kappa_g)), split into fp16 hi + lo
+//    parts and laid out as mma B fragments, plus the column sums of the rate-1 group's
+//    fragments. A column is one query head at one query token: a KV head has Gt = query
+//    heads per KV head x n_q columns (n_q = 1 except in multi-token calls), taken 8 at a
+//    time: a unit is (batch row, KV head, column tile of up to 8 columns).
 //  * split_kernel: one CTA per SM, 8 or 12 warps. The (batch row, KV head) caches are
 //    laid end to end as one sequence of 64-token tiles and every CTA takes an equal slice
 //    of it (one wave). Inside a slice, unit by unit, warp w streams its own tiles w, w+W,
@@ -19,15 +20,21 @@
 //    mbarrier, L2 evict-first, no multicast), contiguous or paged; the tiles left over after
 //    a multiple of W go out whole or as half tiles (row blocks 0-1 and 2-3) so that no warp
 //    runs more than half a tile past the others. Keys: per quad of 4 dimension pairs one
-//    load gives the lane its codes for its 8 tokens (fragment-major format); rate 1 turns
-//    into +-1 pairs with bit operations; rates 2 and 4 look up byte-indexed tables (one
-//    prmt builds the address from a code byte, one 64-bit shared load returns two A
-//    registers, or a hi + lo pair at rate 4); rate 3 indexes a 6-bit pair table. The
-//    tables hold 16 copies of every entry, lane l reading copy l % 16, so a half-warp's
-//    64-bit loads never share a bank. A group's quads go in pairs into mma.m16n8k16
-//    (for G <= 4 the q' hi and lo parts are the eight columns of one product). fp32
-//    accumulators per group, then times the group norm (fp32 or fp16, a template
-//    variant). Each column masks the tokens past its own position (the row's last tiles
+//    load gives the lane its codes for its 8 tokens (fragment-major format); rate 1 gives
+//    0/1 operands straight from the code bits (an fp16 subnormal 2^(m-24) or 0, exact),
+//    turned into +-1 codes afterwards with the rate-1 column sums of q'; rates 2 and 4
+//    look up byte-indexed tables (one prmt builds the address from a code byte, one
+//    64-bit shared load returns two A registers, or a hi + lo pair at rate 4); rate 3
+//    indexes a 6-bit pair table. Rates 3 and 4 put a slot's centroid hi parts in rows g
+//    and their lo parts in rows g+8 of one product, summed afterwards. The tables are
+//    built once per layout (at upload), fetched by one bulk copy per CTA, and hold 16
+//    copies of every entry, lane l reading copy l % 16, so a half-warp's 64-bit loads
+//    never share a bank. A group's quads go in pairs into mma.m16n8k16 (for units of at
+//    most 4 columns the q' hi and lo parts are the eight columns of one product). fp32
+//    accumulators per group (started by the group's first products), then times the
+//    group norm (fp32 or fp16, a template variant). With one layout per KV head (a
+//    layout set) the CTA reloads the layout and its tables when its segment's head
+//    changes. Each column masks the tokens past its own position (the row's last tiles
 //    only). Online softmax in base 2 with warp shuffles. Values: the probabilities times
 //    |v|/sqrt(128) in fp16, transposed with movmatrix, against value codes turned into A
 //    registers the same way (rate 2: the byte table), accumulated in V's rotated space
