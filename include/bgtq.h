@@ -370,6 +370,15 @@ bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* set, const void* q, 
                                      long long max_seq_len, float softmax_scale, float* scores,
                                      long long scores_ld, void* workspace, size_t workspace_bytes,
                                      void* stream);
+/* bgtq_decode_step over a cache written by bgtq_encode_append_heads: appends n_new tokens
+ * per row (k_new, v_new [batch, n_new, h_kv, 128], every KV head coded with its own layout)
+ * and attends the query over the grown cache, in one kernel chain (h_kv = the set's size).
+ * Arguments, ownership and errors otherwise as bgtq_decode_step. */
+bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* set, const void* k_new, const void* v_new,
+                                   int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,
+                                   void* cache, const int* seq_lens_dev, long long capacity,
+                                   long long max_seq_len, float softmax_scale, float* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 /* The set's status bits (BGTQ_STATUS_*), as bgtq_device_status. */
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* set, unsigned* flags, int clear);
 

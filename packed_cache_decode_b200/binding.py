@@ -35,6 +35,7 @@ EXPORTED = [
     "bgtq_block_energy_heads", "bgtq_decode_attention_partial", "bgtq_merge_partials",
     "bgtq_layout_set_create", "bgtq_layout_set_destroy", "bgtq_layout_set_tile_bytes", "bgtq_layout_set_cache_bytes",
     "bgtq_encode_append_heads", "bgtq_decode_attention_heads", "bgtq_decode_scores_heads", "bgtq_layout_set_status",
+    "bgtq_decode_step_heads",
 ]
 
 
@@ -101,6 +102,7 @@ def load():
         "bgtq_decode_attention_heads": (I, [P, P, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
         "bgtq_decode_scores_heads": (I, [P, P, I, I, I, P, P, LL, LL, F, P, LL, P, C.c_size_t, P]),
         "bgtq_layout_set_status": (I, [P, C.POINTER(C.c_uint), I]),
+        "bgtq_decode_step_heads": (I, [P, P, P, I, I, P, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -574,3 +576,19 @@ def decode_scores_heads(layouts: LayoutSet, q, cache, seq_lens, capacity: int, m
                                            max_seq_len, scale, C.c_void_p(scores.data_ptr()), scores.shape[-1],
                                            C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_scores_heads")
+
+
+def decode_step_heads(layouts: LayoutSet, k_new, v_new, q, cache, seq_lens, capacity: int, max_seq_len: int, out,
+                      workspace, softmax_scale: float | None = None, stream=None):
+    """Append k_new, v_new [B, n_new, h_kv, 128] (KV head h with layout h of the set) at
+    seq_lens[b] and attend q [B, h_q, 128] over seq_lens[b] + n_new tokens, one chain."""
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and h_kv == layouts.h_kv and k_new.is_contiguous() and v_new.is_contiguous()
+    assert q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_heads(layouts.handle, C.c_void_p(k_new.data_ptr()), C.c_void_p(v_new.data_ptr()),
+                                         dtype_code(k_new), n_new, C.c_void_p(q.data_ptr()), dtype_code(q), B_,
+                                         q.shape[1], C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()),
+                                         capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                         C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
+           "decode_step_heads")

@@ -326,10 +326,10 @@ bgtq_status decode_impl(const DevLayout& D, const char* who, const void* q, int 
 }
 
 // n_q = 1: one query per row at the newest position; n_q = n_new: the new tokens' queries.
-bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, const void* v_new, int kv_dtype,
+bgtq_status step_impl(const DevLayout& D, const char* who, const void* k_new, const void* v_new, int kv_dtype,
                       int n_new, const void* q, int q_dtype, int batch, int h_q, int h_kv, int n_q, const CacheRef& c,
                       const int* seq_lens_dev, long long max_seq_len, float softmax_scale, float* out,
-                      void* workspace, size_t workspace_bytes, void* stream) {
+                      void* workspace, size_t workspace_bytes, void* stream, const DevLayout* heads = nullptr) {
   if (!valid_dtype(kv_dtype)) return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad dtype");
   if (n_new < 0 || (long long)n_new * kEncodeParts * batch * h_kv + (long long)batch * h_kv > 0x7fffffffLL)
     return fail(BGTQ_ERR_INVALID, std::string(who) + ": bad n_new");
@@ -338,9 +338,9 @@ bgtq_status step_impl(const bgtq_layout* L, const char* who, const void* k_new, 
   bgtq_status st = attention_checks(who, q_dtype, batch, h_q, h_kv, n_q, c.n_tiles * kTile, max_seq_len,
                                     softmax_scale, q, seq_lens_dev, out, workspace, workspace_bytes, &plan);
   if (st != BGTQ_OK) return st;
-  cudaError_t e = launch_decode_step(L->dev, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch,
+  cudaError_t e = launch_decode_step(D, plan, k_new, v_new, kv_dtype, n_new, seq_lens_dev, q, q_dtype, batch,
                                      h_q, h_kv, n_q, c, softmax_scale, out, workspace,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<cudaStream_t>(stream), heads);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return BGTQ_OK;
 }
@@ -435,7 +435,7 @@ bgtq_status bgtq_decode_step(const bgtq_layout* L, const void* k_new, const void
   CacheRef c{};
   if (st == BGTQ_OK) st = contiguous("decode_step", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
-  return step_impl(L, "decode_step", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev,
+  return step_impl(L->dev, "decode_step", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c, seq_lens_dev,
                    max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -480,7 +480,7 @@ bgtq_status bgtq_decode_step_paged(const bgtq_layout* L, const void* k_new, cons
   CacheRef c{};
   if (st == BGTQ_OK) st = paged("decode_step_paged", pool, num_pages, block_table_dev, max_pages, &c);
   if (st != BGTQ_OK) return st;
-  return step_impl(L, "decode_step_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c,
+  return step_impl(L->dev, "decode_step_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, 1, c,
                    seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -506,7 +506,7 @@ bgtq_status bgtq_decode_step_multi(const bgtq_layout* L, const void* k_new, cons
   if (st == BGTQ_OK) st = contiguous("decode_step_multi", cache, capacity, &c);
   if (st != BGTQ_OK) return st;
   if (n_new < 1) return fail(BGTQ_ERR_INVALID, "decode_step_multi: n_new must be >= 1");
-  return step_impl(L, "decode_step_multi", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new, c,
+  return step_impl(L->dev, "decode_step_multi", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new, c,
                    seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -521,7 +521,7 @@ bgtq_status bgtq_decode_step_multi_paged(const bgtq_layout* L, const void* k_new
   if (st == BGTQ_OK) st = paged("decode_step_multi_paged", pool, num_pages, block_table_dev, max_pages, &c);
   if (st != BGTQ_OK) return st;
   if (n_new < 1) return fail(BGTQ_ERR_INVALID, "decode_step_multi_paged: n_new must be >= 1");
-  return step_impl(L, "decode_step_multi_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new,
+  return step_impl(L->dev, "decode_step_multi_paged", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, h_kv, n_new,
                    c, seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream);
 }
 
@@ -691,6 +691,19 @@ bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* S, const void* q, in
   if (st != BGTQ_OK) return st;
   return scores_impl(S->head0, "decode_scores_heads", q, q_dtype, batch, h_q, S->n, cache, seq_lens_dev, capacity,
                      max_seq_len, softmax_scale, scores, scores_ld, workspace, workspace_bytes, stream, S->heads);
+}
+
+bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* S, const void* k_new, const void* v_new, int kv_dtype,
+                                   int n_new, const void* q, int q_dtype, int batch, int h_q, void* cache,
+                                   const int* seq_lens_dev, long long capacity, long long max_seq_len,
+                                   float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  CacheRef c;
+  bgtq_status st = check_set(S, "decode_step_heads");
+  if (st == BGTQ_OK) st = contiguous("decode_step_heads", cache, capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return step_impl(S->head0, "decode_step_heads", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, S->n, 1, c,
+                   seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, S->heads);
 }
 
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* S, unsigned* flags, int clear) {

@@ -1289,9 +1289,11 @@ __global__ void __launch_bounds__(kPrepThreads) qprep_kernel(DevLayout L, const 
 }
 
 // First kernel of a decode step: blocks [0, n_enc) append the new tokens (four blocks per
-// token and KV head), the others prepare q' of one unit each.
-template <bool NC>
-__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const void* __restrict__ k,
+// token and KV head), the others prepare q' of one unit each. PH: heads[h] is the layout of
+// KV head h (else L for every head).
+template <bool NC, bool PH>
+__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, const DevLayout* __restrict__ heads,
+                                                                 const void* __restrict__ k,
                                                                  const void* __restrict__ v, int kv_dtype, int n_new,
                                                                  int batch, const int* __restrict__ seq_lens_before,
                                                                  CacheRef cache,
@@ -1307,10 +1309,17 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(DevLayout L, co
     const int t = rest % n_new;
     rest /= n_new;
     const int b = rest % batch, h = rest / batch;
-    enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
+    if constexpr (PH)
+      enc::encode_token_part<NC>(heads[h], k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
+    else
+      enc::encode_token_part<NC>(L, k, v, kv_dtype, n_new, h_kv, seq_lens_before, cache, t, part, b, h);
   } else if (e - n_enc < batch * h_kv * ((Gt + kMaxG - 1) / kMaxG)) {  // (a cluster launch pads the grid)
     const int u = e - n_enc;
-    prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
+    if constexpr (PH)
+      prep_unit(heads[unit_head(u, h_kv, Gt)], q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u,
+                qfrag + (size_t)u * kQfragWords);
+    else
+      prep_unit(L, q, q_dtype, h_q, h_kv, Gt, n_q, qscale, u, qfrag + (size_t)u * kQfragWords);
   }
 }
 
@@ -1528,14 +1537,15 @@ cudaError_t launch_scores(const DevLayout& L, const DecodePlan& plan, const void
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
                                int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
-                               float* out, void* workspace, cudaStream_t stream) {
+                               float* out, void* workspace, cudaStream_t stream, const DevLayout* heads) {
   const int Gt = h_q * n_q / h_kv;
   const long long cache_units = (long long)batch * h_kv;
   const long long units = cache_units * ((Gt + kMaxG - 1) / kMaxG);  // q' units (column tiles)
   const long long n_enc = (long long)n_new * kEncodeParts * cache_units;
   cudaError_t e;
   if (!L.norm_correct) {
-    e = launch_dependent(step_prep_kernel<false>, unsigned(n_enc + units), kPrepThreads, stream, L, k_new,
+    e = launch_dependent(heads ? step_prep_kernel<false, true> : step_prep_kernel<false, false>,
+                         unsigned(n_enc + units), kPrepThreads, stream, L, heads, k_new,
                          v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, Gt, n_q,
                          softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   } else {
@@ -1553,13 +1563,13 @@ cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, step_prep_kernel<true>, L, k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache,
-                           q, q_dtype, h_q, h_kv, Gt, n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace),
-                           int(n_enc));
+    e = cudaLaunchKernelEx(&cfg, heads ? step_prep_kernel<true, true> : step_prep_kernel<true, false>, L, heads,
+                           k_new, v_new, kv_dtype, n_new, batch, seq_lens_before, cache, q, q_dtype, h_q, h_kv, Gt,
+                           n_q, softmax_scale * kLog2e, static_cast<unsigned*>(workspace), int(n_enc));
   }
   if (e != cudaSuccess) return e;
   return launch_attention(L, plan, batch, h_q, h_kv, n_q, cache, seq_lens_before, out, workspace, n_new,
-                          n_new > 0, stream);
+                          n_new > 0, stream, nullptr, 0, nullptr, heads);
 }
 
 }  // namespace bgtq

@@ -49,7 +49,7 @@ cudaError_t launch_merge_records(const DevLayout& L, const float* recs, int n_re
 cudaError_t launch_decode_step(const DevLayout& L, const DecodePlan& plan, const void* k_new, const void* v_new,
                                int kv_dtype, int n_new, const int* seq_lens_before, const void* q, int q_dtype,
                                int batch, int h_q, int h_kv, int n_q, const CacheRef& cache, float softmax_scale,
-                               float* out, void* workspace, cudaStream_t stream);
+                               float* out, void* workspace, cudaStream_t stream, const DevLayout* heads = nullptr);
 
 // Logits only: scores[(b h_q + hq) scores_ld + t] = softmax_scale q . k_hat_t for every
 // cached token t < seq_lens[b] (the q-preparation kernel, then the split kernel in its

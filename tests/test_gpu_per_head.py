@@ -127,3 +127,46 @@ def test_layout_set_rejects_mixed_layouts():
         assert e.value.status == B.ERR_INVALID
     with pytest.raises(B.BgtqError):
         B.LayoutSet([a, B.Layout(np.full(64, 2), 2, 0)])   # not uploaded
+
+
+@pytest.mark.parametrize("n_new", [1, 5])
+def test_layout_set_step_equals_append_then_attend(n_new):
+    """bgtq_decode_step_heads: the fused append + attend over a layout set gives the cache
+    bytes and outputs of encode_append_heads followed by decode_attention_heads, and each
+    head's outputs match the oracle over the grown rows."""
+    case = Case(16, 4, 2, 400, 2, 2, torch.bfloat16, 5e5, 63, capacity=448)
+    m = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, case.seed + 1, case.theta)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2)
+    q, k, v = synth.make_cache_inputs(m, case.batch, case.length, case.seed, case.theta, case.dtype)
+    layouts = [B.Layout(rates[h], case.v_bits, case.seed).upload(0) for h in range(case.h_kv)]
+    S = B.LayoutSet(layouts)
+    pre = case.length - n_new
+    kd, vd = k.cuda(), v.cuda()
+    base = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    B.encode_append_heads(S, kd[:, :pre].contiguous(), vd[:, :pre].contiguous(),
+                          torch.zeros(case.batch, dtype=torch.int32, device="cuda"), base, case.cap)
+    lens0 = torch.full((case.batch,), pre, dtype=torch.int32, device="cuda")
+    k_new, v_new = kd[:, pre:].contiguous(), vd[:, pre:].contiguous()
+    ws = torch.empty(B.workspace_bytes(layouts[0], case.batch, case.h_q, case.h_kv, case.length), dtype=torch.uint8,
+                     device="cuda")
+    c_sep, c_fus = base.clone(), base.clone()
+    o_sep = torch.empty(case.batch, case.h_q, 128, device="cuda")
+    o_fus = torch.empty_like(o_sep)
+    B.encode_append_heads(S, k_new, v_new, lens0, c_sep, case.cap)
+    B.decode_attention_heads(S, q.cuda(), c_sep, lens0 + n_new, case.cap, case.length, o_sep, ws)
+    B.decode_step_heads(S, k_new, v_new, q.cuda(), c_fus, lens0, case.cap, case.length, o_fus, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    assert torch.equal(c_sep, c_fus)
+    assert torch.equal(o_sep, o_fus)
+    G = case.h_q // case.h_kv
+    got = o_fus.cpu().double().numpy()
+    for h in range(case.h_kv):
+        olay = O.make_layout(rates[h], case.v_bits, case.seed)
+        for b in range(case.batch):
+            enc = O.encode(olay, k[b, :, h].double().numpy(), v[b, :, h].double().numpy())
+            ref = O.decode_attention(olay, q[b, h * G:(h + 1) * G].double().numpy(), O.pack(olay, enc, case.cap),
+                                     case.length, 1 / math.sqrt(128))
+            for i in range(G):
+                assert rel_l2(got[b, h * G + i], ref[i]) <= ATTN_REL_L2, (h, b, i)
