@@ -379,6 +379,20 @@ bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* set, const void* k_new
                                    void* cache, const int* seq_lens_dev, long long capacity,
                                    long long max_seq_len, float softmax_scale, float* out, void* workspace,
                                    size_t workspace_bytes, void* stream);
+/* Paged caches of a layout set: a page holds the h_kv tiles of one 64-token span of one
+ * row at the set's tile stride (-1 on bad arguments); the encode and attention calls take
+ * the pool and block table as bgtq_encode_append_paged / bgtq_decode_attention_paged. */
+long long bgtq_layout_set_paged_pool_bytes(const bgtq_layout_set* set, long long num_pages);
+bgtq_status bgtq_encode_append_paged_heads(const bgtq_layout_set* set, const void* k, const void* v, int dtype,
+                                           int batch, int n_new, const int* seq_lens_dev, void* pool,
+                                           long long num_pages, const int* block_table_dev, long long max_pages,
+                                           void* stream);
+bgtq_status bgtq_decode_attention_paged_heads(const bgtq_layout_set* set, const void* q, int q_dtype,
+                                              int batch, int h_q, const void* pool, long long num_pages,
+                                              const int* block_table_dev, long long max_pages,
+                                              const int* seq_lens_dev, long long max_seq_len,
+                                              float softmax_scale, float* out, void* workspace,
+                                              size_t workspace_bytes, void* stream);
 /* The set's status bits (BGTQ_STATUS_*), as bgtq_device_status. */
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* set, unsigned* flags, int clear);
 

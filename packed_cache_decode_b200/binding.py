@@ -35,7 +35,8 @@ EXPORTED = [
     "bgtq_block_energy_heads", "bgtq_decode_attention_partial", "bgtq_merge_partials",
     "bgtq_layout_set_create", "bgtq_layout_set_destroy", "bgtq_layout_set_tile_bytes", "bgtq_layout_set_cache_bytes",
     "bgtq_encode_append_heads", "bgtq_decode_attention_heads", "bgtq_decode_scores_heads", "bgtq_layout_set_status",
-    "bgtq_decode_step_heads",
+    "bgtq_decode_step_heads", "bgtq_layout_set_paged_pool_bytes", "bgtq_encode_append_paged_heads",
+    "bgtq_decode_attention_paged_heads",
 ]
 
 
@@ -103,6 +104,9 @@ def load():
         "bgtq_decode_scores_heads": (I, [P, P, I, I, I, P, P, LL, LL, F, P, LL, P, C.c_size_t, P]),
         "bgtq_layout_set_status": (I, [P, C.POINTER(C.c_uint), I]),
         "bgtq_decode_step_heads": (I, [P, P, P, I, I, P, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_layout_set_paged_pool_bytes": (LL, [P, LL]),
+        "bgtq_encode_append_paged_heads": (I, [P, P, P, I, I, I, P, P, LL, P, LL, P]),
+        "bgtq_decode_attention_paged_heads": (I, [P, P, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -268,6 +272,12 @@ class LayoutSet:
         n = load().bgtq_layout_set_cache_bytes(self._h, batch, capacity)
         if n == 0:
             _check(ERR_INVALID, "layout_set_cache_bytes")
+        return int(n)
+
+    def paged_pool_bytes(self, num_pages: int) -> int:
+        n = load().bgtq_layout_set_paged_pool_bytes(self._h, num_pages)
+        if n < 0:
+            _check(ERR_INVALID, "layout_set_paged_pool_bytes")
         return int(n)
 
     def status(self, clear: bool = True) -> int:
@@ -592,3 +602,31 @@ def decode_step_heads(layouts: LayoutSet, k_new, v_new, q, cache, seq_lens, capa
                                          capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
                                          C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream)),
            "decode_step_heads")
+
+
+def encode_append_paged_heads(layouts: LayoutSet, k, v, seq_lens, pc, stream=None):
+    """encode_append_heads into a paged cache pc (a PagedCache over a pool of the set's pages)."""
+    B_, n_new, h_kv, d = k.shape
+    assert d == HEAD_DIM and h_kv == layouts.h_kv and k.is_contiguous() and v.is_contiguous()
+    _check(load().bgtq_encode_append_paged_heads(layouts.handle, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()),
+                                                 dtype_code(k), B_, n_new, C.c_void_p(seq_lens.data_ptr()),
+                                                 C.c_void_p(pc.pool.data_ptr()),
+                                                 pc.pool.numel() // (layouts.h_kv * layouts.tile_bytes),
+                                                 C.c_void_p(pc.table.data_ptr()), pc.max_pages, _stream_ptr(stream)),
+           "encode_append_paged_heads")
+
+
+def decode_attention_paged_heads(layouts: LayoutSet, q, pc, seq_lens, max_seq_len: int, out, workspace,
+                                 softmax_scale: float | None = None, stream=None):
+    """decode_attention_heads over a paged cache pc."""
+    B_, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_paged_heads(layouts.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, h_q,
+                                                    C.c_void_p(pc.pool.data_ptr()),
+                                                    pc.pool.numel() // (layouts.h_kv * layouts.tile_bytes),
+                                                    C.c_void_p(pc.table.data_ptr()), pc.max_pages,
+                                                    C.c_void_p(seq_lens.data_ptr()), max_seq_len, scale,
+                                                    C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                                    workspace.numel(), _stream_ptr(stream)),
+           "decode_attention_paged_heads")

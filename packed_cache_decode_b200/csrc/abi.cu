@@ -706,6 +706,40 @@ bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* S, const void* k_new, 
                    seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, S->heads);
 }
 
+long long bgtq_layout_set_paged_pool_bytes(const bgtq_layout_set* S, long long num_pages) {
+  if (!S || num_pages < 0) {
+    set_error("layout_set_paged_pool_bytes: bad arguments");
+    return -1;
+  }
+  return num_pages * S->n * (long long)S->tile_stride;
+}
+
+bgtq_status bgtq_encode_append_paged_heads(const bgtq_layout_set* S, const void* k, const void* v, int dtype,
+                                           int batch, int n_new, const int* seq_lens_dev, void* pool,
+                                           long long num_pages, const int* block_table_dev, long long max_pages,
+                                           void* stream) {
+  CacheRef c{};
+  bgtq_status st = check_set(S, "encode_append_paged_heads");
+  if (st == BGTQ_OK) st = paged("encode_append_paged_heads", pool, num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return encode_impl(S->head0, "encode_append_paged_heads", k, v, dtype, batch, n_new, S->n, seq_lens_dev, c, stream,
+                     S->heads);
+}
+
+bgtq_status bgtq_decode_attention_paged_heads(const bgtq_layout_set* S, const void* q, int q_dtype, int batch,
+                                              int h_q, const void* pool, long long num_pages,
+                                              const int* block_table_dev, long long max_pages,
+                                              const int* seq_lens_dev, long long max_seq_len, float softmax_scale,
+                                              float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  CacheRef c{};
+  bgtq_status st = check_set(S, "decode_attention_paged_heads");
+  if (st == BGTQ_OK)
+    st = paged("decode_attention_paged_heads", const_cast<void*>(pool), num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(S->head0, "decode_attention_paged_heads", q, q_dtype, batch, h_q, S->n, 1, c, seq_lens_dev,
+                     max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, nullptr, S->heads);
+}
+
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* S, unsigned* flags, int clear) {
   bgtq_status st = check_set(S, "layout_set_status");
   if (st != BGTQ_OK) return st;

@@ -170,3 +170,44 @@ def test_layout_set_step_equals_append_then_attend(n_new):
                                      case.length, 1 / math.sqrt(128))
             for i in range(G):
                 assert rel_l2(got[b, h * G + i], ref[i]) <= ATTN_REL_L2, (h, b, i)
+
+
+def test_layout_set_paged_equals_contiguous():
+    """A layout set over a paged cache (pages handed out in shuffled order): the same tiles
+    as the contiguous layout-set cache, byte for byte, and the same outputs, bit for bit."""
+    case = Case(16, 4, 2, 300, 2, 2, torch.bfloat16, 5e5, 64)
+    m = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, case.seed + 1, case.theta)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2)
+    q, k, v = synth.make_cache_inputs(m, case.batch, case.length, case.seed, case.theta, case.dtype)
+    layouts = [B.Layout(rates[h], case.v_bits, case.seed).upload(0) for h in range(case.h_kv)]
+    S = B.LayoutSet(layouts)
+    n_tiles = case.cap // 64
+    num_pages = case.batch * n_tiles + 3
+    perm = np.random.default_rng(5).permutation(num_pages)[:case.batch * n_tiles].astype(np.int32)
+    pc = B.PagedCache(torch.zeros(S.paged_pool_bytes(num_pages), dtype=torch.uint8, device="cuda"),
+                      torch.from_numpy(perm.reshape(case.batch, n_tiles)).cuda())
+    cont = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    kd, vd = k.cuda(), v.cuda()
+    for a0, a1 in ((0, 250), (250, 252), (252, 300)):
+        lens0 = torch.full((case.batch,), a0, dtype=torch.int32, device="cuda")
+        B.encode_append_heads(S, kd[:, a0:a1].contiguous(), vd[:, a0:a1].contiguous(), lens0, cont, case.cap)
+        B.encode_append_paged_heads(S, kd[:, a0:a1].contiguous(), vd[:, a0:a1].contiguous(), lens0, pc)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    tb = S.tile_bytes
+    pv = pc.pool.view(num_pages, case.h_kv, tb)
+    cv = cont.view(case.batch, case.h_kv, n_tiles, tb)
+    for b in range(case.batch):
+        for i in range(n_tiles):
+            assert torch.equal(pv[int(perm[b * n_tiles + i])], cv[b, :, i]), (b, i)
+    lens = torch.tensor([300, 241], dtype=torch.int32, device="cuda")
+    ws = torch.empty(B.workspace_bytes(layouts[0], case.batch, case.h_q, case.h_kv, case.length), dtype=torch.uint8,
+                     device="cuda")
+    o1 = torch.empty(case.batch, case.h_q, 128, device="cuda")
+    o2 = torch.empty_like(o1)
+    B.decode_attention_heads(S, q.cuda(), cont, lens, case.cap, case.length, o1, ws)
+    B.decode_attention_paged_heads(S, q.cuda(), pc, lens, case.length, o2, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    assert torch.equal(o1, o2)
