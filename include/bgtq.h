@@ -363,6 +363,14 @@ bgtq_status bgtq_decode_attention_heads(const bgtq_layout_set* set, const void* 
                                         int h_q, const void* cache, const int* seq_lens_dev,
                                         long long capacity, long long max_seq_len, float softmax_scale,
                                         float* out, void* workspace, size_t workspace_bytes, void* stream);
+/* bgtq_decode_attention_multi over a cache written by bgtq_encode_append_heads (n_q query
+ * tokens per row, causal among them; h_kv = the set's size; workspace as
+ * bgtq_decode_attention_multi). */
+bgtq_status bgtq_decode_attention_multi_heads(const bgtq_layout_set* set, const void* q, int q_dtype,
+                                              int batch, int n_q, int h_q, const void* cache,
+                                              const int* seq_lens_dev, long long capacity,
+                                              long long max_seq_len, float softmax_scale, float* out,
+                                              void* workspace, size_t workspace_bytes, void* stream);
 /* bgtq_decode_scores over a cache written by bgtq_encode_append_heads (h_kv = the set's
  * size). */
 bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* set, const void* q, int q_dtype, int batch,

@@ -36,7 +36,7 @@ EXPORTED = [
     "bgtq_layout_set_create", "bgtq_layout_set_destroy", "bgtq_layout_set_tile_bytes", "bgtq_layout_set_cache_bytes",
     "bgtq_encode_append_heads", "bgtq_decode_attention_heads", "bgtq_decode_scores_heads", "bgtq_layout_set_status",
     "bgtq_decode_step_heads", "bgtq_layout_set_paged_pool_bytes", "bgtq_encode_append_paged_heads",
-    "bgtq_decode_attention_paged_heads",
+    "bgtq_decode_attention_paged_heads", "bgtq_decode_attention_multi_heads",
 ]
 
 
@@ -107,6 +107,7 @@ def load():
         "bgtq_layout_set_paged_pool_bytes": (LL, [P, LL]),
         "bgtq_encode_append_paged_heads": (I, [P, P, P, I, I, I, P, P, LL, P, LL, P]),
         "bgtq_decode_attention_paged_heads": (I, [P, P, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_attention_multi_heads": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -630,3 +631,18 @@ def decode_attention_paged_heads(layouts: LayoutSet, q, pc, seq_lens, max_seq_le
                                                     C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
                                                     workspace.numel(), _stream_ptr(stream)),
            "decode_attention_paged_heads")
+
+
+def decode_attention_multi_heads(layouts: LayoutSet, q, cache, seq_lens, capacity: int, max_seq_len: int, out,
+                                 workspace, softmax_scale: float | None = None, stream=None):
+    """decode_attention_multi over a layout set's cache: q [B, n_q, h_q, 128] CUDA (the last
+    n_q of each row's cached tokens), out [B, n_q, h_q, 128] fp32."""
+    B_, n_q, h_q, d = q.shape
+    assert d == HEAD_DIM and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_attention_multi_heads(layouts.handle, C.c_void_p(q.data_ptr()), dtype_code(q), B_, n_q,
+                                                    h_q, C.c_void_p(cache.data_ptr()),
+                                                    C.c_void_p(seq_lens.data_ptr()), capacity, max_seq_len, scale,
+                                                    C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                                    workspace.numel(), _stream_ptr(stream)),
+           "decode_attention_multi_heads")

@@ -683,6 +683,18 @@ bgtq_status bgtq_decode_attention_heads(const bgtq_layout_set* S, const void* q,
                      max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, nullptr, S->heads);
 }
 
+bgtq_status bgtq_decode_attention_multi_heads(const bgtq_layout_set* S, const void* q, int q_dtype, int batch,
+                                              int n_q, int h_q, const void* cache, const int* seq_lens_dev,
+                                              long long capacity, long long max_seq_len, float softmax_scale,
+                                              float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  CacheRef c;
+  bgtq_status st = check_set(S, "decode_attention_multi_heads");
+  if (st == BGTQ_OK) st = contiguous("decode_attention_multi_heads", const_cast<void*>(cache), capacity, &c);
+  if (st != BGTQ_OK) return st;
+  return decode_impl(S->head0, "decode_attention_multi_heads", q, q_dtype, batch, h_q, S->n, n_q, c, seq_lens_dev,
+                     max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, nullptr, S->heads);
+}
+
 bgtq_status bgtq_decode_scores_heads(const bgtq_layout_set* S, const void* q, int q_dtype, int batch, int h_q,
                                      const void* cache, const int* seq_lens_dev, long long capacity,
                                      long long max_seq_len, float softmax_scale, float* scores, long long scores_ld,

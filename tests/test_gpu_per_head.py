@@ -211,3 +211,46 @@ def test_layout_set_paged_equals_contiguous():
     torch.cuda.synchronize()
     assert S.status() == 0
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("shape", [(16, 4, 2), (12, 4, 3), (32, 2, 2)], ids=["gqa4_nq2", "gqa3_nq3", "gqa16_nq2_32cols"])
+def test_layout_set_multi_token_matches_oracle(shape):
+    """decode_attention_multi_heads: n_q query tokens per row (causal among them) over a
+    layout set, each KV head against the oracle's multi-token attention with its own layout."""
+    h_q, h_kv, n_q = shape
+    case = Case(h_q, h_kv, 2, 400, 2, 2, torch.float16, 5e5, 65)
+    m = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, case.seed + 1, case.theta)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2, min_rate=0)
+    _, k, v = synth.make_cache_inputs(m, case.batch, case.length, case.seed, case.theta, case.dtype)
+    layouts = [B.Layout(rates[h], case.v_bits, case.seed).upload(0) for h in range(h_kv)]
+    S = B.LayoutSet(layouts)
+    cache = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    B.encode_append_heads(S, k.cuda(), v.cuda(), torch.zeros(case.batch, dtype=torch.int32, device="cuda"), cache,
+                          case.cap)
+    lens = torch.tensor([400, 317], dtype=torch.int32)
+    q = torch.empty(case.batch, n_q, h_q, 128, dtype=case.dtype)
+    for b in range(case.batch):
+        for hq in range(h_q):
+            q[b, :, hq] = synth.query_slice(m, b, hq, n_q, int(lens[b]) - n_q, case.seed, case.theta).to(case.dtype)
+    ws = torch.empty(B.workspace_bytes(layouts[0], case.batch, h_q * n_q, h_kv, case.length), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full((case.batch, n_q, h_q, 128), float("nan"), device="cuda")
+    B.decode_attention_multi_heads(S, q.cuda(), cache, lens.cuda(), case.cap, case.length, out, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    G = h_q // h_kv
+    n_tiles = case.cap // 64
+    cv = cache.view(case.batch, h_kv, n_tiles, S.tile_bytes).cpu().numpy()
+    got = out.cpu().double().numpy()
+    for h in range(h_kv):
+        olay = O.make_layout(rates[h], case.v_bits, case.seed)
+        for b in range(case.batch):
+            enc = O.encode(olay, k[b, :, h].double().numpy(), v[b, :, h].double().numpy())
+            want = O.pack(olay, enc, case.cap)
+            compare_packed(olay, enc, want, np.ascontiguousarray(cv[b, h, :, :olay.tile_bytes]).reshape(-1), case.cap)
+            ref = O.decode_attention_multi(olay, q[b, :, h * G:(h + 1) * G].double().numpy(), want, int(lens[b]),
+                                           1 / math.sqrt(128))
+            for j in range(n_q):
+                for c in range(G):
+                    assert rel_l2(got[b, j, h * G + c], ref[j, c]) <= ATTN_REL_L2, (h, b, j, c)
