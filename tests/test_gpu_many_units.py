@@ -6,7 +6,6 @@ tokens per row (12 columns per KV head: two column tiles, twice the units), and 
 set (one layout per KV head, a head change at most segment starts)."""
 import math
 
-import numpy as np
 import pytest
 import torch
 
@@ -97,3 +96,27 @@ def test_many_units_layout_set_match_oracle():
                                      1 / math.sqrt(128))
             for c in range(G):
                 assert rel_l2(got[b, h * G + c], ref[c]) <= ATTN_REL_L2, (b, h, c)
+
+
+def test_many_units_step_equals_append_then_attend(single_layout):
+    """bgtq_decode_step over the 320 units (one new token per row at a ragged position):
+    the cache bytes and outputs of encode_append followed by decode_attention, bit for bit
+    (both of those are checked against the oracle above)."""
+    case, model, lay, cache, olay, packed = single_layout
+    gen = torch.Generator().manual_seed(83)
+    lens0 = (_lens(1) - 1).cuda()  # rows of 0 .. 99 tokens before the step
+    k_new = torch.randn(BATCH, 1, H_KV, 128, generator=gen).to(case.dtype).cuda()
+    v_new = torch.randn(BATCH, 1, H_KV, 128, generator=gen).to(case.dtype).cuda()
+    q = torch.randn(BATCH, H_Q, 128, generator=gen).to(case.dtype).cuda()
+    ws = torch.empty(B.workspace_bytes(lay, BATCH, H_Q, H_KV, LENGTH), dtype=torch.uint8, device="cuda")
+    c_sep, c_fus = cache.clone(), cache.clone()
+    o_sep = torch.empty(BATCH, H_Q, 128, device="cuda")
+    o_fus = torch.empty_like(o_sep)
+    B.encode_append(lay, k_new, v_new, lens0, c_sep, CAP)
+    B.decode_attention(lay, q, c_sep, lens0 + 1, CAP, LENGTH, o_sep, ws, H_KV)
+    B.decode_step(lay, k_new, v_new, q, c_fus, lens0, CAP, LENGTH, o_fus, ws)
+    torch.cuda.synchronize()
+    assert lay.status() == 0
+    assert torch.equal(c_sep, c_fus)
+    assert torch.equal(o_sep, o_fus)
+    assert not torch.isnan(o_fus).any()
