@@ -387,6 +387,16 @@ bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* set, const void* k_new
                                    void* cache, const int* seq_lens_dev, long long capacity,
                                    long long max_seq_len, float softmax_scale, float* out, void* workspace,
                                    size_t workspace_bytes, void* stream);
+/* bgtq_decode_step_multi over a cache written by bgtq_encode_append_heads: appends n_new
+ * >= 1 tokens per row and attends each new token's own queries (q [batch][n_new][h_q][128],
+ * out likewise, causal among the new tokens) over the grown cache, every KV head with its
+ * own layout (h_kv = the set's size). Workspace: bgtq_workspace_bytes(any layout of the
+ * set, batch, h_q * n_new, h_kv, max_seq_len). Errors as bgtq_decode_step_multi. */
+bgtq_status bgtq_decode_step_multi_heads(const bgtq_layout_set* set, const void* k_new, const void* v_new,
+                                         int kv_dtype, int n_new, const void* q, int q_dtype, int batch,
+                                         int h_q, void* cache, const int* seq_lens_dev, long long capacity,
+                                         long long max_seq_len, float softmax_scale, float* out,
+                                         void* workspace, size_t workspace_bytes, void* stream);
 /* Paged caches of a layout set: a page holds the h_kv tiles of one 64-token span of one
  * row at the set's tile stride (-1 on bad arguments); the encode and attention calls take
  * the pool and block table as bgtq_encode_append_paged / bgtq_decode_attention_paged. */
@@ -401,6 +411,14 @@ bgtq_status bgtq_decode_attention_paged_heads(const bgtq_layout_set* set, const 
                                               const int* seq_lens_dev, long long max_seq_len,
                                               float softmax_scale, float* out, void* workspace,
                                               size_t workspace_bytes, void* stream);
+/* bgtq_decode_step_heads over a paged cache of the set (pool and block table as
+ * bgtq_decode_step_paged). */
+bgtq_status bgtq_decode_step_paged_heads(const bgtq_layout_set* set, const void* k_new, const void* v_new,
+                                         int kv_dtype, int n_new, const void* q, int q_dtype, int batch,
+                                         int h_q, void* pool, long long num_pages, const int* block_table_dev,
+                                         long long max_pages, const int* seq_lens_dev, long long max_seq_len,
+                                         float softmax_scale, float* out, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 /* The set's status bits (BGTQ_STATUS_*), as bgtq_device_status. */
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* set, unsigned* flags, int clear);
 

@@ -36,7 +36,8 @@ EXPORTED = [
     "bgtq_layout_set_create", "bgtq_layout_set_destroy", "bgtq_layout_set_tile_bytes", "bgtq_layout_set_cache_bytes",
     "bgtq_encode_append_heads", "bgtq_decode_attention_heads", "bgtq_decode_scores_heads", "bgtq_layout_set_status",
     "bgtq_decode_step_heads", "bgtq_layout_set_paged_pool_bytes", "bgtq_encode_append_paged_heads",
-    "bgtq_decode_attention_paged_heads", "bgtq_decode_attention_multi_heads",
+    "bgtq_decode_attention_paged_heads", "bgtq_decode_attention_multi_heads", "bgtq_decode_step_multi_heads",
+    "bgtq_decode_step_paged_heads",
 ]
 
 
@@ -108,6 +109,9 @@ def load():
         "bgtq_encode_append_paged_heads": (I, [P, P, P, I, I, I, P, P, LL, P, LL, P]),
         "bgtq_decode_attention_paged_heads": (I, [P, P, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t, P]),
         "bgtq_decode_attention_multi_heads": (I, [P, P, I, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_step_multi_heads": (I, [P, P, P, I, I, P, I, I, I, P, P, LL, LL, F, P, P, C.c_size_t, P]),
+        "bgtq_decode_step_paged_heads": (I, [P, P, P, I, I, P, I, I, I, P, LL, P, LL, P, LL, F, P, P, C.c_size_t,
+                                             P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -646,3 +650,41 @@ def decode_attention_multi_heads(layouts: LayoutSet, q, cache, seq_lens, capacit
                                                     C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
                                                     workspace.numel(), _stream_ptr(stream)),
            "decode_attention_multi_heads")
+
+
+def decode_step_multi_heads(layouts: LayoutSet, k_new, v_new, q, cache, seq_lens, capacity: int, max_seq_len: int,
+                            out, workspace, softmax_scale: float | None = None, stream=None):
+    """decode_step_multi over a layout set's cache: append k_new, v_new [B, n_new, h_kv, 128]
+    at seq_lens[b] and attend q [B, n_new, h_q, 128] (the new tokens' queries, causal among
+    them); out [B, n_new, h_q, 128] fp32."""
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and h_kv == layouts.h_kv and k_new.is_contiguous() and v_new.is_contiguous()
+    assert q.shape[:2] == (B_, n_new) and q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_multi_heads(layouts.handle, C.c_void_p(k_new.data_ptr()),
+                                               C.c_void_p(v_new.data_ptr()), dtype_code(k_new), n_new,
+                                               C.c_void_p(q.data_ptr()), dtype_code(q), B_, q.shape[2],
+                                               C.c_void_p(cache.data_ptr()), C.c_void_p(seq_lens.data_ptr()),
+                                               capacity, max_seq_len, scale, C.c_void_p(out.data_ptr()),
+                                               C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                               _stream_ptr(stream)),
+           "decode_step_multi_heads")
+
+
+def decode_step_paged_heads(layouts: LayoutSet, k_new, v_new, q, pc, seq_lens, max_seq_len: int, out, workspace,
+                            softmax_scale: float | None = None, stream=None):
+    """decode_step_heads over a paged cache pc (a PagedCache over a pool of the set's pages)."""
+    B_, n_new, h_kv, d = k_new.shape
+    assert d == HEAD_DIM and h_kv == layouts.h_kv and k_new.is_contiguous() and v_new.is_contiguous()
+    assert q.is_contiguous() and out.is_contiguous()
+    scale = 1.0 / HEAD_DIM ** 0.5 if softmax_scale is None else float(softmax_scale)
+    _check(load().bgtq_decode_step_paged_heads(layouts.handle, C.c_void_p(k_new.data_ptr()),
+                                               C.c_void_p(v_new.data_ptr()), dtype_code(k_new), n_new,
+                                               C.c_void_p(q.data_ptr()), dtype_code(q), B_, q.shape[1],
+                                               C.c_void_p(pc.pool.data_ptr()),
+                                               pc.pool.numel() // (layouts.h_kv * layouts.tile_bytes),
+                                               C.c_void_p(pc.table.data_ptr()), pc.max_pages,
+                                               C.c_void_p(seq_lens.data_ptr()), max_seq_len, scale,
+                                               C.c_void_p(out.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                               workspace.numel(), _stream_ptr(stream)),
+           "decode_step_paged_heads")

@@ -718,6 +718,21 @@ bgtq_status bgtq_decode_step_heads(const bgtq_layout_set* S, const void* k_new, 
                    seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, S->heads);
 }
 
+bgtq_status bgtq_decode_step_multi_heads(const bgtq_layout_set* S, const void* k_new, const void* v_new,
+                                         int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,
+                                         void* cache, const int* seq_lens_dev, long long capacity,
+                                         long long max_seq_len, float softmax_scale, float* out, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  CacheRef c;
+  bgtq_status st = check_set(S, "decode_step_multi_heads");
+  if (st == BGTQ_OK) st = contiguous("decode_step_multi_heads", cache, capacity, &c);
+  if (st != BGTQ_OK) return st;
+  if (n_new < 1) return fail(BGTQ_ERR_INVALID, "decode_step_multi_heads: n_new must be >= 1");
+  return step_impl(S->head0, "decode_step_multi_heads", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, S->n,
+                   n_new, c, seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream,
+                   S->heads);
+}
+
 long long bgtq_layout_set_paged_pool_bytes(const bgtq_layout_set* S, long long num_pages) {
   if (!S || num_pages < 0) {
     set_error("layout_set_paged_pool_bytes: bad arguments");
@@ -750,6 +765,20 @@ bgtq_status bgtq_decode_attention_paged_heads(const bgtq_layout_set* S, const vo
   if (st != BGTQ_OK) return st;
   return decode_impl(S->head0, "decode_attention_paged_heads", q, q_dtype, batch, h_q, S->n, 1, c, seq_lens_dev,
                      max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, nullptr, S->heads);
+}
+
+bgtq_status bgtq_decode_step_paged_heads(const bgtq_layout_set* S, const void* k_new, const void* v_new,
+                                         int kv_dtype, int n_new, const void* q, int q_dtype, int batch, int h_q,
+                                         void* pool, long long num_pages, const int* block_table_dev,
+                                         long long max_pages, const int* seq_lens_dev, long long max_seq_len,
+                                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  CacheRef c{};
+  bgtq_status st = check_set(S, "decode_step_paged_heads");
+  if (st == BGTQ_OK) st = paged("decode_step_paged_heads", pool, num_pages, block_table_dev, max_pages, &c);
+  if (st != BGTQ_OK) return st;
+  return step_impl(S->head0, "decode_step_paged_heads", k_new, v_new, kv_dtype, n_new, q, q_dtype, batch, h_q, S->n,
+                   1, c, seq_lens_dev, max_seq_len, softmax_scale, out, workspace, workspace_bytes, stream, S->heads);
 }
 
 bgtq_status bgtq_layout_set_status(const bgtq_layout_set* S, unsigned* flags, int clear) {

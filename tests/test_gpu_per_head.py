@@ -254,3 +254,76 @@ def test_layout_set_multi_token_matches_oracle(shape):
             for j in range(n_q):
                 for c in range(G):
                     assert rel_l2(got[b, j, h * G + c], ref[j, c]) <= ATTN_REL_L2, (h, b, j, c)
+
+
+def _set_with_prefix(h_q, h_kv, pre, seed, capacity):
+    case = Case(h_q, h_kv, 2, pre + 8, 2, 2, torch.bfloat16, 5e5, seed, capacity=capacity)
+    m = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(m, 256, case.seed + 1, case.theta)
+    rates = B.plan_head_rates(q_cal.numpy(), k_cal.numpy(), 2)
+    _, k, v = synth.make_cache_inputs(m, case.batch, case.length, case.seed, case.theta, case.dtype)
+    S = B.LayoutSet([B.Layout(rates[h], case.v_bits, case.seed).upload(0) for h in range(h_kv)])
+    return case, S, k.cuda(), v.cuda()
+
+
+@pytest.mark.parametrize("n_new", [2, 3])
+def test_layout_set_multi_step_equals_append_then_attend(n_new):
+    """decode_step_multi_heads: the new tokens' own queries over a layout set (12 columns per
+    KV head at n_new = 3: two column tiles) give the cache bytes and outputs of
+    encode_append_heads followed by decode_attention_multi_heads (oracle-checked above)."""
+    case, S, kd, vd = _set_with_prefix(16, 4, 300, 66, 320)
+    pre = 300
+    base = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    B.encode_append_heads(S, kd[:, :pre].contiguous(), vd[:, :pre].contiguous(),
+                          torch.zeros(case.batch, dtype=torch.int32, device="cuda"), base, case.cap)
+    lens0 = torch.tensor([pre, pre - 37], dtype=torch.int32, device="cuda")
+    k_new, v_new = kd[:, pre:pre + n_new].contiguous(), vd[:, pre:pre + n_new].contiguous()
+    q = torch.randn(case.batch, n_new, case.h_q, 128, generator=torch.Generator().manual_seed(7)).to(case.dtype).cuda()
+    ws = torch.empty(B.workspace_bytes(S.layouts[0], case.batch, case.h_q * n_new, case.h_kv, case.length),
+                     dtype=torch.uint8, device="cuda")
+    c_sep, c_fus = base.clone(), base.clone()
+    o_sep = torch.empty(case.batch, n_new, case.h_q, 128, device="cuda")
+    o_fus = torch.empty_like(o_sep)
+    B.encode_append_heads(S, k_new, v_new, lens0, c_sep, case.cap)
+    B.decode_attention_multi_heads(S, q, c_sep, lens0 + n_new, case.cap, case.length, o_sep, ws)
+    B.decode_step_multi_heads(S, k_new, v_new, q, c_fus, lens0, case.cap, case.length, o_fus, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    assert torch.equal(c_sep, c_fus)
+    assert torch.equal(o_sep, o_fus)
+    assert not torch.isnan(o_fus).any()
+
+
+def test_layout_set_paged_step_equals_contiguous_step():
+    """decode_step_paged_heads on a paged cache (shuffled pages) against decode_step_heads on
+    the contiguous cache: the same tiles byte for byte and the same outputs bit for bit."""
+    case, S, kd, vd = _set_with_prefix(16, 4, 250, 67, 320)
+    pre = 250
+    n_tiles = case.cap // 64
+    num_pages = case.batch * n_tiles + 2
+    perm = np.random.default_rng(9).permutation(num_pages)[:case.batch * n_tiles].astype(np.int32)
+    pc = B.PagedCache(torch.zeros(S.paged_pool_bytes(num_pages), dtype=torch.uint8, device="cuda"),
+                      torch.from_numpy(perm.reshape(case.batch, n_tiles)).cuda())
+    cont = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    zero = torch.zeros(case.batch, dtype=torch.int32, device="cuda")
+    B.encode_append_heads(S, kd[:, :pre].contiguous(), vd[:, :pre].contiguous(), zero, cont, case.cap)
+    B.encode_append_paged_heads(S, kd[:, :pre].contiguous(), vd[:, :pre].contiguous(), zero, pc)
+    lens0 = torch.tensor([pre, 191], dtype=torch.int32, device="cuda")  # 191: the new token opens tile 2
+    k_new, v_new = kd[:, pre:pre + 1].contiguous(), vd[:, pre:pre + 1].contiguous()
+    q = torch.randn(case.batch, case.h_q, 128, generator=torch.Generator().manual_seed(8)).to(case.dtype).cuda()
+    ws = torch.empty(B.workspace_bytes(S.layouts[0], case.batch, case.h_q, case.h_kv, case.length),
+                     dtype=torch.uint8, device="cuda")
+    o1 = torch.empty(case.batch, case.h_q, 128, device="cuda")
+    o2 = torch.empty_like(o1)
+    B.decode_step_heads(S, k_new, v_new, q, cont, lens0, case.cap, case.length, o1, ws)
+    B.decode_step_paged_heads(S, k_new, v_new, q, pc, lens0, case.length, o2, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    tb = S.tile_bytes
+    pv = pc.pool.view(num_pages, case.h_kv, tb)
+    cv = cont.view(case.batch, case.h_kv, n_tiles, tb)
+    for b in range(case.batch):
+        for i in range(n_tiles):
+            assert torch.equal(pv[int(perm[b * n_tiles + i])], cv[b, :, i]), (b, i)
+    assert torch.equal(o1, o2)
+    assert not torch.isnan(o1).any()
