@@ -1,7 +1,7 @@
 """Seeded random shapes through the C ABI against the oracle: query heads per KV head,
 query tokens per row (up to 32 columns per KV head), batch, ragged lengths, key and value
 rates, input dtype, norm correction, fp16 norms, rate-0 blocks, one layout per KV head
-(layout sets), and appends split into
+(layout sets, with one or several query tokens per row), and appends split into
 chunks of random sizes (short appends take the per-token encoder, longer ones the bulk
 encoder; a chunk may start anywhere inside a tile). Every packed (row, KV head) slice is
 compared with the oracle's bytes, every query column's output with the oracle's
@@ -141,3 +141,62 @@ def test_random_layout_set_matches_oracle(i):
             for c in range(G):
                 err = rel_l2(got[b, h * G + c], ref[c])
                 assert err <= ATTN_REL_L2, (case, b, h, c, err)
+
+
+@pytest.mark.parametrize("i", range(5))
+def test_random_layout_set_multi_token_matches_oracle(i):
+    """Random shapes with one layout per KV head and n_q query tokens per row (causal among
+    them, up to 32 columns per KV head) through decode_attention_multi_heads; every column
+    against the oracle's multi-token attention with its head's layout."""
+    rng = np.random.default_rng(9500 + i)
+    while True:
+        G = int(rng.choice([1, 2, 3, 4, 6, 8, 16]))
+        n_q = int(rng.choice([2, 3, 4]))
+        if G * n_q <= 32:
+            break
+    h_kv = int(rng.integers(2, 5))
+    case = Case(G * h_kv, h_kv, int(rng.integers(1, 3)), int(rng.integers(n_q + 40, 400)), int(rng.choice([2, 3])),
+                int(rng.integers(1, 5)), DTYPES[int(rng.integers(0, 3))], 5e5, 300 + i,
+                norm_correct=bool(rng.integers(0, 2)), norm_fp16=bool(rng.integers(0, 2)),
+                min_rate=int(rng.integers(0, 2)))
+    model = synth.make_layer_model(case.h_q, case.h_kv, case.seed)
+    q_cal, k_cal = synth.make_calibration(model, 256, case.seed + 1, case.theta)
+    per = O.block_energy_heads(q_cal.double().numpy(), k_cal.double().numpy())
+    rates = [O.greedy_rates(per[h], O.lloyd_max_mse_table(), case.min_rate, 4, 64 * case.k_bits)
+             for h in range(case.h_kv)]
+    _, k, v = synth.make_cache_inputs(model, case.batch, case.length, case.seed, case.theta, case.dtype)
+    layouts = [B.Layout(rates[h], case.v_bits, case.seed, case.norm_correct, case.norm_fp16).upload(0)
+               for h in range(case.h_kv)]
+    S = B.LayoutSet(layouts)
+    cache = torch.zeros(S.cache_bytes(case.batch, case.cap), dtype=torch.uint8, device="cuda")
+    a = int(rng.integers(1, case.length - 10))
+    kd, vd = k.cuda(), v.cuda()
+    for a0, a1 in ((0, a), (a, case.length)):
+        lens0 = torch.full((case.batch,), a0, dtype=torch.int32, device="cuda")
+        B.encode_append_heads(S, kd[:, a0:a1].contiguous(), vd[:, a0:a1].contiguous(), lens0, cache, case.cap)
+    lens = torch.tensor([max(n_q, case.length - 41 * b) for b in range(case.batch)], dtype=torch.int32)
+    q = torch.empty(case.batch, n_q, case.h_q, 128, dtype=case.dtype)
+    for b in range(case.batch):
+        for hq in range(case.h_q):
+            q[b, :, hq] = synth.query_slice(model, b, hq, n_q, int(lens[b]) - n_q, case.seed, case.theta).to(case.dtype)
+    ws = torch.empty(B.workspace_bytes(layouts[0], case.batch, case.h_q * n_q, case.h_kv, case.length),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.full((case.batch, n_q, case.h_q, 128), float("nan"), device="cuda")
+    B.decode_attention_multi_heads(S, q.cuda(), cache, lens.cuda(), case.cap, case.length, out, ws)
+    torch.cuda.synchronize()
+    assert S.status() == 0
+    n_tiles = case.cap // 64
+    cv = cache.view(case.batch, case.h_kv, n_tiles, S.tile_bytes).cpu().numpy()
+    got = out.cpu().double().numpy()
+    for h in range(case.h_kv):
+        olay = O.make_layout(rates[h], case.v_bits, case.seed, case.norm_correct, case.norm_fp16)
+        for b in range(case.batch):
+            enc = O.encode(olay, k[b, :, h].double().numpy(), v[b, :, h].double().numpy())
+            want = O.pack(olay, enc, case.cap)
+            compare_packed(olay, enc, want, np.ascontiguousarray(cv[b, h, :, :olay.tile_bytes]).reshape(-1), case.cap)
+            ref = O.decode_attention_multi(olay, q[b, :, h * G:(h + 1) * G].double().numpy(), want, int(lens[b]),
+                                           1 / math.sqrt(128))
+            for j in range(n_q):
+                for c in range(G):
+                    err = rel_l2(got[b, j, h * G + c], ref[j, c])
+                    assert err <= ATTN_REL_L2, (case, n_q, b, h, j, c, err)
