@@ -235,4 +235,10 @@ def test_layout_set_refuses_bad_arguments_without_device(lib):
     assert lib.bgtq_encode_append_heads(None, None, None, 0, 1, 1, None, None, 64, None) == B.ERR_INVALID
     assert lib.bgtq_decode_attention_heads(None, None, 0, 1, 1, None, None, 64, 64, 0.1, None, None, 0,
                                            None) == B.ERR_INVALID
+    assert lib.bgtq_decode_attention_multi_heads(None, None, 0, 1, 2, 1, None, None, 64, 64, 0.1, None, None, 0,
+                                                 None) == B.ERR_INVALID
+    assert lib.bgtq_decode_step_multi_heads(None, None, None, 0, 2, None, 0, 1, 1, None, None, 64, 64, 0.1, None,
+                                            None, 0, None) == B.ERR_INVALID
+    assert lib.bgtq_decode_step_paged_heads(None, None, None, 0, 1, None, 0, 1, 1, None, 1, None, 1, None, 64, 0.1,
+                                            None, None, 0, None) == B.ERR_INVALID
     lib.bgtq_layout_set_destroy(None)                                          # a no-op
