@@ -1373,9 +1373,13 @@ int split_smem_limit() {
   return optin - kStaticReserve;
 }
 
-// Warps per split CTA: 12 when their ring stages fit next to the tables, else 8.
+// Warps per split CTA: the most, up to 12, whose ring stages fit next to the tables (8 at
+// least). Up to 12 warps a scheduler holds at most 3 of them, so every count keeps the
+// 168-register budget (and 8 warps have up to 255).
 int split_warps(int v_rate, int tile_bytes, int limit) {
-  return split_smem_bytes(v_rate, tile_bytes, 12) <= limit ? 12 : 8;
+  for (int w = 12; w > 8; --w)
+    if (split_smem_bytes(v_rate, tile_bytes, w) <= limit) return w;
+  return 8;
 }
 
 // The split kernel of one call (and, unless scores only, the merge in its last CTA per
@@ -1393,7 +1397,10 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
   if (!sc && (L.v_rate < 1 || L.v_rate > 4)) return cudaErrorInvalidValue;
   const int limit = split_smem_limit();
   const int vr = sc ? 1 : L.v_rate;  // the scores-only variant builds no value table
-  const int W = split_warps(vr, L.tile_bytes, limit);
+  // 9-11 warps only for value rates 1-2: the rate-3/4 value path needs more registers
+  // than 168 and spills there (measured slower than 8 warps); the scores-only form, off the
+  // decode path, keeps to 12 or 8 warps too
+  const int Wf = split_warps(vr, L.tile_bytes, limit), W = (sc || vr >= 3) && Wf < 12 ? 8 : Wf;
   const int smem = split_smem_bytes(vr, L.tile_bytes, W);
   if (smem > limit) return cudaErrorInvalidValue;
   const long long units = (long long)batch * h_kv * CT;
@@ -1427,6 +1434,11 @@ cudaError_t launch_attention(const DevLayout& L, const DecodePlan& plan, int bat
     constexpr bool NPv = decltype(P)::value != 0, SCv = decltype(S)::value != 0, NHv = decltype(H)::value != 0;
     auto go = [&](auto ph) {
       constexpr bool PHv = decltype(ph)::value;
+      if constexpr (!SCv && VR <= 2) {
+        if (W == 11) return launch_split<VR, NPv, SCv, NHv, 11, PHv>(a, L, n_ctas, smem, stream);
+        if (W == 10) return launch_split<VR, NPv, SCv, NHv, 10, PHv>(a, L, n_ctas, smem, stream);
+        if (W == 9) return launch_split<VR, NPv, SCv, NHv, 9, PHv>(a, L, n_ctas, smem, stream);
+      }
       return W == 12 ? launch_split<VR, NPv, SCv, NHv, 12, PHv>(a, L, n_ctas, smem, stream)
                      : launch_split<VR, NPv, SCv, NHv, 8, PHv>(a, L, n_ctas, smem, stream);
     };
