@@ -13,7 +13,7 @@
 //    fragments. A column is one query head at one query token: a KV head has Gt = query
 //    heads per KV head x n_q columns (n_q = 1 except in multi-token calls), taken 8 at a
 //    time: a unit is (batch row, KV head, column tile of up to 8 columns).
-//  * split_kernel: one CTA per SM, 8 or 12 warps. The (batch row, KV head) caches are
+//  * split_kernel: one CTA per SM, 8 to 12 warps. The (batch row, KV head) caches are
 //    laid end to end as one sequence of 64-token tiles and every CTA takes an equal slice
 //    of it (one wave). Inside a slice, unit by unit, warp w streams its own tiles w, w+W,
 //    ... through a private pair of ring stages with 1-D bulk async copies (cp.async.bulk +
